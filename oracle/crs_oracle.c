@@ -1,0 +1,642 @@
+/*
+ * CPU oracle for content-routed sparse attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg load this library.  It shares no code, header, table or
+ * helper with the CUDA path: every function below is the plain definition of
+ * one step, written out in loops, in fp64 unless a step's integer decision is
+ * taken in fp32 (the LSH bucket, see oracle_lsh_hash).  OpenMP only splits
+ * independent rows across cores; it never changes an operation order.
+ *
+ * Pages cited:
+ *   [P1] PaperTrace 2.1.1 "哈希与聚类: 用内容建立稀疏注意力邻域"
+ *   [P2] PaperTrace 2.2 "细粒度索引: 用轻量 selector 召回关键 token"
+ *   [P4] Understanding LLMs ch. 26 "高效、稀疏与替代架构地图"
+ *   [P5] "COBS 阅读笔记: 块稀疏注意力的选择器到底漏掉了什么"
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OAPI __attribute__((visibility("default")))
+
+/* ======================================================================
+ * O1  LSH bucket id.  [P1] §2.1 Eq.(4): u = x R with R in R^{d x b/2};
+ * the bucket is the argmax of the concatenation [u ; -u] over b entries.
+ * The argmax is an integer decided by floating point, so it is taken in the
+ * precision of the kernel: each u_k is one fp32 fused multiply-add per term,
+ * terms in increasing index order starting from 0.  Ties go to the lowest
+ * index (the first maximum met scanning j = 0..b-1).
+ * Layout: X [B,H,n,d] fp32, R [H,rounds,d,b/2] fp32, bucket [B,H,rounds,n].
+ * ====================================================================== */
+OAPI void oracle_lsh_hash(int B, int H, int n, int d, int n_buckets, int n_rounds,
+                          const float *X, const float *R, int32_t *bucket)
+{
+    const int half = n_buckets / 2;
+    const long nbh = (long)B * H;
+#pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < nbh; ++bh) {
+        const int h = (int)(bh % H);
+        for (int i = 0; i < n; ++i) {
+            const float *x = X + (bh * n + i) * (long)d;
+            for (int r = 0; r < n_rounds; ++r) {
+                const float *Rr = R + ((long)h * n_rounds + r) * (long)d * half;
+                int arg = 0;
+                float best = 0.0f;
+                for (int j = 0; j < n_buckets; ++j) {
+                    const int k = (j < half) ? j : j - half;
+                    float u = 0.0f;
+                    for (int t = 0; t < d; ++t)
+                        u = fmaf(x[t], Rr[(long)t * half + k], u);
+                    const float c = (j < half) ? u : -u;
+                    if (j == 0 || c > best) {
+                        best = c;
+                        arg = j;
+                    }
+                }
+                bucket[(bh * n_rounds + r) * (long)n + i] = arg;
+            }
+        }
+    }
+}
+
+/* fp64 companion of O1: the gap between the largest and second largest entry
+ * of [u ; -u] computed in fp64, per (b,h,r,i).  Reported by tests as the
+ * distance of each bucket decision from a tie. */
+OAPI void oracle_lsh_margin(int B, int H, int n, int d, int n_buckets, int n_rounds,
+                            const float *X, const float *R, double *margin)
+{
+    const int half = n_buckets / 2;
+    const long nbh = (long)B * H;
+#pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < nbh; ++bh) {
+        const int h = (int)(bh % H);
+        for (int i = 0; i < n; ++i) {
+            const float *x = X + (bh * n + i) * (long)d;
+            for (int r = 0; r < n_rounds; ++r) {
+                const float *Rr = R + ((long)h * n_rounds + r) * (long)d * half;
+                double b1 = -INFINITY, b2 = -INFINITY;
+                for (int j = 0; j < n_buckets; ++j) {
+                    const int k = (j < half) ? j : j - half;
+                    double u = 0.0;
+                    for (int t = 0; t < d; ++t)
+                        u += (double)x[t] * (double)Rr[(long)t * half + k];
+                    const double c = (j < half) ? u : -u;
+                    if (c > b1) {
+                        b2 = b1;
+                        b1 = c;
+                    } else if (c > b2) {
+                        b2 = c;
+                    }
+                }
+                margin[(bh * n_rounds + r) * (long)n + i] = b1 - b2;
+            }
+        }
+    }
+}
+
+/* ======================================================================
+ * O1  Sort.  [P1] §2.1 (last paragraph) and §2.2: the sort key combines the
+ * bucket id and the position; sorting tokens by it gives the permutation pi
+ * (slot -> original position); pi^{-1} maps a position back to its slot.
+ * Key = bucket * n + pos, ascending.  Keys are unique, so this equals a
+ * stable sort on the bucket id.
+ * ====================================================================== */
+static int cmp_i64(const void *a, const void *b)
+{
+    const int64_t x = *(const int64_t *)a, y = *(const int64_t *)b;
+    return (x > y) - (x < y);
+}
+
+OAPI void oracle_lsh_sort(int n_segments, int n, const int32_t *bucket,
+                          int32_t *perm, int32_t *inv_perm)
+{
+#pragma omp parallel for schedule(static)
+    for (long sg = 0; sg < n_segments; ++sg) {
+        int64_t *key = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
+        const int32_t *bk = bucket + sg * (long)n;
+        for (int p = 0; p < n; ++p)
+            key[p] = (int64_t)bk[p] * n + p;
+        qsort(key, (size_t)n, sizeof(int64_t), cmp_i64);
+        for (int s = 0; s < n; ++s) {
+            const int p = (int)(key[s] % n);
+            perm[sg * (long)n + s] = p;
+            inv_perm[sg * (long)n + p] = s;
+        }
+        free(key);
+    }
+}
+
+/* ======================================================================
+ * O2  Candidate set of query i in one (batch, head).
+ * [P1] §2.1-2.2: after sorting, the sorted array is cut into chunks of m
+ * slots; a query's chunk attends to itself and to the previous chunk (chunk 0
+ * has none); a legal edge still needs the same bucket id and is judged on the
+ * original positions.  [P1] §1.1 Eq.(2): N(i) = B(i) ∩ C(i) ∩ P(i): content,
+ * causal (j <= i) and valid (j < valid_len); optionally no self (j != i).
+ * Several rounds: the union over rounds, a set ([P1] "重复候选和归一化":
+ * duplicates are removed before the softmax).
+ * Arrays bucket/perm/inv_perm point at this (b,h): [rounds, n].
+ * Returns |U(i)|; cand[] receives U(i) in ascending order.  mark[] is n bytes
+ * of zeroed scratch and is left zeroed.
+ * ====================================================================== */
+static int cmp_i32(const void *a, const void *b)
+{
+    const int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+OAPI int oracle_lsh_candidates(int n, int n_rounds, int m, int causal, int no_self,
+                               int valid_len, const int32_t *bucket, const int32_t *perm,
+                               const int32_t *inv_perm, int i, int32_t *cand, uint8_t *mark)
+{
+    int cnt = 0;
+    for (int r = 0; r < n_rounds; ++r) {
+        const int32_t *bk = bucket + (long)r * n;
+        const int32_t *pm = perm + (long)r * n;
+        const int32_t *ip = inv_perm + (long)r * n;
+        const int c = ip[i] / m;
+        for (int cc = c - 1; cc <= c; ++cc) {
+            if (cc < 0)
+                continue;
+            const int s0 = cc * m;
+            const int s1 = (s0 + m < n) ? s0 + m : n;
+            for (int s = s0; s < s1; ++s) {
+                const int j = pm[s];
+                if (bk[j] != bk[i]) continue;
+                if (causal && j > i) continue;
+                if (no_self && j == i) continue;
+                if (j >= valid_len) continue;
+                if (!mark[j]) {
+                    mark[j] = 1;
+                    cand[cnt++] = j;
+                }
+            }
+        }
+    }
+    for (int t = 0; t < cnt; ++t)
+        mark[cand[t]] = 0;
+    qsort(cand, (size_t)cnt, sizeof(int32_t), cmp_i32);
+    return cnt;
+}
+
+/* ======================================================================
+ * O3  LSH attention.  [P1] §1.1 Eq.(1): O_i = sum_{j in N(i)} softmax_j(s_ij) v_j,
+ * with the shared-QK key k_j = q_j / |q_j| ([P1] §2, Reformer: the query
+ * keeps its norm) when key_norm != 0, k_j = q_j otherwise; s_ij = scale * q_i.k_j.
+ * Computed directly over the union set U(i): no per-round merge.  A query
+ * with an empty set, and every padded query (i >= valid_len), gets O_i = 0
+ * and lse = -inf.  A zero-norm key is the zero vector.
+ * Layout: QK, V [B,H,n,d] fp64; bucket/perm/inv_perm [B,H,rounds,n];
+ * valid_len [B]; rows: the query positions to compute (NULL = all n), the
+ * outputs O [B,H,n_rows,d], lse [B,H,n_rows], count [B,H,n_rows].
+ * ====================================================================== */
+OAPI void oracle_lsh_attn(int B, int H, int n, int d, int n_rounds, int m, int causal,
+                          int no_self, int key_norm, double scale, const double *QK,
+                          const double *V, const int32_t *bucket, const int32_t *perm,
+                          const int32_t *inv_perm, const int32_t *valid_len,
+                          const int32_t *rows, int n_rows, double *O, double *lse,
+                          int32_t *count)
+{
+    const long nbh = (long)B * H;
+    const int nr = rows ? n_rows : n;
+#pragma omp parallel
+    {
+        int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+        uint8_t *mark = (uint8_t *)calloc((size_t)n, 1);
+        double *logit = (double *)malloc(sizeof(double) * (size_t)n);
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (long bh = 0; bh < nbh; ++bh) {
+            for (int t = 0; t < nr; ++t) {
+                const int b = (int)(bh / H);
+                const int i = rows ? rows[t] : t;
+                const long seg = bh * (long)n_rounds * n;
+                const double *Qb = QK + bh * (long)n * d;
+                const double *Vb = V + bh * (long)n * d;
+                double *o = O + (bh * nr + t) * (long)d;
+                for (int k = 0; k < d; ++k)
+                    o[k] = 0.0;
+                double l = -INFINITY;
+                int cnt = 0;
+                if (i < valid_len[b]) {
+                    cnt = oracle_lsh_candidates(n, n_rounds, m, causal, no_self, valid_len[b],
+                                                bucket + seg, perm + seg, inv_perm + seg, i,
+                                                cand, mark);
+                    if (cnt > 0) {
+                        const double *qi = Qb + (long)i * d;
+                        double mx = -INFINITY;
+                        for (int c = 0; c < cnt; ++c) {
+                            const double *qj = Qb + (long)cand[c] * d;
+                            double dot = 0.0, nn = 0.0;
+                            for (int k = 0; k < d; ++k) {
+                                dot += qi[k] * qj[k];
+                                nn += qj[k] * qj[k];
+                            }
+                            double s;
+                            if (key_norm)
+                                s = (nn > 0.0) ? scale * dot / sqrt(nn) : 0.0;
+                            else
+                                s = scale * dot;
+                            logit[c] = s;
+                            if (s > mx) mx = s;
+                        }
+                        double z = 0.0;
+                        for (int c = 0; c < cnt; ++c)
+                            z += exp(logit[c] - mx);
+                        for (int c = 0; c < cnt; ++c) {
+                            const double p = exp(logit[c] - mx) / z;
+                            const double *vj = Vb + (long)cand[c] * d;
+                            for (int k = 0; k < d; ++k)
+                                o[k] += p * vj[k];
+                        }
+                        l = mx + log(z);
+                    }
+                }
+                lse[bh * nr + t] = l;
+                count[bh * nr + t] = cnt;
+            }
+        }
+        free(cand);
+        free(mark);
+        free(logit);
+    }
+}
+
+/* ======================================================================
+ * O4  Lightning-indexer score and token top-k.
+ * [P2] §1.1 and §2.1 Eq.(3)-(4): r_{t,s} = sum_h w_{t,h} ReLU(q_{t,h} . k_s)
+ * over the index heads, no extra scale; S_t = Select(r_{t,0:t}, k) keeps the k
+ * largest.  [P2] §2.1 "Select 不等于一次普通 top-k": a row with fewer than k
+ * visible keys returns them all and marks the other slots invalid (-1);
+ * [P2] §3.1 "多卡一致性": ties are broken lexicographically on (score, index),
+ * i.e. equal scores prefer the smaller index.  Output ascending by position.
+ * Layout: q [rows, heads, d]; w [rows, heads]; K: keys of row t are
+ * K[(key_base[t] + s) * d + .] for s < n_visible[t].
+ * ====================================================================== */
+OAPI void oracle_indexer_score(int n_heads, int d, const double *q, const double *w,
+                               const double *K, long n_keys, double *out)
+{
+    for (long s = 0; s < n_keys; ++s) {
+        const double *k = K + s * d;
+        double r = 0.0;
+        for (int h = 0; h < n_heads; ++h) {
+            double dot = 0.0;
+            for (int t = 0; t < d; ++t)
+                dot += q[h * d + t] * k[t];
+            r += w[h] * (dot > 0.0 ? dot : 0.0);
+        }
+        out[s] = r;
+    }
+}
+
+typedef struct {
+    double s;
+    int32_t i;
+} scored_t;
+
+static int cmp_score_desc_idx_asc(const void *a, const void *b)
+{
+    const scored_t *x = (const scored_t *)a, *y = (const scored_t *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->i > y->i) - (x->i < y->i);
+}
+
+OAPI void oracle_indexer_topk(int n_rows, int n_heads, int d, int topk, const double *q,
+                              const double *w, const double *K, const int64_t *key_base,
+                              const int32_t *n_visible, int32_t *out_idx, int32_t *out_count,
+                              double *out_cutoff, double *out_next)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long t = 0; t < n_rows; ++t) {
+        const int nv = n_visible[t];
+        scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(nv > 0 ? nv : 1));
+        double *tmp = (double *)malloc(sizeof(double) * (size_t)(nv > 0 ? nv : 1));
+        oracle_indexer_score(n_heads, d, q + t * (long)n_heads * d, w + t * (long)n_heads,
+                             K + key_base[t] * (long)d, nv, tmp);
+        for (int s = 0; s < nv; ++s) {
+            sc[s].s = tmp[s];
+            sc[s].i = s;
+        }
+        qsort(sc, (size_t)nv, sizeof(scored_t), cmp_score_desc_idx_asc);
+        const int kk = nv < topk ? nv : topk;
+        int32_t *o = out_idx + t * (long)topk;
+        for (int c = 0; c < kk; ++c)
+            o[c] = sc[c].i;
+        qsort(o, (size_t)kk, sizeof(int32_t), cmp_i32);
+        for (int c = kk; c < topk; ++c)
+            o[c] = -1;
+        out_count[t] = kk;
+        out_cutoff[t] = kk > 0 ? sc[kk - 1].s : -INFINITY;
+        out_next[t] = nv > kk ? sc[kk].s : -INFINITY;
+        free(sc);
+        free(tmp);
+    }
+}
+
+/* ======================================================================
+ * O5  Block descriptor.  [P5] Eq.(11): mean key and population covariance
+ * Sigma_b = (1/L) sum (k_r - kbar)(k_r - kbar)^T; Eq.(16): keep the r largest
+ * eigen-directions, xi_i = sqrt(lambda_i) u_i; Eq.(20) / Algorithm 2 (Gram
+ * route): eigen-decompose G = (1/L) Kt Kt^T (L x L) and map back with
+ * xi_i = Kt^T w_i / sqrt(L).  A partial block uses its own count L' for L.
+ * The eigen-decomposition is the cyclic Jacobi method (Jacobi 1846; as in
+ * Golub & Van Loan, "Matrix Computations", symmetric Schur 2x2 rotations),
+ * swept until the off-diagonal mass is below 1e-30 of the total.
+ * Layout: K [n_blocks, L_cap, D] fp64 (rows >= L_eff[b] ignored); outputs
+ * mu [n_blocks, D], xi [n_blocks, rank, D], lam [n_blocks, rank] (descending).
+ * ====================================================================== */
+static void jacobi_eig(int n, double *A, double *Vm)
+{
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j)
+            Vm[i * n + j] = (i == j) ? 1.0 : 0.0;
+    double total = 0.0;
+    for (int i = 0; i < n * n; ++i)
+        total += A[i] * A[i];
+    for (int sweep = 0; sweep < 100; ++sweep) {
+        double off = 0.0;
+        for (int p = 0; p < n; ++p)
+            for (int q = 0; q < n; ++q)
+                if (p != q) off += A[p * n + q] * A[p * n + q];
+        if (off <= 1e-30 * total || off == 0.0)
+            break;
+        for (int p = 0; p < n - 1; ++p) {
+            for (int q = p + 1; q < n; ++q) {
+                const double apq = A[p * n + q];
+                if (apq == 0.0) continue;
+                const double theta = (A[q * n + q] - A[p * n + p]) / (2.0 * apq);
+                const double t = (theta >= 0.0 ? 1.0 : -1.0) /
+                                 (fabs(theta) + sqrt(theta * theta + 1.0));
+                const double c = 1.0 / sqrt(t * t + 1.0);
+                const double s = t * c;
+                /* A <- J^T A J with J the rotation in the (p,q) plane */
+                for (int k = 0; k < n; ++k) {
+                    const double akp = A[k * n + p], akq = A[k * n + q];
+                    A[k * n + p] = c * akp - s * akq;
+                    A[k * n + q] = s * akp + c * akq;
+                }
+                for (int k = 0; k < n; ++k) {
+                    const double apk = A[p * n + k], aqk = A[q * n + k];
+                    A[p * n + k] = c * apk - s * aqk;
+                    A[q * n + k] = s * apk + c * aqk;
+                }
+                for (int k = 0; k < n; ++k) {
+                    const double vkp = Vm[k * n + p], vkq = Vm[k * n + q];
+                    Vm[k * n + p] = c * vkp - s * vkq;
+                    Vm[k * n + q] = s * vkp + c * vkq;
+                }
+            }
+        }
+    }
+}
+
+OAPI void oracle_block_describe(int n_blocks, int L_cap, int D, int rank, const double *K,
+                                const int32_t *L_eff, double *mu, double *xi, double *lam)
+{
+#pragma omp parallel
+    {
+        double *Kt = (double *)malloc(sizeof(double) * (size_t)L_cap * D);
+        double *G = (double *)malloc(sizeof(double) * (size_t)L_cap * L_cap);
+        double *W = (double *)malloc(sizeof(double) * (size_t)L_cap * L_cap);
+        int *order = (int *)malloc(sizeof(int) * (size_t)L_cap);
+#pragma omp for schedule(dynamic, 8)
+        for (long b = 0; b < n_blocks; ++b) {
+            const int L = L_eff ? L_eff[b] : L_cap;
+            const double *Kb = K + b * (long)L_cap * D;
+            double *m = mu + b * (long)D;
+            for (int t = 0; t < D; ++t) {
+                double acc = 0.0;
+                for (int r = 0; r < L; ++r)
+                    acc += Kb[(long)r * D + t];
+                m[t] = (L > 0) ? acc / L : 0.0;
+            }
+            for (int r = 0; r < L; ++r)
+                for (int t = 0; t < D; ++t)
+                    Kt[(long)r * D + t] = Kb[(long)r * D + t] - m[t];
+            for (int i = 0; i < L; ++i)
+                for (int j = 0; j < L; ++j) {
+                    double acc = 0.0;
+                    for (int t = 0; t < D; ++t)
+                        acc += Kt[(long)i * D + t] * Kt[(long)j * D + t];
+                    G[i * L + j] = acc / L;
+                }
+            if (L > 0)
+                jacobi_eig(L, G, W);
+            /* order eigenpairs by eigenvalue, descending (selection sort, ties by index) */
+            for (int i = 0; i < L; ++i)
+                order[i] = i;
+            for (int i = 0; i < L; ++i) {
+                int best = i;
+                for (int j = i + 1; j < L; ++j)
+                    if (G[order[j] * L + order[j]] > G[order[best] * L + order[best]])
+                        best = j;
+                const int tmp = order[i];
+                order[i] = order[best];
+                order[best] = tmp;
+            }
+            for (int e = 0; e < rank; ++e) {
+                double *x = xi + (b * (long)rank + e) * D;
+                if (e >= L) {
+                    for (int t = 0; t < D; ++t)
+                        x[t] = 0.0;
+                    lam[b * (long)rank + e] = 0.0;
+                    continue;
+                }
+                const int col = order[e];
+                lam[b * (long)rank + e] = G[col * L + col];
+                for (int t = 0; t < D; ++t) {
+                    double acc = 0.0;
+                    for (int r = 0; r < L; ++r)
+                        acc += Kt[(long)r * D + t] * W[r * L + col];
+                    x[t] = acc / sqrt((double)L);
+                }
+            }
+        }
+        free(Kt);
+        free(G);
+        free(W);
+        free(order);
+    }
+}
+
+/* Exact block log-mass, [P5] Eq.(1): ln m_b = ln sum_{r in b} exp(q . k_r).
+ * Used by tests as the OSA reference ([P5] Algorithm 1) and for the toy
+ * example of [P5] Eq.(P4)-(P5). */
+OAPI double oracle_block_log_mass(int L, int D, const double *q, const double *Kb)
+{
+    double mx = -INFINITY;
+    for (int r = 0; r < L; ++r) {
+        double s = 0.0;
+        for (int t = 0; t < D; ++t)
+            s += q[t] * Kb[(long)r * D + t];
+        if (s > mx) mx = s;
+    }
+    double z = 0.0;
+    for (int r = 0; r < L; ++r) {
+        double s = 0.0;
+        for (int t = 0; t < D; ++t)
+            s += q[t] * Kb[(long)r * D + t];
+        z += exp(s - mx);
+    }
+    return mx + log(z);
+}
+
+/* ======================================================================
+ * O6  Block selection.  [P5] Eq.(14)/(19): the second-order log-mass
+ * estimate, without the ln L constant that cancels in the ranking,
+ *   s_{g,b} = qt . mu_b + 1/2 sum_i (xi_i . qt)^2,  qt = scale * q_g;
+ * [P5] Eq.(15)/(6): for KV head h the block score is the sum over its
+ * query-head group of each head's softmax over blocks,
+ *   score_b = sum_{g in group(h)} exp(s_{g,b}) / sum_{b'} exp(s_{g,b'});
+ * keep the top_blocks blocks by (score desc, block asc) among the
+ * n_full = floor(T / L) complete blocks; the token set is the union of the
+ * kept blocks' positions and the window [T - window, T), without duplicates,
+ * ascending.  Query heads of group h are [h*G, (h+1)*G) ([P4] §26.2).
+ * Layout: Q [n_seq, n_q, D]; mu [n_seq, n_kv, n_full, D];
+ * xi [n_seq, n_kv, n_full, rank, D]; outputs tok [n_seq, n_kv, cap] (-1 pad),
+ * tok_count [n_seq, n_kv], blk [n_seq, n_kv, top_blocks] (ascending),
+ * blk_score [n_seq, n_kv, n_full].
+ * ====================================================================== */
+OAPI void oracle_block_select(int n_seq, int n_kv, int n_q, int D, int rank, int n_full, int L,
+                              int T, int top_blocks, int window, double scale, const double *Q,
+                              const double *mu, const double *xi, int cap, int32_t *tok,
+                              int32_t *tok_count, int32_t *blk, double *blk_score)
+{
+    const int G = n_q / n_kv;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)n_full);
+        double *qt = (double *)malloc(sizeof(double) * (size_t)D);
+        scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(n_full > 0 ? n_full : 1));
+        uint8_t *mark = (uint8_t *)malloc((size_t)(T > 0 ? T : 1));
+#pragma omp for collapse(2) schedule(dynamic, 1)
+        for (int sq = 0; sq < n_seq; ++sq) {
+            for (int h = 0; h < n_kv; ++h) {
+                const long sh = (long)sq * n_kv + h;
+                double *score = blk_score + sh * n_full;
+                for (int b = 0; b < n_full; ++b)
+                    score[b] = 0.0;
+                for (int g = h * G; g < (h + 1) * G; ++g) {
+                    const double *q = Q + ((long)sq * n_q + g) * D;
+                    for (int t = 0; t < D; ++t)
+                        qt[t] = scale * q[t];
+                    double mx = -INFINITY;
+                    for (int b = 0; b < n_full; ++b) {
+                        const double *m = mu + (sh * n_full + b) * (long)D;
+                        double v = 0.0;
+                        for (int t = 0; t < D; ++t)
+                            v += qt[t] * m[t];
+                        double quad = 0.0;
+                        for (int e = 0; e < rank; ++e) {
+                            const double *x = xi + ((sh * n_full + b) * (long)rank + e) * D;
+                            double p = 0.0;
+                            for (int t = 0; t < D; ++t)
+                                p += x[t] * qt[t];
+                            quad += p * p;
+                        }
+                        s[b] = v + 0.5 * quad;
+                        if (s[b] > mx) mx = s[b];
+                    }
+                    double z = 0.0;
+                    for (int b = 0; b < n_full; ++b)
+                        z += exp(s[b] - mx);
+                    for (int b = 0; b < n_full; ++b)
+                        score[b] += exp(s[b] - mx) / z;
+                }
+                for (int b = 0; b < n_full; ++b) {
+                    sc[b].s = score[b];
+                    sc[b].i = b;
+                }
+                qsort(sc, (size_t)n_full, sizeof(scored_t), cmp_score_desc_idx_asc);
+                const int nk = top_blocks < n_full ? top_blocks : n_full;
+                int32_t *bo = blk + sh * top_blocks;
+                for (int c = 0; c < nk; ++c)
+                    bo[c] = sc[c].i;
+                qsort(bo, (size_t)nk, sizeof(int32_t), cmp_i32);
+                for (int c = nk; c < top_blocks; ++c)
+                    bo[c] = -1;
+                memset(mark, 0, (size_t)T);
+                for (int c = 0; c < nk; ++c)
+                    for (int r = 0; r < L; ++r)
+                        mark[bo[c] * L + r] = 1;
+                for (int p = (T - window > 0 ? T - window : 0); p < T; ++p)
+                    mark[p] = 1;
+                int cnt = 0;
+                int32_t *to = tok + sh * cap;
+                for (int p = 0; p < T; ++p)
+                    if (mark[p]) {
+                        if (cnt < cap) to[cnt] = p;
+                        ++cnt;
+                    }
+                for (int c = cnt; c < cap; ++c)
+                    to[c] = -1;
+                tok_count[sh] = cnt;
+            }
+        }
+        free(s);
+        free(qt);
+        free(sc);
+        free(mark);
+    }
+}
+
+/* ======================================================================
+ * O7  Attention over a given index set.  [P1] §1.1 Eq.(1) restricted to the
+ * candidate set; [P2] §1 (the selected positions are shared by the main
+ * heads); [P4] §26.2 Table 26.1 (query heads [h*G, (h+1)*G) share KV head h).
+ *   O_{t,g} = sum_{j in I} softmax_j(scale * q_{t,g} . k_{j,kv(g)}) v_{j,kv(g)}
+ * over the valid (>= 0) entries of the index list; an empty list gives 0 and
+ * lse = -inf.  Duplicated entries are a caller error and are counted as given.
+ * Layout: Q [rows, n_q, D]; K, V: token j of row t, head h at
+ * ((kv_base[t] + j) * n_kv + h) * D; I [rows, n_lists, max_idx] where
+ * n_lists = n_kv (a list per KV head) or 1 (one list shared by all heads).
+ * ====================================================================== */
+OAPI void oracle_sparse_attn(int n_rows, int n_q, int n_kv, int D, double scale, const double *Q,
+                             const double *K, const double *V, const int64_t *kv_base,
+                             const int32_t *I, int n_lists, int max_idx, double *O, double *lse)
+{
+    const int G = n_q / n_kv;
+#pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(max_idx > 0 ? max_idx : 1));
+#pragma omp for collapse(2) schedule(dynamic, 4)
+        for (long t = 0; t < n_rows; ++t) {
+            for (int g = 0; g < n_q; ++g) {
+                const int h = g / G;
+                const int32_t *idx = I + (t * n_lists + (n_lists == 1 ? 0 : h)) * (long)max_idx;
+                const double *q = Q + (t * n_q + g) * (long)D;
+                double *o = O + (t * n_q + g) * (long)D;
+                for (int k = 0; k < D; ++k)
+                    o[k] = 0.0;
+                double mx = -INFINITY;
+                for (int c = 0; c < max_idx; ++c) {
+                    if (idx[c] < 0) continue;
+                    const double *kj = K + ((kv_base[t] + idx[c]) * n_kv + h) * (long)D;
+                    double dot = 0.0;
+                    for (int k = 0; k < D; ++k)
+                        dot += q[k] * kj[k];
+                    logit[c] = scale * dot;
+                    if (logit[c] > mx) mx = logit[c];
+                }
+                if (mx == -INFINITY) {
+                    lse[t * n_q + g] = -INFINITY;
+                    continue;
+                }
+                double z = 0.0;
+                for (int c = 0; c < max_idx; ++c)
+                    if (idx[c] >= 0) z += exp(logit[c] - mx);
+                for (int c = 0; c < max_idx; ++c) {
+                    if (idx[c] < 0) continue;
+                    const double p = exp(logit[c] - mx) / z;
+                    const double *vj = V + ((kv_base[t] + idx[c]) * n_kv + h) * (long)D;
+                    for (int k = 0; k < D; ++k)
+                        o[k] += p * vj[k];
+                }
+                lse[t * n_q + g] = mx + log(z);
+            }
+        }
+        free(logit);
+    }
+}
