@@ -1,0 +1,601 @@
+"""Throughput of content-routed sparse attention on B200 (one JSON line).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
+                  [--workload lsh|lsh_fp32|prefill|decode|block] [--no-extras]
+
+A step is one pass of the hot path over one batch of the workload:
+  lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
+           b=64 buckets, 4 rounds, chunk 128, causal, last 5% padding:
+           hash -> sort -> chunked attention -> round merge.  Metric: tokens/s.
+  lsh_fp32 fp32 LSH attention, n=1024, b=16, 1 round, chunk 64.
+  prefill  indexer prefill n=32768 (top-2048) + MQA gather attention (16 heads).
+  decode   indexer decode, 64 sequences of ragged context + GQA gather attention.
+  block    block-mass decode: block select (top-64 + 512 window) + GQA attention;
+           the descriptor build is timed separately (it runs once per filled block).
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on
+the launching stream; a 256 MiB buffer (2x L2) is written between steps,
+outside the events.  Multi-GPU: one process per GPU (torchrun), each rank runs
+its own batch (weak scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn prefill tokens/s & decode steps/s on 1 B200; % of HBM/TC roofline"
+FP32_ALU_TFLOPS_NOMINAL = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x 2 x max clock
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ workloads --
+class Workload:
+    name = ""
+    unit = "tokens/s"
+    units_per_step = 1.0
+    dtype = "bf16"
+
+    def step(self):
+        raise NotImplementedError
+
+    def e2e_step(self):
+        raise NotImplementedError
+
+    def roofline_spec(self):
+        """{kernel: (bound, amount per launch, unit)} for kernels we can account."""
+        return {}
+
+
+class LshWorkload(Workload):
+    def __init__(self, crs, dev, fp32=False):
+        import workloads
+        self.crs = crs
+        case = workloads.lsh_fp32_case(device=dev) if fp32 else workloads.lsh_clustered_case(device=dev)
+        self.case = case
+        p = case["params"]
+        self.p = p
+        self.name = case["workload"]
+        self.dtype = "f32" if fp32 else "bf16"
+        self.units_per_step = p["B"] * p["n"]
+        B, H, n, d, R = p["B"], p["H"], p["n"], p["d"], p["n_rounds"]
+        self.route_out = tuple(torch.empty((B, H, R, n), dtype=torch.int32, device=dev) for _ in range(3))
+        self.O = torch.empty(case["QK"].shape, dtype=torch.float32, device=dev)
+        a = crs.LshAttnParams(crs.lsh_params(case["QK"], p["n_buckets"], R, p["chunk"]),
+                              p["causal"], p["no_self"], p["key_norm"], p["scale"])
+        import ctypes
+        ws = int(crs.lib().crs_lsh_attn_workspace_size(ctypes.byref(a)))
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # host copies for the end-to-end pass
+        self.h_in = {k: case[k].cpu().pin_memory() for k in ("QK", "V", "R", "valid_len")}
+        self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.d_in = {k: torch.empty_like(case[k]) for k in self.h_in}
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def _run(self, src):
+        p = self.p
+        b, pm, ip = self.crs.lsh_route(src["QK"], src["R"], p["n_buckets"], p["chunk"],
+                                       out=self.route_out)
+        self.crs.lsh_attn(src["QK"], src["V"], b, pm, ip, src["valid_len"],
+                          n_buckets=p["n_buckets"], chunk=p["chunk"], causal=p["causal"],
+                          no_self=p["no_self"], key_norm=p["key_norm"], scale=p["scale"],
+                          out=self.O, workspace=self.ws)
+
+    def step(self):
+        self._run(self.case)
+
+    def e2e_step(self):
+        for k, h in self.h_in.items():
+            self.d_in[k].copy_(h, non_blocking=True)
+        self._run(self.d_in)
+        self.h_out.copy_(self.O, non_blocking=True)
+
+    def roofline_spec(self):
+        p = self.p
+        B, H, n, d, R, m = p["B"], p["H"], p["n"], p["d"], p["n_rounds"], p["chunk"]
+        rect_flops = B * H * R * n * (2 * m) * d * 4          # QK^T and P.V over own+previous chunk
+        esz = 2 if self.dtype == "bf16" else 4
+        attn_bytes = B * H * R * n * d * esz * 2 + B * H * R * n * (d + 1) * 4
+        return {
+            "lsh_chunk_attn": [("alu", rect_flops / 1e12, "TFLOP/s"),
+                               ("hbm", attn_bytes / 1e9, "GB/s")],
+            "lsh_hash": [("alu", B * H * R * n * d * (p["n_buckets"] // 2) * 2 / 1e12, "TFLOP/s")],
+        }
+
+
+class PrefillWorkload(Workload):
+    unit = "tokens/s"
+
+    def __init__(self, crs, dev):
+        import workloads
+        self.crs = crs
+        c = workloads.indexer_prefill_case(device=dev)
+        self.c = c
+        self.p = c["params"]
+        self.name = c["workload"]
+        n, k = self.p["n"], self.p["topk"]
+        self.units_per_step = n
+        self.idx = torch.empty((n, k), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((n,), dtype=torch.int32, device=dev)
+        self.O = torch.empty(c["Q"].shape, dtype=torch.float32, device=dev)
+        import ctypes
+        ip = crs.IndexerParams(crs.CRS_IDX_PREFILL, n, 4, 64, k, 0)
+        self.ws = torch.empty(max(1, int(crs.lib().crs_indexer_topk_workspace_size(ctypes.byref(ip)))),
+                              dtype=torch.uint8, device=dev)
+        self.h_in = {k2: c[k2].cpu().pin_memory() for k2 in ("Q", "K", "V", "q_idx", "k_idx", "w")}
+        self.d_in = {k2: torch.empty_like(c[k2]) for k2 in self.h_in}
+        self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def _run(self, src):
+        k = self.p["topk"]
+        self.crs.indexer_topk(src["q_idx"], src["w"], src["k_idx"], k, self.crs.CRS_IDX_PREFILL,
+                              out=self.idx, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(src["Q"], src["K"], src["V"], self.idx.view(-1, 1, k), out=self.O)
+
+    def step(self):
+        self._run(self.c)
+
+    def e2e_step(self):
+        for k2, h in self.h_in.items():
+            self.d_in[k2].copy_(h, non_blocking=True)
+        self._run(self.d_in)
+        self.h_out.copy_(self.O, non_blocking=True)
+
+    def roofline_spec(self):
+        n, k = self.p["n"], self.p["topk"]
+        pairs = n * (n + 1) // 2
+        rows = sum(min(k, t + 1) for t in range(n))
+        return {
+            "idx_slice_topk": [("alu", pairs * 4 * 64 * 2 / 1e12, "TFLOP/s")],
+            "sparse_attn": [("hbm", rows * 128 * 2 * 2 / 1e9, "GB/s"),
+                            ("tensor", rows * 16 * 128 * 4 / 1e12, "TFLOP/s")],
+        }
+
+
+class DecodeWorkload(Workload):
+    unit = "steps/s"
+
+    def __init__(self, crs, dev):
+        import workloads
+        self.crs = crs
+        c = workloads.indexer_decode_case(device=dev)
+        self.c = c
+        self.p = c["params"]
+        self.name = c["workload"]
+        ns, k = self.p["n_seq"], self.p["topk"]
+        self.units_per_step = 1
+        self.idx = torch.empty((ns, k), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((ns,), dtype=torch.int32, device=dev)
+        self.O = torch.empty(c["Q"].shape, dtype=torch.float32, device=dev)
+        self.kv_base = c["offsets"][:-1].contiguous()
+        import ctypes
+        ip = crs.IndexerParams(crs.CRS_IDX_DECODE, ns, 4, 64, k, 131072)
+        self.ws = torch.empty(int(crs.lib().crs_indexer_topk_workspace_size(ctypes.byref(ip))),
+                              dtype=torch.uint8, device=dev)
+        ap = crs.AttnParams(ns, 32, 8, 128, k, 1, 0, 0.0)
+        self.ws2 = torch.empty(max(1, int(crs.lib().crs_sparse_attn_workspace_size(ctypes.byref(ap)))),
+                               dtype=torch.uint8, device=dev)
+        # end to end: the per-step inputs are the new queries (caches stay resident)
+        self.h_in = {k2: c[k2].cpu().pin_memory() for k2 in ("q_idx", "w", "Q")}
+        self.d_in = {k2: torch.empty_like(c[k2]) for k2 in self.h_in}
+        self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+        self.total_ctx = int(c["offsets"][-1])
+
+    def _run(self, q_idx, w, Q):
+        k = self.p["topk"]
+        self.crs.indexer_topk(q_idx, w, self.c["k_idx"], k, self.crs.CRS_IDX_DECODE,
+                              k_offsets=self.c["offsets"], max_keys=131072, out=self.idx,
+                              count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(Q, self.c["K"], self.c["V"], self.idx.view(-1, 1, k),
+                             kv_base=self.kv_base, out=self.O, workspace=self.ws2)
+
+    def step(self):
+        self._run(self.c["q_idx"], self.c["w"], self.c["Q"])
+
+    def e2e_step(self):
+        for k2, h in self.h_in.items():
+            self.d_in[k2].copy_(h, non_blocking=True)
+        self._run(self.d_in["q_idx"], self.d_in["w"], self.d_in["Q"])
+        self.h_out.copy_(self.O, non_blocking=True)
+
+    def roofline_spec(self):
+        ns, k = self.p["n_seq"], self.p["topk"]
+        return {
+            "idx_slice_topk": [("hbm", self.total_ctx * 64 * 2 / 1e9, "GB/s")],
+            "sparse_attn": [("hbm", ns * k * 8 * 128 * 2 * 2 / 1e9, "GB/s")],
+        }
+
+
+class BlockWorkload(Workload):
+    unit = "steps/s"
+
+    def __init__(self, crs, dev):
+        import workloads
+        self.crs = crs
+        c = workloads.block_decode_case(device=dev)
+        self.c = c
+        self.p = c["params"]
+        self.name = c["workload"]
+        p = self.p
+        self.units_per_step = 1
+        self.mu, self.xi = crs.block_describe(c["K"], p["L"], p["rank"])   # cache build (once)
+        torch.cuda.synchronize()
+        cap = p["top_blocks"] * p["L"] + p["window"]
+        self.tok = torch.empty((p["n_seq"], p["n_kv_heads"], cap), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((p["n_seq"], p["n_kv_heads"]), dtype=torch.int32, device=dev)
+        self.O = torch.empty(c["Q"].shape, dtype=torch.float32, device=dev)
+        self.Kf = c["K"].view(p["n_seq"] * p["T"], p["n_kv_heads"], p["D"])
+        self.Vf = c["V"].view(p["n_seq"] * p["T"], p["n_kv_heads"], p["D"])
+        self.kv_base = torch.arange(p["n_seq"], device=dev, dtype=torch.int64) * p["T"]
+        import ctypes
+        bp = crs.BlockSelParams(crs.BlockParams(p["n_seq"], p["n_kv_heads"], p["T"], p["D"], p["L"],
+                                                p["rank"], 0, p["T"] // p["L"]),
+                                p["n_q_heads"], p["top_blocks"], p["window"], p["scale"])
+        self.ws = torch.empty(int(crs.lib().crs_block_select_workspace_size(ctypes.byref(bp))),
+                              dtype=torch.uint8, device=dev)
+        ap = crs.AttnParams(p["n_seq"], p["n_q_heads"], p["n_kv_heads"], p["D"], cap,
+                            p["n_kv_heads"], 0, 0.0)
+        self.ws2 = torch.empty(max(1, int(crs.lib().crs_sparse_attn_workspace_size(ctypes.byref(ap)))),
+                               dtype=torch.uint8, device=dev)
+        self.h_in = {"Q": c["Q"].cpu().pin_memory()}
+        self.d_in = {"Q": torch.empty_like(c["Q"])}
+        self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.h2d = self.h_in["Q"].numel() * 2
+        self.d2h = self.h_out.numel() * 2
+
+    def _run(self, Q):
+        p = self.p
+        self.crs.block_select(Q, self.mu, self.xi, p["T"], p["L"], p["top_blocks"], p["window"],
+                              tok=self.tok, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
+                             workspace=self.ws2)
+
+    def step(self):
+        self._run(self.c["Q"])
+
+    def e2e_step(self):
+        self.d_in["Q"].copy_(self.h_in["Q"], non_blocking=True)
+        self._run(self.d_in["Q"])
+        self.h_out.copy_(self.O, non_blocking=True)
+
+    def roofline_spec(self):
+        p = self.p
+        nf = p["T"] // p["L"]
+        desc = p["n_seq"] * p["n_kv_heads"] * nf * (1 + p["rank"]) * p["D"] * 4
+        cap = p["top_blocks"] * p["L"] + p["window"]
+        return {
+            "block_score": [("hbm", desc / 1e9, "GB/s")],
+            "sparse_attn": [("hbm", p["n_seq"] * p["n_kv_heads"] * cap * p["D"] * 2 * 2 / 1e9, "GB/s")],
+        }
+
+
+WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
+             "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
+             "prefill": PrefillWorkload, "decode": DecodeWorkload, "block": BlockWorkload}
+
+
+# ------------------------------------------------------------------- timing --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                power.append(float(r[3]))
+                for k, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(k)
+            except (ValueError, IndexError):
+                continue
+        loaded = [s for s, p in zip(sm, power) if p > 200] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len([p for p in power if p > 200])}
+
+
+def _flush_l2(buf):
+    buf.add_(1)
+
+
+def time_steps(fn, steps, warmup, flush_buf, dist_on):
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+        _flush_l2(flush_buf)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+        _flush_l2(flush_buf)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def roofline(wl, prof, peaks, traffic=None):
+    """The dominant kernel (largest summed device time) with its algorithmic work."""
+    spec = wl.roofline_spec()
+    timed = {k: v for k, v in prof.items() if v["timed_launches"] > 0}
+    if not timed:
+        return None, {}
+    stages = {k: round(v["total_ms"] / v["timed_launches"], 5) for k, v in timed.items()}
+    top = max(timed, key=lambda k: timed[k]["total_ms"])
+    if top not in spec:
+        return {"kernel": top, "bound": None, "achieved": None, "peak": None, "unit": None,
+                "frac": None, "traffic": None}, stages
+    per_launch_s = timed[top]["total_ms"] / timed[top]["timed_launches"] / 1e3
+    bound, amount, unit = spec[top][0]
+    achieved = amount / per_launch_s
+    if bound == "hbm":
+        peak, src = peaks["hbm_gbs"], f"hbm_gbs ({peaks['source']})"
+    elif bound == "tensor":
+        peak, src = peaks["bf16_tflops"], f"bf16_tflops ({peaks['source']})"
+    else:
+        peak, src = FP32_ALU_TFLOPS_NOMINAL, "fp32 FMA: 148 SM x 128 lanes x 2 x 1.965 GHz"
+    out = {"kernel": top, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
+           "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
+           "per_launch_ms": round(per_launch_s * 1e3, 5)}
+    if len(spec[top]) > 1:
+        b2, a2, u2 = spec[top][1]
+        p2 = peaks["hbm_gbs"] if b2 == "hbm" else peaks["bf16_tflops"]
+        out["secondary"] = {"bound": b2, "achieved": round(a2 / per_launch_s, 3), "peak": p2,
+                            "unit": u2, "frac": round(a2 / per_launch_s / p2, 4)}
+    return out, stages
+
+
+def measure(crs, wl, steps, warmup, flush_buf, dist_on, peaks, e2e=True):
+    crs.profile_collect()
+    times = time_steps(wl.step, steps, warmup, flush_buf, dist_on)
+    launched = crs.profile_collect()
+    launches_timed = sum(v["launches"] for v in launched.values())
+    # launches per step, counted over the timed steps only (warm-up excluded by a separate count)
+    crs.profile_collect()
+    for _ in range(1):
+        wl.step()
+    torch.cuda.synchronize()
+    per_step = sum(v["launches"] for v in crs.profile_collect().values())
+    crs.profile_set(True)
+    time_steps(wl.step, steps, 1, flush_buf, False)
+    crs.profile_set(False)
+    prof = crs.profile_collect()
+    rl, stages = roofline(wl, prof, peaks)
+    out = {"times_ms": times, "gpu_launches": per_step * steps, "roofline": rl, "stages_ms": stages,
+           "launches_in_timed_region_incl_warmup": launches_timed}
+    if e2e:
+        out["e2e_times_ms"] = time_steps(wl.e2e_step, steps, warmup, flush_buf, dist_on)
+    return out
+
+
+# ------------------------------------------------------------- CPU baseline --
+def cpu_baseline_lsh(case, n_segments=2):
+    """The oracle on a bounded sample: n_segments of the B*H (batch, head)
+    segments, each routed (hash + sort, all rounds) and attended for all n
+    query rows.  Returns (tokens/s scaled to the metric, seconds, sample text)."""
+    import numpy as np
+
+    import oracle
+    p = case["params"]
+    B, H, n = p["B"], p["H"], p["n"]
+    QK = case["QK"].float().cpu().numpy()
+    V = case["V"].float().cpu().numpy().astype(np.float64)
+    R = case["R"].cpu().numpy()
+    vl = case["valid_len"].cpu().numpy()
+    segs = [(s // H, s % H) for s in range(min(n_segments, B * H))]
+    t0 = time.perf_counter()
+    for b, h in segs:
+        x = QK[b:b + 1, h:h + 1]
+        bk = oracle.lsh_hash(x, R[h:h + 1], p["n_buckets"])
+        pm, ip = oracle.lsh_sort(bk)
+        oracle.lsh_attn(x.astype(np.float64), V[b:b + 1, h:h + 1], bk, pm, ip, vl[b:b + 1],
+                        p["chunk"], p["causal"], p["no_self"], p["key_norm"], p["scale"])
+    dt = time.perf_counter() - t0
+    tokens = B * n * len(segs) / (B * H)      # a (b, h) segment is 1/(B*H) of a step's work
+    sample = (f"{len(segs)} of {B*H} (batch, head) segments: hash + sort + LSH attention for all "
+              f"{n} query rows and {p['n_rounds']} rounds, scaled by segments/(B*H)")
+    return tokens / dt, dt, sample
+
+
+def _omp_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
+
+
+# --------------------------------------------------------------------- main --
+def run_reference(args, rank):
+    """Oracle arm: the CPU oracle on the host cores, bounded sample per step."""
+    if rank != 0:
+        return 0
+    import workloads
+    case = workloads.lsh_clustered_case(device="cpu")
+    p = case["params"]
+    for _ in range(args.warmup):
+        cpu_baseline_lsh(case, n_segments=1)
+    total = 0.0
+    for _ in range(args.steps):
+        _, dt, sample = cpu_baseline_lsh(case, n_segments=1)
+        total += dt
+    tokens = p["B"] * p["n"] / (p["B"] * p["H"]) * args.steps
+    val = tokens / total
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 3), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": case["workload"], "sample": "1 (batch, head) segment per step"},
+            "cpu_baseline": {"value": round(val, 3), "unit": "tokens/s", "cores": _omp_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(val, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="product", choices=["product", "reference"])
+    ap.add_argument("--workload", default="lsh", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import content_routed_sparse_b200 as crs
+
+    peaks = _peaks()
+    flush_buf = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB
+    wl = WORKLOADS[args.workload](crs, dev)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    res = measure(crs, wl, args.steps, args.warmup, flush_buf, dist_on, peaks)
+    clocks = sampler.stop()
+    assert crs.get_device_error() == 0, "device error word set during the bench"
+
+    tot_ms = sum(res["times_ms"])
+    e2e_ms = sum(res["e2e_times_ms"])
+    if dist_on:
+        t = torch.tensor([tot_ms, e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        tot_ms, e2e_ms = float(t[0]), float(t[1])
+    units = wl.units_per_step * args.steps * world
+    value = units / (tot_ms / 1e3)
+    e2e_value = units / (e2e_ms / 1e3)
+
+    extras = {}
+    if not args.no_extras and not dist_on:
+        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block") if w != args.workload]:
+            try:
+                w2 = WORKLOADS[name](crs, dev)
+                r2 = measure(crs, w2, 5, 3, flush_buf, False, peaks)
+                t2 = sum(r2["times_ms"])
+                extras[name] = {"workload": w2.name, "value": round(w2.units_per_step * 5 / (t2 / 1e3), 3),
+                                "unit": w2.unit, "ms_per_step": round(t2 / 5, 4),
+                                "roofline": r2["roofline"], "stages_ms": r2["stages_ms"],
+                                "e2e": {"value": round(w2.units_per_step * 5 / (sum(r2["e2e_times_ms"]) / 1e3), 3),
+                                        "unit": w2.unit, "h2d_bytes_per_step": w2.h2d,
+                                        "d2h_bytes_per_step": w2.d2h},
+                                "gpu_launches": r2["gpu_launches"]}
+                if name == "block":
+                    torch.cuda.synchronize()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    crs.block_describe(w2.c["K"], w2.p["L"], w2.p["rank"], mu=w2.mu, xi=w2.xi)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    extras[name]["cache_build_ms"] = round(e0.elapsed_time(e1), 4)
+                del w2
+                torch.cuda.empty_cache()
+            except Exception as e:   # an extra section must not hide the headline
+                extras[name] = {"error": f"{type(e).__name__}: {e}"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "lsh":
+        v, dt, sample = cpu_baseline_lsh(wl.case)
+        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": _omp_threads(), "kind": "oracle",
+               "sample": sample, "seconds": round(dt, 3)}
+
+    if rank == 0:
+        p = getattr(wl, "p", {})
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic",
+            "config": {"workload": wl.name, **{k: v for k, v in p.items() if not callable(v)},
+                       "l2": "256 MiB buffer written between timed steps (outside the events)",
+                       "parallelism": f"replica per GPU x{world}"},
+            "e2e": {"value": round(e2e_value, 3), "unit": wl.unit, "h2d_bytes_per_step": wl.h2d,
+                    "d2h_bytes_per_step": wl.d2h},
+            "gpu_launches": res["gpu_launches"],
+            "roofline": res["roofline"],
+            "stages_ms": res["stages_ms"],
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

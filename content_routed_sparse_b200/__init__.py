@@ -1,0 +1,363 @@
+"""content_routed_sparse_b200 -- Python binding of libcrs (content-routed sparse
+attention on NVIDIA B200, sm_100a).
+
+Argument marshalling only: every step runs in the CUDA kernels of libcrs.so,
+reached through the C ABI declared in include/crs.h.  PyTorch provides device
+memory and streams.  Importing this module loads libcrs.so and raises if it
+is missing; there is no fallback.
+
+Functions (same names as the C entry points, without the ``crs_`` prefix):
+  lsh_route, lsh_attn, indexer_topk, block_describe, block_select,
+  sparse_attn, get_device_error.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcrs.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libcrs.so not found at {LIB_PATH}; build it with "
+        "`python -m content_routed_sparse_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+CRS_F32, CRS_BF16 = 0, 1
+CRS_IDX_PREFILL, CRS_IDX_DECODE = 0, 1
+STATUS = {0: "CRS_OK", 1: "CRS_ERR_INVALID_ARG", 2: "CRS_ERR_UNSUPPORTED", 3: "CRS_ERR_CUDA",
+          4: "CRS_ERR_NONFINITE", 5: "CRS_ERR_TIMEOUT", 6: "CRS_ERR_WORKSPACE",
+          7: "CRS_ERR_INDEX"}
+DEVERR_NONFINITE, DEVERR_TIMEOUT, DEVERR_INDEX = 0x1, 0x2, 0x4
+
+
+class CrsError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class LshParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("n", ctypes.c_int),
+                ("d", ctypes.c_int), ("n_buckets", ctypes.c_int), ("n_rounds", ctypes.c_int),
+                ("chunk", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class LshAttnParams(ctypes.Structure):
+    _fields_ = [("p", LshParams), ("causal", ctypes.c_int), ("no_self", ctypes.c_int),
+                ("key_norm", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class IndexerParams(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("n_rows", ctypes.c_int), ("n_idx_heads", ctypes.c_int),
+                ("d_idx", ctypes.c_int), ("topk", ctypes.c_int), ("max_keys", ctypes.c_int)]
+
+
+class BlockParams(ctypes.Structure):
+    _fields_ = [("n_seq", ctypes.c_int), ("n_kv", ctypes.c_int), ("T", ctypes.c_int),
+                ("D", ctypes.c_int), ("L", ctypes.c_int), ("rank", ctypes.c_int),
+                ("blk_begin", ctypes.c_int), ("blk_end", ctypes.c_int)]
+
+
+class BlockSelParams(ctypes.Structure):
+    _fields_ = [("b", BlockParams), ("n_q", ctypes.c_int), ("top_blocks", ctypes.c_int),
+                ("window", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class AttnParams(ctypes.Structure):
+    _fields_ = [("n_rows", ctypes.c_int), ("n_q", ctypes.c_int), ("n_kv", ctypes.c_int),
+                ("D", ctypes.c_int), ("max_idx", ctypes.c_int), ("n_lists", ctypes.c_int),
+                ("n_keys", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("timed_launches", ctypes.c_int64), ("total_ms", ctypes.c_double)]
+
+
+_VP = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(_lib, name, None)
+    if f is None:
+        return None
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_lib.crs_status_string.restype = ctypes.c_char_p
+_lib.crs_status_string.argtypes = [ctypes.c_int]
+_lib.crs_version.restype = ctypes.c_int
+_lib.crs_get_device_error.restype = ctypes.c_int
+_lib.crs_get_device_error.argtypes = [_VP, ctypes.POINTER(ctypes.c_uint32)]
+_sig("crs_lsh_route_workspace_size", _SZ, [ctypes.POINTER(LshParams)])
+_sig("crs_lsh_route", ctypes.c_int, [ctypes.POINTER(LshParams), _VP, _VP, _VP, _VP, _VP, _VP,
+                                      _SZ, _VP])
+_sig("crs_lsh_attn_workspace_size", _SZ, [ctypes.POINTER(LshAttnParams)])
+_sig("crs_lsh_attn", ctypes.c_int, [ctypes.POINTER(LshAttnParams), _VP, _VP, _VP, _VP, _VP, _VP,
+                                     _VP, _VP, _VP, _SZ, _VP])
+_sig("crs_indexer_topk_workspace_size", _SZ, [ctypes.POINTER(IndexerParams)])
+_sig("crs_indexer_topk", ctypes.c_int, [ctypes.POINTER(IndexerParams), _VP, _VP, _VP, _VP, _VP,
+                                         _VP, _VP, _SZ, _VP])
+_sig("crs_block_describe", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP])
+_sig("crs_block_select_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams)])
+_sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
+                                         _VP, _SZ, _VP])
+_sig("crs_sparse_attn_workspace_size", _SZ, [ctypes.POINTER(AttnParams)])
+_sig("crs_sparse_attn", ctypes.c_int, [ctypes.POINTER(AttnParams), _VP, _VP, _VP, _VP, _VP, _VP,
+                                        _VP, _VP, _SZ, _VP])
+
+
+_sig("crs_profile_set", ctypes.c_int, [ctypes.c_int])
+_sig("crs_profile_collect", ctypes.c_int, [ctypes.POINTER(KernelStat), ctypes.c_int,
+                                            ctypes.POINTER(ctypes.c_int)])
+
+
+def lib():
+    """The loaded ctypes handle of libcrs.so."""
+    return _lib
+
+
+# ------------------------------------------------------------------ utils --
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, st):
+    if st != 0:
+        raise CrsError(fn, st)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
+    if nbytes == 0:
+        return None, 0
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return workspace, workspace.numel() * workspace.element_size()
+    return torch.empty(nbytes, dtype=torch.uint8, device=device), nbytes
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return CRS_F32
+    if t.dtype == torch.bfloat16:
+        return CRS_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronize, read and clear the device error word (CRS_DEVERR_* bits)."""
+    v = ctypes.c_uint32(0)
+    _check("crs_get_device_error", _lib.crs_get_device_error(_stream(stream), ctypes.byref(v)))
+    return int(v.value)
+
+
+def profile_set(enabled: bool) -> None:
+    """Turn per-launch CUDA-event timing on or off (launch counting is always on)."""
+    _check("crs_profile_set", _lib.crs_profile_set(1 if enabled else 0))
+
+
+def profile_collect() -> dict:
+    """{kernel: {"launches", "timed_launches", "total_ms"}} since the last collect (then reset)."""
+    buf = (KernelStat * 64)()
+    n = ctypes.c_int(0)
+    _check("crs_profile_collect", _lib.crs_profile_collect(buf, 64, ctypes.byref(n)))
+    out = {}
+    for i in range(min(n.value, 64)):
+        out[buf[i].name.decode()] = {"launches": int(buf[i].launches),
+                                     "timed_launches": int(buf[i].timed_launches),
+                                     "total_ms": float(buf[i].total_ms)}
+    return out
+
+
+# -------------------------------------------------------------------- LSH --
+def lsh_params(QK: torch.Tensor, n_buckets: int, n_rounds: int, chunk: int) -> LshParams:
+    B, H, n, d = QK.shape
+    return LshParams(B, H, n, d, int(n_buckets), int(n_rounds), int(chunk), _dtype_code(QK))
+
+
+def lsh_route(X: torch.Tensor, R: torch.Tensor, n_buckets: int, chunk: int = 1,
+              out=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Bucket ids, perm (slot -> position) and inv_perm, each [B,H,rounds,n] int32."""
+    _need(X, "X")
+    B, H, n, d = X.shape
+    n_rounds = R.shape[1]
+    _need(R, "R", torch.float32, (H, n_rounds, d, n_buckets // 2))
+    p = lsh_params(X, n_buckets, n_rounds, chunk)
+    shape = (B, H, n_rounds, n)
+    if out is None:
+        out = tuple(torch.empty(shape, dtype=torch.int32, device=X.device) for _ in range(3))
+    bucket, perm, inv = out
+    for t, nm in ((bucket, "bucket"), (perm, "perm"), (inv, "inv_perm")):
+        _need(t, nm, torch.int32, shape)
+    st = _lib.crs_lsh_route(ctypes.byref(p), _ptr(X), _ptr(R), _ptr(bucket), _ptr(perm),
+                            _ptr(inv), None, 0, _stream(stream))
+    _check("crs_lsh_route", st)
+    return bucket, perm, inv
+
+
+def lsh_attn(QK, V, bucket, perm, inv_perm, valid_len=None, *, n_buckets, chunk, causal=1,
+             no_self=0, key_norm=1, scale=None, out=None, lse=None, workspace=None,
+             stream=None):
+    """Chunked multi-round LSH attention; returns (O [B,H,n,d] fp32, lse [B,H,n] or None)."""
+    _need(QK, "QK")
+    B, H, n, d = QK.shape
+    _need(V, "V", QK.dtype, QK.shape)
+    n_rounds = bucket.shape[2]
+    for t, nm in ((bucket, "bucket"), (perm, "perm"), (inv_perm, "inv_perm")):
+        _need(t, nm, torch.int32, (B, H, n_rounds, n))
+    if valid_len is not None:
+        _need(valid_len, "valid_len", torch.int32, (B,))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    a = LshAttnParams(lsh_params(QK, n_buckets, n_rounds, chunk), int(causal), int(no_self),
+                      int(key_norm), float(scale))
+    if out is None:
+        out = torch.empty(QK.shape, dtype=torch.float32, device=QK.device)
+    _need(out, "out", torch.float32, QK.shape)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, H, n))
+    ws, wsb = _workspace(int(_lib.crs_lsh_attn_workspace_size(ctypes.byref(a))), QK.device,
+                         workspace)
+    st = _lib.crs_lsh_attn(ctypes.byref(a), _ptr(QK), _ptr(V), _ptr(bucket), _ptr(perm),
+                           _ptr(inv_perm), _ptr(valid_len), _ptr(out), _ptr(lse), _ptr(ws), wsb,
+                           _stream(stream))
+    _check("crs_lsh_attn", st)
+    return out, lse
+
+
+# ---------------------------------------------------------------- indexer --
+def indexer_topk(q_idx, w, k_idx, topk: int, mode: int = CRS_IDX_PREFILL, k_offsets=None,
+                 max_keys: int = 0, out=None, count=None, workspace=None, stream=None):
+    """Lightning-indexer top-k; returns (idx [rows, topk] int32 ascending, -1 pad; count [rows])."""
+    _need(q_idx, "q_idx", torch.bfloat16)
+    rows, heads, d = q_idx.shape
+    _need(w, "w", torch.float32, (rows, heads))
+    _need(k_idx, "k_idx", torch.bfloat16)
+    if mode == CRS_IDX_DECODE:
+        _need(k_offsets, "k_offsets", torch.int64, (rows + 1,))
+    p = IndexerParams(int(mode), rows, heads, d, int(topk), int(max_keys))
+    if out is None:
+        out = torch.empty((rows, topk), dtype=torch.int32, device=q_idx.device)
+    if count is None:
+        count = torch.empty((rows,), dtype=torch.int32, device=q_idx.device)
+    _need(out, "out", torch.int32, (rows, topk))
+    _need(count, "count", torch.int32, (rows,))
+    ws, wsb = _workspace(int(_lib.crs_indexer_topk_workspace_size(ctypes.byref(p))),
+                         q_idx.device, workspace)
+    st = _lib.crs_indexer_topk(ctypes.byref(p), _ptr(q_idx), _ptr(w), _ptr(k_idx),
+                               _ptr(k_offsets), _ptr(out), _ptr(count), _ptr(ws), wsb,
+                               _stream(stream))
+    _check("crs_indexer_topk", st)
+    return out, count
+
+
+# ----------------------------------------------------------------- blocks --
+def block_describe(K, L: int, rank: int, blk_range=None, mu=None, xi=None, stream=None):
+    """Block descriptors of K [n_seq, T, n_kv, D] bf16 -> (mu, xi) fp32."""
+    _need(K, "K", torch.bfloat16)
+    n_seq, T, n_kv, D = K.shape
+    nfull = T // L
+    b0, b1 = (0, nfull) if blk_range is None else blk_range
+    p = BlockParams(n_seq, n_kv, T, D, int(L), int(rank), int(b0), int(b1))
+    if mu is None:
+        mu = torch.empty((n_seq, n_kv, nfull, D), dtype=torch.float32, device=K.device)
+    if xi is None:
+        xi = torch.empty((n_seq, n_kv, nfull, rank, D), dtype=torch.float32, device=K.device)
+    _need(mu, "mu", torch.float32, (n_seq, n_kv, nfull, D))
+    _need(xi, "xi", torch.float32, (n_seq, n_kv, nfull, rank, D))
+    st = _lib.crs_block_describe(ctypes.byref(p), _ptr(K), _ptr(mu), _ptr(xi), _stream(stream))
+    _check("crs_block_describe", st)
+    return mu, xi
+
+
+def block_select(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=None,
+                 tok=None, count=None, workspace=None, stream=None):
+    """Block-mass selection -> (tok [n_seq, n_kv, top_blocks*L + window], count [n_seq, n_kv])."""
+    _need(Q, "Q", torch.bfloat16)
+    n_seq, n_q, D = Q.shape
+    n_kv, nfull, rank = mu.shape[1], mu.shape[2], xi.shape[3]
+    _need(mu, "mu", torch.float32, (n_seq, n_kv, nfull, D))
+    _need(xi, "xi", torch.float32, (n_seq, n_kv, nfull, rank, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull), n_q,
+                       int(top_blocks), int(window), float(scale))
+    cap = top_blocks * L + window
+    if tok is None:
+        tok = torch.empty((n_seq, n_kv, cap), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((n_seq, n_kv), dtype=torch.int32, device=Q.device)
+    _need(tok, "tok", torch.int32, (n_seq, n_kv, cap))
+    _need(count, "count", torch.int32, (n_seq, n_kv))
+    ws, wsb = _workspace(int(_lib.crs_block_select_workspace_size(ctypes.byref(p))), Q.device,
+                         workspace)
+    st = _lib.crs_block_select(ctypes.byref(p), _ptr(Q), _ptr(mu), _ptr(xi), _ptr(tok),
+                               _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_block_select", st)
+    return tok, count
+
+
+# -------------------------------------------------------------- attention --
+def sparse_attn(Q, K, V, I, kv_base=None, scale=None, n_keys: int = 0, out=None, lse=None,
+                workspace=None, stream=None):
+    """Attention over index lists -> (O [rows, n_q, D] fp32, lse).  Q [rows, n_q, D];
+    K, V [tokens, n_kv, D] (token j of row t at kv_base[t] + j); I [rows, n_lists,
+    max_idx] (n_lists 1 or n_kv)."""
+    _need(Q, "Q", torch.bfloat16)
+    rows, n_q, D = Q.shape
+    _need(K, "K", torch.bfloat16)
+    _need(V, "V", torch.bfloat16, K.shape)
+    n_kv = K.shape[-2]
+    if I.dim() == 2:
+        I = I.view(rows, 1, I.shape[1])
+    _need(I, "I", torch.int32)
+    n_lists, max_idx = I.shape[1], I.shape[2]
+    if kv_base is not None:
+        _need(kv_base, "kv_base", torch.int64, (rows,))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = AttnParams(rows, n_q, n_kv, D, max_idx, n_lists, int(n_keys), float(scale))
+    if out is None:
+        out = torch.empty((rows, n_q, D), dtype=torch.float32, device=Q.device)
+    _need(out, "out", torch.float32, (rows, n_q, D))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (rows, n_q))
+    ws, wsb = _workspace(int(_lib.crs_sparse_attn_workspace_size(ctypes.byref(p))), Q.device,
+                         workspace)
+    st = _lib.crs_sparse_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(kv_base),
+                              _ptr(I), _ptr(out), _ptr(lse), _ptr(ws), wsb, _stream(stream))
+    _check("crs_sparse_attn", st)
+    return out, lse

@@ -1,0 +1,110 @@
+// Library-wide entry points: status strings, version, the device error word.
+#include <mutex>
+#include <string.h>
+#include <vector>
+
+#include "common.cuh"
+
+namespace crs {
+static const char *kKernelNames[K_COUNT] = {
+    "lsh_hash", "lsh_sort", "lsh_chunk_attn", "lsh_combine", "idx_slice_topk", "idx_merge_topk",
+    "sparse_attn", "sparse_attn_merge", "block_describe", "block_score", "block_pick",
+    "lsh_chunk_attn_tc", "idx_prefill_tc", "idx_select", "noalloc"};
+struct PendingEv {
+    int id;
+    cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static bool g_prof_on = false;
+static long long g_launches[K_COUNT];
+static double g_ms[K_COUNT];
+static long long g_timed[K_COUNT];
+static std::vector<PendingEv> g_pending;
+
+void prof_begin(int id, cudaStream_t s, void **ev_start) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_launches[id] += 1;
+    *ev_start = nullptr;
+    if (!g_prof_on) return;
+    cudaEvent_t a;
+    if (cudaEventCreate(&a) != cudaSuccess) return;
+    cudaEventRecord(a, s);
+    *ev_start = a;
+}
+void prof_end(int id, cudaStream_t s, void *ev_start) {
+    if (!ev_start) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b;
+    if (cudaEventCreate(&b) != cudaSuccess) return;
+    cudaEventRecord(b, s);
+    g_pending.push_back({id, static_cast<cudaEvent_t>(ev_start), b});
+}
+}  // namespace crs
+
+extern "C" int crs_profile_set(int enabled) {
+    std::lock_guard<std::mutex> lk(crs::g_prof_mu);
+    crs::g_prof_on = enabled != 0;
+    return CRS_OK;
+}
+
+extern "C" int crs_profile_collect(crs_kernel_stat *out, int max_out, int *n_out) {
+    if (!n_out || (max_out > 0 && !out)) return CRS_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(crs::g_prof_mu);
+    int st = CRS_OK;
+    for (auto &p : crs::g_pending) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+            crs::g_ms[p.id] += ms;
+            crs::g_timed[p.id] += 1;
+        } else {
+            st = CRS_ERR_CUDA;
+        }
+        cudaEventDestroy(p.a);
+        cudaEventDestroy(p.b);
+    }
+    crs::g_pending.clear();
+    int n = 0;
+    for (int k = 0; k < crs::K_COUNT; ++k) {
+        if (crs::g_launches[k] == 0) continue;
+        if (n < max_out) {
+            memset(&out[n], 0, sizeof(crs_kernel_stat));
+            strncpy(out[n].name, crs::kKernelNames[k], sizeof(out[n].name) - 1);
+            out[n].launches = crs::g_launches[k];
+            out[n].timed_launches = crs::g_timed[k];
+            out[n].total_ms = crs::g_ms[k];
+        }
+        ++n;
+        crs::g_launches[k] = 0;
+        crs::g_timed[k] = 0;
+        crs::g_ms[k] = 0.0;
+    }
+    *n_out = n;
+    return st;
+}
+
+extern "C" const char *crs_status_string(int status) {
+    switch (status) {
+        case CRS_OK: return "CRS_OK";
+        case CRS_ERR_INVALID_ARG: return "CRS_ERR_INVALID_ARG";
+        case CRS_ERR_UNSUPPORTED: return "CRS_ERR_UNSUPPORTED";
+        case CRS_ERR_CUDA: return "CRS_ERR_CUDA";
+        case CRS_ERR_NONFINITE: return "CRS_ERR_NONFINITE";
+        case CRS_ERR_TIMEOUT: return "CRS_ERR_TIMEOUT";
+        case CRS_ERR_WORKSPACE: return "CRS_ERR_WORKSPACE";
+        case CRS_ERR_INDEX: return "CRS_ERR_INDEX";
+        default: return "CRS_ERR_UNKNOWN";
+    }
+}
+
+extern "C" int crs_version(void) { return 100; }
+
+extern "C" int crs_get_device_error(void *stream, uint32_t *flags) {
+    if (!flags) return CRS_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CRS_TRY_CUDA(cudaStreamSynchronize(s));
+    uint32_t v = 0, zero = 0;
+    CRS_TRY_CUDA(cudaMemcpyFromSymbol(&v, crs::g_device_error, sizeof(v)));
+    CRS_TRY_CUDA(cudaMemcpyToSymbol(crs::g_device_error, &zero, sizeof(zero)));
+    *flags = v;
+    return CRS_OK;
+}

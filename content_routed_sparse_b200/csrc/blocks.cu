@@ -1,0 +1,479 @@
+// Block-mass selector (COBS-style): block descriptors and block selection, sm_100a.
+//
+// [P5] "COBS 阅读笔记": Eq.(11) (block mean, population covariance), Eq.(16)
+// (rank-r factor xi_i = sqrt(lambda_i) u_i), Eq.(20) and Algorithm 2 (Gram
+// route: eigen-decompose G = Kt Kt^T / L, xi_i = Kt^T w_i / sqrt(L)), Eq.(14)
+// and (19) (second-order log-mass score), Eq.(15)/(6) (GQA group score = sum
+// over the group of each head's softmax over blocks), "可缓存性约束" (the
+// descriptor is computed once, when the block is full).
+#include <math.h>
+
+#include "common.cuh"
+
+namespace crs {
+
+// ---------------------------------------------------------------------------
+// K8: one warp per block.  Keys (bf16) are staged in shared memory; the mean
+// and the Gram matrix are formed in fp32; the L x L symmetric eigenproblem is
+// solved by the cyclic Jacobi method in the parallel "round-robin" ordering
+// (Brent & Luk, 1985): each round applies L/2 disjoint plane rotations, one
+// sweep is L-1 rounds, sweeps repeat until the off-diagonal mass is below
+// 1e-12 of the total (at most 15 sweeps).  Lane k owns row/column k.
+// ---------------------------------------------------------------------------
+constexpr int kBdWarps = 4;
+constexpr int kBdMaxL = 32;
+constexpr int kBdD = 128;
+
+struct BdWarpSmem {
+    __nv_bfloat16 k[kBdMaxL][kBdD];
+    float mu[kBdD];
+    float g[kBdMaxL][kBdMaxL + 1];
+    float v[kBdMaxL][kBdMaxL + 1];
+    float rc[kBdMaxL], rs[kBdMaxL];
+    int partner[kBdMaxL];
+};
+
+__global__ void __launch_bounds__(kBdWarps * 32)
+block_describe_kernel(const __nv_bfloat16 *__restrict__ K, float *__restrict__ mu_out,
+                      float *__restrict__ xi_out, int n_kv, int T, int L, int rank, int blk_begin,
+                      int n_blk, int n_full) {
+    extern __shared__ __align__(16) unsigned char bd_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BdWarpSmem &S = reinterpret_cast<BdWarpSmem *>(bd_smem)[warp];
+    const long long item = (long long)blockIdx.x * kBdWarps + warp;
+    const int sh = blockIdx.y;                 // seq * n_kv + h
+    if (item >= n_blk) return;
+    const int blk = blk_begin + (int)item;
+    const int seq = sh / n_kv, h = sh - seq * n_kv;
+    const size_t tok0 = (size_t)seq * T + (size_t)blk * L;
+
+    // stage the block's keys: L rows x 256 B
+    for (int e = lane; e < L * 16; e += 32) {
+        const int r = e >> 4, c = e & 15;
+        const uint4 v = *reinterpret_cast<const uint4 *>(K + ((tok0 + r) * n_kv + h) * kBdD + c * 8);
+        *reinterpret_cast<uint4 *>(&S.k[r][c * 8]) = v;
+    }
+    __syncwarp();
+    const float invL = 1.0f / (float)L;
+    for (int d = lane; d < kBdD; d += 32) {
+        float acc = 0.0f;
+        for (int r = 0; r < L; ++r) acc += __bfloat162float(S.k[r][d]);
+        S.mu[d] = acc * invL;
+    }
+    __syncwarp();
+    // Gram row `lane`: G[i][j] = (1/L) sum_d Kt[i][d] Kt[j][d]
+    if (lane < L) {
+        float grow[kBdMaxL];
+#pragma unroll
+        for (int j = 0; j < kBdMaxL; ++j) grow[j] = 0.0f;
+        for (int d = 0; d < kBdD; ++d) {
+            const float md = S.mu[d];
+            const float ki = __bfloat162float(S.k[lane][d]) - md;
+#pragma unroll
+            for (int j = 0; j < kBdMaxL; ++j)
+                if (j < L) grow[j] = fmaf(ki, __bfloat162float(S.k[j][d]) - md, grow[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < kBdMaxL; ++j)
+            if (j < L) {
+                S.g[lane][j] = grow[j] * invL;
+                S.v[lane][j] = (lane == j) ? 1.0f : 0.0f;
+            }
+    }
+    __syncwarp();
+
+    // ---- parallel cyclic Jacobi
+    const int nm1 = L - 1;                    // L even: players 0..L-1, player L-1 fixed
+    for (int sweep = 0; sweep < 15; ++sweep) {
+        float off = 0.0f, tot = 0.0f;
+        if (lane < L)
+            for (int j = 0; j < L; ++j) {
+                const float x = S.g[lane][j];
+                tot += x * x;
+                if (j != lane) off += x * x;
+            }
+        off = warp_sum(off);
+        tot = warp_sum(tot);
+        if (off <= 1e-12f * tot || off == 0.0f) break;
+        for (int t = 0; t < nm1; ++t) {
+            if (lane < L) {
+                int q;
+                if (lane == nm1) {
+                    // the p with 2p = t (mod L-1)
+                    q = 0;
+                    for (int p = 0; p < nm1; ++p)
+                        if ((2 * p) % nm1 == t % nm1) q = p;
+                } else {
+                    q = ((t - lane) % nm1 + nm1) % nm1;
+                    if (q == lane) q = nm1;
+                }
+                S.partner[lane] = q;
+                if (lane < q) {
+                    const float app = S.g[lane][lane], aqq = S.g[q][q], apq = S.g[lane][q];
+                    float c = 1.0f, s = 0.0f;
+                    if (apq != 0.0f && fabsf(apq) > 1e-30f * (fabsf(app) + fabsf(aqq))) {
+                        const float theta = (aqq - app) / (2.0f * apq);
+                        float tt;
+                        if (fabsf(theta) > 1e18f)
+                            tt = 0.5f / theta;
+                        else
+                            tt = copysignf(1.0f, theta) / (fabsf(theta) + sqrtf(theta * theta + 1.0f));
+                        c = rsqrtf(tt * tt + 1.0f);
+                        s = tt * c;
+                    }
+                    S.rc[lane] = c;
+                    S.rs[lane] = s;
+                }
+            }
+            __syncwarp();
+            // columns: A <- A J, V <- V J (lane = row k)
+            if (lane < L) {
+                for (int p = 0; p < L; ++p) {
+                    const int q = S.partner[p];
+                    if (p < q) {
+                        const float c = S.rc[p], s = S.rs[p];
+                        const float akp = S.g[lane][p], akq = S.g[lane][q];
+                        S.g[lane][p] = c * akp - s * akq;
+                        S.g[lane][q] = s * akp + c * akq;
+                        const float vkp = S.v[lane][p], vkq = S.v[lane][q];
+                        S.v[lane][p] = c * vkp - s * vkq;
+                        S.v[lane][q] = s * vkp + c * vkq;
+                    }
+                }
+            }
+            __syncwarp();
+            // rows: A <- J^T A (lane = column k)
+            if (lane < L) {
+                for (int p = 0; p < L; ++p) {
+                    const int q = S.partner[p];
+                    if (p < q) {
+                        const float c = S.rc[p], s = S.rs[p];
+                        const float apk = S.g[p][lane], aqk = S.g[q][lane];
+                        S.g[p][lane] = c * apk - s * aqk;
+                        S.g[q][lane] = s * apk + c * aqk;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+
+    // ---- the `rank` largest eigenvalues (ties: lower index), xi = Kt^T w / sqrt(L)
+    float lam = (lane < L) ? S.g[lane][lane] : -INFINITY;
+    bool taken = false;
+    const float rs_L = rsqrtf((float)L);
+    const size_t dbase = ((size_t)sh * n_full + blk);
+    for (int e = 0; e < rank; ++e) {
+        float best = taken ? -INFINITY : lam;
+        int bi = taken ? 0x7fffffff : lane;
+        if (lane >= L) { best = -INFINITY; bi = 0x7fffffff; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+        }
+        if (lane == bi) taken = true;
+        float *xo = xi_out + (dbase * rank + e) * kBdD;
+        if (e >= L || bi >= L) {
+            for (int d = lane; d < kBdD; d += 32) xo[d] = 0.0f;
+            continue;
+        }
+        for (int d = lane; d < kBdD; d += 32) {
+            const float md = S.mu[d];
+            float acc = 0.0f;
+            for (int r = 0; r < L; ++r) acc = fmaf(__bfloat162float(S.k[r][d]) - md, S.v[r][bi], acc);
+            xo[d] = acc * rs_L;
+        }
+    }
+    for (int d = lane; d < kBdD; d += 32) mu_out[dbase * kBdD + d] = S.mu[d];
+}
+
+// ---------------------------------------------------------------------------
+// K9a: second-order scores s_{g,b}.  One thread per (block, query head) of a
+// tile of blocks; descriptors and the scaled queries are staged in shared
+// memory (rows padded by one float against bank conflicts).
+// ---------------------------------------------------------------------------
+constexpr int kBsThreads = 128;
+
+__global__ void __launch_bounds__(kBsThreads)
+block_score_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ mu,
+                   const float *__restrict__ xi, float *__restrict__ sc_out, int n_kv, int n_q,
+                   int G, int rank, int n_full, float scale) {
+    extern __shared__ float bs_smem[];
+    const int nbt = kBsThreads / G;             // blocks per CTA
+    const int DP = kBdD + 1;
+    float *sq = bs_smem;                        // [G][DP]
+    float *sd = sq + G * DP;                    // [nbt][(1+rank)][DP]
+    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
+    const int b0 = blockIdx.x * nbt;
+    const int nb = min(nbt, n_full - b0);
+    for (int e = threadIdx.x; e < G * kBdD; e += kBsThreads) {
+        const int g = e / kBdD, d = e - g * kBdD;
+        sq[g * DP + d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+    }
+    const int rows = 1 + rank;
+    for (int e = threadIdx.x; e < nb * rows * kBdD; e += kBsThreads) {
+        const int bl = e / (rows * kBdD), rem = e - bl * rows * kBdD;
+        const int rr = rem / kBdD, d = rem - rr * kBdD;
+        const size_t blk = (size_t)sh * n_full + b0 + bl;
+        sd[(bl * rows + rr) * DP + d] =
+            (rr == 0) ? mu[blk * kBdD + d] : xi[(blk * rank + (rr - 1)) * kBdD + d];
+    }
+    __syncthreads();
+    const int bl = threadIdx.x / G, g = threadIdx.x - bl * G;
+    if (bl >= nb) return;
+    const float *q = sq + g * DP;
+    const float *dsc = sd + bl * rows * DP;
+    float lin = 0.0f;
+    for (int d = 0; d < kBdD; ++d) lin = fmaf(q[d], dsc[d], lin);
+    float quad = 0.0f;
+    for (int e = 0; e < rank; ++e) {
+        float p = 0.0f;
+        const float *x = dsc + (1 + e) * DP;
+        for (int d = 0; d < kBdD; ++d) p = fmaf(q[d], x[d], p);
+        quad = fmaf(p, p, quad);
+    }
+    sc_out[((size_t)sh * G + g) * n_full + b0 + bl] = fmaf(0.5f, quad, lin);
+}
+
+// ---------------------------------------------------------------------------
+// K9b: group softmax sum, top blocks, token list.  One CTA per (seq, KV head).
+// ---------------------------------------------------------------------------
+constexpr int kSelT = 512;
+
+__device__ float block_reduce_max(float v, float *sh) {
+    v = warp_max(v);
+    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = -INFINITY;
+    for (int w = 0; w < kSelT / 32; ++w) r = fmaxf(r, sh[w]);
+    __syncthreads();
+    return r;
+}
+__device__ float block_reduce_sum(float v, float *sh) {
+    v = warp_sum(v);
+    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = 0.0f;
+    for (int w = 0; w < kSelT / 32; ++w) r += sh[w];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kSelT)
+block_pick_kernel(const float *__restrict__ sc, int32_t *__restrict__ tok, int32_t *__restrict__ cnt,
+                  int G, int n_full, int L, int T, int top, int window, int cap) {
+    extern __shared__ __align__(16) unsigned char bp_smem[];
+    float *score = reinterpret_cast<float *>(bp_smem);                 // [n_full]
+    uint32_t *keyv = reinterpret_cast<uint32_t *>(score + n_full);      // [n_full]
+    int *sel = reinterpret_cast<int *>(keyv + n_full);                  // [top]
+    __shared__ float red[kSelT / 32];
+    __shared__ int hist[256];
+    __shared__ int bc[2];
+    __shared__ int scan_sh[kSelT / 32 + 1];
+    const int sh = blockIdx.x;
+    for (int b = threadIdx.x; b < n_full; b += kSelT) score[b] = 0.0f;
+    __syncthreads();
+    for (int g = 0; g < G; ++g) {
+        const float *s = sc + ((size_t)sh * G + g) * n_full;
+        float m = -INFINITY;
+        for (int b = threadIdx.x; b < n_full; b += kSelT) m = fmaxf(m, s[b]);
+        m = block_reduce_max(m, red);
+        float z = 0.0f;
+        for (int b = threadIdx.x; b < n_full; b += kSelT) z += __expf(s[b] - m);
+        z = block_reduce_sum(z, red);
+        const float iz = 1.0f / z;
+        for (int b = threadIdx.x; b < n_full; b += kSelT) score[b] += __expf(s[b] - m) * iz;
+        __syncthreads();
+    }
+    for (int b = threadIdx.x; b < n_full; b += kSelT) keyv[b] = score_key(score[b]);
+    __syncthreads();
+    // exact top `top` by (score desc, block asc): 4-pass radix select on the keys
+    const int k = min(top, n_full);
+    uint32_t prefix = 0, mask = 0;
+    int remaining = k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int b = threadIdx.x; b < 256; b += kSelT) hist[b] = 0;
+        __syncthreads();
+        for (int b = threadIdx.x; b < n_full; b += kSelT) {
+            const uint32_t kk = keyv[b];
+            if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int acc = 0;
+            for (int d = 255; d >= 0; --d) {
+                if (acc + hist[d] >= remaining) { bc[0] = d; bc[1] = remaining - acc; break; }
+                acc += hist[d];
+            }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)bc[0] << shift;
+        mask |= 0xffu << shift;
+        remaining = bc[1];
+        __syncthreads();
+    }
+    const uint32_t Tk = prefix;
+    // compaction in block order; equal keys: the first `remaining` blocks
+    int out_base = 0, eq_base = 0;
+    for (int t0 = 0; t0 < n_full; t0 += kSelT) {
+        const int b = t0 + threadIdx.x;
+        const uint32_t kk = (b < n_full) ? keyv[b] : 0u;
+        const bool gt = (b < n_full) && kk > Tk;
+        const bool eq = (b < n_full) && kk == Tk;
+        // exclusive scans via warp ballots
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        const unsigned be = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) scan_sh[w] = __popc(be);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int s = 0;
+            for (int i = 0; i < kSelT / 32; ++i) { const int c = scan_sh[i]; scan_sh[i] = s; s += c; }
+            scan_sh[kSelT / 32] = s;
+        }
+        __syncthreads();
+        const int eq_rank = eq_base + scan_sh[w] + __popc(be & ((1u << lane) - 1u));
+        const int eq_tot = scan_sh[kSelT / 32];
+        __syncthreads();
+        const bool take = gt || (eq && eq_rank < remaining);
+        const unsigned bt = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) scan_sh[w] = __popc(bt);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int s = 0;
+            for (int i = 0; i < kSelT / 32; ++i) { const int c = scan_sh[i]; scan_sh[i] = s; s += c; }
+            scan_sh[kSelT / 32] = s;
+        }
+        __syncthreads();
+        if (take) sel[out_base + scan_sh[w] + __popc(bt & ((1u << lane) - 1u))] = b;
+        out_base += scan_sh[kSelT / 32];
+        eq_base += eq_tot;
+        __syncthreads();
+    }
+    // token list: kept blocks' positions before the window (blocks ascending),
+    // then the window [wstart, T)
+    int *tstart = sel + top;                 // [top] first output slot of each kept block
+    const int wstart = max(0, T - window);
+    int32_t *to = tok + (size_t)sh * cap;
+    if (threadIdx.x == 0) {
+        int pos = 0;
+        for (int i = 0; i < out_base; ++i) {
+            tstart[i] = pos;
+            pos += min(L, max(0, wstart - sel[i] * L));
+        }
+        bc[0] = pos;
+    }
+    __syncthreads();
+    const int nblk_tok = bc[0];
+    for (int e = threadIdx.x; e < out_base * L; e += kSelT) {
+        const int i = e / L, r = e - i * L;
+        const int b = sel[i];
+        if (b * L + r < wstart) to[tstart[i] + r] = b * L + r;
+    }
+    const int nwin = T - wstart;
+    for (int i = threadIdx.x; i < nwin; i += kSelT) to[nblk_tok + i] = wstart + i;
+    const int total = nblk_tok + nwin;
+    for (int i = total + threadIdx.x; i < cap; i += kSelT) to[i] = -1;
+    if (threadIdx.x == 0) cnt[sh] = total;
+}
+
+static int bd_validate(const crs_block_params *p) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    if (p->n_seq < 1 || p->n_kv < 1 || p->T < 1) return CRS_ERR_INVALID_ARG;
+    if (p->D != kBdD) return CRS_ERR_UNSUPPORTED;
+    if (p->L < 2 || p->L > kBdMaxL || (p->L & 1)) return CRS_ERR_UNSUPPORTED;
+    if (p->rank < 1 || p->rank > 8 || p->rank > p->L) return CRS_ERR_INVALID_ARG;
+    return CRS_OK;
+}
+
+}  // namespace crs
+
+using namespace crs;
+
+extern "C" int crs_block_describe(const crs_block_params *p, const void *K, float *mu, float *xi,
+                                  void *stream) {
+    int st = bd_validate(p);
+    if (st) return st;
+    if (!K || !mu || !xi) return CRS_ERR_INVALID_ARG;
+    const int n_full = p->T / p->L;
+    if (p->blk_begin < 0 || p->blk_end > n_full || p->blk_begin > p->blk_end)
+        return CRS_ERR_INVALID_ARG;
+    const int n_blk = p->blk_end - p->blk_begin;
+    if (n_blk == 0) return CRS_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t smem = sizeof(BdWarpSmem) * kBdWarps;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_describe_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid(ceil_div(n_blk, kBdWarps), p->n_seq * p->n_kv);
+    {
+        ProfScope _ps(K_BLK_DESCRIBE, s);
+        block_describe_kernel<<<grid, kBdWarps * 32, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(K), mu, xi, p->n_kv, p->T, p->L, p->rank, p->blk_begin,
+            n_blk, n_full);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+
+static int bs_validate(const crs_block_sel_params *p) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    crs_block_params b = p->b;
+    b.blk_begin = 0;
+    b.blk_end = 0;
+    int st = bd_validate(&b);
+    if (st) return st;
+    if (p->n_q < 1 || p->n_q % p->b.n_kv) return CRS_ERR_INVALID_ARG;
+    const int G = p->n_q / p->b.n_kv;
+    if (G > 16 || (16 % G) != 0) return CRS_ERR_UNSUPPORTED;
+    const int n_full = p->b.T / p->b.L;
+    if (n_full < 1 || n_full > 8192) return CRS_ERR_UNSUPPORTED;
+    if (p->top_blocks < 1 || p->top_blocks > n_full) return CRS_ERR_INVALID_ARG;
+    if (p->window < 0 || p->window > p->b.T) return CRS_ERR_INVALID_ARG;
+    return CRS_OK;
+}
+
+extern "C" size_t crs_block_select_workspace_size(const crs_block_sel_params *p) {
+    if (bs_validate(p)) return 0;
+    const size_t n_full = p->b.T / p->b.L;
+    return (size_t)p->b.n_seq * p->n_q * n_full * sizeof(float);
+}
+
+extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, const float *mu,
+                                const float *xi, int32_t *tok_idx, int32_t *tok_count, void *ws,
+                                size_t ws_bytes, void *stream) {
+    int st = bs_validate(p);
+    if (st) return st;
+    if (!Q || !mu || !xi || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_block_select_workspace_size(p);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int G = p->n_q / p->b.n_kv;
+    const int n_full = p->b.T / p->b.L;
+    const int nbt = kBsThreads / G;
+    const size_t smem_a = ((size_t)G * (kBdD + 1) + (size_t)nbt * (1 + p->b.rank) * (kBdD + 1)) * 4;
+    if (smem_a > 227 * 1024) return CRS_ERR_UNSUPPORTED;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a));
+    float *sc = static_cast<float *>(ws);
+    dim3 ga(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv);
+    {
+        ProfScope _ps(K_BLK_SCORE, s);
+        block_score_kernel<<<ga, kBsThreads, smem_a, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu, xi,
+                                                          sc, p->b.n_kv, p->n_q, G, p->b.rank, n_full,
+                                                          p->scale);
+    }
+    CRS_CHECK_LAUNCH();
+    const int cap = p->top_blocks * p->b.L + p->window;
+    const size_t smem_b = (size_t)n_full * 8 + (size_t)p->top_blocks * 8;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_pick_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b));
+    {
+        ProfScope _ps(K_BLK_PICK, s);
+        block_pick_kernel<<<p->b.n_seq * p->b.n_kv, kSelT, smem_b, s>>>(
+            sc, tok_idx, tok_count, G, n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}

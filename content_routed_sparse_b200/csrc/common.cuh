@@ -1,0 +1,115 @@
+// Shared device helpers for libcrs kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "crs.h"
+
+namespace crs {
+
+// Per-device error word (CRS_DEVERR_* bits), read and cleared by crs_get_device_error.
+// The library is built as one translation unit (libcrs.cu), so this is its only definition.
+__device__ uint32_t g_device_error = 0;
+
+__device__ __forceinline__ void raise_error(uint32_t bit) { atomicOr(&g_device_error, bit); }
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Order-preserving map of an fp32 score to uint32: a > b  <=>  key(a) > key(b)
+// for non-NaN a, b, with -0 and +0 mapped to the same key.  NaN maps to 0,
+// below every number.
+__device__ __forceinline__ uint32_t score_key(float s) {
+    if (s != s) return 0u;
+    s = s + 0.0f;  // -0 -> +0
+    uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ long long ceil_div_ll(long long a, long long b) {
+    return (a + b - 1) / b;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte asynchronous global -> shared copy (sm_80+ path, valid on sm_100a).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async16_zfill(void *smem, const void *gmem, bool valid) {
+    int src_size = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
+                 "l"(gmem), "r"(src_size));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+}  // namespace crs
+
+// Host-side helpers shared by the entry points.
+#define CRS_TRY_CUDA(expr)                          \
+    do {                                            \
+        cudaError_t _e = (expr);                    \
+        if (_e != cudaSuccess) return CRS_ERR_CUDA; \
+    } while (0)
+
+#define CRS_CHECK_LAUNCH()                                   \
+    do {                                                     \
+        if (cudaGetLastError() != cudaSuccess) return CRS_ERR_CUDA; \
+    } while (0)
+
+// ---------------------------------------------------------------------------
+// Launch tracing: every kernel launch site opens a ProfScope.  Launches are
+// always counted; while tracing is enabled (crs_profile_set) each launch is
+// also bracketed by a pair of CUDA events recorded on its own stream, and
+// crs_profile_collect turns them into per-kernel device times.
+// ---------------------------------------------------------------------------
+namespace crs {
+enum KernelId {
+    K_LSH_HASH = 0, K_LSH_SORT, K_LSH_ATTN, K_LSH_COMBINE, K_IDX_SLICE, K_IDX_MERGE,
+    K_SA_MAIN, K_SA_MERGE, K_BLK_DESCRIBE, K_BLK_SCORE, K_BLK_PICK, K_LSH_ATTN_TC,
+    K_IDX_PREFILL_TC, K_IDX_SELECT, K_NOALLOC, K_COUNT
+};
+void prof_begin(int id, cudaStream_t s, void **ev_start);
+void prof_end(int id, cudaStream_t s, void *ev_start);
+struct ProfScope {
+    int id;
+    cudaStream_t s;
+    void *ev;
+    ProfScope(int id_, cudaStream_t s_) : id(id_), s(s_), ev(nullptr) { prof_begin(id, s, &ev); }
+    ~ProfScope() { prof_end(id, s, ev); }
+};
+}  // namespace crs

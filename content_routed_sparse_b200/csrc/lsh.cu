@@ -1,0 +1,476 @@
+// LSH routing and chunked LSH attention (Reformer-style), sm_100a.
+//
+// [P1] PaperTrace 2.1.1 "哈希与聚类" §2.1 Eq.(4) (bucket = argmax [xR; -xR]),
+// §2.1-2.2 (stable sort on (bucket, position) -> pi, pi^-1; chunks of m slots
+// attend to themselves and the previous chunk; causal and padding masks on
+// original positions), "重复候选和归一化" (a pair counts once, in its first
+// round; rounds merge by log-sum-exp weights).
+#include <math.h>
+
+#include "common.cuh"
+
+namespace crs {
+
+// --------------------------------------------------------------------------
+// K1: hash.  One thread per (token, round).  R_{h,r} and a tile of 128 token
+// rows are staged in shared memory; every u_k is a chain of fp32 FMAs over
+// the head dim in increasing index order (bit-reproducible bucket ids).
+// --------------------------------------------------------------------------
+constexpr int kHashTok = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(kHashTok) lsh_hash_kernel(const T *__restrict__ X,
+                                                            const float *__restrict__ R,
+                                                            int32_t *__restrict__ bucket, int H,
+                                                            int n, int d, int nb, int rounds) {
+    extern __shared__ float sm[];
+    const int half = nb / 2;
+    const int bh = blockIdx.z, r = blockIdx.y, h = bh % H;
+    float *Rs = sm;               // [d][half]
+    float *Xs = sm + d * half;    // [kHashTok][d+1]
+    const float *Rg = R + ((size_t)h * rounds + r) * (size_t)d * half;
+    for (int e = threadIdx.x; e < d * half; e += blockDim.x) Rs[e] = Rg[e];
+    const int i0 = blockIdx.x * kHashTok;
+    for (int e = threadIdx.x; e < kHashTok * d; e += blockDim.x) {
+        const int t = e / d, k = e - t * d, i = i0 + t;
+        Xs[t * (d + 1) + k] = (i < n) ? to_f32(X[((size_t)bh * n + i) * d + k]) : 0.0f;
+    }
+    __syncthreads();
+    const int i = i0 + threadIdx.x;
+    if (i >= n) return;
+    const float *x = Xs + threadIdx.x * (d + 1);
+    float bp = 0.0f, bn = 0.0f;
+    int ap = 0, an = 0;
+    for (int k0 = 0; k0 < half; k0 += 32) {
+        float u[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) u[j] = 0.0f;
+        for (int t = 0; t < d; ++t) {
+            const float xv = x[t];
+            const float *rr = Rs + t * half + k0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (k0 + j < half) u[j] = __fmaf_rn(xv, rr[j], u[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int k = k0 + j;
+            if (k < half) {
+                if (k == 0 || u[j] > bp) { bp = u[j]; ap = k; }
+                const float nu = -u[j];
+                if (k == 0 || nu > bn) { bn = nu; an = k; }
+            }
+        }
+    }
+    // first maximum of [u ; -u] in index order: the +u group precedes the -u group
+    const int arg = (bp >= bn) ? ap : half + an;
+    bucket[((size_t)bh * rounds + r) * n + i] = arg;
+}
+
+// --------------------------------------------------------------------------
+// K2: stable counting sort of one (b, h, round) segment per CTA.
+// Histogram -> exclusive scan (bucket bases) -> tiles of blockDim positions
+// in increasing order; inside a tile, the rank of a position among equal
+// buckets comes from __match_any_sync within the warp plus the counts of
+// earlier warps, so equal buckets keep position order (the (bucket, pos) key).
+// --------------------------------------------------------------------------
+constexpr int kSortThreads = 512;
+
+__global__ void __launch_bounds__(kSortThreads) lsh_sort_kernel(const int32_t *__restrict__ bucket,
+                                                                 int32_t *__restrict__ perm,
+                                                                 int32_t *__restrict__ inv_perm,
+                                                                 int n, int nb) {
+    extern __shared__ int smi[];
+    constexpr int NW = kSortThreads / 32;
+    int *base = smi;              // [nb]
+    int *running = base + nb;     // [nb]
+    int *wcnt = running + nb;     // [NW][nb]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t seg = blockIdx.x;
+    const int32_t *bk = bucket + seg * n;
+    int32_t *pm = perm + seg * n;
+    int32_t *ip = inv_perm + seg * n;
+    for (int e = tid; e < nb; e += kSortThreads) { base[e] = 0; running[e] = 0; }
+    for (int e = tid; e < NW * nb; e += kSortThreads) wcnt[e] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kSortThreads) {
+        const int b = bk[i];
+        if (b >= 0 && b < nb) atomicAdd(&base[b], 1);
+        else raise_error(CRS_DEVERR_INDEX);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int per = (nb + 31) / 32, b0 = lane * per, b1 = min(b0 + per, nb);
+        int s = 0;
+        for (int b = b0; b < b1; ++b) s += base[b];
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int excl = incl - s;
+        for (int b = b0; b < b1; ++b) { const int c = base[b]; base[b] = excl; excl += c; }
+    }
+    __syncthreads();
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int t0 = 0; t0 < n; t0 += kSortThreads) {
+        const int i = t0 + tid;
+        int b = (i < n) ? bk[i] : -1;
+        if (b >= nb) b = -1;
+        const bool valid = b >= 0;
+        const unsigned active = __ballot_sync(0xffffffffu, valid);
+        int rank = 0, cnt = 0;
+        if (valid) {
+            const unsigned peers = __match_any_sync(active, b);
+            rank = __popc(peers & lt_mask);
+            cnt = __popc(peers);
+            if (rank == 0) wcnt[warp * nb + b] = cnt;
+        }
+        __syncthreads();
+        if (valid) {
+            int off = 0;
+            for (int w = 0; w < warp; ++w) off += wcnt[w * nb + b];
+            const int slot = base[b] + running[b] + off + rank;
+            pm[slot] = i;
+            ip[i] = slot;
+        }
+        __syncthreads();
+        if (valid && rank == 0) { atomicAdd(&running[b], cnt); wcnt[warp * nb + b] = 0; }
+        __syncthreads();
+    }
+}
+
+// --------------------------------------------------------------------------
+// K3 (CUDA-core path): one CTA per (chunk, round, b*h).  Keys = the slots of
+// the previous and the own chunk, gathered through perm into shared memory;
+// each warp owns query rows of the chunk; lanes split the keys for the
+// logits, then split the head dim for P.V.  Masks per pair: same bucket in
+// this round, causal / no-self / padding on original positions, and "not an
+// edge of an earlier round" (a pair is counted in its first round only).
+// Writes o_r (normalised, fp32) and lse_r at the ORIGINAL position.
+// --------------------------------------------------------------------------
+constexpr int kAttnWarps = 8;
+constexpr int kMaxRounds = 8;
+
+template <typename T, int DH>
+__global__ void __launch_bounds__(kAttnWarps * 32)
+lsh_chunk_attn_kernel(const T *__restrict__ QK, const T *__restrict__ V,
+                      const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
+                      const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
+                      float *__restrict__ o_ws, float *__restrict__ lse_ws, int H, int n, int m,
+                      int rounds, int causal, int no_self, int key_norm, float scale) {
+    extern __shared__ float smf[];
+    const int c = blockIdx.x, r = blockIdx.y, bh = blockIdx.z;
+    const int b = bh / H;
+    const int vl = valid_len ? valid_len[b] : n;
+    const int ks0 = max(0, (c - 1) * m), ks1 = min((c + 1) * m, n);
+    const int nk = ks1 - ks0;                    // <= 2m
+    const int qs0 = c * m, qs1 = min(qs0 + m, n);
+    const int KM = 2 * m;
+    float *Ks = smf;                             // [KM][DH+1]
+    float *Vs = Ks + KM * (DH + 1);              // [KM][DH]
+    float *inv_norm = Vs + KM * DH;              // [KM]
+    float *prob = inv_norm + KM;                 // [kAttnWarps][KM]
+    int *kpos = reinterpret_cast<int *>(prob + kAttnWarps * KM);  // [KM]
+    int *kbkt = kpos + KM;                       // [KM]
+    int *pinfo = kbkt + KM;                      // [KM][kMaxRounds-1][2] (slot, bucket) of earlier rounds
+
+    const size_t seg_r = ((size_t)bh * rounds + r) * n;
+    const int32_t *pm = perm + seg_r;
+    const int32_t *bkr = bucket + seg_r;
+    const T *Qb = QK + (size_t)bh * n * DH;
+    const T *Vb = V + (size_t)bh * n * DH;
+    const int tid = threadIdx.x;
+    for (int j = tid; j < nk; j += blockDim.x) {
+        int pos = pm[ks0 + j];
+        int bkt;
+        if (pos < 0 || pos >= n) {            // a caller-supplied permutation out of range
+            raise_error(CRS_DEVERR_INDEX);
+            pos = 0;
+            bkt = -1;                         // matches no query: the key is never used
+        } else {
+            bkt = bkr[pos];
+        }
+        kpos[j] = pos;
+        kbkt[j] = bkt;
+        for (int rr = 0; rr < r; ++rr) {
+            const size_t seg = ((size_t)bh * rounds + rr) * n;
+            pinfo[(j * (kMaxRounds - 1) + rr) * 2 + 0] = inv_perm[seg + pos];
+            pinfo[(j * (kMaxRounds - 1) + rr) * 2 + 1] = bucket[seg + pos];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < nk * DH; e += blockDim.x) {
+        const int j = e / DH, k = e - j * DH;
+        const size_t g = (size_t)kpos[j] * DH + k;
+        Ks[j * (DH + 1) + k] = to_f32(Qb[g]);
+        Vs[j * DH + k] = to_f32(Vb[g]);
+    }
+    __syncthreads();
+    for (int j = tid; j < nk; j += blockDim.x) {
+        float ss = 0.0f;
+        for (int k = 0; k < DH; ++k) ss = fmaf(Ks[j * (DH + 1) + k], Ks[j * (DH + 1) + k], ss);
+        inv_norm[j] = key_norm ? (ss > 0.0f ? rsqrtf(ss) : 0.0f) : 1.0f;
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5, lane = tid & 31;
+    float *pw = prob + warp * KM;
+    for (int qs = qs0 + warp; qs < qs1; qs += kAttnWarps) {
+        const int jq = qs - ks0;                 // the query row is one of the keys
+        const int pos_i = kpos[jq];
+        float *o_out = o_ws + (((size_t)r * gridDim.z + bh) * n + pos_i) * DH;
+        float *l_out = lse_ws + ((size_t)r * gridDim.z + bh) * n + pos_i;
+        if (pos_i >= vl) {
+            for (int k = lane; k < DH; k += 32) o_out[k] = 0.0f;
+            if (lane == 0) *l_out = -INFINITY;
+            continue;
+        }
+        const int bk_i = kbkt[jq];
+        int ps[kMaxRounds - 1], pb[kMaxRounds - 1];
+#pragma unroll
+        for (int rr = 0; rr < kMaxRounds - 1; ++rr) {
+            if (rr < r) {
+                ps[rr] = pinfo[(jq * (kMaxRounds - 1) + rr) * 2 + 0] / m;
+                pb[rr] = pinfo[(jq * (kMaxRounds - 1) + rr) * 2 + 1];
+            }
+        }
+        float mx = -INFINITY;
+        for (int j = lane; j < nk; j += 32) {
+            const int pj = kpos[j];
+            bool ok = (kbkt[j] == bk_i) && (pj < vl) && !(causal && pj > pos_i) &&
+                      !(no_self && pj == pos_i);
+#pragma unroll
+            for (int rr = 0; rr < kMaxRounds - 1; ++rr) {
+                if (rr < r && ok) {
+                    const int cj = pinfo[(j * (kMaxRounds - 1) + rr) * 2 + 0] / m;
+                    const int bj = pinfo[(j * (kMaxRounds - 1) + rr) * 2 + 1];
+                    if (bj == pb[rr] && (cj == ps[rr] || cj == ps[rr] - 1)) ok = false;
+                }
+            }
+            float s = -INFINITY;
+            if (ok) {
+                float dot = 0.0f;
+                const float *kr = Ks + j * (DH + 1);
+                const float *qr = Ks + jq * (DH + 1);
+#pragma unroll 16
+                for (int k = 0; k < DH; ++k) dot = fmaf(qr[k], kr[k], dot);
+                s = scale * dot * inv_norm[j];
+                mx = fmaxf(mx, s);
+            }
+            pw[j] = s;
+        }
+        mx = warp_max(mx);
+        __syncwarp();
+        if (mx == -INFINITY) {
+            for (int k = lane; k < DH; k += 32) o_out[k] = 0.0f;
+            if (lane == 0) *l_out = -INFINITY;
+            __syncwarp();
+            continue;
+        }
+        float sum = 0.0f;
+        for (int j = lane; j < nk; j += 32) {
+            const float p = (pw[j] == -INFINITY) ? 0.0f : __expf(pw[j] - mx);
+            pw[j] = p;
+            sum += p;
+        }
+        sum = warp_sum(sum);
+        __syncwarp();
+        float acc[DH / 32 > 0 ? DH / 32 : 1];
+#pragma unroll
+        for (int u = 0; u < DH / 32; ++u) acc[u] = 0.0f;
+        for (int j = 0; j < nk; ++j) {
+            const float p = pw[j];
+            if (p != 0.0f) {
+#pragma unroll
+                for (int u = 0; u < DH / 32; ++u) acc[u] = fmaf(p, Vs[j * DH + lane + 32 * u], acc[u]);
+            }
+        }
+        const float inv = 1.0f / sum;
+#pragma unroll
+        for (int u = 0; u < DH / 32; ++u) o_out[lane + 32 * u] = acc[u] * inv;
+        if (lane == 0) *l_out = mx + logf(sum);
+        __syncwarp();
+    }
+}
+
+// --------------------------------------------------------------------------
+// K4: merge the rounds.  One warp per (b*h, position):
+//   LSE = log sum_r exp(lse_r),  O = sum_r exp(lse_r - LSE) o_r.
+// Padded positions and queries with no edge in any round give 0 / -inf.
+// --------------------------------------------------------------------------
+template <int DH>
+__global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
+                                   const int32_t *__restrict__ valid_len, float *__restrict__ O,
+                                   float *__restrict__ lse_out, int BH, int H, int n, int rounds) {
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= BH * n) return;
+    const int bh = gw / n, pos = gw - bh * n;
+    const int vl = valid_len ? valid_len[bh / H] : n;
+    float l[kMaxRounds];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        l[r] = (r < rounds) ? lse_ws[((size_t)r * BH + bh) * n + pos] : -INFINITY;
+        mx = fmaxf(mx, l[r]);
+    }
+    float *o = O + ((size_t)bh * n + pos) * DH;
+    if (pos >= vl || mx == -INFINITY) {
+        for (int k = lane; k < DH; k += 32) o[k] = 0.0f;
+        if (lse_out && lane == 0) lse_out[(size_t)bh * n + pos] = -INFINITY;
+        return;
+    }
+    float z = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) z += (r < rounds && l[r] != -INFINITY) ? __expf(l[r] - mx) : 0.0f;
+    const float LSE = mx + logf(z);
+    for (int k = lane; k < DH; k += 32) {
+        float acc = 0.0f;
+        for (int r = 0; r < rounds; ++r)
+            if (l[r] != -INFINITY)
+                acc = fmaf(__expf(l[r] - LSE), o_ws[(((size_t)r * BH + bh) * n + pos) * DH + k], acc);
+        o[k] = acc;
+    }
+    if (lse_out && lane == 0) lse_out[(size_t)bh * n + pos] = LSE;
+}
+
+// ------------------------------------------------------------ host side --
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int validate_lsh(const crs_lsh_params *p) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    if (p->B < 1 || p->H < 1 || p->n < 1) return CRS_ERR_INVALID_ARG;
+    if (p->d < 8 || p->d % 8 != 0 || p->d > 128) return CRS_ERR_INVALID_ARG;
+    if (p->n_buckets < 2 || p->n_buckets % 2 != 0 || p->n_buckets > 1024) return CRS_ERR_INVALID_ARG;
+    if (p->n_rounds < 1 || p->n_rounds > kMaxRounds) return CRS_ERR_INVALID_ARG;
+    if (p->dtype != CRS_F32 && p->dtype != CRS_BF16) return CRS_ERR_INVALID_ARG;
+    if ((long long)p->n_buckets * p->n > 0x7fffffffLL) return CRS_ERR_INVALID_ARG;
+    return CRS_OK;
+}
+
+}  // namespace crs
+
+using namespace crs;
+
+extern "C" size_t crs_lsh_route_workspace_size(const crs_lsh_params *) { return 0; }
+
+extern "C" int crs_lsh_route(const crs_lsh_params *p, const void *X, const float *R,
+                             int32_t *bucket, int32_t *perm, int32_t *inv_perm, void *,
+                             size_t, void *stream) {
+    int st = validate_lsh(p);
+    if (st) return st;
+    if (!X || !R || !bucket || !perm || !inv_perm) return CRS_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int half = p->n_buckets / 2;
+    const size_t smem = ((size_t)p->d * half + (size_t)kHashTok * (p->d + 1)) * sizeof(float);
+    if (smem > 200 * 1024) return CRS_ERR_UNSUPPORTED;
+    dim3 grid(ceil_div(p->n, kHashTok), p->n_rounds, p->B * p->H);
+    if (p->dtype == CRS_F32) {
+        CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_hash_kernel<float>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        {
+            ProfScope _ps(K_LSH_HASH, s);
+            lsh_hash_kernel<float><<<grid, kHashTok, smem, s>>>(
+                static_cast<const float *>(X), R, bucket, p->H, p->n, p->d, p->n_buckets, p->n_rounds);
+        }
+    } else {
+        CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_hash_kernel<__nv_bfloat16>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        {
+            ProfScope _ps(K_LSH_HASH, s);
+            lsh_hash_kernel<__nv_bfloat16><<<grid, kHashTok, smem, s>>>(
+                static_cast<const __nv_bfloat16 *>(X), R, bucket, p->H, p->n, p->d, p->n_buckets,
+                p->n_rounds);
+        }
+    }
+    CRS_CHECK_LAUNCH();
+    const size_t ssm = (size_t)(2 + kSortThreads / 32) * p->n_buckets * sizeof(int);
+    CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)ssm));
+    {
+        ProfScope _ps(K_LSH_SORT, s);
+        lsh_sort_kernel<<<p->B * p->H * p->n_rounds, kSortThreads, ssm, s>>>(bucket, perm, inv_perm,
+                                                                             p->n, p->n_buckets);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+
+extern "C" size_t crs_lsh_attn_workspace_size(const crs_lsh_attn_params *a) {
+    if (!a || validate_lsh(&a->p)) return 0;
+    const crs_lsh_params &p = a->p;
+    const size_t rows = (size_t)p.n_rounds * p.B * p.H * p.n;
+    return align256(rows * p.d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+namespace crs {
+template <typename T, int DH>
+static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const void *V,
+                           const int32_t *bucket, const int32_t *perm, const int32_t *inv_perm,
+                           const int32_t *valid_len, void *O, float *lse, float *o_ws,
+                           float *lse_ws, cudaStream_t s) {
+    const crs_lsh_params &p = a->p;
+    const int KM = 2 * p.chunk;
+    const size_t smem = (size_t)KM * (DH + 1) * 4 + (size_t)KM * DH * 4 + (size_t)KM * 4 +
+                        (size_t)kAttnWarps * KM * 4 + (size_t)KM * 4 * 2 +
+                        (size_t)KM * (kMaxRounds - 1) * 2 * 4;
+    if (smem > 227 * 1024) return CRS_ERR_UNSUPPORTED;
+    auto kern = lsh_chunk_attn_kernel<T, DH>;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid(ceil_div(p.n, p.chunk), p.n_rounds, p.B * p.H);
+    {
+        ProfScope _ps(K_LSH_ATTN, s);
+        kern<<<grid, kAttnWarps * 32, smem, s>>>(static_cast<const T *>(QK), static_cast<const T *>(V),
+                                                  bucket, perm, inv_perm, valid_len, o_ws, lse_ws, p.H,
+                                                  p.n, p.chunk, p.n_rounds, a->causal, a->no_self,
+                                                  a->key_norm, a->scale);
+    }
+    CRS_CHECK_LAUNCH();
+    const long long warps = (long long)p.B * p.H * p.n;
+    const int threads = 256;
+    {
+        ProfScope _ps(K_LSH_COMBINE, s);
+        lsh_combine_kernel<DH><<<(unsigned)ceil_div_ll(warps * 32, threads), threads, 0, s>>>(
+            o_ws, lse_ws, valid_len, static_cast<float *>(O), lse, p.B * p.H, p.H, p.n, p.n_rounds);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+}  // namespace crs
+
+extern "C" int crs_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const void *V,
+                            const int32_t *bucket, const int32_t *perm, const int32_t *inv_perm,
+                            const int32_t *valid_len, void *O, float *lse, void *ws,
+                            size_t ws_bytes, void *stream) {
+    if (!a) return CRS_ERR_INVALID_ARG;
+    int st = validate_lsh(&a->p);
+    if (st) return st;
+    const crs_lsh_params &p = a->p;
+    if (p.chunk < 1 || p.chunk > 128) return CRS_ERR_INVALID_ARG;
+    if (!QK || !V || !bucket || !perm || !inv_perm || !O) return CRS_ERR_INVALID_ARG;
+    if (!(a->scale == a->scale)) return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_lsh_attn_workspace_size(a);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    const size_t rows = (size_t)p.n_rounds * p.B * p.H * p.n;
+    float *o_ws = static_cast<float *>(ws);
+    float *lse_ws = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                              align256(rows * p.d * sizeof(float)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p.d == 64) {
+        if (p.dtype == CRS_F32)
+            return launch_lsh_attn<float, 64>(a, QK, V, bucket, perm, inv_perm, valid_len, O, lse,
+                                              o_ws, lse_ws, s);
+        return launch_lsh_attn<__nv_bfloat16, 64>(a, QK, V, bucket, perm, inv_perm, valid_len, O,
+                                                  lse, o_ws, lse_ws, s);
+    }
+    if (p.d == 32) {
+        if (p.dtype == CRS_F32)
+            return launch_lsh_attn<float, 32>(a, QK, V, bucket, perm, inv_perm, valid_len, O, lse,
+                                              o_ws, lse_ws, s);
+        return launch_lsh_attn<__nv_bfloat16, 32>(a, QK, V, bucket, perm, inv_perm, valid_len, O,
+                                                  lse, o_ws, lse_ws, s);
+    }
+    return CRS_ERR_UNSUPPORTED;
+}

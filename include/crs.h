@@ -1,0 +1,272 @@
+/*
+ * crs.h -- C ABI of libcrs, content-routed sparse attention on NVIDIA B200 (sm_100a).
+ *
+ * A selector computes, for every query, a candidate set of key positions; exact
+ * softmax attention then runs over the gathered K/V only.  Three selectors:
+ *   - Reformer-style LSH routing (crs_lsh_route + crs_lsh_attn),
+ *   - a DSA-style lightning indexer with token top-k (crs_indexer_topk),
+ *   - a COBS-style block-mass selector (crs_block_describe + crs_block_select),
+ * and one attention kernel over explicit index lists (crs_sparse_attn).
+ *
+ * Pages cited:
+ *   [P1] PaperTrace 2.1.1 "哈希与聚类: 用内容建立稀疏注意力邻域"
+ *   [P2] PaperTrace 2.2 "细粒度索引: 用轻量 selector 召回关键 token"
+ *   [P4] Understanding LLMs ch. 26 "高效、稀疏与替代架构地图"
+ *   [P5] "COBS 阅读笔记: 块稀疏注意力的选择器到底漏掉了什么"
+ *
+ * Conventions (all entry points):
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; libcrs
+ *     never allocates, frees or keeps a pointer after the call returns.
+ *     Tensors are dense, row-major (C order), in the layouts stated below.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous on that stream.
+ *   - Scratch memory comes from the caller: `ws`/`ws_bytes`, sized by the
+ *     matching *_workspace_size() call.  A short workspace returns
+ *     CRS_ERR_WORKSPACE with nothing launched.
+ *   - Host-side validation errors return immediately with nothing launched.
+ *     A failed launch returns CRS_ERR_CUDA.
+ *   - Problems a kernel detects in the data (a non-finite indexer score, an
+ *     index out of range, a bounded wait that ran out) are OR-ed into a
+ *     per-device error word; crs_get_device_error() reads and clears it.
+ *   - Index lists hold int32 positions within their sequence, ascending;
+ *     -1 marks an unused slot.
+ *   - bf16 means IEEE bfloat16 stored in 16 bits; f32 means IEEE binary32.
+ */
+#ifndef CRS_H
+#define CRS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status -- */
+typedef enum {
+    CRS_OK = 0,
+    CRS_ERR_INVALID_ARG = 1,  /* a size, pointer or parameter is out of range     */
+    CRS_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement   */
+    CRS_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed          */
+    CRS_ERR_NONFINITE = 4,    /* (device word bit) NaN/Inf met where not allowed */
+    CRS_ERR_TIMEOUT = 5,      /* (device word bit) a bounded wait ran out        */
+    CRS_ERR_WORKSPACE = 6,    /* ws is NULL or shorter than required             */
+    CRS_ERR_INDEX = 7         /* (device word bit) an index list entry is out of range */
+} crs_status;
+
+typedef enum { CRS_F32 = 0, CRS_BF16 = 1 } crs_dtype;
+
+/* Bits of the device error word. */
+#define CRS_DEVERR_NONFINITE 0x1u
+#define CRS_DEVERR_TIMEOUT   0x2u
+#define CRS_DEVERR_INDEX     0x4u
+
+/* Human-readable name of a crs_status value (static string, never NULL). */
+const char *crs_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int crs_version(void);
+
+/* Synchronizes `stream`, then reads and clears the error word of the current
+ * device.  *flags receives the CRS_DEVERR_* bits set since the last call
+ * (0 = none).  Returns CRS_ERR_CUDA if the synchronization fails. */
+int crs_get_device_error(void *stream, uint32_t *flags);
+
+/* Launch tracing.  [P1] "一个可复现的评测矩阵" and [P2] §1.1 "性能轴" ask for the
+ * time of every stage (routing, sort, selection, gather, attention) reported
+ * separately; this is how the library provides it.  Every kernel
+ * launch is counted.  While enabled, each launch is also bracketed by two
+ * CUDA events recorded on the launch's own stream.
+ * crs_profile_collect() synchronizes on those events, writes one record per
+ * kernel that launched since the previous collect (up to max_out records;
+ * *n_out receives how many kernels there were) and resets the counters. */
+typedef struct {
+    char name[32];           /* kernel family, e.g. "lsh_chunk_attn"            */
+    int64_t launches;        /* launches since the previous collect             */
+    int64_t timed_launches;  /* of those, launches made while tracing was on    */
+    double total_ms;         /* summed device time of the timed launches        */
+} crs_kernel_stat;
+
+int crs_profile_set(int enabled);
+int crs_profile_collect(crs_kernel_stat *out, int max_out, int *n_out);
+
+/* ====================================================================== *
+ * LSH routing.  [P1] §2.1 Eq.(4): per head h and round r, u = x R_{h,r} with
+ * R_{h,r} in R^{d x b/2}; bucket = argmax_j [u ; -u]_j (0-based, lowest
+ * index on ties).  [P1] §2.1-2.2: tokens are stably sorted on the bucket id
+ * (sort key = bucket * n + position); perm maps a sorted slot to its
+ * original position, inv_perm maps a position to its slot.
+ * The projection is evaluated in fp32 as one fused multiply-add per term in
+ * increasing index order starting from 0, so the bucket ids are reproducible
+ * bit for bit.
+ * ====================================================================== */
+typedef struct {
+    int B;          /* batch                                                    */
+    int H;          /* heads                                                    */
+    int n;          /* tokens per sequence, >= 1                                */
+    int d;          /* head dim, multiple of 8, <= 128                          */
+    int n_buckets;  /* b, even, 2..1024                                         */
+    int n_rounds;   /* independent hash rounds, 1..8                            */
+    int chunk;      /* m, slots per chunk (used by crs_lsh_attn), 1..128       */
+    int dtype;      /* crs_dtype of X / QK / V / O                              */
+} crs_lsh_params;
+
+/* X: [B,H,n,d] (dtype); R: [H,n_rounds,d,n_buckets/2] f32.
+ * Outputs (int32, [B,H,n_rounds,n]): bucket, perm (slot -> position),
+ * inv_perm (position -> slot).  Needs no workspace (ws may be NULL). */
+size_t crs_lsh_route_workspace_size(const crs_lsh_params *p);
+int crs_lsh_route(const crs_lsh_params *p, const void *X, const float *R, int32_t *bucket,
+                  int32_t *perm, int32_t *inv_perm, void *ws, size_t ws_bytes, void *stream);
+
+/* ====================================================================== *
+ * LSH attention.  [P1] §2.2: each round's sorted array is cut into chunks of
+ * m slots; a query chunk attends to itself and the previous chunk (chunk 0
+ * has none).  A pair (i, j) is an edge of round r iff bucket_r(j) ==
+ * bucket_r(i), j <= i when causal, j != i when no_self, j < valid_len[b]
+ * ([P1] §1.1 Eq.(2); causality on ORIGINAL positions, [P1] §"8.2").  Shared
+ * QK ([P1] §2): keys are q_j/|q_j| when key_norm != 0 (a zero vector stays
+ * zero), logits scale * q_i . k_j.  Rounds are merged by their log-sum-exp
+ * weights with each pair counted only in the first round it appears in
+ * ([P1] "重复候选和归一化"), which equals one softmax over the union of the
+ * rounds' candidates.  A query with no edge, and every padded query
+ * (i >= valid_len[b]), gets O = 0 and lse = -inf.
+ * ====================================================================== */
+typedef struct {
+    crs_lsh_params p;
+    int causal;     /* 1: j <= i                                              */
+    int no_self;    /* 1: j != i                                              */
+    int key_norm;   /* 1: k_j = q_j / |q_j| (Reformer shared-QK), 0: k_j = q_j */
+    float scale;    /* logit scale, typically 1/sqrt(d)                       */
+} crs_lsh_attn_params;
+
+/* QK, V: [B,H,n,d] (p.dtype); bucket/perm/inv_perm: [B,H,n_rounds,n] from
+ * crs_lsh_route; valid_len: [B] int32 (NULL = n for all).
+ * O: [B,H,n,d] f32, written in original token order (f32 whatever p.dtype:
+ * the 2e-3 output tolerance for bf16 inputs is below bf16's unit roundoff
+ * 2^-8, so the result keeps the fp32 accumulator's precision);
+ * lse: [B,H,n] f32 natural-log normaliser of the merged softmax, or NULL. */
+size_t crs_lsh_attn_workspace_size(const crs_lsh_attn_params *p);
+int crs_lsh_attn(const crs_lsh_attn_params *p, const void *QK, const void *V,
+                 const int32_t *bucket, const int32_t *perm, const int32_t *inv_perm,
+                 const int32_t *valid_len, void *O, float *lse, void *ws, size_t ws_bytes,
+                 void *stream);
+
+/* ====================================================================== *
+ * Lightning indexer + token top-k.  [P2] §1.1 / §2.1 Eq.(2)-(4):
+ *   r_{t,s} = sum_h w_{t,h} ReLU(q_{t,h} . k_s)   (no extra scale)
+ * S_t = the topk positions with the largest r_{t,s}, ties to the smaller
+ * position ([P2] §3.1 "多卡一致性"), returned ascending; a row with fewer
+ * than topk visible keys returns all of them and -1 in the other slots
+ * ([P2] §2.1).  The score matrix is never stored whole ([P2] §2.1).
+ * Modes:
+ *   CRS_IDX_PREFILL: one causal sequence of n_rows tokens; row t sees keys
+ *                    0..t; k_offsets is ignored.
+ *   CRS_IDX_DECODE:  n_rows sequences, one query each; row s sees the keys
+ *                    k_idx[k_offsets[s] .. k_offsets[s+1]) (int64 offsets,
+ *                    [n_rows+1]); positions are relative to k_offsets[s].
+ * A NaN score sets CRS_DEVERR_NONFINITE and ranks below every number.
+ * ====================================================================== */
+enum { CRS_IDX_PREFILL = 0, CRS_IDX_DECODE = 1 };
+
+typedef struct {
+    int mode;         /* CRS_IDX_PREFILL or CRS_IDX_DECODE                      */
+    int n_rows;       /* queries                                                */
+    int n_idx_heads;  /* index heads, 1..8                                      */
+    int d_idx;        /* index head dim, 64                                     */
+    int topk;         /* 1..4096                                                */
+    int max_keys;     /* DECODE: an upper bound of the longest row (sizes ws)   */
+} crs_indexer_params;
+
+/* q_idx: [n_rows, n_idx_heads, d_idx] bf16; w: [n_rows, n_idx_heads] f32;
+ * k_idx: [keys, d_idx] bf16; out_idx: [n_rows, topk] int32; out_count:
+ * [n_rows] int32 (number of valid entries). */
+size_t crs_indexer_topk_workspace_size(const crs_indexer_params *p);
+int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, const float *w,
+                     const void *k_idx, const int64_t *k_offsets, int32_t *out_idx,
+                     int32_t *out_count, void *ws, size_t ws_bytes, void *stream);
+
+/* ====================================================================== *
+ * Block descriptors.  [P5] Eq.(11), (16), (20) and Algorithm 2: for each
+ * complete block of L consecutive keys of one (sequence, KV head):
+ *   mu = mean key; Kt = K - mu; G = Kt Kt^T / L (L x L);
+ *   (lambda_i, w_i) = the `rank` largest eigenpairs of G;
+ *   xi_i = Kt^T w_i / sqrt(L)   (= sqrt(lambda_i) u_i, sign arbitrary).
+ * The descriptor depends on the block alone and is computed once, when the
+ * block is full ([P5] "可缓存性约束").  Blocks [blk_begin, blk_end) are
+ * (re)computed; others are left untouched.
+ * ====================================================================== */
+typedef struct {
+    int n_seq;      /* sequences                                             */
+    int n_kv;       /* KV heads                                              */
+    int T;          /* tokens per sequence in the cache                      */
+    int D;          /* head dim, 128                                         */
+    int L;          /* block size, 32                                        */
+    int rank;       /* kept eigen-directions, 1..8                           */
+    int blk_begin;  /* first block to compute                                */
+    int blk_end;    /* one past the last block to compute, <= T / L          */
+} crs_block_params;
+
+/* K: [n_seq, T, n_kv, D] bf16.  mu: [n_seq, n_kv, T/L, D] f32;
+ * xi: [n_seq, n_kv, T/L, rank, D] f32. */
+int crs_block_describe(const crs_block_params *p, const void *K, float *mu, float *xi,
+                       void *stream);
+
+/* ====================================================================== *
+ * Block selection.  [P5] Eq.(14)/(19): s_{g,b} = qt . mu_b + 1/2 sum_i (xi_i . qt)^2
+ * with qt = scale * q_g (the ln L constant cancels); [P5] Eq.(15)/(6): KV head
+ * h scores block b by sum over its query-head group g of softmax_b(s_{g,.});
+ * the top_blocks complete blocks by (score desc, block asc) are kept; the
+ * token list is their positions united with the window [T-window, T),
+ * without duplicates, ascending.  Query heads [h*G, (h+1)*G) share KV head h
+ * ([P4] §26.2).
+ * ====================================================================== */
+typedef struct {
+    crs_block_params b;  /* n_seq, n_kv, T, D, L, rank (blk_* ignored)       */
+    int n_q;             /* query heads, multiple of n_kv, G = n_q/n_kv <= 16 */
+    int top_blocks;      /* kept blocks, 1..T/L                              */
+    int window;          /* trailing window, 0..T                            */
+    float scale;         /* typically 1/sqrt(D)                              */
+} crs_block_sel_params;
+
+/* Q: [n_seq, n_q, D] bf16; mu, xi from crs_block_describe.
+ * tok_idx: [n_seq, n_kv, top_blocks*L + window] int32; tok_count: [n_seq, n_kv]. */
+size_t crs_block_select_workspace_size(const crs_block_sel_params *p);
+int crs_block_select(const crs_block_sel_params *p, const void *Q, const float *mu,
+                     const float *xi, int32_t *tok_idx, int32_t *tok_count, void *ws,
+                     size_t ws_bytes, void *stream);
+
+/* ====================================================================== *
+ * Attention over explicit index lists.  [P1] §1.1 Eq.(1) restricted to the
+ * candidate set; [P2] §1.1 (one selected set shared by the main heads);
+ * [P4] §26.2 (query heads [h*G, (h+1)*G) share KV head h):
+ *   O_{t,g} = sum_{j in I} softmax_j(scale * q_{t,g} . k_{j,h}) v_{j,h},  h = g / G,
+ * over the entries of the row's list that are >= 0.  An empty list gives
+ * O = 0 and lse = -inf.  Duplicated entries are a caller error.
+ * ====================================================================== */
+typedef struct {
+    int n_rows;     /* queries                                               */
+    int n_q;        /* query heads per row                                   */
+    int n_kv;       /* KV heads; G = n_q / n_kv <= 16                        */
+    int D;          /* head dim, 128                                         */
+    int max_idx;    /* slots per index list                                  */
+    int n_lists;    /* 1: one list per row shared by all KV heads;
+                       n_kv: one list per (row, KV head)                     */
+    int n_keys;     /* entries must be < n_keys (bounds check); 0 = no check  */
+    float scale;    /* typically 1/sqrt(D)                                   */
+} crs_attn_params;
+
+/* Q: [n_rows, n_q, D] bf16.  K, V: bf16, token j of row t and KV head h at
+ * element ((kv_base[t] + j) * n_kv + h) * D (kv_base: [n_rows] int64, NULL =
+ * 0).  I: [n_rows, n_lists, max_idx] int32.  O: [n_rows, n_q, D] f32 (the
+ * fp32 accumulator's precision; P.V runs on bf16 tensor cores with P split
+ * into a bf16 value and a bf16 residual);
+ * lse: [n_rows, n_q] f32 or NULL. */
+size_t crs_sparse_attn_workspace_size(const crs_attn_params *p);
+int crs_sparse_attn(const crs_attn_params *p, const void *Q, const void *K, const void *V,
+                    const int64_t *kv_base, const int32_t *I, void *O, float *lse, void *ws,
+                    size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CRS_H */

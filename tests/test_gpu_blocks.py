@@ -1,0 +1,108 @@
+"""GPU parity: block descriptors and block selection vs the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().cpu().float().numpy().astype(np.float64)
+
+
+def _blocks(K, L):
+    """[n_seq, T, n_kv, D] -> [n_seq, n_kv, n_full, L, D] (full blocks only)."""
+    n_seq, T, n_kv, D = K.shape
+    nf = T // L
+    return K[:, : nf * L].reshape(n_seq, nf, L, n_kv, D).transpose(0, 3, 1, 2, 4)
+
+
+def _oracle_describe(Kd, L, rank):
+    kb = _blocks(Kd, L)
+    s, h, nf = kb.shape[:3]
+    mu, xi, lam = oracle.block_describe(kb.reshape(-1, L, kb.shape[-1]), rank + 1)
+    return (mu.reshape(s, h, nf, -1), xi.reshape(s, h, nf, rank + 1, -1),
+            lam.reshape(s, h, nf, rank + 1))
+
+
+def test_describe_small(crs, cuda_dev):
+    case = workloads.block_decode_case(n_seq=2, T=32 * 40 + 7, seed=3, device=cuda_dev)
+    p = case["params"]
+    L, r = p["L"], p["rank"]
+    mu, xi = crs.block_describe(case["K"], L, r)
+    torch.cuda.synchronize()
+    Kd = _np(case["K"])
+    omu, oxi, olam = _oracle_describe(Kd, L, r)
+    assert rel_err(_np(mu), omu).max() < 1e-5
+    g = _np(xi)
+    glam = (g ** 2).sum(-1)                          # |xi_i|^2 = lambda_i
+    assert np.abs(glam - olam[..., :r]).max() <= 1e-4 * olam[..., 0].max()
+    # the rank-r factor sum xi xi^T where the r-th eigengap is clear of fp32 noise
+    gap = (olam[..., r - 1] - olam[..., r]) / olam[..., 0]
+    P = np.einsum("shbrd,shbre->shbde", g, g)
+    Po = np.einsum("shbrd,shbre->shbde", oxi[..., :r, :], oxi[..., :r, :])
+    err = np.abs(P - Po).max(axis=(-1, -2)) / olam[..., 0]
+    ok = gap > 1e-3
+    assert ok.mean() > 0.9
+    assert (err[ok] <= 1e-4 / gap[ok]).all()
+
+
+def _check_select(tok, cnt, o_tok, o_cnt, o_blk, o_bs, L, T, window, top, what):
+    n_seq, n_kv = cnt.shape
+    for s in range(n_seq):
+        for h in range(n_kv):
+            gt = tok[s, h, : cnt[s, h]]
+            ot = o_tok[s, h, : o_cnt[s, h]]
+            assert (np.diff(gt) > 0).all() and (tok[s, h, cnt[s, h]:] == -1).all()
+            gb = np.unique(gt[gt < max(0, T - window)] // L)
+            ob = np.unique(ot[ot < max(0, T - window)] // L)
+            diff = np.setxor1d(gb, ob)
+            if diff.size:
+                sc = o_bs[s, h]
+                cut = np.sort(sc)[::-1][top - 1]
+                assert np.all(np.abs(sc[diff] - cut) <= 1e-5 * abs(cut) + 1e-6), \
+                    f"{what} ({s},{h}): blocks {diff} not at the cutoff"
+            else:
+                assert cnt[s, h] == o_cnt[s, h]
+
+
+def test_select_on_oracle_descriptors(crs, cuda_dev):
+    """Selection alone: the GPU reads the oracle's descriptors (rounded to fp32)."""
+    case = workloads.block_decode_case(n_seq=3, T=4096, seed=5, device=cuda_dev)
+    p = case["params"]
+    L, r, top, win = p["L"], p["rank"], 16, 256
+    omu, oxi, _ = _oracle_describe(_np(case["K"]), L, r)
+    oxi = oxi[..., :r, :]
+    mu32 = torch.from_numpy(omu.astype(np.float32)).to(cuda_dev)
+    xi32 = torch.from_numpy(oxi.astype(np.float32)).to(cuda_dev)
+    tok, cnt = crs.block_select(case["Q"], mu32, xi32, p["T"], L, top, win)
+    torch.cuda.synchronize()
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(
+        _np(case["Q"]), mu32.double().cpu().numpy(), xi32.double().cpu().numpy(), p["T"], L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, p["T"], win,
+                  top, "select")
+
+
+def test_describe_select_end_to_end_small(crs, cuda_dev):
+    case = workloads.block_decode_case(n_seq=2, T=2048, seed=6, device=cuda_dev)
+    p = case["params"]
+    L, r, top, win = p["L"], p["rank"], 8, 128
+    mu, xi = crs.block_describe(case["K"], L, r)
+    tok, cnt = crs.block_select(case["Q"], mu, xi, p["T"], L, top, win)
+    torch.cuda.synchronize()
+    omu, oxi, _ = _oracle_describe(_np(case["K"]), L, r)
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), omu, oxi[..., :r, :], p["T"], L,
+                                                    top, win)
+    g_tok, g_cnt = tok.cpu().numpy(), cnt.cpu().numpy()
+    # descriptors carry fp32 rounding: a differing block must sit within 1e-3 of the cutoff
+    for s in range(2):
+        for h in range(4):
+            gb = np.unique(g_tok[s, h, : g_cnt[s, h]] // L)
+            ob = np.unique(o_tok[s, h, : o_cnt[s, h]] // L)
+            d = np.setxor1d(gb, ob)
+            cut = np.sort(o_bs[s, h])[::-1][top - 1]
+            assert np.all(np.abs(o_bs[s, h][d] - cut) <= 1e-3 * abs(cut))

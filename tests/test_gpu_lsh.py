@@ -1,0 +1,115 @@
+"""GPU parity: LSH routing (bit-exact) and LSH attention (float tolerance) vs the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+# |gpu - oracle| <= TOL * max(1, |oracle|): 1e-5 for fp32 inputs, 2e-3 for bf16
+# inputs with fp32 accumulation (the tolerances the workloads state).
+TOL = {"f32": 1e-5, "bf16": 2e-3}
+
+
+def _host(x):
+    return x.detach().cpu()
+
+
+def _route_and_check(crs, case):
+    p = case["params"]
+    X = case["QK"]
+    bucket, perm, inv = crs.lsh_route(X, case["R"], p["n_buckets"], p["chunk"])
+    torch.cuda.synchronize()
+    Xh = _host(X).float().numpy()
+    Rh = _host(case["R"]).numpy()
+    ob = oracle.lsh_hash(Xh, Rh, p["n_buckets"])
+    op, oi = oracle.lsh_sort(ob)
+    gb, gp, gi = (_host(t).numpy() for t in (bucket, perm, inv))
+    assert (gb == ob).all(), f"bucket mismatch at {np.argwhere(gb != ob)[:5]}"
+    assert (gp == op).all()
+    assert (gi == oi).all()
+    return bucket, perm, inv, ob, op, oi
+
+
+def _attn_and_check(crs, case, bucket, perm, inv, ob, op, oi, rows=None):
+    p = case["params"]
+    O, lse = crs.lsh_attn(case["QK"], case["V"], bucket, perm, inv, case["valid_len"],
+                          n_buckets=p["n_buckets"], chunk=p["chunk"], causal=p["causal"],
+                          no_self=p["no_self"], key_norm=p["key_norm"], scale=p["scale"],
+                          lse=torch.empty(bucket.shape[0], bucket.shape[1], bucket.shape[3],
+                                          device=bucket.device))
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    Qh = _host(case["QK"]).double().numpy()
+    Vh = _host(case["V"]).double().numpy()
+    vl = _host(case["valid_len"]).numpy()
+    oO, olse, ocnt = oracle.lsh_attn(Qh, Vh, ob, op, oi, vl, p["chunk"], p["causal"],
+                                     p["no_self"], p["key_norm"], p["scale"], rows=rows)
+    gO = _host(O).double().numpy()
+    gl = _host(lse).double().numpy()
+    if rows is not None:
+        gO = gO[:, :, rows]
+        gl = gl[:, :, rows]
+    tol = TOL[p["dtype"]]
+    err = np.abs(gO - oO) / np.maximum(1.0, np.abs(oO))
+    assert err.max() <= tol, f"max rel err {err.max():.3e} > {tol}"
+    fin = np.isfinite(olse)
+    assert (np.isfinite(gl) == fin).all()
+    assert np.abs(gl[fin] - olse[fin]).max() <= tol * max(1.0, np.abs(olse[fin]).max())
+    return ocnt
+
+
+def test_lsh_fp32_full_config(crs, cuda_dev):
+    """n=1024 fp32, one round, b=16, m=64, causal, no self (the fp32 LSH workload)."""
+    case = workloads.lsh_fp32_case(device=cuda_dev)
+    r = _route_and_check(crs, case)
+    cnt = _attn_and_check(crs, case, *r)
+    assert (cnt[0, 0, 0] == 0)  # position 0 has no legal key (causal + no self)
+
+
+@pytest.mark.parametrize("n,chunk,rounds,nb,vl_frac", [
+    (1000, 64, 2, 16, 0.05),    # ragged last chunk, padding
+    (2048, 128, 4, 64, 0.05),   # the bf16 workload's shape per head, 4 rounds
+    (77, 128, 3, 8, 0.0),       # n < chunk: one chunk, no previous
+    (333, 32, 8, 4, 0.3),       # many rounds, heavy duplication
+])
+def test_lsh_bf16_small(crs, cuda_dev, n, chunk, rounds, nb, vl_frac):
+    case = workloads.lsh_clustered_case(B=2, H=2, n=n, n_buckets=nb, n_rounds=rounds, chunk=chunk,
+                                        n_centres=16, pad_frac=vl_frac, seed=n, device=cuda_dev)
+    r = _route_and_check(crs, case)
+    _attn_and_check(crs, case, *r)
+
+
+def test_lsh_fp32_variants(crs, cuda_dev):
+    """fp32, causal off / self allowed / raw keys."""
+    case = workloads.lsh_fp32_case(n=300, n_rounds=3, chunk=16, causal=0, no_self=0, seed=9,
+                                   device=cuda_dev)
+    case["params"]["key_norm"] = 0
+    r = _route_and_check(crs, case)
+    _attn_and_check(crs, case, *r)
+
+
+def test_lsh_bf16_full_config_sampled(crs, cuda_dev):
+    """The full bf16 multi-round workload (B=2, H=8, n=16384, 4 rounds); routing is
+    compared everywhere, attention on 96 sampled query rows per (b, h)."""
+    case = workloads.lsh_clustered_case(device=cuda_dev)
+    r = _route_and_check(crs, case)
+    n = case["params"]["n"]
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([rng.choice(n, 90, replace=False),
+                                     [0, 1, 127, 128, n - 1, int(case["valid_len"][0]) - 1]]))
+    _attn_and_check(crs, case, *r, rows=rows.astype(np.int32))
+
+
+def test_lsh_rejects_bad_args(crs, cuda_dev):
+    case = workloads.lsh_fp32_case(n=64, device=cuda_dev)
+    with pytest.raises(ValueError):
+        crs.lsh_route(case["QK"], case["R"][:, :, :, :4], 16)   # R shape mismatch
+    X = case["QK"][..., :7].contiguous()                        # d not a multiple of 8
+    R = torch.zeros(1, 1, 7, 8, device=cuda_dev)
+    with pytest.raises(crs.CrsError):
+        crs.lsh_route(X, R, 16)

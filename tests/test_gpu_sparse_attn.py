@@ -1,0 +1,83 @@
+"""GPU parity: attention over explicit index lists vs the oracle (same index set)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import rel_err
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3   # bf16 inputs, fp32 accumulation
+
+
+def _np(t):
+    return t.detach().cpu().float().numpy().astype(np.float64)
+
+
+def _random_lists(rng, n_rows, n_lists, max_idx, n_keys, fill):
+    I = np.full((n_rows, n_lists, max_idx), -1, np.int32)
+    for r in range(n_rows):
+        for l in range(n_lists):
+            m = int(rng.integers(0, max_idx + 1)) if fill is None else min(fill, max_idx)
+            I[r, l, :m] = np.sort(rng.choice(n_keys, min(m, n_keys), replace=False))
+    return I
+
+
+def _run(crs, dev, n_rows, n_q, n_kv, max_idx, n_tok, n_lists, seed, kv_base=None, fill=None,
+         per_row_tokens=None):
+    rng = np.random.default_rng(seed)
+    g = torch.Generator(device=dev).manual_seed(seed)
+    Q = torch.randn(n_rows, n_q, 128, generator=g, device=dev).to(torch.bfloat16)
+    K = torch.randn(n_tok, n_kv, 128, generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn(n_tok, n_kv, 128, generator=g, device=dev).to(torch.bfloat16)
+    I = _random_lists(rng, n_rows, n_lists, max_idx, per_row_tokens or n_tok, fill)
+    It = torch.from_numpy(I).to(dev)
+    kb = None if kv_base is None else torch.from_numpy(kv_base).to(dev)
+    lse = torch.empty(n_rows, n_q, device=dev)
+    O, _ = crs.sparse_attn(Q, K, V, It, kv_base=kb, lse=lse)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    oO, olse = oracle.sparse_attn(_np(Q), _np(K), _np(V), I, kv_base=kv_base)
+    err = rel_err(_np(O), oO)
+    assert err.max() <= TOL, f"max rel err {err.max():.3e}"
+    gl = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(olse)
+    assert (np.isfinite(gl) == fin).all()
+    if fin.any():
+        assert rel_err(gl[fin], olse[fin]).max() <= TOL
+    return I
+
+
+def test_mqa_ragged_lists(crs, cuda_dev):
+    """16 heads share one KV head; list lengths 0..max (empty lists included)."""
+    _run(crs, cuda_dev, n_rows=60, n_q=16, n_kv=1, max_idx=300, n_tok=1000, n_lists=1, seed=1)
+
+
+def test_gqa_shared_list_multi_sequence(crs, cuda_dev):
+    """32 q heads over 8 KV heads, one list per row, rows in different sequences."""
+    lens = [500, 1200, 64, 3000]
+    base = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+    rng = np.random.default_rng(0)
+    rows = len(lens)
+    _run(crs, cuda_dev, n_rows=rows, n_q=32, n_kv=8, max_idx=64, n_tok=sum(lens), n_lists=1,
+         seed=2, kv_base=base, per_row_tokens=min(lens))
+
+
+@pytest.mark.parametrize("n_q,n_kv", [(32, 4), (8, 8), (12, 4)])
+def test_per_kv_lists_and_splits(crs, cuda_dev, n_q, n_kv):
+    """A list per (row, KV head); few rows and long lists force split-KV + merge."""
+    _run(crs, cuda_dev, n_rows=3, n_q=n_q, n_kv=n_kv, max_idx=2560, n_tok=5000, n_lists=n_kv,
+         seed=n_q + n_kv, fill=2560)
+
+
+def test_out_of_range_index_is_flagged_and_skipped(crs, cuda_dev):
+    Q = torch.randn(2, 16, 128, device=cuda_dev).to(torch.bfloat16)
+    K = torch.randn(100, 1, 128, device=cuda_dev).to(torch.bfloat16)
+    V = torch.randn(100, 1, 128, device=cuda_dev).to(torch.bfloat16)
+    I = torch.tensor([[[3, 5, 150]], [[1, 2, -1]]], dtype=torch.int32, device=cuda_dev)
+    crs.get_device_error()
+    O, _ = crs.sparse_attn(Q, K, V, I, n_keys=100)
+    assert crs.get_device_error() & crs.DEVERR_INDEX
+    Ir = np.array([[[3, 5, -1]], [[1, 2, -1]]], np.int32)
+    oO, _ = oracle.sparse_attn(_np(Q), _np(K), _np(V), Ir)
+    assert rel_err(_np(O), oO).max() <= TOL
