@@ -112,6 +112,8 @@ _sig("crs_block_describe", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP,
 _sig("crs_block_select_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams)])
 _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                          _VP, _SZ, _VP])
+_sig("crs_block_select_noalloc", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP,
+                                                 _VP, _VP, _VP])
 _sig("crs_sparse_attn_workspace_size", _SZ, [ctypes.POINTER(AttnParams)])
 _sig("crs_sparse_attn", ctypes.c_int, [ctypes.POINTER(AttnParams), _VP, _VP, _VP, _VP, _VP, _VP,
                                         _VP, _VP, _SZ, _VP])
@@ -327,6 +329,41 @@ def block_select(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=
     st = _lib.crs_block_select(ctypes.byref(p), _ptr(Q), _ptr(mu), _ptr(xi), _ptr(tok),
                                _ptr(count), _ptr(ws), wsb, _stream(stream))
     _check("crs_block_select", st)
+    return tok, count
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def block_select_noalloc(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=None,
+                         tok=None, count=None, stream=None):
+    """block_select for callers that cannot allocate device memory at call time.
+
+    Same inputs and outputs as block_select, but the scratch is a static 16 MiB
+    device array inside libcrs (no workspace is allocated): problems with
+    n_seq * n_q * (T // L) > 4,194,304 scores are rejected.  The first call on a
+    device looks up that array's address; calls that overlap on the GPU share
+    the array and race.  Pass preallocated ``tok``/``count`` to allocate nothing
+    on the Python side either."""
+    _need(Q, "Q", torch.bfloat16)
+    n_seq, n_q, D = Q.shape
+    n_kv, nfull, rank = mu.shape[1], mu.shape[2], xi.shape[3]
+    _need(mu, "mu", torch.float32, (n_seq, n_kv, nfull, D))
+    _need(xi, "xi", torch.float32, (n_seq, n_kv, nfull, rank, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull), n_q,
+                       int(top_blocks), int(window), float(scale))
+    cap = top_blocks * L + window
+    if tok is None:
+        tok = torch.empty((n_seq, n_kv, cap), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((n_seq, n_kv), dtype=torch.int32, device=Q.device)
+    _need(tok, "tok", torch.int32, (n_seq, n_kv, cap))
+    _need(count, "count", torch.int32, (n_seq, n_kv))
+    st = _lib.crs_block_select_noalloc(ctypes.byref(p), _ptr(Q), _ptr(mu), _ptr(xi), _ptr(tok),
+                                       _ptr(count), _stream(stream))
+    _check("crs_block_select_noalloc", st)
     return tok, count
 
 

@@ -5,3 +5,4 @@
 #include "sparse_attn.cu"
 #include "indexer.cu"
 #include "blocks.cu"
+#include "noalloc.cu"

@@ -235,6 +235,31 @@ int crs_block_select(const crs_block_sel_params *p, const void *Q, const float *
                      const float *xi, int32_t *tok_idx, int32_t *tok_count, void *ws,
                      size_t ws_bytes, void *stream);
 
+/* Allocation-free variant of crs_block_select.  The pages have no counterpart
+ * of this call; it exists for callers that cannot allocate device memory when
+ * they call the library (an engine whose pool owns all device memory and
+ * refuses allocations after start-up, a plugin host that passes only input
+ * and output buffers, a latency-bound loop that must not pay for cudaMalloc /
+ * cudaFree or their implicit synchronization).  Same parameters, inputs,
+ * outputs and result as crs_block_select, but no workspace argument: the
+ * scratch is a static device array of CRS_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads libcrs holds until the process exits.
+ *   - Limit: crs_block_select_workspace_size(p) (n_seq * n_q * (T/L) * 4
+ *     bytes) must not exceed CRS_NOALLOC_SCRATCH_BYTES, i.e. at most 4,194,304
+ *     (sequence, query head, block) scores; larger problems return
+ *     CRS_ERR_WORKSPACE with nothing launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on the device.
+ *   - Every call, on any stream, shares the one array and it keeps the last
+ *     call's contents: calls that overlap on the GPU (concurrent streams)
+ *     race on it and must be serialized by the caller.  Nothing needs
+ *     clearing between calls: the kernels write every scratch entry they read.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine. */
+#define CRS_NOALLOC_SCRATCH_BYTES (16u << 20)
+int crs_block_select_noalloc(const crs_block_sel_params *p, const void *Q, const float *mu,
+                             const float *xi, int32_t *tok_idx, int32_t *tok_count, void *stream);
+
 /* ====================================================================== *
  * Attention over explicit index lists.  [P1] §1.1 Eq.(1) restricted to the
  * candidate set; [P2] §1.1 (one selected set shared by the main heads);
