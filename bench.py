@@ -374,6 +374,26 @@ def time_steps(fn, steps, warmup, flush_buf, dist_on):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def _traffic(kernel):
+    """DRAM bytes per launch from profiles/traffic.json, only while the kernel's
+    source file is unchanged since the capture (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f).get(kernel)
+    if not t:
+        return None
+    src = os.path.join(ROOT, t["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != t["sha256_16"]:
+            return None
+    return t["bytes_per_launch"]
+
+
 def roofline(wl, prof, peaks, traffic=None):
     """The dominant kernel (largest summed device time) with its algorithmic work."""
     spec = wl.roofline_spec()
@@ -395,7 +415,8 @@ def roofline(wl, prof, peaks, traffic=None):
     else:
         peak, src = FP32_ALU_TFLOPS_NOMINAL, "fp32 FMA: 148 SM x 128 lanes x 2 x 1.965 GHz"
     out = {"kernel": top, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
-           "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
+           "unit": unit, "frac": round(achieved / peak, 4), "traffic": _traffic(top),
+           "peak_source": src,
            "per_launch_ms": round(per_launch_s * 1e3, 5)}
     if len(spec[top]) > 1:
         b2, a2, u2 = spec[top][1]
@@ -429,7 +450,7 @@ def measure(crs, wl, steps, warmup, flush_buf, dist_on, peaks, e2e=True):
 
 
 # ------------------------------------------------------------- CPU baseline --
-def cpu_baseline_lsh(case, n_segments=2):
+def cpu_baseline_lsh(case, n_segments=16):
     """The oracle on a bounded sample: n_segments of the B*H (batch, head)
     segments, each routed (hash + sort, all rounds) and attended for all n
     query rows.  Returns (tokens/s scaled to the metric, seconds, sample text)."""
