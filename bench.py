@@ -123,6 +123,8 @@ class LshWorkload(Workload):
         return {
             "lsh_chunk_attn": [("alu", rect_flops / 1e12, "TFLOP/s"),
                                ("hbm", attn_bytes / 1e9, "GB/s")],
+            "lsh_chunk_attn_tc": [("tensor", rect_flops / 1e12, "TFLOP/s"),
+                                  ("hbm", attn_bytes / 1e9, "GB/s")],
             "lsh_hash": [("alu", B * H * R * n * d * (p["n_buckets"] // 2) * 2 / 1e12, "TFLOP/s")],
         }
 

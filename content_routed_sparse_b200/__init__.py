@@ -186,6 +186,16 @@ def get_device_error(stream=None) -> int:
     return int(v.value)
 
 
+_sig("crs_get_device_diag", ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int])
+
+
+def get_device_diag(stream=None) -> list:
+    """Synchronize, read and clear the kernels' diagnostic record (16 words, [0] == 0: none)."""
+    buf = (ctypes.c_uint32 * 16)()
+    _check("crs_get_device_diag", _lib.crs_get_device_diag(_stream(stream), buf, 16))
+    return [int(x) for x in buf]
+
+
 def profile_set(enabled: bool) -> None:
     """Turn per-launch CUDA-event timing on or off (launch counting is always on)."""
     _check("crs_profile_set", _lib.crs_profile_set(1 if enabled else 0))

@@ -98,6 +98,18 @@ extern "C" const char *crs_status_string(int status) {
 
 extern "C" int crs_version(void) { return 100; }
 
+extern "C" int crs_get_device_diag(void *stream, uint32_t *out, int n) {
+    if (!out || n < 1) return CRS_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CRS_TRY_CUDA(cudaStreamSynchronize(s));
+    uint32_t v[16] = {0};
+    uint32_t zero[16] = {0};
+    CRS_TRY_CUDA(cudaMemcpyFromSymbol(v, crs::g_device_diag, sizeof(v)));
+    CRS_TRY_CUDA(cudaMemcpyToSymbol(crs::g_device_diag, zero, sizeof(zero)));
+    for (int i = 0; i < n && i < 16; ++i) out[i] = v[i];
+    return CRS_OK;
+}
+
 extern "C" int crs_get_device_error(void *stream, uint32_t *flags) {
     if (!flags) return CRS_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -15,6 +15,30 @@ __device__ uint32_t g_device_error = 0;
 
 __device__ __forceinline__ void raise_error(uint32_t bit) { atomicOr(&g_device_error, bit); }
 
+// Diagnostic record of the first failure a kernel reports about itself:
+// [0] = kernel id + 1 (0: none), [1] = where (kernel-defined site), [2..4] =
+// blockIdx.x/y/z, [5..] = kernel-defined values.  Read by crs_get_device_diag.
+__device__ uint32_t g_device_diag[16] = {};
+__device__ __forceinline__ void diag_record(uint32_t kernel, uint32_t site, uint32_t a,
+                                            uint32_t b, uint32_t c, uint32_t d) {
+    if (atomicCAS(&g_device_diag[0], 0u, kernel + 1u) == 0u) {
+        g_device_diag[1] = site;
+        g_device_diag[2] = blockIdx.x;
+        g_device_diag[3] = blockIdx.y;
+        g_device_diag[4] = blockIdx.z;
+        g_device_diag[5] = a;
+        g_device_diag[6] = b;
+        g_device_diag[7] = c;
+        g_device_diag[8] = d;
+    }
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -53,6 +77,8 @@ __device__ __forceinline__ float key_score(uint32_t k) {
     uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
     return __uint_as_float(u);
 }
+
+constexpr int kMaxRounds = 8;   // LSH hash rounds supported by the attention kernels
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ long long ceil_div_ll(long long a, long long b) {

@@ -1,6 +1,7 @@
 // libcrs: the whole library as one translation unit (device globals such as the
 // error word are shared by every kernel without relocatable device code).
 #include "api.cu"
+#include "lsh_tc.cu"
 #include "lsh.cu"
 #include "sparse_attn.cu"
 #include "indexer.cu"

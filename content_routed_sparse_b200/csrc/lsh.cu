@@ -7,6 +7,8 @@
 // round; rounds merge by log-sum-exp weights).
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace crs {
@@ -151,7 +153,6 @@ __global__ void __launch_bounds__(kSortThreads) lsh_sort_kernel(const int32_t *_
 // Writes o_r (normalised, fp32) and lse_r at the ORIGINAL position.
 // --------------------------------------------------------------------------
 constexpr int kAttnWarps = 8;
-constexpr int kMaxRounds = 8;
 
 template <typename T, int DH>
 __global__ void __launch_bounds__(kAttnWarps * 32)
@@ -412,10 +413,30 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
                            const int32_t *valid_len, void *O, float *lse, float *o_ws,
                            float *lse_ws, cudaStream_t s) {
     const crs_lsh_params &p = a->p;
+    bool tc_done = false;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && DH == kTcD) {
+        if (p.chunk == kTcM) {
+            // tensor-core path: bf16, d = 64, chunk = 128
+            const size_t smem = sizeof(LshTcSmem) + 1024;
+            CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_chunk_attn_tc_kernel,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+            dim3 grid(ceil_div(p.n, kTcM), p.n_rounds, p.B * p.H);
+            {
+                ProfScope _ps(K_LSH_ATTN_TC, s);
+                lsh_chunk_attn_tc_kernel<<<grid, kTcThreads, smem, s>>>(
+                    static_cast<const __nv_bfloat16 *>(QK), static_cast<const __nv_bfloat16 *>(V),
+                    bucket, perm, inv_perm, valid_len, o_ws, lse_ws, p.H, p.n, p.n_rounds,
+                    a->causal, a->no_self, a->key_norm, a->scale * 1.4426950408889634f);
+            }
+            CRS_CHECK_LAUNCH();
+            tc_done = true;
+        }
+    }
     const int KM = 2 * p.chunk;
     const size_t smem = (size_t)KM * (DH + 1) * 4 + (size_t)KM * DH * 4 + (size_t)KM * 4 +
                         (size_t)kAttnWarps * KM * 4 + (size_t)KM * 4 * 2 +
                         (size_t)KM * (kMaxRounds - 1) * 2 * 4;
+    if (!tc_done) {
     if (smem > 227 * 1024) return CRS_ERR_UNSUPPORTED;
     auto kern = lsh_chunk_attn_kernel<T, DH>;
     CRS_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -428,6 +449,7 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
                                                   a->key_norm, a->scale);
     }
     CRS_CHECK_LAUNCH();
+    }
     const long long warps = (long long)p.B * p.H * p.n;
     const int threads = 256;
     {

@@ -1,0 +1,309 @@
+// K3 on the tensor cores: chunked LSH attention for bf16, d = 64, chunk m = 128.
+//
+// [P1] PaperTrace 2.1.1 §2.1-2.2 (sorted array cut into chunks of m slots; a
+// chunk attends to itself and the previous chunk; edges need the same bucket
+// and are judged on original positions), "重复候选和归一化" (a pair counts once).
+//
+// One CTA (8 warps) per (chunk, round, batch*head):
+//   1. per key slot: original position (via perm), bucket, earlier-round
+//      (bucket, chunk) codes;
+//   2. 16-byte cp.async gathers of the 256 key rows (previous + own chunk)
+//      of Q(=K) and V into 128B-swizzled shared tiles; the own chunk's 128
+//      rows are also the query tile (A operand);
+//   3. one thread issues S = Q K^T (M=128, N=256, K=64) into TMEM;
+//   4. both warpgroups read S from TMEM (warpgroup g owns columns
+//      [128g, 128g+128) of every row), apply the masks and the key scale
+//      (1/|k_j| * scale), exchange row maxima, and write P = exp(S - max) to
+//      shared memory as a bf16 value plus a bf16 residual (K-major tiles);
+//   5. one thread issues O = P_hi V + P_lo V (M=128, N=64, K=2x256, V as an
+//      MN-major operand) into TMEM;
+//   6. the epilogue divides by the row sum and writes o_r and lse_r at the
+//      ORIGINAL position; lsh_combine_kernel merges the rounds.
+#include <math.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace crs {
+
+constexpr int kTcM = 128;        // queries per chunk
+constexpr int kTcN = 256;        // keys: previous + own chunk
+constexpr int kTcD = 64;
+constexpr int kTcThreads = 256;
+constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s: a wait that long means a fault
+
+struct LshTcSmem {
+    unsigned char k[kTcN * 128];        // K tile, rows = keys; rows 128..255 = Q tile
+    unsigned char v[kTcN * 128];        // V tile, rows = keys
+    unsigned char p_hi[4][kTcM * 128];  // P (bf16) in 4 K-blocks of 64 keys
+    unsigned char p_lo[4][kTcM * 128];  // P - bf16(P)
+    int kpos[kTcN];
+    int kbkt[kTcN];
+    int kcode[kMaxRounds - 1][kTcN];
+    float kscale[kTcN];
+    float rowmax[2][kTcM];
+    float rowsum[2][kTcM];
+    uint64_t bar[2];
+    uint32_t tmem_base;
+    int fail;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
+                         const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
+                         const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
+                         float *__restrict__ o_ws, float *__restrict__ lse_ws, int H, int n,
+                         int rounds, int causal, int no_self, int key_norm, float scale_log2) {
+    extern __shared__ unsigned char lsh_tc_raw[];
+    const uint32_t mis = smem_u32(lsh_tc_raw) & 1023u;
+    LshTcSmem &S = *reinterpret_cast<LshTcSmem *>(lsh_tc_raw + ((1024u - mis) & 1023u));
+
+    const int c = blockIdx.x, r = blockIdx.y, bh = blockIdx.z;
+    const int BH = gridDim.z;
+    const int b = bh / H;
+    const int vl = valid_len ? valid_len[b] : n;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int C1 = (n + kTcM - 1) / kTcM + 1;      // chunk-code stride
+    const size_t seg_r = ((size_t)bh * rounds + r) * n;
+
+    // ---- 1. key metadata; key j is slot (c-1)*128 + j
+    {
+        const int j = tid;                       // 256 threads, 256 keys
+        const int s = (c - 1) * kTcM + j;
+        int pos = -1, bk = -1;
+        if (s >= 0 && s < n) {
+            pos = perm[seg_r + s];
+            if (pos < 0 || pos >= n) {
+                raise_error(CRS_DEVERR_INDEX);
+                pos = -1;
+            } else {
+                bk = bucket[seg_r + pos];
+            }
+        }
+        S.kpos[j] = pos;
+        S.kbkt[j] = bk;
+        for (int rr = 0; rr < r; ++rr) {
+            int code = -8;                        // matches no query code
+            if (pos >= 0) {
+                const size_t sg = ((size_t)bh * rounds + rr) * n;
+                code = bucket[sg + pos] * C1 + inv_perm[sg + pos] / kTcM + 1;
+            }
+            S.kcode[rr][j] = code;
+        }
+    }
+    if (tid == 0) {
+        tc::mbar_init(&S.bar[0], 1);
+        tc::mbar_init(&S.bar[1], 1);
+        tc::mbar_fence_init();
+        S.fail = 0;
+    }
+    __syncthreads();
+
+    // ---- 2. gather K (= Q) and V rows
+    const __nv_bfloat16 *Qb = QK + (size_t)bh * n * kTcD;
+    const __nv_bfloat16 *Vb = V + (size_t)bh * n * kTcD;
+#pragma unroll
+    for (int u = 0; u < (kTcN * 8) / kTcThreads; ++u) {
+        const int e = tid + u * kTcThreads;
+        const int j = e >> 3, ch = e & 7;
+        const int pos = S.kpos[j];
+        const bool ok = pos >= 0;
+        const size_t off = ok ? (size_t)pos * kTcD + ch * 8 : 0;
+        cp_async16_zfill(S.k + tc::sw128(j, ch), Qb + off, ok);
+        cp_async16_zfill(S.v + tc::sw128(j, ch), Vb + off, ok);
+    }
+    cp_async_commit();
+    if (warp == 0) tc::tmem_alloc(&S.tmem_base, 512);
+    cp_async_wait<0>();
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    {
+        const int j = tid;
+        float ss = 0.0f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(S.k + tc::sw128(j, ch));
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 f = __bfloat1622float2(p2[t]);
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+            }
+        }
+        const float inv = key_norm ? (ss > 0.0f ? rsqrtf(ss) : 0.0f) : 1.0f;
+        S.kscale[j] = inv * scale_log2;
+    }
+    tc::fence_proxy_async();
+    __syncthreads();
+    const uint32_t tmem = S.tmem_base;
+    const uint32_t kbase = smem_u32(S.k), vbase = smem_u32(S.v);
+
+    // ---- 3. S = Q K^T into TMEM columns [0, 256)
+    if (tid == 0) {
+        constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcM, kTcN, 0, 0);
+#pragma unroll
+        for (int k = 0; k < kTcD / 16; ++k) {
+            const uint64_t a = tc::smem_desc(kbase + kTcM * 128 + k * 32, 16, 1024, tc::kLayoutSW128);
+            const uint64_t bd = tc::smem_desc(kbase + k * 32, 16, 1024, tc::kLayoutSW128);
+            tc::mma_bf16(tmem, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        tc::commit(&S.bar[0]);
+    }
+    bool ok_wait = tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 1);
+    if (__syncthreads_or(!ok_wait)) {
+        if (tid == 0) {
+            const uint64_t a0 = tc::smem_desc(kbase + kTcM * 128, 16, 1024, tc::kLayoutSW128);
+            g_device_diag[9] = tmem;
+            g_device_diag[10] = (uint32_t)a0;
+            g_device_diag[11] = (uint32_t)(a0 >> 32);
+            g_device_diag[12] = tc::idesc_bf16_f32(kTcM, kTcN, 0, 0);
+            g_device_diag[13] = kbase;
+        }
+        tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 2);   // let the MMA drain
+        goto teardown;
+    }
+    tc::fence_after();
+
+    {
+        // ---- 4. masked softmax; warpgroup wg owns columns [128 wg, 128 wg + 128)
+        const int wg = warp >> 2, q = warp & 3, row = q * 32 + lane;
+        const int jq = kTcM + row;
+        const int pos_i = S.kpos[jq];
+        const bool qvalid = pos_i >= 0 && pos_i < vl;
+        const int bk_i = S.kbkt[jq];
+        int code_i[kMaxRounds - 1];
+#pragma unroll
+        for (int rr = 0; rr < kMaxRounds - 1; ++rr) code_i[rr] = (rr < r) ? S.kcode[rr][jq] : 0;
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        uint32_t mbits[4];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            const int col0 = wg * 128 + cb * 32;
+            uint32_t v[32];
+            tc::tmem_ld32(trow + col0, v);
+            tc::tmem_ld_wait();
+            uint32_t mb = 0;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int j = col0 + t;
+                const int pj = S.kpos[j];
+                bool ok = qvalid && pj >= 0 && S.kbkt[j] == bk_i && pj < vl &&
+                          !(causal && pj > pos_i) && !(no_self && pj == pos_i);
+#pragma unroll
+                for (int rr = 0; rr < kMaxRounds - 1; ++rr)
+                    if (rr < r) ok = ok && ((uint32_t)(code_i[rr] - S.kcode[rr][j]) > 1u);
+                if (ok) {
+                    mx = fmaxf(mx, __uint_as_float(v[t]) * S.kscale[j]);
+                    mb |= 1u << t;
+                }
+            }
+            mbits[cb] = mb;
+        }
+        S.rowmax[wg][row] = mx;
+        __syncthreads();
+        const float M = fmaxf(S.rowmax[0][row], S.rowmax[1][row]);
+        float sum = 0.0f;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            const int col0 = wg * 128 + cb * 32;
+            uint32_t v[32];
+            tc::tmem_ld32(trow + col0, v);
+            tc::tmem_ld_wait();
+            const int kb = col0 >> 6;             // 64-key block of P
+            const int ch0 = (col0 & 63) >> 3;     // first 16-byte chunk in the block row
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int t2 = 0; t2 < 4; ++t2) {
+                    float pv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int t = u * 8 + t2 * 2 + e;
+                        const int j = col0 + t;
+                        pv[e] = ((mbits[cb] >> t) & 1u)
+                                    ? exp2f(__uint_as_float(v[t]) * S.kscale[j] - M)
+                                    : 0.0f;
+                        sum += pv[e];
+                    }
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[0], pv[1]);
+                    const float2 hf = __bfloat1622float2(h2);
+                    __nv_bfloat162 l2 = __floats2bfloat162_rn(pv[0] - hf.x, pv[1] - hf.y);
+                    hi[t2] = *reinterpret_cast<uint32_t *>(&h2);
+                    lo[t2] = *reinterpret_cast<uint32_t *>(&l2);
+                }
+                const uint32_t off = tc::sw128(row, ch0 + u);
+                *reinterpret_cast<uint4 *>(S.p_hi[kb] + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(S.p_lo[kb] + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        S.rowsum[wg][row] = sum;
+        tc::fence_proxy_async();
+        tc::fence_before();
+        __syncthreads();
+        tc::fence_after();
+
+        // ---- 5. O = P_hi V + P_lo V into TMEM columns [256, 320)
+        if (tid == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcM, kTcD, 0, 1);
+            uint32_t acc = 0;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                for (int kb2 = 0; kb2 < 4; ++kb2) {
+                    const uint32_t pbase = smem_u32(part ? S.p_lo[kb2] : S.p_hi[kb2]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t a = tc::smem_desc(pbase + k * 32, 16, 1024, tc::kLayoutSW128);
+                        const uint64_t bd = tc::smem_desc(vbase + (kb2 * 64 + k * 16) * 128, 32768,
+                                                          1024, tc::kLayoutSW128);
+                        tc::mma_bf16(tmem + 256, a, bd, idesc, acc);
+                        acc = 1;
+                    }
+                }
+            }
+            tc::commit(&S.bar[1]);
+        }
+        ok_wait = tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 3);
+        if (__syncthreads_or(!ok_wait)) {
+            tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 4);
+            goto teardown;
+        }
+        tc::fence_after();
+
+        // ---- 6. epilogue: warpgroup wg writes output columns [32 wg, 32 wg + 32).
+        // tcgen05.ld is warp-collective (.sync.aligned): every lane loads, rows
+        // without a position (a partial last chunk) only skip the stores.
+        uint32_t v[32];
+        tc::tmem_ld32(trow + 256 + wg * 32, v);
+        tc::tmem_ld_wait();
+        if (pos_i >= 0) {
+            const float L = S.rowsum[0][row] + S.rowsum[1][row];
+            float *o = o_ws + (((size_t)r * BH + bh) * n + pos_i) * kTcD + wg * 32;
+            const bool has = qvalid && L > 0.0f;
+            const float inv = has ? 1.0f / L : 0.0f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                float4 f;
+                f.x = __uint_as_float(v[u * 4 + 0]) * inv;
+                f.y = __uint_as_float(v[u * 4 + 1]) * inv;
+                f.z = __uint_as_float(v[u * 4 + 2]) * inv;
+                f.w = __uint_as_float(v[u * 4 + 3]) * inv;
+                *reinterpret_cast<float4 *>(o + u * 4) = f;
+            }
+            if (wg == 0)
+                lse_ws[((size_t)r * BH + bh) * n + pos_i] =
+                    has ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+
+teardown:
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(S.tmem_base, 512);
+}
+
+}  // namespace crs

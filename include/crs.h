@@ -72,6 +72,13 @@ int crs_version(void);
  * (0 = none).  Returns CRS_ERR_CUDA if the synchronization fails. */
 int crs_get_device_error(void *stream, uint32_t *flags);
 
+/* Diagnostic record of the first failure a kernel reported about itself
+ * since the last call (a bounded wait that gave up, an operand check):
+ * out[0] = kernel id + 1 (0 = none), out[1] = site within the kernel,
+ * out[2..4] = the CTA's blockIdx, out[5..15] = kernel-specific values.
+ * Synchronizes `stream`, copies min(n, 16) words and clears the record. */
+int crs_get_device_diag(void *stream, uint32_t *out, int n);
+
 /* Launch tracing.  [P1] "一个可复现的评测矩阵" and [P2] §1.1 "性能轴" ask for the
  * time of every stage (routing, sort, selection, gather, attention) reported
  * separately; this is how the library provides it.  Every kernel

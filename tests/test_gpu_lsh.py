@@ -84,6 +84,24 @@ def test_lsh_bf16_small(crs, cuda_dev, n, chunk, rounds, nb, vl_frac):
     _attn_and_check(crs, case, *r)
 
 
+@pytest.mark.parametrize("n,rounds,nb,causal,no_self,key_norm,vl_frac", [
+    (1000, 2, 16, 1, 0, 1, 0.05),   # ragged last chunk (n % 128 != 0)
+    (1280, 8, 4, 1, 1, 1, 0.2),     # 8 rounds: dedup against 7 earlier rounds
+    (640, 3, 8, 0, 0, 0, 0.0),      # no causal mask, raw keys
+    (129, 1, 2, 1, 1, 1, 0.0),      # two chunks, the second of one slot
+])
+def test_lsh_bf16_tensor_core_path(crs, cuda_dev, n, rounds, nb, causal, no_self, key_norm, vl_frac):
+    """bf16, d = 64, chunk = 128 runs on the tcgen05 kernel."""
+    case = workloads.lsh_clustered_case(B=1, H=3, n=n, n_buckets=nb, n_rounds=rounds, chunk=128,
+                                        n_centres=8, pad_frac=vl_frac, causal=causal,
+                                        no_self=no_self, seed=n + rounds, device=cuda_dev)
+    case["params"]["key_norm"] = key_norm
+    crs.profile_collect()
+    r = _route_and_check(crs, case)
+    _attn_and_check(crs, case, *r)
+    assert "lsh_chunk_attn_tc" in crs.profile_collect()
+
+
 def test_lsh_fp32_variants(crs, cuda_dev):
     """fp32, causal off / self allowed / raw keys."""
     case = workloads.lsh_fp32_case(n=300, n_rounds=3, chunk=16, causal=0, no_self=0, seed=9,
