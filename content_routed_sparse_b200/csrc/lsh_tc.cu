@@ -4,17 +4,22 @@
 // chunk attends to itself and the previous chunk; edges need the same bucket
 // and are judged on original positions), "重复候选和归一化" (a pair counts once).
 //
-// One CTA (8 warps) per (chunk, round, batch*head):
-//   1. per key slot: original position (via perm), bucket, earlier-round
-//      (bucket, chunk) codes;
-//   2. 16-byte cp.async gathers of the 256 key rows (previous + own chunk)
-//      of Q(=K) and V into 128B-swizzled shared tiles; the own chunk's 128
-//      rows are also the query tile (A operand);
+// One CTA (16 warps) per (chunk, round, batch*head):
+//   1. per key slot of the 256-slot window (previous + own chunk): original
+//      position (via perm), bucket, earlier-round (bucket, chunk) codes;
+//   2. 16-byte cp.async gathers of the 256 rows of Q(=K) and V into
+//      128B-swizzled shared tiles; the own chunk's 128 rows are also the
+//      query tile (A operand);
 //   3. one thread issues S = Q K^T (M=128, N=256, K=64) into TMEM;
-//   4. both warpgroups read S from TMEM (warpgroup g owns columns
-//      [128g, 128g+128) of every row), apply the masks and the key scale
-//      (1/|k_j| * scale), exchange row maxima, and write P = exp(S - max) to
-//      shared memory as a bf16 value plus a bf16 residual (K-major tiles);
+//   4. the masked softmax reads S from TMEM; warpgroup g owns columns
+//      [64g, 64g+64) of every row.  Slots are sorted by (bucket, position),
+//      so the keys of a query that share its bucket and precede it form ONE
+//      contiguous column range [run start, own slot]: the bucket, causal and
+//      padding masks are a range test, and 32-column chunks outside the range
+//      are skipped warp-uniformly (tcgen05.ld is warp-collective).  Pairs seen
+//      in an earlier round are masked per element (specialised per round).
+//      P = exp(S - max) goes to shared memory as a bf16 value plus a bf16
+//      residual (K-major tiles);
 //   5. one thread issues O = P_hi V + P_lo V (M=128, N=64, K=2x256, V as an
 //      MN-major operand) into TMEM;
 //   6. the epilogue divides by the row sum and writes o_r and lse_r at the
@@ -29,24 +34,115 @@ namespace crs {
 constexpr int kTcM = 128;        // queries per chunk
 constexpr int kTcN = 256;        // keys: previous + own chunk
 constexpr int kTcD = 64;
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 512;  // 4 warpgroups
 constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s: a wait that long means a fault
+constexpr int kBktBefore = -1;                  // absent slot before the sequence
+constexpr int kBktAfter = 0x7fffffff;           // absent slot after the sequence
 
 struct LshTcSmem {
     unsigned char k[kTcN * 128];        // K tile, rows = keys; rows 128..255 = Q tile
     unsigned char v[kTcN * 128];        // V tile, rows = keys
-    unsigned char p_hi[4][kTcM * 128];  // P (bf16) in 4 K-blocks of 64 keys
+    unsigned char p_hi[4][kTcM * 128];  // P (bf16), K-block g = columns of warpgroup g
     unsigned char p_lo[4][kTcM * 128];  // P - bf16(P)
     int kpos[kTcN];
-    int kbkt[kTcN];
-    int kcode[kMaxRounds - 1][kTcN];
-    float kscale[kTcN];
-    float rowmax[2][kTcM];
-    float rowsum[2][kTcM];
+    int kbkt[kTcN];                     // nondecreasing over the window
+    int krun0[kTcN];                    // first slot of this key's bucket run
+    int krun1[kTcN];                    // last slot of the run whose position < valid_len
+    int kcode[kMaxRounds - 1][kTcN];    // earlier rounds: bucket * C1 + chunk + 1
+    float kscale[kTcN];                 // scale * log2(e) / |k_j|
+    float rowmax[4][kTcM];
+    float rowsum[4][kTcM];
     uint64_t bar[2];
     uint32_t tmem_base;
-    int fail;
 };
+
+struct LshTcRow {
+    int row, jq, lo, hi, pos_i;
+    bool qvalid, excl_self;
+};
+
+// Step 4 for rounds with R earlier rounds: returns the row maximum (log2 units).
+template <int R>
+__device__ __forceinline__ float lsh_tc_softmax(LshTcSmem &S, const LshTcRow &q, uint32_t trow,
+                                                int wg) {
+    int code_i[R > 0 ? R : 1];
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr) code_i[rr] = S.kcode[rr][q.jq];
+    uint32_t mbits[2];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int col0 = wg * 64 + cc * 32;
+        const bool need = q.qvalid && col0 <= q.hi && col0 + 31 >= q.lo;
+        uint32_t mb = 0;
+        if (__any_sync(0xffffffffu, need)) {
+            uint32_t v[32];
+            tc::tmem_ld32(trow + col0, v);
+            tc::tmem_ld_wait();
+            if (need) {
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int j = col0 + t;
+                    bool ok = j >= q.lo && j <= q.hi && !(q.excl_self && j == q.jq);
+#pragma unroll
+                    for (int rr = 0; rr < R; ++rr)
+                        ok = ok && ((uint32_t)(code_i[rr] - S.kcode[rr][j]) > 1u);
+                    if (ok) {
+                        mx = fmaxf(mx, __uint_as_float(v[t]) * S.kscale[j]);
+                        mb |= 1u << t;
+                    }
+                }
+            }
+        }
+        mbits[cc] = mb;
+    }
+    S.rowmax[wg][q.row] = mx;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(S.rowmax[0][q.row], S.rowmax[1][q.row]),
+                          fmaxf(S.rowmax[2][q.row], S.rowmax[3][q.row]));
+    float sum = 0.0f;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int col0 = wg * 64 + cc * 32;
+        const int ch0 = cc * 4;            // first 16-byte chunk of these 32 keys in the block row
+        uint32_t hi[16], lo[16];
+        if (__any_sync(0xffffffffu, mbits[cc] != 0u)) {
+            uint32_t v[32];
+            tc::tmem_ld32(trow + col0, v);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int t2 = 0; t2 < 16; ++t2) {
+                float pv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = t2 * 2 + e;
+                    pv[e] = ((mbits[cc] >> t) & 1u)
+                                ? exp2f(__uint_as_float(v[t]) * S.kscale[col0 + t] - M)
+                                : 0.0f;
+                    sum += pv[e];
+                }
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[0], pv[1]);
+                const float2 hf = __bfloat1622float2(h2);
+                __nv_bfloat162 l2 = __floats2bfloat162_rn(pv[0] - hf.x, pv[1] - hf.y);
+                hi[t2] = *reinterpret_cast<uint32_t *>(&h2);
+                lo[t2] = *reinterpret_cast<uint32_t *>(&l2);
+            }
+        } else {
+#pragma unroll
+            for (int t2 = 0; t2 < 16; ++t2) hi[t2] = lo[t2] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t off = tc::sw128(q.row, ch0 + u);
+            *reinterpret_cast<uint4 *>(S.p_hi[wg] + off) =
+                make_uint4(hi[u * 4], hi[u * 4 + 1], hi[u * 4 + 2], hi[u * 4 + 3]);
+            *reinterpret_cast<uint4 *>(S.p_lo[wg] + off) =
+                make_uint4(lo[u * 4], lo[u * 4 + 1], lo[u * 4 + 2], lo[u * 4 + 3]);
+        }
+    }
+    S.rowsum[wg][q.row] = sum;
+    return M;
+}
 
 __global__ void __launch_bounds__(kTcThreads, 1)
 lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
@@ -66,11 +162,11 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     const int C1 = (n + kTcM - 1) / kTcM + 1;      // chunk-code stride
     const size_t seg_r = ((size_t)bh * rounds + r) * n;
 
-    // ---- 1. key metadata; key j is slot (c-1)*128 + j
-    {
-        const int j = tid;                       // 256 threads, 256 keys
+    // ---- 1. key metadata; window key j is slot (c-1)*128 + j
+    if (tid < kTcN) {
+        const int j = tid;
         const int s = (c - 1) * kTcM + j;
-        int pos = -1, bk = -1;
+        int pos = -1, bk = (s < 0) ? kBktBefore : kBktAfter;
         if (s >= 0 && s < n) {
             pos = perm[seg_r + s];
             if (pos < 0 || pos >= n) {
@@ -95,11 +191,10 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         tc::mbar_init(&S.bar[0], 1);
         tc::mbar_init(&S.bar[1], 1);
         tc::mbar_fence_init();
-        S.fail = 0;
     }
     __syncthreads();
 
-    // ---- 2. gather K (= Q) and V rows
+    // ---- 2. gather K (= Q) and V rows; bucket runs of the window
     const __nv_bfloat16 *Qb = QK + (size_t)bh * n * kTcD;
     const __nv_bfloat16 *Vb = V + (size_t)bh * n * kTcD;
 #pragma unroll
@@ -114,11 +209,28 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     }
     cp_async_commit();
     if (warp == 0) tc::tmem_alloc(&S.tmem_base, 512);
+    if (tid < kTcN) {
+        // the window's buckets are nondecreasing: binary searches give the run
+        const int j = tid, bk = S.kbkt[j];
+        int a = 0, z = j;                         // first index with kbkt >= bk
+        while (a < z) {
+            const int mid = (a + z) >> 1;
+            if (S.kbkt[mid] < bk) a = mid + 1; else z = mid;
+        }
+        S.krun0[j] = a;
+        a = j;                                    // last index in the run with pos < vl
+        z = kTcN - 1;
+        while (a < z) {
+            const int mid = (a + z + 1) >> 1;
+            if (S.kbkt[mid] == bk && S.kpos[mid] < vl) a = mid; else z = mid - 1;
+        }
+        S.krun1[j] = a;
+    }
     cp_async_wait<0>();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
-    {
+    if (tid < kTcN) {
         const int j = tid;
         float ss = 0.0f;
 #pragma unroll
@@ -153,94 +265,34 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     }
     bool ok_wait = tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 1);
     if (__syncthreads_or(!ok_wait)) {
-        if (tid == 0) {
-            const uint64_t a0 = tc::smem_desc(kbase + kTcM * 128, 16, 1024, tc::kLayoutSW128);
-            g_device_diag[9] = tmem;
-            g_device_diag[10] = (uint32_t)a0;
-            g_device_diag[11] = (uint32_t)(a0 >> 32);
-            g_device_diag[12] = tc::idesc_bf16_f32(kTcM, kTcN, 0, 0);
-            g_device_diag[13] = kbase;
-        }
         tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 2);   // let the MMA drain
         goto teardown;
     }
     tc::fence_after();
 
     {
-        // ---- 4. masked softmax; warpgroup wg owns columns [128 wg, 128 wg + 128)
-        const int wg = warp >> 2, q = warp & 3, row = q * 32 + lane;
-        const int jq = kTcM + row;
-        const int pos_i = S.kpos[jq];
-        const bool qvalid = pos_i >= 0 && pos_i < vl;
-        const int bk_i = S.kbkt[jq];
-        int code_i[kMaxRounds - 1];
-#pragma unroll
-        for (int rr = 0; rr < kMaxRounds - 1; ++rr) code_i[rr] = (rr < r) ? S.kcode[rr][jq] : 0;
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        uint32_t mbits[4];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            const int col0 = wg * 128 + cb * 32;
-            uint32_t v[32];
-            tc::tmem_ld32(trow + col0, v);
-            tc::tmem_ld_wait();
-            uint32_t mb = 0;
-#pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const int j = col0 + t;
-                const int pj = S.kpos[j];
-                bool ok = qvalid && pj >= 0 && S.kbkt[j] == bk_i && pj < vl &&
-                          !(causal && pj > pos_i) && !(no_self && pj == pos_i);
-#pragma unroll
-                for (int rr = 0; rr < kMaxRounds - 1; ++rr)
-                    if (rr < r) ok = ok && ((uint32_t)(code_i[rr] - S.kcode[rr][j]) > 1u);
-                if (ok) {
-                    mx = fmaxf(mx, __uint_as_float(v[t]) * S.kscale[j]);
-                    mb |= 1u << t;
-                }
-            }
-            mbits[cb] = mb;
+        // ---- 4. masked softmax; warpgroup wg owns columns [64 wg, 64 wg + 64)
+        const int wg = warp >> 2, quad = warp & 3;
+        LshTcRow q;
+        q.row = quad * 32 + lane;
+        q.jq = kTcM + q.row;
+        q.pos_i = S.kpos[q.jq];
+        q.qvalid = q.pos_i >= 0 && q.pos_i < vl;
+        q.lo = S.krun0[q.jq];
+        q.hi = causal ? (no_self ? q.jq - 1 : q.jq) : S.krun1[q.jq];
+        q.excl_self = (!causal) && no_self;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        float M;
+        switch (r) {
+            case 0: M = lsh_tc_softmax<0>(S, q, trow, wg); break;
+            case 1: M = lsh_tc_softmax<1>(S, q, trow, wg); break;
+            case 2: M = lsh_tc_softmax<2>(S, q, trow, wg); break;
+            case 3: M = lsh_tc_softmax<3>(S, q, trow, wg); break;
+            case 4: M = lsh_tc_softmax<4>(S, q, trow, wg); break;
+            case 5: M = lsh_tc_softmax<5>(S, q, trow, wg); break;
+            case 6: M = lsh_tc_softmax<6>(S, q, trow, wg); break;
+            default: M = lsh_tc_softmax<7>(S, q, trow, wg); break;
         }
-        S.rowmax[wg][row] = mx;
-        __syncthreads();
-        const float M = fmaxf(S.rowmax[0][row], S.rowmax[1][row]);
-        float sum = 0.0f;
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            const int col0 = wg * 128 + cb * 32;
-            uint32_t v[32];
-            tc::tmem_ld32(trow + col0, v);
-            tc::tmem_ld_wait();
-            const int kb = col0 >> 6;             // 64-key block of P
-            const int ch0 = (col0 & 63) >> 3;     // first 16-byte chunk in the block row
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int t2 = 0; t2 < 4; ++t2) {
-                    float pv[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int t = u * 8 + t2 * 2 + e;
-                        const int j = col0 + t;
-                        pv[e] = ((mbits[cb] >> t) & 1u)
-                                    ? exp2f(__uint_as_float(v[t]) * S.kscale[j] - M)
-                                    : 0.0f;
-                        sum += pv[e];
-                    }
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[0], pv[1]);
-                    const float2 hf = __bfloat1622float2(h2);
-                    __nv_bfloat162 l2 = __floats2bfloat162_rn(pv[0] - hf.x, pv[1] - hf.y);
-                    hi[t2] = *reinterpret_cast<uint32_t *>(&h2);
-                    lo[t2] = *reinterpret_cast<uint32_t *>(&l2);
-                }
-                const uint32_t off = tc::sw128(row, ch0 + u);
-                *reinterpret_cast<uint4 *>(S.p_hi[kb] + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(S.p_lo[kb] + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-        }
-        S.rowsum[wg][row] = sum;
         tc::fence_proxy_async();
         tc::fence_before();
         __syncthreads();
@@ -274,19 +326,20 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         }
         tc::fence_after();
 
-        // ---- 6. epilogue: warpgroup wg writes output columns [32 wg, 32 wg + 32).
-        // tcgen05.ld is warp-collective (.sync.aligned): every lane loads, rows
-        // without a position (a partial last chunk) only skip the stores.
-        uint32_t v[32];
-        tc::tmem_ld32(trow + 256 + wg * 32, v);
+        // ---- 6. epilogue: warpgroup wg writes output columns [16 wg, 16 wg + 16).
+        // tcgen05.ld is warp-collective: every lane loads; rows without a
+        // position (a partial last chunk) only skip the stores.
+        uint32_t v[16];
+        tc::tmem_ld16(trow + 256 + wg * 16, v);
         tc::tmem_ld_wait();
-        if (pos_i >= 0) {
-            const float L = S.rowsum[0][row] + S.rowsum[1][row];
-            float *o = o_ws + (((size_t)r * BH + bh) * n + pos_i) * kTcD + wg * 32;
-            const bool has = qvalid && L > 0.0f;
+        if (q.pos_i >= 0) {
+            const float L = S.rowsum[0][q.row] + S.rowsum[1][q.row] + S.rowsum[2][q.row] +
+                            S.rowsum[3][q.row];
+            float *o = o_ws + (((size_t)r * BH + bh) * n + q.pos_i) * kTcD + wg * 16;
+            const bool has = q.qvalid && L > 0.0f;
             const float inv = has ? 1.0f / L : 0.0f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 float4 f;
                 f.x = __uint_as_float(v[u * 4 + 0]) * inv;
                 f.y = __uint_as_float(v[u * 4 + 1]) * inv;
@@ -295,7 +348,7 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
                 *reinterpret_cast<float4 *>(o + u * 4) = f;
             }
             if (wg == 0)
-                lse_ws[((size_t)r * BH + bh) * n + pos_i] =
+                lse_ws[((size_t)r * BH + bh) * n + q.pos_i] =
                     has ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
         }
     }
