@@ -69,6 +69,64 @@ __global__ void __launch_bounds__(kHashTok) lsh_hash_kernel(const T *__restrict_
     bucket[((size_t)bh * rounds + r) * n + i] = arg;
 }
 
+// K1 specialised for a compile-time head dim D and half-width HALF: the token
+// row lives in registers, R_{h,r} is read from shared memory as broadcast
+// float4s; the FMA chain of every u_k is the same as above (index order from
+// 0), so the bucket ids are identical.
+template <typename T, int D, int HALF>
+__global__ void __launch_bounds__(kHashTok) lsh_hash_fixed_kernel(const T *__restrict__ X,
+                                                                  const float *__restrict__ R,
+                                                                  int32_t *__restrict__ bucket,
+                                                                  int H, int n, int rounds) {
+    __shared__ __align__(16) float Rs[D * HALF];
+    const int bh = blockIdx.z, h = bh % H;
+    const int i = blockIdx.x * kHashTok + threadIdx.x;
+    float x[D];
+    if (i < n) {
+        const T *xr = X + ((size_t)bh * n + i) * D;
+#pragma unroll
+        for (int t = 0; t < D; ++t) x[t] = to_f32(xr[t]);
+    }
+    for (int r = blockIdx.y; r < rounds; r += gridDim.y) {
+        __syncthreads();
+        const float4 *Rg = reinterpret_cast<const float4 *>(R + ((size_t)h * rounds + r) * D * HALF);
+        for (int e = threadIdx.x; e < D * HALF / 4; e += kHashTok)
+            reinterpret_cast<float4 *>(Rs)[e] = Rg[e];
+        __syncthreads();
+        if (i >= n) continue;
+        float bp = 0.0f, bn = 0.0f;
+        int ap = 0, an = 0;
+#pragma unroll
+        for (int k0 = 0; k0 < HALF; k0 += 32) {
+            constexpr int W = HALF < 32 ? HALF : 32;
+            float u[W];
+#pragma unroll
+            for (int j = 0; j < W; ++j) u[j] = 0.0f;
+#pragma unroll
+            for (int t = 0; t < D; ++t) {
+                const float xv = x[t];
+                const float4 *rr = reinterpret_cast<const float4 *>(Rs + t * HALF + k0);
+#pragma unroll
+                for (int j4 = 0; j4 < W / 4; ++j4) {
+                    const float4 rv = rr[j4];
+                    u[4 * j4 + 0] = __fmaf_rn(xv, rv.x, u[4 * j4 + 0]);
+                    u[4 * j4 + 1] = __fmaf_rn(xv, rv.y, u[4 * j4 + 1]);
+                    u[4 * j4 + 2] = __fmaf_rn(xv, rv.z, u[4 * j4 + 2]);
+                    u[4 * j4 + 3] = __fmaf_rn(xv, rv.w, u[4 * j4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                const int k = k0 + j;
+                if (k == 0 || u[j] > bp) { bp = u[j]; ap = k; }
+                const float nu = -u[j];
+                if (k == 0 || nu > bn) { bn = nu; an = k; }
+            }
+        }
+        bucket[((size_t)bh * rounds + r) * n + i] = (bp >= bn) ? ap : HALF + an;
+    }
+}
+
 // --------------------------------------------------------------------------
 // K2: stable counting sort of one (b, h, round) segment per CTA.
 // Histogram -> exclusive scan (bucket bases) -> tiles of blockDim positions
@@ -297,7 +355,7 @@ lsh_chunk_attn_kernel(const T *__restrict__ QK, const T *__restrict__ V,
 }
 
 // --------------------------------------------------------------------------
-// K4: merge the rounds.  One warp per (b*h, position):
+// K4: merge the rounds.  One thread per (b*h, position, 4 output dims):
 //   LSE = log sum_r exp(lse_r),  O = sum_r exp(lse_r - LSE) o_r.
 // Padded positions and queries with no edge in any round give 0 / -inf.
 // --------------------------------------------------------------------------
@@ -305,10 +363,12 @@ template <int DH>
 __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
                                    const int32_t *__restrict__ valid_len, float *__restrict__ O,
                                    float *__restrict__ lse_out, int BH, int H, int n, int rounds) {
-    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (gw >= BH * n) return;
-    const int bh = gw / n, pos = gw - bh * n;
+    constexpr int G4 = DH / 4;                  // float4 groups per row
+    const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gt >= (long long)BH * n * G4) return;
+    const int g = (int)(gt % G4);
+    const long long rowi = gt / G4;
+    const int bh = (int)(rowi / n), pos = (int)(rowi - (long long)bh * n);
     const int vl = valid_len ? valid_len[bh / H] : n;
     float l[kMaxRounds];
     float mx = -INFINITY;
@@ -317,24 +377,30 @@ __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *
         l[r] = (r < rounds) ? lse_ws[((size_t)r * BH + bh) * n + pos] : -INFINITY;
         mx = fmaxf(mx, l[r]);
     }
-    float *o = O + ((size_t)bh * n + pos) * DH;
+    float4 *o = reinterpret_cast<float4 *>(O + ((size_t)bh * n + pos) * DH) + g;
     if (pos >= vl || mx == -INFINITY) {
-        for (int k = lane; k < DH; k += 32) o[k] = 0.0f;
-        if (lse_out && lane == 0) lse_out[(size_t)bh * n + pos] = -INFINITY;
+        *o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (lse_out && g == 0) lse_out[(size_t)bh * n + pos] = -INFINITY;
         return;
     }
     float z = 0.0f;
 #pragma unroll
     for (int r = 0; r < kMaxRounds; ++r) z += (r < rounds && l[r] != -INFINITY) ? __expf(l[r] - mx) : 0.0f;
     const float LSE = mx + logf(z);
-    for (int k = lane; k < DH; k += 32) {
-        float acc = 0.0f;
-        for (int r = 0; r < rounds; ++r)
-            if (l[r] != -INFINITY)
-                acc = fmaf(__expf(l[r] - LSE), o_ws[(((size_t)r * BH + bh) * n + pos) * DH + k], acc);
-        o[k] = acc;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        if (r < rounds && l[r] != -INFINITY) {
+            const float wgt = __expf(l[r] - LSE);
+            const float4 v = reinterpret_cast<const float4 *>(o_ws + (((size_t)r * BH + bh) * n + pos) * DH)[g];
+            acc.x = fmaf(wgt, v.x, acc.x);
+            acc.y = fmaf(wgt, v.y, acc.y);
+            acc.z = fmaf(wgt, v.z, acc.z);
+            acc.w = fmaf(wgt, v.w, acc.w);
+        }
     }
-    if (lse_out && lane == 0) lse_out[(size_t)bh * n + pos] = LSE;
+    *o = acc;
+    if (lse_out && g == 0) lse_out[(size_t)bh * n + pos] = LSE;
 }
 
 // ------------------------------------------------------------ host side --
@@ -368,7 +434,26 @@ extern "C" int crs_lsh_route(const crs_lsh_params *p, const void *X, const float
     const size_t smem = ((size_t)p->d * half + (size_t)kHashTok * (p->d + 1)) * sizeof(float);
     if (smem > 200 * 1024) return CRS_ERR_UNSUPPORTED;
     dim3 grid(ceil_div(p->n, kHashTok), p->n_rounds, p->B * p->H);
-    if (p->dtype == CRS_F32) {
+    if (p->d == 64 && (half == 32 || half == 8)) {
+        // specialised kernel: one CTA per 128 tokens covers every round
+        dim3 g2(ceil_div(p->n, kHashTok), 1, p->B * p->H);
+        ProfScope _ps(K_LSH_HASH, s);
+        if (p->dtype == CRS_F32) {
+            if (half == 32)
+                lsh_hash_fixed_kernel<float, 64, 32><<<g2, kHashTok, 0, s>>>(
+                    static_cast<const float *>(X), R, bucket, p->H, p->n, p->n_rounds);
+            else
+                lsh_hash_fixed_kernel<float, 64, 8><<<g2, kHashTok, 0, s>>>(
+                    static_cast<const float *>(X), R, bucket, p->H, p->n, p->n_rounds);
+        } else {
+            if (half == 32)
+                lsh_hash_fixed_kernel<__nv_bfloat16, 64, 32><<<g2, kHashTok, 0, s>>>(
+                    static_cast<const __nv_bfloat16 *>(X), R, bucket, p->H, p->n, p->n_rounds);
+            else
+                lsh_hash_fixed_kernel<__nv_bfloat16, 64, 8><<<g2, kHashTok, 0, s>>>(
+                    static_cast<const __nv_bfloat16 *>(X), R, bucket, p->H, p->n, p->n_rounds);
+        }
+    } else if (p->dtype == CRS_F32) {
         CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_hash_kernel<float>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         {
@@ -420,6 +505,9 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
             const size_t smem = sizeof(LshTcSmem) + 1024;
             CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_chunk_attn_tc_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+            CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_chunk_attn_tc_kernel,
+                                              cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              (int)cudaSharedmemCarveoutMaxShared));
             dim3 grid(ceil_div(p.n, kTcM), p.n_rounds, p.B * p.H);
             {
                 ProfScope _ps(K_LSH_ATTN_TC, s);
@@ -450,11 +538,11 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
     }
     CRS_CHECK_LAUNCH();
     }
-    const long long warps = (long long)p.B * p.H * p.n;
+    const long long work = (long long)p.B * p.H * p.n * (DH / 4);
     const int threads = 256;
     {
         ProfScope _ps(K_LSH_COMBINE, s);
-        lsh_combine_kernel<DH><<<(unsigned)ceil_div_ll(warps * 32, threads), threads, 0, s>>>(
+        lsh_combine_kernel<DH><<<(unsigned)ceil_div_ll(work, threads), threads, 0, s>>>(
             o_ws, lse_ws, valid_len, static_cast<float *>(O), lse, p.B * p.H, p.H, p.n, p.n_rounds);
     }
     CRS_CHECK_LAUNCH();

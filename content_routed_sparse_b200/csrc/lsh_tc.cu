@@ -4,26 +4,30 @@
 // chunk attends to itself and the previous chunk; edges need the same bucket
 // and are judged on original positions), "重复候选和归一化" (a pair counts once).
 //
-// One CTA (16 warps) per (chunk, round, batch*head):
+// One CTA (8 warps, two CTAs resident per SM) per (chunk, round, batch*head):
 //   1. per key slot of the 256-slot window (previous + own chunk): original
 //      position (via perm), bucket, earlier-round (bucket, chunk) codes;
 //   2. 16-byte cp.async gathers of the 256 rows of Q(=K) and V into
 //      128B-swizzled shared tiles; the own chunk's 128 rows are also the
 //      query tile (A operand);
 //   3. one thread issues S = Q K^T (M=128, N=256, K=64) into TMEM;
-//   4. the masked softmax reads S from TMEM; warpgroup g owns columns
-//      [64g, 64g+64) of every row.  Slots are sorted by (bucket, position),
+//   4. the masked softmax reads S from TMEM (pass 1: row maxima, warpgroup g
+//      owns columns [128g, 128g+128)).  Slots are sorted by (bucket, position),
 //      so the keys of a query that share its bucket and precede it form ONE
 //      contiguous column range [run start, own slot]: the bucket, causal and
 //      padding masks are a range test, and 32-column chunks outside the range
 //      are skipped warp-uniformly (tcgen05.ld is warp-collective).  Pairs seen
 //      in an earlier round are masked per element (specialised per round).
-//      P = exp(S - max) goes to shared memory as a bf16 value plus a bf16
-//      residual (K-major tiles);
-//   5. one thread issues O = P_hi V + P_lo V (M=128, N=64, K=2x256, V as an
-//      MN-major operand) into TMEM;
+//      Pass 2 writes P = exp(S - max) for one 128-key half at a time into
+//      shared memory as a bf16 value plus a bf16 residual (K-major tiles),
+//      reusing the K tile's space (S is complete by then);
+//   5. after each half, one thread issues O += P_hi V_half + P_lo V_half
+//      (M=128, N=64, V as an MN-major operand) into TMEM columns [0, 64),
+//      which the first half's S no longer needs;
 //   6. the epilogue divides by the row sum and writes o_r and lse_r at the
 //      ORIGINAL position; lsh_combine_kernel merges the rounds.
+// Resources per CTA: 256 TMEM columns, ~107 KB shared memory, 256 threads,
+// so two CTAs share an SM and overlap each other's latency.
 #include <math.h>
 
 #include "common.cuh"
@@ -34,25 +38,31 @@ namespace crs {
 constexpr int kTcM = 128;        // queries per chunk
 constexpr int kTcN = 256;        // keys: previous + own chunk
 constexpr int kTcD = 64;
-constexpr int kTcThreads = 512;  // 4 warpgroups
+constexpr int kTcThreads = 256;  // 2 warpgroups
+constexpr uint32_t kTcCols = 256;
 constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s: a wait that long means a fault
 constexpr int kBktBefore = -1;                  // absent slot before the sequence
 constexpr int kBktAfter = 0x7fffffff;           // absent slot after the sequence
 
 struct LshTcSmem {
-    unsigned char k[kTcN * 128];        // K tile, rows = keys; rows 128..255 = Q tile
+    // K tile (rows = keys; rows 128..255 = Q tile) until S is computed, then
+    // the P buffer of one 128-key half: hi[2 blocks], lo[2 blocks] (K-major)
+    unsigned char kp[4][kTcM * 128];
     unsigned char v[kTcN * 128];        // V tile, rows = keys
-    unsigned char p_hi[4][kTcM * 128];  // P (bf16), K-block g = columns of warpgroup g
-    unsigned char p_lo[4][kTcM * 128];  // P - bf16(P)
     int kpos[kTcN];
-    int kbkt[kTcN];                     // nondecreasing over the window
-    int krun0[kTcN];                    // first slot of this key's bucket run
-    int krun1[kTcN];                    // last slot of the run whose position < valid_len
+    union {                             // lifetimes do not overlap:
+        int kbkt[kTcN];                 //   buckets (nondecreasing), until the runs are known
+        uint32_t mbits[kTcN / 32][kTcM];//   pass-1 masks: [32-key chunk][row]
+    } u1;
+    union {
+        uint32_t krun[kTcN];            //   bucket run of a key: first slot | (last slot with
+                                        //   position < valid_len) << 16, read before pass 1
+        float rowsum[2][kTcM];          //   written after pass 2
+    } u2;
     int kcode[kMaxRounds - 1][kTcN];    // earlier rounds: bucket * C1 + chunk + 1
     float kscale[kTcN];                 // scale * log2(e) / |k_j|
-    float rowmax[4][kTcM];
-    float rowsum[4][kTcM];
-    uint64_t bar[2];
+    float rowmax[2][kTcM];
+    uint64_t bar[3];
     uint32_t tmem_base;
 };
 
@@ -61,18 +71,17 @@ struct LshTcRow {
     bool qvalid, excl_self;
 };
 
-// Step 4 for rounds with R earlier rounds: returns the row maximum (log2 units).
+// Pass 1 for a query row with R earlier rounds: warpgroup wg scans columns
+// [128 wg, 128 wg + 128); stores the per-chunk masks, returns the partial max.
 template <int R>
-__device__ __forceinline__ float lsh_tc_softmax(LshTcSmem &S, const LshTcRow &q, uint32_t trow,
-                                                int wg) {
+__device__ __forceinline__ float lsh_tc_pass1(LshTcSmem &S, const LshTcRow &q, uint32_t trow, int wg) {
     int code_i[R > 0 ? R : 1];
 #pragma unroll
     for (int rr = 0; rr < R; ++rr) code_i[rr] = S.kcode[rr][q.jq];
-    uint32_t mbits[2];
     float mx = -INFINITY;
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-        const int col0 = wg * 64 + cc * 32;
+    for (int cc = 0; cc < 4; ++cc) {
+        const int col0 = wg * 128 + cc * 32;
         const bool need = q.qvalid && col0 <= q.hi && col0 + 31 >= q.lo;
         uint32_t mb = 0;
         if (__any_sync(0xffffffffu, need)) {
@@ -94,21 +103,26 @@ __device__ __forceinline__ float lsh_tc_softmax(LshTcSmem &S, const LshTcRow &q,
                 }
             }
         }
-        mbits[cc] = mb;
+        S.u1.mbits[col0 >> 5][q.row] = mb;
     }
-    S.rowmax[wg][q.row] = mx;
-    __syncthreads();
-    const float M = fmaxf(fmaxf(S.rowmax[0][q.row], S.rowmax[1][q.row]),
-                          fmaxf(S.rowmax[2][q.row], S.rowmax[3][q.row]));
+    return mx;
+}
+
+// Pass 2 for the 64 keys [col0, col0 + 64) of one row: P into K-block `blk`
+// of the P buffer (value and residual); returns the partial row sum.
+__device__ __forceinline__ float lsh_tc_pass2(LshTcSmem &S, const LshTcRow &q, uint32_t trow,
+                                              int col0, int blk, float M) {
     float sum = 0.0f;
+    unsigned char *p_hi = S.kp[blk];
+    unsigned char *p_lo = S.kp[2 + blk];
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
-        const int col0 = wg * 64 + cc * 32;
-        const int ch0 = cc * 4;            // first 16-byte chunk of these 32 keys in the block row
+        const int c0 = col0 + cc * 32;
+        const uint32_t mb = S.u1.mbits[c0 >> 5][q.row];
         uint32_t hi[16], lo[16];
-        if (__any_sync(0xffffffffu, mbits[cc] != 0u)) {
+        if (__any_sync(0xffffffffu, mb != 0u)) {
             uint32_t v[32];
-            tc::tmem_ld32(trow + col0, v);
+            tc::tmem_ld32(trow + c0, v);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int t2 = 0; t2 < 16; ++t2) {
@@ -116,9 +130,8 @@ __device__ __forceinline__ float lsh_tc_softmax(LshTcSmem &S, const LshTcRow &q,
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int t = t2 * 2 + e;
-                    pv[e] = ((mbits[cc] >> t) & 1u)
-                                ? exp2f(__uint_as_float(v[t]) * S.kscale[col0 + t] - M)
-                                : 0.0f;
+                    pv[e] = ((mb >> t) & 1u) ? exp2f(__uint_as_float(v[t]) * S.kscale[c0 + t] - M)
+                                             : 0.0f;
                     sum += pv[e];
                 }
                 __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[0], pv[1]);
@@ -133,18 +146,40 @@ __device__ __forceinline__ float lsh_tc_softmax(LshTcSmem &S, const LshTcRow &q,
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const uint32_t off = tc::sw128(q.row, ch0 + u);
-            *reinterpret_cast<uint4 *>(S.p_hi[wg] + off) =
+            const uint32_t off = tc::sw128(q.row, cc * 4 + u);
+            *reinterpret_cast<uint4 *>(p_hi + off) =
                 make_uint4(hi[u * 4], hi[u * 4 + 1], hi[u * 4 + 2], hi[u * 4 + 3]);
-            *reinterpret_cast<uint4 *>(S.p_lo[wg] + off) =
+            *reinterpret_cast<uint4 *>(p_lo + off) =
                 make_uint4(lo[u * 4], lo[u * 4 + 1], lo[u * 4 + 2], lo[u * 4 + 3]);
         }
     }
-    S.rowsum[wg][q.row] = sum;
-    return M;
+    return sum;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+// O (TMEM columns [0, 64)) += P_hi V_half + P_lo V_half for keys [128 half, +128).
+__device__ __forceinline__ void lsh_tc_issue_pv(LshTcSmem &S, uint32_t tmem, int half,
+                                                bool first) {
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcM, kTcD, 0, 1);
+    const uint32_t vbase = smem_u32(S.v);
+    uint32_t acc = first ? 0u : 1u;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            const uint32_t pbase = smem_u32(S.kp[part * 2 + blk]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t a = tc::smem_desc(pbase + k * 32, 16, 1024, tc::kLayoutSW128);
+                const uint64_t bd = tc::smem_desc(vbase + (half * 128 + blk * 64 + k * 16) * 128,
+                                                  32768, 1024, tc::kLayoutSW128);
+                tc::mma_bf16(tmem, a, bd, idesc, acc);
+                acc = 1u;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 2)
 lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
                          const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
                          const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
@@ -162,8 +197,8 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     const int C1 = (n + kTcM - 1) / kTcM + 1;      // chunk-code stride
     const size_t seg_r = ((size_t)bh * rounds + r) * n;
 
-    // ---- 1. key metadata; window key j is slot (c-1)*128 + j
-    if (tid < kTcN) {
+    // ---- 1. key metadata; window key j = tid is slot (c-1)*128 + j
+    {
         const int j = tid;
         const int s = (c - 1) * kTcM + j;
         int pos = -1, bk = (s < 0) ? kBktBefore : kBktAfter;
@@ -177,7 +212,7 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
             }
         }
         S.kpos[j] = pos;
-        S.kbkt[j] = bk;
+        S.u1.kbkt[j] = bk;
         for (int rr = 0; rr < r; ++rr) {
             int code = -8;                        // matches no query code
             if (pos >= 0) {
@@ -190,52 +225,55 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     if (tid == 0) {
         tc::mbar_init(&S.bar[0], 1);
         tc::mbar_init(&S.bar[1], 1);
+        tc::mbar_init(&S.bar[2], 1);
         tc::mbar_fence_init();
     }
     __syncthreads();
 
     // ---- 2. gather K (= Q) and V rows; bucket runs of the window
-    const __nv_bfloat16 *Qb = QK + (size_t)bh * n * kTcD;
-    const __nv_bfloat16 *Vb = V + (size_t)bh * n * kTcD;
+    {
+        const __nv_bfloat16 *Qb = QK + (size_t)bh * n * kTcD;
+        const __nv_bfloat16 *Vb = V + (size_t)bh * n * kTcD;
 #pragma unroll
-    for (int u = 0; u < (kTcN * 8) / kTcThreads; ++u) {
-        const int e = tid + u * kTcThreads;
-        const int j = e >> 3, ch = e & 7;
-        const int pos = S.kpos[j];
-        const bool ok = pos >= 0;
-        const size_t off = ok ? (size_t)pos * kTcD + ch * 8 : 0;
-        cp_async16_zfill(S.k + tc::sw128(j, ch), Qb + off, ok);
-        cp_async16_zfill(S.v + tc::sw128(j, ch), Vb + off, ok);
+        for (int u = 0; u < (kTcN * 8) / kTcThreads; ++u) {
+            const int e = tid + u * kTcThreads;
+            const int j = e >> 3, ch = e & 7;
+            const int pos = S.kpos[j];
+            const bool ok = pos >= 0;
+            const size_t off = ok ? (size_t)pos * kTcD + ch * 8 : 0;
+            cp_async16_zfill(&S.kp[0][0] + tc::sw128(j, ch), Qb + off, ok);
+            cp_async16_zfill(S.v + tc::sw128(j, ch), Vb + off, ok);
+        }
+        cp_async_commit();
     }
-    cp_async_commit();
-    if (warp == 0) tc::tmem_alloc(&S.tmem_base, 512);
-    if (tid < kTcN) {
+    if (warp == 0) tc::tmem_alloc(&S.tmem_base, kTcCols);
+    {
         // the window's buckets are nondecreasing: binary searches give the run
-        const int j = tid, bk = S.kbkt[j];
+        const int j = tid, bk = S.u1.kbkt[j];
         int a = 0, z = j;                         // first index with kbkt >= bk
         while (a < z) {
             const int mid = (a + z) >> 1;
-            if (S.kbkt[mid] < bk) a = mid + 1; else z = mid;
+            if (S.u1.kbkt[mid] < bk) a = mid + 1; else z = mid;
         }
-        S.krun0[j] = a;
+        const int run0 = a;
         a = j;                                    // last index in the run with pos < vl
         z = kTcN - 1;
         while (a < z) {
             const int mid = (a + z + 1) >> 1;
-            if (S.kbkt[mid] == bk && S.kpos[mid] < vl) a = mid; else z = mid - 1;
+            if (S.u1.kbkt[mid] == bk && S.kpos[mid] < vl) a = mid; else z = mid - 1;
         }
-        S.krun1[j] = a;
+        S.u2.krun[j] = (uint32_t)run0 | ((uint32_t)a << 16);
     }
     cp_async_wait<0>();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
-    if (tid < kTcN) {
+    {
         const int j = tid;
         float ss = 0.0f;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(S.k + tc::sw128(j, ch));
+            const uint4 v = *reinterpret_cast<const uint4 *>(&S.kp[0][0] + tc::sw128(j, ch));
             const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
@@ -250,11 +288,11 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     tc::fence_proxy_async();
     __syncthreads();
     const uint32_t tmem = S.tmem_base;
-    const uint32_t kbase = smem_u32(S.k), vbase = smem_u32(S.v);
 
     // ---- 3. S = Q K^T into TMEM columns [0, 256)
     if (tid == 0) {
         constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcM, kTcN, 0, 0);
+        const uint32_t kbase = smem_u32(&S.kp[0][0]);
 #pragma unroll
         for (int k = 0; k < kTcD / 16; ++k) {
             const uint64_t a = tc::smem_desc(kbase + kTcM * 128 + k * 32, 16, 1024, tc::kLayoutSW128);
@@ -271,75 +309,71 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     tc::fence_after();
 
     {
-        // ---- 4. masked softmax; warpgroup wg owns columns [64 wg, 64 wg + 64)
         const int wg = warp >> 2, quad = warp & 3;
         LshTcRow q;
         q.row = quad * 32 + lane;
         q.jq = kTcM + q.row;
         q.pos_i = S.kpos[q.jq];
         q.qvalid = q.pos_i >= 0 && q.pos_i < vl;
-        q.lo = S.krun0[q.jq];
-        q.hi = causal ? (no_self ? q.jq - 1 : q.jq) : S.krun1[q.jq];
+        const uint32_t run = S.u2.krun[q.jq];
+        q.lo = (int)(run & 0xffffu);
+        q.hi = causal ? (no_self ? q.jq - 1 : q.jq) : (int)(run >> 16);
         q.excl_self = (!causal) && no_self;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        float M;
+
+        // ---- 4a. pass 1: masks and row maxima
+        float mx;
         switch (r) {
-            case 0: M = lsh_tc_softmax<0>(S, q, trow, wg); break;
-            case 1: M = lsh_tc_softmax<1>(S, q, trow, wg); break;
-            case 2: M = lsh_tc_softmax<2>(S, q, trow, wg); break;
-            case 3: M = lsh_tc_softmax<3>(S, q, trow, wg); break;
-            case 4: M = lsh_tc_softmax<4>(S, q, trow, wg); break;
-            case 5: M = lsh_tc_softmax<5>(S, q, trow, wg); break;
-            case 6: M = lsh_tc_softmax<6>(S, q, trow, wg); break;
-            default: M = lsh_tc_softmax<7>(S, q, trow, wg); break;
+            case 0: mx = lsh_tc_pass1<0>(S, q, trow, wg); break;
+            case 1: mx = lsh_tc_pass1<1>(S, q, trow, wg); break;
+            case 2: mx = lsh_tc_pass1<2>(S, q, trow, wg); break;
+            case 3: mx = lsh_tc_pass1<3>(S, q, trow, wg); break;
+            case 4: mx = lsh_tc_pass1<4>(S, q, trow, wg); break;
+            case 5: mx = lsh_tc_pass1<5>(S, q, trow, wg); break;
+            case 6: mx = lsh_tc_pass1<6>(S, q, trow, wg); break;
+            default: mx = lsh_tc_pass1<7>(S, q, trow, wg); break;
         }
-        tc::fence_proxy_async();
-        tc::fence_before();
+        S.rowmax[wg][q.row] = mx;
         __syncthreads();
-        tc::fence_after();
+        const float M = fmaxf(S.rowmax[0][q.row], S.rowmax[1][q.row]);
 
-        // ---- 5. O = P_hi V + P_lo V into TMEM columns [256, 320)
-        if (tid == 0) {
-            constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcM, kTcD, 0, 1);
-            uint32_t acc = 0;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-#pragma unroll
-                for (int kb2 = 0; kb2 < 4; ++kb2) {
-                    const uint32_t pbase = smem_u32(part ? S.p_lo[kb2] : S.p_hi[kb2]);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t a = tc::smem_desc(pbase + k * 32, 16, 1024, tc::kLayoutSW128);
-                        const uint64_t bd = tc::smem_desc(vbase + (kb2 * 64 + k * 16) * 128, 32768,
-                                                          1024, tc::kLayoutSW128);
-                        tc::mma_bf16(tmem + 256, a, bd, idesc, acc);
-                        acc = 1;
-                    }
-                }
+        // ---- 4b/5. per 128-key half: P into the buffer, then O += P V_half
+        float sum = 0.0f;
+        for (int half = 0; half < 2; ++half) {
+            if (half == 1) {
+                // the buffer is free once the first half's P.V has completed
+                ok_wait = tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 3);
+                if (__syncthreads_or(!ok_wait)) goto teardown;
+                tc::fence_after();
             }
-            tc::commit(&S.bar[1]);
+            sum += lsh_tc_pass2(S, q, trow, half * 128 + wg * 64, wg, M);
+            tc::fence_proxy_async();
+            tc::fence_before();
+            __syncthreads();
+            tc::fence_after();
+            if (tid == 0) {
+                lsh_tc_issue_pv(S, tmem, half, half == 0);
+                tc::commit(&S.bar[1 + half]);
+            }
         }
-        ok_wait = tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 3);
-        if (__syncthreads_or(!ok_wait)) {
-            tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 4);
-            goto teardown;
-        }
+        S.u2.rowsum[wg][q.row] = sum;
+        ok_wait = tc::mbar_wait_bounded(&S.bar[2], 0, kTcWaitNs, K_LSH_ATTN_TC, 4);
+        if (__syncthreads_or(!ok_wait)) goto teardown;
         tc::fence_after();
 
-        // ---- 6. epilogue: warpgroup wg writes output columns [16 wg, 16 wg + 16).
+        // ---- 6. epilogue: warpgroup wg writes output columns [32 wg, 32 wg + 32).
         // tcgen05.ld is warp-collective: every lane loads; rows without a
         // position (a partial last chunk) only skip the stores.
-        uint32_t v[16];
-        tc::tmem_ld16(trow + 256 + wg * 16, v);
+        uint32_t v[32];
+        tc::tmem_ld32(trow + wg * 32, v);
         tc::tmem_ld_wait();
         if (q.pos_i >= 0) {
-            const float L = S.rowsum[0][q.row] + S.rowsum[1][q.row] + S.rowsum[2][q.row] +
-                            S.rowsum[3][q.row];
-            float *o = o_ws + (((size_t)r * BH + bh) * n + q.pos_i) * kTcD + wg * 16;
+            const float L = S.u2.rowsum[0][q.row] + S.u2.rowsum[1][q.row];
+            float *o = o_ws + (((size_t)r * BH + bh) * n + q.pos_i) * kTcD + wg * 32;
             const bool has = q.qvalid && L > 0.0f;
             const float inv = has ? 1.0f / L : 0.0f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 float4 f;
                 f.x = __uint_as_float(v[u * 4 + 0]) * inv;
                 f.y = __uint_as_float(v[u * 4 + 1]) * inv;
@@ -356,7 +390,7 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
 teardown:
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(S.tmem_base, 512);
+    if (warp == 0) tc::tmem_dealloc(S.tmem_base, kTcCols);
 }
 
 }  // namespace crs
