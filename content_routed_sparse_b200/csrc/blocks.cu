@@ -237,6 +237,65 @@ block_score_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict_
     sc_out[((size_t)sh * G + g) * n_full + b0 + bl] = fmaf(0.5f, quad, lin);
 }
 
+// K9a specialised for G query heads and rank R: one thread per block holds
+// the G x (1 + R) dot products in registers; the block's descriptor rows are
+// streamed once with 16-byte loads and the scaled queries are read from
+// shared memory (the same address for every lane: a broadcast).
+template <int G, int R>
+__global__ void __launch_bounds__(128)
+block_score_fixed_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ mu,
+                         const float *__restrict__ xi, float *__restrict__ sc_out, int n_kv,
+                         int n_q, int n_full, float scale) {
+    __shared__ __align__(16) float sq[G][kBdD];
+    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
+    for (int e = threadIdx.x; e < G * kBdD; e += blockDim.x) {
+        const int g = e / kBdD, d = e - g * kBdD;
+        sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+    }
+    __syncthreads();
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= n_full) return;
+    const size_t blk = (size_t)sh * n_full + b;
+    const float4 *m4 = reinterpret_cast<const float4 *>(mu + blk * kBdD);
+    const float4 *x4 = reinterpret_cast<const float4 *>(xi + blk * R * kBdD);
+    float lin[G], pr[G][R];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        lin[g] = 0.0f;
+#pragma unroll
+        for (int e = 0; e < R; ++e) pr[g][e] = 0.0f;
+    }
+#pragma unroll 2
+    for (int d4 = 0; d4 < kBdD / 4; ++d4) {
+        const float4 mv = __ldg(m4 + d4);
+        float4 xv[R];
+#pragma unroll
+        for (int e = 0; e < R; ++e) xv[e] = __ldg(x4 + e * (kBdD / 4) + d4);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float4 qv = *reinterpret_cast<const float4 *>(&sq[g][d4 * 4]);
+            lin[g] = fmaf(qv.x, mv.x, lin[g]);
+            lin[g] = fmaf(qv.y, mv.y, lin[g]);
+            lin[g] = fmaf(qv.z, mv.z, lin[g]);
+            lin[g] = fmaf(qv.w, mv.w, lin[g]);
+#pragma unroll
+            for (int e = 0; e < R; ++e) {
+                pr[g][e] = fmaf(qv.x, xv[e].x, pr[g][e]);
+                pr[g][e] = fmaf(qv.y, xv[e].y, pr[g][e]);
+                pr[g][e] = fmaf(qv.z, xv[e].z, pr[g][e]);
+                pr[g][e] = fmaf(qv.w, xv[e].w, pr[g][e]);
+            }
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float quad = 0.0f;
+#pragma unroll
+        for (int e = 0; e < R; ++e) quad = fmaf(pr[g][e], pr[g][e], quad);
+        sc_out[((size_t)sh * G + g) * n_full + b] = fmaf(0.5f, quad, lin[g]);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // K9b: group softmax sum, top blocks, token list.  One CTA per (seq, KV head).
 // ---------------------------------------------------------------------------
@@ -457,12 +516,19 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
     CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a));
     float *sc = static_cast<float *>(ws);
+    if (G == 8 && p->b.rank == 4) {
+        dim3 gf(ceil_div(n_full, 128), p->b.n_seq * p->b.n_kv);
+        ProfScope _ps(K_BLK_SCORE, s);
+        block_score_fixed_kernel<8, 4><<<gf, 128, 0, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu,
+                                                         xi, sc, p->b.n_kv, p->n_q, n_full, p->scale);
+    } else {
     dim3 ga(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv);
     {
         ProfScope _ps(K_BLK_SCORE, s);
         block_score_kernel<<<ga, kBsThreads, smem_a, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu, xi,
                                                           sc, p->b.n_kv, p->n_q, G, p->b.rank, n_full,
                                                           p->scale);
+    }
     }
     CRS_CHECK_LAUNCH();
     const int cap = p->top_blocks * p->b.L + p->window;

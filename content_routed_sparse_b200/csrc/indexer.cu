@@ -120,25 +120,49 @@ __device__ uint32_t block_radix_select(KeyFn key, int n, int k, SelScratch &sc, 
 
 // Writes, in index order, the selected elements: key > T, plus the first
 // need_eq elements with key == T.  emit(pos, i, key) is called per element.
+// Each thread owns kCompactItems consecutive elements of a tile, so a tile of
+// kSelThreads * kCompactItems elements costs two block-wide scans.
+constexpr int kCompactItems = 16;
+
 template <typename KeyFn, typename EmitFn>
 __device__ int block_compact(KeyFn key, int n, uint32_t T, int need_eq, bool take_all,
                              SelScratch &sc, EmitFn emit) {
     int out_base = 0, eq_base = 0;
-    for (int t0 = 0; t0 < n; t0 += kSelThreads) {
-        const int i = t0 + threadIdx.x;
-        uint32_t kk = 0;
-        bool gt = false, eq = false;
-        if (i < n) {
-            kk = key(i);
-            gt = take_all || kk > T;
-            eq = !take_all && kk == T;
+    constexpr int kTile = kSelThreads * kCompactItems;
+    for (int t0 = 0; t0 < n; t0 += kTile) {
+        const int i0 = t0 + threadIdx.x * kCompactItems;
+        uint32_t kk[kCompactItems];
+        int ce = 0;
+#pragma unroll
+        for (int u = 0; u < kCompactItems; ++u) {
+            const int i = i0 + u;
+            kk[u] = (i < n) ? key(i) : 0u;
+            ce += (i < n && !take_all && kk[u] == T) ? 1 : 0;
         }
         int eq_tot;
-        const int eq_rank = eq_base + block_excl_scan(eq ? 1 : 0, sc.warp, eq_tot);
-        const bool take = gt || (eq && eq_rank < need_eq);
+        int eq_rank = eq_base + block_excl_scan(ce, sc.warp, eq_tot);
+        bool tk[kCompactItems];
+        int ct = 0;
+#pragma unroll
+        for (int u = 0; u < kCompactItems; ++u) {
+            const int i = i0 + u;
+            bool take = false;
+            if (i < n) {
+                if (take_all || kk[u] > T) {
+                    take = true;
+                } else if (kk[u] == T) {
+                    take = eq_rank < need_eq;
+                    ++eq_rank;
+                }
+            }
+            tk[u] = take;
+            ct += take ? 1 : 0;
+        }
         int tk_tot;
-        const int pos = out_base + block_excl_scan(take ? 1 : 0, sc.warp, tk_tot);
-        if (take) emit(pos, i, kk);
+        int pos = out_base + block_excl_scan(ct, sc.warp, tk_tot);
+#pragma unroll
+        for (int u = 0; u < kCompactItems; ++u)
+            if (tk[u]) emit(pos++, i0 + u, kk[u]);
         out_base += tk_tot;
         eq_base += eq_tot;
     }
@@ -309,6 +333,231 @@ __global__ void __launch_bounds__(kSelThreads) idx_merge_kernel(IdxArgs a, int r
     if (threadIdx.x == 0) a.out_cnt[row] = cnt;
 }
 
+// ---------------------------------------------------------------------------
+// Decode path.  A decode row's scores are O(ctx) (one query per sequence), so
+// they are written once as order-preserving keys (4 B per cached key) while
+// the index-key cache is streamed; no score matrix exists.
+//   idx_decode_score_kernel: grid (tile, row): 4096 keys per CTA, scores ->
+//     keys, and a histogram of the keys' top 12 bits added to the row's
+//     global histogram;
+//   idx_decode_select_kernel: one CTA per row: the histogram locates the
+//     12-bit bucket holding the k-th largest key; only that bucket's keys are
+//     resolved exactly (radix select on the low bits), then one ordered
+//     compaction over the row writes the ascending index list.
+// ---------------------------------------------------------------------------
+constexpr int kDecTile = 4096;
+constexpr int kDecBins = 4096;            // top 12 bits of the key
+constexpr int kDecThreads = 256;
+constexpr int kDecEqCap = 16384;          // bucket size resolved in shared memory
+
+struct DecArgs {
+    const __nv_bfloat16 *q;
+    const float *w;
+    const __nv_bfloat16 *k;
+    const int64_t *k_off;
+    uint32_t *keys;                       // [total keys] score keys
+    uint32_t *hist;                       // [rows][kDecBins]
+    int32_t *out_idx;
+    int32_t *out_cnt;
+    int n_rows, H, topk, max_tiles;
+};
+
+// Scores on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+// 16 keys form the M side (A operand, ldmatrix from a swizzled shared tile),
+// the index heads (padded to 8) the N side, the 64 dims K.  Thread (g, t4)
+// receives the dot products of keys g and g+8 with heads 2 t4 and 2 t4 + 1;
+// the weighted ReLU sum over heads 0..3 needs one shuffle.  Each warp streams
+// its own 16-key slices of the 4096-key tile through a 2-deep cp.async ring.
+__device__ __forceinline__ void ldsm_x4_a(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecSlice = 16;                           // keys per mma slice
+
+__global__ void __launch_bounds__(kDecThreads) idx_decode_score_kernel(DecArgs a) {
+    __shared__ __align__(128) unsigned char ktile[kDecWarps][2][kDecSlice * 128];
+    __shared__ uint32_t sh[kDecBins];
+    const int tile = blockIdx.x, row = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t kb = a.k_off[row];
+    int nv = (int)(a.k_off[row + 1] - kb);
+    if (nv > a.max_tiles * kDecTile) {
+        if (tile == 0 && threadIdx.x == 0) raise_error(CRS_DEVERR_INDEX);
+        nv = a.max_tiles * kDecTile;
+    }
+    if (nv <= a.topk) return;                 // every key is selected; no score needed
+    const int s0 = tile * kDecTile;
+    if (s0 >= nv) return;
+    const int ns = min(kDecTile, nv - s0);
+    const int H = a.H;
+    const int g = lane >> 2, t4 = lane & 3;
+    // B fragments: head n = g (zero for n >= H), dims 16 kk + 2 t4 (+8)
+    uint32_t bq[4][2];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v = 0u;
+            if (g < H) {
+                const __nv_bfloat16 *qp = a.q + ((size_t)row * H + g) * kIdxDim + kk * 16 + hh * 8 + t4 * 2;
+                v = *reinterpret_cast<const uint32_t *>(qp);
+            }
+            bq[kk][hh] = v;
+        }
+    }
+    const float w0 = (2 * t4 < H) ? a.w[(size_t)row * H + 2 * t4] : 0.0f;
+    const float w1 = (2 * t4 + 1 < H) ? a.w[(size_t)row * H + 2 * t4 + 1] : 0.0f;
+    for (int e = threadIdx.x; e < kDecBins; e += kDecThreads) sh[e] = 0u;
+    __syncthreads();
+
+    const int nsl = (ns + kDecSlice - 1) / kDecSlice;     // 16-key slices in the tile
+    bool nonfinite = false;
+    auto issue = [&](int sl, int buf) {
+        // 16 keys x 8 chunks of 16 B: lane handles chunks lane and lane + 32
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = lane + u * 32;
+            const int r = e >> 3, c = e & 7;
+            const int key = sl * kDecSlice + r;
+            const bool ok = key < ns;
+            const __nv_bfloat16 *src = a.k + (size_t)(kb + s0 + (ok ? key : 0)) * kIdxDim + c * 8;
+            cp_async16_zfill(&ktile[warp][buf][0] + r * 128 + ((c ^ (r & 7)) << 4), src, ok);
+        }
+        cp_async_commit();
+    };
+    int sl = warp;
+    if (sl < nsl) issue(sl, 0);
+    for (int it = 0; sl < nsl; ++it, sl += kDecWarps) {
+        const int buf = it & 1;
+        const int nxt = sl + kDecWarps;
+        if (nxt < nsl) {
+            issue(nxt, buf ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncwarp();
+        float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint32_t base = smem_u32(&ktile[warp][buf][0]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            // A: rows = keys; matrices (keys 0-7, k lo), (8-15, lo), (0-7, hi), (8-15, hi)
+            const int mi = lane >> 3;
+            const int r = (lane & 7) + ((mi & 1) << 3);
+            const int ch = kk * 2 + (mi >> 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_a(base + r * 128 + ((ch ^ (r & 7)) << 4), a0, a1, a2, a3);
+            mma16816(c, a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
+        }
+        // c0, c1: key g, heads 2 t4, 2 t4 + 1; c2, c3: key g + 8
+        if (!isfinite(c[0]) || !isfinite(c[1]) || !isfinite(c[2]) || !isfinite(c[3])) nonfinite = true;
+        float s_lo = fmaf(w0, fmaxf(c[0], 0.0f), w1 * fmaxf(c[1], 0.0f));
+        float s_hi = fmaf(w0, fmaxf(c[2], 0.0f), w1 * fmaxf(c[3], 0.0f));
+        // heads 2 t4 .. 2 t4 + 1 live in lanes t4 = 0..3 of the quad: sum the quad
+        s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 1);
+        s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 1);
+        s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 2);
+        s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 2);
+        if (t4 == 0) {
+            const int k_lo = sl * kDecSlice + g, k_hi = k_lo + 8;
+            if (k_lo < ns) {
+                const uint32_t key = score_key(s_lo);
+                a.keys[kb + s0 + k_lo] = key;
+                atomicAdd(&sh[key >> 20], 1u);
+            }
+            if (k_hi < ns) {
+                const uint32_t key = score_key(s_hi);
+                a.keys[kb + s0 + k_hi] = key;
+                atomicAdd(&sh[key >> 20], 1u);
+            }
+        }
+        __syncwarp();
+    }
+    if (__syncthreads_or(nonfinite) && threadIdx.x == 0) raise_error(CRS_DEVERR_NONFINITE);
+    uint32_t *gh = a.hist + (size_t)row * kDecBins;
+    for (int e = threadIdx.x; e < kDecBins; e += kDecThreads)
+        if (sh[e]) atomicAdd(gh + e, sh[e]);
+}
+
+__global__ void __launch_bounds__(kSelThreads) idx_decode_select_kernel(DecArgs a) {
+    __shared__ SelScratch sc;
+    extern __shared__ uint32_t eqk[];         // [kDecEqCap]
+    __shared__ int bc[4];
+    const int row = blockIdx.x;
+    const int64_t kb = a.k_off[row];
+    int nv = (int)(a.k_off[row + 1] - kb);
+    nv = min(max(nv, 0), a.max_tiles * kDecTile);
+    const int topk = a.topk;
+    int32_t *o = a.out_idx + (size_t)row * topk;
+    if (nv <= topk) {
+        for (int i = threadIdx.x; i < topk; i += kSelThreads) o[i] = (i < nv) ? i : -1;
+        if (threadIdx.x == 0) a.out_cnt[row] = nv;
+        return;
+    }
+    const uint32_t *keys = a.keys + kb;
+    const uint32_t *gh = a.hist + (size_t)row * kDecBins;
+    // 1. the 12-bit bucket B holding the topk-th largest key (scan from the top)
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        constexpr int per = kDecBins / 32;             // bins per lane, top-down
+        int cnt = 0;
+        for (int u = 0; u < per; ++u) cnt += (int)gh[kDecBins - 1 - (lane * per + u)];
+        int incl = cnt;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o2);
+            if (lane >= o2) incl += t;
+        }
+        const int before = incl - cnt;
+        if (before < topk && topk <= incl) {
+            int acc = before;
+            for (int u = 0; u < per; ++u) {
+                const int bin = kDecBins - 1 - (lane * per + u);
+                const int c = (int)gh[bin];
+                if (acc < topk && topk <= acc + c) {
+                    bc[0] = bin;
+                    bc[1] = topk - acc;                 // to take from bucket B
+                    bc[2] = c;                          // size of bucket B
+                }
+                acc += c;
+            }
+        }
+    }
+    __syncthreads();
+    const uint32_t B = (uint32_t)bc[0];
+    const int need_b = bc[1], size_b = bc[2];
+    uint32_t T;
+    int need_eq;
+    if (size_b <= kDecEqCap) {
+        // 2. gather bucket B's keys (index order) and resolve them exactly
+        auto inb = [&](int i) { return (keys[i] >> 20) == B; };
+        block_compact([&](int i) { return inb(i) ? 1u : 0u; }, nv, 0u, 0, false, sc,
+                      [&](int pos, int i, uint32_t) { eqk[pos] = keys[i]; });
+        __syncthreads();
+        T = block_radix_select([&](int i) { return eqk[i]; }, size_b, need_b, sc, need_eq);
+    } else {
+        // a very populated bucket (e.g. many exactly-equal scores): select over the whole row
+        T = block_radix_select([&](int i) { return keys[i]; }, nv, topk, sc, need_eq);
+    }
+    // 3. ordered compaction over the row
+    const int cnt = block_compact([&](int i) { return keys[i]; }, nv, T, need_eq, false, sc,
+                                  [&](int pos, int i, uint32_t) { o[pos] = i; });
+    for (int i = cnt + threadIdx.x; i < topk; i += kSelThreads) o[i] = -1;
+    if (threadIdx.x == 0) a.out_cnt[row] = cnt;
+}
+
 static int idx_validate(const crs_indexer_params *p) {
     if (!p) return CRS_ERR_INVALID_ARG;
     if (p->mode != CRS_IDX_PREFILL && p->mode != CRS_IDX_DECODE) return CRS_ERR_INVALID_ARG;
@@ -334,8 +583,18 @@ static void idx_geometry(const crs_indexer_params *p, int &max_slices, int &ws_r
 
 using namespace crs;
 
+static size_t dec_ws_parts(const crs_indexer_params *p, size_t &keys_bytes) {
+    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    keys_bytes = al((size_t)p->n_rows * (size_t)max(p->max_keys, 1) * 4);
+    return keys_bytes + al((size_t)p->n_rows * kDecBins * 4);
+}
+
 extern "C" size_t crs_indexer_topk_workspace_size(const crs_indexer_params *p) {
     if (idx_validate(p)) return 0;
+    if (p->mode == CRS_IDX_DECODE) {
+        size_t kbytes;
+        return dec_ws_parts(p, kbytes);
+    }
     int max_slices, ws_rows;
     idx_geometry(p, max_slices, ws_rows);
     if (max_slices <= 1 || ws_rows == 0) return 0;
@@ -353,6 +612,39 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
     if (p->mode == CRS_IDX_DECODE && !k_offsets) return CRS_ERR_INVALID_ARG;
     const size_t need = crs_indexer_topk_workspace_size(p);
     if (need > 0 && (!ws || ws_bytes < need)) return CRS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p->mode == CRS_IDX_DECODE) {
+        size_t kbytes;
+        dec_ws_parts(p, kbytes);
+        DecArgs d;
+        d.q = static_cast<const __nv_bfloat16 *>(q_idx);
+        d.w = w;
+        d.k = static_cast<const __nv_bfloat16 *>(k_idx);
+        d.k_off = k_offsets;
+        d.keys = static_cast<uint32_t *>(ws);
+        d.hist = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kbytes);
+        d.out_idx = out_idx;
+        d.out_cnt = out_count;
+        d.n_rows = p->n_rows;
+        d.H = p->n_idx_heads;
+        d.topk = p->topk;
+        d.max_tiles = max(1, ceil_div(p->max_keys, kDecTile));
+        CRS_TRY_CUDA(cudaMemsetAsync(d.hist, 0, (size_t)p->n_rows * kDecBins * 4, s));
+        {
+            ProfScope _ps(K_IDX_SLICE, s);
+            idx_decode_score_kernel<<<dim3(d.max_tiles, p->n_rows), kDecThreads, 0, s>>>(d);
+        }
+        CRS_CHECK_LAUNCH();
+        CRS_TRY_CUDA(cudaFuncSetAttribute(idx_decode_select_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          kDecEqCap * 4));
+        {
+            ProfScope _ps(K_IDX_SELECT, s);
+            idx_decode_select_kernel<<<p->n_rows, kSelThreads, kDecEqCap * 4, s>>>(d);
+        }
+        CRS_CHECK_LAUNCH();
+        return CRS_OK;
+    }
     int max_slices, ws_rows;
     idx_geometry(p, max_slices, ws_rows);
     if (max_slices > 64) return CRS_ERR_UNSUPPORTED;
@@ -379,7 +671,6 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
         a.cand_idx = reinterpret_cast<int32_t *>(b + al(cand * 4));
         a.cand_cnt = reinterpret_cast<int32_t *>(b + 2 * al(cand * 4));
     }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t smem = (size_t)kSlice * 4 + (kMaxIdxHeads * kIdxDim + kMaxIdxHeads) * 4;
     CRS_TRY_CUDA(cudaFuncSetAttribute(idx_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem));
