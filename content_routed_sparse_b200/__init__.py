@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libcrs.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libcrs.so not found at {LIB_PATH}; build it with "
-        "`python -m content_routed_sparse_b200.build` (nvcc, sm_100a)")
+        "`python content_routed_sparse_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -1,6 +1,8 @@
 """Build libcrs.so in-tree for sm_100a with nvcc.
 
-    python -m content_routed_sparse_b200.build [--force]
+    python content_routed_sparse_b200/build.py [--force] [--ptxas-v]
+
+(run by path: importing the package loads the library this script builds)
 
 The library is one translation unit (csrc/libcrs.cu) and exports only the
 crs_* C symbols declared in include/crs.h.

@@ -181,6 +181,8 @@ struct IdxArgs {
     int32_t *cand_idx;            // [ws_rows, max_slices, topk]
     int32_t *cand_cnt;            // [ws_rows, max_slices]
     int n_rows, H, topk, max_slices;
+    const int32_t *row_list;      // optional: rows to process (blockIdx -> row_list[i])
+    const int32_t *list_count;    //   and how many entries of row_list are live
 };
 
 __device__ __forceinline__ void row_range(const IdxArgs &a, int row, int64_t &kb, int &nv) {
@@ -206,7 +208,15 @@ __global__ void __launch_bounds__(kSelThreads) idx_slice_kernel(IdxArgs a) {
     float *sw = sq + kMaxIdxHeads * kIdxDim;                          // [H]
     __shared__ SelScratch sc;
 
-    const int slice = blockIdx.x, row = blockIdx.y;
+    const int slice = blockIdx.x;
+    int row = blockIdx.y, wrow;
+    if (a.row_list) {
+        if ((int)blockIdx.y >= *a.list_count) return;
+        row = a.row_list[blockIdx.y];
+        wrow = blockIdx.y;
+    } else {
+        wrow = ws_row(a, row);
+    }
     int64_t kb;
     int nv;
     row_range(a, row, kb, nv);
@@ -280,7 +290,7 @@ __global__ void __launch_bounds__(kSelThreads) idx_slice_kernel(IdxArgs a) {
         for (int i = cnt + threadIdx.x; i < topk; i += kSelThreads) o[i] = -1;
         if (threadIdx.x == 0) a.out_cnt[row] = cnt;
     } else {
-        const size_t base = ((size_t)ws_row(a, row) * a.max_slices + slice) * topk;
+        const size_t base = ((size_t)wrow * a.max_slices + slice) * topk;
         uint32_t *ck = a.cand_key + base;
         int32_t *ci = a.cand_idx + base;
         const int cnt = block_compact(key, ns, T, need_eq, take_all, sc,
@@ -288,21 +298,27 @@ __global__ void __launch_bounds__(kSelThreads) idx_slice_kernel(IdxArgs a) {
                                           ck[pos] = kk;
                                           ci[pos] = s0 + i;
                                       });
-        if (threadIdx.x == 0) a.cand_cnt[(size_t)ws_row(a, row) * a.max_slices + slice] = cnt;
+        if (threadIdx.x == 0) a.cand_cnt[(size_t)wrow * a.max_slices + slice] = cnt;
     }
 }
 
 __global__ void __launch_bounds__(kSelThreads) idx_merge_kernel(IdxArgs a, int row0) {
     __shared__ SelScratch sc;
     __shared__ int soff[65];
-    const int row = row0 + blockIdx.x;
+    int row = row0 + blockIdx.x, wr;
+    if (a.row_list) {
+        if ((int)blockIdx.x >= *a.list_count) return;
+        row = a.row_list[blockIdx.x];
+        wr = blockIdx.x;
+    } else {
+        wr = ws_row(a, row);
+    }
     int64_t kb;
     int nv;
     row_range(a, row, kb, nv);
     nv = min(max(nv, 0), a.max_slices * kSlice);
     const int n_slices = ceil_div(nv, kSlice);
     if (n_slices <= 1 || nv <= a.topk) return;   // answered by idx_slice_kernel
-    const int wr = ws_row(a, row);
     const int topk = a.topk;
     if (threadIdx.x == 0) {
         int s = 0;
@@ -583,6 +599,15 @@ static void idx_geometry(const crs_indexer_params *p, int &max_slices, int &ws_r
 
 using namespace crs;
 
+// tensor-core prefill path (indexer_tc.cu, same translation unit)
+namespace crs {
+static bool prefill_tc_applicable(const crs_indexer_params *p);
+static size_t prefill_tc_workspace(const crs_indexer_params *p);
+static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, const float *wgt,
+                             const void *k_idx, int32_t *out_idx, int32_t *out_count, void *ws,
+                             cudaStream_t s);
+}  // namespace crs
+
 static size_t dec_ws_parts(const crs_indexer_params *p, size_t &keys_bytes) {
     auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
     keys_bytes = al((size_t)p->n_rows * (size_t)max(p->max_keys, 1) * 4);
@@ -595,6 +620,7 @@ extern "C" size_t crs_indexer_topk_workspace_size(const crs_indexer_params *p) {
         size_t kbytes;
         return dec_ws_parts(p, kbytes);
     }
+    if (prefill_tc_applicable(p)) return prefill_tc_workspace(p);
     int max_slices, ws_rows;
     idx_geometry(p, max_slices, ws_rows);
     if (max_slices <= 1 || ws_rows == 0) return 0;
@@ -645,10 +671,14 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
         CRS_CHECK_LAUNCH();
         return CRS_OK;
     }
+    if (prefill_tc_applicable(p))
+        return launch_prefill_tc(p, q_idx, w, k_idx, out_idx, out_count, ws, s);
     int max_slices, ws_rows;
     idx_geometry(p, max_slices, ws_rows);
     if (max_slices > 64) return CRS_ERR_UNSUPPORTED;
     IdxArgs a;
+    a.row_list = nullptr;
+    a.list_count = nullptr;
     a.mode = p->mode;
     a.q = static_cast<const __nv_bfloat16 *>(q_idx);
     a.w = w;

@@ -5,5 +5,6 @@
 #include "lsh.cu"
 #include "sparse_attn.cu"
 #include "indexer.cu"
+#include "indexer_tc.cu"
 #include "blocks.cu"
 #include "noalloc.cu"

@@ -46,6 +46,79 @@ def test_prefill_small(crs, cuda_dev, n, topk):
                 rows, topk, "prefill")
 
 
+def test_prefill_tensor_core_path_traced(crs, cuda_dev):
+    """4 index heads of dim 64 run on the tcgen05 kernel (sample, threshold, filter, select)."""
+    n, topk = 5000, 512
+    case = workloads.indexer_prefill_case(n=n, topk=topk, seed=11, device=cuda_dev)
+    crs.profile_collect()
+    idx, cnt = crs.indexer_topk(case["q_idx"], case["w"], case["k_idx"], topk,
+                                crs.CRS_IDX_PREFILL)
+    torch.cuda.synchronize()
+    names = crs.profile_collect()
+    assert "idx_prefill_tc" in names
+    assert crs.get_device_error() == 0
+    g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    assert (g_cnt == np.minimum(topk, np.arange(n) + 1)).all()
+    rows = np.unique(np.concatenate([np.arange(0, n, 37), [topk - 1, topk, 1279, 1280, n - 1]]))
+    _check_rows(g_idx, g_cnt, _np(case["q_idx"]), _np(case["w"]), _np(case["k_idx"]),
+                np.zeros(n, np.int64), np.arange(1, n + 1, dtype=np.int32), rows, topk,
+                "prefill-tc")
+
+
+@pytest.mark.parametrize("n_idx_heads", [2, 8])
+def test_prefill_cuda_core_path(crs, cuda_dev, n_idx_heads):
+    """Index-head counts other than 4 take the CUDA-core slice path."""
+    n, topk = 2500, 256
+    case = workloads.indexer_prefill_case(n=n, topk=topk, n_idx_heads=n_idx_heads, seed=5,
+                                          device=cuda_dev)
+    crs.profile_collect()
+    idx, cnt = crs.indexer_topk(case["q_idx"], case["w"], case["k_idx"], topk,
+                                crs.CRS_IDX_PREFILL)
+    torch.cuda.synchronize()
+    assert "idx_prefill_tc" not in crs.profile_collect()
+    assert crs.get_device_error() == 0
+    g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    rows = np.unique(np.concatenate([np.arange(0, n, 41), [topk - 1, topk, n - 1]]))
+    _check_rows(g_idx, g_cnt, _np(case["q_idx"]), _np(case["w"]), _np(case["k_idx"]),
+                np.zeros(n, np.int64), np.arange(1, n + 1, dtype=np.int32), rows, topk,
+                "prefill-cc")
+
+
+def test_prefill_all_tied_rows_take_exact_fallback(crs, cuda_dev):
+    """Every key identical: each row's scores tie, the sampled threshold lets all
+    keys through, lists overflow and those rows are recomputed exactly; ties go to
+    the smallest positions."""
+    n, topk = 6000, 1024
+    g = torch.Generator(device=cuda_dev).manual_seed(3)
+    q = torch.randn(n, 4, 64, generator=g, device=cuda_dev).to(torch.bfloat16)
+    w = torch.randn(n, 4, generator=g, device=cuda_dev)
+    k = torch.randn(1, 64, generator=g, device=cuda_dev).to(torch.bfloat16).expand(n, 64).contiguous()
+    crs.profile_collect()
+    idx, cnt = crs.indexer_topk(q, w, k, topk, crs.CRS_IDX_PREFILL)
+    torch.cuda.synchronize()
+    names = crs.profile_collect()
+    assert "idx_prefill_tc" in names and "idx_slice_topk" in names
+    assert crs.get_device_error() == 0
+    g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    assert (g_cnt == np.minimum(topk, np.arange(n) + 1)).all()
+    for r in (0, 100, topk, 4095, 4096, 4097, n - 1):
+        m = min(topk, r + 1)
+        assert (g_idx[r, :m] == np.arange(m)).all(), f"row {r}"
+        assert (g_idx[r, m:] == -1).all()
+
+
+def test_prefill_nan_score_flags_device_error(crs, cuda_dev):
+    g = torch.Generator(device=cuda_dev).manual_seed(4)
+    q = torch.randn(600, 4, 64, generator=g, device=cuda_dev).to(torch.bfloat16)
+    w = torch.randn(600, 4, generator=g, device=cuda_dev)
+    k = torch.randn(600, 64, generator=g, device=cuda_dev).to(torch.bfloat16)
+    k[300, 5] = float("nan")
+    crs.get_device_error()
+    crs.indexer_topk(q, w, k, 64, crs.CRS_IDX_PREFILL)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() & crs.DEVERR_NONFINITE
+
+
 @pytest.mark.parametrize("lens,topk", [([100, 2048, 2049, 5000], 2048), ([40000, 17, 16384, 16385, 33000], 512)])
 def test_decode_small(crs, cuda_dev, lens, topk):
     g = torch.Generator(device=cuda_dev).manual_seed(len(lens))
