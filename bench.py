@@ -175,6 +175,9 @@ class PrefillWorkload(Workload):
         rows = sum(min(k, t + 1) for t in range(n))
         return {
             "idx_slice_topk": [("alu", pairs * 4 * 64 * 2 / 1e12, "TFLOP/s")],
+            # two launches per step (sampled threshold pass + filter pass): the
+            # step's causal score FLOPs split evenly over them
+            "idx_prefill_tc": [("tensor", pairs * 4 * 64 * 2 / 2 / 1e12, "TFLOP/s")],
             "sparse_attn": [("hbm", rows * 128 * 2 * 2 / 1e9, "GB/s"),
                             ("tensor", rows * 16 * 128 * 4 / 1e12, "TFLOP/s")],
         }

@@ -183,6 +183,7 @@ struct IdxArgs {
     int n_rows, H, topk, max_slices;
     const int32_t *row_list;      // optional: rows to process (blockIdx -> row_list[i])
     const int32_t *list_count;    //   and how many entries of row_list are live
+    int list_cap;                 //   capacity of row_list
 };
 
 __device__ __forceinline__ void row_range(const IdxArgs &a, int row, int64_t &kb, int &nv) {
@@ -201,22 +202,10 @@ __device__ __forceinline__ int ws_row(const IdxArgs &a, int row) {
     return a.mode == CRS_IDX_PREFILL ? row - kSlice : row;
 }
 
-__global__ void __launch_bounds__(kSelThreads) idx_slice_kernel(IdxArgs a) {
-    extern __shared__ __align__(16) unsigned char idx_smem[];
-    uint32_t *skey = reinterpret_cast<uint32_t *>(idx_smem);          // [kSlice]
-    float *sq = reinterpret_cast<float *>(skey + kSlice);             // [H][64]
-    float *sw = sq + kMaxIdxHeads * kIdxDim;                          // [H]
-    __shared__ SelScratch sc;
-
-    const int slice = blockIdx.x;
-    int row = blockIdx.y, wrow;
-    if (a.row_list) {
-        if ((int)blockIdx.y >= *a.list_count) return;
-        row = a.row_list[blockIdx.y];
-        wrow = blockIdx.y;
-    } else {
-        wrow = ws_row(a, row);
-    }
+// One (row, slice): wrow is the row's slot in the candidate workspace.
+__device__ __forceinline__ void idx_slice_row(const IdxArgs &a, const int slice, const int row,
+                                              const int wrow, uint32_t *skey, float *sq, float *sw,
+                                              SelScratch &sc) {
     int64_t kb;
     int nv;
     row_range(a, row, kb, nv);
@@ -302,17 +291,43 @@ __global__ void __launch_bounds__(kSelThreads) idx_slice_kernel(IdxArgs a) {
     }
 }
 
+// grid (slice, row); with a row list, grid.y CTAs stride over the list's live entries
+__global__ void __launch_bounds__(kSelThreads) idx_slice_kernel(IdxArgs a) {
+    extern __shared__ __align__(16) unsigned char idx_smem[];
+    uint32_t *skey = reinterpret_cast<uint32_t *>(idx_smem);          // [kSlice]
+    float *sq = reinterpret_cast<float *>(skey + kSlice);             // [H][64]
+    float *sw = sq + kMaxIdxHeads * kIdxDim;                          // [H]
+    __shared__ SelScratch sc;
+    if (a.row_list) {
+        const int live = min(*a.list_count, a.list_cap);
+        for (int i = blockIdx.y; i < live; i += gridDim.y) {
+            idx_slice_row(a, blockIdx.x, a.row_list[i], i, skey, sq, sw, sc);
+            __syncthreads();
+        }
+    } else {
+        idx_slice_row(a, blockIdx.x, blockIdx.y, ws_row(a, blockIdx.y), skey, sq, sw, sc);
+    }
+}
+
+__device__ __forceinline__ void idx_merge_row(const IdxArgs &a, const int row, const int wr,
+                                              SelScratch &sc, int *soff);
+
 __global__ void __launch_bounds__(kSelThreads) idx_merge_kernel(IdxArgs a, int row0) {
     __shared__ SelScratch sc;
     __shared__ int soff[65];
-    int row = row0 + blockIdx.x, wr;
     if (a.row_list) {
-        if ((int)blockIdx.x >= *a.list_count) return;
-        row = a.row_list[blockIdx.x];
-        wr = blockIdx.x;
+        const int live = min(*a.list_count, a.list_cap);
+        for (int i = blockIdx.x; i < live; i += gridDim.x) {
+            idx_merge_row(a, a.row_list[i], i, sc, soff);
+            __syncthreads();
+        }
     } else {
-        wr = ws_row(a, row);
+        idx_merge_row(a, row0 + blockIdx.x, ws_row(a, row0 + blockIdx.x), sc, soff);
     }
+}
+
+__device__ __forceinline__ void idx_merge_row(const IdxArgs &a, const int row, const int wr,
+                                              SelScratch &sc, int *soff) {
     int64_t kb;
     int nv;
     row_range(a, row, kb, nv);
@@ -679,6 +694,7 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
     IdxArgs a;
     a.row_list = nullptr;
     a.list_count = nullptr;
+    a.list_cap = 0;
     a.mode = p->mode;
     a.q = static_cast<const __nv_bfloat16 *>(q_idx);
     a.w = w;

@@ -9,20 +9,22 @@
 // last row).  Warp roles: warp 0 loads Q (once) and K tiles with TMA into a
 // ring of shared buffers; warp 1 issues tcgen05.mma for the 4 index heads
 // (M=128, N=64, K=64 each) into one of two TMEM accumulator sets
-// (4 heads x 64 columns); warps 4..11 read the accumulators (warp quadrant =
-// rows, two warps per quadrant split the 64 keys), form the weighted ReLU sum
-// and act on the scores.  Two modes:
+// (4 heads x 64 columns); warp 2 owns the TMEM allocation; warps 4..19 read
+// the accumulators (warp % 4 = TMEM lane quadrant = 32 query rows, four warps
+// per quadrant take 16 keys each), release them at once, and form the
+// weighted ReLU sum with paired fp32 FMAs.  Two modes:
 //   SAMPLE: every 8th key tile; scores (top 16 bits of the order-preserving
 //           key) are written out per row;
 //   FILTER: every key tile; a score whose key is >= the row's threshold is
-//           appended to that (row, key half)'s candidate list.
+//           appended to that (row, part)'s candidate list, in position order.
 // idx_tc_tau_kernel picks each row's threshold from its samples so that about
-// 1.25 k scores pass; idx_tc_final_kernel merges a row's two candidate lists by
-// position and selects the exact top-k (ties to the smaller position); a row
-// whose candidates number fewer than k or overflowed a list is recomputed by
-// the exact CUDA-core slice path.  The threshold only decides how much work
+// 1.25 k scores pass; idx_tc_final_kernel merges a row's four candidate lists
+// by position and selects the exact top-k (ties to the smaller position); a
+// row whose candidates number fewer than k or overflowed a list is recomputed
+// by the exact CUDA-core slice path.  The threshold only decides how much work
 // the final selection sees, never the result.
 #include <cuda.h>
+#include <float.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -30,15 +32,45 @@
 
 namespace crs {
 
+// packed fp32 pairs (sm_100 f32x2 arithmetic) and a NaN-propagating ReLU
+__device__ __forceinline__ uint64_t f32x2_pack(float x, float y) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+    return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float &x, float &y) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ float relu_nan(float x) {
+    float r;
+    asm("max.NaN.f32 %0, %1, 0f00000000;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float fmax_nan(float x, float y) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(x), "f"(y));
+    return r;
+}
+
 constexpr int kIqM = 128;           // query rows per CTA
 constexpr int kIkN = 64;            // keys per tile
 constexpr int kIH = 4;              // index heads on this path
 constexpr int kID = 64;             // index head dim
-constexpr int kIStages = 8;         // K-tile ring
+constexpr int kIStages = 3;         // K-tile ring
 constexpr int kISampStride = 8;     // SAMPLE mode: every 8th key tile
-constexpr int kICapHalf = 2048;     // candidates per (row, key half)
+constexpr int kIParts = 4;          // a key tile is split in 4 parts of 16 keys (one epilogue warp each)
+constexpr int kIPartKeys = kIkN / kIParts;
+constexpr int kICap = 2048;         // candidates per (row, part) list
 constexpr int kIFallbackRows = 4096;
-constexpr int kIThreads = 384;      // 12 warps
+constexpr int kIRing = 24;          // FILTER: staged candidates per row (<= 7 pending + 16 new)
+constexpr int kIFlush = 8;          //   written out 8 at a time (one 32-byte run per array)
+constexpr int kIEpiWarps = 4 * kIParts;             // 4 TMEM lane quadrants x 4 parts
+constexpr int kIThreads = 32 * (4 + kIEpiWarps);    // TMA, MMA, TMEM-alloc, spare + epilogue
 constexpr uint64_t kIWaitNs = 2000000000ull;
 constexpr float kIBeta = 1.25f;
 
@@ -47,6 +79,8 @@ struct IdxTcSmem {
     unsigned char k[kIStages][kIkN * 128];   // key tiles: 64 keys x 64 dims, SW128
     float w[kIqM][kIH];
     uint32_t tau[kIqM];
+    uint64_t ring[kIEpiWarps][kIRing][32];   // FILTER: (score bits << 32 | position) per lane (row)
+    float stage[kIEpiWarps][kIPartKeys][32]; // FILTER: a tile's 16 scores per lane
     uint64_t qfull;
     uint64_t kfull[kIStages];
     uint64_t kempty[kIStages];
@@ -60,11 +94,41 @@ struct IdxTcArgs {
     const float *w;           // [n, 4]
     const uint32_t *tau;      // [n] FILTER thresholds (order-preserving keys)
     uint16_t *samples;        // [n, samp_slots] SAMPLE output (0 = no sample)
-    uint32_t *cand_key;       // [n, 2, kICapHalf]
-    int32_t *cand_idx;        // [n, 2, kICapHalf]
-    int32_t *cand_cnt;        // [n, 2]
+    uint32_t *cand_key;       // [n, kIParts, kICap]
+    int32_t *cand_idx;        // [n, kIParts, kICap]
+    int32_t *cand_cnt;        // [n, kIParts]
     int n, samp_slots, n_tiles_rows;
 };
+
+// One flush round of a FILTER epilogue warp: up to 4 rows (the lowest set bits
+// of `rows`, lanes = rows of the warp's quadrant); lanes [8g, 8g + 8) write the
+// next (at most 8) staged entries of the g-th row to its candidate list, as one
+// 32-byte run per array.  Entries past the list capacity are dropped (the count
+// still records them, so the row falls back).  Returns the rows served.
+__device__ __forceinline__ unsigned flush_round(const IdxTcArgs &a, const uint64_t *ring,
+                                                unsigned rows, int flushed, int cnt, int t_base,
+                                                int part) {
+    const int lane = threadIdx.x & 31, g = lane >> 3;
+    int src[4];
+    unsigned m = rows;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        src[u] = m ? __ffs(m) - 1 : -1;
+        m &= m - 1u;
+    }
+    const int mine = g == 0 ? src[0] : g == 1 ? src[1] : g == 2 ? src[2] : src[3];
+    const int sl = mine < 0 ? 0 : mine;
+    const int f = __shfl_sync(0xffffffffu, flushed, sl);
+    const int c = __shfl_sync(0xffffffffu, cnt, sl);
+    const int e = f + (lane & 7);
+    if (mine >= 0 && e < c && e < kICap) {
+        const uint64_t v = ring[(e % kIRing) * 32 + mine];
+        const size_t base = ((size_t)(t_base + mine) * kIParts + part) * kICap;
+        a.cand_key[base + e] = score_key(__uint_as_float((uint32_t)(v >> 32)));
+        a.cand_idx[base + e] = (int32_t)(uint32_t)v;
+    }
+    return rows & ~m;
+}
 
 template <int MODE>   // 0 = SAMPLE, 1 = FILTER
 __global__ void __launch_bounds__(kIThreads, 1)
@@ -89,7 +153,7 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&S.tfull[i], 1);
-            tc::mbar_init(&S.tempty[i], 8);       // one arrival per epilogue warp
+            tc::mbar_init(&S.tempty[i], kIEpiWarps);   // one arrival per epilogue warp
         }
         tc::mbar_fence_init();
         S.fail = 0;
@@ -153,19 +217,22 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             if (!ok) atomicOr(&S.fail, 1);
         }
     } else if (warp >= 4) {
-        // ---------------- epilogue: row = quadrant * 32 + lane, key half hf
-        const int quad = warp & 3, hf = (warp - 4) >> 2;
+        // ---------------- epilogue: row = quadrant * 32 + lane, keys [16 part, 16 part + 16)
+        const int ew = warp - 4, quad = warp & 3, part = ew >> 2;
         const int row = quad * 32 + lane;
         const int t = r0 + row;
         const bool row_ok = t < a.n;
-        float wr[kIH];
+        uint64_t w2[kIH];                        // (w_h, w_h) for the paired FMA
 #pragma unroll
-        for (int h = 0; h < kIH; ++h) wr[h] = S.w[row][h];
+        for (int h = 0; h < kIH; ++h) w2[h] = f32x2_pack(S.w[row][h], S.w[row][h]);
         const uint32_t tau = MODE == 1 ? S.tau[row] : 0u;
-        int cnt = 0;
-        const size_t cbase = ((size_t)(row_ok ? t : 0) * 2 + hf) * kICapHalf;
-        const uint32_t tq_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        bool nonfinite = false;
+        // key >= tau  <=>  score >= key_score(tau) for every non-NaN score
+        const float tauf = tau == 0u ? -INFINITY : key_score(tau);
+        int cnt = 0, flushed = 0, slot = 0;          // FILTER: appended, written out, ring slot
+        uint64_t *ring = &S.ring[ew][0][0];
+        const uint32_t tq_lane = tmem + ((uint32_t)(quad * 32) << 16) + part * kIPartKeys;
+        uint64_t nanacc = 0ull;                  // score pairs x 0: stays 0 unless a score is NaN/inf
+        float *stage = &S.stage[ew][0][0];
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1, v = j >> 1;
             const bool ok = tc::mbar_wait_bounded(&S.tfull[b], v & 1, kIWaitNs, K_IDX_PREFILL_TC, 5);
@@ -174,61 +241,91 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
                 break;
             }
             tc::fence_after();
-            float sc[32];
+            uint32_t d[kIH][kIPartKeys];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sc[i] = 0.0f;
-#pragma unroll
-            for (int h = 0; h < kIH; ++h) {
-                uint32_t d[32];
-                tc::tmem_ld32(tq_lane + b * 256 + h * 64 + hf * 32, d);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float x = __uint_as_float(d[i]);
-                    nonfinite |= !isfinite(x);
-                    sc[i] = fmaf(wr[h], fmaxf(x, 0.0f), sc[i]);
-                }
-            }
+            for (int h = 0; h < kIH; ++h) tc::tmem_ld16(tq_lane + b * 256 + h * 64, d[h]);
+            tc::tmem_ld_wait();
             tc::fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&S.tempty[b]);
+            if (lane == 0) tc::mbar_arrive(&S.tempty[b]);     // accumulators free for tile j + 2
+            // score = sum_h w_h ReLU(q_h . k); a NaN dot survives the ReLU (max.NaN)
+            uint64_t acc[kIPartKeys / 2];
+#pragma unroll
+            for (int i = 0; i < kIPartKeys / 2; ++i) acc[i] = 0ull;
+#pragma unroll
+            for (int h = 0; h < kIH; ++h)
+#pragma unroll
+                for (int i = 0; i < kIPartKeys / 2; ++i)
+                    acc[i] = f32x2_fma(w2[h],
+                                       f32x2_pack(relu_nan(__uint_as_float(d[h][2 * i])),
+                                                  relu_nan(__uint_as_float(d[h][2 * i + 1]))),
+                                       acc[i]);
+            float sc[kIPartKeys];
+#pragma unroll
+            for (int i = 0; i < kIPartKeys / 2; ++i) {
+                nanacc = f32x2_fma(acc[i], 0ull, nanacc);
+                f32x2_unpack(acc[i], sc[2 * i], sc[2 * i + 1]);
+            }
             const int kt = MODE == 0 ? j * kISampStride : j;
-            const int key0 = kt * kIkN + hf * 32;
+            const int key0 = kt * kIkN + part * kIPartKeys;
+            // keys > t (causal) exist only in the CTA's last two tiles
+            const int lim = t - key0 + 1;            // keys [key0, key0 + lim) are visible
+            const uint32_t vis = lim >= kIPartKeys ? 0xffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
             if constexpr (MODE == 0) {
                 if (row_ok) {
-                    uint32_t pk[16];
+                    uint32_t pk[kIPartKeys / 2];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        uint32_t lo = 0u, hi = 0u;
-                        const int ka = key0 + 2 * i, kb2 = ka + 1;
-                        if (ka <= t) lo = score_key(sc[2 * i]) >> 16;
-                        if (kb2 <= t) hi = score_key(sc[2 * i + 1]) >> 16;
+                    for (int i = 0; i < kIPartKeys / 2; ++i) {
+                        const uint32_t lo = ((vis >> (2 * i)) & 1u) ? score_key(sc[2 * i]) >> 16 : 0u;
+                        const uint32_t hi = ((vis >> (2 * i + 1)) & 1u) ? score_key(sc[2 * i + 1]) >> 16 : 0u;
                         pk[i] = lo | (hi << 16);
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(a.samples + (size_t)t * a.samp_slots +
-                                                           j * kIkN + hf * 32);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                                                           j * kIkN + part * kIPartKeys);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             } else {
-                if (row_ok) {
+                uint32_t pm = 0u;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int key = key0 + i;
-                        const uint32_t kk = score_key(sc[i]);
-                        if (key <= t && kk >= tau) {
-                            if (cnt < kICapHalf) {
-                                a.cand_key[cbase + cnt] = kk;
-                                a.cand_idx[cbase + cnt] = key;
-                            }
-                            ++cnt;
-                        }
+                for (int i = 0; i < kIPartKeys; ++i) pm |= (sc[i] >= tauf ? 1u : 0u) << i;
+                pm &= row_ok ? vis : 0u;
+                if (__any_sync(0xffffffffu, pm != 0u)) {
+                    // the scores go through shared memory so that the set bits can
+                    // be visited with a dynamic index; each lane stages its row's
+                    // passing (score, position) pairs in its ring
+#pragma unroll
+                    for (int i = 0; i < kIPartKeys; ++i) stage[i * 32 + lane] = sc[i];
+                    while (pm) {
+                        const int i = __ffs(pm) - 1;
+                        pm &= pm - 1u;
+                        ring[slot * 32 + lane] =
+                            ((uint64_t)__float_as_uint(stage[i * 32 + lane]) << 32) | (uint32_t)(key0 + i);
+                        slot = slot + 1 == kIRing ? 0 : slot + 1;
+                        ++cnt;
+                    }
+                    __syncwarp();
+                    // until every row has < 8 staged entries: 8 entries of up to 4
+                    // rows per round, one 32-byte run per row and array
+                    unsigned full;
+                    while ((full = __ballot_sync(0xffffffffu, cnt - flushed >= kIFlush)) != 0u) {
+                        const unsigned done = flush_round(a, ring, full, flushed, cnt, r0 + quad * 32, part);
+                        if ((done >> lane) & 1u) flushed += kIFlush;
                     }
                 }
             }
         }
-        if (MODE == 1 && row_ok) a.cand_cnt[(size_t)t * 2 + hf] = cnt;
-        if (nonfinite) raise_error(CRS_DEVERR_NONFINITE);
+        if (MODE == 1) {
+            unsigned left;
+            while ((left = __ballot_sync(0xffffffffu, cnt > flushed)) != 0u) {
+                const unsigned done = flush_round(a, ring, left, flushed, cnt, r0 + quad * 32, part);
+                if ((done >> lane) & 1u) flushed = min(cnt, flushed + kIFlush);
+            }
+        }
+        if (MODE == 1 && row_ok) a.cand_cnt[(size_t)t * kIParts + part] = cnt;
+        float n0, n1;
+        f32x2_unpack(nanacc, n0, n1);
+        if (row_ok && (n0 != 0.0f || n1 != 0.0f)) raise_error(CRS_DEVERR_NONFINITE);
     }
     tc::fence_before();
     __syncthreads();
@@ -318,66 +415,152 @@ __global__ void __launch_bounds__(256) idx_tc_tau_kernel(const uint16_t *__restr
 }
 
 // ---------------------------------------------------------------------------
-// Per row: merge the two candidate lists by position, exact top-k, ascending
-// output.  Rows whose lists overflowed, or hold fewer than k candidates, are
-// queued for the exact slice path.
+// Per row (one warp): exact top-k over the row's candidates, ascending output.
+//   1. 4 radix passes of 8 bits over the candidate keys (warp histogram)
+//      give the k-th largest key T and how many keys equal to T are taken;
+//   2. positions with key > T are set in a bitmap over [0, t], positions with
+//      key == T in a second one;
+//   3. one ordered sweep over the bitmap words emits the positions ascending,
+//      taking the tied positions smallest first.
+// Rows whose lists overflowed, or hold fewer than k candidates, are queued
+// for the exact slice path.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kSelThreads)
+constexpr int kFinWarps = 8;
+
+__host__ __device__ __forceinline__ size_t fin_warp_words(int n) { return 256 + 2 * (size_t)((n + 31) / 32); }
+
+// Finds, from the top bin down, the bin holding the need-th largest count; need
+// is then replaced by its rank inside that bin.  Warp-collective.
+__device__ __forceinline__ int warp_top_bin(const uint32_t *hist, int &need) {
+    const int lane = threadIdx.x & 31;
+    int c[8], s = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) { c[u] = (int)hist[255 - (lane * 8 + u)]; s += c[u]; }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    const int before = incl - s;
+    int fb = -1, fr = 0;
+    if (before < need && need <= incl) {
+        int acc = before;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (fb < 0 && acc < need && need <= acc + c[u]) { fb = 255 - (lane * 8 + u); fr = need - acc; }
+            acc += c[u];
+        }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, fb >= 0);
+    const int src = m ? __ffs(m) - 1 : 0;
+    need = __shfl_sync(0xffffffffu, fr, src);
+    return __shfl_sync(0xffffffffu, fb, src);
+}
+
+__global__ void __launch_bounds__(kFinWarps * 32)
 idx_tc_final_kernel(const uint32_t *__restrict__ cand_key, const int32_t *__restrict__ cand_idx,
                     const int32_t *__restrict__ cand_cnt, int32_t *__restrict__ out_idx,
                     int32_t *__restrict__ out_cnt, int32_t *__restrict__ fb_list,
                     int32_t *__restrict__ fb_count, int n, int topk) {
-    __shared__ SelScratch sc;
-    __shared__ int32_t aidx[kICapHalf], bidx[kICapHalf];
-    extern __shared__ uint32_t mrg[];            // [2 * kICapHalf] keys, then [2 * kICapHalf] positions
-    const int t = blockIdx.x;
+    extern __shared__ uint32_t fin_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t >= n) return;                                   // warp-uniform; no block barriers below
+    uint32_t *hist = fin_smem + (size_t)warp * fin_warp_words(n);
+    const int nwords = (t + 1 + 31) >> 5;                 // bitmap words over positions [0, t]
+    uint32_t *bm_gt = hist + 256;
+    uint32_t *bm_eq = bm_gt + (n + 31) / 32;
     int32_t *o = out_idx + (size_t)t * topk;
     if (t + 1 <= topk) {
-        for (int i = threadIdx.x; i < topk; i += kSelThreads) o[i] = (i <= t) ? i : -1;
-        if (threadIdx.x == 0) out_cnt[t] = t + 1;
+        for (int i = lane; i < topk; i += 32) o[i] = (i <= t) ? i : -1;
+        if (lane == 0) out_cnt[t] = t + 1;
         return;
     }
-    const int c0 = cand_cnt[(size_t)t * 2], c1 = cand_cnt[(size_t)t * 2 + 1];
-    if (c0 > kICapHalf || c1 > kICapHalf || c0 + c1 < topk) {
-        if (threadIdx.x == 0) {
+    int c[kIParts], N = 0;
+    bool over = false;
+#pragma unroll
+    for (int q = 0; q < kIParts; ++q) {
+        c[q] = cand_cnt[(size_t)t * kIParts + q];
+        over |= c[q] > kICap;
+        N += c[q];
+    }
+    if (over || N < topk) {
+        if (lane == 0) {
             const int pos = atomicAdd(fb_count, 1);
             if (pos < kIFallbackRows) fb_list[pos] = t;
             else raise_error(CRS_DEVERR_INDEX);
         }
         return;
     }
-    const size_t ba = (size_t)t * 2 * kICapHalf, bb = ba + kICapHalf;
-    for (int i = threadIdx.x; i < c0; i += kSelThreads) aidx[i] = cand_idx[ba + i];
-    for (int i = threadIdx.x; i < c1; i += kSelThreads) bidx[i] = cand_idx[bb + i];
-    __syncthreads();
-    uint32_t *mk = mrg;
-    int32_t *mi = reinterpret_cast<int32_t *>(mrg + 2 * kICapHalf);
-    auto lower = [](const int32_t *arr, int len, int x) {
-        int lo = 0, hi = len;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (arr[mid] < x) lo = mid + 1; else hi = mid;
+    const uint32_t *ck = cand_key + (size_t)t * kIParts * kICap;
+    const int32_t *ci = cand_idx + (size_t)t * kIParts * kICap;
+    // 1. radix select
+    uint32_t prefix = 0u, mask = 0u;
+    int need = topk;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0u;
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < kIParts; ++q)
+            for (int i = lane; i < c[q]; i += 32) {
+                const uint32_t kk = ck[q * kICap + i];
+                if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1u);
+            }
+        __syncwarp();
+        const int bin = warp_top_bin(hist, need);
+        prefix |= (uint32_t)bin << shift;
+        mask |= 0xffu << shift;
+        __syncwarp();
+    }
+    const uint32_t T = prefix;                            // the k-th largest key; take `need` ties
+    // 2. bitmaps
+    for (int w = lane; w < nwords; w += 32) { bm_gt[w] = 0u; bm_eq[w] = 0u; }
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < kIParts; ++q)
+        for (int i = lane; i < c[q]; i += 32) {
+            const uint32_t kk = ck[q * kICap + i];
+            if (kk >= T) {
+                const int pos = ci[q * kICap + i];
+                atomicOr(kk > T ? &bm_gt[pos >> 5] : &bm_eq[pos >> 5], 1u << (pos & 31));
+            }
         }
-        return lo;
-    };
-    for (int i = threadIdx.x; i < c0; i += kSelThreads) {
-        const int p = i + lower(bidx, c1, aidx[i]);
-        mk[p] = cand_key[ba + i];
-        mi[p] = aidx[i];
+    __syncwarp();
+    // 3. ordered sweep: word w = round * 32 + lane
+    int eq_base = 0, out_base = 0;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t g = 0u, e = 0u;
+        if (w < nwords) { g = bm_gt[w]; e = bm_eq[w]; }
+        const int pe = __popc(e);
+        int incl = pe;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += x;
+        }
+        const int allow = need - (eq_base + incl - pe);   // ties this word may still take
+        if (allow <= 0) e = 0u;
+        else
+            for (int r = pe - allow; r > 0; --r) e &= ~(0x80000000u >> __clz(e));   // keep the lowest `allow`
+        const uint32_t sel = g | e;
+        const int ps = __popc(sel);
+        int oin = ps;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, oin, off);
+            if (lane >= off) oin += x;
+        }
+        int dst = out_base + oin - ps;
+        for (uint32_t m = sel; m; m &= m - 1u) o[dst++] = w * 32 + (__ffs(m) - 1);
+        eq_base += __shfl_sync(0xffffffffu, incl, 31);
+        out_base += __shfl_sync(0xffffffffu, oin, 31);
     }
-    for (int i = threadIdx.x; i < c1; i += kSelThreads) {
-        const int p = i + lower(aidx, c0, bidx[i]);
-        mk[p] = cand_key[bb + i];
-        mi[p] = bidx[i];
-    }
-    __syncthreads();
-    const int N = c0 + c1;
-    int need_eq = 0;
-    const uint32_t T = block_radix_select([&](int i) { return mk[i]; }, N, topk, sc, need_eq);
-    const int cnt = block_compact([&](int i) { return mk[i]; }, N, T, need_eq, false, sc,
-                                  [&](int pos, int i, uint32_t) { o[pos] = mi[i]; });
-    for (int i = cnt + threadIdx.x; i < topk; i += kSelThreads) o[i] = -1;
-    if (threadIdx.x == 0) out_cnt[t] = cnt;
+    for (int i = out_base + lane; i < topk; i += 32) o[i] = -1;
+    if (lane == 0) out_cnt[t] = out_base;
 }
 
 // ----------------------------------------------------------------- host --
@@ -418,9 +601,9 @@ static void prefill_tc_layout(int n, int topk, PrefillTcWs &w, char *base) {
     auto take = [&](size_t bytes) { char *p = base ? base + off : nullptr; off += al(bytes); return p; };
     w.samples = reinterpret_cast<uint16_t *>(take((size_t)n * w.samp_slots * 2));
     w.tau = reinterpret_cast<uint32_t *>(take((size_t)n * 4));
-    w.cand_key = reinterpret_cast<uint32_t *>(take((size_t)n * 2 * kICapHalf * 4));
-    w.cand_idx = reinterpret_cast<int32_t *>(take((size_t)n * 2 * kICapHalf * 4));
-    w.cand_cnt = reinterpret_cast<int32_t *>(take((size_t)n * 2 * 4));
+    w.cand_key = reinterpret_cast<uint32_t *>(take((size_t)n * kIParts * kICap * 4));
+    w.cand_idx = reinterpret_cast<int32_t *>(take((size_t)n * kIParts * kICap * 4));
+    w.cand_cnt = reinterpret_cast<int32_t *>(take((size_t)n * kIParts * 4));
     w.fb_list = reinterpret_cast<int32_t *>(take((size_t)fbr * 4));
     w.fb_count = reinterpret_cast<int32_t *>(take(4));
     w.fb_ckey = reinterpret_cast<uint32_t *>(take((size_t)fbr * w.fb_slices * topk * 4));
@@ -431,7 +614,7 @@ static void prefill_tc_layout(int n, int topk, PrefillTcWs &w, char *base) {
 
 static bool prefill_tc_applicable(const crs_indexer_params *p) {
     return p->mode == CRS_IDX_PREFILL && p->n_idx_heads == kIH && p->d_idx == kID &&
-           p->topk <= kICapHalf && p->n_rows >= 1 && p->n_rows <= 64 * kSlice;
+           p->topk <= 2048 && p->n_rows >= 1 && p->n_rows <= (1 << 19);
 }
 
 static size_t prefill_tc_workspace(const crs_indexer_params *p) {
@@ -500,12 +683,15 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
         idx_prefill_tc_kernel<1><<<a.n_tiles_rows, kIThreads, smem, s>>>(tq, tk, a);
     }
     CRS_CHECK_LAUNCH();
-    const int dsm = 4 * kICapHalf * 4;
+    const size_t per_warp = fin_warp_words(n) * 4;
+    const int fin_warps = (int)min((size_t)kFinWarps, ((size_t)200 << 10) / per_warp);
+    if (fin_warps < 1) return CRS_ERR_UNSUPPORTED;
+    const int dsm = (int)(per_warp * fin_warps);
     CRS_TRY_CUDA(cudaFuncSetAttribute(idx_tc_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm));
     {
         ProfScope _ps(K_IDX_SELECT, s);
-        idx_tc_final_kernel<<<n, kSelThreads, dsm, s>>>(w.cand_key, w.cand_idx, w.cand_cnt, out_idx,
-                                                          out_count, w.fb_list, w.fb_count, n, topk);
+        idx_tc_final_kernel<<<ceil_div(n, fin_warps), fin_warps * 32, dsm, s>>>(
+            w.cand_key, w.cand_idx, w.cand_cnt, out_idx, out_count, w.fb_list, w.fb_count, n, topk);
     }
     CRS_CHECK_LAUNCH();
     // exact slice path for the queued rows (usually none)
@@ -527,16 +713,18 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
     f.row_list = w.fb_list;
     f.list_count = w.fb_count;
     const int fbr = min(n, kIFallbackRows);
+    f.list_cap = fbr;
+    const int fb_grid = min(fbr, 2 * 148);      // CTAs stride over the live list entries
     const size_t ssm = (size_t)kSlice * 4 + (kMaxIdxHeads * kIdxDim + kMaxIdxHeads) * 4;
     CRS_TRY_CUDA(cudaFuncSetAttribute(idx_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm));
     {
         ProfScope _ps(K_IDX_SLICE, s);
-        idx_slice_kernel<<<dim3(w.fb_slices, fbr), kSelThreads, ssm, s>>>(f);
+        idx_slice_kernel<<<dim3(w.fb_slices, fb_grid), kSelThreads, ssm, s>>>(f);
     }
     CRS_CHECK_LAUNCH();
     if (w.fb_slices > 1) {
         ProfScope _ps(K_IDX_MERGE, s);
-        idx_merge_kernel<<<fbr, kSelThreads, 0, s>>>(f, 0);
+        idx_merge_kernel<<<fb_grid, kSelThreads, 0, s>>>(f, 0);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;

@@ -8,7 +8,8 @@
 // One CTA = one (row, KV head, split of the list).  The G <= 16 query heads
 // of the KV head form the M = 16 side of mma.sync.m16n8k16 (bf16 in, fp32
 // accumulate).  Keys are gathered 64 per stage with 16-byte cp.async into
-// XOR-swizzled shared rows (double-buffered); each of the 4 warps owns 16
+// XOR-swizzled shared rows (a ring of 3 tiles, two in flight while one is
+// consumed; one barrier per tile); each of the 4 warps owns 16
 // keys of a stage and keeps its own online-softmax state; the warps merge at
 // the end.  The path is bound by the gather bandwidth.
 #include <math.h>
@@ -23,6 +24,7 @@ constexpr int kSaWarps = 4;
 constexpr int kSaThreads = kSaWarps * 32;
 constexpr int kSaRowBytes = kSaD * 2;                 // 256 B per K or V row
 constexpr int kSaTileBytes = kSaKeys * kSaRowBytes;   // 16 KB
+constexpr int kSaStages = 3;                          // K/V tiles in the ring
 constexpr float kLog2e = 1.4426950408889634f;
 
 // swizzled byte offset of 16-byte chunk c (0..15) of row r inside a tile
@@ -75,11 +77,11 @@ struct SaArgs {
 
 __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
     extern __shared__ __align__(128) unsigned char sa_smem[];
-    unsigned char *sK = sa_smem;                          // [2][kSaTileBytes]
-    unsigned char *sV = sK + 2 * kSaTileBytes;            // [2][kSaTileBytes]
-    unsigned char *sQ = sV + 2 * kSaTileBytes;            // [16 rows][256 B] swizzled
-    int *sIdx = reinterpret_cast<int *>(sQ + 16 * kSaRowBytes);   // [2][kSaKeys]
-    float *sRed = reinterpret_cast<float *>(sIdx + 2 * kSaKeys);   // merge scratch
+    unsigned char *sK = sa_smem;                                  // [kSaStages][kSaTileBytes]
+    unsigned char *sV = sK + kSaStages * kSaTileBytes;            // [kSaStages][kSaTileBytes]
+    unsigned char *sQ = sV + kSaStages * kSaTileBytes;            // [16 rows][256 B] swizzled
+    float *sRed = reinterpret_cast<float *>(sQ + 16 * kSaRowBytes);   // [4][16] m, [4][16] l
+    int *sIdx = reinterpret_cast<int *>(sRed + kSaWarps * 16 * 2);      // the split's list, -1 padded
 
     const int split = blockIdx.x;
     const int item = blockIdx.y;                 // row * n_kv + h
@@ -104,35 +106,41 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
         *reinterpret_cast<uint4 *>(sQ + sw_off(r, c)) = v;
     }
 
-    auto load_tile = [&](int t, int buf) {
-        const int base = s0 + t * kSaKeys;
-        int *si = sIdx + buf * kSaKeys;
-        if (tid < kSaKeys) {
-            const int s = base + tid;
-            int j = (s < s1) ? idx[s] : -1;
-            if (j >= 0 && a.n_keys > 0 && j >= a.n_keys) {
-                raise_error(CRS_DEVERR_INDEX);
-                j = -1;
-            }
-            si[tid] = j;
+    // the split's index list, once, into shared memory (padded with -1 to whole tiles)
+    for (int i = tid; i < n_tiles * kSaKeys; i += kSaThreads) {
+        int j = (s0 + i < s1) ? __ldg(idx + s0 + i) : -1;
+        if (j >= 0 && a.n_keys > 0 && j >= a.n_keys) {
+            raise_error(CRS_DEVERR_INDEX);
+            j = -1;
         }
-        __syncthreads();
-        unsigned char *k_dst = sK + buf * kSaTileBytes;
-        unsigned char *v_dst = sV + buf * kSaTileBytes;
+        sIdx[i] = j;
+    }
+    __syncthreads();
+
+    // Issue the gathers of tile t into ring slot t % kSaStages (one commit group per
+    // call, empty past the last tile).
+    auto load_tile = [&](int t) {
+        if (t < n_tiles) {
+            const int buf = t % kSaStages;
+            const int *si = sIdx + t * kSaKeys;
+            unsigned char *k_dst = sK + buf * kSaTileBytes;
+            unsigned char *v_dst = sV + buf * kSaTileBytes;
 #pragma unroll
-        for (int u = 0; u < (kSaKeys * 16) / kSaThreads; ++u) {
-            const int e = tid + u * kSaThreads;
-            const int r = e >> 4, c = e & 15;
-            const int j = si[r];
-            const bool ok = j >= 0;
-            const size_t off = ok ? ((size_t)(kbase + j) * tok_stride + c * 8) : 0;
-            cp_async16_zfill(k_dst + sw_off(r, c), Kh + off, ok);
-            cp_async16_zfill(v_dst + sw_off(r, c), Vh + off, ok);
+            for (int u = 0; u < (kSaKeys * 16) / kSaThreads; ++u) {
+                const int e = tid + u * kSaThreads;
+                const int r = e >> 4, c = e & 15;
+                const int j = si[r];
+                const bool ok = j >= 0;
+                const size_t off = ok ? ((size_t)(kbase + j) * tok_stride + c * 8) : 0;
+                cp_async16_zfill(k_dst + sw_off(r, c), Kh + off, ok);
+                cp_async16_zfill(v_dst + sw_off(r, c), Vh + off, ok);
+            }
         }
         cp_async_commit();
     };
 
-    if (n_tiles > 0) load_tile(0, 0);
+#pragma unroll
+    for (int t = 0; t < kSaStages - 1; ++t) load_tile(t);
     __syncthreads();
 
     // ---- Q fragments (A operand, 16 x 128): 8 k-steps x 4 regs
@@ -154,15 +162,11 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
     const int g_row = lane >> 2, tig = lane & 3;
 
     for (int t = 0; t < n_tiles; ++t) {
-        const int buf = t & 1;
-        if (t + 1 < n_tiles) {
-            load_tile(t + 1, buf ^ 1);   // contains a __syncthreads before issuing
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const int *si = sIdx + buf * kSaKeys;
+        const int buf = t % kSaStages;
+        cp_async_wait<kSaStages - 2>();          // tile t has landed (this thread's copies)
+        __syncthreads();                         // ... everyone's; tile t-1 is no longer read
+        load_tile(t + kSaStages - 1);            // into the slot tile t-1 used
+        const int *si = sIdx + t * kSaKeys;
         const int kw = warp * 16;        // this warp's 16 keys
         const bool any = (si[kw + (lane & 15)] >= 0);
         if (__any_sync(0xffffffffu, any)) {
@@ -244,8 +248,9 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
                 mma_bf16(o[2 * jj + 1], pl, b2, b3);
             }
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();                             // the ring is free: it holds the merge scratch
 
     // ---- merge the 4 warps: row sums across the quad, then across warps in smem
     l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
@@ -254,7 +259,7 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
     l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
     float *sM = sRed;                        // [4 warps][16]
     float *sL = sM + kSaWarps * 16;          // [4][16]
-    float *sO = sL + kSaWarps * 16;          // [4][16][128]  (reuses nothing else)
+    float *sO = reinterpret_cast<float *>(sK);   // [4][16][128], over the K/V ring
     if (tig == 0) {
         sM[warp * 16 + g_row] = m_lo;
         sM[warp * 16 + g_row + 8] = m_hi;
@@ -330,10 +335,13 @@ __global__ void sparse_attn_merge_kernel(const float *__restrict__ part_o,
     if (lse && lane == 0) lse[gw] = (L > 0.0f) ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
-static size_t sa_smem_bytes() {
-    const size_t main = 4 * (size_t)kSaTileBytes + 16 * kSaRowBytes + 2 * kSaKeys * 4;
-    const size_t red = (size_t)kSaWarps * 16 * 2 * 4 + (size_t)kSaWarps * 16 * kSaD * 4;
-    return main + red;
+constexpr int kSaMaxSplit = 4096;     // keys per split: the split's list sits in shared memory
+
+static size_t sa_smem_bytes(int split_len) {
+    static_assert((size_t)kSaWarps * 16 * kSaD * 4 <= 2 * kSaStages * (size_t)kSaTileBytes,
+                  "merge scratch must fit in the K/V ring");
+    return 2 * kSaStages * (size_t)kSaTileBytes + 16 * kSaRowBytes + (size_t)kSaWarps * 16 * 2 * 4 +
+           (size_t)split_len * 4;
 }
 
 static int sa_splits(const crs_attn_params *p) {
@@ -341,7 +349,8 @@ static int sa_splits(const crs_attn_params *p) {
     const int max_split = max(1, ceil_div(p->max_idx, 256));   // >= 256 keys per split
     const long long target = 148LL * 8;
     int s = (int)((target + items - 1) / items);
-    return max(1, min(s, max_split));
+    s = max(1, min(s, max_split));
+    return max(s, ceil_div(p->max_idx, kSaMaxSplit));
 }
 
 static int sa_validate(const crs_attn_params *p) {
@@ -392,7 +401,7 @@ extern "C" int crs_sparse_attn(const crs_attn_params *p, const void *Q, const vo
     a.n_lists = p->n_lists;
     a.n_keys = p->n_keys;
     a.splits = sa_splits(p);
-    a.split_len = ceil_div(ceil_div(p->max_idx, a.splits), kSaKeys) * kSaKeys;
+    a.split_len = min(kSaMaxSplit, ceil_div(ceil_div(p->max_idx, a.splits), kSaKeys) * kSaKeys);
     a.splits = ceil_div(p->max_idx, a.split_len);
     a.scale_log2 = p->scale * kLog2e;
     const size_t qrows = (size_t)p->n_rows * p->n_q;
@@ -401,7 +410,7 @@ extern "C" int crs_sparse_attn(const crs_attn_params *p, const void *Q, const vo
                                                          ((qrows * a.splits * kSaD * 4 + 255) &
                                                           ~size_t(255)))
                              : nullptr;
-    const size_t smem = sa_smem_bytes();
+    const size_t smem = sa_smem_bytes(a.split_len);
     CRS_TRY_CUDA(cudaFuncSetAttribute(sparse_attn_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     dim3 grid(a.splits, p->n_rows * p->n_kv);

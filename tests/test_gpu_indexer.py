@@ -85,10 +85,11 @@ def test_prefill_cuda_core_path(crs, cuda_dev, n_idx_heads):
 
 
 def test_prefill_all_tied_rows_take_exact_fallback(crs, cuda_dev):
-    """Every key identical: each row's scores tie, the sampled threshold lets all
-    keys through, lists overflow and those rows are recomputed exactly; ties go to
-    the smallest positions."""
-    n, topk = 6000, 1024
+    """Every key identical: each row's scores tie and the sampled threshold lets all
+    keys through.  Rows up to ~8k keys select among the ties (smallest positions
+    first); longer rows overflow their candidate lists and are recomputed by the
+    exact slice path."""
+    n, topk = 10000, 1024
     g = torch.Generator(device=cuda_dev).manual_seed(3)
     q = torch.randn(n, 4, 64, generator=g, device=cuda_dev).to(torch.bfloat16)
     w = torch.randn(n, 4, generator=g, device=cuda_dev)
@@ -101,7 +102,7 @@ def test_prefill_all_tied_rows_take_exact_fallback(crs, cuda_dev):
     assert crs.get_device_error() == 0
     g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
     assert (g_cnt == np.minimum(topk, np.arange(n) + 1)).all()
-    for r in (0, 100, topk, 4095, 4096, 4097, n - 1):
+    for r in (0, 100, topk, 4095, 4096, 4097, 8191, 8192, 8193, 9000, n - 1):
         m = min(topk, r + 1)
         assert (g_idx[r, :m] == np.arange(m)).all(), f"row {r}"
         assert (g_idx[r, m:] == -1).all()
