@@ -9,6 +9,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace crs {
 
@@ -237,62 +238,126 @@ block_score_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict_
     sc_out[((size_t)sh * G + g) * n_full + b0 + bl] = fmaf(0.5f, quad, lin);
 }
 
-// K9a specialised for G query heads and rank R: one thread per block holds
-// the G x (1 + R) dot products in registers; the block's descriptor rows are
-// streamed once with 16-byte loads and the scaled queries are read from
-// shared memory (the same address for every lane: a broadcast).
+// K9a specialised for G query heads and rank R, streaming the descriptors
+// through shared memory.  A CTA owns a contiguous range of blocks of one
+// (sequence, KV head); chunks of 16 blocks (mu 8 KB + xi 32 KB, contiguous in
+// HBM) arrive by two bulk copies each into a 2-stage ring, so one chunk is in
+// flight while the previous is scored (two CTAs per SM).  Eight lanes share a block: lane s reads
+// 16-byte chunks s, s + 8, s + 16, s + 24 of each 512-byte row (a group's
+// reads are 128 contiguous bytes: no bank conflicts), forms its G x (1 + R)
+// partial dot products with the scaled queries (read the same way), and the
+// group sums them with three shuffle steps.
+constexpr int kBsChunk = 16;                        // blocks per chunk
+constexpr int kBsThreadsT = 8 * kBsChunk;          // 8 lanes per block
+constexpr int kBsStages = 2;
+constexpr uint64_t kBsWaitNs = 1000000000ull;
+
 template <int G, int R>
-__global__ void __launch_bounds__(128)
-block_score_fixed_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ mu,
-                         const float *__restrict__ xi, float *__restrict__ sc_out, int n_kv,
-                         int n_q, int n_full, float scale) {
-    __shared__ __align__(16) float sq[G][kBdD];
+struct BsSmem {
+    float mu[kBsStages][kBsChunk][kBdD];
+    float xi[kBsStages][kBsChunk][R][kBdD];
+    float sq[G][kBdD];
+    uint64_t full[kBsStages];
+};
+
+template <int G, int R>
+__global__ void __launch_bounds__(kBsThreadsT, 2)
+block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ mu,
+                       const float *__restrict__ xi, float *__restrict__ sc_out, int n_kv, int n_q,
+                       int n_full, int blocks_per_cta, float scale) {
+    extern __shared__ __align__(128) unsigned char bs_raw[];
+    BsSmem<G, R> &S = *reinterpret_cast<BsSmem<G, R> *>(bs_raw);
     const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
-    for (int e = threadIdx.x; e < G * kBdD; e += blockDim.x) {
-        const int g = e / kBdD, d = e - g * kBdD;
-        sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+    const int b_lo = blockIdx.x * blocks_per_cta;
+    const int b_hi = min(n_full, b_lo + blocks_per_cta);
+    if (b_lo >= b_hi) return;
+    const int n_chunks = ceil_div(b_hi - b_lo, kBsChunk);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float *mu_sh = mu + (size_t)sh * n_full * kBdD;
+    const float *xi_sh = xi + (size_t)sh * n_full * R * kBdD;
+    auto issue = [&](int c) {                      // one thread
+        const int st = c % kBsStages;
+        const int b0 = b_lo + c * kBsChunk;
+        const int nb = min(kBsChunk, b_hi - b0);
+        const uint32_t mb = (uint32_t)nb * kBdD * 4, xb = mb * R;
+        tc::mbar_arrive_expect_tx(&S.full[st], mb + xb);
+        tc::bulk_load(&S.mu[st][0][0], mu_sh + (size_t)b0 * kBdD, mb, &S.full[st]);
+        tc::bulk_load(&S.xi[st][0][0][0], xi_sh + (size_t)b0 * R * kBdD, xb, &S.full[st]);
+    };
+    if (tid == 0) {
+        for (int st = 0; st < kBsStages; ++st) tc::mbar_init(&S.full[st], 1);
+        tc::mbar_fence_init();
     }
     __syncthreads();
-    const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= n_full) return;
-    const size_t blk = (size_t)sh * n_full + b;
-    const float4 *m4 = reinterpret_cast<const float4 *>(mu + blk * kBdD);
-    const float4 *x4 = reinterpret_cast<const float4 *>(xi + blk * R * kBdD);
-    float lin[G], pr[G][R];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        lin[g] = 0.0f;
-#pragma unroll
-        for (int e = 0; e < R; ++e) pr[g][e] = 0.0f;
+    if (tid == 0)
+        for (int c = 0; c < min(kBsStages, n_chunks); ++c) issue(c);
+    for (int e = tid; e < G * kBdD; e += blockDim.x) {
+        const int g = e / kBdD, d = e - g * kBdD;
+        S.sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
     }
-#pragma unroll 2
-    for (int d4 = 0; d4 < kBdD / 4; ++d4) {
-        const float4 mv = __ldg(m4 + d4);
-        float4 xv[R];
+    __syncthreads();
+    const int sub = lane & 7, grp = warp * 4 + (lane >> 3);     // block of the chunk
+    const float4 *q4 = reinterpret_cast<const float4 *>(&S.sq[0][0]);
+    bool ok = true;
+    for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % kBsStages;
+        ok = ok && tc::mbar_wait_bounded(&S.full[st], (c / kBsStages) & 1, kBsWaitNs, K_BLK_SCORE, 1);
+        if (__syncthreads_or(!ok)) break;
+        const int b = b_lo + c * kBsChunk + grp;
+        if (b < b_hi) {
+            const float4 *m4 = reinterpret_cast<const float4 *>(&S.mu[st][grp][0]);
+            const float4 *x4 = reinterpret_cast<const float4 *>(&S.xi[st][grp][0][0]);
+            float lin[G], pr[G][R];
 #pragma unroll
-        for (int e = 0; e < R; ++e) xv[e] = __ldg(x4 + e * (kBdD / 4) + d4);
+            for (int g = 0; g < G; ++g) {
+                lin[g] = 0.0f;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float4 qv = *reinterpret_cast<const float4 *>(&sq[g][d4 * 4]);
-            lin[g] = fmaf(qv.x, mv.x, lin[g]);
-            lin[g] = fmaf(qv.y, mv.y, lin[g]);
-            lin[g] = fmaf(qv.z, mv.z, lin[g]);
-            lin[g] = fmaf(qv.w, mv.w, lin[g]);
+                for (int e = 0; e < R; ++e) pr[g][e] = 0.0f;
+            }
 #pragma unroll
-            for (int e = 0; e < R; ++e) {
-                pr[g][e] = fmaf(qv.x, xv[e].x, pr[g][e]);
-                pr[g][e] = fmaf(qv.y, xv[e].y, pr[g][e]);
-                pr[g][e] = fmaf(qv.z, xv[e].z, pr[g][e]);
-                pr[g][e] = fmaf(qv.w, xv[e].w, pr[g][e]);
+            for (int u = 0; u < 4; ++u) {
+                const int f = u * 8 + sub;                 // 16-byte chunk of the row
+                const float4 mv = m4[f];
+                float4 xv[R];
+#pragma unroll
+                for (int e = 0; e < R; ++e) xv[e] = x4[e * (kBdD / 4) + f];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float4 qv = q4[g * (kBdD / 4) + f];
+                    lin[g] = fmaf(qv.x, mv.x, lin[g]);
+                    lin[g] = fmaf(qv.y, mv.y, lin[g]);
+                    lin[g] = fmaf(qv.z, mv.z, lin[g]);
+                    lin[g] = fmaf(qv.w, mv.w, lin[g]);
+#pragma unroll
+                    for (int e = 0; e < R; ++e) {
+                        pr[g][e] = fmaf(qv.x, xv[e].x, pr[g][e]);
+                        pr[g][e] = fmaf(qv.y, xv[e].y, pr[g][e]);
+                        pr[g][e] = fmaf(qv.z, xv[e].z, pr[g][e]);
+                        pr[g][e] = fmaf(qv.w, xv[e].w, pr[g][e]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    lin[g] += __shfl_xor_sync(0xffffffffu, lin[g], off);
+#pragma unroll
+                    for (int e = 0; e < R; ++e) pr[g][e] += __shfl_xor_sync(0xffffffffu, pr[g][e], off);
+                }
+            }
+            if (sub == 0) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float quad = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < R; ++e) quad = fmaf(pr[g][e], pr[g][e], quad);
+                    sc_out[((size_t)sh * G + g) * n_full + b] = fmaf(0.5f, quad, lin[g]);
+                }
             }
         }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float quad = 0.0f;
-#pragma unroll
-        for (int e = 0; e < R; ++e) quad = fmaf(pr[g][e], pr[g][e], quad);
-        sc_out[((size_t)sh * G + g) * n_full + b] = fmaf(0.5f, quad, lin[g]);
+        __syncthreads();                                  // stage st is read: refill it
+        if (tid == 0 && c + kBsStages < n_chunks) issue(c + kBsStages);
     }
 }
 
@@ -517,10 +582,16 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a));
     float *sc = static_cast<float *>(ws);
     if (G == 8 && p->b.rank == 4) {
-        dim3 gf(ceil_div(n_full, 128), p->b.n_seq * p->b.n_kv);
+        const int n_sh = p->b.n_seq * p->b.n_kv;
+        const int per_sh = max(1, min(ceil_div(n_full, kBsChunk), ceil_div(148 * 4, n_sh)));
+        const int bpc = ceil_div(ceil_div(n_full, per_sh), kBsChunk) * kBsChunk;
+        const size_t smem_s = sizeof(BsSmem<8, 4>);
+        CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_tma_kernel<8, 4>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
+        dim3 gf(ceil_div(n_full, bpc), n_sh);
         ProfScope _ps(K_BLK_SCORE, s);
-        block_score_fixed_kernel<8, 4><<<gf, 128, 0, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu,
-                                                         xi, sc, p->b.n_kv, p->n_q, n_full, p->scale);
+        block_score_tma_kernel<8, 4><<<gf, kBsThreadsT, smem_s, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu, xi,
+                                                            sc, p->b.n_kv, p->n_q, n_full, bpc, p->scale);
     } else {
     dim3 ga(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv);
     {
