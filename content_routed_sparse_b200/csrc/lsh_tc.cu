@@ -43,6 +43,7 @@ constexpr uint32_t kTcCols = 256;
 constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s: a wait that long means a fault
 constexpr int kBktBefore = -1;                  // absent slot before the sequence
 constexpr int kBktAfter = 0x7fffffff;           // absent slot after the sequence
+constexpr float kTcBoundMax = 48.0f;            // single pass while 2^(-2 bound) stays normal
 
 struct LshTcSmem {
     // K tile (rows = keys; rows 128..255 = Q tile) until S is computed, then
@@ -65,6 +66,12 @@ struct LshTcSmem {
     uint64_t bar[3];
     uint32_t tmem_base;
 };
+
+__device__ __forceinline__ float ex2_approx(float x) {   // 2^x, PTX ex2.approx (rel. err ~2^-22)
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
 
 struct LshTcRow {
     int row, jq, lo, hi, pos_i;
@@ -130,7 +137,7 @@ __device__ __forceinline__ float lsh_tc_pass2(LshTcSmem &S, const LshTcRow &q, u
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int t = t2 * 2 + e;
-                    pv[e] = ((mb >> t) & 1u) ? exp2f(__uint_as_float(v[t]) * S.kscale[c0 + t] - M)
+                    pv[e] = ((mb >> t) & 1u) ? ex2_approx(__uint_as_float(v[t]) * S.kscale[c0 + t] - M)
                                              : 0.0f;
                     sum += pv[e];
                 }
@@ -139,6 +146,91 @@ __device__ __forceinline__ float lsh_tc_pass2(LshTcSmem &S, const LshTcRow &q, u
                 __nv_bfloat162 l2 = __floats2bfloat162_rn(pv[0] - hf.x, pv[1] - hf.y);
                 hi[t2] = *reinterpret_cast<uint32_t *>(&h2);
                 lo[t2] = *reinterpret_cast<uint32_t *>(&l2);
+            }
+        } else {
+#pragma unroll
+            for (int t2 = 0; t2 < 16; ++t2) hi[t2] = lo[t2] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t off = tc::sw128(q.row, cc * 4 + u);
+            *reinterpret_cast<uint4 *>(p_hi + off) =
+                make_uint4(hi[u * 4], hi[u * 4 + 1], hi[u * 4 + 2], hi[u * 4 + 3]);
+            *reinterpret_cast<uint4 *>(p_lo + off) =
+                make_uint4(lo[u * 4], lo[u * 4 + 1], lo[u * 4 + 2], lo[u * 4 + 3]);
+        }
+    }
+    return sum;
+}
+
+// Bits t of the 32 columns [c0, c0 + 32) with lo <= c0 + t <= hi.
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int c0) {
+    const int a = lo - c0, b = hi - c0;
+    if (b < 0 || a > 31 || a > b) return 0u;
+    const uint32_t low = a <= 0 ? 0xffffffffu : (0xffffffffu << a);
+    const uint32_t high = b >= 31 ? 0xffffffffu : ((2u << b) - 1u);
+    return low & high;
+}
+
+// Single pass for normalised keys: every logit of row i is at most
+// M_i = scale |q_i| (log2 units), so P = 2^(S - M_i) needs no row maximum.
+// Keys [col0, col0 + 64) of the row: masks (range bits, earlier-round
+// pairs), P into K-block `blk` of the P buffer (value and residual); returns
+// the partial row sum.  NR = earlier rounds (R < 0: runtime count r).
+template <int NR>
+__device__ __forceinline__ float lsh_tc_fused(LshTcSmem &S, const LshTcRow &q, uint32_t trow,
+                                              int col0, int blk, float M, int r) {
+    const int R = NR >= 0 ? NR : r;
+    float sum = 0.0f;
+    unsigned char *p_hi = S.kp[blk];
+    unsigned char *p_lo = S.kp[2 + blk];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = col0 + cc * 32;
+        uint32_t mb = q.qvalid ? range_bits(q.lo, q.hi, c0) : 0u;
+        if (q.excl_self && q.jq >= c0 && q.jq < c0 + 32) mb &= ~(1u << (q.jq - c0));
+        uint32_t hi[16], lo[16];
+        if (__any_sync(0xffffffffu, mb != 0u)) {
+            uint32_t v[32];
+            tc::tmem_ld32(trow + c0, v);
+            // pairs met in an earlier round (same bucket, key chunk = query chunk or the one before)
+#pragma unroll
+            for (int rr = 0; rr < (NR >= 0 ? NR : kMaxRounds - 1); ++rr) {
+                if (NR < 0 && rr >= R) break;
+                const int4 *kc = reinterpret_cast<const int4 *>(&S.kcode[rr][c0]);
+                const int ci = S.kcode[rr][q.jq];
+                uint32_t dup = 0u;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int4 k4 = kc[u];
+                    dup |= ((uint32_t)(ci - k4.x) <= 1u ? 1u : 0u) << (4 * u);
+                    dup |= ((uint32_t)(ci - k4.y) <= 1u ? 1u : 0u) << (4 * u + 1);
+                    dup |= ((uint32_t)(ci - k4.z) <= 1u ? 1u : 0u) << (4 * u + 2);
+                    dup |= ((uint32_t)(ci - k4.w) <= 1u ? 1u : 0u) << (4 * u + 3);
+                }
+                mb &= ~dup;
+            }
+            tc::tmem_ld_wait();
+            const float4 *ks = reinterpret_cast<const float4 *>(&S.kscale[c0]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 k4 = ks[u];
+                const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+                float pv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = 4 * u + e;
+                    pv[e] = ((mb >> t) & 1u) ? ex2_approx(fmaf(__uint_as_float(v[t]), kk[e], -M)) : 0.0f;
+                    sum += pv[e];
+                }
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[2 * e2], pv[2 * e2 + 1]);
+                    const float2 hf = __bfloat1622float2(h2);
+                    __nv_bfloat162 l2 = __floats2bfloat162_rn(pv[2 * e2] - hf.x, pv[2 * e2 + 1] - hf.y);
+                    hi[2 * u + e2] = *reinterpret_cast<uint32_t *>(&h2);
+                    lo[2 * u + e2] = *reinterpret_cast<uint32_t *>(&l2);
+                }
             }
         } else {
 #pragma unroll
@@ -268,6 +360,7 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
+    bool big = false;
     {
         const int j = tid;
         float ss = 0.0f;
@@ -284,9 +377,16 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         }
         const float inv = key_norm ? (ss > 0.0f ? rsqrtf(ss) : 0.0f) : 1.0f;
         S.kscale[j] = inv * scale_log2;
+        // own-chunk row: with normalised keys its logits are at most scale |q| (log2 units)
+        if (j >= kTcM) {
+            const float bound = sqrtf(ss) * fabsf(scale_log2);
+            S.rowmax[1][j - kTcM] = bound;
+            big = bound > kTcBoundMax;
+        }
     }
     tc::fence_proxy_async();
-    __syncthreads();
+    // single pass unless keys are raw or some bound is so large that 2^(S - bound) could underflow
+    const bool single = key_norm && !__syncthreads_or(big);
     const uint32_t tmem = S.tmem_base;
 
     // ---- 3. S = Q K^T into TMEM columns [0, 256)
@@ -321,21 +421,28 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         q.excl_self = (!causal) && no_self;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
 
-        // ---- 4a. pass 1: masks and row maxima
-        float mx;
-        switch (r) {
-            case 0: mx = lsh_tc_pass1<0>(S, q, trow, wg); break;
-            case 1: mx = lsh_tc_pass1<1>(S, q, trow, wg); break;
-            case 2: mx = lsh_tc_pass1<2>(S, q, trow, wg); break;
-            case 3: mx = lsh_tc_pass1<3>(S, q, trow, wg); break;
-            case 4: mx = lsh_tc_pass1<4>(S, q, trow, wg); break;
-            case 5: mx = lsh_tc_pass1<5>(S, q, trow, wg); break;
-            case 6: mx = lsh_tc_pass1<6>(S, q, trow, wg); break;
-            default: mx = lsh_tc_pass1<7>(S, q, trow, wg); break;
+        // ---- 4a. the exponent shift M: the row bound (single pass), or pass 1's
+        // masks and row maxima
+        float M;
+        if (single) {
+            M = S.rowmax[1][q.row];
+        } else {
+            float mx;
+            switch (r) {
+                case 0: mx = lsh_tc_pass1<0>(S, q, trow, wg); break;
+                case 1: mx = lsh_tc_pass1<1>(S, q, trow, wg); break;
+                case 2: mx = lsh_tc_pass1<2>(S, q, trow, wg); break;
+                case 3: mx = lsh_tc_pass1<3>(S, q, trow, wg); break;
+                case 4: mx = lsh_tc_pass1<4>(S, q, trow, wg); break;
+                case 5: mx = lsh_tc_pass1<5>(S, q, trow, wg); break;
+                case 6: mx = lsh_tc_pass1<6>(S, q, trow, wg); break;
+                default: mx = lsh_tc_pass1<7>(S, q, trow, wg); break;
+            }
+            __syncthreads();                     // row bounds in rowmax[1] are no longer needed
+            S.rowmax[wg][q.row] = mx;
+            __syncthreads();
+            M = fmaxf(S.rowmax[0][q.row], S.rowmax[1][q.row]);
         }
-        S.rowmax[wg][q.row] = mx;
-        __syncthreads();
-        const float M = fmaxf(S.rowmax[0][q.row], S.rowmax[1][q.row]);
 
         // ---- 4b/5. per 128-key half: P into the buffer, then O += P V_half
         float sum = 0.0f;
@@ -346,7 +453,18 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
                 if (__syncthreads_or(!ok_wait)) goto teardown;
                 tc::fence_after();
             }
-            sum += lsh_tc_pass2(S, q, trow, half * 128 + wg * 64, wg, M);
+            const int col0 = half * 128 + wg * 64;
+            if (single) {
+                switch (r) {
+                    case 0: sum += lsh_tc_fused<0>(S, q, trow, col0, wg, M, r); break;
+                    case 1: sum += lsh_tc_fused<1>(S, q, trow, col0, wg, M, r); break;
+                    case 2: sum += lsh_tc_fused<2>(S, q, trow, col0, wg, M, r); break;
+                    case 3: sum += lsh_tc_fused<3>(S, q, trow, col0, wg, M, r); break;
+                    default: sum += lsh_tc_fused<-1>(S, q, trow, col0, wg, M, r); break;
+                }
+            } else {
+                sum += lsh_tc_pass2(S, q, trow, col0, wg, M);
+            }
             tc::fence_proxy_async();
             tc::fence_before();
             __syncthreads();
