@@ -99,22 +99,25 @@ __global__ void __launch_bounds__(kHashTok) lsh_hash_fixed_kernel(const T *__res
 #pragma unroll
         for (int k0 = 0; k0 < HALF; k0 += 32) {
             constexpr int W = HALF < 32 ? HALF : 32;
-            float u[W];
+            // u_k pairs (k, k + 1) advance together with one paired fused multiply-add:
+            // each lane rounds exactly like __fmaf_rn, in the same index order
+            uint64_t u2[W / 2];
 #pragma unroll
-            for (int j = 0; j < W; ++j) u[j] = 0.0f;
+            for (int j = 0; j < W / 2; ++j) u2[j] = 0ull;
 #pragma unroll
             for (int t = 0; t < D; ++t) {
-                const float xv = x[t];
-                const float4 *rr = reinterpret_cast<const float4 *>(Rs + t * HALF + k0);
+                const uint64_t xx = f32x2_pack(x[t], x[t]);
+                const ulonglong2 *rr = reinterpret_cast<const ulonglong2 *>(Rs + t * HALF + k0);
 #pragma unroll
                 for (int j4 = 0; j4 < W / 4; ++j4) {
-                    const float4 rv = rr[j4];
-                    u[4 * j4 + 0] = __fmaf_rn(xv, rv.x, u[4 * j4 + 0]);
-                    u[4 * j4 + 1] = __fmaf_rn(xv, rv.y, u[4 * j4 + 1]);
-                    u[4 * j4 + 2] = __fmaf_rn(xv, rv.z, u[4 * j4 + 2]);
-                    u[4 * j4 + 3] = __fmaf_rn(xv, rv.w, u[4 * j4 + 3]);
+                    const ulonglong2 rv = rr[j4];
+                    u2[2 * j4] = f32x2_fma(xx, rv.x, u2[2 * j4]);
+                    u2[2 * j4 + 1] = f32x2_fma(xx, rv.y, u2[2 * j4 + 1]);
                 }
             }
+            float u[W];
+#pragma unroll
+            for (int j = 0; j < W / 2; ++j) f32x2_unpack(u2[j], u[2 * j], u[2 * j + 1]);
 #pragma unroll
             for (int j = 0; j < W; ++j) {
                 const int k = k0 + j;
@@ -370,11 +373,19 @@ __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *
     const long long rowi = gt / G4;
     const int bh = (int)(rowi / n), pos = (int)(rowi - (long long)bh * n);
     const int vl = valid_len ? valid_len[bh / H] : n;
+    // every round's lse and partial output are requested before any is used
     float l[kMaxRounds];
+    float4 ov[kMaxRounds];
     float mx = -INFINITY;
 #pragma unroll
     for (int r = 0; r < kMaxRounds; ++r) {
-        l[r] = (r < rounds) ? lse_ws[((size_t)r * BH + bh) * n + pos] : -INFINITY;
+        if (r < rounds) {
+            l[r] = __ldcs(lse_ws + ((size_t)r * BH + bh) * n + pos);
+            ov[r] = __ldcs(reinterpret_cast<const float4 *>(o_ws + (((size_t)r * BH + bh) * n + pos) * DH) + g);
+        } else {
+            l[r] = -INFINITY;
+            ov[r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
         mx = fmaxf(mx, l[r]);
     }
     float4 *o = reinterpret_cast<float4 *>(O + ((size_t)bh * n + pos) * DH) + g;
@@ -392,7 +403,7 @@ __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *
     for (int r = 0; r < kMaxRounds; ++r) {
         if (r < rounds && l[r] != -INFINITY) {
             const float wgt = __expf(l[r] - LSE);
-            const float4 v = reinterpret_cast<const float4 *>(o_ws + (((size_t)r * BH + bh) * n + pos) * DH)[g];
+            const float4 v = ov[r];
             acc.x = fmaf(wgt, v.x, acc.x);
             acc.y = fmaf(wgt, v.y, acc.y);
             acc.z = fmaf(wgt, v.z, acc.z);
