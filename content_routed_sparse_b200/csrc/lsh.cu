@@ -130,6 +130,85 @@ __global__ void __launch_bounds__(kHashTok) lsh_hash_fixed_kernel(const T *__res
     }
 }
 
+// K1 for bf16 rows, two tokens per thread (i and i + 128 of a 256-token tile):
+// each R value read from shared memory feeds both tokens, halving the
+// shared-memory loads per FMA (the limit of the one-token kernel).  Rows stay
+// packed as bf16 pairs in registers and are upcast exactly when used; the FMA
+// chain of every u_k is unchanged (index order from 0, one rounding per step),
+// so the bucket ids are identical.
+constexpr int kHash2Tok = 2 * kHashTok;
+
+template <int D, int HALF>
+__global__ void __launch_bounds__(kHashTok) lsh_hash_bf16x2_kernel(const __nv_bfloat16 *__restrict__ X,
+                                                                   const float *__restrict__ R,
+                                                                   int32_t *__restrict__ bucket,
+                                                                   int H, int n, int rounds) {
+    __shared__ __align__(16) float Rs[D * HALF];
+    const int bh = blockIdx.z, h = bh % H;
+    const int i0 = blockIdx.x * kHash2Tok + threadIdx.x, i1 = i0 + kHashTok;
+    uint32_t xa[D / 2], xb[D / 2];
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
+        if (i0 < n) va = reinterpret_cast<const uint4 *>(X + ((size_t)bh * n + i0) * D)[c];
+        if (i1 < n) vb = reinterpret_cast<const uint4 *>(X + ((size_t)bh * n + i1) * D)[c];
+        xa[4 * c] = va.x; xa[4 * c + 1] = va.y; xa[4 * c + 2] = va.z; xa[4 * c + 3] = va.w;
+        xb[4 * c] = vb.x; xb[4 * c + 1] = vb.y; xb[4 * c + 2] = vb.z; xb[4 * c + 3] = vb.w;
+    }
+    for (int r = 0; r < rounds; ++r) {
+        __syncthreads();
+        const float4 *Rg = reinterpret_cast<const float4 *>(R + ((size_t)h * rounds + r) * D * HALF);
+        for (int e = threadIdx.x; e < D * HALF / 4; e += kHashTok)
+            reinterpret_cast<float4 *>(Rs)[e] = Rg[e];
+        __syncthreads();
+        float bp[2] = {0.0f, 0.0f}, bn[2] = {0.0f, 0.0f};
+        int ap[2] = {0, 0}, an[2] = {0, 0};
+#pragma unroll 1
+        for (int k0 = 0; k0 < HALF; k0 += 16) {
+            constexpr int W = HALF < 16 ? HALF : 16;
+            uint64_t ua[W / 2], ub[W / 2];
+#pragma unroll
+            for (int j = 0; j < W / 2; ++j) ua[j] = ub[j] = 0ull;
+#pragma unroll
+            for (int t = 0; t < D; ++t) {
+                // exact bf16 -> fp32: the 16 bits become the high half of the float
+                const uint32_t wa = xa[t >> 1], wb = xb[t >> 1];
+                const float fa = __uint_as_float((t & 1) ? (wa & 0xffff0000u) : (wa << 16));
+                const float fb = __uint_as_float((t & 1) ? (wb & 0xffff0000u) : (wb << 16));
+                const uint64_t pa = f32x2_pack(fa, fa), pb = f32x2_pack(fb, fb);
+                const ulonglong2 *rr = reinterpret_cast<const ulonglong2 *>(Rs + t * HALF + k0);
+#pragma unroll
+                for (int j4 = 0; j4 < W / 4; ++j4) {
+                    const ulonglong2 rv = rr[j4];
+                    ua[2 * j4] = f32x2_fma(pa, rv.x, ua[2 * j4]);
+                    ua[2 * j4 + 1] = f32x2_fma(pa, rv.y, ua[2 * j4 + 1]);
+                    ub[2 * j4] = f32x2_fma(pb, rv.x, ub[2 * j4]);
+                    ub[2 * j4 + 1] = f32x2_fma(pb, rv.y, ub[2 * j4 + 1]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < W / 2; ++j) {
+                float u[2][2];
+                f32x2_unpack(ua[j], u[0][0], u[0][1]);
+                f32x2_unpack(ub[j], u[1][0], u[1][1]);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int k = k0 + 2 * j + e;
+#pragma unroll
+                    for (int z = 0; z < 2; ++z) {
+                        if (k == 0 || u[z][e] > bp[z]) { bp[z] = u[z][e]; ap[z] = k; }
+                        const float nu = -u[z][e];
+                        if (k == 0 || nu > bn[z]) { bn[z] = nu; an[z] = k; }
+                    }
+                }
+            }
+        }
+        int32_t *bo = bucket + ((size_t)bh * rounds + r) * n;
+        if (i0 < n) bo[i0] = (bp[0] >= bn[0]) ? ap[0] : HALF + an[0];
+        if (i1 < n) bo[i1] = (bp[1] >= bn[1]) ? ap[1] : HALF + an[1];
+    }
+}
+
 // --------------------------------------------------------------------------
 // K2: stable counting sort of one (b, h, round) segment per CTA.
 // Histogram -> exclusive scan (bucket bases) -> tiles of blockDim positions
@@ -457,11 +536,12 @@ extern "C" int crs_lsh_route(const crs_lsh_params *p, const void *X, const float
                 lsh_hash_fixed_kernel<float, 64, 8><<<g2, kHashTok, 0, s>>>(
                     static_cast<const float *>(X), R, bucket, p->H, p->n, p->n_rounds);
         } else {
+            dim3 g3(ceil_div(p->n, kHash2Tok), 1, p->B * p->H);
             if (half == 32)
-                lsh_hash_fixed_kernel<__nv_bfloat16, 64, 32><<<g2, kHashTok, 0, s>>>(
+                lsh_hash_bf16x2_kernel<64, 32><<<g3, kHashTok, 0, s>>>(
                     static_cast<const __nv_bfloat16 *>(X), R, bucket, p->H, p->n, p->n_rounds);
             else
-                lsh_hash_fixed_kernel<__nv_bfloat16, 64, 8><<<g2, kHashTok, 0, s>>>(
+                lsh_hash_bf16x2_kernel<64, 8><<<g3, kHashTok, 0, s>>>(
                     static_cast<const __nv_bfloat16 *>(X), R, bucket, p->H, p->n, p->n_rounds);
         }
     } else if (p->dtype == CRS_F32) {
