@@ -235,6 +235,8 @@ class DecodeWorkload(Workload):
         ns, k = self.p["n_seq"], self.p["topk"]
         return {
             "idx_slice_topk": [("hbm", self.total_ctx * 64 * 2 / 1e9, "GB/s")],
+            # the select reads each row's score keys (4 B per cached token)
+            "idx_select": [("hbm", self.total_ctx * 4 / 1e9, "GB/s")],
             "sparse_attn": [("hbm", ns * k * 8 * 128 * 2 * 2 / 1e9, "GB/s")],
         }
 
@@ -379,15 +381,15 @@ def time_steps(fn, steps, warmup, flush_buf, dist_on):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def _traffic(kernel):
-    """DRAM bytes per launch from profiles/traffic.json, only while the kernel's
-    source file is unchanged since the capture (else None)."""
+def _traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from profiles/traffic.json,
+    only while the kernel's source file is unchanged since the capture (else None)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        t = json.load(f).get(kernel)
+        t = json.load(f).get(f"{kernel}@{workload}")
     if not t:
         return None
     src = os.path.join(ROOT, t["source"])
@@ -420,7 +422,7 @@ def roofline(wl, prof, peaks, traffic=None):
     else:
         peak, src = FP32_ALU_TFLOPS_NOMINAL, "fp32 FMA: 148 SM x 128 lanes x 2 x 1.965 GHz"
     out = {"kernel": top, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
-           "unit": unit, "frac": round(achieved / peak, 4), "traffic": _traffic(top),
+           "unit": unit, "frac": round(achieved / peak, 4), "traffic": _traffic(top, wl.name),
            "peak_source": src,
            "per_launch_ms": round(per_launch_s * 1e3, 5)}
     if len(spec[top]) > 1:
