@@ -16,10 +16,10 @@
 //   SAMPLE: every 8th key tile; scores (top 16 bits of the order-preserving
 //           key) are written out per row;
 //   FILTER: every key tile; a score whose key is >= the row's threshold is
-//           appended to that (row, part)'s candidate list, in position order.
+//           appended to that (row, part)'s candidate list.
 // idx_tc_tau_kernel picks each row's threshold from its samples so that about
-// 1.25 k scores pass; idx_tc_final_kernel merges a row's four candidate lists
-// by position and selects the exact top-k (ties to the smaller position); a
+// 1.25 k scores pass; idx_tc_final_kernel selects the exact top-k over a row's
+// four candidate lists (ties to the smaller position, output ascending); a
 // row whose candidates number fewer than k or overflowed a list is recomputed
 // by the exact CUDA-core slice path.  The threshold only decides how much work
 // the final selection sees, never the result.
@@ -47,6 +47,7 @@ constexpr int kIFlush = 8;          //   written out 8 at a time (one 32-byte ru
 constexpr int kIEpiWarps = 4 * kIParts;             // 4 TMEM lane quadrants x 4 parts
 constexpr int kIThreads = 32 * (4 + kIEpiWarps);    // TMA, MMA, TMEM-alloc, spare + epilogue
 constexpr uint64_t kIWaitNs = 2000000000ull;
+constexpr uint32_t kISuspendNs = 128;    // pipeline waits: short suspends, prompt wake-up
 constexpr float kIBeta = 1.25f;
 
 struct IdxTcSmem {
@@ -105,6 +106,13 @@ __device__ __forceinline__ unsigned flush_round(const IdxTcArgs &a, const uint64
     return rows & ~m;
 }
 
+// 0xffffffff if a >= b (false for NaN), else 0
+__device__ __forceinline__ uint32_t set_ge_mask(float a, float b) {
+    uint32_t r;
+    asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 template <int MODE>   // 0 = SAMPLE, 1 = FILTER
 __global__ void __launch_bounds__(kIThreads, 1)
 idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -119,6 +127,9 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
     const int key_end = min(a.n, r0 + kIqM);                  // causal: keys < key_end
     const int nt_all = (key_end + kIkN - 1) / kIkN;
     const int ntiles = MODE == 0 ? (nt_all + kISampStride - 1) / kISampStride : nt_all;
+    // CTAs start at different key tiles (and wrap), so they do not all read the same
+    // tile of K at once; a row's candidate order does not matter to the selection
+    const int t_off = ntiles > 0 ? (int)((blockIdx.x * 37u) % (unsigned)ntiles) : 0;
 
     if (tid == 0) {
         tc::mbar_init(&S.qfull, 1);
@@ -154,11 +165,12 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             for (int j = 0; j < ntiles; ++j) {
                 const int s = j % kIStages, u = j / kIStages;
                 if (u > 0 &&
-                    !tc::mbar_wait_bounded(&S.kempty[s], (u - 1) & 1, kIWaitNs, K_IDX_PREFILL_TC, 1)) {
+                    !tc::mbar_wait_bounded(&S.kempty[s], (u - 1) & 1, kIWaitNs, K_IDX_PREFILL_TC, 1, kISuspendNs)) {
                     atomicOr(&S.fail, 1);
                     break;
                 }
-                const int kt = MODE == 0 ? j * kISampStride : j;
+                const int js = j + t_off < ntiles ? j + t_off : j + t_off - ntiles;
+                const int kt = MODE == 0 ? js * kISampStride : js;
                 tc::mbar_arrive_expect_tx(&S.kfull[s], kIkN * 128);
                 tc::tma_load_2d(S.k[s], &tk, 0, kt * kIkN, &S.kfull[s]);
             }
@@ -167,12 +179,12 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         // ---------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_bf16_f32(kIqM, kIkN, 0, 0);
-            bool ok = tc::mbar_wait_bounded(&S.qfull, 0, kIWaitNs, K_IDX_PREFILL_TC, 2);
+            bool ok = tc::mbar_wait_bounded(&S.qfull, 0, kIWaitNs, K_IDX_PREFILL_TC, 2, kISuspendNs);
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int s = j % kIStages, u = j / kIStages;
                 const int b = j & 1, v = j >> 1;
-                ok = tc::mbar_wait_bounded(&S.kfull[s], u & 1, kIWaitNs, K_IDX_PREFILL_TC, 3);
-                if (ok && v > 0) ok = tc::mbar_wait_bounded(&S.tempty[b], (v - 1) & 1, kIWaitNs, K_IDX_PREFILL_TC, 4);
+                ok = tc::mbar_wait_bounded(&S.kfull[s], u & 1, kIWaitNs, K_IDX_PREFILL_TC, 3, kISuspendNs);
+                if (ok && v > 0) ok = tc::mbar_wait_bounded(&S.tempty[b], (v - 1) & 1, kIWaitNs, K_IDX_PREFILL_TC, 4, kISuspendNs);
                 if (!ok) break;
                 tc::fence_after();
                 const uint32_t kbase = smem_u32(S.k[s]);
@@ -210,7 +222,7 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         float *stage = &S.stage[ew][0][0];
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1, v = j >> 1;
-            const bool ok = tc::mbar_wait_bounded(&S.tfull[b], v & 1, kIWaitNs, K_IDX_PREFILL_TC, 5);
+            const bool ok = tc::mbar_wait_bounded(&S.tfull[b], v & 1, kIWaitNs, K_IDX_PREFILL_TC, 5, kISuspendNs);
             if (__any_sync(0xffffffffu, !ok)) {
                 if (lane == 0) atomicOr(&S.fail, 1);
                 break;
@@ -241,7 +253,8 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
                 nanacc = f32x2_fma(acc[i], 0ull, nanacc);
                 f32x2_unpack(acc[i], sc[2 * i], sc[2 * i + 1]);
             }
-            const int kt = MODE == 0 ? j * kISampStride : j;
+            const int js = j + t_off < ntiles ? j + t_off : j + t_off - ntiles;
+            const int kt = MODE == 0 ? js * kISampStride : js;
             const int key0 = kt * kIkN + part * kIPartKeys;
             // keys > t (causal) exist only in the CTA's last two tiles
             const int lim = t - key0 + 1;            // keys [key0, key0 + lim) are visible
@@ -256,14 +269,15 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
                         pk[i] = lo | (hi << 16);
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(a.samples + (size_t)t * a.samp_slots +
-                                                           j * kIkN + part * kIPartKeys);
+                                                           js * kIkN + part * kIPartKeys);
                     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             } else {
+                // pass mask: set.ge gives an all-ones word per passing key, one LOP3 merges it
                 uint32_t pm = 0u;
 #pragma unroll
-                for (int i = 0; i < kIPartKeys; ++i) pm |= (sc[i] >= tauf ? 1u : 0u) << i;
+                for (int i = 0; i < kIPartKeys; ++i) pm |= set_ge_mask(sc[i], tauf) & (1u << i);
                 pm &= row_ok ? vis : 0u;
                 if (__any_sync(0xffffffffu, pm != 0u)) {
                     // the scores go through shared memory so that the set bits can

@@ -120,22 +120,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *mbar, uint32_t parity, u
         : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after `limit_ns` of wall time (globaltimer, checked
-// after every poll of at most 10 us), raises CRS_DEVERR_TIMEOUT and records
-// (kernel, site) in the diagnostic record.
+// Bounded wait: gives up after `limit_ns` of wall time, raises
+// CRS_DEVERR_TIMEOUT and records (kernel, site) in the diagnostic record.  The
+// phase is polled with try_wait (each poll suspends at most `suspend_ns`); the
+// global timer is read only every 256 polls, because reading it is slow and a
+// read between polls would delay the wake-up of every pipeline handoff.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parity,
                                                   uint64_t limit_ns, uint32_t kernel,
-                                                  uint32_t site) {
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t polls = 0;
-    while (true) {
-        if (mbar_try_wait(mbar, parity, 10000u)) return true;
-        ++polls;
-        if (globaltimer_ns() - t0 > limit_ns) break;
+                                                  uint32_t site, uint32_t suspend_ns = 10000u) {
+    uint64_t t0 = 0;
+    for (uint32_t polls = 1;; ++polls) {
+        if (mbar_try_wait(mbar, parity, suspend_ns)) return true;
+        if ((polls & 255u) == 0u) {
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > limit_ns) {
+                raise_error(CRS_DEVERR_TIMEOUT);
+                diag_record(kernel, site, polls, threadIdx.x, 0, 0);
+                return false;
+            }
+        }
     }
-    raise_error(CRS_DEVERR_TIMEOUT);
-    diag_record(kernel, site, polls, threadIdx.x, 0, 0);
-    return false;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *mbar) {
