@@ -347,7 +347,7 @@ static size_t sa_smem_bytes(int split_len) {
 static int sa_splits(const crs_attn_params *p) {
     const long long items = (long long)p->n_rows * p->n_kv;
     const int max_split = max(1, ceil_div(p->max_idx, 256));   // >= 256 keys per split
-    const long long target = 148LL * 8;
+    const long long target = 148LL * 2;   // two CTAs per SM are resident
     int s = (int)((target + items - 1) / items);
     s = max(1, min(s, max_split));
     return max(s, ceil_div(p->max_idx, kSaMaxSplit));
