@@ -386,11 +386,15 @@ struct DecArgs {
     const float *w;
     const __nv_bfloat16 *k;
     const int64_t *k_off;
-    uint32_t *keys;                       // [total keys] score keys
+    uint32_t *keys;                       // [rows][max_words * 32] score keys
     uint32_t *hist;                       // [rows][kDecBins]
+    uint32_t *bm_gt, *bm_eq;              // [rows][max_words] position bitmaps
+    uint2 *eq_buf;                        // [rows][kDecEqCap] (key, position) of bucket B
+    int *eq_cnt;                          // [rows]
+    int4 *info;                           // [rows]: bucket B, to take from B, |B|, 0
     int32_t *out_idx;
     int32_t *out_cnt;
-    int n_rows, H, topk, max_tiles;
+    int n_rows, H, topk, max_tiles, max_words;
 };
 
 // Scores on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
@@ -424,9 +428,9 @@ __global__ void __launch_bounds__(kDecThreads) idx_decode_score_kernel(DecArgs a
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t kb = a.k_off[row];
     int nv = (int)(a.k_off[row + 1] - kb);
-    if (nv > a.max_tiles * kDecTile) {
+    if (nv > a.max_words * 32) {                 // longer than the caller's bound
         if (tile == 0 && threadIdx.x == 0) raise_error(CRS_DEVERR_INDEX);
-        nv = a.max_tiles * kDecTile;
+        nv = a.max_words * 32;
     }
     if (nv <= a.topk) return;                 // every key is selected; no score needed
     const int s0 = tile * kDecTile;
@@ -505,12 +509,12 @@ __global__ void __launch_bounds__(kDecThreads) idx_decode_score_kernel(DecArgs a
             const int k_lo = sl * kDecSlice + g, k_hi = k_lo + 8;
             if (k_lo < ns) {
                 const uint32_t key = score_key(s_lo);
-                a.keys[kb + s0 + k_lo] = key;
+                a.keys[(size_t)row * a.max_words * 32 + s0 + k_lo] = key;
                 atomicAdd(&sh[key >> 20], 1u);
             }
             if (k_hi < ns) {
                 const uint32_t key = score_key(s_hi);
-                a.keys[kb + s0 + k_hi] = key;
+                a.keys[(size_t)row * a.max_words * 32 + s0 + k_hi] = key;
                 atomicAdd(&sh[key >> 20], 1u);
             }
         }
@@ -522,14 +526,82 @@ __global__ void __launch_bounds__(kDecThreads) idx_decode_score_kernel(DecArgs a
         if (sh[e]) atomicAdd(gh + e, sh[e]);
 }
 
+// Per row (one warp): the 12-bit bucket B that holds the topk-th largest key
+// (from the top of the histogram), how many keys to take from it, and its size.
+__global__ void __launch_bounds__(256) idx_decode_bucket_kernel(DecArgs a) {
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= a.n_rows) return;
+    const uint32_t *gh = a.hist + (size_t)row * kDecBins;
+    constexpr int per = kDecBins / 32;             // bins per lane, top-down
+    int cnt = 0;
+    for (int u = 0; u < per; ++u) cnt += (int)gh[kDecBins - 1 - (lane * per + u)];
+    int incl = cnt;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o2);
+        if (lane >= o2) incl += t;
+    }
+    const int before = incl - cnt, topk = a.topk;
+    if (lane == 0) a.eq_cnt[row] = 0;
+    if (lane == 31 && incl < topk) a.info[row] = make_int4(-1, 0, 0, 0);   // every key is taken
+    if (before < topk && topk <= incl) {
+        int acc = before;
+        for (int u = 0; u < per; ++u) {
+            const int bin = kDecBins - 1 - (lane * per + u);
+            const int c = (int)gh[bin];
+            if (acc < topk && topk <= acc + c) a.info[row] = make_int4(bin, topk - acc, c, 0);
+            acc += c;
+        }
+    }
+}
+
+// grid (8192-key part, row): one warp per 32 keys writes the bitmap words of
+// "bucket above B" (ballot) and clears the tie words; keys of bucket B go to
+// the row's (key, position) list when it fits.
+constexpr int kDecMarkKeys = 8192;
+__global__ void __launch_bounds__(256) idx_decode_mark_kernel(DecArgs a) {
+    const int row = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t kb = a.k_off[row];
+    const int nv = min((int)(a.k_off[row + 1] - kb), a.max_words * 32);
+    if (nv <= a.topk) return;
+    const int4 inf = a.info[row];
+    const uint32_t B = (uint32_t)inf.x;
+    const bool collect = inf.z <= kDecEqCap;
+    const uint32_t *keys = a.keys + (size_t)row * a.max_words * 32;
+    const int w0 = blockIdx.x * (kDecMarkKeys / 32), w1 = min((nv + 31) / 32, w0 + kDecMarkKeys / 32);
+    uint32_t *gt = a.bm_gt + (size_t)row * a.max_words;
+    uint32_t *eqm = a.bm_eq + (size_t)row * a.max_words;
+    for (int w = w0 + warp; w < w1; w += 8) {
+        const int i = w * 32 + lane;
+        const uint32_t kk = i < nv ? keys[i] : 0u;
+        const bool in = i < nv;
+        const unsigned g = __ballot_sync(0xffffffffu, in && (kk >> 20) > B);
+        const unsigned e = __ballot_sync(0xffffffffu, in && (kk >> 20) == B);
+        if (lane == 0) {
+            gt[w] = g;
+            eqm[w] = 0u;
+        }
+        if (collect && e) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(a.eq_cnt + row, __popc(e));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if ((e >> lane) & 1u) {
+                const int slot = base + __popc(e & ((1u << lane) - 1u));
+                if (slot < kDecEqCap) a.eq_buf[(size_t)row * kDecEqCap + slot] = make_uint2(kk, (uint32_t)i);
+            }
+        }
+    }
+}
+
+// Per row: exact threshold inside bucket B, ties marked, then one ordered sweep
+// over the position bitmaps writes the ascending index list (ties smallest
+// position first).  A bucket too large for the list selects over the whole row.
 __global__ void __launch_bounds__(kSelThreads) idx_decode_select_kernel(DecArgs a) {
     __shared__ SelScratch sc;
-    extern __shared__ uint32_t eqk[];         // [kDecEqCap]
-    __shared__ int bc[4];
     const int row = blockIdx.x;
     const int64_t kb = a.k_off[row];
     int nv = (int)(a.k_off[row + 1] - kb);
-    nv = min(max(nv, 0), a.max_tiles * kDecTile);
+    nv = min(max(nv, 0), a.max_words * 32);
     const int topk = a.topk;
     int32_t *o = a.out_idx + (size_t)row * topk;
     if (nv <= topk) {
@@ -537,56 +609,54 @@ __global__ void __launch_bounds__(kSelThreads) idx_decode_select_kernel(DecArgs 
         if (threadIdx.x == 0) a.out_cnt[row] = nv;
         return;
     }
-    const uint32_t *keys = a.keys + kb;
-    const uint32_t *gh = a.hist + (size_t)row * kDecBins;
-    // 1. the 12-bit bucket B holding the topk-th largest key (scan from the top)
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        constexpr int per = kDecBins / 32;             // bins per lane, top-down
-        int cnt = 0;
-        for (int u = 0; u < per; ++u) cnt += (int)gh[kDecBins - 1 - (lane * per + u)];
-        int incl = cnt;
-#pragma unroll
-        for (int o2 = 1; o2 < 32; o2 <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o2);
-            if (lane >= o2) incl += t;
-        }
-        const int before = incl - cnt;
-        if (before < topk && topk <= incl) {
-            int acc = before;
-            for (int u = 0; u < per; ++u) {
-                const int bin = kDecBins - 1 - (lane * per + u);
-                const int c = (int)gh[bin];
-                if (acc < topk && topk <= acc + c) {
-                    bc[0] = bin;
-                    bc[1] = topk - acc;                 // to take from bucket B
-                    bc[2] = c;                          // size of bucket B
-                }
-                acc += c;
-            }
-        }
+    const uint32_t *keys = a.keys + (size_t)row * a.max_words * 32;
+    const int4 inf = a.info[row];
+    int need_eq;
+    if (inf.z > kDecEqCap) {
+        // a very populated bucket (e.g. many exactly-equal scores): select over the whole row
+        const uint32_t T = block_radix_select([&](int i) { return keys[i]; }, nv, topk, sc, need_eq);
+        const int cnt = block_compact([&](int i) { return keys[i]; }, nv, T, need_eq, false, sc,
+                                      [&](int pos, int i, uint32_t) { o[pos] = i; });
+        for (int i = cnt + threadIdx.x; i < topk; i += kSelThreads) o[i] = -1;
+        if (threadIdx.x == 0) a.out_cnt[row] = cnt;
+        return;
+    }
+    // 1. exact threshold among bucket B's keys, then mark them
+    const uint2 *eb = a.eq_buf + (size_t)row * kDecEqCap;
+    const int size_b = min(a.eq_cnt[row], kDecEqCap);
+    const uint32_t T = block_radix_select([&](int i) { return eb[i].x; }, size_b, inf.y, sc, need_eq);
+    uint32_t *gt = a.bm_gt + (size_t)row * a.max_words;
+    uint32_t *eqm = a.bm_eq + (size_t)row * a.max_words;
+    for (int i = threadIdx.x; i < size_b; i += kSelThreads) {
+        const uint2 v = eb[i];
+        if (v.x > T) atomicOr(gt + (v.y >> 5), 1u << (v.y & 31));
+        else if (v.x == T) atomicOr(eqm + (v.y >> 5), 1u << (v.y & 31));
     }
     __syncthreads();
-    const uint32_t B = (uint32_t)bc[0];
-    const int need_b = bc[1], size_b = bc[2];
-    uint32_t T;
-    int need_eq;
-    if (size_b <= kDecEqCap) {
-        // 2. gather bucket B's keys (index order) and resolve them exactly
-        auto inb = [&](int i) { return (keys[i] >> 20) == B; };
-        block_compact([&](int i) { return inb(i) ? 1u : 0u; }, nv, 0u, 0, false, sc,
-                      [&](int pos, int i, uint32_t) { eqk[pos] = keys[i]; });
-        __syncthreads();
-        T = block_radix_select([&](int i) { return eqk[i]; }, size_b, need_b, sc, need_eq);
-    } else {
-        // a very populated bucket (e.g. many exactly-equal scores): select over the whole row
-        T = block_radix_select([&](int i) { return keys[i]; }, nv, topk, sc, need_eq);
+    // 2. ordered sweep: thread t owns a contiguous run of words
+    const int nwords = (nv + 31) / 32;
+    const int per = (nwords + kSelThreads - 1) / kSelThreads;
+    const int wa = min(nwords, threadIdx.x * per), wz = min(nwords, wa + per);
+    int gtc = 0, eqc = 0;
+    for (int w = wa; w < wz; ++w) {
+        gtc += __popc(gt[w]);
+        eqc += __popc(eqm[w]);
     }
-    // 3. ordered compaction over the row
-    const int cnt = block_compact([&](int i) { return keys[i]; }, nv, T, need_eq, false, sc,
-                                  [&](int pos, int i, uint32_t) { o[pos] = i; });
-    for (int i = cnt + threadIdx.x; i < topk; i += kSelThreads) o[i] = -1;
-    if (threadIdx.x == 0) a.out_cnt[row] = cnt;
+    int tot;
+    const int eq_before = block_excl_scan(eqc, sc.warp, tot);
+    int allow = min(max(need_eq - eq_before, 0), eqc);   // ties this thread may take
+    const int out0 = block_excl_scan(gtc + allow, sc.warp, tot);
+    int pos = out0;
+    for (int w = wa; w < wz; ++w) {
+        uint32_t e = eqm[w];
+        const int pe = __popc(e);
+        if (pe > allow)
+            for (int r = pe - allow; r > 0; --r) e &= ~(0x80000000u >> __clz(e));   // keep the lowest
+        allow -= __popc(e);
+        for (uint32_t m = gt[w] | e; m; m &= m - 1u) o[pos++] = w * 32 + (__ffs(m) - 1);
+    }
+    for (int i = tot + threadIdx.x; i < topk; i += kSelThreads) o[i] = -1;
+    if (threadIdx.x == 0) a.out_cnt[row] = tot;
 }
 
 static int idx_validate(const crs_indexer_params *p) {
@@ -623,18 +693,27 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
                              cudaStream_t s);
 }  // namespace crs
 
-static size_t dec_ws_parts(const crs_indexer_params *p, size_t &keys_bytes) {
+struct DecWs {
+    size_t keys, hist, bm, eq_buf, eq_cnt, info, total;   // byte offsets
+};
+static DecWs dec_ws_layout(const crs_indexer_params *p) {
     auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-    keys_bytes = al((size_t)p->n_rows * (size_t)max(p->max_keys, 1) * 4);
-    return keys_bytes + al((size_t)p->n_rows * kDecBins * 4);
+    const size_t rows = (size_t)p->n_rows;
+    const size_t words = (size_t)ceil_div(max(p->max_keys, 1), 32);
+    DecWs w;
+    w.keys = 0;
+    w.hist = w.keys + al(rows * words * 32 * 4);   // score keys, fixed stride per row
+    w.bm = w.hist + al(rows * kDecBins * 4);
+    w.eq_buf = w.bm + al(rows * words * 4 * 2);
+    w.eq_cnt = w.eq_buf + al(rows * kDecEqCap * 8);
+    w.info = w.eq_cnt + al(rows * 4);
+    w.total = w.info + al(rows * 16);
+    return w;
 }
 
 extern "C" size_t crs_indexer_topk_workspace_size(const crs_indexer_params *p) {
     if (idx_validate(p)) return 0;
-    if (p->mode == CRS_IDX_DECODE) {
-        size_t kbytes;
-        return dec_ws_parts(p, kbytes);
-    }
+    if (p->mode == CRS_IDX_DECODE) return dec_ws_layout(p).total;
     if (prefill_tc_applicable(p)) return prefill_tc_workspace(p);
     int max_slices, ws_rows;
     idx_geometry(p, max_slices, ws_rows);
@@ -655,15 +734,21 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
     if (need > 0 && (!ws || ws_bytes < need)) return CRS_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p->mode == CRS_IDX_DECODE) {
-        size_t kbytes;
-        dec_ws_parts(p, kbytes);
+        const DecWs L = dec_ws_layout(p);
+        char *wb = static_cast<char *>(ws);
         DecArgs d;
         d.q = static_cast<const __nv_bfloat16 *>(q_idx);
         d.w = w;
         d.k = static_cast<const __nv_bfloat16 *>(k_idx);
         d.k_off = k_offsets;
-        d.keys = static_cast<uint32_t *>(ws);
-        d.hist = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kbytes);
+        d.keys = reinterpret_cast<uint32_t *>(wb + L.keys);
+        d.hist = reinterpret_cast<uint32_t *>(wb + L.hist);
+        d.max_words = ceil_div(max(p->max_keys, 1), 32);
+        d.bm_gt = reinterpret_cast<uint32_t *>(wb + L.bm);
+        d.bm_eq = d.bm_gt + (size_t)p->n_rows * d.max_words;
+        d.eq_buf = reinterpret_cast<uint2 *>(wb + L.eq_buf);
+        d.eq_cnt = reinterpret_cast<int *>(wb + L.eq_cnt);
+        d.info = reinterpret_cast<int4 *>(wb + L.info);
         d.out_idx = out_idx;
         d.out_cnt = out_count;
         d.n_rows = p->n_rows;
@@ -676,12 +761,19 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
             idx_decode_score_kernel<<<dim3(d.max_tiles, p->n_rows), kDecThreads, 0, s>>>(d);
         }
         CRS_CHECK_LAUNCH();
-        CRS_TRY_CUDA(cudaFuncSetAttribute(idx_decode_select_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          kDecEqCap * 4));
         {
             ProfScope _ps(K_IDX_SELECT, s);
-            idx_decode_select_kernel<<<p->n_rows, kSelThreads, kDecEqCap * 4, s>>>(d);
+            idx_decode_bucket_kernel<<<ceil_div(p->n_rows, 8), 256, 0, s>>>(d);
+        }
+        CRS_CHECK_LAUNCH();
+        {
+            ProfScope _ps(K_IDX_SELECT, s);
+            idx_decode_mark_kernel<<<dim3(ceil_div(d.max_tiles * kDecTile, kDecMarkKeys), p->n_rows), 256, 0, s>>>(d);
+        }
+        CRS_CHECK_LAUNCH();
+        {
+            ProfScope _ps(K_IDX_SELECT, s);
+            idx_decode_select_kernel<<<p->n_rows, kSelThreads, 0, s>>>(d);
         }
         CRS_CHECK_LAUNCH();
         return CRS_OK;
