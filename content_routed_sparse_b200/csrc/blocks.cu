@@ -364,142 +364,116 @@ block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restr
 // ---------------------------------------------------------------------------
 // K9b: group softmax sum, top blocks, token list.  One CTA per (seq, KV head).
 // ---------------------------------------------------------------------------
-constexpr int kSelT = 512;
+constexpr int kPickT = 256;
 
-__device__ float block_reduce_max(float v, float *sh) {
-    v = warp_max(v);
-    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float r = -INFINITY;
-    for (int w = 0; w < kSelT / 32; ++w) r = fmaxf(r, sh[w]);
-    __syncthreads();
-    return r;
-}
-__device__ float block_reduce_sum(float v, float *sh) {
-    v = warp_sum(v);
-    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float r = 0.0f;
-    for (int w = 0; w < kSelT / 32; ++w) r += sh[w];
-    __syncthreads();
-    return r;
-}
-
-__global__ void __launch_bounds__(kSelT)
+// One CTA per (sequence, KV head).  Warp g takes query heads g, g + 8, ...:
+// the head's softmax over blocks (max and sum by shuffles) goes to its own
+// shared row, so the group sum is formed in a fixed order; warp 0 then selects
+// the top blocks exactly (4 radix passes over order-preserving keys, no block
+// barriers) and lists them in block order (ties: smaller block first).
+__global__ void __launch_bounds__(kPickT)
 block_pick_kernel(const float *__restrict__ sc, int32_t *__restrict__ tok, int32_t *__restrict__ cnt,
                   int G, int n_full, int L, int T, int top, int window, int cap) {
     extern __shared__ __align__(16) unsigned char bp_smem[];
-    float *score = reinterpret_cast<float *>(bp_smem);                 // [n_full]
-    uint32_t *keyv = reinterpret_cast<uint32_t *>(score + n_full);      // [n_full]
-    int *sel = reinterpret_cast<int *>(keyv + n_full);                  // [top]
-    __shared__ float red[kSelT / 32];
-    __shared__ int hist[256];
+    float *prob = reinterpret_cast<float *>(bp_smem);                  // [G][n_full]
+    uint32_t *keyv = reinterpret_cast<uint32_t *>(prob + (size_t)G * n_full);   // [n_full]
+    int *sel = reinterpret_cast<int *>(keyv + n_full);                  // [top] kept blocks
+    int *tstart = sel + top;                                            // [top] output offsets
+    __shared__ uint32_t hist[256];
     __shared__ int bc[2];
-    __shared__ int scan_sh[kSelT / 32 + 1];
     const int sh = blockIdx.x;
-    for (int b = threadIdx.x; b < n_full; b += kSelT) score[b] = 0.0f;
-    __syncthreads();
-    for (int g = 0; g < G; ++g) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int g = warp; g < G; g += kPickT / 32) {
         const float *s = sc + ((size_t)sh * G + g) * n_full;
+        float *pr = prob + (size_t)g * n_full;
         float m = -INFINITY;
-        for (int b = threadIdx.x; b < n_full; b += kSelT) m = fmaxf(m, s[b]);
-        m = block_reduce_max(m, red);
+        for (int b = lane; b < n_full; b += 32) m = fmaxf(m, s[b]);
+        m = warp_max(m);
         float z = 0.0f;
-        for (int b = threadIdx.x; b < n_full; b += kSelT) z += __expf(s[b] - m);
-        z = block_reduce_sum(z, red);
+        for (int b = lane; b < n_full; b += 32) {
+            const float e = __expf(s[b] - m);
+            pr[b] = e;
+            z += e;
+        }
+        z = warp_sum(z);
         const float iz = 1.0f / z;
-        for (int b = threadIdx.x; b < n_full; b += kSelT) score[b] += __expf(s[b] - m) * iz;
-        __syncthreads();
+        for (int b = lane; b < n_full; b += 32) pr[b] *= iz;
     }
-    for (int b = threadIdx.x; b < n_full; b += kSelT) keyv[b] = score_key(score[b]);
     __syncthreads();
-    // exact top `top` by (score desc, block asc): 4-pass radix select on the keys
-    const int k = min(top, n_full);
-    uint32_t prefix = 0, mask = 0;
-    int remaining = k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int b = threadIdx.x; b < 256; b += kSelT) hist[b] = 0;
-        __syncthreads();
-        for (int b = threadIdx.x; b < n_full; b += kSelT) {
-            const uint32_t kk = keyv[b];
-            if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int acc = 0;
-            for (int d = 255; d >= 0; --d) {
-                if (acc + hist[d] >= remaining) { bc[0] = d; bc[1] = remaining - acc; break; }
-                acc += hist[d];
+    for (int b = threadIdx.x; b < n_full; b += kPickT) {
+        float acc = 0.0f;
+        for (int g = 0; g < G; ++g) acc += prob[(size_t)g * n_full + b];
+        keyv[b] = score_key(acc);
+    }
+    __syncthreads();
+    const int wstart = max(0, T - window);
+    if (warp == 0) {
+        // exact top `top` by (score desc, block asc)
+        const int k = min(top, n_full);
+        uint32_t prefix = 0u, mask = 0u;
+        int need = k;
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0u;
+            __syncwarp();
+            for (int b = lane; b < n_full; b += 32) {
+                const uint32_t kk = keyv[b];
+                if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1u);
             }
+            __syncwarp();
+            const int bin = warp_top_bin(hist, need);
+            prefix |= (uint32_t)bin << shift;
+            mask |= 0xffu << shift;
+            __syncwarp();
         }
-        __syncthreads();
-        prefix |= (uint32_t)bc[0] << shift;
-        mask |= 0xffu << shift;
-        remaining = bc[1];
-        __syncthreads();
+        const uint32_t Tk = prefix;
+        // compaction in block order: block b = j * 32 + lane
+        int out = 0, eq_seen = 0, tok_pos = 0;
+        for (int j0 = 0; j0 < n_full; j0 += 32) {
+            const int b = j0 + lane;
+            const uint32_t kk = b < n_full ? keyv[b] : 0u;
+            const bool eq = b < n_full && kk == Tk;
+            const unsigned be = __ballot_sync(0xffffffffu, eq);
+            const bool take = (b < n_full && kk > Tk) ||
+                              (eq && eq_seen + __popc(be & ((1u << lane) - 1u)) < need);
+            const unsigned bt = __ballot_sync(0xffffffffu, take);
+            // tokens of block b that lie before the window
+            const int nt = take ? min(L, max(0, wstart - b * L)) : 0;
+            int incl = nt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += x;
+            }
+            if (take) {
+                const int slot = out + __popc(bt & ((1u << lane) - 1u));
+                sel[slot] = b;
+                tstart[slot] = tok_pos + incl - nt;
+            }
+            out += __popc(bt);
+            eq_seen += __popc(be);
+            tok_pos += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            bc[0] = out;
+            bc[1] = tok_pos;
+        }
     }
-    const uint32_t Tk = prefix;
-    // compaction in block order; equal keys: the first `remaining` blocks
-    int out_base = 0, eq_base = 0;
-    for (int t0 = 0; t0 < n_full; t0 += kSelT) {
-        const int b = t0 + threadIdx.x;
-        const uint32_t kk = (b < n_full) ? keyv[b] : 0u;
-        const bool gt = (b < n_full) && kk > Tk;
-        const bool eq = (b < n_full) && kk == Tk;
-        // exclusive scans via warp ballots
-        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-        const unsigned be = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) scan_sh[w] = __popc(be);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int s = 0;
-            for (int i = 0; i < kSelT / 32; ++i) { const int c = scan_sh[i]; scan_sh[i] = s; s += c; }
-            scan_sh[kSelT / 32] = s;
-        }
-        __syncthreads();
-        const int eq_rank = eq_base + scan_sh[w] + __popc(be & ((1u << lane) - 1u));
-        const int eq_tot = scan_sh[kSelT / 32];
-        __syncthreads();
-        const bool take = gt || (eq && eq_rank < remaining);
-        const unsigned bt = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) scan_sh[w] = __popc(bt);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int s = 0;
-            for (int i = 0; i < kSelT / 32; ++i) { const int c = scan_sh[i]; scan_sh[i] = s; s += c; }
-            scan_sh[kSelT / 32] = s;
-        }
-        __syncthreads();
-        if (take) sel[out_base + scan_sh[w] + __popc(bt & ((1u << lane) - 1u))] = b;
-        out_base += scan_sh[kSelT / 32];
-        eq_base += eq_tot;
-        __syncthreads();
-    }
+    __syncthreads();
     // token list: kept blocks' positions before the window (blocks ascending),
     // then the window [wstart, T)
-    int *tstart = sel + top;                 // [top] first output slot of each kept block
-    const int wstart = max(0, T - window);
+    const int n_sel = bc[0], nblk_tok = bc[1];
     int32_t *to = tok + (size_t)sh * cap;
-    if (threadIdx.x == 0) {
-        int pos = 0;
-        for (int i = 0; i < out_base; ++i) {
-            tstart[i] = pos;
-            pos += min(L, max(0, wstart - sel[i] * L));
-        }
-        bc[0] = pos;
-    }
-    __syncthreads();
-    const int nblk_tok = bc[0];
-    for (int e = threadIdx.x; e < out_base * L; e += kSelT) {
+    for (int e = threadIdx.x; e < n_sel * L; e += kPickT) {
         const int i = e / L, r = e - i * L;
         const int b = sel[i];
         if (b * L + r < wstart) to[tstart[i] + r] = b * L + r;
     }
     const int nwin = T - wstart;
-    for (int i = threadIdx.x; i < nwin; i += kSelT) to[nblk_tok + i] = wstart + i;
+    for (int i = threadIdx.x; i < nwin; i += kPickT) to[nblk_tok + i] = wstart + i;
     const int total = nblk_tok + nwin;
-    for (int i = total + threadIdx.x; i < cap; i += kSelT) to[i] = -1;
+    for (int i = total + threadIdx.x; i < cap; i += kPickT) to[i] = -1;
     if (threadIdx.x == 0) cnt[sh] = total;
 }
 
@@ -603,12 +577,13 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
     }
     CRS_CHECK_LAUNCH();
     const int cap = p->top_blocks * p->b.L + p->window;
-    const size_t smem_b = (size_t)n_full * 8 + (size_t)p->top_blocks * 8;
+    const size_t smem_b = ((size_t)G + 1) * n_full * 4 + (size_t)p->top_blocks * 8;
+    if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
     CRS_TRY_CUDA(cudaFuncSetAttribute(block_pick_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b));
     {
         ProfScope _ps(K_BLK_PICK, s);
-        block_pick_kernel<<<p->b.n_seq * p->b.n_kv, kSelT, smem_b, s>>>(
+        block_pick_kernel<<<p->b.n_seq * p->b.n_kv, kPickT, smem_b, s>>>(
             sc, tok_idx, tok_count, G, n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
     }
     CRS_CHECK_LAUNCH();
