@@ -7,9 +7,13 @@
 // round; rounds merge by log-sum-exp weights).
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include <type_traits>
 
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace crs {
 
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(kHashTok) lsh_hash_bf16x2_kernel(const __nv_bf
 }
 
 // --------------------------------------------------------------------------
-// K2: stable counting sort of one (b, h, round) segment per CTA.
+// K2: stable counting sort of one (b, h, round) segment per 8-CTA cluster.
 // Histogram -> exclusive scan (bucket bases) -> tiles of blockDim positions
 // in increasing order; inside a tile, the rank of a position among equal
 // buckets comes from __match_any_sync within the warp plus the counts of
@@ -218,47 +222,75 @@ __global__ void __launch_bounds__(kHashTok) lsh_hash_bf16x2_kernel(const __nv_bf
 // --------------------------------------------------------------------------
 constexpr int kSortThreads = 512;
 
-__global__ void __launch_bounds__(kSortThreads) lsh_sort_kernel(const int32_t *__restrict__ bucket,
-                                                                 int32_t *__restrict__ perm,
-                                                                 int32_t *__restrict__ inv_perm,
-                                                                 int n, int nb) {
-    extern __shared__ int smi[];
+// The 8 CTAs of a cluster split one segment into 8
+// contiguous position ranges.  Each counts its range's buckets in shared
+// memory; after a cluster barrier every CTA reads the other CTAs' counts
+// through distributed shared memory, so the slot of the first position of
+// bucket b in range p is (positions in buckets < b) + (positions of bucket b
+// in ranges < p).  No global scratch is needed.
+constexpr int kSortCluster = 8;
+
+__global__ void __cluster_dims__(kSortCluster, 1, 1) __launch_bounds__(kSortThreads)
+lsh_sort_cluster_kernel(const int32_t *__restrict__ bucket, int32_t *__restrict__ perm,
+                        int32_t *__restrict__ inv_perm, int n, int nb) {
+    extern __shared__ int smc[];
     constexpr int NW = kSortThreads / 32;
-    int *base = smi;              // [nb]
-    int *running = base + nb;     // [nb]
-    int *wcnt = running + nb;     // [NW][nb]
+    int *hist = smc;               // [nb] counts of this range (read by the cluster)
+    int *base = hist + nb;         // [nb]
+    int *running = base + nb;      // [nb]
+    int *wcnt = running + nb;      // [NW][nb]
+    __shared__ int scan_w[NW + 1];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int part = (int)cluster.block_rank();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const size_t seg = blockIdx.x;
+    const size_t seg = blockIdx.y;
+    const int len = (n + kSortCluster - 1) / kSortCluster;
+    const int p0 = min(n, part * len), p1 = min(n, p0 + len);
     const int32_t *bk = bucket + seg * n;
     int32_t *pm = perm + seg * n;
     int32_t *ip = inv_perm + seg * n;
-    for (int e = tid; e < nb; e += kSortThreads) { base[e] = 0; running[e] = 0; }
+    for (int e = tid; e < nb; e += kSortThreads) { hist[e] = 0; running[e] = 0; }
     for (int e = tid; e < NW * nb; e += kSortThreads) wcnt[e] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kSortThreads) {
+    for (int i = p0 + tid; i < p1; i += kSortThreads) {
         const int b = bk[i];
-        if (b >= 0 && b < nb) atomicAdd(&base[b], 1);
+        if (b >= 0 && b < nb) atomicAdd(&hist[b], 1);
         else raise_error(CRS_DEVERR_INDEX);
     }
-    __syncthreads();
-    if (warp == 0) {
-        const int per = (nb + 31) / 32, b0 = lane * per, b1 = min(b0 + per, nb);
-        int s = 0;
-        for (int b = b0; b < b1; ++b) s += base[b];
-        int incl = s;
+    cluster.sync();
+    // base[b] = sum over ranges of buckets < b, plus bucket b in earlier ranges
+    for (int b0 = 0; b0 < nb; b0 += kSortThreads) {
+        const int b = b0 + tid;
+        int tot = 0, before = 0;
+        if (b < nb) {
+            for (int q = 0; q < kSortCluster; ++q) {
+                const int c = *cluster.map_shared_rank(hist + b, q);
+                tot += c;
+                if (q < part) before += c;
+            }
+        }
+        int incl = tot;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        int excl = incl - s;
-        for (int b = b0; b < b1; ++b) { const int c = base[b]; base[b] = excl; excl += c; }
+        if (lane == 31) scan_w[warp] = incl;
+        __syncthreads();
+        if (tid == 0) {
+            int acc = b0 == 0 ? 0 : scan_w[NW];
+            for (int w = 0; w < NW; ++w) { const int c = scan_w[w]; scan_w[w] = acc; acc += c; }
+            scan_w[NW] = acc;
+        }
+        __syncthreads();
+        if (b < nb) base[b] = scan_w[warp] + incl - tot + before;
+        __syncthreads();
     }
-    __syncthreads();
+    cluster.sync();                // every CTA has read the counts it needs
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int t0 = 0; t0 < n; t0 += kSortThreads) {
+    for (int t0 = p0; t0 < p1; t0 += kSortThreads) {
         const int i = t0 + tid;
-        int b = (i < n) ? bk[i] : -1;
+        int b = (i < p1) ? bk[i] : -1;
         if (b >= nb) b = -1;
         const bool valid = b >= 0;
         const unsigned active = __ballot_sync(0xffffffffu, valid);
@@ -563,13 +595,14 @@ extern "C" int crs_lsh_route(const crs_lsh_params *p, const void *X, const float
         }
     }
     CRS_CHECK_LAUNCH();
-    const size_t ssm = (size_t)(2 + kSortThreads / 32) * p->n_buckets * sizeof(int);
-    CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)ssm));
+    const size_t ssm = (size_t)(3 + kSortThreads / 32) * p->n_buckets * sizeof(int);
+    if (ssm > 200 * 1024) return CRS_ERR_UNSUPPORTED;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_sort_cluster_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm));
     {
         ProfScope _ps(K_LSH_SORT, s);
-        lsh_sort_kernel<<<p->B * p->H * p->n_rounds, kSortThreads, ssm, s>>>(bucket, perm, inv_perm,
-                                                                             p->n, p->n_buckets);
+        lsh_sort_cluster_kernel<<<dim3(kSortCluster, p->B * p->H * p->n_rounds), kSortThreads, ssm, s>>>(
+            bucket, perm, inv_perm, p->n, p->n_buckets);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;
