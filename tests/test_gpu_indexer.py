@@ -171,6 +171,28 @@ def test_prefill_full_config_sampled(crs, cuda_dev):
                 "prefill-full")
 
 
+def test_decode_all_tied_row_selects_whole_row(crs, cuda_dev):
+    """Every cached index key equal: one histogram bucket holds the whole row (more than the
+    bucket list holds), so the select runs over the whole row; ties go to the smallest
+    positions.  A second, ordinary row shares the launch."""
+    g = torch.Generator(device=cuda_dev).manual_seed(21)
+    lens = [40000, 9000]
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    k_idx = torch.randn(int(off[-1]), 64, generator=g, device=cuda_dev).to(torch.bfloat16)
+    k_idx[:lens[0]] = k_idx[0]
+    q_idx = torch.randn(2, 4, 64, generator=g, device=cuda_dev).to(torch.bfloat16)
+    w = torch.randn(2, 4, generator=g, device=cuda_dev)
+    topk = 1024
+    idx, cnt = crs.indexer_topk(q_idx, w, k_idx, topk, crs.CRS_IDX_DECODE,
+                                k_offsets=torch.from_numpy(off).to(cuda_dev), max_keys=max(lens))
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    assert g_cnt[0] == topk and (g_idx[0] == np.arange(topk)).all()
+    _check_rows(g_idx, g_cnt, _np(q_idx), _np(w), _np(k_idx), off[:-1], np.array(lens, np.int32),
+                np.array([1]), topk, "decode-tied")
+
+
 def test_nan_score_flags_device_error(crs, cuda_dev):
     q = torch.randn(1, 4, 64, device=cuda_dev).to(torch.bfloat16)
     w = torch.randn(1, 4, device=cuda_dev)
