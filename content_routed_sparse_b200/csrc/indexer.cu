@@ -534,7 +534,15 @@ __global__ void __launch_bounds__(256) idx_decode_bucket_kernel(DecArgs a) {
     const uint32_t *gh = a.hist + (size_t)row * kDecBins;
     constexpr int per = kDecBins / 32;             // bins per lane, top-down
     int cnt = 0;
-    for (int u = 0; u < per; ++u) cnt += (int)gh[kDecBins - 1 - (lane * per + u)];
+    {
+        // lane l owns bins [kDecBins - per (l + 1), kDecBins - per l): 16-byte loads, all in flight
+        const uint4 *g4 = reinterpret_cast<const uint4 *>(gh + kDecBins - per * (lane + 1));
+        uint4 v[per / 4];
+#pragma unroll
+        for (int u = 0; u < per / 4; ++u) v[u] = g4[u];
+#pragma unroll
+        for (int u = 0; u < per / 4; ++u) cnt += (int)(v[u].x + v[u].y + v[u].z + v[u].w);
+    }
     int incl = cnt;
 #pragma unroll
     for (int o2 = 1; o2 < 32; o2 <<= 1) {
@@ -571,9 +579,20 @@ __global__ void __launch_bounds__(256) idx_decode_mark_kernel(DecArgs a) {
     const int w0 = blockIdx.x * (kDecMarkKeys / 32), w1 = min((nv + 31) / 32, w0 + kDecMarkKeys / 32);
     uint32_t *gt = a.bm_gt + (size_t)row * a.max_words;
     uint32_t *eqm = a.bm_eq + (size_t)row * a.max_words;
-    for (int w = w0 + warp; w < w1; w += 8) {
+    for (int wb = w0 + warp * 4; wb < w1; wb += 32) {
+        // four words per warp and iteration: four 128-byte loads in flight
+        uint32_t kv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = (wb + u) * 32 + lane;
+            kv[u] = (wb + u < w1 && i < nv) ? keys[i] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+        const int w = wb + u;
+        if (w >= w1) break;
         const int i = w * 32 + lane;
-        const uint32_t kk = i < nv ? keys[i] : 0u;
+        const uint32_t kk = kv[u];
         const bool in = i < nv;
         const unsigned g = __ballot_sync(0xffffffffu, in && (kk >> 20) > B);
         const unsigned e = __ballot_sync(0xffffffffu, in && (kk >> 20) == B);
@@ -589,6 +608,7 @@ __global__ void __launch_bounds__(256) idx_decode_mark_kernel(DecArgs a) {
                 const int slot = base + __popc(e & ((1u << lane) - 1u));
                 if (slot < kDecEqCap) a.eq_buf[(size_t)row * kDecEqCap + slot] = make_uint2(kk, (uint32_t)i);
             }
+        }
         }
     }
 }
