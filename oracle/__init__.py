@@ -50,6 +50,8 @@ def _lib():
         lib.oracle_block_describe.argtypes = [I, I, I, I, _f64p, _i32p, _f64p, _f64p, _f64p]
         lib.oracle_block_log_mass.argtypes = [I, I, _f64p, _f64p]
         lib.oracle_block_log_mass.restype = D
+        lib.oracle_fp4_quantize.argtypes = [I, I, _f32p, _u8p, _f32p]
+        lib.oracle_fp4_dequantize.argtypes = [I, I, _u8p, _f32p, _f64p]
         lib.oracle_block_select.argtypes = [I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
                                             I, _i32p, _i32p, _i32p, _f64p]
         lib.oracle_sparse_attn.argtypes = [I, I, I, I, D, _f64p, _f64p, _f64p, _i64p, _i32p, I, I,
@@ -234,6 +236,29 @@ def block_select(Q, mu, xi, T, L, top_blocks, window, scale=None):
                                float(scale), _p(Q, _f64p), _p(mu, _f64p), _p(xi, _f64p), cap,
                                _p(tok, _i32p), _p(cnt, _i32p), _p(blk, _i32p), _p(bs, _f64p))
     return tok, cnt, blk, bs
+
+
+def fp4_quantize(xi):
+    """xi [..., D] float32 -> (codes [..., D/2] uint8, scale [...] float32): E2M1 with one
+    fp32 absmax/6 scale per vector ([P5] §5.5; rounding reading in crs_oracle.c)."""
+    x = _c(xi, np.float32)
+    D = x.shape[-1]
+    n = x.size // D
+    codes = np.empty(x.shape[:-1] + (D // 2,), dtype=np.uint8)
+    scale = np.empty(x.shape[:-1], dtype=np.float32)
+    _lib().oracle_fp4_quantize(n, D, _p(x, _f32p), _p(codes, _u8p), _p(scale, _f32p))
+    return codes, scale
+
+
+def fp4_dequantize(codes, scale):
+    """Inverse map of fp4_quantize's codes: sign * E2M1 value * scale, fp64."""
+    c = _c(codes, np.uint8)
+    s = _c(scale, np.float32)
+    D = c.shape[-1] * 2
+    n = c.size // (D // 2)
+    out = np.empty(c.shape[:-1] + (D,), dtype=np.float64)
+    _lib().oracle_fp4_dequantize(n, D, _p(c, _u8p), _p(s, _f32p), _p(out, _f64p))
+    return out
 
 
 # ---------------------------------------------------------- attention --

@@ -640,3 +640,66 @@ OAPI void oracle_sparse_attn(int n_rows, int n_q, int n_kv, int D, double scale,
         free(logit);
     }
 }
+
+/* ======================================================================
+ * f1  Deployed descriptor compression.  [P5] §5.5 "量化：对存储的特征向量做
+ * FP4": each scaled eigenvector xi_i is stored in E2M1 FP4 (2 exponent bits,
+ * 1 mantissa bit) with one fp32 scale per vector; the block mean is stored
+ * in bf16 (Algorithm 2 steps 7-8).  The page fixes the format but not the
+ * scale rule or the rounding; the reading taken here: scale = max_d |xi_d| / 6
+ * (6 is the largest E2M1 magnitude), each element x / scale rounded to the
+ * nearest E2M1 value {0, 0.5, 1, 1.5, 2, 3, 4, 6}, a tie going to the value
+ * with a zero mantissa bit (the even code), a zero vector getting scale 0.
+ * The codes are integers decided by floating point, so the division and the
+ * comparisons are taken in fp32, the kernel's precision.
+ * Code: bit 3 = sign, bits 0-2 = magnitude index into the list above; two
+ * codes per byte, the even element in the low nibble.
+ * Layout: xi [n_vec, D] fp32 -> codes [n_vec, D/2] bytes, scale [n_vec].
+ * ====================================================================== */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+static int e2m1_index(float a)   /* a = |x / scale| in fp32 */
+{
+    int best = 0;
+    for (int i = 1; i < 8; ++i) {
+        const float d_new = fabsf(a - kE2M1[i]);
+        const float d_best = fabsf(a - kE2M1[best]);
+        /* strictly closer wins; an exact tie goes to the even index */
+        if (d_new < d_best || (d_new == d_best && (i & 1) == 0)) best = i;
+    }
+    return best;
+}
+
+OAPI void oracle_fp4_quantize(int n_vec, int D, const float *xi, uint8_t *codes, float *scale)
+{
+    for (int v = 0; v < n_vec; ++v) {
+        const float *x = xi + (size_t)v * D;
+        float amax = 0.0f;
+        for (int d = 0; d < D; ++d) amax = fmaxf(amax, fabsf(x[d]));
+        const float s = amax / 6.0f;
+        scale[v] = s;
+        for (int d = 0; d < D; d += 2) {
+            uint8_t c[2] = {0, 0};
+            for (int e = 0; e < 2; ++e) {
+                if (s > 0.0f) {
+                    const float y = x[d + e] / s;
+                    const int idx = e2m1_index(fabsf(y));
+                    c[e] = (uint8_t)(((y < 0.0f && idx != 0) ? 8 : 0) | idx);
+                }
+            }
+            codes[(size_t)v * (D / 2) + d / 2] = (uint8_t)(c[0] | (c[1] << 4));
+        }
+    }
+}
+
+OAPI void oracle_fp4_dequantize(int n_vec, int D, const uint8_t *codes, const float *scale,
+                                double *out)
+{
+    for (int v = 0; v < n_vec; ++v)
+        for (int d = 0; d < D; ++d) {
+            const uint8_t byte = codes[(size_t)v * (D / 2) + d / 2];
+            const int c = (d & 1) ? (byte >> 4) : (byte & 15);
+            const double mag = (double)kE2M1[c & 7] * (double)scale[v];
+            out[(size_t)v * D + d] = (c & 8) ? -mag : mag;
+        }
+}
