@@ -8,7 +8,7 @@ is missing; there is no fallback.
 
 Functions (same names as the C entry points, without the ``crs_`` prefix):
   lsh_route, lsh_attn, indexer_topk, block_describe, block_select,
-  sparse_attn, get_device_error.
+  block_quantize, block_select_fp4, sparse_attn, get_device_error.
 """
 from __future__ import annotations
 
@@ -112,6 +112,9 @@ _sig("crs_block_describe", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP,
 _sig("crs_block_select_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams)])
 _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                          _VP, _SZ, _VP])
+_sig("crs_block_quantize", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP, _VP, _VP])
+_sig("crs_block_select_fp4", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
+                                             _VP, _VP, _SZ, _VP])
 _sig("crs_block_select_noalloc", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP,
                                                  _VP, _VP, _VP])
 _sig("crs_sparse_attn_workspace_size", _SZ, [ctypes.POINTER(AttnParams)])
@@ -339,6 +342,55 @@ def block_select(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=
     st = _lib.crs_block_select(ctypes.byref(p), _ptr(Q), _ptr(mu), _ptr(xi), _ptr(tok),
                                _ptr(count), _ptr(ws), wsb, _stream(stream))
     _check("crs_block_select", st)
+    return tok, count
+
+
+def block_quantize(mu, xi, T: int, L: int, out=None, stream=None):
+    """Deployed descriptor compression: mu -> bf16, xi -> FP4 codes + fp32 scales.
+    Returns (mu16 [.., D] bf16, xi4 [.., rank, D/2] uint8, xi_scale [.., rank] fp32)."""
+    _need(mu, "mu", torch.float32)
+    n_seq, n_kv, nfull, D = mu.shape
+    rank = xi.shape[3]
+    _need(xi, "xi", torch.float32, (n_seq, n_kv, nfull, rank, D))
+    if out is None:
+        out = (torch.empty((n_seq, n_kv, nfull, D), dtype=torch.bfloat16, device=mu.device),
+               torch.empty((n_seq, n_kv, nfull, rank, D // 2), dtype=torch.uint8, device=mu.device),
+               torch.empty((n_seq, n_kv, nfull, rank), dtype=torch.float32, device=mu.device))
+    mu16, xi4, xs = out
+    _need(mu16, "mu16", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    _need(xi4, "xi4", torch.uint8, (n_seq, n_kv, nfull, rank, D // 2))
+    _need(xs, "xi_scale", torch.float32, (n_seq, n_kv, nfull, rank))
+    p = BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull)
+    _check("crs_block_quantize", _lib.crs_block_quantize(ctypes.byref(p), _ptr(mu), _ptr(xi), _ptr(mu16),
+                                                         _ptr(xi4), _ptr(xs), _stream(stream)))
+    return mu16, xi4, xs
+
+
+def block_select_fp4(Q, mu16, xi4, xi_scale, T: int, L: int, top_blocks: int, window: int,
+                     scale=None, tok=None, count=None, workspace=None, stream=None):
+    """block_select on compressed descriptors (from block_quantize)."""
+    _need(Q, "Q", torch.bfloat16)
+    n_seq, n_q, D = Q.shape
+    n_kv, nfull, rank = mu16.shape[1], mu16.shape[2], xi4.shape[3]
+    _need(mu16, "mu16", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    _need(xi4, "xi4", torch.uint8, (n_seq, n_kv, nfull, rank, D // 2))
+    _need(xi_scale, "xi_scale", torch.float32, (n_seq, n_kv, nfull, rank))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull), n_q,
+                       int(top_blocks), int(window), float(scale))
+    cap = top_blocks * L + window
+    if tok is None:
+        tok = torch.empty((n_seq, n_kv, cap), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((n_seq, n_kv), dtype=torch.int32, device=Q.device)
+    _need(tok, "tok", torch.int32, (n_seq, n_kv, cap))
+    _need(count, "count", torch.int32, (n_seq, n_kv))
+    ws, wsb = _workspace(int(_lib.crs_block_select_workspace_size(ctypes.byref(p))), Q.device,
+                         workspace)
+    st = _lib.crs_block_select_fp4(ctypes.byref(p), _ptr(Q), _ptr(mu16), _ptr(xi4), _ptr(xi_scale),
+                                   _ptr(tok), _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_block_select_fp4", st)
     return tok, count
 
 

@@ -304,7 +304,7 @@ block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restr
         ok = ok && tc::mbar_wait_bounded(&S.full[st], (c / kBsStages) & 1, kBsWaitNs, K_BLK_SCORE, 1);
         if (__syncthreads_or(!ok)) break;
         const int b = b_lo + c * kBsChunk + grp;
-        if (b < b_hi) {
+        {   // every lane computes (the group shuffles need all 32); invalid blocks only skip the store
             const float4 *m4 = reinterpret_cast<const float4 *>(&S.mu[st][grp][0]);
             const float4 *x4 = reinterpret_cast<const float4 *>(&S.xi[st][grp][0][0]);
             float lin[G], pr[G][R];
@@ -346,7 +346,7 @@ block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restr
                     for (int e = 0; e < R; ++e) pr[g][e] += __shfl_xor_sync(0xffffffffu, pr[g][e], off);
                 }
             }
-            if (sub == 0) {
+            if (sub == 0 && b < b_hi) {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     float quad = 0.0f;
@@ -477,6 +477,186 @@ block_pick_kernel(const float *__restrict__ sc, int32_t *__restrict__ tok, int32
     if (threadIdx.x == 0) cnt[sh] = total;
 }
 
+// ---------------------------------------------------------------------------
+// Deployed descriptor compression ([P5] §5.5): the block mean in bf16 and each
+// scaled eigenvector in E2M1 FP4 with one fp32 scale (absmax / 6).  One warp
+// per vector, four elements per lane; codes: bit 3 sign, bits 0-2 index into
+// {0, 0.5, 1, 1.5, 2, 3, 4, 6}, nearest value, ties to the zero-mantissa code
+// (decided in fp32 on the quotient x / scale).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1_code(float x, float s) {
+    if (!(s > 0.0f)) return 0u;
+    const float y = x / s;
+    const float a = fabsf(y);
+    const uint32_t idx = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                         (a >= 3.5f) + (a > 5.0f);
+    return ((y < 0.0f && idx != 0u) ? 8u : 0u) | idx;
+}
+
+// grid (vectors / 8, 1): warps 0..7 take vectors; vector v < n_mu is a mean
+// (bf16), the rest are scaled eigenvectors (FP4 + scale)
+__global__ void __launch_bounds__(256) block_quantize_kernel(const float *__restrict__ mu,
+                                                             const float *__restrict__ xi,
+                                                             __nv_bfloat16 *__restrict__ mu16,
+                                                             uint8_t *__restrict__ xi4,
+                                                             float *__restrict__ xi_scale,
+                                                             long long n_mu, long long n_xi) {
+    const long long v = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (v < n_mu) {
+        const float4 x = reinterpret_cast<const float4 *>(mu + v * kBdD)[lane];
+        __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t *>(&a);
+        o.y = *reinterpret_cast<uint32_t *>(&b);
+        reinterpret_cast<uint2 *>(mu16 + v * kBdD)[lane] = o;
+        return;
+    }
+    const long long w = v - n_mu;
+    if (w >= n_xi) return;
+    const float4 x = reinterpret_cast<const float4 *>(xi + w * kBdD)[lane];
+    const float amax = warp_max(fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+    const float sc = amax / 6.0f;
+    const uint32_t c = e2m1_code(x.x, sc) | (e2m1_code(x.y, sc) << 4) | (e2m1_code(x.z, sc) << 8) |
+                       (e2m1_code(x.w, sc) << 12);
+    reinterpret_cast<uint16_t *>(xi4 + w * (kBdD / 2))[lane] = (uint16_t)c;
+    if (lane == 0) xi_scale[w] = sc;
+}
+
+// E2M1 code (4 bits) -> float: index 0/1 -> 0/0.5, else (1 + m/2) 2^(e-1)
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const uint32_t mag = e ? (((126u + e) << 23) | (m << 22)) : (m ? 0x3f000000u : 0u);
+    return __uint_as_float(mag | ((c & 8u) << 28));
+}
+
+// K9a on compressed descriptors: the FP4 counterpart of block_score_tma_kernel.
+// A chunk of 16 blocks is 4 KB of bf16 means, 4 KB of FP4 codes and 256 B of
+// scales (three bulk copies); lane s of a block's 8-lane group covers dims
+// [8s, 8s + 8) and [64 + 8s, 64 + 8s + 8).  Projections are formed on the code
+// values and scaled once per vector.
+constexpr int kBqChunk = 16;
+template <int G, int R>
+struct BqSmem {
+    __nv_bfloat16 mu[kBsStages][kBqChunk][kBdD];
+    uint8_t xi[kBsStages][kBqChunk][R][kBdD / 2];
+    float scale[kBsStages][kBqChunk][R];
+    float sq[G][kBdD];
+    uint64_t full[kBsStages];
+};
+
+template <int G, int R>
+__global__ void __launch_bounds__(8 * kBqChunk)
+block_score_fp4_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ mu16,
+                       const uint8_t *__restrict__ xi4, const float *__restrict__ xi_scale,
+                       float *__restrict__ sc_out, int n_kv, int n_q, int n_full, int blocks_per_cta,
+                       float scale) {
+    extern __shared__ __align__(128) unsigned char bq_raw[];
+    BqSmem<G, R> &S = *reinterpret_cast<BqSmem<G, R> *>(bq_raw);
+    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
+    const int b_lo = blockIdx.x * blocks_per_cta;
+    const int b_hi = min(n_full, b_lo + blocks_per_cta);
+    if (b_lo >= b_hi) return;
+    const int n_chunks = ceil_div(b_hi - b_lo, kBqChunk);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t blk0 = (size_t)sh * n_full;
+    auto issue = [&](int c) {                      // one thread
+        const int st = c % kBsStages;
+        const size_t b0 = blk0 + b_lo + (size_t)c * kBqChunk;
+        const int nb = min(kBqChunk, b_hi - (b_lo + c * kBqChunk));
+        const uint32_t mb = (uint32_t)nb * kBdD * 2, xb = (uint32_t)nb * R * (kBdD / 2);
+        const uint32_t sb = (uint32_t)((nb * R * 4 + 15) & ~15);
+        tc::mbar_arrive_expect_tx(&S.full[st], mb + xb + sb);
+        tc::bulk_load(&S.mu[st][0][0], mu16 + b0 * kBdD, mb, &S.full[st]);
+        tc::bulk_load(&S.xi[st][0][0][0], xi4 + b0 * R * (kBdD / 2), xb, &S.full[st]);
+        tc::bulk_load(&S.scale[st][0][0], xi_scale + b0 * R, sb, &S.full[st]);
+    };
+    if (tid == 0) {
+        for (int st = 0; st < kBsStages; ++st) tc::mbar_init(&S.full[st], 1);
+        tc::mbar_fence_init();
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int c = 0; c < min(kBsStages, n_chunks); ++c) issue(c);
+    for (int e = tid; e < G * kBdD; e += blockDim.x) {
+        const int g = e / kBdD, d = e - g * kBdD;
+        S.sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+    }
+    __syncthreads();
+    const int sub = lane & 7, grp = warp * 4 + (lane >> 3);
+    bool ok = true;
+    for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % kBsStages;
+        ok = ok && tc::mbar_wait_bounded(&S.full[st], (c / kBsStages) & 1, kBsWaitNs, K_BLK_SCORE, 2);
+        if (__syncthreads_or(!ok)) break;
+        const int b = b_lo + c * kBqChunk + grp;
+        {   // every lane computes (the group shuffles need all 32); invalid blocks only skip the store
+            float lin[G], pr[G][R];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                lin[g] = 0.0f;
+#pragma unroll
+                for (int e = 0; e < R; ++e) pr[g][e] = 0.0f;
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int d0 = half * 64 + sub * 8;              // 8 dims of this lane
+                const uint4 mraw = *reinterpret_cast<const uint4 *>(&S.mu[st][grp][d0]);
+                const __nv_bfloat162 *m2 = reinterpret_cast<const __nv_bfloat162 *>(&mraw);
+                float mv[8];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = __bfloat1622float2(m2[t]);
+                    mv[2 * t] = f.x;
+                    mv[2 * t + 1] = f.y;
+                }
+                float cv[R][8];
+#pragma unroll
+                for (int e = 0; e < R; ++e) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(&S.xi[st][grp][e][d0 / 2]);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) cv[e][t] = e2m1_value((w >> (4 * t)) & 15u);
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float4 q0 = *reinterpret_cast<const float4 *>(&S.sq[g][d0]);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(&S.sq[g][d0 + 4]);
+                    const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        lin[g] = fmaf(qv[t], mv[t], lin[g]);
+#pragma unroll
+                        for (int e = 0; e < R; ++e) pr[g][e] = fmaf(qv[t], cv[e][t], pr[g][e]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    lin[g] += __shfl_xor_sync(0xffffffffu, lin[g], off);
+#pragma unroll
+                    for (int e = 0; e < R; ++e) pr[g][e] += __shfl_xor_sync(0xffffffffu, pr[g][e], off);
+                }
+            }
+            if (sub == 0 && b < b_hi) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float quad = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < R; ++e) {
+                        const float pe = pr[g][e] * S.scale[st][grp][e];
+                        quad = fmaf(pe, pe, quad);
+                    }
+                    sc_out[((size_t)sh * G + g) * n_full + b] = fmaf(0.5f, quad, lin[g]);
+                }
+            }
+        }
+        __syncthreads();                                  // stage st is read: refill it
+        if (tid == 0 && c + kBsStages < n_chunks) issue(c + kBsStages);
+    }
+}
+
 static int bd_validate(const crs_block_params *p) {
     if (!p) return CRS_ERR_INVALID_ARG;
     if (p->n_seq < 1 || p->n_kv < 1 || p->T < 1) return CRS_ERR_INVALID_ARG;
@@ -585,6 +765,76 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
         ProfScope _ps(K_BLK_PICK, s);
         block_pick_kernel<<<p->b.n_seq * p->b.n_kv, kPickT, smem_b, s>>>(
             sc, tok_idx, tok_count, G, n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+
+extern "C" int crs_block_quantize(const crs_block_params *p, const float *mu, const float *xi,
+                                  void *mu16, uint8_t *xi4, float *xi_scale, void *stream) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    crs_block_params b = *p;
+    b.blk_begin = 0;
+    b.blk_end = 0;
+    int st = bd_validate(&b);
+    if (st) return st;
+    if (!mu || !xi || !mu16 || !xi4 || !xi_scale) return CRS_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mu) | reinterpret_cast<uintptr_t>(xi) |
+         reinterpret_cast<uintptr_t>(mu16) | reinterpret_cast<uintptr_t>(xi4)) & 15)
+        return CRS_ERR_INVALID_ARG;
+    const long long n_mu = (long long)p->n_seq * p->n_kv * (p->T / p->L);
+    const long long n_xi = n_mu * p->rank;
+    if (n_mu == 0) return CRS_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        ProfScope _ps(K_BLK_SCORE, s);
+        block_quantize_kernel<<<(unsigned)ceil_div_ll(n_mu + n_xi, 8), 256, 0, s>>>(
+            mu, xi, static_cast<__nv_bfloat16 *>(mu16), xi4, xi_scale, n_mu, n_xi);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+
+extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q, const void *mu16,
+                                    const uint8_t *xi4, const float *xi_scale, int32_t *tok_idx,
+                                    int32_t *tok_count, void *ws, size_t ws_bytes, void *stream) {
+    int st = bs_validate(p);
+    if (st) return st;
+    if (!Q || !mu16 || !xi4 || !xi_scale || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
+    const int G = p->n_q / p->b.n_kv;
+    if (G != 8 || p->b.rank != 4) return CRS_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(mu16) | reinterpret_cast<uintptr_t>(xi4) |
+         reinterpret_cast<uintptr_t>(xi_scale)) & 15)
+        return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_block_select_workspace_size(p);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int n_full = p->b.T / p->b.L;
+    float *sc = static_cast<float *>(ws);
+    const int n_sh = p->b.n_seq * p->b.n_kv;
+    // every block's slice of the three arrays (256 B, 256 B, 16 B) starts on a
+    // 16-byte boundary, as the bulk copies require
+    const int per_sh = max(1, min(ceil_div(n_full, kBqChunk), ceil_div(148 * 4, n_sh)));
+    const int bpc = ceil_div(ceil_div(n_full, per_sh), kBqChunk) * kBqChunk;
+    const size_t smem_s = sizeof(BqSmem<8, 4>);
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_fp4_kernel<8, 4>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
+    {
+        ProfScope _ps(K_BLK_SCORE, s);
+        block_score_fp4_kernel<8, 4><<<dim3(ceil_div(n_full, bpc), n_sh), 8 * kBqChunk, smem_s, s>>>(
+            static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(mu16), xi4,
+            xi_scale, sc, p->b.n_kv, p->n_q, n_full, bpc, p->scale);
+    }
+    CRS_CHECK_LAUNCH();
+    const int cap = p->top_blocks * p->b.L + p->window;
+    const size_t smem_b = ((size_t)G + 1) * n_full * 4 + (size_t)p->top_blocks * 8;
+    if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_pick_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b));
+    {
+        ProfScope _ps(K_BLK_PICK, s);
+        block_pick_kernel<<<n_sh, kPickT, smem_b, s>>>(sc, tok_idx, tok_count, G, n_full, p->b.L,
+                                                       p->b.T, p->top_blocks, p->window, cap);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;

@@ -267,6 +267,33 @@ int crs_block_select(const crs_block_sel_params *p, const void *Q, const float *
 int crs_block_select_noalloc(const crs_block_sel_params *p, const void *Q, const float *mu,
                              const float *xi, int32_t *tok_idx, int32_t *tok_count, void *stream);
 
+/* Deployed descriptor compression.  [P5] §5.5 ("量化：对存储的特征向量做
+ * FP4") and Algorithm 2 steps 7-8: the block mean is stored in bf16 and each
+ * scaled eigenvector in E2M1 FP4 with one fp32 scale per vector.
+ *   mu, xi:   from crs_block_describe (fp32, [n_seq, n_kv, T/L, D] and
+ *             [n_seq, n_kv, T/L, rank, D]).
+ *   mu16:     [n_seq, n_kv, T/L, D] bf16 (round to nearest even).
+ *   xi4:      [n_seq, n_kv, T/L, rank, D/2] bytes: two 4-bit codes per byte,
+ *             the even element in the low nibble; code bit 3 = sign, bits 0-2
+ *             index {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *   xi_scale: [n_seq, n_kv, T/L, rank] fp32, = max |xi| / 6 of the vector; an
+ *             element is ~ sign * value(code) * scale.
+ * Rounding (the page leaves it open): the nearest value of xi / scale, a tie
+ * going to the zero-mantissa code, decided in fp32.  At r = 4, D = 128 the
+ * factors take 272 bytes per block instead of 1024 in bf16 ([P5] §5.5); with
+ * the mean, 528 bytes instead of 2560 in fp32.  All pointers 16-byte aligned
+ * (else CRS_ERR_INVALID_ARG); blk_begin / blk_end are ignored. */
+int crs_block_quantize(const crs_block_params *p, const float *mu, const float *xi, void *mu16,
+                       uint8_t *xi4, float *xi_scale, void *stream);
+
+/* crs_block_select on compressed descriptors (same selection rule, outputs and
+ * workspace as crs_block_select; the score uses the dequantised mean and
+ * eigenvectors).  Supported: 8 query heads per KV head, rank 4
+ * (else CRS_ERR_UNSUPPORTED); mu16, xi4, xi_scale 16-byte aligned. */
+int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q, const void *mu16,
+                         const uint8_t *xi4, const float *xi_scale, int32_t *tok_idx,
+                         int32_t *tok_count, void *ws, size_t ws_bytes, void *stream);
+
 /* ====================================================================== *
  * Attention over explicit index lists.  [P1] §1.1 Eq.(1) restricted to the
  * candidate set; [P2] §1.1 (one selected set shared by the main heads);

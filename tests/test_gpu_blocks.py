@@ -87,6 +87,24 @@ def test_select_on_oracle_descriptors(crs, cuda_dev):
                   top, "select")
 
 
+def test_select_ragged_block_count(crs, cuda_dev):
+    """50 complete blocks (a partial last chunk of the streamed descriptors) and a partial
+    last block of tokens: selection alone on the oracle's descriptors."""
+    T = 32 * 50 + 13
+    case = workloads.block_decode_case(n_seq=2, T=T, seed=17, device=cuda_dev)
+    p = case["params"]
+    L, r, top, win = p["L"], p["rank"], 9, 100
+    omu, oxi, _ = _oracle_describe(_np(case["K"]), L, r)
+    mu32 = torch.from_numpy(omu.astype(np.float32)).to(cuda_dev)
+    xi32 = torch.from_numpy(oxi[..., :r, :].astype(np.float32)).to(cuda_dev)
+    tok, cnt = crs.block_select(case["Q"], mu32, xi32, T, L, top, win)
+    torch.cuda.synchronize()
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(
+        _np(case["Q"]), mu32.double().cpu().numpy(), xi32.double().cpu().numpy(), T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
+                  "select-ragged")
+
+
 def test_describe_select_end_to_end_small(crs, cuda_dev):
     case = workloads.block_decode_case(n_seq=2, T=2048, seed=6, device=cuda_dev)
     p = case["params"]
@@ -106,3 +124,60 @@ def test_describe_select_end_to_end_small(crs, cuda_dev):
             d = np.setxor1d(gb, ob)
             cut = np.sort(o_bs[s, h])[::-1][top - 1]
             assert np.all(np.abs(o_bs[s, h][d] - cut) <= 1e-3 * abs(cut))
+
+
+def test_quantize_matches_oracle_bit_exact(crs, cuda_dev):
+    """FP4 codes and scales equal the oracle's (integers decided in fp32), the bf16 mean is
+    round-to-nearest-even ([P5] §5.5)."""
+    case = workloads.block_decode_case(n_seq=2, T=32 * 37, seed=8, device=cuda_dev)
+    p = case["params"]
+    mu, xi = crs.block_describe(case["K"], p["L"], p["rank"])
+    # a few planted values on the rounding midpoints and an all-zero vector
+    xi[0, 0, 0, 0] = 0.0
+    xi[0, 0, 1, 0, :8] = torch.tensor([6.0, 2.5, 0.25, 0.75, 1.25, 1.75, 3.5, 5.0], device=cuda_dev)
+    xi[0, 0, 1, 0, 8:] = 0.1
+    mu16, xi4, xs = crs.block_quantize(mu, xi, p["T"], p["L"])
+    torch.cuda.synchronize()
+    o_codes, o_scale = oracle.fp4_quantize(xi.cpu().numpy())
+    assert np.array_equal(xi4.cpu().numpy(), o_codes)
+    assert np.array_equal(xs.cpu().numpy(), o_scale)
+    assert torch.equal(mu16.cpu(), mu.cpu().to(torch.bfloat16))
+    assert xs[0, 0, 0, 0].item() == 0.0 and (xi4[0, 0, 0, 0] == 0).all()
+
+
+@pytest.mark.parametrize("n_seq,T,top,win", [(3, 4096, 16, 256), (2, 32 * 50 + 13, 9, 100)])
+def test_select_fp4_on_its_own_descriptors(crs, cuda_dev, n_seq, T, top, win):
+    """Selection over compressed descriptors equals the oracle's selection over the same
+    dequantised descriptors (set rule at the cutoff)."""
+    case = workloads.block_decode_case(n_seq=n_seq, T=T, seed=T, device=cuda_dev)
+    p = case["params"]
+    L, r = p["L"], p["rank"]
+    mu, xi = crs.block_describe(case["K"], L, r)
+    mu16, xi4, xs = crs.block_quantize(mu, xi, T, L)
+    tok, cnt = crs.block_select_fp4(case["Q"], mu16, xi4, xs, T, L, top, win)
+    torch.cuda.synchronize()
+    omu = _np(mu16)
+    oxi = oracle.fp4_dequantize(xi4.cpu().numpy(), xs.cpu().numpy())
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), omu, oxi, T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win,
+                  top, "select-fp4")
+
+
+def test_select_fp4_full_config_sampled(crs, cuda_dev):
+    """The block-sparse decode workload (32 seqs, T = 32768) on FP4 descriptors: every
+    (sequence, KV head) set checked against the oracle on the dequantised descriptors for
+    4 sampled sequences."""
+    case = workloads.block_decode_case(device=cuda_dev)
+    p = case["params"]
+    T, L, r, top, win = p["T"], p["L"], p["rank"], p["top_blocks"], p["window"]
+    mu, xi = crs.block_describe(case["K"], L, r)
+    mu16, xi4, xs = crs.block_quantize(mu, xi, T, L)
+    tok, cnt = crs.block_select_fp4(case["Q"], mu16, xi4, xs, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    seqs = [0, 7, 19, 31]
+    omu = _np(mu16)[seqs]
+    oxi = oracle.fp4_dequantize(xi4.cpu().numpy()[seqs], xs.cpu().numpy()[seqs])
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"])[seqs], omu, oxi, T, L, top, win)
+    _check_select(tok.cpu().numpy()[seqs], cnt.cpu().numpy()[seqs], o_tok, o_cnt, o_blk, o_bs, L, T,
+                  win, top, "select-fp4-full")
