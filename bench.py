@@ -1,7 +1,7 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|prefill|decode|block] [--no-extras]
+                  [--workload lsh|lsh_fp32|prefill|decode|block|block_fp4] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
@@ -12,6 +12,7 @@ A step is one pass of the hot path over one batch of the workload:
   decode   indexer decode, 64 sequences of ragged context + GQA gather attention.
   block    block-mass decode: block select (top-64 + 512 window) + GQA attention;
            the descriptor build is timed separately (it runs once per filled block).
+  block_fp4 the same on bf16 means + FP4 (E2M1) eigenvectors (528 B per block).
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on
 the launching stream; a 256 MiB buffer (2x L2) is written between steps,
 outside the events.  Multi-GPU: one process per GPU (torchrun), each rank runs
@@ -304,9 +305,42 @@ class BlockWorkload(Workload):
         }
 
 
+class BlockFp4Workload(BlockWorkload):
+    """The block workload on the deployed descriptor format: bf16 block means and
+    FP4 (E2M1) eigenvectors with one fp32 scale per vector (528 B per block of
+    D=128, rank 4, against 2560 B in fp32).  Cache build: describe + quantise."""
+
+    def __init__(self, crs, dev):
+        super().__init__(crs, dev)
+        p = self.p
+        self.name = self.c["workload"].replace("block_", "block_fp4_", 1)
+        self.mu16, self.xi4, self.xs = crs.block_quantize(self.mu, self.xi, p["T"], p["L"])
+        torch.cuda.synchronize()
+        del self.mu, self.xi
+        torch.cuda.empty_cache()
+
+    def _run(self, Q):
+        p = self.p
+        self.crs.block_select_fp4(Q, self.mu16, self.xi4, self.xs, p["T"], p["L"], p["top_blocks"],
+                                  p["window"], tok=self.tok, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
+                             workspace=self.ws2)
+
+    def roofline_spec(self):
+        p = self.p
+        nf = p["T"] // p["L"]
+        per_block = p["D"] * 2 + p["rank"] * (p["D"] // 2 + 4)
+        cap = p["top_blocks"] * p["L"] + p["window"]
+        return {
+            "block_score": [("hbm", p["n_seq"] * p["n_kv_heads"] * nf * per_block / 1e9, "GB/s")],
+            "sparse_attn": [("hbm", p["n_seq"] * p["n_kv_heads"] * cap * p["D"] * 2 * 2 / 1e9, "GB/s")],
+        }
+
+
 WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
-             "prefill": PrefillWorkload, "decode": DecodeWorkload, "block": BlockWorkload}
+             "prefill": PrefillWorkload, "decode": DecodeWorkload, "block": BlockWorkload,
+             "block_fp4": BlockFp4Workload}
 
 
 # ------------------------------------------------------------------- timing --
@@ -568,7 +602,7 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block") if w != args.workload]:
+        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block", "block_fp4") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)
                 r2 = measure(crs, w2, 5, 3, flush_buf, False, peaks)
@@ -588,6 +622,11 @@ def main():
                     e1.record()
                     torch.cuda.synchronize()
                     extras[name]["cache_build_ms"] = round(e0.elapsed_time(e1), 4)
+                    e0.record()
+                    crs.block_quantize(w2.mu, w2.xi, w2.p["T"], w2.p["L"])
+                    e1.record()
+                    torch.cuda.synchronize()
+                    extras[name]["fp4_quantize_ms"] = round(e0.elapsed_time(e1), 4)
                 del w2
                 torch.cuda.empty_cache()
             except Exception as e:   # an extra section must not hide the headline

@@ -787,7 +787,7 @@ extern "C" int crs_block_quantize(const crs_block_params *p, const float *mu, co
     if (n_mu == 0) return CRS_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
-        ProfScope _ps(K_BLK_SCORE, s);
+        ProfScope _ps(K_BLK_QUANTIZE, s);
         block_quantize_kernel<<<(unsigned)ceil_div_ll(n_mu + n_xi, 8), 256, 0, s>>>(
             mu, xi, static_cast<__nv_bfloat16 *>(mu16), xi4, xi_scale, n_mu, n_xi);
     }
