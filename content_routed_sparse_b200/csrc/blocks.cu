@@ -364,117 +364,200 @@ block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restr
 // ---------------------------------------------------------------------------
 // K9b: group softmax sum, top blocks, token list.  One CTA per (seq, KV head).
 // ---------------------------------------------------------------------------
-constexpr int kPickT = 256;
+constexpr int kPickT = 1024;
 
-// One CTA per (sequence, KV head).  Warp g takes query heads g, g + 8, ...:
-// the head's softmax over blocks (max and sum by shuffles) goes to its own
-// shared row, so the group sum is formed in a fixed order; warp 0 then selects
-// the top blocks exactly (4 radix passes over order-preserving keys, no block
-// barriers) and lists them in block order (ties: smaller block first).
+__host__ __device__ inline size_t pick_smem_bytes(int G, int n_full, int top) {
+    return (size_t)G * n_full * 4 + (size_t)top * 8;
+}
+
+// Exclusive prefix sums over the CTA of two per-thread counts (thread order).
+__device__ __forceinline__ void cta_exscan2(int a, int b, int &ea, int &eb, int &ta, int &tb, int2 *wtot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int xa = __shfl_up_sync(0xffffffffu, ia, o), xb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += xa;
+            ib += xb;
+        }
+    }
+    if (lane == 31) wtot[warp] = make_int2(ia, ib);
+    __syncthreads();
+    if (warp == 0) {
+        int2 v = lane < kPickT / 32 ? wtot[lane] : make_int2(0, 0);
+        int sa = v.x, sb = v.y;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int xa = __shfl_up_sync(0xffffffffu, sa, o), xb = __shfl_up_sync(0xffffffffu, sb, o);
+            if (lane >= o) {
+                sa += xa;
+                sb += xb;
+            }
+        }
+        if (lane < kPickT / 32) wtot[lane] = make_int2(sa - v.x, sb - v.y);   // exclusive per warp
+        if (lane == 31) wtot[kPickT / 32] = make_int2(sa, sb);                 // totals
+    }
+    __syncthreads();
+    const int2 base = wtot[warp], tot = wtot[kPickT / 32];
+    ea = base.x + ia - a;
+    eb = base.y + ib - b;
+    ta = tot.x;
+    tb = tot.y;
+    __syncthreads();                                    // wtot is reused by the next scan
+}
+
+// One CTA per (sequence, KV head), thread t owning blocks [t KPT, t KPT + KPT).
+// The 32 / G warps of query head g form its softmax over blocks (max and sum
+// by shuffles, combined across the warps in a fixed order; exponentials kept
+// in shared memory); the group sum of the heads' probabilities is formed per
+// block in head order.  The k-th largest block key is built bit by bit from
+// the top (32 CTA-wide counts), ties at it go to the smaller blocks, and the
+// kept blocks are listed in block order by CTA-wide prefix sums.
+template <int KPT>
 __global__ void __launch_bounds__(kPickT)
 block_pick_kernel(const float *__restrict__ sc, int32_t *__restrict__ tok, int32_t *__restrict__ cnt,
                   int G, int n_full, int L, int T, int top, int window, int cap) {
     extern __shared__ __align__(16) unsigned char bp_smem[];
-    float *prob = reinterpret_cast<float *>(bp_smem);                  // [G][n_full]
-    uint32_t *keyv = reinterpret_cast<uint32_t *>(prob + (size_t)G * n_full);   // [n_full]
-    int *sel = reinterpret_cast<int *>(keyv + n_full);                  // [top] kept blocks
-    int *tstart = sel + top;                                            // [top] output offsets
-    __shared__ uint32_t hist[256];
-    __shared__ int bc[2];
-    const int sh = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int g = warp; g < G; g += kPickT / 32) {
+    float *ex = reinterpret_cast<float *>(bp_smem);                       // [G][n_full]
+    int *sel = reinterpret_cast<int *>(ex + (size_t)G * n_full);         // [top] kept blocks
+    int *tstart = sel + top;                                              // [top] output offsets
+    __shared__ float iz[16];
+    __shared__ float part_red[kPickT / 32];
+    __shared__ int2 wtot[kPickT / 32 + 1];
+    const int sh = blockIdx.x, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    {   // G divides 16, so the 32 warps split evenly over the heads
+        const int wph = (kPickT / 32) / G, g = warp / wph, part = warp - g * wph;
         const float *s = sc + ((size_t)sh * G + g) * n_full;
-        float *pr = prob + (size_t)g * n_full;
+        float *e = ex + (size_t)g * n_full;
         float m = -INFINITY;
-        for (int b = lane; b < n_full; b += 32) m = fmaxf(m, s[b]);
+        for (int b0 = part * 32; b0 < n_full; b0 += 8 * wph * 32) {    // 8 loads in flight per lane
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int b = b0 + u * wph * 32 + lane;
+                v[u] = b < n_full ? s[b] : -INFINITY;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int b = b0 + u * wph * 32 + lane;
+                if (b < n_full) e[b] = v[u];
+                m = fmaxf(m, v[u]);
+            }
+        }
         m = warp_max(m);
+        if (lane == 0) part_red[warp] = m;
+        __syncthreads();
+        m = -INFINITY;
+        for (int q = 0; q < wph; ++q) m = fmaxf(m, part_red[g * wph + q]);
+        __syncthreads();
         float z = 0.0f;
-        for (int b = lane; b < n_full; b += 32) {
-            const float e = __expf(s[b] - m);
-            pr[b] = e;
-            z += e;
+        for (int b = part * 32 + lane; b < n_full; b += wph * 32) {
+            const float x = __expf(e[b] - m);
+            e[b] = x;
+            z += x;
         }
         z = warp_sum(z);
-        const float iz = 1.0f / z;
-        for (int b = lane; b < n_full; b += 32) pr[b] *= iz;
+        if (lane == 0) part_red[warp] = z;
+        __syncthreads();
+        if (part == 0 && lane == 0) {
+            float zt = 0.0f;
+            for (int q = 0; q < wph; ++q) zt += part_red[g * wph + q];
+            iz[g] = 1.0f / zt;
+        }
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < n_full; b += kPickT) {
-        float acc = 0.0f;
-        for (int g = 0; g < G; ++g) acc += prob[(size_t)g * n_full + b];
-        keyv[b] = score_key(acc);
+    const int bt0 = tid * KPT;
+    uint32_t key[KPT];
+    bool valid[KPT];
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+        const int b = bt0 + u;
+        valid[u] = b < n_full;
+        key[u] = 0u;
+        if (valid[u]) {
+            float acc = 0.0f;
+            for (int g = 0; g < G; ++g) acc += __fmul_rn(ex[(size_t)g * n_full + b], iz[g]);
+            key[u] = score_key(acc);
+        }
     }
-    __syncthreads();
+    auto count_ge = [&](uint32_t c) -> int {
+        int local = 0;
+#pragma unroll
+        for (int u = 0; u < KPT; ++u) local += (valid[u] && key[u] >= c) ? 1 : 0;
+        if (KPT == 1) return __syncthreads_count(local);
+        int total = 0;
+#pragma unroll
+        for (int bit = 0; (1 << bit) <= KPT; ++bit) total += __syncthreads_count(local & (1 << bit)) << bit;
+        return total;
+    };
+    // exact top k by (key desc, block asc): Tk = the largest key with >= k keys at or above it
+    const int k = min(top, n_full);
+    uint32_t Tk = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t c = Tk | (1u << bit);
+        if (count_ge(c) >= k) Tk = c;
+    }
+    const int need = k - (Tk == 0xffffffffu ? 0 : count_ge(Tk + 1u));   // ties at Tk to keep
+    int n_eq = 0;
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) n_eq += (valid[u] && key[u] == Tk) ? 1 : 0;
+    int eq_before, dummy, t0, t1;
+    cta_exscan2(n_eq, 0, eq_before, dummy, t0, t1, wtot);
     const int wstart = max(0, T - window);
-    if (warp == 0) {
-        // exact top `top` by (score desc, block asc)
-        const int k = min(top, n_full);
-        uint32_t prefix = 0u, mask = 0u;
-        int need = k;
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
+    bool take[KPT];
+    int n_take = 0, n_tok = 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0u;
-            __syncwarp();
-            for (int b = lane; b < n_full; b += 32) {
-                const uint32_t kk = keyv[b];
-                if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1u);
-            }
-            __syncwarp();
-            const int bin = warp_top_bin(hist, need);
-            prefix |= (uint32_t)bin << shift;
-            mask |= 0xffu << shift;
-            __syncwarp();
-        }
-        const uint32_t Tk = prefix;
-        // compaction in block order: block b = j * 32 + lane
-        int out = 0, eq_seen = 0, tok_pos = 0;
-        for (int j0 = 0; j0 < n_full; j0 += 32) {
-            const int b = j0 + lane;
-            const uint32_t kk = b < n_full ? keyv[b] : 0u;
-            const bool eq = b < n_full && kk == Tk;
-            const unsigned be = __ballot_sync(0xffffffffu, eq);
-            const bool take = (b < n_full && kk > Tk) ||
-                              (eq && eq_seen + __popc(be & ((1u << lane) - 1u)) < need);
-            const unsigned bt = __ballot_sync(0xffffffffu, take);
-            // tokens of block b that lie before the window
-            const int nt = take ? min(L, max(0, wstart - b * L)) : 0;
-            int incl = nt;
+    for (int u = 0; u < KPT; ++u) {
+        const int b = bt0 + u;
+        const bool eq = valid[u] && key[u] == Tk;
+        take[u] = (valid[u] && key[u] > Tk) || (eq && eq_before < need);
+        eq_before += eq ? 1 : 0;
+        n_take += take[u] ? 1 : 0;
+        n_tok += take[u] ? min(L, max(0, wstart - b * L)) : 0;   // tokens of b before the window
+    }
+    int slot, tpos, n_sel, nblk_tok;
+    cta_exscan2(n_take, n_tok, slot, tpos, n_sel, nblk_tok, wtot);
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int x = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += x;
-            }
-            if (take) {
-                const int slot = out + __popc(bt & ((1u << lane) - 1u));
-                sel[slot] = b;
-                tstart[slot] = tok_pos + incl - nt;
-            }
-            out += __popc(bt);
-            eq_seen += __popc(be);
-            tok_pos += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) {
-            bc[0] = out;
-            bc[1] = tok_pos;
-        }
+    for (int u = 0; u < KPT; ++u) {
+        if (!take[u]) continue;
+        const int b = bt0 + u;
+        sel[slot] = b;
+        tstart[slot] = tpos;
+        ++slot;
+        tpos += min(L, max(0, wstart - b * L));
     }
     __syncthreads();
     // token list: kept blocks' positions before the window (blocks ascending),
     // then the window [wstart, T)
-    const int n_sel = bc[0], nblk_tok = bc[1];
     int32_t *to = tok + (size_t)sh * cap;
-    for (int e = threadIdx.x; e < n_sel * L; e += kPickT) {
+    for (int e = tid; e < n_sel * L; e += kPickT) {
         const int i = e / L, r = e - i * L;
         const int b = sel[i];
         if (b * L + r < wstart) to[tstart[i] + r] = b * L + r;
     }
     const int nwin = T - wstart;
-    for (int i = threadIdx.x; i < nwin; i += kPickT) to[nblk_tok + i] = wstart + i;
+    for (int i = tid; i < nwin; i += kPickT) to[nblk_tok + i] = wstart + i;
     const int total = nblk_tok + nwin;
-    for (int i = total + threadIdx.x; i < cap; i += kPickT) to[i] = -1;
-    if (threadIdx.x == 0) cnt[sh] = total;
+    for (int i = total + tid; i < cap; i += kPickT) to[i] = -1;
+    if (tid == 0) cnt[sh] = total;
+}
+
+// Host: the instantiation for n_full blocks (KPT = blocks per thread).
+template <typename... A>
+static void launch_pick(int n_full, int grid, size_t smem, cudaStream_t s, A... args) {
+    if (n_full <= kPickT) block_pick_kernel<1><<<grid, kPickT, smem, s>>>(args...);
+    else if (n_full <= 2 * kPickT) block_pick_kernel<2><<<grid, kPickT, smem, s>>>(args...);
+    else if (n_full <= 4 * kPickT) block_pick_kernel<4><<<grid, kPickT, smem, s>>>(args...);
+    else block_pick_kernel<8><<<grid, kPickT, smem, s>>>(args...);
+}
+static cudaError_t pick_prepare(int n_full, size_t smem) {
+    const void *f = n_full <= kPickT ? (const void *)block_pick_kernel<1>
+                    : n_full <= 2 * kPickT ? (const void *)block_pick_kernel<2>
+                    : n_full <= 4 * kPickT ? (const void *)block_pick_kernel<4>
+                                           : (const void *)block_pick_kernel<8>;
+    return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -523,138 +606,306 @@ __global__ void __launch_bounds__(256) block_quantize_kernel(const float *__rest
     if (lane == 0) xi_scale[w] = sc;
 }
 
-// E2M1 code (4 bits) -> float: index 0/1 -> 0/0.5, else (1 + m/2) 2^(e-1)
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-    const uint32_t mag = e ? (((126u + e) << 23) | (m << 22)) : (m ? 0x3f000000u : 0u);
-    return __uint_as_float(mag | ((c & 8u) << 28));
+// bf16 bit patterns of the eight E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6},
+// split into high and low bytes so that one byte permute looks up four codes.
+constexpr uint32_t kE2m1HiLo = 0x3F3F3F00u, kE2m1HiHi = 0x40404040u;
+constexpr uint32_t kE2m1LoLo = 0xC0800000u, kE2m1LoHi = 0xC0804000u;
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 
-// K9a on compressed descriptors: the FP4 counterpart of block_score_tma_kernel.
-// A chunk of 16 blocks is 4 KB of bf16 means, 4 KB of FP4 codes and 256 B of
-// scales (three bulk copies); lane s of a block's 8-lane group covers dims
-// [8s, 8s + 8) and [64 + 8s, 64 + 8s + 8).  Projections are formed on the code
-// values and scaled once per vector.
-constexpr int kBqChunk = 16;
-template <int G, int R>
-struct BqSmem {
-    __nv_bfloat16 mu[kBsStages][kBqChunk][kBdD];
-    uint8_t xi[kBsStages][kBqChunk][R][kBdD / 2];
-    float scale[kBsStages][kBqChunk][R];
-    float sq[G][kBdD];
-    uint64_t full[kBsStages];
+// Eight E2M1 codes (element j in bits [4j, 4j+4): magnitude index in the low
+// three bits, sign in the fourth) -> eight bf16, two per word, element 2k in
+// the low half of word k.  Every E2M1 value is exact in bf16.  The high and
+// low bytes of each magnitude come from the byte tables above (one permute
+// looks up four codes); a code's sign is the top bit of its byte in w (odd
+// elements) or in w << 4 (even elements), replicated by the permute's sign
+// mode into the high byte before the two bytes are interleaved.
+__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t w) {
+    const uint32_t m = w & 0x77777777u, mh = m >> 16, w4 = w << 4;
+    const uint32_t hiA = prmt(kE2m1HiLo, kE2m1HiHi, m) | (prmt(w4, w, 0xD9C8u) & 0x80808080u);
+    const uint32_t hiB = prmt(kE2m1HiLo, kE2m1HiHi, mh) | (prmt(w4, w, 0xFBEAu) & 0x80808080u);
+    const uint32_t loA = prmt(kE2m1LoLo, kE2m1LoHi, m), loB = prmt(kE2m1LoLo, kE2m1LoHi, mh);
+    uint4 o;
+    o.x = prmt(loA, hiA, 0x5140u);
+    o.y = prmt(loA, hiA, 0x7362u);
+    o.z = prmt(loB, hiB, 0x5140u);
+    o.w = prmt(loB, hiB, 0x7362u);
+    return o;
+}
+
+// K9a on compressed descriptors, on the tensor cores.  A tile is 128
+// consecutive blocks of one (sequence, KV head); per tile the CTA forms
+//   lin_g   = Q_g . mu_b                  (A = the bf16 means, TMA, 128B swizzle)
+//   p_{e,g} = Q_g . code(xi_{b,e})        (A = the codes widened to bf16)
+// as M=128 (blocks) x N=16 (query heads, zero-padded) x K=128 products with
+// fp32 accumulators in TMEM; Q is the raw bf16 query (every product of two
+// bf16 is exact in fp32, so nothing is split), and the softmax scale and the
+// per-vector FP4 scale are applied in the epilogue:
+//   score_g = s lin_g + 1/2 sum_e (s sigma_e p_{e,g})^2.
+// Warp roles: 0 loads the mean tile and query rows (TMA, two stages); 1
+// owns TMEM and issues the MMAs; 4..7 read the accumulators (warp % 4 = lane
+// quadrant = 32 blocks); 8..15 read the codes of the next tile into registers while widening the
+// current one, one eigenvector at a time, into a four-buffer ring of bf16
+// operand tiles.  Persistent: each CTA walks a contiguous range of tiles.
+constexpr int kFtM = 128;                     // blocks per tile
+constexpr int kFtN = 16;                      // query-head columns (G <= 16)
+constexpr int kFtMaxR = 4;
+constexpr int kFtStages = 2;                  // mean + query tiles
+constexpr int kFtDecBufs = 4;                 // widened eigenvector tiles
+constexpr int kFtDecWarps = 8;
+constexpr int kFtThreads = 32 * (8 + kFtDecWarps);
+constexpr uint32_t kFtSuspendNs = 256;
+
+struct FtSmem {
+    unsigned char mu[kFtStages][2][kFtM * 128];    // [stage][K half]: 128 blocks x 64 dims, SW128
+    unsigned char dec[kFtDecBufs][2][kFtM * 128];  // [buffer][K half]: one eigenvector as bf16
+    unsigned char q[kFtStages][2][kFtN * 128];     // [stage][K half]: 16 rows x 64 dims, rows >= G zero
+    uint64_t full[kFtStages], raw_empty[kFtStages], dec_full[kFtDecBufs], dec_empty[kFtDecBufs];
+    uint64_t tm_full[2], tm_empty[2];
+    uint32_t tmem_base;
+    int fail;
 };
 
-template <int G, int R>
-__global__ void __launch_bounds__(8 * kBqChunk)
-block_score_fp4_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ mu16,
-                       const uint8_t *__restrict__ xi4, const float *__restrict__ xi_scale,
-                       float *__restrict__ sc_out, int n_kv, int n_q, int n_full, int blocks_per_cta,
-                       float scale) {
-    extern __shared__ __align__(128) unsigned char bq_raw[];
-    BqSmem<G, R> &S = *reinterpret_cast<BqSmem<G, R> *>(bq_raw);
-    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
-    const int b_lo = blockIdx.x * blocks_per_cta;
-    const int b_hi = min(n_full, b_lo + blocks_per_cta);
-    if (b_lo >= b_hi) return;
-    const int n_chunks = ceil_div(b_hi - b_lo, kBqChunk);
+struct FtArgs {
+    const __nv_bfloat16 *mu16;
+    const uint8_t *xi4;
+    const float *xi_scale;
+    float *sc_out;
+    int n_kv, n_q, G, R, n_full, tiles_per_sh, total_tiles, tiles_per_cta;
+    float scale;
+};
+
+__global__ void __launch_bounds__(kFtThreads, 1)
+block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_constant__ CUtensorMap tq,
+                          FtArgs a) {
+    extern __shared__ unsigned char ft_raw[];
+    const uint32_t mis = smem_u32(ft_raw) & 1023u;
+    FtSmem &S = *reinterpret_cast<FtSmem *>(ft_raw + ((1024u - mis) & 1023u));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const size_t blk0 = (size_t)sh * n_full;
-    auto issue = [&](int c) {                      // one thread
-        const int st = c % kBsStages;
-        const size_t b0 = blk0 + b_lo + (size_t)c * kBqChunk;
-        const int nb = min(kBqChunk, b_hi - (b_lo + c * kBqChunk));
-        const uint32_t mb = (uint32_t)nb * kBdD * 2, xb = (uint32_t)nb * R * (kBdD / 2);
-        const uint32_t sb = (uint32_t)((nb * R * 4 + 15) & ~15);
-        tc::mbar_arrive_expect_tx(&S.full[st], mb + xb + sb);
-        tc::bulk_load(&S.mu[st][0][0], mu16 + b0 * kBdD, mb, &S.full[st]);
-        tc::bulk_load(&S.xi[st][0][0][0], xi4 + b0 * R * (kBdD / 2), xb, &S.full[st]);
-        tc::bulk_load(&S.scale[st][0][0], xi_scale + b0 * R, sb, &S.full[st]);
-    };
+    const int t_lo = blockIdx.x * a.tiles_per_cta;
+    const int nt = min(a.total_tiles, t_lo + a.tiles_per_cta) - t_lo;
+    if (nt <= 0) return;
+    const int R = a.R;
     if (tid == 0) {
-        for (int st = 0; st < kBsStages; ++st) tc::mbar_init(&S.full[st], 1);
+        for (int i = 0; i < kFtStages; ++i) {
+            tc::mbar_init(&S.full[i], 1);
+            tc::mbar_init(&S.raw_empty[i], 1);
+        }
+        for (int i = 0; i < kFtDecBufs; ++i) {
+            tc::mbar_init(&S.dec_full[i], kFtDecWarps);
+            tc::mbar_init(&S.dec_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&S.tm_full[i], 1);
+            tc::mbar_init(&S.tm_empty[i], 4);
+        }
         tc::mbar_fence_init();
+        S.fail = 0;
     }
-    __syncthreads();
-    if (tid == 0)
-        for (int c = 0; c < min(kBsStages, n_chunks); ++c) issue(c);
-    for (int e = tid; e < G * kBdD; e += blockDim.x) {
-        const int g = e / kBdD, d = e - g * kBdD;
-        S.sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+    {   // query rows G..15 of every stage stay zero (the TMA box writes rows 0..G-1)
+        uint4 *qz = reinterpret_cast<uint4 *>(&S.q[0][0][0]);
+        for (int i = tid; i < (int)(sizeof(S.q) / 16); i += kFtThreads) qz[i] = make_uint4(0, 0, 0, 0);
     }
+    tc::fence_proxy_async();
+    if (warp == 1) tc::tmem_alloc(&S.tmem_base, 256);
+    tc::fence_before();
     __syncthreads();
-    const int sub = lane & 7, grp = warp * 4 + (lane >> 3);
-    bool ok = true;
-    for (int c = 0; c < n_chunks; ++c) {
-        const int st = c % kBsStages;
-        ok = ok && tc::mbar_wait_bounded(&S.full[st], (c / kBsStages) & 1, kBsWaitNs, K_BLK_SCORE, 2);
-        if (__syncthreads_or(!ok)) break;
-        const int b = b_lo + c * kBqChunk + grp;
-        {   // every lane computes (the group shuffles need all 32); invalid blocks only skip the store
-            float lin[G], pr[G][R];
+    tc::fence_after();
+    const uint32_t tmem = S.tmem_base;
+    auto tile_of = [&](int i, int &sh, int &b0, int &nb) {
+        const int t = t_lo + i;
+        sh = t / a.tiles_per_sh;
+        b0 = (t - sh * a.tiles_per_sh) * kFtM;
+        nb = min(kFtM, a.n_full - b0);
+    };
+
+    if (warp == 0) {
+        // ---------------- loads
+        if (lane == 0) {
+            for (int i = 0; i < nt; ++i) {
+                const int s = i % kFtStages, u = i / kFtStages;
+                if (u > 0 && !tc::mbar_wait_bounded(&S.raw_empty[s], (u - 1) & 1, kBsWaitNs, K_BLK_SCORE, 10,
+                                                    kFtSuspendNs)) {
+                    atomicOr(&S.fail, 1);
+                    break;
+                }
+                int sh, b0, nb;
+                tile_of(i, sh, b0, nb);
+                const int seq = sh / a.n_kv, h = sh - seq * a.n_kv;
+                tc::mbar_arrive_expect_tx(&S.full[s], 2 * kFtM * 128 + 2 * a.G * 128);
+                const int row = sh * a.n_full + b0;
+                tc::tma_load_2d(S.mu[s][0], &tmu, 0, row, &S.full[s]);
+                tc::tma_load_2d(S.mu[s][1], &tmu, 64, row, &S.full[s]);
+                const int qrow = seq * a.n_q + h * a.G;
+                tc::tma_load_2d(S.q[s][0], &tq, 0, qrow, &S.full[s]);
+                tc::tma_load_2d(S.q[s][1], &tq, 64, qrow, &S.full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(kFtM, kFtN, 0, 0);
+            bool ok = true;
+            int j = 0;                                   // eigenvector tiles consumed so far
+            for (int i = 0; ok && i < nt; ++i) {
+                const int s = i % kFtStages, u = i / kFtStages, acc = i & 1, w = i >> 1;
+                ok = tc::mbar_wait_bounded(&S.full[s], u & 1, kBsWaitNs, K_BLK_SCORE, 11, kFtSuspendNs);
+                if (ok && w > 0)
+                    ok = tc::mbar_wait_bounded(&S.tm_empty[acc], (w - 1) & 1, kBsWaitNs, K_BLK_SCORE, 12,
+                                               kFtSuspendNs);
+                if (!ok) break;
+                tc::fence_after();
+                const uint32_t d0 = tmem + acc * 128;
+                auto mma_tile = [&](unsigned char (*A)[kFtM * 128], uint32_t d) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                lin[g] = 0.0f;
+                    for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
-                for (int e = 0; e < R; ++e) pr[g][e] = 0.0f;
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t ad = tc::smem_desc(smem_u32(A[kh]) + k * 32, 16, 1024, tc::kLayoutSW128);
+                            const uint64_t bd = tc::smem_desc(smem_u32(S.q[s][kh]) + k * 32, 16, 1024,
+                                                              tc::kLayoutSW128);
+                            tc::mma_bf16(d, ad, bd, idesc, (kh | k) ? 1u : 0u);
+                        }
+                };
+                mma_tile(S.mu[s], d0);
+                for (int e = 0; e < R; ++e, ++j) {
+                    const int b = j % kFtDecBufs, v = j / kFtDecBufs;
+                    ok = tc::mbar_wait_bounded(&S.dec_full[b], v & 1, kBsWaitNs, K_BLK_SCORE, 13, kFtSuspendNs);
+                    if (!ok) break;
+                    tc::fence_after();
+                    mma_tile(S.dec[b], d0 + 16 * (1 + e));
+                    tc::commit(&S.dec_empty[b]);
+                }
+                if (!ok) break;
+                tc::commit(&S.raw_empty[s]);
+                tc::commit(&S.tm_full[acc]);
+            }
+            if (!ok) atomicOr(&S.fail, 1);
+        }
+    } else if (warp >= 8) {
+        // ---------------- widen the codes.  A thread owns, per eigenvector e and
+        // K half kh, words [c0, c0 + 4) of block r: dims [64 kh + 8 c, +8) for
+        // c in that range, which become 16-byte chunks c of row r.  A quarter
+        // warp covers 4 consecutive rows x both c0, so its swizzled 16-byte
+        // stores hit 8 distinct bank groups.  The codes of tile i+1 are read
+        // (16-byte loads) into registers while tile i is widened.
+        const int dw = warp - 8;
+        const int r = dw * 16 + (lane >> 3) * 4 + ((lane & 7) >> 1), c0 = (lane & 1) * 4;
+        uint4 cur[kFtMaxR][2], nxt[kFtMaxR][2];
+        auto fetch = [&](int i, uint4 (&dst)[kFtMaxR][2]) {
+            int sh, b0, nb;
+            tile_of(i, sh, b0, nb);
+            const uint8_t *src = a.xi4 + ((size_t)sh * a.n_full + b0 + r) * R * 64 + c0 * 4;
+#pragma unroll
+            for (int e = 0; e < kFtMaxR; ++e)
+#pragma unroll
+                for (int kh = 0; kh < 2; ++kh)
+                    dst[e][kh] = (e < R && r < nb) ? __ldg(reinterpret_cast<const uint4 *>(src + e * 64 + kh * 32))
+                                                   : make_uint4(0, 0, 0, 0);
+        };
+        fetch(0, cur);
+        int j = 0;
+        bool ok = true;
+        for (int i = 0; ok && i < nt; ++i) {
+            if (i + 1 < nt) fetch(i + 1, nxt);
+#pragma unroll
+            for (int e = 0; e < kFtMaxR; ++e) {
+                if (e >= R) break;
+                const int b = j % kFtDecBufs, v = j / kFtDecBufs;
+                ++j;
+                if (v > 0) {
+                    ok = tc::mbar_wait_bounded(&S.dec_empty[b], (v - 1) & 1, kBsWaitNs, K_BLK_SCORE, 15,
+                                               kFtSuspendNs);
+                    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                }
+#pragma unroll
+                for (int kh = 0; kh < 2; ++kh) {
+                    const uint32_t wv[4] = {cur[e][kh].x, cur[e][kh].y, cur[e][kh].z, cur[e][kh].w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        *reinterpret_cast<uint4 *>(S.dec[b][kh] + tc::sw128(r, c0 + k)) = e2m1x8_to_bf16(wv[k]);
+                }
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&S.dec_full[b]);
             }
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int d0 = half * 64 + sub * 8;              // 8 dims of this lane
-                const uint4 mraw = *reinterpret_cast<const uint4 *>(&S.mu[st][grp][d0]);
-                const __nv_bfloat162 *m2 = reinterpret_cast<const __nv_bfloat162 *>(&mraw);
-                float mv[8];
+            for (int e = 0; e < kFtMaxR; ++e)
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float2 f = __bfloat1622float2(m2[t]);
-                    mv[2 * t] = f.x;
-                    mv[2 * t + 1] = f.y;
-                }
-                float cv[R][8];
+                for (int kh = 0; kh < 2; ++kh) cur[e][kh] = nxt[e][kh];
+        }
+        if (!ok && lane == 0) atomicOr(&S.fail, 1);
+    } else if (warp >= 4) {
+        // ---------------- epilogue: thread = TMEM lane = block b0 + row
+        const int quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        // this block's FP4 scales, read kFtScaleAhead tiles ahead so that no
+        // global-load latency sits between two accumulator hand-offs
+        constexpr int kFtScaleAhead = 3;
+        float sring[kFtScaleAhead + 1][kFtMaxR];
+        auto load_sig = [&](int i, float (&dst)[kFtMaxR]) {
+            int sh, b0, nb;
+            tile_of(i, sh, b0, nb);
+            const bool valid = i < nt && row < nb;
+            const size_t blk = (size_t)sh * a.n_full + b0 + row;
 #pragma unroll
-                for (int e = 0; e < R; ++e) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(&S.xi[st][grp][e][d0 / 2]);
+            for (int e = 0; e < kFtMaxR; ++e)
+                dst[e] = (valid && e < R) ? __ldg(a.xi_scale + blk * R + e) : 0.0f;
+        };
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) cv[e][t] = e2m1_value((w >> (4 * t)) & 15u);
-                }
+        for (int k = 0; k < kFtScaleAhead; ++k) load_sig(k, sring[k]);
+        for (int i = 0; i < nt; ++i) {
+            const int acc = i & 1, w = i >> 1;
+            int sh, b0, nb;
+            tile_of(i, sh, b0, nb);
+            const bool valid = row < nb;
+            load_sig(i + kFtScaleAhead, sring[kFtScaleAhead]);
+            float sig[kFtMaxR];
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float4 q0 = *reinterpret_cast<const float4 *>(&S.sq[g][d0]);
-                    const float4 q1 = *reinterpret_cast<const float4 *>(&S.sq[g][d0 + 4]);
-                    const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            for (int e = 0; e < kFtMaxR; ++e) sig[e] = a.scale * sring[0][e];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        lin[g] = fmaf(qv[t], mv[t], lin[g]);
+            for (int k = 0; k < kFtScaleAhead; ++k)
 #pragma unroll
-                        for (int e = 0; e < R; ++e) pr[g][e] = fmaf(qv[t], cv[e][t], pr[g][e]);
+                for (int e = 0; e < kFtMaxR; ++e) sring[k][e] = sring[k + 1][e];
+            const bool ok = tc::mbar_wait_bounded(&S.tm_full[acc], w & 1, kBsWaitNs, K_BLK_SCORE, 16, kFtSuspendNs);
+            if (__any_sync(0xffffffffu, !ok)) {
+                if (lane == 0) atomicOr(&S.fail, 1);
+                break;
+            }
+            tc::fence_after();
+            uint32_t d[1 + kFtMaxR][16];
+            tc::tmem_ld16(tl + acc * 128, d[0]);
+#pragma unroll
+            for (int e = 0; e < kFtMaxR; ++e)
+                if (e < R) tc::tmem_ld16(tl + acc * 128 + 16 * (1 + e), d[1 + e]);
+            tc::tmem_ld_wait();
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&S.tm_empty[acc]);
+            if (valid) {
+#pragma unroll
+                for (int g = 0; g < kFtN; ++g) {
+                    if (g >= a.G) break;
+                    float quad2 = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < kFtMaxR; ++e) {      // sig[e] = 0 for e >= R
+                        const float pe = sig[e] * __uint_as_float(e < R ? d[1 + e][g] : 0u);
+                        quad2 = fmaf(pe, pe, quad2);
                     }
-                }
-            }
-#pragma unroll
-            for (int off = 1; off < 8; off <<= 1) {
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    lin[g] += __shfl_xor_sync(0xffffffffu, lin[g], off);
-#pragma unroll
-                    for (int e = 0; e < R; ++e) pr[g][e] += __shfl_xor_sync(0xffffffffu, pr[g][e], off);
-                }
-            }
-            if (sub == 0 && b < b_hi) {
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float quad = 0.0f;
-#pragma unroll
-                    for (int e = 0; e < R; ++e) {
-                        const float pe = pr[g][e] * S.scale[st][grp][e];
-                        quad = fmaf(pe, pe, quad);
-                    }
-                    sc_out[((size_t)sh * G + g) * n_full + b] = fmaf(0.5f, quad, lin[g]);
+                    a.sc_out[((size_t)sh * a.G + g) * a.n_full + b0 + row] =
+                        fmaf(0.5f, quad2, a.scale * __uint_as_float(d[0][g]));
                 }
             }
         }
-        __syncthreads();                                  // stage st is read: refill it
-        if (tid == 0 && c + kBsStages < n_chunks) issue(c + kBsStages);
     }
+    tc::fence_before();
+    __syncthreads();
+    if (S.fail && tid == 0) raise_error(CRS_DEVERR_TIMEOUT);
+    if (warp == 1) tc::tmem_dealloc(tmem, 256);
 }
 
 static int bd_validate(const crs_block_params *p) {
@@ -757,14 +1008,13 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
     }
     CRS_CHECK_LAUNCH();
     const int cap = p->top_blocks * p->b.L + p->window;
-    const size_t smem_b = ((size_t)G + 1) * n_full * 4 + (size_t)p->top_blocks * 8;
+    const size_t smem_b = pick_smem_bytes(G, n_full, p->top_blocks);
     if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
-    CRS_TRY_CUDA(cudaFuncSetAttribute(block_pick_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b));
+    CRS_TRY_CUDA(pick_prepare(n_full, smem_b));
     {
         ProfScope _ps(K_BLK_PICK, s);
-        block_pick_kernel<<<p->b.n_seq * p->b.n_kv, kPickT, smem_b, s>>>(
-            sc, tok_idx, tok_count, G, n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
+        launch_pick(n_full, p->b.n_seq * p->b.n_kv, smem_b, s, static_cast<const float *>(sc), tok_idx,
+                    tok_count, G, n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;
@@ -801,10 +1051,10 @@ extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q
     int st = bs_validate(p);
     if (st) return st;
     if (!Q || !mu16 || !xi4 || !xi_scale || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
-    const int G = p->n_q / p->b.n_kv;
-    if (G != 8 || p->b.rank != 4) return CRS_ERR_UNSUPPORTED;
-    if ((reinterpret_cast<uintptr_t>(mu16) | reinterpret_cast<uintptr_t>(xi4) |
-         reinterpret_cast<uintptr_t>(xi_scale)) & 15)
+    const int G = p->n_q / p->b.n_kv, R = p->b.rank;
+    if (R > kFtMaxR) return CRS_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(mu16) |
+         reinterpret_cast<uintptr_t>(xi4)) & 15)
         return CRS_ERR_INVALID_ARG;
     const size_t need = crs_block_select_workspace_size(p);
     if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
@@ -812,29 +1062,63 @@ extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q
     const int n_full = p->b.T / p->b.L;
     float *sc = static_cast<float *>(ws);
     const int n_sh = p->b.n_seq * p->b.n_kv;
-    // every block's slice of the three arrays (256 B, 256 B, 16 B) starts on a
-    // 16-byte boundary, as the bulk copies require
-    const int per_sh = max(1, min(ceil_div(n_full, kBqChunk), ceil_div(148 * 4, n_sh)));
-    const int bpc = ceil_div(ceil_div(n_full, per_sh), kBqChunk) * kBqChunk;
-    const size_t smem_s = sizeof(BqSmem<8, 4>);
-    CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_fp4_kernel<8, 4>,
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tc::tensor_map_encoder();
+    if (!enc) return CRS_ERR_CUDA;
+    CUtensorMap tmu, tq;
+    {   // means: [n_sh * n_full rows, 128 dims] bf16; a box is 128 blocks x 64 dims
+        cuuint64_t dims[2] = {(cuuint64_t)kBdD, (cuuint64_t)n_sh * n_full};
+        cuuint64_t strides[1] = {(cuuint64_t)kBdD * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)kFtM};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&tmu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(mu16), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CRS_ERR_CUDA;
+    }
+    {   // queries: [n_seq * n_q rows, 128 dims] bf16; a box is one KV head's G rows x 64 dims
+        cuuint64_t dims[2] = {(cuuint64_t)kBdD, (cuuint64_t)p->b.n_seq * p->n_q};
+        cuuint64_t strides[1] = {(cuuint64_t)kBdD * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)G};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(Q), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CRS_ERR_CUDA;
+    }
+    FtArgs fa;
+    fa.mu16 = static_cast<const __nv_bfloat16 *>(mu16);
+    fa.xi4 = xi4;
+    fa.xi_scale = xi_scale;
+    fa.sc_out = sc;
+    fa.n_kv = p->b.n_kv;
+    fa.n_q = p->n_q;
+    fa.G = G;
+    fa.R = R;
+    fa.n_full = n_full;
+    fa.tiles_per_sh = ceil_div(n_full, kFtM);
+    fa.total_tiles = n_sh * fa.tiles_per_sh;
+    fa.scale = p->scale;
+    int dev = 0, sms = 148;
+    CRS_TRY_CUDA(cudaGetDevice(&dev));
+    CRS_TRY_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    fa.tiles_per_cta = ceil_div(fa.total_tiles, max(1, sms));     // one CTA per SM
+    const int grid = ceil_div(fa.total_tiles, fa.tiles_per_cta);
+    const size_t smem_s = sizeof(FtSmem) + 1024;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_fp4_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
     {
         ProfScope _ps(K_BLK_SCORE, s);
-        block_score_fp4_kernel<8, 4><<<dim3(ceil_div(n_full, bpc), n_sh), 8 * kBqChunk, smem_s, s>>>(
-            static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(mu16), xi4,
-            xi_scale, sc, p->b.n_kv, p->n_q, n_full, bpc, p->scale);
+        block_score_fp4_tc_kernel<<<grid, kFtThreads, smem_s, s>>>(tmu, tq, fa);
     }
     CRS_CHECK_LAUNCH();
     const int cap = p->top_blocks * p->b.L + p->window;
-    const size_t smem_b = ((size_t)G + 1) * n_full * 4 + (size_t)p->top_blocks * 8;
+    const size_t smem_b = pick_smem_bytes(G, n_full, p->top_blocks);
     if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
-    CRS_TRY_CUDA(cudaFuncSetAttribute(block_pick_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b));
+    CRS_TRY_CUDA(pick_prepare(n_full, smem_b));
     {
         ProfScope _ps(K_BLK_PICK, s);
-        block_pick_kernel<<<n_sh, kPickT, smem_b, s>>>(sc, tok_idx, tok_count, G, n_full, p->b.L,
-                                                       p->b.T, p->top_blocks, p->window, cap);
+        launch_pick(n_full, n_sh, smem_b, s, static_cast<const float *>(sc), tok_idx, tok_count, G,
+                    n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;

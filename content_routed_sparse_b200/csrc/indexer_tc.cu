@@ -553,17 +553,6 @@ idx_tc_final_kernel(const uint32_t *__restrict__ cand_key, const int32_t *__rest
 }
 
 // ----------------------------------------------------------------- host --
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
 
 struct PrefillTcWs {
     uint16_t *samples;
@@ -616,7 +605,7 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
                              const void *k_idx, int32_t *out_idx, int32_t *out_count, void *ws,
                              cudaStream_t s) {
     const int n = p->n_rows, topk = p->topk;
-    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tc::tensor_map_encoder();
     if (!enc) return CRS_ERR_CUDA;
     if ((reinterpret_cast<uintptr_t>(q_idx) & 15) || (reinterpret_cast<uintptr_t>(k_idx) & 15))
         return CRS_ERR_INVALID_ARG;

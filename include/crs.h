@@ -288,8 +288,12 @@ int crs_block_quantize(const crs_block_params *p, const float *mu, const float *
 
 /* crs_block_select on compressed descriptors (same selection rule, outputs and
  * workspace as crs_block_select; the score uses the dequantised mean and
- * eigenvectors).  Supported: 8 query heads per KV head, rank 4
- * (else CRS_ERR_UNSUPPORTED); mu16, xi4, xi_scale 16-byte aligned. */
+ * eigenvectors).  Supported: up to 16 query heads per KV head (a divisor of
+ * 16, as for crs_block_select), rank 1..4 (else CRS_ERR_UNSUPPORTED); Q,
+ * mu16 and xi4 16-byte aligned (else CRS_ERR_INVALID_ARG).  The products
+ * Q . mu and Q . code are formed on the tensor cores from the bf16 query and
+ * the codes widened to bf16 (both exact), accumulated in fp32; the softmax
+ * scale and the per-vector FP4 scale are applied afterwards. */
 int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q, const void *mu16,
                          const uint8_t *xi4, const float *xi_scale, int32_t *tok_idx,
                          int32_t *tok_count, void *ws, size_t ws_bytes, void *stream);

@@ -181,3 +181,49 @@ def test_select_fp4_full_config_sampled(crs, cuda_dev):
     o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"])[seqs], omu, oxi, T, L, top, win)
     _check_select(tok.cpu().numpy()[seqs], cnt.cpu().numpy()[seqs], o_tok, o_cnt, o_blk, o_bs, L, T,
                   win, top, "select-fp4-full")
+
+
+@pytest.mark.parametrize("n_q,n_kv,rank,T,top,win", [
+    (16, 4, 2, 32 * 300 + 5, 20, 64),     # G = 4, three tiles of 128 blocks, ragged last tile
+    (64, 4, 1, 32 * 130, 7, 0),           # G = 16 (every column of the MMA), rank 1
+    (8, 2, 3, 32 * 257, 31, 300),         # G = 4, rank 3, one block past two full tiles
+])
+def test_select_fp4_head_and_rank_shapes(crs, cuda_dev, n_q, n_kv, rank, T, top, win):
+    """Compressed-descriptor selection for other query-group sizes and ranks, several
+    (sequence, KV head) pairs per CTA, against the oracle on the dequantised descriptors."""
+    case = workloads.block_decode_case(n_seq=3, T=T, n_kv_heads=n_kv, n_q_heads=n_q, rank=rank,
+                                       seed=T + n_q, device=cuda_dev)
+    p = case["params"]
+    L = p["L"]
+    mu, xi = crs.block_describe(case["K"], L, rank)
+    mu16, xi4, xs = crs.block_quantize(mu, xi, T, L)
+    tok, cnt = crs.block_select_fp4(case["Q"], mu16, xi4, xs, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    omu = _np(mu16)
+    oxi = oracle.fp4_dequantize(xi4.cpu().numpy(), xs.cpu().numpy())
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), omu, oxi, T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win,
+                  top, f"select-fp4-G{n_q // n_kv}-r{rank}")
+
+
+@pytest.mark.parametrize("n_full,n_q,n_kv,top", [(1500, 16, 2, 40), (3000, 8, 2, 100), (5000, 16, 2, 64),
+                                                 (8192, 4, 2, 300)])
+def test_select_many_blocks(crs, cuda_dev, n_full, n_q, n_kv, top):
+    """More than 1024 blocks per (sequence, KV head): several blocks per thread in the
+    pick kernel.  Random descriptors with planted exact ties at the cutoff."""
+    rng = np.random.default_rng(n_full)
+    L, D, rank, win = 32, 128, 2, 200
+    T = n_full * L + 7
+    mu = rng.standard_normal((1, n_kv, n_full, D)).astype(np.float32)
+    xi = (0.3 * rng.standard_normal((1, n_kv, n_full, rank, D))).astype(np.float32)
+    mu[0, 0, 7] = mu[0, 0, 3]            # identical descriptors -> identical block scores
+    xi[0, 0, 7] = xi[0, 0, 3]
+    Q = torch.from_numpy(rng.standard_normal((1, n_q, D)).astype(np.float32)).to(torch.bfloat16)
+    tok, cnt = crs.block_select(Q.to(cuda_dev), torch.from_numpy(mu).to(cuda_dev),
+                                torch.from_numpy(xi).to(cuda_dev), T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(Q.float().numpy(), mu, xi, T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
+                  f"select-{n_full}")
