@@ -344,13 +344,48 @@ static size_t sa_smem_bytes(int split_len) {
            (size_t)split_len * 4;
 }
 
+// Splits per (row, KV head), chosen on a makespan model of the grid.  A wave
+// runs n CTAs of k tiles on the SMs; an SM's gather rate is set by the CTAs it
+// holds, c = n / SMs: one CTA per SM gives rate 1 (c <= 1: the busy SMs' share),
+// each further resident CTA adds 0.35 (a lone CTA's gather is latency-bound).
+// A wave costs n k / (SMs rate(c)); splitting adds a merge pass, costed as
+// 4 + s/2 tiles (its partial rows grow with s).  At least 256 keys and at most kSaMaxSplit keys per split.
 static int sa_splits(const crs_attn_params *p) {
     const long long items = (long long)p->n_rows * p->n_kv;
-    const int max_split = max(1, ceil_div(p->max_idx, 256));   // >= 256 keys per split
-    const long long target = 148LL * 2;   // two CTAs per SM are resident
-    int s = (int)((target + items - 1) / items);
-    s = max(1, min(s, max_split));
-    return max(s, ceil_div(p->max_idx, kSaMaxSplit));
+    const int s_min = ceil_div(p->max_idx, kSaMaxSplit);
+    const int s_max = max(s_min, min(16, ceil_div(p->max_idx, 256)));
+    int dev = 0, sms = 148, smem_sm = 233472, smem_rsv = 1024;
+    cudaFuncAttributes fa;
+    fa.numRegs = 255;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, sparse_attn_kernel) != cudaSuccess) {
+        cudaGetLastError();          // model with the defaults; the launch reports real errors
+        sms = 148;
+    }
+    const int by_regs = 65536 / (kSaThreads * max(fa.numRegs, 1));
+    int best = s_min;
+    double best_cost = -1.0;
+    for (int s = s_min; s <= s_max; ++s) {
+        const int len = min(kSaMaxSplit, ceil_div(ceil_div(p->max_idx, s), kSaKeys) * kSaKeys);
+        const int per_sm = max(1, min(by_regs, smem_sm / (int)(sa_smem_bytes(len) + smem_rsv)));
+        const long long slots = (long long)per_sm * sms;
+        const long long ctas = items * ceil_div(p->max_idx, len);
+        const int k = len / kSaKeys;
+        double cost = s > 1 ? 4.0 + 0.5 * s : 0.0;
+        for (long long left = ctas; left > 0; left -= slots) {
+            const double n = (double)min(left, slots), c = n / sms;
+            const double rate = c <= 1.0 ? c : 1.0 + 0.35 * (min(c, (double)per_sm) - 1.0);
+            cost += n * k / (sms * rate);
+        }
+        if (best_cost < 0.0 || cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
 }
 
 static int sa_validate(const crs_attn_params *p) {
