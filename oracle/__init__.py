@@ -8,7 +8,9 @@ package.  It shares no code with the CUDA path; the arithmetic lives in
 Parity status per function (pins in ``tests/test_oracle_*.py``):
   lsh_hash / lsh_sort / lsh_candidates / lsh_attn  -- pinned
   indexer_topk / indexer_score                     -- pinned
-  block_describe / block_log_mass / block_select   -- pinned
+  block_describe / block_log_mass / block_select   -- pinned (rank 0 = mean-pool selector)
+  quest_describe / quest_select                    -- pinned
+  fp4_quantize / fp4_dequantize                    -- pinned
   sparse_attn                                      -- pinned
 """
 from __future__ import annotations
@@ -54,6 +56,9 @@ def _lib():
         lib.oracle_fp4_dequantize.argtypes = [I, I, _u8p, _f32p, _f64p]
         lib.oracle_block_select.argtypes = [I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
                                             I, _i32p, _i32p, _i32p, _f64p]
+        lib.oracle_quest_describe.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p]
+        lib.oracle_quest_select.argtypes = [I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p, I,
+                                            _i32p, _i32p, _i32p, _f64p]
         lib.oracle_sparse_attn.argtypes = [I, I, I, I, D, _f64p, _f64p, _f64p, _i64p, _i32p, I, I,
                                            _f64p, _f64p]
         _LIB = lib
@@ -235,6 +240,38 @@ def block_select(Q, mu, xi, T, L, top_blocks, window, scale=None):
     _lib().oracle_block_select(n_seq, n_kv, n_q, D, rank, n_full, L, T, top_blocks, window,
                                float(scale), _p(Q, _f64p), _p(mu, _f64p), _p(xi, _f64p), cap,
                                _p(tok, _i32p), _p(cnt, _i32p), _p(blk, _i32p), _p(bs, _f64p))
+    return tok, cnt, blk, bs
+
+
+def quest_describe(K, L):
+    """K [n_seq, T, n_kv, D] -> (kmin, kmax) [n_seq, n_kv, T // L, D] ([P5] Eq.(23))."""
+    K = _c(K, np.float64)
+    n_seq, T, n_kv, D = K.shape
+    n_full = T // L
+    kmin = np.empty((n_seq, n_kv, n_full, D), dtype=np.float64)
+    kmax = np.empty((n_seq, n_kv, n_full, D), dtype=np.float64)
+    _lib().oracle_quest_describe(n_seq, T, n_kv, D, L, _p(K, _f64p), _p(kmin, _f64p), _p(kmax, _f64p))
+    return kmin, kmax
+
+
+def quest_select(Q, kmin, kmax, T, L, top_blocks, window, scale=None):
+    """Quest box score ([P5] Eq.(24)) under the block_select rule.  Q [n_seq, n_q, D];
+    kmin, kmax [n_seq, n_kv, n_full, D].  Returns (tok, tok_count, blk, blk_score)."""
+    Q = _c(Q, np.float64)
+    kmin = _c(kmin, np.float64)
+    kmax = _c(kmax, np.float64)
+    n_seq, n_q, D = Q.shape
+    n_kv, n_full = kmin.shape[1], kmin.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cap = top_blocks * L + window
+    tok = np.empty((n_seq, n_kv, cap), dtype=np.int32)
+    cnt = np.empty((n_seq, n_kv), dtype=np.int32)
+    blk = np.empty((n_seq, n_kv, top_blocks), dtype=np.int32)
+    bs = np.empty((n_seq, n_kv, n_full), dtype=np.float64)
+    _lib().oracle_quest_select(n_seq, n_kv, n_q, D, n_full, L, T, top_blocks, window, float(scale),
+                               _p(Q, _f64p), _p(kmin, _f64p), _p(kmax, _f64p), cap, _p(tok, _i32p),
+                               _p(cnt, _i32p), _p(blk, _i32p), _p(bs, _f64p))
     return tok, cnt, blk, bs
 
 

@@ -499,10 +499,40 @@ OAPI double oracle_block_log_mass(int L, int D, const double *q, const double *K
  * tok_count [n_seq, n_kv], blk [n_seq, n_kv, top_blocks] (ascending),
  * blk_score [n_seq, n_kv, n_full].
  * ====================================================================== */
-OAPI void oracle_block_select(int n_seq, int n_kv, int n_q, int D, int rank, int n_full, int L,
-                              int T, int top_blocks, int window, double scale, const double *Q,
-                              const double *mu, const double *xi, int cap, int32_t *tok,
-                              int32_t *tok_count, int32_t *blk, double *blk_score)
+enum { SEL_COBS = 0, SEL_QUEST = 1 };
+
+/* One query head's block score s_{g,b} for selector `kind`:
+ *   SEL_COBS:  qt . A_b + 1/2 sum_i (B_{b,i} . qt)^2      (A = mu, B = xi, [P5] Eq.(14)/(19);
+ *              rank 0 is the mean-pool selector qt . kbar_b, [P5] Table 1)
+ *   SEL_QUEST: sum_t max(qt_t A_{b,t}, qt_t B_{b,t})       (A = kmin, B = kmax, [P5] Eq.(24)) */
+static double head_block_score(int kind, int D, int rank, const double *qt, const double *A,
+                               const double *B)
+{
+    double v = 0.0;
+    if (kind == SEL_QUEST) {
+        for (int t = 0; t < D; ++t) {
+            const double lo = qt[t] * A[t], hi = qt[t] * B[t];
+            v += lo > hi ? lo : hi;
+        }
+        return v;
+    }
+    for (int t = 0; t < D; ++t)
+        v += qt[t] * A[t];
+    double quad = 0.0;
+    for (int e = 0; e < rank; ++e) {
+        const double *x = B + (long)e * D;
+        double p = 0.0;
+        for (int t = 0; t < D; ++t)
+            p += x[t] * qt[t];
+        quad += p * p;
+    }
+    return v + 0.5 * quad;
+}
+
+static void block_select_run(int kind, int n_seq, int n_kv, int n_q, int D, int rank, int n_full,
+                             int L, int T, int top_blocks, int window, double scale, const double *Q,
+                             const double *Ab, const double *Bb, int cap, int32_t *tok,
+                             int32_t *tok_count, int32_t *blk, double *blk_score)
 {
     const int G = n_q / n_kv;
 #pragma omp parallel
@@ -524,19 +554,11 @@ OAPI void oracle_block_select(int n_seq, int n_kv, int n_q, int D, int rank, int
                         qt[t] = scale * q[t];
                     double mx = -INFINITY;
                     for (int b = 0; b < n_full; ++b) {
-                        const double *m = mu + (sh * n_full + b) * (long)D;
-                        double v = 0.0;
-                        for (int t = 0; t < D; ++t)
-                            v += qt[t] * m[t];
-                        double quad = 0.0;
-                        for (int e = 0; e < rank; ++e) {
-                            const double *x = xi + ((sh * n_full + b) * (long)rank + e) * D;
-                            double p = 0.0;
-                            for (int t = 0; t < D; ++t)
-                                p += x[t] * qt[t];
-                            quad += p * p;
-                        }
-                        s[b] = v + 0.5 * quad;
+                        const long blkid = sh * n_full + b;
+                        const double *a = Ab + blkid * (long)D;
+                        const double *bb = kind == SEL_QUEST ? Bb + blkid * (long)D
+                                                             : Bb + blkid * (long)rank * D;
+                        s[b] = head_block_score(kind, D, rank, qt, a, bb);
                         if (s[b] > mx) mx = s[b];
                     }
                     double z = 0.0;
@@ -580,6 +602,58 @@ OAPI void oracle_block_select(int n_seq, int n_kv, int n_q, int D, int rank, int
         free(sc);
         free(mark);
     }
+}
+
+
+OAPI void oracle_block_select(int n_seq, int n_kv, int n_q, int D, int rank, int n_full, int L,
+                              int T, int top_blocks, int window, double scale, const double *Q,
+                              const double *mu, const double *xi, int cap, int32_t *tok,
+                              int32_t *tok_count, int32_t *blk, double *blk_score)
+{
+    block_select_run(SEL_COBS, n_seq, n_kv, n_q, D, rank, n_full, L, T, top_blocks, window, scale,
+                     Q, mu, xi, cap, tok, tok_count, blk, blk_score);
+}
+
+/* ======================================================================
+ * O6q  Quest selection.  [P5] Eq.(23): per block the element-wise minimum
+ * and maximum of its keys (an axis-aligned box); Eq.(24): the block's score
+ * for a query is the largest inner product any point of the box reaches,
+ *   s_{g,b} = sum_t max(qt_t kmin_{b,t}, qt_t kmax_{b,t}),  qt = scale * q_g.
+ * Reading: the same group aggregation, top-k and window rule as O6 (the
+ * pages compare the selectors inside one block-sparse pipeline, [P5] Table 1).
+ * Layout: K [n_seq, T, n_kv, D]; kmin, kmax [n_seq, n_kv, n_full, D].
+ * ====================================================================== */
+OAPI void oracle_quest_describe(int n_seq, int T, int n_kv, int D, int L, const double *K,
+                                double *kmin, double *kmax)
+{
+    const int n_full = T / L;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int sq = 0; sq < n_seq; ++sq)
+        for (int h = 0; h < n_kv; ++h)
+            for (int b = 0; b < n_full; ++b) {
+                double *lo = kmin + (((long)sq * n_kv + h) * n_full + b) * D;
+                double *hi = kmax + (((long)sq * n_kv + h) * n_full + b) * D;
+                for (int t = 0; t < D; ++t) {
+                    lo[t] = INFINITY;
+                    hi[t] = -INFINITY;
+                }
+                for (int r = 0; r < L; ++r) {
+                    const double *k = K + (((long)sq * T + (long)b * L + r) * n_kv + h) * D;
+                    for (int t = 0; t < D; ++t) {
+                        if (k[t] < lo[t]) lo[t] = k[t];
+                        if (k[t] > hi[t]) hi[t] = k[t];
+                    }
+                }
+            }
+}
+
+OAPI void oracle_quest_select(int n_seq, int n_kv, int n_q, int D, int n_full, int L, int T,
+                              int top_blocks, int window, double scale, const double *Q,
+                              const double *kmin, const double *kmax, int cap, int32_t *tok,
+                              int32_t *tok_count, int32_t *blk, double *blk_score)
+{
+    block_select_run(SEL_QUEST, n_seq, n_kv, n_q, D, 0, n_full, L, T, top_blocks, window, scale, Q,
+                     kmin, kmax, cap, tok, tok_count, blk, blk_score);
 }
 
 /* ======================================================================
