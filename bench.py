@@ -1,7 +1,7 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|prefill|decode|block|block_fp4] [--no-extras]
+                  [--workload lsh|lsh_fp32|prefill|decode|block|block_fp4|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
@@ -13,6 +13,8 @@ A step is one pass of the hot path over one batch of the workload:
   block    block-mass decode: block select (top-64 + 512 window) + GQA attention;
            the descriptor build is timed separately (it runs once per filled block).
   block_fp4 the same on bf16 means + FP4 (E2M1) eigenvectors (528 B per block).
+  block_quest / block_meanpool  the same step with the baseline selectors (Quest boxes;
+           block means alone).
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on
 the launching stream; a 256 MiB buffer (2x L2) is written between steps,
 outside the events.  Multi-GPU: one process per GPU (torchrun), each rank runs
@@ -254,7 +256,7 @@ class BlockWorkload(Workload):
         self.name = c["workload"]
         p = self.p
         self.units_per_step = 1
-        self.mu, self.xi = crs.block_describe(c["K"], p["L"], p["rank"])   # cache build (once)
+        self._build_cache()                     # descriptor cache build (once, untimed)
         torch.cuda.synchronize()
         cap = p["top_blocks"] * p["L"] + p["window"]
         self.tok = torch.empty((p["n_seq"], p["n_kv_heads"], cap), dtype=torch.int32, device=dev)
@@ -278,6 +280,9 @@ class BlockWorkload(Workload):
         self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
         self.h2d = self.h_in["Q"].numel() * 2
         self.d2h = self.h_out.numel() * 2
+
+    def _build_cache(self):
+        self.mu, self.xi = self.crs.block_describe(self.c["K"], self.p["L"], self.p["rank"])
 
     def _run(self, Q):
         p = self.p
@@ -337,10 +342,56 @@ class BlockFp4Workload(BlockWorkload):
         }
 
 
+class BlockQuestWorkload(BlockWorkload):
+    """Baseline selector: Quest boxes (element-wise key min / max per block, bf16, 512 B
+    per block) under the same selection rule, then the gather attention."""
+
+    def __init__(self, crs, dev):
+        super().__init__(crs, dev)
+        self.name = self.c["workload"].replace("block_", "block_quest_", 1)
+
+    def _build_cache(self):
+        self.kmin, self.kmax = self.crs.quest_describe(self.c["K"], self.p["L"])
+
+    def _run(self, Q):
+        p = self.p
+        self.crs.block_select_quest(Q, self.kmin, self.kmax, p["T"], p["L"], p["top_blocks"], p["window"],
+                                    tok=self.tok, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
+                             workspace=self.ws2)
+
+    def roofline_spec(self):
+        p = self.p
+        spec = super().roofline_spec()
+        spec["block_score"] = [("hbm", p["n_seq"] * p["n_kv_heads"] * (p["T"] // p["L"]) * p["D"] * 4 / 1e9,
+                                "GB/s")]
+        return spec
+
+
+class BlockMeanPoolWorkload(BlockWorkload):
+    """Baseline selector: the block mean alone (first-order score, fp32, 512 B per block)."""
+
+    def __init__(self, crs, dev):
+        super().__init__(crs, dev)
+        self.name = self.c["workload"].replace("block_", "block_meanpool_", 1)
+
+    def _build_cache(self):
+        self.mu, _ = self.crs.block_describe(self.c["K"], self.p["L"], 1)
+        self.xi = None
+
+    def roofline_spec(self):
+        p = self.p
+        spec = super().roofline_spec()
+        spec["block_score"] = [("hbm", p["n_seq"] * p["n_kv_heads"] * (p["T"] // p["L"]) * p["D"] * 4 / 1e9,
+                                "GB/s")]
+        return spec
+
+
 WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
              "prefill": PrefillWorkload, "decode": DecodeWorkload, "block": BlockWorkload,
-             "block_fp4": BlockFp4Workload}
+             "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
+             "block_meanpool": BlockMeanPoolWorkload}
 
 
 # ------------------------------------------------------------------- timing --
@@ -602,7 +653,8 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block", "block_fp4") if w != args.workload]:
+        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block", "block_fp4", "block_quest",
+                                  "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)
                 r2 = measure(crs, w2, 5, 3, flush_buf, False, peaks)

@@ -115,6 +115,9 @@ _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP
 _sig("crs_block_quantize", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP, _VP, _VP])
 _sig("crs_block_select_fp4", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                              _VP, _VP, _SZ, _VP])
+_sig("crs_block_quest_describe", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP])
+_sig("crs_block_select_quest", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
+                                               _VP, _SZ, _VP])
 _sig("crs_block_select_noalloc", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP,
                                                  _VP, _VP, _VP])
 _sig("crs_sparse_attn_workspace_size", _SZ, [ctypes.POINTER(AttnParams)])
@@ -320,12 +323,15 @@ def block_describe(K, L: int, rank: int, blk_range=None, mu=None, xi=None, strea
 
 def block_select(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=None,
                  tok=None, count=None, workspace=None, stream=None):
-    """Block-mass selection -> (tok [n_seq, n_kv, top_blocks*L + window], count [n_seq, n_kv])."""
+    """Block-mass selection -> (tok [n_seq, n_kv, top_blocks*L + window], count [n_seq, n_kv]).
+    xi=None selects on the block means alone (the mean-pool selector, rank 0)."""
     _need(Q, "Q", torch.bfloat16)
     n_seq, n_q, D = Q.shape
-    n_kv, nfull, rank = mu.shape[1], mu.shape[2], xi.shape[3]
+    n_kv, nfull = mu.shape[1], mu.shape[2]
+    rank = 0 if xi is None else xi.shape[3]
     _need(mu, "mu", torch.float32, (n_seq, n_kv, nfull, D))
-    _need(xi, "xi", torch.float32, (n_seq, n_kv, nfull, rank, D))
+    if xi is not None:
+        _need(xi, "xi", torch.float32, (n_seq, n_kv, nfull, rank, D))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull), n_q,
@@ -342,6 +348,50 @@ def block_select(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=
     st = _lib.crs_block_select(ctypes.byref(p), _ptr(Q), _ptr(mu), _ptr(xi), _ptr(tok),
                                _ptr(count), _ptr(ws), wsb, _stream(stream))
     _check("crs_block_select", st)
+    return tok, count
+
+
+def quest_describe(K, L: int, out=None, stream=None):
+    """Quest summaries: K [n_seq, T, n_kv, D] bf16 -> (kmin, kmax) [n_seq, n_kv, T // L, D] bf16."""
+    _need(K, "K", torch.bfloat16)
+    n_seq, T, n_kv, D = K.shape
+    nfull = T // L
+    if out is None:
+        out = (torch.empty((n_seq, n_kv, nfull, D), dtype=torch.bfloat16, device=K.device),
+               torch.empty((n_seq, n_kv, nfull, D), dtype=torch.bfloat16, device=K.device))
+    kmin, kmax = out
+    _need(kmin, "kmin", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    _need(kmax, "kmax", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    p = BlockParams(n_seq, n_kv, int(T), D, int(L), 0, 0, nfull)
+    _check("crs_block_quest_describe", _lib.crs_block_quest_describe(ctypes.byref(p), _ptr(K), _ptr(kmin),
+                                                                     _ptr(kmax), _stream(stream)))
+    return kmin, kmax
+
+
+def block_select_quest(Q, kmin, kmax, T: int, L: int, top_blocks: int, window: int, scale=None,
+                       tok=None, count=None, workspace=None, stream=None):
+    """block_select with the Quest box score (summaries from quest_describe)."""
+    _need(Q, "Q", torch.bfloat16)
+    n_seq, n_q, D = Q.shape
+    n_kv, nfull = kmin.shape[1], kmin.shape[2]
+    _need(kmin, "kmin", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    _need(kmax, "kmax", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), 0, 0, nfull), n_q,
+                       int(top_blocks), int(window), float(scale))
+    cap = top_blocks * L + window
+    if tok is None:
+        tok = torch.empty((n_seq, n_kv, cap), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((n_seq, n_kv), dtype=torch.int32, device=Q.device)
+    _need(tok, "tok", torch.int32, (n_seq, n_kv, cap))
+    _need(count, "count", torch.int32, (n_seq, n_kv))
+    ws, wsb = _workspace(int(_lib.crs_block_select_workspace_size(ctypes.byref(p))), Q.device,
+                         workspace)
+    st = _lib.crs_block_select_quest(ctypes.byref(p), _ptr(Q), _ptr(kmin), _ptr(kmax), _ptr(tok),
+                                     _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_block_select_quest", st)
     return tok, count
 
 

@@ -561,6 +561,149 @@ static cudaError_t pick_prepare(int n_full, size_t smem) {
 }
 
 // ---------------------------------------------------------------------------
+// First-order and box selectors ([P5] Table 1): per-block summaries that are
+// scored without a quadratic term.
+//   Quest ([P5] Eq.(23)-(24)): kmin, kmax = element-wise key minimum and
+//     maximum of the block (bf16, exact: they are key values); score
+//     sum_t max(q_t kmin_t, q_t kmax_t) = sum_t q_t (q_t > 0 ? kmax_t : kmin_t).
+//   Mean-pool: the block mean (fp32), score q . mu (crs_block_select, rank 0).
+// ---------------------------------------------------------------------------
+constexpr int kQdWarps = 8;
+
+// One warp per block: lane l takes dims [4l, 4l + 4) of each of the L keys.
+__global__ void __launch_bounds__(kQdWarps * 32)
+quest_describe_kernel(const __nv_bfloat16 *__restrict__ K, __nv_bfloat16 *__restrict__ kmin,
+                      __nv_bfloat16 *__restrict__ kmax, int T, int n_kv, int L, int n_full, int blk_begin,
+                      int n_blk) {
+    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * kQdWarps + warp;
+    if (i >= n_blk) return;
+    const int blk = blk_begin + i;
+    float lo[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+    float hi[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    const __nv_bfloat16 *k0 = K + (((size_t)seq * T + (size_t)blk * L) * n_kv + h) * kBdD + 4 * lane;
+    const size_t row = (size_t)n_kv * kBdD;
+#pragma unroll 8
+    for (int r = 0; r < L; ++r) {
+        const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(k0 + r * row));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+        const float v[4] = {a.x, a.y, b.x, b.y};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            lo[t] = fminf(lo[t], v[t]);
+            hi[t] = fmaxf(hi[t], v[t]);
+        }
+    }
+    const size_t o = ((size_t)sh * n_full + blk) * kBdD + 4 * lane;
+    __nv_bfloat162 l0 = __floats2bfloat162_rn(lo[0], lo[1]), l1 = __floats2bfloat162_rn(lo[2], lo[3]);
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(hi[0], hi[1]), h1 = __floats2bfloat162_rn(hi[2], hi[3]);
+    *reinterpret_cast<uint2 *>(kmin + o) = make_uint2(*reinterpret_cast<uint32_t *>(&l0), *reinterpret_cast<uint32_t *>(&l1));
+    *reinterpret_cast<uint2 *>(kmax + o) = make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
+}
+
+// K9a for these selectors.  One warp scores 32 / G blocks at a time: lane l
+// holds dims [4l, 4l + 4) of the G scaled queries (registers) and of each
+// block's summary, forms the 32 partial sums (block j, head g) -> index
+// j G + g, and a five-step butterfly reduce-scatter leaves lane v with the
+// total of index v.
+constexpr int kWsWarps = 8;
+constexpr int kWsGroups = 2;              // block groups per warp
+enum { kWsQuest = 0, kWsMean = 1 };
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(kWsWarps * 32)
+block_score_warp_kernel(const __nv_bfloat16 *__restrict__ Q, const void *__restrict__ A,
+                        const void *__restrict__ B, float *__restrict__ sc_out, int n_kv, int n_q,
+                        int n_full, float scale) {
+    constexpr int BPW = 32 / G;
+    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float q[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(Q + ((size_t)seq * n_q + h * G + g) * kBdD + 4 * lane));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+        q[g][0] = scale * a.x;
+        q[g][1] = scale * a.y;
+        q[g][2] = scale * b.x;
+        q[g][3] = scale * b.y;
+    }
+    const int n_groups = ceil_div(n_full, BPW);
+    const int grp0 = (blockIdx.x * kWsWarps + warp) * kWsGroups;
+    for (int gi = 0; gi < kWsGroups; ++gi) {
+        const int b0 = (grp0 + gi) * BPW;
+        if (grp0 + gi >= n_groups) break;                 // warp-uniform
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < BPW; ++j) {
+            const int b = b0 + j;
+            const size_t o = ((size_t)sh * n_full + b) * kBdD + 4 * lane;
+            float lo[4] = {0.0f, 0.0f, 0.0f, 0.0f}, hi[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if (b < n_full) {
+                if constexpr (MODE == kWsQuest) {
+                    const uint2 rl = __ldcs(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(A) + o));
+                    const uint2 rh = __ldcs(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(B) + o));
+                    const float2 l0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&rl.x));
+                    const float2 l1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&rl.y));
+                    const float2 h0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&rh.x));
+                    const float2 h1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&rh.y));
+                    lo[0] = l0.x; lo[1] = l0.y; lo[2] = l1.x; lo[3] = l1.y;
+                    hi[0] = h0.x; hi[1] = h0.y; hi[2] = h1.x; hi[3] = h1.y;
+                } else {
+                    const float4 m = __ldcs(reinterpret_cast<const float4 *>(static_cast<const float *>(A) + o));
+                    lo[0] = m.x; lo[1] = m.y; lo[2] = m.z; lo[3] = m.w;
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if constexpr (MODE == kWsQuest) acc = fmaf(q[g][t], q[g][t] > 0.0f ? hi[t] : lo[t], acc);
+                    else acc = fmaf(q[g][t], lo[t], acc);
+                }
+                v[j * G + g] = acc;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < o; ++i) {
+                const float send = up ? v[i] : v[i + o];
+                const float keep = up ? v[i + o] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        const int j = lane / G, g = lane - j * G, b = b0 + j;
+        if (b < n_full) sc_out[((size_t)sh * G + g) * n_full + b] = v[0];
+    }
+}
+
+template <int MODE>
+static cudaError_t launch_score_warp(int G, dim3 grid, cudaStream_t s, const void *Q, const void *A,
+                                     const void *B, float *sc, int n_kv, int n_q, int n_full, float scale) {
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(Q);
+    switch (G) {
+    case 1: block_score_warp_kernel<1, MODE><<<grid, kWsWarps * 32, 0, s>>>(q, A, B, sc, n_kv, n_q, n_full, scale); break;
+    case 2: block_score_warp_kernel<2, MODE><<<grid, kWsWarps * 32, 0, s>>>(q, A, B, sc, n_kv, n_q, n_full, scale); break;
+    case 4: block_score_warp_kernel<4, MODE><<<grid, kWsWarps * 32, 0, s>>>(q, A, B, sc, n_kv, n_q, n_full, scale); break;
+    case 8: block_score_warp_kernel<8, MODE><<<grid, kWsWarps * 32, 0, s>>>(q, A, B, sc, n_kv, n_q, n_full, scale); break;
+    case 16: block_score_warp_kernel<16, MODE><<<grid, kWsWarps * 32, 0, s>>>(q, A, B, sc, n_kv, n_q, n_full, scale); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+static dim3 score_warp_grid(int G, int n_full, int n_sh) {
+    const int n_groups = ceil_div(n_full, 32 / G);
+    return dim3(ceil_div(n_groups, kWsWarps * kWsGroups), n_sh);
+}
+
+// ---------------------------------------------------------------------------
 // Deployed descriptor compression ([P5] §5.5): the block mean in bf16 and each
 // scaled eigenvector in E2M1 FP4 with one fp32 scale (absmax / 6).  One warp
 // per vector, four elements per lane; codes: bit 3 sign, bits 0-2 index into
@@ -948,9 +1091,11 @@ extern "C" int crs_block_describe(const crs_block_params *p, const void *K, floa
 
 static int bs_validate(const crs_block_sel_params *p) {
     if (!p) return CRS_ERR_INVALID_ARG;
+    if (p->b.rank < 0) return CRS_ERR_INVALID_ARG;
     crs_block_params b = p->b;
     b.blk_begin = 0;
     b.blk_end = 0;
+    b.rank = max(1, b.rank);                 // rank 0: the first-order (mean-pool) score
     int st = bd_validate(&b);
     if (st) return st;
     if (p->n_q < 1 || p->n_q % p->b.n_kv) return CRS_ERR_INVALID_ARG;
@@ -960,6 +1105,23 @@ static int bs_validate(const crs_block_sel_params *p) {
     if (n_full < 1 || n_full > 8192) return CRS_ERR_UNSUPPORTED;
     if (p->top_blocks < 1 || p->top_blocks > n_full) return CRS_ERR_INVALID_ARG;
     if (p->window < 0 || p->window > p->b.T) return CRS_ERR_INVALID_ARG;
+    return CRS_OK;
+}
+
+// K9b launch shared by every selector: scores sc [n_seq * n_kv][G][n_full] -> token lists.
+static int launch_block_pick(const crs_block_sel_params *p, const float *sc, int32_t *tok_idx,
+                             int32_t *tok_count, cudaStream_t s) {
+    const int G = p->n_q / p->b.n_kv, n_full = p->b.T / p->b.L;
+    const int cap = p->top_blocks * p->b.L + p->window;
+    const size_t smem_b = pick_smem_bytes(G, n_full, p->top_blocks);
+    if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
+    CRS_TRY_CUDA(pick_prepare(n_full, smem_b));
+    {
+        ProfScope _ps(K_BLK_PICK, s);
+        launch_pick(n_full, p->b.n_seq * p->b.n_kv, smem_b, s, sc, tok_idx, tok_count, G, n_full, p->b.L,
+                    p->b.T, p->top_blocks, p->window, cap);
+    }
+    CRS_CHECK_LAUNCH();
     return CRS_OK;
 }
 
@@ -974,12 +1136,23 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
                                 size_t ws_bytes, void *stream) {
     int st = bs_validate(p);
     if (st) return st;
-    if (!Q || !mu || !xi || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
+    if (!Q || !mu || (!xi && p->b.rank > 0) || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
     const size_t need = crs_block_select_workspace_size(p);
     if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int G = p->n_q / p->b.n_kv;
     const int n_full = p->b.T / p->b.L;
+    if (p->b.rank == 0) {                    // mean-pool: q . mu only
+        if ((reinterpret_cast<uintptr_t>(Q) & 7) || (reinterpret_cast<uintptr_t>(mu) & 15))
+            return CRS_ERR_INVALID_ARG;
+        float *sc = static_cast<float *>(ws);
+        {
+            ProfScope _ps(K_BLK_SCORE, s);
+            CRS_TRY_CUDA(launch_score_warp<kWsMean>(G, score_warp_grid(G, n_full, p->b.n_seq * p->b.n_kv), s,
+                                                    Q, mu, nullptr, sc, p->b.n_kv, p->n_q, n_full, p->scale));
+        }
+        return launch_block_pick(p, sc, tok_idx, tok_count, s);
+    }
     const int nbt = kBsThreads / G;
     const size_t smem_a = ((size_t)G * (kBdD + 1) + (size_t)nbt * (1 + p->b.rank) * (kBdD + 1)) * 4;
     if (smem_a > 227 * 1024) return CRS_ERR_UNSUPPORTED;
@@ -1007,17 +1180,7 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
     }
     }
     CRS_CHECK_LAUNCH();
-    const int cap = p->top_blocks * p->b.L + p->window;
-    const size_t smem_b = pick_smem_bytes(G, n_full, p->top_blocks);
-    if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
-    CRS_TRY_CUDA(pick_prepare(n_full, smem_b));
-    {
-        ProfScope _ps(K_BLK_PICK, s);
-        launch_pick(n_full, p->b.n_seq * p->b.n_kv, smem_b, s, static_cast<const float *>(sc), tok_idx,
-                    tok_count, G, n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
-    }
-    CRS_CHECK_LAUNCH();
-    return CRS_OK;
+    return launch_block_pick(p, sc, tok_idx, tok_count, s);
 }
 
 extern "C" int crs_block_quantize(const crs_block_params *p, const float *mu, const float *xi,
@@ -1052,6 +1215,7 @@ extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q
     if (st) return st;
     if (!Q || !mu16 || !xi4 || !xi_scale || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
     const int G = p->n_q / p->b.n_kv, R = p->b.rank;
+    if (R < 1) return CRS_ERR_INVALID_ARG;
     if (R > kFtMaxR) return CRS_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(mu16) |
          reinterpret_cast<uintptr_t>(xi4)) & 15)
@@ -1111,15 +1275,51 @@ extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q
         block_score_fp4_tc_kernel<<<grid, kFtThreads, smem_s, s>>>(tmu, tq, fa);
     }
     CRS_CHECK_LAUNCH();
-    const int cap = p->top_blocks * p->b.L + p->window;
-    const size_t smem_b = pick_smem_bytes(G, n_full, p->top_blocks);
-    if (smem_b > 200 * 1024) return CRS_ERR_UNSUPPORTED;
-    CRS_TRY_CUDA(pick_prepare(n_full, smem_b));
+    return launch_block_pick(p, sc, tok_idx, tok_count, s);
+}
+
+extern "C" int crs_block_quest_describe(const crs_block_params *p, const void *K, void *kmin, void *kmax,
+                                        void *stream) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    crs_block_params b = *p;
+    b.rank = 1;                              // no eigenvectors here
+    int st = bd_validate(&b);
+    if (st) return st;
+    if (!K || !kmin || !kmax) return CRS_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax)) & 7)
+        return CRS_ERR_INVALID_ARG;
+    const int n_full = p->T / p->L;
+    if (p->blk_begin < 0 || p->blk_end > n_full || p->blk_begin > p->blk_end) return CRS_ERR_INVALID_ARG;
+    const int n_blk = p->blk_end - p->blk_begin;
+    if (n_blk == 0) return CRS_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
-        ProfScope _ps(K_BLK_PICK, s);
-        launch_pick(n_full, n_sh, smem_b, s, static_cast<const float *>(sc), tok_idx, tok_count, G,
-                    n_full, p->b.L, p->b.T, p->top_blocks, p->window, cap);
+        ProfScope _ps(K_BLK_DESCRIBE, s);
+        quest_describe_kernel<<<dim3(ceil_div(n_blk, kQdWarps), p->n_seq * p->n_kv), kQdWarps * 32, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(K), static_cast<__nv_bfloat16 *>(kmin),
+            static_cast<__nv_bfloat16 *>(kmax), p->T, p->n_kv, p->L, n_full, p->blk_begin, n_blk);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;
+}
+
+extern "C" int crs_block_select_quest(const crs_block_sel_params *p, const void *Q, const void *kmin,
+                                      const void *kmax, int32_t *tok_idx, int32_t *tok_count, void *ws,
+                                      size_t ws_bytes, void *stream) {
+    int st = bs_validate(p);
+    if (st) return st;
+    if (!Q || !kmin || !kmax || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(kmin) | reinterpret_cast<uintptr_t>(kmax)) & 7)
+        return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_block_select_workspace_size(p);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int G = p->n_q / p->b.n_kv, n_full = p->b.T / p->b.L;
+    float *sc = static_cast<float *>(ws);
+    {
+        ProfScope _ps(K_BLK_SCORE, s);
+        CRS_TRY_CUDA(launch_score_warp<kWsQuest>(G, score_warp_grid(G, n_full, p->b.n_seq * p->b.n_kv), s, Q,
+                                                 kmin, kmax, sc, p->b.n_kv, p->n_q, n_full, p->scale));
+    }
+    return launch_block_pick(p, sc, tok_idx, tok_count, s);
 }

@@ -236,7 +236,9 @@ typedef struct {
 } crs_block_sel_params;
 
 /* Q: [n_seq, n_q, D] bf16; mu, xi from crs_block_describe.
- * tok_idx: [n_seq, n_kv, top_blocks*L + window] int32; tok_count: [n_seq, n_kv]. */
+ * tok_idx: [n_seq, n_kv, top_blocks*L + window] int32; tok_count: [n_seq, n_kv].
+ * rank 0 is the mean-pool selector of [P5] Table 1 (s_{g,b} = qt . mu_b, the
+ * first-order term alone): xi may then be NULL; Q 8-byte and mu 16-byte aligned. */
 size_t crs_block_select_workspace_size(const crs_block_sel_params *p);
 int crs_block_select(const crs_block_sel_params *p, const void *Q, const float *mu,
                      const float *xi, int32_t *tok_idx, int32_t *tok_count, void *ws,
@@ -297,6 +299,26 @@ int crs_block_quantize(const crs_block_params *p, const float *mu, const float *
 int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q, const void *mu16,
                          const uint8_t *xi4, const float *xi_scale, int32_t *tok_idx,
                          int32_t *tok_count, void *ws, size_t ws_bytes, void *stream);
+
+/* ====================================================================== *
+ * Quest box selector ([P5] Quest section, Eq.(23)-(24), Table 1).
+ * crs_block_quest_describe: per complete block b of L keys and KV head h the
+ * element-wise minimum and maximum of its keys, kmin_b, kmax_b (the keys'
+ * own bf16 values: exact).  Blocks [blk_begin, blk_end) of every (sequence,
+ * KV head) are written; p->rank is ignored.
+ *   K: [n_seq, T, n_kv, D] bf16; kmin, kmax: [n_seq, n_kv, T/L, D] bf16.
+ * crs_block_select_quest: the block selection rule of crs_block_select with
+ * the box score s_{g,b} = sum_t max(qt_t kmin_{b,t}, qt_t kmax_{b,t}),
+ * qt = scale * q_g, the largest inner product a point of the box reaches.
+ * kmin <= kmax element-wise (as crs_block_quest_describe writes them); same
+ * workspace size as crs_block_select; Q, kmin, kmax 8-byte aligned (else
+ * CRS_ERR_INVALID_ARG); D = 128, G <= 16 dividing 16 (else CRS_ERR_UNSUPPORTED).
+ * ====================================================================== */
+int crs_block_quest_describe(const crs_block_params *p, const void *K, void *kmin, void *kmax,
+                             void *stream);
+int crs_block_select_quest(const crs_block_sel_params *p, const void *Q, const void *kmin,
+                           const void *kmax, int32_t *tok_idx, int32_t *tok_count, void *ws,
+                           size_t ws_bytes, void *stream);
 
 /* ====================================================================== *
  * Attention over explicit index lists.  [P1] §1.1 Eq.(1) restricted to the

@@ -227,3 +227,70 @@ def test_select_many_blocks(crs, cuda_dev, n_full, n_q, n_kv, top):
     o_tok, o_cnt, o_blk, o_bs = oracle.block_select(Q.float().numpy(), mu, xi, T, L, top, win)
     _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
                   f"select-{n_full}")
+
+
+# ---------------------------------------------------------------- Quest / mean-pool --
+def test_quest_describe_matches_oracle_bit_exact(crs, cuda_dev):
+    """kmin / kmax are key values: bf16 on the GPU, equal to the oracle's min / max."""
+    case = workloads.block_decode_case(n_seq=2, T=32 * 37 + 5, seed=9, device=cuda_dev)
+    p = case["params"]
+    kmin, kmax = crs.quest_describe(case["K"], p["L"])
+    torch.cuda.synchronize()
+    o_min, o_max = oracle.quest_describe(_np(case["K"]), p["L"])
+    assert np.array_equal(kmin.double().cpu().numpy(), o_min)
+    assert np.array_equal(kmax.double().cpu().numpy(), o_max)
+
+
+@pytest.mark.parametrize("n_q,n_kv,T,top,win", [
+    (32, 4, 4096, 16, 256),          # G = 8
+    (16, 4, 32 * 300 + 5, 20, 64),   # G = 4, ragged
+    (64, 4, 32 * 130, 7, 0),         # G = 16
+    (4, 4, 32 * 77, 9, 100),         # G = 1
+])
+def test_select_quest_matches_oracle(crs, cuda_dev, n_q, n_kv, T, top, win):
+    case = workloads.block_decode_case(n_seq=3, T=T, n_kv_heads=n_kv, n_q_heads=n_q, seed=T + n_q,
+                                       device=cuda_dev)
+    L = case["params"]["L"]
+    kmin, kmax = crs.quest_describe(case["K"], L)
+    tok, cnt = crs.block_select_quest(case["Q"], kmin, kmax, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    o_tok, o_cnt, o_blk, o_bs = oracle.quest_select(_np(case["Q"]), kmin.double().cpu().numpy(),
+                                                    kmax.double().cpu().numpy(), T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
+                  f"quest-G{n_q // n_kv}")
+
+
+@pytest.mark.parametrize("n_q,n_kv,T,top,win", [(32, 4, 4096, 16, 256), (16, 4, 32 * 300 + 5, 20, 64),
+                                                (64, 4, 32 * 130, 7, 0)])
+def test_select_meanpool_matches_oracle(crs, cuda_dev, n_q, n_kv, T, top, win):
+    """Rank 0 (xi = None): the first-order score q . mu alone."""
+    case = workloads.block_decode_case(n_seq=3, T=T, n_kv_heads=n_kv, n_q_heads=n_q, seed=T + 1,
+                                       device=cuda_dev)
+    L = case["params"]["L"]
+    mu, _ = crs.block_describe(case["K"], L, 1)
+    tok, cnt = crs.block_select(case["Q"], mu, None, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    omu = mu.double().cpu().numpy()
+    oxi = np.zeros(omu.shape[:3] + (0, omu.shape[3]))
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), omu, oxi, T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
+                  f"meanpool-G{n_q // n_kv}")
+
+
+def test_select_quest_full_config_sampled(crs, cuda_dev):
+    """The block-sparse decode workload (32 seqs, T = 32768) with the Quest selector; 4
+    sampled sequences checked against the oracle."""
+    case = workloads.block_decode_case(device=cuda_dev)
+    p = case["params"]
+    T, L, top, win = p["T"], p["L"], p["top_blocks"], p["window"]
+    kmin, kmax = crs.quest_describe(case["K"], L)
+    tok, cnt = crs.block_select_quest(case["Q"], kmin, kmax, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    seqs = [0, 11, 22, 31]
+    o_tok, o_cnt, o_blk, o_bs = oracle.quest_select(_np(case["Q"])[seqs], kmin.double().cpu().numpy()[seqs],
+                                                    kmax.double().cpu().numpy()[seqs], T, L, top, win)
+    _check_select(tok.cpu().numpy()[seqs], cnt.cpu().numpy()[seqs], o_tok, o_cnt, o_blk, o_bs, L, T,
+                  win, top, "quest-full")
