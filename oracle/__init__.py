@@ -10,6 +10,7 @@ Parity status per function (pins in ``tests/test_oracle_*.py``):
   indexer_topk / indexer_score                     -- pinned
   block_describe / block_log_mass / block_select   -- pinned (rank 0 = mean-pool selector)
   quest_describe / quest_select                    -- pinned
+  block_describe_ss / block_select_ss              -- pinned
   fp4_quantize / fp4_dequantize                    -- pinned
   sparse_attn                                      -- pinned
 """
@@ -56,6 +57,9 @@ def _lib():
         lib.oracle_fp4_dequantize.argtypes = [I, I, _u8p, _f32p, _f64p]
         lib.oracle_block_select.argtypes = [I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
                                             I, _i32p, _i32p, _i32p, _f64p]
+        lib.oracle_block_describe_ss.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p, _f64p, _f64p]
+        lib.oracle_block_select_ss.argtypes = [I, I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
+                                               _f64p, I, _i32p, _i32p, _i32p, _f64p]
         lib.oracle_quest_describe.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p]
         lib.oracle_quest_select.argtypes = [I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p, I,
                                             _i32p, _i32p, _i32p, _f64p]
@@ -240,6 +244,43 @@ def block_select(Q, mu, xi, T, L, top_blocks, window, scale=None):
     _lib().oracle_block_select(n_seq, n_kv, n_q, D, rank, n_full, L, T, top_blocks, window,
                                float(scale), _p(Q, _f64p), _p(mu, _f64p), _p(xi, _f64p), cap,
                                _p(tok, _i32p), _p(cnt, _i32p), _p(blk, _i32p), _p(bs, _f64p))
+    return tok, cnt, blk, bs
+
+
+def block_describe_ss(Kblocks, U, rank):
+    """Subspace descriptors: Kblocks [nb, L, D], U [D, s] -> (mu [nb, D], xi [nb, rank, s],
+    lam [nb, rank]) with xi the scaled eigenvectors of U^T Sigma_b U ([P5] Eq.(17))."""
+    Kb = _c(Kblocks, np.float64)
+    U = _c(U, np.float64)
+    nb, L, D = Kb.shape
+    sd = U.shape[1]
+    mu = np.empty((nb, D), dtype=np.float64)
+    xi = np.empty((nb, rank, sd), dtype=np.float64)
+    lam = np.empty((nb, rank), dtype=np.float64)
+    _lib().oracle_block_describe_ss(nb, L, D, sd, rank, _p(Kb, _f64p), _p(U, _f64p), _p(mu, _f64p),
+                                    _p(xi, _f64p), _p(lam, _f64p))
+    return mu, xi, lam
+
+
+def block_select_ss(Q, U, mu, xi, T, L, top_blocks, window, scale=None):
+    """block_select with the subspace quadratic term ([P5] Eq.(18)): Q [n_seq, n_q, D],
+    U [D, s], mu [n_seq, n_kv, n_full, D], xi [n_seq, n_kv, n_full, rank, s]."""
+    Q = _c(Q, np.float64)
+    U = _c(U, np.float64)
+    mu = _c(mu, np.float64)
+    xi = _c(xi, np.float64)
+    n_seq, n_q, D = Q.shape
+    n_kv, n_full, rank, sd = mu.shape[1], mu.shape[2], xi.shape[3], xi.shape[4]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cap = top_blocks * L + window
+    tok = np.empty((n_seq, n_kv, cap), dtype=np.int32)
+    cnt = np.empty((n_seq, n_kv), dtype=np.int32)
+    blk = np.empty((n_seq, n_kv, top_blocks), dtype=np.int32)
+    bs = np.empty((n_seq, n_kv, n_full), dtype=np.float64)
+    _lib().oracle_block_select_ss(n_seq, n_kv, n_q, D, sd, rank, n_full, L, T, top_blocks, window,
+                                  float(scale), _p(Q, _f64p), _p(U, _f64p), _p(mu, _f64p), _p(xi, _f64p),
+                                  cap, _p(tok, _i32p), _p(cnt, _i32p), _p(blk, _i32p), _p(bs, _f64p))
     return tok, cnt, blk, bs
 
 

@@ -392,12 +392,18 @@ static void jacobi_eig(int n, double *A, double *Vm)
     }
 }
 
-OAPI void oracle_block_describe(int n_blocks, int L_cap, int D, int rank, const double *K,
-                                const int32_t *L_eff, double *mu, double *xi, double *lam)
+/* U == NULL: the descriptors of the full key space (Y = Kt, sd = D).  Else
+ * U [D, sd] (row-major) spans the query subspace and the eigenvectors are
+ * taken of the projected covariance B = U^T Sigma U, [P5] Eq.(17), by the
+ * same Gram route on Y = Kt U: G = Y Y^T / L, xi_i = Y^T w_i / sqrt(L) in R^sd. */
+static void block_describe_core(int n_blocks, int L_cap, int D, int rank, const double *K,
+                                const int32_t *L_eff, const double *U, int sd, double *mu, double *xi,
+                                double *lam)
 {
 #pragma omp parallel
     {
         double *Kt = (double *)malloc(sizeof(double) * (size_t)L_cap * D);
+        double *Y = (double *)malloc(sizeof(double) * (size_t)L_cap * sd);
         double *G = (double *)malloc(sizeof(double) * (size_t)L_cap * L_cap);
         double *W = (double *)malloc(sizeof(double) * (size_t)L_cap * L_cap);
         int *order = (int *)malloc(sizeof(int) * (size_t)L_cap);
@@ -415,11 +421,22 @@ OAPI void oracle_block_describe(int n_blocks, int L_cap, int D, int rank, const 
             for (int r = 0; r < L; ++r)
                 for (int t = 0; t < D; ++t)
                     Kt[(long)r * D + t] = Kb[(long)r * D + t] - m[t];
+            for (int r = 0; r < L; ++r)
+                for (int j = 0; j < sd; ++j) {
+                    if (!U) {
+                        Y[(long)r * sd + j] = Kt[(long)r * D + j];
+                        continue;
+                    }
+                    double acc = 0.0;
+                    for (int t = 0; t < D; ++t)
+                        acc += Kt[(long)r * D + t] * U[(long)t * sd + j];
+                    Y[(long)r * sd + j] = acc;
+                }
             for (int i = 0; i < L; ++i)
                 for (int j = 0; j < L; ++j) {
                     double acc = 0.0;
-                    for (int t = 0; t < D; ++t)
-                        acc += Kt[(long)i * D + t] * Kt[(long)j * D + t];
+                    for (int t = 0; t < sd; ++t)
+                        acc += Y[(long)i * sd + t] * Y[(long)j * sd + t];
                     G[i * L + j] = acc / L;
                 }
             if (L > 0)
@@ -437,28 +454,45 @@ OAPI void oracle_block_describe(int n_blocks, int L_cap, int D, int rank, const 
                 order[best] = tmp;
             }
             for (int e = 0; e < rank; ++e) {
-                double *x = xi + (b * (long)rank + e) * D;
+                double *x = xi + (b * (long)rank + e) * sd;
                 if (e >= L) {
-                    for (int t = 0; t < D; ++t)
+                    for (int t = 0; t < sd; ++t)
                         x[t] = 0.0;
                     lam[b * (long)rank + e] = 0.0;
                     continue;
                 }
                 const int col = order[e];
                 lam[b * (long)rank + e] = G[col * L + col];
-                for (int t = 0; t < D; ++t) {
+                for (int t = 0; t < sd; ++t) {
                     double acc = 0.0;
                     for (int r = 0; r < L; ++r)
-                        acc += Kt[(long)r * D + t] * W[r * L + col];
+                        acc += Y[(long)r * sd + t] * W[r * L + col];
                     x[t] = acc / sqrt((double)L);
                 }
             }
         }
         free(Kt);
+        free(Y);
         free(G);
         free(W);
         free(order);
     }
+}
+
+OAPI void oracle_block_describe(int n_blocks, int L_cap, int D, int rank, const double *K,
+                                const int32_t *L_eff, double *mu, double *xi, double *lam)
+{
+    block_describe_core(n_blocks, L_cap, D, rank, K, L_eff, NULL, D, mu, xi, lam);
+}
+
+/* O5s  Subspace descriptors ([P5] "子空间方法", Eq.(17)-(18)): U [D, sd] holds
+ * the query-subspace basis (orthonormal columns, computed offline from the
+ * queries' second moment); xi [n_blocks, rank, sd] are the scaled top-rank
+ * eigenvectors of U^T Sigma_b U; mu as in O5. */
+OAPI void oracle_block_describe_ss(int n_blocks, int L_cap, int D, int sd, int rank, const double *K,
+                                   const double *U, double *mu, double *xi, double *lam)
+{
+    block_describe_core(n_blocks, L_cap, D, rank, K, NULL, U, sd, mu, xi, lam);
 }
 
 /* Exact block log-mass, [P5] Eq.(1): ln m_b = ln sum_{r in b} exp(q . k_r).
@@ -499,14 +533,16 @@ OAPI double oracle_block_log_mass(int L, int D, const double *q, const double *K
  * tok_count [n_seq, n_kv], blk [n_seq, n_kv, top_blocks] (ascending),
  * blk_score [n_seq, n_kv, n_full].
  * ====================================================================== */
-enum { SEL_COBS = 0, SEL_QUEST = 1 };
+enum { SEL_COBS = 0, SEL_QUEST = 1, SEL_SUBSPACE = 2 };
 
 /* One query head's block score s_{g,b} for selector `kind`:
  *   SEL_COBS:  qt . A_b + 1/2 sum_i (B_{b,i} . qt)^2      (A = mu, B = xi, [P5] Eq.(14)/(19);
  *              rank 0 is the mean-pool selector qt . kbar_b, [P5] Table 1)
- *   SEL_QUEST: sum_t max(qt_t A_{b,t}, qt_t B_{b,t})       (A = kmin, B = kmax, [P5] Eq.(24)) */
-static double head_block_score(int kind, int D, int rank, const double *qt, const double *A,
-                               const double *B)
+ *   SEL_QUEST: sum_t max(qt_t A_{b,t}, qt_t B_{b,t})       (A = kmin, B = kmax, [P5] Eq.(24))
+ *   SEL_SUBSPACE: qt . A_b + 1/2 sum_i (B_{b,i} . qs)^2    (B = xi in R^sd, qs = U^T qt,
+ *              [P5] Eq.(18): q^T Sigma q ~ qs^T B_b qs) */
+static double head_block_score(int kind, int D, int rank, int sd, const double *qt, const double *qs,
+                               const double *A, const double *B)
 {
     double v = 0.0;
     if (kind == SEL_QUEST) {
@@ -518,27 +554,30 @@ static double head_block_score(int kind, int D, int rank, const double *qt, cons
     }
     for (int t = 0; t < D; ++t)
         v += qt[t] * A[t];
+    const double *qq = kind == SEL_SUBSPACE ? qs : qt;
+    const int n = kind == SEL_SUBSPACE ? sd : D;
     double quad = 0.0;
     for (int e = 0; e < rank; ++e) {
-        const double *x = B + (long)e * D;
+        const double *x = B + (long)e * n;
         double p = 0.0;
-        for (int t = 0; t < D; ++t)
-            p += x[t] * qt[t];
+        for (int t = 0; t < n; ++t)
+            p += x[t] * qq[t];
         quad += p * p;
     }
     return v + 0.5 * quad;
 }
 
-static void block_select_run(int kind, int n_seq, int n_kv, int n_q, int D, int rank, int n_full,
-                             int L, int T, int top_blocks, int window, double scale, const double *Q,
-                             const double *Ab, const double *Bb, int cap, int32_t *tok,
-                             int32_t *tok_count, int32_t *blk, double *blk_score)
+static void block_select_run(int kind, int n_seq, int n_kv, int n_q, int D, int rank, int sd,
+                             const double *U, int n_full, int L, int T, int top_blocks, int window,
+                             double scale, const double *Q, const double *Ab, const double *Bb, int cap,
+                             int32_t *tok, int32_t *tok_count, int32_t *blk, double *blk_score)
 {
     const int G = n_q / n_kv;
 #pragma omp parallel
     {
         double *s = (double *)malloc(sizeof(double) * (size_t)n_full);
         double *qt = (double *)malloc(sizeof(double) * (size_t)D);
+        double *qs = (double *)malloc(sizeof(double) * (size_t)(sd > 0 ? sd : 1));
         scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(n_full > 0 ? n_full : 1));
         uint8_t *mark = (uint8_t *)malloc((size_t)(T > 0 ? T : 1));
 #pragma omp for collapse(2) schedule(dynamic, 1)
@@ -552,13 +591,21 @@ static void block_select_run(int kind, int n_seq, int n_kv, int n_q, int D, int 
                     const double *q = Q + ((long)sq * n_q + g) * D;
                     for (int t = 0; t < D; ++t)
                         qt[t] = scale * q[t];
+                    if (kind == SEL_SUBSPACE)
+                        for (int j = 0; j < sd; ++j) {
+                            double acc = 0.0;
+                            for (int t = 0; t < D; ++t)
+                                acc += U[(long)t * sd + j] * qt[t];
+                            qs[j] = acc;
+                        }
                     double mx = -INFINITY;
                     for (int b = 0; b < n_full; ++b) {
                         const long blkid = sh * n_full + b;
                         const double *a = Ab + blkid * (long)D;
-                        const double *bb = kind == SEL_QUEST ? Bb + blkid * (long)D
-                                                             : Bb + blkid * (long)rank * D;
-                        s[b] = head_block_score(kind, D, rank, qt, a, bb);
+                        const double *bb = kind == SEL_QUEST      ? Bb + blkid * (long)D
+                                           : kind == SEL_SUBSPACE ? Bb + blkid * (long)rank * sd
+                                                                  : Bb + blkid * (long)rank * D;
+                        s[b] = head_block_score(kind, D, rank, sd, qt, qs, a, bb);
                         if (s[b] > mx) mx = s[b];
                     }
                     double z = 0.0;
@@ -599,6 +646,7 @@ static void block_select_run(int kind, int n_seq, int n_kv, int n_q, int D, int 
         }
         free(s);
         free(qt);
+        free(qs);
         free(sc);
         free(mark);
     }
@@ -610,8 +658,20 @@ OAPI void oracle_block_select(int n_seq, int n_kv, int n_q, int D, int rank, int
                               const double *mu, const double *xi, int cap, int32_t *tok,
                               int32_t *tok_count, int32_t *blk, double *blk_score)
 {
-    block_select_run(SEL_COBS, n_seq, n_kv, n_q, D, rank, n_full, L, T, top_blocks, window, scale,
-                     Q, mu, xi, cap, tok, tok_count, blk, blk_score);
+    block_select_run(SEL_COBS, n_seq, n_kv, n_q, D, rank, D, NULL, n_full, L, T, top_blocks, window,
+                     scale, Q, mu, xi, cap, tok, tok_count, blk, blk_score);
+}
+
+/* O6s  Subspace block selection: O6 with the quadratic term of [P5] Eq.(18),
+ * (xi_i . U^T qt)^2 with xi in R^sd (from O5s).  U [D, sd]; xi [n_seq, n_kv,
+ * n_full, rank, sd]; other layouts as O6. */
+OAPI void oracle_block_select_ss(int n_seq, int n_kv, int n_q, int D, int sd, int rank, int n_full,
+                                 int L, int T, int top_blocks, int window, double scale, const double *Q,
+                                 const double *U, const double *mu, const double *xi, int cap,
+                                 int32_t *tok, int32_t *tok_count, int32_t *blk, double *blk_score)
+{
+    block_select_run(SEL_SUBSPACE, n_seq, n_kv, n_q, D, rank, sd, U, n_full, L, T, top_blocks, window,
+                     scale, Q, mu, xi, cap, tok, tok_count, blk, blk_score);
 }
 
 /* ======================================================================
@@ -652,8 +712,8 @@ OAPI void oracle_quest_select(int n_seq, int n_kv, int n_q, int D, int n_full, i
                               const double *kmin, const double *kmax, int cap, int32_t *tok,
                               int32_t *tok_count, int32_t *blk, double *blk_score)
 {
-    block_select_run(SEL_QUEST, n_seq, n_kv, n_q, D, 0, n_full, L, T, top_blocks, window, scale, Q,
-                     kmin, kmax, cap, tok, tok_count, blk, blk_score);
+    block_select_run(SEL_QUEST, n_seq, n_kv, n_q, D, 0, D, NULL, n_full, L, T, top_blocks, window,
+                     scale, Q, kmin, kmax, cap, tok, tok_count, blk, blk_score);
 }
 
 /* ======================================================================
