@@ -1,7 +1,7 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|prefill|decode|block|block_fp4|block_quest|block_meanpool] [--no-extras]
+                  [--workload lsh|lsh_fp32|prefill|decode|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
@@ -13,6 +13,7 @@ A step is one pass of the hot path over one batch of the workload:
   block    block-mass decode: block select (top-64 + 512 window) + GQA attention;
            the descriptor build is timed separately (it runs once per filled block).
   block_fp4 the same on bf16 means + FP4 (E2M1) eigenvectors (528 B per block).
+  block_ss  the same on descriptors in a query subspace of 85 dims (fp32).
   block_quest / block_meanpool  the same step with the baseline selectors (Quest boxes;
            block means alone).
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on
@@ -368,6 +369,43 @@ class BlockQuestWorkload(BlockWorkload):
         return spec
 
 
+class BlockSubspaceWorkload(BlockWorkload):
+    """COBS descriptors in a query subspace of s = 85 dims: fp32 mean (512 B) and four
+    scaled eigenvectors of U^T Sigma U (4 x 85 x 4 B) per block."""
+    SD = 85
+
+    def __init__(self, crs, dev):
+        import workloads
+        self.U = workloads.query_subspace(128, self.SD, device=dev)
+        super().__init__(crs, dev)
+        self.name = self.c["workload"].replace("block_", f"block_ss{self.SD}_", 1)
+        import ctypes
+        p = self.p
+        bp = crs.BlockSelParams(crs.BlockParams(p["n_seq"], p["n_kv_heads"], p["T"], p["D"], p["L"],
+                                                p["rank"], 0, p["T"] // p["L"]),
+                                p["n_q_heads"], p["top_blocks"], p["window"], p["scale"])
+        self.ws = torch.empty(int(crs.lib().crs_block_select_ss_workspace_size(ctypes.byref(bp), self.SD)),
+                              dtype=torch.uint8, device=dev)
+
+    def _build_cache(self):
+        self.mu, self.xi = self.crs.block_describe_ss(self.c["K"], self.p["L"], self.p["rank"], self.U)
+
+    def _run(self, Q):
+        p = self.p
+        self.crs.block_select_ss(Q, self.U, self.mu, self.xi, p["T"], p["L"], p["top_blocks"], p["window"],
+                                 tok=self.tok, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
+                             workspace=self.ws2)
+
+    def roofline_spec(self):
+        p = self.p
+        spec = super().roofline_spec()
+        per_block = p["D"] * 4 + p["rank"] * self.SD * 4
+        spec["block_score"] = [("hbm", p["n_seq"] * p["n_kv_heads"] * (p["T"] // p["L"]) * per_block / 1e9,
+                                "GB/s")]
+        return spec
+
+
 class BlockMeanPoolWorkload(BlockWorkload):
     """Baseline selector: the block mean alone (first-order score, fp32, 512 B per block)."""
 
@@ -391,7 +429,7 @@ WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
              "prefill": PrefillWorkload, "decode": DecodeWorkload, "block": BlockWorkload,
              "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
-             "block_meanpool": BlockMeanPoolWorkload}
+             "block_meanpool": BlockMeanPoolWorkload, "block_ss": BlockSubspaceWorkload}
 
 
 # ------------------------------------------------------------------- timing --
@@ -653,8 +691,8 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block", "block_fp4", "block_quest",
-                                  "block_meanpool") if w != args.workload]:
+        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block", "block_fp4", "block_ss",
+                                  "block_quest", "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)
                 r2 = measure(crs, w2, 5, 3, flush_buf, False, peaks)

@@ -115,6 +115,11 @@ _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP
 _sig("crs_block_quantize", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP, _VP, _VP])
 _sig("crs_block_select_fp4", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                              _VP, _VP, _SZ, _VP])
+_sig("crs_block_describe_ss", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, ctypes.c_int, _VP, _VP,
+                                              _VP])
+_sig("crs_block_select_ss_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams), ctypes.c_int])
+_sig("crs_block_select_ss", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, ctypes.c_int, _VP, _VP,
+                                            _VP, _VP, _VP, _SZ, _VP])
 _sig("crs_block_quest_describe", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP])
 _sig("crs_block_select_quest", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                                _VP, _SZ, _VP])
@@ -348,6 +353,55 @@ def block_select(Q, mu, xi, T: int, L: int, top_blocks: int, window: int, scale=
     st = _lib.crs_block_select(ctypes.byref(p), _ptr(Q), _ptr(mu), _ptr(xi), _ptr(tok),
                                _ptr(count), _ptr(ws), wsb, _stream(stream))
     _check("crs_block_select", st)
+    return tok, count
+
+
+def block_describe_ss(K, L: int, rank: int, U, out=None, stream=None):
+    """Query-subspace descriptors: K [n_seq, T, n_kv, D] bf16, U [D, s] f32 ->
+    (mu [n_seq, n_kv, T//L, D], xi_ss [n_seq, n_kv, T//L, rank, s]) f32."""
+    _need(K, "K", torch.bfloat16)
+    n_seq, T, n_kv, D = K.shape
+    _need(U, "U", torch.float32)
+    sd = U.shape[1]
+    _need(U, "U", torch.float32, (D, sd))
+    nfull = T // L
+    if out is None:
+        out = (torch.empty((n_seq, n_kv, nfull, D), dtype=torch.float32, device=K.device),
+               torch.empty((n_seq, n_kv, nfull, rank, sd), dtype=torch.float32, device=K.device))
+    mu, xi = out
+    _need(mu, "mu", torch.float32, (n_seq, n_kv, nfull, D))
+    _need(xi, "xi_ss", torch.float32, (n_seq, n_kv, nfull, rank, sd))
+    p = BlockParams(n_seq, n_kv, int(T), D, int(L), int(rank), 0, nfull)
+    _check("crs_block_describe_ss", _lib.crs_block_describe_ss(ctypes.byref(p), _ptr(K), _ptr(U), sd, _ptr(mu),
+                                                               _ptr(xi), _stream(stream)))
+    return mu, xi
+
+
+def block_select_ss(Q, U, mu, xi_ss, T: int, L: int, top_blocks: int, window: int, scale=None,
+                    tok=None, count=None, workspace=None, stream=None):
+    """block_select on query-subspace descriptors (from block_describe_ss)."""
+    _need(Q, "Q", torch.bfloat16)
+    n_seq, n_q, D = Q.shape
+    n_kv, nfull, rank, sd = xi_ss.shape[1], xi_ss.shape[2], xi_ss.shape[3], xi_ss.shape[4]
+    _need(U, "U", torch.float32, (D, sd))
+    _need(mu, "mu", torch.float32, (n_seq, n_kv, nfull, D))
+    _need(xi_ss, "xi_ss", torch.float32, (n_seq, n_kv, nfull, rank, sd))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull), n_q,
+                       int(top_blocks), int(window), float(scale))
+    cap = top_blocks * L + window
+    if tok is None:
+        tok = torch.empty((n_seq, n_kv, cap), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((n_seq, n_kv), dtype=torch.int32, device=Q.device)
+    _need(tok, "tok", torch.int32, (n_seq, n_kv, cap))
+    _need(count, "count", torch.int32, (n_seq, n_kv))
+    ws, wsb = _workspace(int(_lib.crs_block_select_ss_workspace_size(ctypes.byref(p), sd)), Q.device,
+                         workspace)
+    st = _lib.crs_block_select_ss(ctypes.byref(p), _ptr(Q), _ptr(U), sd, _ptr(mu), _ptr(xi_ss), _ptr(tok),
+                                  _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_block_select_ss", st)
     return tok, count
 
 

@@ -33,14 +33,28 @@ struct BdWarpSmem {
     float rc[kBdMaxL], rs[kBdMaxL];
     int partner[kBdMaxL];
 };
+// subspace descriptors ([P5] Eq.(17)): the projected centred keys Y = Kt U (L x sd)
+struct BdWarpSmemSS {
+    float y[kBdMaxL][kBdD + 1];
+};
 
+// SS: the eigenvectors are those of U^T Sigma U, taken by the same Gram route on
+// Y = Kt U (U [D, sd] staged once per CTA in shared memory, after the warps'
+// areas); xi then has sd entries per vector.
+template <bool SS>
 __global__ void __launch_bounds__(kBdWarps * 32)
 block_describe_kernel(const __nv_bfloat16 *__restrict__ K, float *__restrict__ mu_out,
                       float *__restrict__ xi_out, int n_kv, int T, int L, int rank, int blk_begin,
-                      int n_blk, int n_full) {
+                      int n_blk, int n_full, const float *__restrict__ U, int sd) {
     extern __shared__ __align__(16) unsigned char bd_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     BdWarpSmem &S = reinterpret_cast<BdWarpSmem *>(bd_smem)[warp];
+    BdWarpSmemSS *SY = reinterpret_cast<BdWarpSmemSS *>(bd_smem + kBdWarps * sizeof(BdWarpSmem));
+    float *sU = reinterpret_cast<float *>(bd_smem + kBdWarps * (sizeof(BdWarpSmem) + sizeof(BdWarpSmemSS)));
+    if constexpr (SS) {
+        for (int e = threadIdx.x; e < kBdD * sd; e += kBdWarps * 32) sU[e] = U[e];
+        __syncthreads();
+    }
     const long long item = (long long)blockIdx.x * kBdWarps + warp;
     const int sh = blockIdx.y;                 // seq * n_kv + h
     if (item >= n_blk) return;
@@ -62,17 +76,37 @@ block_describe_kernel(const __nv_bfloat16 *__restrict__ K, float *__restrict__ m
         S.mu[d] = acc * invL;
     }
     __syncwarp();
-    // Gram row `lane`: G[i][j] = (1/L) sum_d Kt[i][d] Kt[j][d]
+    if constexpr (SS) {
+        // Y[r][j] = sum_d Kt[r][d] U[d][j]; lane owns columns j = lane, lane + 32, ...
+        for (int j = lane; j < sd; j += 32)
+            for (int r = 0; r < L; ++r) {
+                float acc = 0.0f;
+                for (int d = 0; d < kBdD; ++d)
+                    acc = fmaf(__bfloat162float(S.k[r][d]) - S.mu[d], sU[d * sd + j], acc);
+                SY[warp].y[r][j] = acc;
+            }
+        __syncwarp();
+    }
+    // Gram row `lane`: G[i][j] = (1/L) sum_d Kt[i][d] Kt[j][d]  (SS: over Y's sd columns)
     if (lane < L) {
         float grow[kBdMaxL];
 #pragma unroll
         for (int j = 0; j < kBdMaxL; ++j) grow[j] = 0.0f;
-        for (int d = 0; d < kBdD; ++d) {
-            const float md = S.mu[d];
-            const float ki = __bfloat162float(S.k[lane][d]) - md;
+        if constexpr (SS) {
+            for (int t = 0; t < sd; ++t) {
+                const float yi = SY[warp].y[lane][t];
 #pragma unroll
-            for (int j = 0; j < kBdMaxL; ++j)
-                if (j < L) grow[j] = fmaf(ki, __bfloat162float(S.k[j][d]) - md, grow[j]);
+                for (int j = 0; j < kBdMaxL; ++j)
+                    if (j < L) grow[j] = fmaf(yi, SY[warp].y[j][t], grow[j]);
+            }
+        } else {
+            for (int d = 0; d < kBdD; ++d) {
+                const float md = S.mu[d];
+                const float ki = __bfloat162float(S.k[lane][d]) - md;
+#pragma unroll
+                for (int j = 0; j < kBdMaxL; ++j)
+                    if (j < L) grow[j] = fmaf(ki, __bfloat162float(S.k[j][d]) - md, grow[j]);
+            }
         }
 #pragma unroll
         for (int j = 0; j < kBdMaxL; ++j)
@@ -175,15 +209,20 @@ block_describe_kernel(const __nv_bfloat16 *__restrict__ K, float *__restrict__ m
             if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
         }
         if (lane == bi) taken = true;
-        float *xo = xi_out + (dbase * rank + e) * kBdD;
+        const int xd = SS ? sd : kBdD;
+        float *xo = xi_out + (dbase * rank + e) * xd;
         if (e >= L || bi >= L) {
-            for (int d = lane; d < kBdD; d += 32) xo[d] = 0.0f;
+            for (int d = lane; d < xd; d += 32) xo[d] = 0.0f;
             continue;
         }
-        for (int d = lane; d < kBdD; d += 32) {
-            const float md = S.mu[d];
+        for (int d = lane; d < xd; d += 32) {
             float acc = 0.0f;
-            for (int r = 0; r < L; ++r) acc = fmaf(__bfloat162float(S.k[r][d]) - md, S.v[r][bi], acc);
+            if constexpr (SS) {
+                for (int r = 0; r < L; ++r) acc = fmaf(SY[warp].y[r][d], S.v[r][bi], acc);
+            } else {
+                const float md = S.mu[d];
+                for (int r = 0; r < L; ++r) acc = fmaf(__bfloat162float(S.k[r][d]) - md, S.v[r][bi], acc);
+            }
             xo[d] = acc * rs_L;
         }
     }
@@ -196,35 +235,49 @@ block_describe_kernel(const __nv_bfloat16 *__restrict__ K, float *__restrict__ m
 // memory (rows padded by one float against bank conflicts).
 // ---------------------------------------------------------------------------
 constexpr int kBsThreads = 128;
+constexpr int kBsMaxTile = 32;              // blocks per CTA at most (G = 1 would stage 128)
+__host__ __device__ inline int bs_tile(int G) { return min(kBsThreads / G, kBsMaxTile); }
 
+// xdim: entries per eigenvector (D, or the subspace size with qx != nullptr:
+// the queries projected and scaled, [n_seq * n_q][xdim], [P5] Eq.(18)).
 __global__ void __launch_bounds__(kBsThreads)
 block_score_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ mu,
                    const float *__restrict__ xi, float *__restrict__ sc_out, int n_kv, int n_q,
-                   int G, int rank, int n_full, float scale) {
+                   int G, int rank, int n_full, float scale, int xdim, const float *__restrict__ qx) {
     extern __shared__ float bs_smem[];
-    const int nbt = kBsThreads / G;             // blocks per CTA
+    const int nbt = bs_tile(G);                 // blocks per CTA
     const int DP = kBdD + 1;
     float *sq = bs_smem;                        // [G][DP]
-    float *sd = sq + G * DP;                    // [nbt][(1+rank)][DP]
+    float *sqx = sq + G * DP;                   // [G][DP] projected queries (subspace)
+    float *sd = sqx + G * DP;                   // [nbt][(1+rank)][DP]
     const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
     const int b0 = blockIdx.x * nbt;
     const int nb = min(nbt, n_full - b0);
     for (int e = threadIdx.x; e < G * kBdD; e += kBsThreads) {
         const int g = e / kBdD, d = e - g * kBdD;
-        sq[g * DP + d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+        const size_t row = (size_t)seq * n_q + h * G + g;
+        sq[g * DP + d] = scale * __bfloat162float(Q[row * kBdD + d]);
+        if (qx && d < xdim) sqx[g * DP + d] = qx[row * xdim + d];
     }
     const int rows = 1 + rank;
-    for (int e = threadIdx.x; e < nb * rows * kBdD; e += kBsThreads) {
-        const int bl = e / (rows * kBdD), rem = e - bl * rows * kBdD;
-        const int rr = rem / kBdD, d = rem - rr * kBdD;
-        const size_t blk = (size_t)sh * n_full + b0 + bl;
-        sd[(bl * rows + rr) * DP + d] =
-            (rr == 0) ? mu[blk * kBdD + d] : xi[(blk * rank + (rr - 1)) * kBdD + d];
+    {   // every descriptor row of the tile in flight at once (4-byte async copies
+        // into the padded rows); warp w copies rows w, w + 4, ...
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        for (int row = warp; row < nb * rows; row += kBsThreads / 32) {
+            const int bl = row / rows, rr = row - bl * rows;
+            const size_t blk = (size_t)sh * n_full + b0 + bl;
+            const float *src = rr == 0 ? mu + blk * kBdD : xi + (blk * rank + (rr - 1)) * xdim;
+            const int len = rr == 0 ? kBdD : xdim;
+            for (int d = lane; d < len; d += 32) cp_async4(&sd[row * DP + d], src + d);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
     }
     __syncthreads();
     const int bl = threadIdx.x / G, g = threadIdx.x - bl * G;
     if (bl >= nb) return;
     const float *q = sq + g * DP;
+    const float *qq = qx ? sqx + g * DP : q;
     const float *dsc = sd + bl * rows * DP;
     float lin = 0.0f;
     for (int d = 0; d < kBdD; ++d) lin = fmaf(q[d], dsc[d], lin);
@@ -232,10 +285,24 @@ block_score_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict_
     for (int e = 0; e < rank; ++e) {
         float p = 0.0f;
         const float *x = dsc + (1 + e) * DP;
-        for (int d = 0; d < kBdD; ++d) p = fmaf(q[d], x[d], p);
+        for (int d = 0; d < xdim; ++d) p = fmaf(qq[d], x[d], p);
         quad = fmaf(p, p, quad);
     }
     sc_out[((size_t)sh * G + g) * n_full + b0 + bl] = fmaf(0.5f, quad, lin);
+}
+
+// qx[row][j] = sum_d U[d][j] scale q[row][d]: one warp per query row, lanes over j.
+__global__ void __launch_bounds__(256)
+query_project_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ U,
+                     float *__restrict__ qx, int n_rows, int sd, float scale) {
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= n_rows) return;
+    const __nv_bfloat16 *q = Q + (size_t)row * kBdD;
+    for (int j = lane; j < sd; j += 32) {
+        float acc = 0.0f;
+        for (int d = 0; d < kBdD; ++d) acc = fmaf(U[(size_t)d * sd + j], scale * __bfloat162float(q[d]), acc);
+        qx[(size_t)row * sd + j] = acc;
+    }
 }
 
 // K9a specialised for G query heads and rank R, streaming the descriptors
@@ -1076,14 +1143,40 @@ extern "C" int crs_block_describe(const crs_block_params *p, const void *K, floa
     if (n_blk == 0) return CRS_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t smem = sizeof(BdWarpSmem) * kBdWarps;
-    CRS_TRY_CUDA(cudaFuncSetAttribute(block_describe_kernel,
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_describe_kernel<false>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     dim3 grid(ceil_div(n_blk, kBdWarps), p->n_seq * p->n_kv);
     {
         ProfScope _ps(K_BLK_DESCRIBE, s);
-        block_describe_kernel<<<grid, kBdWarps * 32, smem, s>>>(
+        block_describe_kernel<false><<<grid, kBdWarps * 32, smem, s>>>(
             static_cast<const __nv_bfloat16 *>(K), mu, xi, p->n_kv, p->T, p->L, p->rank, p->blk_begin,
-            n_blk, n_full);
+            n_blk, n_full, nullptr, 0);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+
+extern "C" int crs_block_describe_ss(const crs_block_params *p, const void *K, const float *U, int sd,
+                                     float *mu, float *xi_ss, void *stream) {
+    int st = bd_validate(p);
+    if (st) return st;
+    if (!K || !U || !mu || !xi_ss) return CRS_ERR_INVALID_ARG;
+    if (sd < 1 || sd > kBdD) return CRS_ERR_INVALID_ARG;
+    const int n_full = p->T / p->L;
+    if (p->blk_begin < 0 || p->blk_end > n_full || p->blk_begin > p->blk_end)
+        return CRS_ERR_INVALID_ARG;
+    const int n_blk = p->blk_end - p->blk_begin;
+    if (n_blk == 0) return CRS_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t smem = (sizeof(BdWarpSmem) + sizeof(BdWarpSmemSS)) * kBdWarps + (size_t)kBdD * sd * 4;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_describe_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid(ceil_div(n_blk, kBdWarps), p->n_seq * p->n_kv);
+    {
+        ProfScope _ps(K_BLK_DESCRIBE, s);
+        block_describe_kernel<true><<<grid, kBdWarps * 32, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(K), mu, xi_ss, p->n_kv, p->T, p->L, p->rank, p->blk_begin,
+            n_blk, n_full, U, sd);
     }
     CRS_CHECK_LAUNCH();
     return CRS_OK;
@@ -1153,8 +1246,8 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
         }
         return launch_block_pick(p, sc, tok_idx, tok_count, s);
     }
-    const int nbt = kBsThreads / G;
-    const size_t smem_a = ((size_t)G * (kBdD + 1) + (size_t)nbt * (1 + p->b.rank) * (kBdD + 1)) * 4;
+    const int nbt = bs_tile(G);
+    const size_t smem_a = ((size_t)2 * G * (kBdD + 1) + (size_t)nbt * (1 + p->b.rank) * (kBdD + 1)) * 4;
     if (smem_a > 227 * 1024) return CRS_ERR_UNSUPPORTED;
     CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a));
@@ -1176,7 +1269,7 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
         ProfScope _ps(K_BLK_SCORE, s);
         block_score_kernel<<<ga, kBsThreads, smem_a, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu, xi,
                                                           sc, p->b.n_kv, p->n_q, G, p->b.rank, n_full,
-                                                          p->scale);
+                                                          p->scale, kBdD, nullptr);
     }
     }
     CRS_CHECK_LAUNCH();
@@ -1321,5 +1414,44 @@ extern "C" int crs_block_select_quest(const crs_block_sel_params *p, const void 
         CRS_TRY_CUDA(launch_score_warp<kWsQuest>(G, score_warp_grid(G, n_full, p->b.n_seq * p->b.n_kv), s, Q,
                                                  kmin, kmax, sc, p->b.n_kv, p->n_q, n_full, p->scale));
     }
+    return launch_block_pick(p, sc, tok_idx, tok_count, s);
+}
+
+extern "C" size_t crs_block_select_ss_workspace_size(const crs_block_sel_params *p, int sd) {
+    const size_t sc = crs_block_select_workspace_size(p);
+    if (sc == 0 || sd < 1 || sd > kBdD) return 0;
+    return ((sc + 255) & ~size_t(255)) + (size_t)p->b.n_seq * p->n_q * sd * sizeof(float);
+}
+
+extern "C" int crs_block_select_ss(const crs_block_sel_params *p, const void *Q, const float *U, int sd,
+                                   const float *mu, const float *xi_ss, int32_t *tok_idx, int32_t *tok_count,
+                                   void *ws, size_t ws_bytes, void *stream) {
+    int st = bs_validate(p);
+    if (st) return st;
+    if (p->b.rank < 1) return CRS_ERR_INVALID_ARG;
+    if (!Q || !U || !mu || !xi_ss || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
+    if (sd < 1 || sd > kBdD) return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_block_select_ss_workspace_size(p, sd);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int G = p->n_q / p->b.n_kv, n_full = p->b.T / p->b.L;
+    float *sc = static_cast<float *>(ws);
+    float *qx = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                          ((crs_block_select_workspace_size(p) + 255) & ~size_t(255)));
+    const int n_rows = p->b.n_seq * p->n_q;
+    const int nbt = bs_tile(G);
+    const size_t smem_a = ((size_t)2 * G * (kBdD + 1) + (size_t)nbt * (1 + p->b.rank) * (kBdD + 1)) * 4;
+    if (smem_a > 227 * 1024) return CRS_ERR_UNSUPPORTED;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem_a));
+    {
+        ProfScope _ps(K_BLK_SCORE, s);
+        query_project_kernel<<<ceil_div(n_rows, 8), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Q), U, qx,
+                                                                  n_rows, sd, p->scale);
+        block_score_kernel<<<dim3(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv), kBsThreads, smem_a, s>>>(
+            static_cast<const __nv_bfloat16 *>(Q), mu, xi_ss, sc, p->b.n_kv, p->n_q, G, p->b.rank, n_full,
+            p->scale, sd, qx);
+    }
+    CRS_CHECK_LAUNCH();
     return launch_block_pick(p, sc, tok_idx, tok_count, s);
 }

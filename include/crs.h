@@ -301,6 +301,24 @@ int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q, const voi
                          int32_t *tok_count, void *ws, size_t ws_bytes, void *stream);
 
 /* ====================================================================== *
+ * Query-subspace descriptors ([P5] "子空间方法", Eq.(17)-(18)).  U: [D, sd] f32
+ * (row-major), orthonormal columns spanning the query subspace (the top sd
+ * eigenvectors of the queries' second moment, computed offline; an input).
+ * crs_block_describe_ss: mu as crs_block_describe; xi_ss [n_seq, n_kv, T/L,
+ * rank, sd] f32 = the rank scaled eigenvectors of B_b = U^T Sigma_b U, formed
+ * by the Gram route on the projected centred keys Y = Kt U (1 <= sd <= D).
+ * crs_block_select_ss: the crs_block_select rule with the quadratic term
+ * (xi_i . U^T qt)^2 ([P5] Eq.(18)); workspace from
+ * crs_block_select_ss_workspace_size (scores + projected queries).
+ * ====================================================================== */
+int crs_block_describe_ss(const crs_block_params *p, const void *K, const float *U, int sd, float *mu,
+                          float *xi_ss, void *stream);
+size_t crs_block_select_ss_workspace_size(const crs_block_sel_params *p, int sd);
+int crs_block_select_ss(const crs_block_sel_params *p, const void *Q, const float *U, int sd,
+                        const float *mu, const float *xi_ss, int32_t *tok_idx, int32_t *tok_count,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/* ====================================================================== *
  * Quest box selector ([P5] Quest section, Eq.(23)-(24), Table 1).
  * crs_block_quest_describe: per complete block b of L keys and KV head h the
  * element-wise minimum and maximum of its keys, kmin_b, kmax_b (the keys'

@@ -294,3 +294,62 @@ def test_select_quest_full_config_sampled(crs, cuda_dev):
                                                     kmax.double().cpu().numpy()[seqs], T, L, top, win)
     _check_select(tok.cpu().numpy()[seqs], cnt.cpu().numpy()[seqs], o_tok, o_cnt, o_blk, o_bs, L, T,
                   win, top, "quest-full")
+
+
+# ---------------------------------------------------------------- query subspace --
+def test_describe_ss_matches_oracle(crs, cuda_dev):
+    """Subspace descriptors (s = 85 of D = 128): the mean, the eigenvalues of U^T Sigma U and
+    the rank-r factor sum xi xi^T (where the r-th eigengap is clear of fp32 noise)."""
+    case = workloads.block_decode_case(n_seq=2, T=32 * 40 + 7, seed=14, device=cuda_dev)
+    p = case["params"]
+    L, r = p["L"], p["rank"]
+    U = workloads.query_subspace(128, 85, device=cuda_dev)
+    mu, xi = crs.block_describe_ss(case["K"], L, r, U)
+    torch.cuda.synchronize()
+    kb = _blocks(_np(case["K"]), L)
+    s_, h_, nf = kb.shape[:3]
+    omu, oxi, olam = oracle.block_describe_ss(kb.reshape(-1, L, 128), U.double().cpu().numpy(), r + 1)
+    omu, oxi, olam = omu.reshape(s_, h_, nf, -1), oxi.reshape(s_, h_, nf, r + 1, -1), olam.reshape(s_, h_, nf, r + 1)
+    assert rel_err(_np(mu), omu).max() < 1e-5
+    g = _np(xi)
+    assert np.abs((g ** 2).sum(-1) - olam[..., :r]).max() <= 1e-4 * olam[..., 0].max()
+    gap = (olam[..., r - 1] - olam[..., r]) / olam[..., 0]
+    P = np.einsum("shbrd,shbre->shbde", g, g)
+    Po = np.einsum("shbrd,shbre->shbde", oxi[..., :r, :], oxi[..., :r, :])
+    err = np.abs(P - Po).max(axis=(-1, -2)) / olam[..., 0]
+    ok = gap > 1e-3
+    assert ok.mean() > 0.9
+    assert (err[ok] <= 1e-4 / gap[ok]).all()
+
+
+@pytest.mark.parametrize("n_q,n_kv,T,top,win,sd", [(32, 4, 4096, 16, 256, 85), (16, 4, 32 * 300 + 5, 20, 64, 48),
+                                                   (4, 4, 32 * 90, 9, 100, 128)])
+def test_select_ss_matches_oracle(crs, cuda_dev, n_q, n_kv, T, top, win, sd):
+    case = workloads.block_decode_case(n_seq=3, T=T, n_kv_heads=n_kv, n_q_heads=n_q, seed=T + sd,
+                                       device=cuda_dev)
+    p = case["params"]
+    L, r = p["L"], p["rank"]
+    U = workloads.query_subspace(128, sd, seed=sd, device=cuda_dev)
+    mu, xi = crs.block_describe_ss(case["K"], L, r, U)
+    tok, cnt = crs.block_select_ss(case["Q"], U, mu, xi, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select_ss(_np(case["Q"]), U.double().cpu().numpy(),
+                                                       mu.double().cpu().numpy(), xi.double().cpu().numpy(),
+                                                       T, L, top, win)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
+                  f"ss{sd}-G{n_q // n_kv}")
+
+
+def test_select_one_query_head_per_kv_head(crs, cuda_dev):
+    """G = 1 with rank 4 on the generic scorer (a tile of 32 blocks per CTA)."""
+    case = workloads.block_decode_case(n_seq=2, T=32 * 200, n_kv_heads=4, n_q_heads=4, seed=15,
+                                       device=cuda_dev)
+    p = case["params"]
+    L, r = p["L"], p["rank"]
+    mu, xi = crs.block_describe(case["K"], L, r)
+    tok, cnt = crs.block_select(case["Q"], mu, xi, p["T"], L, 12, 64)
+    torch.cuda.synchronize()
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), mu.double().cpu().numpy(),
+                                                    xi.double().cpu().numpy(), p["T"], L, 12, 64)
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, p["T"], 64, 12, "G1")

@@ -12,5 +12,6 @@ from .gen import (  # noqa: F401
     indexer_prefill_case,
     indexer_decode_case,
     block_decode_case,
+    query_subspace,
     make_config,
 )

@@ -224,6 +224,16 @@ CONFIGS = {
 }
 
 
+def query_subspace(D=128, s=85, seed=21, device="cpu") -> "torch.Tensor":
+    """An orthonormal basis U [D, s] (fp32) of a query subspace.  The synthetic
+    queries are isotropic N(0, I), so no subspace captures more of their second
+    moment than another: U is the Q factor of a seeded Gaussian D x s matrix."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    A = torch.randn(D, s, generator=g, dtype=torch.float64)
+    Uq, _ = torch.linalg.qr(A)
+    return Uq.to(torch.float32).contiguous().to(device)
+
+
 def make_config(i: int, device="cpu") -> Dict:
     """Full-size workload ``i`` (1..5); seed = i - 1."""
     return CONFIGS[int(i)](device=device)
