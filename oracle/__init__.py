@@ -11,6 +11,7 @@ Parity status per function (pins in ``tests/test_oracle_*.py``):
   block_describe / block_log_mass / block_select   -- pinned (rank 0 = mean-pool selector)
   quest_describe / quest_select                    -- pinned
   block_describe_ss / block_select_ss              -- pinned
+  hisa_describe / hisa_topk                        -- pinned
   fp4_quantize / fp4_dequantize                    -- pinned
   sparse_attn                                      -- pinned
 """
@@ -60,6 +61,9 @@ def _lib():
         lib.oracle_block_describe_ss.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p, _f64p, _f64p]
         lib.oracle_block_select_ss.argtypes = [I, I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
                                                _f64p, I, _i32p, _i32p, _i32p, _f64p]
+        lib.oracle_hisa_describe.argtypes = [I, I, I, _f64p, _i64p, _i64p, _f64p]
+        lib.oracle_hisa_topk.argtypes = [I, I, I, I, I, I, _f64p, _f64p, _f64p, _i64p, _f64p, _i64p, _i32p,
+                                         _i32p, _i32p, _i32p, _f64p]
         lib.oracle_quest_describe.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p]
         lib.oracle_quest_select.argtypes = [I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p, I,
                                             _i32p, _i32p, _i32p, _f64p]
@@ -197,6 +201,45 @@ def indexer_topk(q, w, K, key_base, n_visible, topk):
                                _p(kb, _i64p), _p(nv, _i32p), _p(idx, _i32p), _p(cnt, _i32p),
                                _p(cut, _f64p), _p(nxt, _f64p))
     return idx, cnt, cut, nxt
+
+
+def hisa_block_offsets(k_offsets, blk):
+    """[n_rows + 1] int64: first representative of each row (complete blocks only)."""
+    ko = np.asarray(k_offsets, dtype=np.int64)
+    nb = (ko[1:] - ko[:-1]) // blk
+    return np.concatenate([[0], np.cumsum(nb)]).astype(np.int64)
+
+
+def hisa_describe(K, k_offsets, blk):
+    """Block representatives (mean index key per complete block).  K [keys, d]."""
+    K = _c(K, np.float64)
+    ko = _c(k_offsets, np.int64)
+    bo = hisa_block_offsets(ko, blk)
+    n_rows, d = len(ko) - 1, K.shape[1]
+    rep = np.zeros((int(bo[-1]), d), dtype=np.float64)
+    _lib().oracle_hisa_describe(n_rows, d, blk, _p(K, _f64p), _p(ko, _i64p), _p(bo, _i64p), _p(rep, _f64p))
+    return rep, bo
+
+
+def hisa_topk(q, w, K, k_offsets, rep, blk_offsets, topk, blk, top_blocks, given_blocks=None):
+    """Hierarchical top-k for decode rows.  Returns (blocks [rows, top_blocks] ascending,
+    idx [rows, topk] ascending, count [rows], coarse scores [n_blocks])."""
+    q = _c(q, np.float64)
+    w = _c(w, np.float64)
+    K = _c(K, np.float64)
+    ko = _c(k_offsets, np.int64)
+    rep = _c(rep, np.float64)
+    bo = _c(blk_offsets, np.int64)
+    rows, heads, d = q.shape
+    blocks = np.empty((rows, top_blocks), dtype=np.int32)
+    idx = np.empty((rows, topk), dtype=np.int32)
+    cnt = np.empty(rows, dtype=np.int32)
+    coarse = np.zeros(max(1, rep.shape[0]), dtype=np.float64)
+    gb = None if given_blocks is None else _c(given_blocks, np.int32)
+    _lib().oracle_hisa_topk(rows, heads, d, topk, blk, top_blocks, _p(q, _f64p), _p(w, _f64p), _p(K, _f64p),
+                            _p(ko, _i64p), _p(rep, _f64p), _p(bo, _i64p), None if gb is None else _p(gb, _i32p),
+                            _p(blocks, _i32p), _p(idx, _i32p), _p(cnt, _i32p), _p(coarse, _f64p))
+    return blocks, idx, cnt, coarse[: rep.shape[0]]
 
 
 # -------------------------------------------------------------- blocks --

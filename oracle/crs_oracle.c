@@ -336,6 +336,110 @@ OAPI void oracle_indexer_topk(int n_rows, int n_heads, int d, int topk, const do
 }
 
 /* ======================================================================
+ * O4h  Hierarchical indexer (HISA), decode rows.  [P2] "索引器的三种降本方向"
+ * and §2.2 Eq.(7): the history of a row is cut into blocks of `blk` keys;
+ * each complete block has a representative (reading: the mean of its index
+ * keys, d_c = d) scored with the indexer's own formula,
+ *   c_j = sum_h w_h ReLU(q_h . rep_j);
+ * the top_blocks blocks by (c desc, block asc) are kept (all of them when the
+ * row has fewer); the original token indexer then runs only on the kept
+ * blocks' keys and on the open (incomplete) trailing block ([P2] "未满块由局部
+ * 或单独 open-block 路径处理"), and returns the same top-k interface as O4
+ * (ties to the smaller position, ascending, -1 padded).  The kept blocks are
+ * returned too (ascending, -1 padded): the pages keep each level's candidates
+ * to locate a miss ([P2] "失败样本怎样定位到具体层级").
+ * Layout: keys of row s are K[k_offsets[s] .. k_offsets[s+1]); block j of row s
+ * has rep[(blk_offsets[s] + j) * d + .], j < (k_offsets[s+1]-k_offsets[s])/blk.
+ * given_blocks (optional, [n_rows, top_blocks], -1 padded) replaces the
+ * coarse selection: the fine stage on a given candidate set.
+ * ====================================================================== */
+OAPI void oracle_hisa_describe(int n_rows, int d, int blk, const double *K, const int64_t *k_offsets,
+                               const int64_t *blk_offsets, double *rep)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long t = 0; t < n_rows; ++t) {
+        const long ctx = (long)(k_offsets[t + 1] - k_offsets[t]);
+        const long nb = ctx / blk;
+        for (long j = 0; j < nb; ++j) {
+            double *r = rep + (blk_offsets[t] + j) * d;
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int i = 0; i < blk; ++i)
+                    acc += K[(k_offsets[t] + j * blk + i) * d + c];
+                r[c] = acc / blk;
+            }
+        }
+    }
+}
+
+OAPI void oracle_hisa_topk(int n_rows, int n_heads, int d, int topk, int blk, int top_blocks,
+                           const double *q, const double *w, const double *K, const int64_t *k_offsets,
+                           const double *rep, const int64_t *blk_offsets, const int32_t *given_blocks,
+                           int32_t *out_blocks, int32_t *out_idx, int32_t *out_count,
+                           double *coarse_score)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long t = 0; t < n_rows; ++t) {
+        const long ctx = (long)(k_offsets[t + 1] - k_offsets[t]);
+        const int nb = (int)(ctx / blk);
+        const double *qt = q + t * (long)n_heads * d, *wt = w + t * (long)n_heads;
+        int32_t *ob = out_blocks + t * (long)top_blocks;
+        int nkeep = 0;
+        if (given_blocks) {
+            for (int c = 0; c < top_blocks; ++c)
+                if (given_blocks[t * (long)top_blocks + c] >= 0)
+                    ob[nkeep++] = given_blocks[t * (long)top_blocks + c];
+        } else {
+            scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(nb > 0 ? nb : 1));
+            double *cs = (double *)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
+            oracle_indexer_score(n_heads, d, qt, wt, rep + blk_offsets[t] * (long)d, nb, cs);
+            for (int j = 0; j < nb; ++j) {
+                sc[j].s = cs[j];
+                sc[j].i = j;
+                if (coarse_score) coarse_score[blk_offsets[t] + j] = cs[j];
+            }
+            qsort(sc, (size_t)nb, sizeof(scored_t), cmp_score_desc_idx_asc);
+            nkeep = nb < top_blocks ? nb : top_blocks;
+            for (int c = 0; c < nkeep; ++c)
+                ob[c] = sc[c].i;
+            free(sc);
+            free(cs);
+        }
+        qsort(ob, (size_t)nkeep, sizeof(int32_t), cmp_i32);
+        for (int c = nkeep; c < top_blocks; ++c)
+            ob[c] = -1;
+        /* candidates: the kept blocks' keys, then the open block's */
+        const long open0 = (long)nb * blk;
+        const long ncand = (long)nkeep * blk + (ctx - open0);
+        scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(ncand > 0 ? ncand : 1));
+        double one;
+        long c = 0;
+        for (int b = 0; b < nkeep; ++b)
+            for (int i = 0; i < blk; ++i, ++c) {
+                const long pos = (long)ob[b] * blk + i;
+                oracle_indexer_score(n_heads, d, qt, wt, K + (k_offsets[t] + pos) * d, 1, &one);
+                sc[c].s = one;
+                sc[c].i = (int32_t)pos;
+            }
+        for (long pos = open0; pos < ctx; ++pos, ++c) {
+            oracle_indexer_score(n_heads, d, qt, wt, K + (k_offsets[t] + pos) * d, 1, &one);
+            sc[c].s = one;
+            sc[c].i = (int32_t)pos;
+        }
+        qsort(sc, (size_t)ncand, sizeof(scored_t), cmp_score_desc_idx_asc);
+        const int kk = ncand < topk ? (int)ncand : topk;
+        int32_t *o = out_idx + t * (long)topk;
+        for (int i = 0; i < kk; ++i)
+            o[i] = sc[i].i;
+        qsort(o, (size_t)kk, sizeof(int32_t), cmp_i32);
+        for (int i = kk; i < topk; ++i)
+            o[i] = -1;
+        out_count[t] = kk;
+        free(sc);
+    }
+}
+
+/* ======================================================================
  * O5  Block descriptor.  [P5] Eq.(11): mean key and population covariance
  * Sigma_b = (1/L) sum (k_r - kbar)(k_r - kbar)^T; Eq.(16): keep the r largest
  * eigen-directions, xi_i = sqrt(lambda_i) u_i; Eq.(20) / Algorithm 2 (Gram
