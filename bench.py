@@ -1,7 +1,7 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|prefill|decode|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
+                  [--workload lsh|lsh_fp32|prefill|decode|decode_hisa|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
@@ -10,6 +10,7 @@ A step is one pass of the hot path over one batch of the workload:
   lsh_fp32 fp32 LSH attention, n=1024, b=16, 1 round, chunk 64.
   prefill  indexer prefill n=32768 (top-2048) + MQA gather attention (16 heads).
   decode   indexer decode, 64 sequences of ragged context + GQA gather attention.
+  decode_hisa  the same with the hierarchical indexer (64-key blocks, 128 kept).
   block    block-mass decode: block select (top-64 + 512 window) + GQA attention;
            the descriptor build is timed separately (it runs once per filled block).
   block_fp4 the same on bf16 means + FP4 (E2M1) eigenvectors (528 B per block).
@@ -245,6 +246,42 @@ class DecodeWorkload(Workload):
         }
 
 
+class DecodeHisaWorkload(DecodeWorkload):
+    """The indexer decode step with the hierarchical indexer: mean representatives of
+    64-key blocks (a cache, built once per filled block), 128 kept blocks per row, the
+    token indexer on their keys and the open block, then the gather attention."""
+    BLK, TOP_BLOCKS = 64, 128
+
+    def __init__(self, crs, dev):
+        super().__init__(crs, dev)
+        self.name = self.c["workload"].replace("indexer_decode_", f"hisa_b{self.BLK}_kb{self.TOP_BLOCKS}_decode_", 1)
+        self.rep, self.bo = crs.hisa_describe(self.c["k_idx"], self.c["offsets"], self.BLK, 131072)
+        torch.cuda.synchronize()
+        import ctypes
+        hp = crs.HisaParams(self.p["n_seq"], 4, 64, self.p["topk"], self.BLK, self.TOP_BLOCKS, 131072)
+        self.ws = torch.empty(int(crs.lib().crs_hisa_topk_workspace_size(ctypes.byref(hp))),
+                              dtype=torch.uint8, device=dev)
+        self.blocks = torch.empty((self.p["n_seq"], self.TOP_BLOCKS), dtype=torch.int32, device=dev)
+
+    def _run(self, q_idx, w, Q):
+        k = self.p["topk"]
+        self.crs.hisa_topk(q_idx, w, self.c["k_idx"], self.c["offsets"], self.rep, self.bo, k, self.BLK,
+                           self.TOP_BLOCKS, 131072, out_blocks=self.blocks, out=self.idx, count=self.cnt,
+                           workspace=self.ws)
+        self.crs.sparse_attn(Q, self.c["K"], self.c["V"], self.idx.view(-1, 1, k),
+                             kv_base=self.kv_base, out=self.O, workspace=self.ws2)
+
+    def roofline_spec(self):
+        ns, k = self.p["n_seq"], self.p["topk"]
+        n_blocks = int(self.bo[-1])
+        cand = ns * (self.TOP_BLOCKS * self.BLK + self.BLK // 2)
+        return {
+            # representatives (256 B each) + the candidates' index keys (128 B each)
+            "hisa": [("hbm", (n_blocks * 256 + cand * 128) / 1e9, "GB/s")],
+            "sparse_attn": [("hbm", ns * k * 8 * 128 * 2 * 2 / 1e9, "GB/s")],
+        }
+
+
 class BlockWorkload(Workload):
     unit = "steps/s"
 
@@ -427,7 +464,8 @@ class BlockMeanPoolWorkload(BlockWorkload):
 
 WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
-             "prefill": PrefillWorkload, "decode": DecodeWorkload, "block": BlockWorkload,
+             "prefill": PrefillWorkload, "decode": DecodeWorkload, "decode_hisa": DecodeHisaWorkload,
+             "block": BlockWorkload,
              "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
              "block_meanpool": BlockMeanPoolWorkload, "block_ss": BlockSubspaceWorkload}
 
@@ -691,7 +729,7 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "prefill", "decode", "block", "block_fp4", "block_ss",
+        for name in [w for w in ("lsh_fp32", "prefill", "decode", "decode_hisa", "block", "block_fp4", "block_ss",
                                   "block_quest", "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)

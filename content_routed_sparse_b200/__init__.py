@@ -59,6 +59,12 @@ class IndexerParams(ctypes.Structure):
                 ("d_idx", ctypes.c_int), ("topk", ctypes.c_int), ("max_keys", ctypes.c_int)]
 
 
+class HisaParams(ctypes.Structure):
+    _fields_ = [("n_rows", ctypes.c_int), ("n_idx_heads", ctypes.c_int), ("d_idx", ctypes.c_int),
+                ("topk", ctypes.c_int), ("blk", ctypes.c_int), ("top_blocks", ctypes.c_int),
+                ("max_keys", ctypes.c_int)]
+
+
 class BlockParams(ctypes.Structure):
     _fields_ = [("n_seq", ctypes.c_int), ("n_kv", ctypes.c_int), ("T", ctypes.c_int),
                 ("D", ctypes.c_int), ("L", ctypes.c_int), ("rank", ctypes.c_int),
@@ -115,6 +121,10 @@ _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP
 _sig("crs_block_quantize", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP, _VP, _VP])
 _sig("crs_block_select_fp4", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                              _VP, _VP, _SZ, _VP])
+_sig("crs_hisa_describe", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP])
+_sig("crs_hisa_topk_workspace_size", _SZ, [ctypes.POINTER(HisaParams)])
+_sig("crs_hisa_topk", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                      _VP, _SZ, _VP])
 _sig("crs_block_describe_ss", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, ctypes.c_int, _VP, _VP,
                                               _VP])
 _sig("crs_block_select_ss_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams), ctypes.c_int])
@@ -305,6 +315,62 @@ def indexer_topk(q_idx, w, k_idx, topk: int, mode: int = CRS_IDX_PREFILL, k_offs
                                _stream(stream))
     _check("crs_indexer_topk", st)
     return out, count
+
+
+# ------------------------------------------------------------------- HISA --
+def hisa_block_offsets(k_offsets, blk: int):
+    """[rows + 1] int64 on k_offsets' device: first representative of each row (complete
+    blocks of `blk` keys only).  Cache-layout bookkeeping, done when blocks fill."""
+    ko = k_offsets.to("cpu", torch.int64)
+    nb = (ko[1:] - ko[:-1]) // int(blk)
+    bo = torch.zeros(ko.numel(), dtype=torch.int64)
+    bo[1:] = torch.cumsum(nb, 0)
+    return bo.to(k_offsets.device)
+
+
+def hisa_describe(k_idx, k_offsets, blk: int, max_keys: int, blk_offsets=None, rep=None, stream=None):
+    """Block representatives (mean index key per complete block) -> (rep [blocks, 64] f32,
+    blk_offsets [rows + 1] int64)."""
+    _need(k_idx, "k_idx", torch.bfloat16)
+    rows = k_offsets.numel() - 1
+    _need(k_offsets, "k_offsets", torch.int64, (rows + 1,))
+    if blk_offsets is None:
+        blk_offsets = hisa_block_offsets(k_offsets, blk)
+    n_blocks = int(blk_offsets[-1].item())
+    if rep is None:
+        rep = torch.empty((max(1, n_blocks), k_idx.shape[1]), dtype=torch.float32, device=k_idx.device)
+    p = HisaParams(rows, 1, k_idx.shape[1], 1, int(blk), 1, int(max_keys))
+    _check("crs_hisa_describe", _lib.crs_hisa_describe(ctypes.byref(p), _ptr(k_idx), _ptr(k_offsets),
+                                                       _ptr(blk_offsets), _ptr(rep), _stream(stream)))
+    return rep, blk_offsets
+
+
+def hisa_topk(q_idx, w, k_idx, k_offsets, rep, blk_offsets, topk: int, blk: int, top_blocks: int,
+              max_keys: int, out_blocks=None, out=None, count=None, workspace=None, stream=None):
+    """Hierarchical top-k for decode rows -> (blocks [rows, top_blocks], idx [rows, topk], count)."""
+    _need(q_idx, "q_idx", torch.bfloat16)
+    rows, heads, d = q_idx.shape
+    _need(w, "w", torch.float32, (rows, heads))
+    _need(k_idx, "k_idx", torch.bfloat16)
+    _need(k_offsets, "k_offsets", torch.int64, (rows + 1,))
+    _need(blk_offsets, "blk_offsets", torch.int64, (rows + 1,))
+    _need(rep, "rep", torch.float32)
+    p = HisaParams(rows, heads, d, int(topk), int(blk), int(top_blocks), int(max_keys))
+    if out_blocks is None:
+        out_blocks = torch.empty((rows, top_blocks), dtype=torch.int32, device=q_idx.device)
+    if out is None:
+        out = torch.empty((rows, topk), dtype=torch.int32, device=q_idx.device)
+    if count is None:
+        count = torch.empty((rows,), dtype=torch.int32, device=q_idx.device)
+    _need(out_blocks, "out_blocks", torch.int32, (rows, top_blocks))
+    _need(out, "out", torch.int32, (rows, topk))
+    _need(count, "count", torch.int32, (rows,))
+    ws, wsb = _workspace(int(_lib.crs_hisa_topk_workspace_size(ctypes.byref(p))), q_idx.device, workspace)
+    st = _lib.crs_hisa_topk(ctypes.byref(p), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_offsets), _ptr(rep),
+                            _ptr(blk_offsets), _ptr(out_blocks), _ptr(out), _ptr(count), _ptr(ws), wsb,
+                            _stream(stream))
+    _check("crs_hisa_topk", st)
+    return out_blocks, out, count
 
 
 # ----------------------------------------------------------------- blocks --

@@ -7,4 +7,5 @@
 #include "indexer.cu"
 #include "indexer_tc.cu"
 #include "blocks.cu"
+#include "hisa.cu"
 #include "noalloc.cu"

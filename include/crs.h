@@ -193,6 +193,41 @@ int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, const float
                      int32_t *out_count, void *ws, size_t ws_bytes, void *stream);
 
 /* ====================================================================== *
+ * Hierarchical indexer (HISA) for decode rows.  [P2] "索引器的三种降本方向",
+ * §2.2 Eq.(7): each complete block of `blk` keys of a row has a representative
+ * rep_j (the mean of its index keys, f32, from crs_hisa_describe, once per
+ * filled block); the row scores c_j = sum_h w_h ReLU(q_h . rep_j), keeps the
+ * top_blocks blocks by (c desc, block asc), and runs the token indexer of
+ * crs_indexer_topk (same score, ties, ascending -1-padded output) on the kept
+ * blocks' keys plus the open trailing block only.  out_blocks (optional,
+ * [n_rows, top_blocks], ascending, -1 padded) returns the kept blocks: the
+ * pages keep each level's candidates to locate a miss.
+ * k_offsets: [n_rows + 1] int64, row s owns keys k_offsets[s]..k_offsets[s+1]
+ * (at most max_keys, else CRS_DEVERR_INDEX and an empty row); blk_offsets:
+ * [n_rows + 1] int64, blk_offsets[s+1] - blk_offsets[s] = floor(keys_s / blk);
+ * rep: [blk_offsets[n_rows], 64] f32.  d_idx = 64, n_idx_heads <= 8,
+ * blk <= 256, top_blocks * blk + blk <= 16384, max_keys / blk <= 8192
+ * (else CRS_ERR_UNSUPPORTED); k_idx 16-byte aligned.
+ * ====================================================================== */
+typedef struct {
+    int n_rows;       /* decode rows, one query each                            */
+    int n_idx_heads;  /* index heads, 1..8                                      */
+    int d_idx;        /* 64                                                     */
+    int topk;         /* tokens returned, 1..4096                               */
+    int blk;          /* keys per block                                         */
+    int top_blocks;   /* blocks kept by the coarse level                        */
+    int max_keys;     /* an upper bound of the longest row                      */
+} crs_hisa_params;
+
+int crs_hisa_describe(const crs_hisa_params *p, const void *k_idx, const int64_t *k_offsets,
+                      const int64_t *blk_offsets, float *rep, void *stream);
+size_t crs_hisa_topk_workspace_size(const crs_hisa_params *p);
+int crs_hisa_topk(const crs_hisa_params *p, const void *q_idx, const float *w, const void *k_idx,
+                  const int64_t *k_offsets, const float *rep, const int64_t *blk_offsets,
+                  int32_t *out_blocks, int32_t *out_idx, int32_t *out_count, void *ws, size_t ws_bytes,
+                  void *stream);
+
+/* ====================================================================== *
  * Block descriptors.  [P5] Eq.(11), (16), (20) and Algorithm 2: for each
  * complete block of L consecutive keys of one (sequence, KV head):
  *   mu = mean key; Kt = K - mu; G = Kt Kt^T / L (L x L);
