@@ -574,22 +574,27 @@ def roofline(wl, prof, peaks, traffic=None):
         return {"kernel": top, "bound": None, "achieved": None, "peak": None, "unit": None,
                 "frac": None, "traffic": None}, stages
     per_launch_s = timed[top]["total_ms"] / timed[top]["timed_launches"] / 1e3
-    bound, amount, unit = spec[top][0]
+
+    def peak_of(bound):
+        if bound == "hbm":
+            return peaks["hbm_gbs"], f"hbm_gbs ({peaks['source']})"
+        if bound == "tensor":
+            return peaks["bf16_tflops"], f"bf16_tflops ({peaks['source']})"
+        return FP32_ALU_TFLOPS_NOMINAL, "fp32 FMA: 148 SM x 128 lanes x 2 x 1.965 GHz"
+
+    # the binding roofline: the resource whose algorithmic work takes longest at its peak
+    entries = sorted(spec[top], key=lambda e: -e[1] / peak_of(e[0])[0])
+    bound, amount, unit = entries[0]
+    peak, src = peak_of(bound)
     achieved = amount / per_launch_s
-    if bound == "hbm":
-        peak, src = peaks["hbm_gbs"], f"hbm_gbs ({peaks['source']})"
-    elif bound == "tensor":
-        peak, src = peaks["bf16_tflops"], f"bf16_tflops ({peaks['source']})"
-    else:
-        peak, src = FP32_ALU_TFLOPS_NOMINAL, "fp32 FMA: 148 SM x 128 lanes x 2 x 1.965 GHz"
     out = {"kernel": top, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
            "unit": unit, "frac": round(achieved / peak, 4), "traffic": _traffic(top, wl.name),
            "peak_source": src,
            "per_launch_ms": round(per_launch_s * 1e3, 5)}
-    if len(spec[top]) > 1:
-        b2, a2, u2 = spec[top][1]
-        p2 = peaks["hbm_gbs"] if b2 == "hbm" else peaks["bf16_tflops"]
-        out["secondary"] = {"bound": b2, "achieved": round(a2 / per_launch_s, 3), "peak": p2,
+    if len(entries) > 1:
+        b2, a2, u2 = entries[1]
+        p2 = peak_of(b2)[0]
+        out["secondary"] = {"bound": b2, "achieved": round(a2 / per_launch_s, 3), "peak": round(p2, 1),
                             "unit": u2, "frac": round(a2 / per_launch_s / p2, 4)}
     return out, stages
 
