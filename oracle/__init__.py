@@ -12,6 +12,7 @@ Parity status per function (pins in ``tests/test_oracle_*.py``):
   quest_describe / quest_select                    -- pinned
   block_describe_ss / block_select_ss              -- pinned
   hisa_describe / hisa_topk                        -- pinned
+  lsh_decode                                       -- pinned
   fp4_quantize / fp4_dequantize                    -- pinned
   sparse_attn                                      -- pinned
 """
@@ -61,6 +62,8 @@ def _lib():
         lib.oracle_block_describe_ss.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p, _f64p, _f64p]
         lib.oracle_block_select_ss.argtypes = [I, I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
                                                _f64p, I, _i32p, _i32p, _i32p, _f64p]
+        lib.oracle_lsh_decode.argtypes = [I, I, I, I, I, I, I, D, _f64p, _f64p, _i32p, _i32p, _f64p, _f64p,
+                                          _i32p]
         lib.oracle_hisa_describe.argtypes = [I, I, I, _f64p, _i64p, _i64p, _f64p]
         lib.oracle_hisa_topk.argtypes = [I, I, I, I, I, I, _f64p, _f64p, _f64p, _i64p, _f64p, _i64p, _i32p,
                                          _i32p, _i32p, _i32p, _f64p]
@@ -201,6 +204,28 @@ def indexer_topk(q, w, K, key_base, n_visible, topk):
                                _p(kb, _i64p), _p(nv, _i32p), _p(idx, _i32p), _p(cnt, _i32p),
                                _p(cut, _f64p), _p(nxt, _f64p))
     return idx, cnt, cut, nxt
+
+
+def lsh_decode(X, V, R, n_buckets, lengths, no_self=True, key_norm=True, scale=None):
+    """LSH decode step for the newest token of each row.  X, V [S, H, n_max, d] (X also
+    hashed in fp32 by lsh_hash), R [H, rounds, d, b/2]; lengths [S] (tokens including the
+    new one).  Returns (O [S, H, d], lse [S, H], count [S, H])."""
+    Xf = np.ascontiguousarray(X, dtype=np.float32)
+    S, H, n_max, d = Xf.shape
+    rounds = np.asarray(R).shape[1]
+    bucket = lsh_hash(Xf, R, n_buckets)
+    Xd = _c(X, np.float64)
+    Vd = _c(V, np.float64)
+    ln = _c(lengths, np.int32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros((S, H, d), dtype=np.float64)
+    lse = np.empty((S, H), dtype=np.float64)
+    cnt = np.empty((S, H), dtype=np.int32)
+    _lib().oracle_lsh_decode(S, H, n_max, d, rounds, int(no_self), int(key_norm), float(scale), _p(Xd, _f64p),
+                             _p(Vd, _f64p), _p(_c(bucket, np.int32), _i32p), _p(ln, _i32p), _p(O, _f64p),
+                             _p(lse, _f64p), _p(cnt, _i32p))
+    return O, lse, cnt
 
 
 def hisa_block_offsets(k_offsets, blk):

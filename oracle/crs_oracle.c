@@ -264,6 +264,79 @@ OAPI void oracle_lsh_attn(int B, int H, int n, int d, int n_rounds, int m, int c
 }
 
 /* ======================================================================
+ * O3d  LSH decode step.  [P1] §5.2 "Prefill、Decode 与 KV 状态": with the hash
+ * fixed, a new key's bucket ids are computed once and appended to the bucket
+ * lists; the new query reads the lists of its own buckets.  Reading: the
+ * newest token t = len-1 of a row attends to
+ *   U(t) = { j <= t : bucket_r(j) == bucket_r(t) for some round r },
+ * without j == t when no_self, each j once (pairs counted once across rounds,
+ * as O3), with no chunk window (the whole bucket is the neighbourhood in
+ * decode); keys, scale, the empty set and lse as O3.
+ * Layout: X, V [S, H, n_max, d] fp64; bucket [S, H, rounds, n_max] (from O1
+ * on the fp32 vectors); len [S] = tokens of row s including the new one;
+ * outputs O [S, H, d], lse [S, H], count [S, H].
+ * ====================================================================== */
+OAPI void oracle_lsh_decode(int S, int H, int n_max, int d, int n_rounds, int no_self, int key_norm,
+                            double scale, const double *X, const double *V, const int32_t *bucket,
+                            const int32_t *len, double *O, double *lse, int32_t *count)
+{
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < S; ++s)
+        for (int h = 0; h < H; ++h) {
+            const long sh = (long)s * H + h;
+            const int t = len[s] - 1;
+            const double *x = X + sh * n_max * d, *v = V + sh * n_max * d;
+            const int32_t *bk = bucket + sh * (long)n_rounds * n_max;
+            double *o = O + sh * d;
+            double mx = -INFINITY;
+            int cnt = 0;
+            for (int pass = 0; pass < 2; ++pass) {          /* 0: max logit, 1: accumulate */
+                double z = 0.0;
+                if (pass == 1)
+                    for (int c = 0; c < d; ++c)
+                        o[c] = 0.0;
+                for (int j = 0; j <= t; ++j) {
+                    if (no_self && j == t) continue;
+                    int hit = 0;
+                    for (int r = 0; r < n_rounds && !hit; ++r)
+                        hit = bk[(long)r * n_max + j] == bk[(long)r * n_max + t];
+                    if (!hit) continue;
+                    double nrm = 1.0;
+                    if (key_norm) {
+                        nrm = 0.0;
+                        for (int c = 0; c < d; ++c)
+                            nrm += x[(long)j * d + c] * x[(long)j * d + c];
+                        nrm = sqrt(nrm);
+                    }
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        dot += x[(long)t * d + c] * x[(long)j * d + c];
+                    const double lg = nrm > 0.0 ? scale * dot / nrm : 0.0;
+                    if (pass == 0) {
+                        if (lg > mx) mx = lg;
+                        ++cnt;
+                    } else {
+                        const double e = exp(lg - mx);
+                        z += e;
+                        for (int c = 0; c < d; ++c)
+                            o[c] += e * v[(long)j * d + c];
+                    }
+                }
+                if (pass == 1) {
+                    if (cnt == 0) {
+                        lse[sh] = -INFINITY;
+                    } else {
+                        for (int c = 0; c < d; ++c)
+                            o[c] /= z;
+                        lse[sh] = mx + log(z);
+                    }
+                }
+            }
+            count[sh] = cnt;
+        }
+}
+
+/* ======================================================================
  * O4  Lightning-indexer score and token top-k.
  * [P2] §1.1 and §2.1 Eq.(3)-(4): r_{t,s} = sum_h w_{t,h} ReLU(q_{t,h} . k_s)
  * over the index heads, no extra scale; S_t = Select(r_{t,0:t}, k) keeps the k
