@@ -1,13 +1,16 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|prefill|decode|decode_hisa|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
+                  [--workload lsh|lsh_fp32|lsh_decode|prefill|decode|decode_hisa|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
            b=64 buckets, 4 rounds, chunk 128, causal, last 5% padding:
            hash -> sort -> chunked attention -> round merge.  Metric: tokens/s.
   lsh_fp32 fp32 LSH attention, n=1024, b=16, 1 round, chunk 64.
+  lsh_decode  LSH attention in decode: 64 rows x 8 heads, 16384-token prompts in bucket
+           lists (64 buckets x 4 rounds) and paged K/V; a step appends one token per row
+           and attends with it.
   prefill  indexer prefill n=32768 (top-2048) + MQA gather attention (16 heads).
   decode   indexer decode, 64 sequences of ragged context + GQA gather attention.
   decode_hisa  the same with the hierarchical indexer (64-key blocks, 128 kept).
@@ -132,6 +135,54 @@ class LshWorkload(Workload):
                                   ("hbm", attn_bytes / 1e9, "GB/s")],
             "lsh_hash": [("alu", B * H * R * n * d * (p["n_buckets"] // 2) * 2 / 1e12, "TFLOP/s")],
         }
+
+
+class LshDecodeWorkload(Workload):
+    """LSH attention in decode: 64 rows x 8 heads (d = 64) whose 16384-token prompts were
+    hashed into 64 buckets x 4 rounds (bucket lists, paged K/V behind a shuffled block
+    table); a step appends one token per row and attends with it."""
+    unit = "steps/s"
+
+    def __init__(self, crs, dev):
+        self.crs = crs
+        S, H, d, b, R, n = 64, 8, 64, 64, 4, 16384
+        self.p = dict(n_seq=S, n_heads=H, d=d, n_buckets=b, n_rounds=R, prompt=n, page_size=64, list_page=64)
+        self.name = f"lsh_decode_seq{S}_H{H}_d{d}_b{b}_r{R}_ctx{n}"
+        self.units_per_step = 1
+        g = torch.Generator(device="cpu").manual_seed(61)
+        self.rot = torch.randn(H, R, d, b // 2, generator=g).to(dev)
+        self.cache = crs.LshDecodeCache(S, H, b, R, max_len=n + 256, device=dev)
+        for c0 in range(0, n, 4096):              # the prompt, in pieces (device memory for inputs)
+            x = torch.randn(S, 4096, H, d, generator=g).to(torch.bfloat16).to(dev)
+            v = torch.randn(S, 4096, H, d, generator=g).to(torch.bfloat16).to(dev)
+            self.cache.prefill(x, v, self.rot)
+        self.x = torch.randn(S, 1, H, d, generator=g).to(torch.bfloat16).to(dev)
+        self.v = torch.randn(S, 1, H, d, generator=g).to(torch.bfloat16).to(dev)
+        self.O = torch.empty((S, H, d), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((S, H), dtype=torch.float32, device=dev)
+        self.cnt = torch.empty((S, H), dtype=torch.int32, device=dev)
+        self.cache.step(self.x, self.v, self.rot, out=self.O, lse=self.lse, count=self.cnt)
+        torch.cuda.synchronize()
+        self.cand = int(self.cnt.sum())            # candidates of a step (K + V rows read)
+        self.h_in = {"x": self.x.cpu().pin_memory(), "v": self.v.cpu().pin_memory()}
+        self.d_in = {k: torch.empty_like(t, device=dev) for k, t in self.h_in.items()}
+        self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def step(self):
+        self.cache.step(self.x, self.v, self.rot, out=self.O, lse=self.lse, count=self.cnt)
+
+    def e2e_step(self):
+        for k, h in self.h_in.items():
+            self.d_in[k].copy_(h, non_blocking=True)
+        self.cache.step(self.d_in["x"], self.d_in["v"], self.rot, out=self.O, lse=self.lse, count=self.cnt)
+        self.h_out.copy_(self.O, non_blocking=True)
+
+    def roofline_spec(self):
+        # per candidate: its key and value rows (2 x 128 B), its list entry (4 B) and the
+        # earlier rounds' bucket bytes; per step and (row, head): the new rows written
+        return {"lsh_decode": [("hbm", self.cand * (256 + 4 + self.p["n_rounds"]) / 1e9, "GB/s")]}
 
 
 class PrefillWorkload(Workload):
@@ -465,6 +516,7 @@ class BlockMeanPoolWorkload(BlockWorkload):
 WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
              "prefill": PrefillWorkload, "decode": DecodeWorkload, "decode_hisa": DecodeHisaWorkload,
+             "lsh_decode": LshDecodeWorkload,
              "block": BlockWorkload,
              "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
              "block_meanpool": BlockMeanPoolWorkload, "block_ss": BlockSubspaceWorkload}
@@ -734,7 +786,7 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "prefill", "decode", "decode_hisa", "block", "block_fp4", "block_ss",
+        for name in [w for w in ("lsh_fp32", "lsh_decode", "prefill", "decode", "decode_hisa", "block", "block_fp4", "block_ss",
                                   "block_quest", "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)

@@ -65,6 +65,18 @@ class HisaParams(ctypes.Structure):
                 ("max_keys", ctypes.c_int)]
 
 
+class LshDecodeParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("n_seq", "n_heads", "d", "n_buckets", "n_rounds", "page_size",
+                                              "max_pages", "list_page", "list_pages", "n_list_pages",
+                                              "max_len", "no_self", "key_norm")] + [("scale", ctypes.c_float)]
+
+
+class LshDecodeState(ctypes.Structure):
+    _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("bucket_store", ctypes.c_void_p), ("list_table", ctypes.c_void_p), ("list_len", ctypes.c_void_p),
+                ("list_pool", ctypes.c_void_p), ("alloc", ctypes.c_void_p), ("seq_len", ctypes.c_void_p)]
+
+
 class BlockParams(ctypes.Structure):
     _fields_ = [("n_seq", ctypes.c_int), ("n_kv", ctypes.c_int), ("T", ctypes.c_int),
                 ("D", ctypes.c_int), ("L", ctypes.c_int), ("rank", ctypes.c_int),
@@ -121,6 +133,10 @@ _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP
 _sig("crs_block_quantize", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP, _VP, _VP])
 _sig("crs_block_select_fp4", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                              _VP, _VP, _SZ, _VP])
+_sig("crs_lsh_decode_prefill", ctypes.c_int, [ctypes.POINTER(LshDecodeParams), ctypes.POINTER(LshDecodeState),
+                                                _VP, _VP, _VP, ctypes.c_int, _VP])
+_sig("crs_lsh_decode_step", ctypes.c_int, [ctypes.POINTER(LshDecodeParams), ctypes.POINTER(LshDecodeState),
+                                             _VP, _VP, _VP, _VP, _VP, _VP, _VP])
 _sig("crs_hisa_describe", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP])
 _sig("crs_hisa_topk_workspace_size", _SZ, [ctypes.POINTER(HisaParams)])
 _sig("crs_hisa_topk", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
@@ -315,6 +331,69 @@ def indexer_topk(q_idx, w, k_idx, topk: int, mode: int = CRS_IDX_PREFILL, k_offs
                                _stream(stream))
     _check("crs_indexer_topk", st)
     return out, count
+
+
+# ------------------------------------------------------------- LSH decode --
+class LshDecodeCache:
+    """Device state of LSH attention in decode (paged K/V behind a block table, bucket
+    lists of logical positions): see crs_lsh_decode_* in include/crs.h.  block_table maps
+    each row's logical pages to physical pages of one pool (a permutation when given as
+    "shuffled", so that rows' pages interleave as in a shared page pool)."""
+
+    def __init__(self, n_seq, n_heads, n_buckets, n_rounds, max_len, d=64, page_size=64, list_page=64,
+                 list_cap=None, n_list_pages=None, no_self=True, key_norm=True, scale=None, device="cuda",
+                 shuffled=True, seed=0):
+        max_pages = -(-max_len // page_size)
+        if list_cap is None:
+            list_cap = max(list_page, 4 * max_len // n_buckets)
+        list_pages = -(-list_cap // list_page)
+        if n_list_pages is None:
+            n_list_pages = n_seq * n_heads * n_rounds * (n_buckets + -(-max_len // list_page))
+        self.p = LshDecodeParams(n_seq, n_heads, d, n_buckets, n_rounds, page_size, max_pages, list_page,
+                                 list_pages, n_list_pages, max_len, int(no_self), int(key_norm),
+                                 float(scale if scale is not None else 1.0 / math.sqrt(d)))
+        n_pages = n_seq * max_pages
+        g = torch.Generator(device="cpu").manual_seed(seed)
+        order = torch.randperm(n_pages, generator=g) if shuffled else torch.arange(n_pages)
+        self.block_table = order.to(torch.int32).view(n_seq, max_pages).to(device)
+        self.k_pool = torch.zeros((n_pages, page_size, n_heads, d), dtype=torch.bfloat16, device=device)
+        self.v_pool = torch.zeros_like(self.k_pool)
+        self.bucket_store = torch.zeros((n_seq, n_heads, n_rounds, max_len), dtype=torch.uint8, device=device)
+        self.list_table = torch.full((n_seq, n_heads, n_rounds, n_buckets, list_pages), -1, dtype=torch.int32,
+                                     device=device)
+        self.list_len = torch.zeros((n_seq, n_heads, n_rounds, n_buckets), dtype=torch.int32, device=device)
+        self.list_pool = torch.zeros((n_list_pages, list_page), dtype=torch.int32, device=device)
+        self.alloc = torch.zeros((1,), dtype=torch.int32, device=device)
+        self.seq_len = torch.zeros((n_seq,), dtype=torch.int32, device=device)
+        self.st = LshDecodeState(*(t.data_ptr() for t in (self.k_pool, self.v_pool, self.block_table,
+                                                         self.bucket_store, self.list_table, self.list_len,
+                                                         self.list_pool, self.alloc, self.seq_len)))
+
+    def prefill(self, x, v, rot, stream=None):
+        """Append x, v [n_seq, n_tokens, n_heads, d] bf16 (rot [H, rounds, d, b/2] f32)."""
+        _need(x, "x", torch.bfloat16)
+        _need(v, "v", torch.bfloat16, tuple(x.shape))
+        _need(rot, "rot", torch.float32)
+        _check("crs_lsh_decode_prefill", _lib.crs_lsh_decode_prefill(ctypes.byref(self.p), ctypes.byref(self.st),
+                                                                     _ptr(x), _ptr(v), _ptr(rot), x.shape[1],
+                                                                     _stream(stream)))
+
+    def step(self, x, v, rot, out=None, lse=None, count=None, stream=None):
+        """Append one token per row (x, v [n_seq, 1, n_heads, d]) and attend with it ->
+        (O [n_seq, n_heads, d] f32, lse [n_seq, n_heads], count [n_seq, n_heads])."""
+        _need(x, "x", torch.bfloat16)
+        _need(v, "v", torch.bfloat16, tuple(x.shape))
+        S, H, d = self.p.n_seq, self.p.n_heads, self.p.d
+        if out is None:
+            out = torch.empty((S, H, d), dtype=torch.float32, device=x.device)
+        if lse is None:
+            lse = torch.empty((S, H), dtype=torch.float32, device=x.device)
+        if count is None:
+            count = torch.empty((S, H), dtype=torch.int32, device=x.device)
+        _check("crs_lsh_decode_step", _lib.crs_lsh_decode_step(ctypes.byref(self.p), ctypes.byref(self.st), _ptr(x),
+                                                               _ptr(v), _ptr(rot), _ptr(out), _ptr(lse), _ptr(count),
+                                                               _stream(stream)))
+        return out, lse, count
 
 
 # ------------------------------------------------------------------- HISA --

@@ -60,6 +60,7 @@ typedef enum { CRS_F32 = 0, CRS_BF16 = 1 } crs_dtype;
 #define CRS_DEVERR_NONFINITE 0x1u
 #define CRS_DEVERR_TIMEOUT   0x2u
 #define CRS_DEVERR_INDEX     0x4u
+#define CRS_DEVERR_CAPACITY  0x8u   /* a bounded structure was full: an entry was dropped */
 
 /* Human-readable name of a crs_status value (static string, never NULL). */
 const char *crs_status_string(int status);
@@ -157,6 +158,57 @@ int crs_lsh_attn(const crs_lsh_attn_params *p, const void *QK, const void *V,
                  const int32_t *bucket, const int32_t *perm, const int32_t *inv_perm,
                  const int32_t *valid_len, void *O, float *lse, void *ws, size_t ws_bytes,
                  void *stream);
+
+/* ====================================================================== *
+ * LSH attention in decode.  [P1] §5.2 "Prefill、Decode 与 KV 状态": the hash is
+ * fixed (R as crs_lsh_route); each new token's bucket ids (one per round, O(d R))
+ * are appended to that (row, head, round, bucket)'s list of logical positions;
+ * K/V stay paged by time behind a block table ([P2] §2.1 "主 KV gather 的物理代价").
+ * The newest token t of a row attends to every token j <= t sharing a bucket
+ * with it in some round, each once, without t itself when no_self; keys are
+ * the shared-QK vectors normalised when key_norm (stored normalised in bf16),
+ * logits scale * q . k, fp32 softmax; an empty set gives O = 0, lse = -inf.
+ * State (caller-owned, zero-initialised except k/v pools and block_table):
+ *   k_pool, v_pool [n_pages, page_size, n_heads, d] bf16 (16-byte aligned);
+ *   block_table [n_seq, max_pages] int32 (logical page -> physical page);
+ *   bucket_store [n_seq, n_heads, n_rounds, max_len] uint8;
+ *   list_table [n_seq, n_heads, n_rounds, n_buckets, list_pages] int32,
+ *   list_len [n_seq, n_heads, n_rounds, n_buckets] int32,
+ *   list_pool [n_list_pages, list_page] int32, alloc [1] int32 (pages used);
+ *   seq_len [n_seq] int32 (tokens already in each row).
+ * A list holds at most list_pages * list_page entries; a full list, an
+ * exhausted list pool, or a row beyond max_len / max_pages * page_size sets
+ * CRS_DEVERR_CAPACITY and drops the entry.  d = 64, n_buckets even <= 256,
+ * n_rounds <= 8 (else CRS_ERR_UNSUPPORTED).
+ * crs_lsh_decode_prefill appends n_tokens tokens per row (x, v [n_seq,
+ * n_tokens, n_heads, d] bf16) in position order; crs_lsh_decode_step appends
+ * one token per row (x, v [n_seq, 1, n_heads, d]) and attends with it:
+ * O [n_seq, n_heads, d] f32, lse [n_seq, n_heads] f32 (natural log), count
+ * [n_seq, n_heads] int32 (candidates, may be NULL).  Both advance seq_len.
+ * ====================================================================== */
+typedef struct {
+    int n_seq, n_heads, d, n_buckets, n_rounds;
+    int page_size;     /* tokens per KV page                                   */
+    int max_pages;     /* block_table row length                               */
+    int list_page;     /* positions per bucket-list page                       */
+    int list_pages;    /* page-table length of one bucket list                 */
+    int n_list_pages;  /* pages in list_pool                                   */
+    int max_len;       /* tokens per row at most (bucket_store row length)     */
+    int no_self, key_norm;
+    float scale;
+} crs_lsh_decode_params;
+
+typedef struct {
+    void *k_pool, *v_pool;
+    const int32_t *block_table;
+    uint8_t *bucket_store;
+    int32_t *list_table, *list_len, *list_pool, *alloc, *seq_len;
+} crs_lsh_decode_state;
+
+int crs_lsh_decode_prefill(const crs_lsh_decode_params *p, const crs_lsh_decode_state *st, const void *x,
+                           const void *v, const float *rot, int n_tokens, void *stream);
+int crs_lsh_decode_step(const crs_lsh_decode_params *p, const crs_lsh_decode_state *st, const void *x,
+                        const void *v, const float *rot, float *O, float *lse, int32_t *count, void *stream);
 
 /* ====================================================================== *
  * Lightning indexer + token top-k.  [P2] §1.1 / §2.1 Eq.(2)-(4):
