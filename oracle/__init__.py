@@ -13,6 +13,7 @@ Parity status per function (pins in ``tests/test_oracle_*.py``):
   block_describe_ss / block_select_ss              -- pinned
   hisa_describe / hisa_topk                        -- pinned
   lsh_decode                                       -- pinned
+  kmeans_route                                     -- pinned
   fp4_quantize / fp4_dequantize                    -- pinned
   sparse_attn                                      -- pinned
 """
@@ -62,6 +63,8 @@ def _lib():
         lib.oracle_block_describe_ss.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p, _f64p, _f64p]
         lib.oracle_block_select_ss.argtypes = [I, I, I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p,
                                                _f64p, I, _i32p, _i32p, _i32p, _f64p]
+        lib.oracle_kmeans_route.argtypes = [I, I, I, I, I, I, I, I, D, _f32p, _f32p, _f32p, _f64p, _f64p, _f64p,
+                                            _i32p, _i32p, _f64p, _f64p, _i32p]
         lib.oracle_lsh_decode.argtypes = [I, I, I, I, I, I, I, D, _f64p, _f64p, _i32p, _i32p, _f64p, _f64p,
                                           _i32p]
         lib.oracle_hisa_describe.argtypes = [I, I, I, _f64p, _i64p, _i64p, _f64p]
@@ -204,6 +207,29 @@ def indexer_topk(q, w, K, key_base, n_visible, topk):
                                _p(kb, _i64p), _p(nv, _i32p), _p(idx, _i32p), _p(cnt, _i32p),
                                _p(cut, _f64p), _p(nxt, _f64p))
     return idx, cnt, cut, nxt
+
+
+def kmeans_route(Q, K, V, M, m, causal=True, no_self=False, scale=None):
+    """Routing attention with quota execution.  Q, K, V [B, H, n, d] (Q, K also scored in
+    fp32), M [H, C, d] frozen centres, quota m.  Returns (JQ, JK [B, H, C, m] ascending,
+    -1 padded; O [B, H, n, d]; lse [B, H, n]; count [B, H, n])."""
+    Qf = _c(Q, np.float32)
+    Kf = _c(K, np.float32)
+    Mf = _c(M, np.float32)
+    B, H, n, d = Qf.shape
+    C = Mf.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    JQ = np.empty((B, H, C, m), dtype=np.int32)
+    JK = np.empty((B, H, C, m), dtype=np.int32)
+    O = np.empty((B, H, n, d), dtype=np.float64)
+    lse = np.empty((B, H, n), dtype=np.float64)
+    cnt = np.empty((B, H, n), dtype=np.int32)
+    _lib().oracle_kmeans_route(B, H, n, d, C, m, int(causal), int(no_self), float(scale), _p(Qf, _f32p),
+                               _p(Kf, _f32p), _p(Mf, _f32p), _p(_c(Q, np.float64), _f64p),
+                               _p(_c(K, np.float64), _f64p), _p(_c(V, np.float64), _f64p), _p(JQ, _i32p),
+                               _p(JK, _i32p), _p(O, _f64p), _p(lse, _f64p), _p(cnt, _i32p))
+    return JQ, JK, O, lse, cnt
 
 
 def lsh_decode(X, V, R, n_buckets, lengths, no_self=True, key_norm=True, scale=None):

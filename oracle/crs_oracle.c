@@ -409,6 +409,109 @@ OAPI void oracle_indexer_topk(int n_rows, int n_heads, int d, int topk, const do
 }
 
 /* ======================================================================
+ * O3k  Routing (k-means) attention with quota execution.  [P1] §3.1: with the
+ * centres M frozen (inference), the routing scores are S_Q = Q M^T and
+ * S_K = K M^T; each centre c takes its m best queries and m best keys,
+ *   J_c^Q = Top_m(S_Q[:, c]),  J_c^K = Top_m(S_K[:, c]),
+ * a token may belong to several centres, and each query's outputs over its
+ * centres must be combined at its original index ("定额执行").  The score is
+ * an integer decision taken in fp32 as O1: one fused multiply-add per term in
+ * increasing index order from 0; Top_m keeps (score desc, index asc).
+ * Reading: query i attends to the union U(i) of J_c^K over the centres c with
+ * i in J_c^Q, each key once (pairs counted once, as O3), restricted to j <= i
+ * when causal and to j != i when no_self; logits scale * q_i . k_j (separate
+ * Q and K, no normalisation); an empty set gives O = 0, lse = -inf.
+ * Layout: Qf, Kf [B,H,n,d] fp32 (for the scores), Q, K, V [B,H,n,d] fp64,
+ * M [H, C, d] fp32; outputs JQ, JK [B,H,C,m] (ascending), O [B,H,n,d],
+ * lse [B,H,n], count [B,H,n].
+ * ====================================================================== */
+static float route_score(const float *x, const float *mu, int d)
+{
+    float acc = 0.0f;
+    for (int t = 0; t < d; ++t)
+        acc = fmaf(x[t], mu[t], acc);
+    return acc;
+}
+
+OAPI void oracle_kmeans_route(int B, int H, int n, int d, int C, int m, int causal, int no_self, double scale,
+                              const float *Qf, const float *Kf, const float *M, const double *Q,
+                              const double *K, const double *V, int32_t *JQ, int32_t *JK, double *O,
+                              double *lse, int32_t *count)
+{
+    const int mm = m < n ? m : n;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const long bh = (long)b * H + h;
+            scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)n);
+            uint8_t *inq = (uint8_t *)calloc((size_t)n * C, 1);   /* [i][c]: i in J_c^Q */
+            uint8_t *ink = (uint8_t *)calloc((size_t)n * C, 1);
+            for (int role = 0; role < 2; ++role) {
+                const float *X = (role == 0 ? Qf : Kf) + bh * (long)n * d;
+                int32_t *J = (role == 0 ? JQ : JK) + bh * (long)C * m;
+                uint8_t *in = role == 0 ? inq : ink;
+                for (int c = 0; c < C; ++c) {
+                    const float *mu = M + ((long)h * C + c) * d;
+                    for (int i = 0; i < n; ++i) {
+                        sc[i].s = (double)route_score(X + (long)i * d, mu, d);
+                        sc[i].i = i;
+                    }
+                    qsort(sc, (size_t)n, sizeof(scored_t), cmp_score_desc_idx_asc);
+                    int32_t *Jc = J + (long)c * m;
+                    for (int k = 0; k < mm; ++k)
+                        Jc[k] = sc[k].i;
+                    qsort(Jc, (size_t)mm, sizeof(int32_t), cmp_i32);
+                    for (int k = mm; k < m; ++k)
+                        Jc[k] = -1;
+                    for (int k = 0; k < mm; ++k)
+                        in[(long)Jc[k] * C + c] = 1;
+                }
+            }
+            const double *q = Q + bh * (long)n * d, *k = K + bh * (long)n * d, *v = V + bh * (long)n * d;
+            for (int i = 0; i < n; ++i) {
+                double *o = O + (bh * n + i) * d;
+                for (int t = 0; t < d; ++t)
+                    o[t] = 0.0;
+                double mx = -INFINITY, z = 0.0;
+                int cnt = 0;
+                for (int pass = 0; pass < 2; ++pass)
+                    for (int j = 0; j < n; ++j) {
+                        if (causal && j > i) continue;
+                        if (no_self && j == i) continue;
+                        int hit = 0;
+                        for (int c = 0; c < C && !hit; ++c)
+                            hit = inq[(long)i * C + c] && ink[(long)j * C + c];
+                        if (!hit) continue;
+                        double dot = 0.0;
+                        for (int t = 0; t < d; ++t)
+                            dot += q[(long)i * d + t] * k[(long)j * d + t];
+                        const double lg = scale * dot;
+                        if (pass == 0) {
+                            if (lg > mx) mx = lg;
+                            ++cnt;
+                        } else {
+                            const double e = exp(lg - mx);
+                            z += e;
+                            for (int t = 0; t < d; ++t)
+                                o[t] += e * v[(long)j * d + t];
+                        }
+                    }
+                if (cnt > 0) {
+                    for (int t = 0; t < d; ++t)
+                        o[t] /= z;
+                    lse[bh * n + i] = mx + log(z);
+                } else {
+                    lse[bh * n + i] = -INFINITY;
+                }
+                count[bh * n + i] = cnt;
+            }
+            free(sc);
+            free(inq);
+            free(ink);
+        }
+}
+
+/* ======================================================================
  * O4h  Hierarchical indexer (HISA), decode rows.  [P2] "索引器的三种降本方向"
  * and §2.2 Eq.(7): the history of a row is cut into blocks of `blk` keys;
  * each complete block has a representative (reading: the mean of its index
