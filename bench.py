@@ -1,13 +1,14 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|lsh_decode|prefill|decode|decode_hisa|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
+                  [--workload lsh|lsh_fp32|lsh_decode|route|prefill|decode|decode_hisa|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
            b=64 buckets, 4 rounds, chunk 128, causal, last 5% padding:
            hash -> sort -> chunked attention -> round merge.  Metric: tokens/s.
   lsh_fp32 fp32 LSH attention, n=1024, b=16, 1 round, chunk 64.
+  route    routing (k-means) attention with quotas, B=2, H=8, n=16384, C=128, m=128.
   lsh_decode  LSH attention in decode: 64 rows x 8 heads, 16384-token prompts in bucket
            lists (64 buckets x 4 rounds) and paged K/V; a step appends one token per row
            and attends with it.
@@ -135,6 +136,61 @@ class LshWorkload(Workload):
                                   ("hbm", attn_bytes / 1e9, "GB/s")],
             "lsh_hash": [("alu", B * H * R * n * d * (p["n_buckets"] // 2) * 2 / 1e12, "TFLOP/s")],
         }
+
+
+class RouteWorkload(Workload):
+    """Routing (k-means) attention with quota execution: B = 2, H = 8, n = 16384, d = 64,
+    C = 128 frozen unit centres, quota m = 128 (C m = n), causal.  A step = routing
+    scores -> quotas -> per-centre attention -> merge.  Metric: tokens/s."""
+
+    def __init__(self, crs, dev):
+        self.crs = crs
+        B, H, n, d, C, m = 2, 8, 16384, 64, 128, 128
+        self.p = dict(B=B, H=H, n=n, d=d, C=C, m=m, causal=1)
+        self.name = f"route_B{B}_H{H}_n{n}_d{d}_C{C}_m{m}_causal"
+        self.units_per_step = B * n
+        g = torch.Generator(device="cpu").manual_seed(81)
+        self.Q = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16).to(dev)
+        self.K = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16).to(dev)
+        self.V = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16).to(dev)
+        M = torch.randn(H, C, d, generator=g)
+        self.M = (M / M.norm(dim=-1, keepdim=True)).to(dev)
+        self.JQ = torch.empty((B, H, C, m), dtype=torch.int32, device=dev)
+        self.JK = torch.empty_like(self.JQ)
+        self.O = torch.empty((B, H, n, d), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((B, H, n), dtype=torch.float32, device=dev)
+        self.cnt = torch.empty((B, H, n), dtype=torch.int32, device=dev)
+        import ctypes
+        rp = crs.RouteParams(B, H, n, d, C, m, 1, 0, 1.0 / math.sqrt(d))
+        self.ws = torch.empty(int(crs.lib().crs_route_attn_workspace_size(ctypes.byref(rp))), dtype=torch.uint8,
+                              device=dev)
+        self.h_in = {k: getattr(self, k).cpu().pin_memory() for k in ("Q", "K", "V")}
+        self.d_in = {k: torch.empty_like(getattr(self, k)) for k in self.h_in}
+        self.h_out = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def _run(self, Q, K, V):
+        self.crs.route_attn(Q, K, V, self.M, self.p["m"], causal=True, out=self.O, lse=self.lse, count=self.cnt,
+                            JQ=self.JQ, JK=self.JK, workspace=self.ws)
+
+    def step(self):
+        self._run(self.Q, self.K, self.V)
+
+    def e2e_step(self):
+        for k, h in self.h_in.items():
+            self.d_in[k].copy_(h, non_blocking=True)
+        self._run(self.d_in["Q"], self.d_in["K"], self.d_in["V"])
+        self.h_out.copy_(self.O, non_blocking=True)
+
+    def roofline_spec(self):
+        p = self.p
+        BH = p["B"] * p["H"]
+        # scores n C d per role (ALU) vs the bytes: Q, K read for the scores, Q, K, V gathered
+        # per centre, O written
+        flops = BH * 2 * p["n"] * p["C"] * p["d"] * 2 + BH * p["C"] * p["m"] * p["m"] * p["d"] * 4
+        byts = BH * (2 * p["n"] * p["d"] * 2 + p["C"] * p["m"] * p["d"] * 2 * 3 + p["n"] * p["d"] * 4)
+        return {"route": [("alu", flops / 1e12, "TFLOP/s"), ("hbm", byts / 1e9, "GB/s")]}
 
 
 class LshDecodeWorkload(Workload):
@@ -516,7 +572,7 @@ class BlockMeanPoolWorkload(BlockWorkload):
 WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
              "prefill": PrefillWorkload, "decode": DecodeWorkload, "decode_hisa": DecodeHisaWorkload,
-             "lsh_decode": LshDecodeWorkload,
+             "lsh_decode": LshDecodeWorkload, "route": RouteWorkload,
              "block": BlockWorkload,
              "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
              "block_meanpool": BlockMeanPoolWorkload, "block_ss": BlockSubspaceWorkload}
@@ -786,7 +842,7 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "lsh_decode", "prefill", "decode", "decode_hisa", "block", "block_fp4", "block_ss",
+        for name in [w for w in ("lsh_fp32", "lsh_decode", "route", "prefill", "decode", "decode_hisa", "block", "block_fp4", "block_ss",
                                   "block_quest", "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)

@@ -77,6 +77,11 @@ class LshDecodeState(ctypes.Structure):
                 ("list_pool", ctypes.c_void_p), ("alloc", ctypes.c_void_p), ("seq_len", ctypes.c_void_p)]
 
 
+class RouteParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "n", "d", "C", "m", "causal", "no_self")] + \
+               [("scale", ctypes.c_float)]
+
+
 class BlockParams(ctypes.Structure):
     _fields_ = [("n_seq", ctypes.c_int), ("n_kv", ctypes.c_int), ("T", ctypes.c_int),
                 ("D", ctypes.c_int), ("L", ctypes.c_int), ("rank", ctypes.c_int),
@@ -133,6 +138,9 @@ _sig("crs_block_select", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP
 _sig("crs_block_quantize", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, _VP, _VP, _VP, _VP])
 _sig("crs_block_select_fp4", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, _VP, _VP, _VP,
                                              _VP, _VP, _SZ, _VP])
+_sig("crs_route_attn_workspace_size", _SZ, [ctypes.POINTER(RouteParams)])
+_sig("crs_route_attn", ctypes.c_int, [ctypes.POINTER(RouteParams), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                       _VP, _SZ, _VP])
 _sig("crs_lsh_decode_prefill", ctypes.c_int, [ctypes.POINTER(LshDecodeParams), ctypes.POINTER(LshDecodeState),
                                                 _VP, _VP, _VP, ctypes.c_int, _VP])
 _sig("crs_lsh_decode_step", ctypes.c_int, [ctypes.POINTER(LshDecodeParams), ctypes.POINTER(LshDecodeState),
@@ -331,6 +339,34 @@ def indexer_topk(q_idx, w, k_idx, topk: int, mode: int = CRS_IDX_PREFILL, k_offs
                                _stream(stream))
     _check("crs_indexer_topk", st)
     return out, count
+
+
+# ---------------------------------------------------------------- routing --
+def route_attn(Q, K, V, M, m: int, causal=True, no_self=False, scale=None, out=None, lse=None, count=None,
+               JQ=None, JK=None, workspace=None, stream=None):
+    """Routing attention with quota execution: Q, K, V [B, H, n, d] bf16, M [H, C, d] f32
+    (frozen centres), quota m -> (JQ, JK [B, H, C, m], O [B, H, n, d] f32, lse, count)."""
+    _need(Q, "Q", torch.bfloat16)
+    B, H, n, d = Q.shape
+    _need(K, "K", torch.bfloat16, (B, H, n, d))
+    _need(V, "V", torch.bfloat16, (B, H, n, d))
+    _need(M, "M", torch.float32)
+    C = M.shape[1]
+    _need(M, "M", torch.float32, (H, C, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    p = RouteParams(B, H, n, d, C, int(m), int(causal), int(no_self), float(scale))
+    dev = Q.device
+    JQ = torch.empty((B, H, C, m), dtype=torch.int32, device=dev) if JQ is None else JQ
+    JK = torch.empty((B, H, C, m), dtype=torch.int32, device=dev) if JK is None else JK
+    out = torch.empty((B, H, n, d), dtype=torch.float32, device=dev) if out is None else out
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=dev) if lse is None else lse
+    count = torch.empty((B, H, n), dtype=torch.int32, device=dev) if count is None else count
+    ws, wsb = _workspace(int(_lib.crs_route_attn_workspace_size(ctypes.byref(p))), dev, workspace)
+    st = _lib.crs_route_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(M), _ptr(JQ), _ptr(JK), _ptr(out),
+                             _ptr(lse), _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_route_attn", st)
+    return JQ, JK, out, lse, count
 
 
 # ------------------------------------------------------------- LSH decode --

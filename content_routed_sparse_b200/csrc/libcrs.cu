@@ -9,4 +9,5 @@
 #include "indexer_tc.cu"
 #include "blocks.cu"
 #include "hisa.cu"
+#include "route.cu"
 #include "noalloc.cu"

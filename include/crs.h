@@ -211,6 +211,32 @@ int crs_lsh_decode_step(const crs_lsh_decode_params *p, const crs_lsh_decode_sta
                         const void *v, const float *rot, float *O, float *lse, int32_t *count, void *stream);
 
 /* ====================================================================== *
+ * Routing (k-means) attention with quota execution.  [P1] §3.1: frozen
+ * centres M [H, C, d] f32; routing scores S_Q = Q M^T, S_K = K M^T, each an
+ * integer decision taken in fp32 as one FMA per term in increasing index order
+ * from 0; centre c keeps its m best queries J_c^Q and m best keys J_c^K
+ * (score desc, index asc), returned ascending in JQ, JK [B, H, C, m] (-1 past
+ * n).  Query i attends to the union of J_c^K over the centres with i in J_c^Q,
+ * each key once, j <= i when causal, j != i when no_self; logits scale * q.k;
+ * fp32 softmax; an empty set gives O = 0, lse = -inf.
+ * Q, K, V: [B, H, n, d] bf16 (16-byte aligned); O [B, H, n, d] f32; lse [B, H, n]
+ * f32 (natural log); count [B, H, n] int32 (keys attended, may be NULL).
+ * d = 64, C <= 256, m <= 256, n <= 16384 (else CRS_ERR_UNSUPPORTED).
+ * ====================================================================== */
+typedef struct {
+    int B, H, n, d;
+    int C;            /* centres per head                                     */
+    int m;            /* quota: queries and keys kept per centre              */
+    int causal, no_self;
+    float scale;
+} crs_route_params;
+
+size_t crs_route_attn_workspace_size(const crs_route_params *p);
+int crs_route_attn(const crs_route_params *p, const void *Q, const void *K, const void *V, const float *M,
+                   int32_t *JQ, int32_t *JK, float *O, float *lse, int32_t *count, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/* ====================================================================== *
  * Lightning indexer + token top-k.  [P2] §1.1 / §2.1 Eq.(2)-(4):
  *   r_{t,s} = sum_h w_{t,h} ReLU(q_{t,h} . k_s)   (no extra scale)
  * S_t = the topk positions with the largest r_{t,s}, ties to the smaller
