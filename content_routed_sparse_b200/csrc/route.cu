@@ -12,8 +12,8 @@
 //                         (an integer decision, taken as the oracle takes it),
 //                         stored as order-preserving keys [role][c][token]
 //   route_quota_kernel    one 1024-thread CTA per (b, h, role, c): 4-pass 8-bit
-//                         radix select of the m-th key (warp-aggregated shared
-//                         histograms), ties to the smaller index by prefix sums,
+//                         radix select of the m-th key (one shared histogram per
+//                         warp, then summed), ties to the smaller index by prefix sums,
 //                         the kept tokens ascending + membership bitmaps
 //   route_attn_kernel     one CTA per (b, h, c): thread = query of the centre,
 //                         the centre's keys and values staged in shared memory,
@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(256) route_score_kernel(RtArgs a) {
 
 template <int KPT>
 __global__ void __launch_bounds__(kPickT) route_quota_kernel(RtArgs a) {
+    __shared__ uint32_t whist[kPickT / 32][256];           // one histogram per warp
     __shared__ uint32_t hist[256];
     __shared__ int sbin, sneed;
     __shared__ int2 wtot[kPickT / 32 + 1];
@@ -96,14 +97,17 @@ __global__ void __launch_bounds__(kPickT) route_quota_kernel(RtArgs a) {
     int need = a.mm;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
-        for (int e = tid; e < 256; e += kPickT) hist[e] = 0u;
-        __syncthreads();
+        for (int e = lane; e < 256; e += 32) whist[warp][e] = 0u;
+        __syncwarp();
 #pragma unroll
-        for (int u = 0; u < KPT; ++u) {
-            const bool in = valid[u] && (key[u] & mask) == prefix;
-            const int dg = in ? (int)((key[u] >> shift) & 255u) : -1 - lane;
-            const unsigned grp = __match_any_sync(0xffffffffu, dg);
-            if (in && (__ffs(grp) - 1) == lane) atomicAdd(&hist[dg], (uint32_t)__popc(grp));
+        for (int u = 0; u < KPT; ++u)
+            if (valid[u] && (key[u] & mask) == prefix) atomicAdd(&whist[warp][(key[u] >> shift) & 255u], 1u);
+        __syncthreads();
+        for (int e = tid; e < 256; e += kPickT) {
+            uint32_t v = 0u;
+#pragma unroll 8
+            for (int w = 0; w < kPickT / 32; ++w) v += whist[w][e];
+            hist[e] = v;
         }
         __syncthreads();
         if (warp == 0) {
