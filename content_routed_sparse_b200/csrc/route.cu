@@ -15,12 +15,14 @@
 //                         radix select of the m-th key (one shared histogram per
 //                         warp, then summed), ties to the smaller index by prefix sums,
 //                         the kept tokens ascending + membership bitmaps
-//   route_attn_kernel     one CTA per (b, h, c): thread = query of the centre,
+//   route_attn_tc_kernel  one CTA per (b, h, c) for m <= 128: S = Q K^T and P V on
+//                         mma.sync tiles, masks per element, exact softmax;
+//   route_attn_kernel     (m > 128) one CTA per (b, h, c): thread = query of the centre,
 //                         the centre's keys and values staged in shared memory,
 //                         causal / self / earlier-centre pairs masked, online
 //                         softmax; partial (o, lse, count) per (c, slot)
 //   route_merge_kernel    one warp per query: its centres' partials combined
-//                         by log-sum-exp (slot found by binary search)
+//                         by log-sum-exp (slots recorded by the quota kernel)
 #include "common.cuh"
 
 namespace crs {
@@ -35,6 +37,7 @@ struct RtArgs {
     const float *M;                        // [H, C, d]
     uint32_t *keys;                        // [B, H, 2, C, n]
     uint32_t *memb;                        // [B, H, 2, n, C/32]
+    uint8_t *qslot;                        // [B, H, n, C]: slot of query i in J_c^Q
     int32_t *JQ, *JK;                      // [B, H, C, m]
     float *part_o, *part_lse;              // [B, H, C, m, d], [B, H, C, m]
     int32_t *part_cnt;                     // [B, H, C, m]
@@ -66,12 +69,27 @@ __global__ void __launch_bounds__(256) route_score_kernel(RtArgs a) {
         }
     }
     uint32_t *out = a.keys + ((size_t)bh * 2 + role) * a.C * a.n;
-    for (int c = threadIdx.x >> 6; c < a.C; c += 4) {
-        const float *mu = rt_mu + c * kRtD;
-        float acc = 0.0f;
+    // two centres at a time (two independent chains), the centre read 4 values per load;
+    // each chain is still one FMA per term in index order from 0
+    for (int c = threadIdx.x >> 6; c < a.C; c += 8) {
+        const int c2 = c + 4 < a.C ? c + 4 : c;
+        const float4 *mu0 = reinterpret_cast<const float4 *>(rt_mu + c * kRtD);
+        const float4 *mu1 = reinterpret_cast<const float4 *>(rt_mu + c2 * kRtD);
+        float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
-        for (int i = 0; i < kRtD; ++i) acc = fmaf(xv[i], mu[i], acc);   // index order from 0
-        out[(size_t)c * a.n + t] = score_key(acc);
+        for (int i4 = 0; i4 < kRtD / 4; ++i4) {
+            const float4 m0 = mu0[i4], m1 = mu1[i4];
+            acc0 = fmaf(xv[4 * i4], m0.x, acc0);
+            acc1 = fmaf(xv[4 * i4], m1.x, acc1);
+            acc0 = fmaf(xv[4 * i4 + 1], m0.y, acc0);
+            acc1 = fmaf(xv[4 * i4 + 1], m1.y, acc1);
+            acc0 = fmaf(xv[4 * i4 + 2], m0.z, acc0);
+            acc1 = fmaf(xv[4 * i4 + 2], m1.z, acc1);
+            acc0 = fmaf(xv[4 * i4 + 3], m0.w, acc0);
+            acc1 = fmaf(xv[4 * i4 + 3], m1.w, acc1);
+        }
+        out[(size_t)c * a.n + t] = score_key(acc0);
+        if (c2 != c) out[(size_t)c2 * a.n + t] = score_key(acc1);
     }
 }
 
@@ -147,6 +165,7 @@ __global__ void __launch_bounds__(kPickT) route_quota_kernel(RtArgs a) {
     for (int u = 0; u < KPT; ++u)
         if (take[u]) {
             const int i = tid * KPT + u;
+            if (role == 0) a.qslot[((size_t)bh * a.n + i) * a.C + c] = (uint8_t)slot;
             J[slot++] = i;
             atomicOr(&mb[(size_t)i * a.words + (c >> 5)], 1u << (c & 31));
         }
@@ -239,6 +258,184 @@ __global__ void __launch_bounds__(kRtMaxM) route_attn_kernel(RtArgs a) {
     a.part_cnt[ps] = cnt;
 }
 
+// The same per-centre attention on the tensor cores (mma.sync m16n8k16, bf16 in,
+// fp32 accumulate) for quotas up to 128: the centre's query, key and value rows
+// are staged in 128B-swizzled shared rows; warp w takes query slots 16w..16w+15
+// against all 128 key slots: S = Q K^T (16 n-tiles), the causal / self /
+// earlier-centre masks per element (key membership words in shared memory,
+// the query's earlier-centre words in registers), an exact softmax over the
+// 128 slots, then O = P V with P carried as a bf16 value + bf16 residual.
+constexpr int kRtTcM = 128;
+constexpr int kRtMaxWords = kRtMaxC / 32;
+
+__device__ __forceinline__ uint32_t rt_sw(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
+struct RtTcSmem {
+    unsigned char q[kRtTcM * 128], k[kRtTcM * 128], v[kRtTcM * 128];   // 64 bf16 per row
+    int qi[kRtTcM], kj[kRtTcM];
+    uint32_t km[kRtTcM][kRtMaxWords];
+};
+
+__global__ void __launch_bounds__(256) route_attn_tc_kernel(RtArgs a) {
+    extern __shared__ __align__(128) unsigned char rt_tc_raw[];
+    RtTcSmem &S = *reinterpret_cast<RtTcSmem *>(rt_tc_raw);
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t *JQ = a.JQ + ((size_t)bh * a.C + c) * a.m, *JK = a.JK + ((size_t)bh * a.C + c) * a.m;
+    const uint32_t *mkb = a.memb + ((size_t)bh * 2 + 1) * a.n * a.words;
+    for (int e = tid; e < kRtTcM * 8; e += 256) {
+        const int r = e >> 3, ch = e & 7;
+        const int i = r < a.mm ? JQ[r] : -1, j = r < a.mm ? JK[r] : -1;
+        uint4 qv = make_uint4(0, 0, 0, 0), kv = qv, vv = qv;
+        if (i >= 0) qv = __ldg(reinterpret_cast<const uint4 *>(a.Q + ((size_t)bh * a.n + i) * kRtD) + ch);
+        if (j >= 0) {
+            kv = __ldg(reinterpret_cast<const uint4 *>(a.K + ((size_t)bh * a.n + j) * kRtD) + ch);
+            vv = __ldg(reinterpret_cast<const uint4 *>(a.V + ((size_t)bh * a.n + j) * kRtD) + ch);
+        }
+        *reinterpret_cast<uint4 *>(S.q + rt_sw(r, ch)) = qv;
+        *reinterpret_cast<uint4 *>(S.k + rt_sw(r, ch)) = kv;
+        *reinterpret_cast<uint4 *>(S.v + rt_sw(r, ch)) = vv;
+        if (ch == 0) {
+            S.qi[r] = i;
+            S.kj[r] = j;
+        }
+        if (ch < kRtMaxWords) S.km[r][ch] = (j >= 0 && ch < a.words) ? mkb[(size_t)j * a.words + ch] : 0u;
+    }
+    __syncthreads();
+    const int r0 = warp * 16;
+    if (r0 >= a.mm) return;
+    const int g_row = lane >> 2, tig = lane & 3;
+    // query fragments: 16 rows x 64 dims, 4 k-steps
+    uint32_t qf[4][4];
+    {
+        const uint32_t qb = smem_u32(S.q);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int mi = lane >> 3, r = r0 + (lane & 7) + ((mi & 1) << 3), ch = kk * 2 + (mi >> 1);
+            ldsm_x4(qb + rt_sw(r, ch), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+        }
+    }
+    float sc[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
+    {
+        const uint32_t kb = smem_u32(S.k);
+#pragma unroll
+        for (int np = 0; np < 8; ++np)                  // pairs of n-tiles: 16 keys
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int mi = lane >> 3;
+                const int r = np * 16 + (lane & 7) + ((mi >> 1) << 3), ch = kk * 2 + (mi & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kb + rt_sw(r, ch), b0, b1, b2, b3);
+                mma_bf16(sc[2 * np], qf[kk], b0, b1);
+                mma_bf16(sc[2 * np + 1], qf[kk], b2, b3);
+            }
+    }
+    // masks: rows g_row (lo) and g_row + 8 (hi) of this warp's 16
+    const int rl = r0 + g_row, rh = r0 + g_row + 8;
+    const int il = rl < a.mm ? S.qi[rl] : -1, ih = rh < a.mm ? S.qi[rh] : -1;
+    uint32_t ql[kRtMaxWords], qh[kRtMaxWords];
+    const uint32_t *mqb = a.memb + ((size_t)bh * 2 + 0) * a.n * a.words;
+#pragma unroll
+    for (int w = 0; w < kRtMaxWords; ++w) {
+        const uint32_t lowmask = w < (c >> 5) ? 0xffffffffu : (w == (c >> 5) ? (1u << (c & 31)) - 1u : 0u);
+        ql[w] = (il >= 0 && w < a.words) ? mqb[(size_t)il * a.words + w] & lowmask : 0u;
+        qh[w] = (ih >= 0 && w < a.words) ? mqb[(size_t)ih * a.words + w] & lowmask : 0u;
+    }
+    const float sl2 = a.scale * 1.4426950408889634f;
+    float mxl = -INFINITY, mxh = -INFINITY;
+    int cl = 0, ch_ = 0;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int col = nt * 8 + tig * 2 + e;
+            const int j = S.kj[col];
+            bool metl = false, meth = false;
+#pragma unroll
+            for (int w = 0; w < kRtMaxWords; ++w) {
+                const uint32_t kw = S.km[col][w];
+                metl |= (ql[w] & kw) != 0u;
+                meth |= (qh[w] & kw) != 0u;
+            }
+            const bool okl = il >= 0 && j >= 0 && !(a.causal && j > il) && !(a.no_self && j == il) && !metl;
+            const bool okh = ih >= 0 && j >= 0 && !(a.causal && j > ih) && !(a.no_self && j == ih) && !meth;
+            sc[nt][e] = okl ? sc[nt][e] * sl2 : -INFINITY;
+            sc[nt][2 + e] = okh ? sc[nt][2 + e] * sl2 : -INFINITY;
+            mxl = fmaxf(mxl, sc[nt][e]);
+            mxh = fmaxf(mxh, sc[nt][2 + e]);
+            cl += okl ? 1 : 0;
+            ch_ += okh ? 1 : 0;
+        }
+    mxl = fmaxf(mxl, __shfl_xor_sync(0xffffffffu, mxl, 1));
+    mxl = fmaxf(mxl, __shfl_xor_sync(0xffffffffu, mxl, 2));
+    mxh = fmaxf(mxh, __shfl_xor_sync(0xffffffffu, mxh, 1));
+    mxh = fmaxf(mxh, __shfl_xor_sync(0xffffffffu, mxh, 2));
+    float sum_l = 0.0f, sum_h = 0.0f;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            sc[nt][e] = sc[nt][e] == -INFINITY ? 0.0f : exp2f(sc[nt][e] - mxl);
+            sc[nt][2 + e] = sc[nt][2 + e] == -INFINITY ? 0.0f : exp2f(sc[nt][2 + e] - mxh);
+            sum_l += sc[nt][e];
+            sum_h += sc[nt][2 + e];
+        }
+    sum_l += __shfl_xor_sync(0xffffffffu, sum_l, 1);
+    sum_l += __shfl_xor_sync(0xffffffffu, sum_l, 2);
+    sum_h += __shfl_xor_sync(0xffffffffu, sum_h, 1);
+    sum_h += __shfl_xor_sync(0xffffffffu, sum_h, 2);
+    cl += __shfl_xor_sync(0xffffffffu, cl, 1);
+    cl += __shfl_xor_sync(0xffffffffu, cl, 2);
+    ch_ += __shfl_xor_sync(0xffffffffu, ch_, 1);
+    ch_ += __shfl_xor_sync(0xffffffffu, ch_, 2);
+    // O = P V
+    float o[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
+    const uint32_t vb = smem_u32(S.v);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {                      // 16 key slots per k-step
+        uint32_t pa[4], pl[4];
+        pack_bf16_split(sc[2 * kk][0], sc[2 * kk][1], pa[0], pl[0]);
+        pack_bf16_split(sc[2 * kk][2], sc[2 * kk][3], pa[1], pl[1]);
+        pack_bf16_split(sc[2 * kk + 1][0], sc[2 * kk + 1][1], pa[2], pl[2]);
+        pack_bf16_split(sc[2 * kk + 1][2], sc[2 * kk + 1][3], pa[3], pl[3]);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {                  // 16 dims per step
+            const int mi = lane >> 3;
+            const int r = kk * 16 + (lane & 7) + ((mi & 1) << 3), chn = jj * 2 + (mi >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vb + rt_sw(r, chn), b0, b1, b2, b3);
+            mma_bf16(o[2 * jj], pa, b0, b1);
+            mma_bf16(o[2 * jj], pl, b0, b1);
+            mma_bf16(o[2 * jj + 1], pa, b2, b3);
+            mma_bf16(o[2 * jj + 1], pl, b2, b3);
+        }
+    }
+    const float il_ = sum_l > 0.0f ? 1.0f / sum_l : 0.0f, ih_ = sum_h > 0.0f ? 1.0f / sum_h : 0.0f;
+    const size_t pbase = ((size_t)bh * a.C + c) * a.m;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int col = nt * 8 + tig * 2;
+        if (rl < a.mm)
+            *reinterpret_cast<float2 *>(a.part_o + (pbase + rl) * kRtD + col) = make_float2(o[nt][0] * il_, o[nt][1] * il_);
+        if (rh < a.mm)
+            *reinterpret_cast<float2 *>(a.part_o + (pbase + rh) * kRtD + col) = make_float2(o[nt][2] * ih_, o[nt][3] * ih_);
+    }
+    if (tig == 0) {
+        const float ln2 = 0.6931471805599453f;
+        if (rl < a.mm) {
+            a.part_lse[pbase + rl] = cl > 0 ? (mxl + log2f(sum_l)) * ln2 : -INFINITY;
+            a.part_cnt[pbase + rl] = cl;
+        }
+        if (rh < a.mm) {
+            a.part_lse[pbase + rh] = ch_ > 0 ? (mxh + log2f(sum_h)) * ln2 : -INFINITY;
+            a.part_cnt[pbase + rh] = ch_;
+        }
+    }
+}
+
 // one warp per (b, h, i): lanes own dims 2l, 2l + 1
 __global__ void __launch_bounds__(256) route_merge_kernel(RtArgs a) {
     const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -255,14 +452,8 @@ __global__ void __launch_bounds__(256) route_merge_kernel(RtArgs a) {
             while (bits) {
                 const int c = wd * 32 + __ffs(bits) - 1;
                 bits &= bits - 1u;
-                const int32_t *J = a.JQ + ((size_t)bh * a.C + c) * a.m;
-                int lo = 0, hi = a.mm - 1;                         // J ascending: find i
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (J[mid] < i) lo = mid + 1;
-                    else hi = mid;
-                }
-                const size_t ps = ((size_t)bh * a.C + c) * a.m + lo;
+                const int slot = a.qslot[((size_t)bh * a.n + i) * a.C + c];
+                const size_t ps = ((size_t)bh * a.C + c) * a.m + slot;
                 const float ls = a.part_lse[ps];
                 if (pass == 0) {
                     M = fmaxf(M, ls);
@@ -290,6 +481,7 @@ __global__ void __launch_bounds__(256) route_merge_kernel(RtArgs a) {
 
 struct RtWs {
     uint32_t *keys, *memb;
+    uint8_t *qslot;
     float *part_o, *part_lse;
     int32_t *part_cnt;
     size_t total;
@@ -310,6 +502,7 @@ static void rt_ws_layout(const crs_route_params *p, RtWs &w, char *base) {
     auto take = [&](size_t bytes) { char *q = base ? base + off : nullptr; off += al(bytes); return q; };
     w.keys = reinterpret_cast<uint32_t *>(take(bh * 2 * p->C * p->n * 4));
     w.memb = reinterpret_cast<uint32_t *>(take(bh * 2 * p->n * words * 4));
+    w.qslot = reinterpret_cast<uint8_t *>(take(bh * p->n * p->C));
     w.part_o = reinterpret_cast<float *>(take(bh * p->C * p->m * kRtD * 4));
     w.part_lse = reinterpret_cast<float *>(take(bh * p->C * p->m * 4));
     w.part_cnt = reinterpret_cast<int32_t *>(take(bh * p->C * p->m * 4));
@@ -346,6 +539,7 @@ extern "C" int crs_route_attn(const crs_route_params *p, const void *Q, const vo
     a.M = M;
     a.keys = w.keys;
     a.memb = w.memb;
+    a.qslot = w.qslot;
     a.JQ = JQ;
     a.JK = JK;
     a.part_o = w.part_o;
@@ -379,9 +573,15 @@ extern "C" int crs_route_attn(const crs_route_params *p, const void *Q, const vo
     else if (kpt <= 4) route_quota_kernel<4><<<gq, kPickT, 0, s>>>(a);
     else if (kpt <= 8) route_quota_kernel<8><<<gq, kPickT, 0, s>>>(a);
     else route_quota_kernel<16><<<gq, kPickT, 0, s>>>(a);
-    CRS_TRY_CUDA(cudaFuncSetAttribute(route_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)rt_attn_smem(a.mm)));
-    route_attn_kernel<<<dim3(p->C, BH), max(32, ceil_div(a.mm, 32) * 32), rt_attn_smem(a.mm), s>>>(a);
+    if (a.mm <= kRtTcM) {
+        CRS_TRY_CUDA(cudaFuncSetAttribute(route_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)sizeof(RtTcSmem)));
+        route_attn_tc_kernel<<<dim3(p->C, BH), 256, sizeof(RtTcSmem), s>>>(a);
+    } else {
+        CRS_TRY_CUDA(cudaFuncSetAttribute(route_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)rt_attn_smem(a.mm)));
+        route_attn_kernel<<<dim3(p->C, BH), max(32, ceil_div(a.mm, 32) * 32), rt_attn_smem(a.mm), s>>>(a);
+    }
     route_merge_kernel<<<(unsigned)ceil_div((long long)BH * p->n, 8), 256, 0, s>>>(a);
     CRS_CHECK_LAUNCH();
     return CRS_OK;
