@@ -23,11 +23,15 @@
 //      reusing the K tile's space (S is complete by then);
 //   5. after each half, one thread issues O += P_hi V_half + P_lo V_half
 //      (M=128, N=64, V as an MN-major operand) into TMEM columns [0, 64),
-//      which the first half's S no longer needs;
+//      which the first half's S no longer needs.  When every row bound is
+//      small and V is fp16-representable (the usual case), the CTA instead
+//      converts its V tile to fp16, writes P = 2^(S - bound + 15) for all 256
+//      keys as fp16 in one sweep and issues a single fp16 chain O = P V;
 //   6. the epilogue divides by the row sum and writes o_r and lse_r at the
 //      ORIGINAL position; lsh_combine_kernel merges the rounds.
 // Resources per CTA: 256 TMEM columns, ~107 KB shared memory, 256 threads,
 // so two CTAs share an SM and overlap each other's latency.
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -44,6 +48,7 @@ constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s: a wait that long means a
 constexpr int kBktBefore = -1;                  // absent slot before the sequence
 constexpr int kBktAfter = 0x7fffffff;           // absent slot after the sequence
 constexpr float kTcBoundMax = 48.0f;            // single pass while 2^(-2 bound) stays normal
+constexpr float kTcBoundMax16 = 14.0f;          // fp16 P while 2^(15 - 2 bound) stays fp16-normal
 
 struct LshTcSmem {
     // K tile (rows = keys; rows 128..255 = Q tile) until S is computed, then
@@ -248,6 +253,88 @@ __device__ __forceinline__ float lsh_tc_fused(LshTcSmem &S, const LshTcRow &q, u
     return sum;
 }
 
+// Single pass with fp16 P for all 256 keys at once (the CTA has checked that
+// every bound is at most kTcBoundMax16 and that every V value is below 2^16 in
+// magnitude, so its fp16 copy is exact from 2^-14 up and within 2^-25 below):
+// P = 2^(S - M) with M = bound - 15 lies in [2^(15 - 2 bound), 2^15], inside
+// the fp16 normal range, so one rounding (relative 2^-12) is the only error P
+// adds.  Warpgroup wg writes keys [128 wg, 128 wg + 128) = P blocks 2wg, 2wg+1.
+// The earlier-round pair test is folded into each element's predicate.
+template <int NR>
+__device__ __forceinline__ float lsh_tc_fused16(LshTcSmem &S, const LshTcRow &q, uint32_t trow, int wg,
+                                                float M, int r) {
+    constexpr int NRR = NR >= 0 ? NR : kMaxRounds - 1;
+    const int R = NR >= 0 ? NR : r;
+    int ci[NRR > 0 ? NRR : 1];
+#pragma unroll
+    for (int rr = 0; rr < NRR; ++rr) ci[rr] = rr < R ? S.kcode[rr][q.jq] : 0;
+    float2 sum2 = make_float2(0.0f, 0.0f);
+    const float2 negM = make_float2(-M, -M);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        const int c0 = wg * 128 + cc * 32;
+        uint32_t mb = q.qvalid ? range_bits(q.lo, q.hi, c0) : 0u;
+        if (q.excl_self && q.jq >= c0 && q.jq < c0 + 32) mb &= ~(1u << (q.jq - c0));
+        uint32_t ph[16];
+        if (__any_sync(0xffffffffu, mb != 0u)) {
+            uint32_t v[32];
+            tc::tmem_ld32(trow + c0, v);
+            tc::tmem_ld_wait();
+            const float4 *ks = reinterpret_cast<const float4 *>(&S.kscale[c0]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 k4 = ks[u];
+                bool ok[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ok[e] = (mb >> (4 * u + e)) & 1u;
+#pragma unroll
+                for (int rr = 0; rr < NRR; ++rr) {
+                    if (NR < 0 && rr >= R) break;
+                    const int4 kc = reinterpret_cast<const int4 *>(&S.kcode[rr][c0])[u];
+                    ok[0] = ok[0] && (uint32_t)(ci[rr] - kc.x) > 1u;
+                    ok[1] = ok[1] && (uint32_t)(ci[rr] - kc.y) > 1u;
+                    ok[2] = ok[2] && (uint32_t)(ci[rr] - kc.z) > 1u;
+                    ok[3] = ok[3] && (uint32_t)(ci[rr] - kc.w) > 1u;
+                }
+                const float2 a = __ffma2_rn(make_float2(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1])),
+                                            make_float2(k4.x, k4.y), negM);
+                const float2 b = __ffma2_rn(make_float2(__uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3])),
+                                            make_float2(k4.z, k4.w), negM);
+                const float2 p01 = make_float2(ok[0] ? ex2_approx(a.x) : 0.0f, ok[1] ? ex2_approx(a.y) : 0.0f);
+                const float2 p23 = make_float2(ok[2] ? ex2_approx(b.x) : 0.0f, ok[3] ? ex2_approx(b.y) : 0.0f);
+                sum2 = __fadd2_rn(sum2, p01);
+                sum2 = __fadd2_rn(sum2, p23);
+                const __half2 h01 = __floats2half2_rn(p01.x, p01.y);
+                const __half2 h23 = __floats2half2_rn(p23.x, p23.y);
+                ph[2 * u] = *reinterpret_cast<const uint32_t *>(&h01);
+                ph[2 * u + 1] = *reinterpret_cast<const uint32_t *>(&h23);
+            }
+        } else {
+#pragma unroll
+            for (int t2 = 0; t2 < 16; ++t2) ph[t2] = 0u;
+        }
+        unsigned char *pb = S.kp[2 * wg + (cc >> 1)];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4 *>(pb + tc::sw128(q.row, (cc & 1) * 4 + u)) =
+                make_uint4(ph[u * 4], ph[u * 4 + 1], ph[u * 4 + 2], ph[u * 4 + 3]);
+    }
+    return sum2.x + sum2.y;
+}
+
+// O (TMEM columns [0, 64)) = P V over all 256 keys, fp16 operands (P K-major
+// in blocks of 64 keys, V MN-major), one chain of 16 MMAs.
+__device__ __forceinline__ void lsh_tc_issue_pv16(LshTcSmem &S, uint32_t tmem) {
+    constexpr uint32_t idesc = tc::idesc_f16_f32(kTcM, kTcD, 0, 1);
+    const uint32_t vbase = smem_u32(S.v);
+#pragma unroll
+    for (int kk = 0; kk < kTcN / 16; ++kk) {
+        const uint64_t a = tc::smem_desc(smem_u32(S.kp[kk >> 2]) + (kk & 3) * 32, 16, 1024, tc::kLayoutSW128);
+        const uint64_t bd = tc::smem_desc(vbase + kk * 16 * 128, 32768, 1024, tc::kLayoutSW128);
+        tc::mma_bf16(tmem, a, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
 // O (TMEM columns [0, 64)) += P_hi V_half + P_lo V_half for keys [128 half, +128).
 __device__ __forceinline__ void lsh_tc_issue_pv(LshTcSmem &S, uint32_t tmem, int half,
                                                 bool first) {
@@ -360,9 +447,27 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
-    bool big = false;
+    bool big = false, no16 = false;
+    uint4 v16[8];                                 // row j of V as fp16, stored if the CTA takes fp16 P
     {
         const int j = tid;
+        uint32_t vbad = 0u;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(S.v + tc::sw128(j, ch));
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            uint32_t hh[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                // |bf16| >= 2^16 (or Inf / NaN) does not convert exactly: bit 15 of each half of
+                // (w & 0x7fff7fff) + 0x38803880 is set exactly when the half's magnitude bits reach 0x4780
+                vbad |= ((ww[t] & 0x7fff7fffu) + 0x38803880u) & 0x80008000u;
+                const __half2 h = __floats2half2_rn(__uint_as_float(ww[t] << 16), __uint_as_float(ww[t] & 0xffff0000u));
+                hh[t] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            v16[ch] = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+        }
+        no16 = vbad != 0u;
         float ss = 0.0f;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -382,11 +487,18 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
             const float bound = sqrtf(ss) * fabsf(scale_log2);
             S.rowmax[1][j - kTcM] = bound;
             big = bound > kTcBoundMax;
+            no16 = no16 || !(bound <= kTcBoundMax16);
         }
     }
-    tc::fence_proxy_async();
-    // single pass unless keys are raw or some bound is so large that 2^(S - bound) could underflow
+    // single pass unless keys are raw or some bound is so large that 2^(S - bound) could underflow;
+    // fp16 P when, in addition, all of V is exact in fp16 and 2^(S - bound + 15) stays fp16-normal
     const bool single = key_norm && !__syncthreads_or(big);
+    const bool use16 = single && !__syncthreads_or(no16);
+    if (use16) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(S.v + tc::sw128(tid, ch)) = v16[ch];
+    }
+    tc::fence_proxy_async();
     const uint32_t tmem = S.tmem_base;
 
     // ---- 3. S = Q K^T into TMEM columns [0, 256)
@@ -424,7 +536,9 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         // ---- 4a. the exponent shift M: the row bound (single pass), or pass 1's
         // masks and row maxima
         float M;
-        if (single) {
+        if (use16) {
+            M = S.rowmax[1][q.row] - 15.0f;
+        } else if (single) {
             M = S.rowmax[1][q.row];
         } else {
             float mx;
@@ -444,9 +558,27 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
             M = fmaxf(S.rowmax[0][q.row], S.rowmax[1][q.row]);
         }
 
-        // ---- 4b/5. per 128-key half: P into the buffer, then O += P V_half
+        // ---- 4b/5. fp16 P: all 256 keys, then O = P V in one chain; otherwise per
+        // 128-key half: P (value + residual) into the buffer, then O += P V_half
         float sum = 0.0f;
-        for (int half = 0; half < 2; ++half) {
+        if (use16) {
+            switch (r) {
+                case 0: sum = lsh_tc_fused16<0>(S, q, trow, wg, M, r); break;
+                case 1: sum = lsh_tc_fused16<1>(S, q, trow, wg, M, r); break;
+                case 2: sum = lsh_tc_fused16<2>(S, q, trow, wg, M, r); break;
+                case 3: sum = lsh_tc_fused16<3>(S, q, trow, wg, M, r); break;
+                default: sum = lsh_tc_fused16<-1>(S, q, trow, wg, M, r); break;
+            }
+            tc::fence_proxy_async();
+            tc::fence_before();
+            __syncthreads();
+            tc::fence_after();
+            if (tid == 0) {
+                lsh_tc_issue_pv16(S, tmem);
+                tc::commit(&S.bar[2]);
+            }
+        }
+        for (int half = 0; half < 2 && !use16; ++half) {
             if (half == 1) {
                 // the buffer is free once the first half's P.V has completed
                 ok_wait = tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 3);

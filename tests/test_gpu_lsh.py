@@ -35,7 +35,7 @@ def _route_and_check(crs, case):
     return bucket, perm, inv, ob, op, oi
 
 
-def _attn_and_check(crs, case, bucket, perm, inv, ob, op, oi, rows=None):
+def _attn_and_check(crs, case, bucket, perm, inv, ob, op, oi, rows=None, unit=None):
     p = case["params"]
     O, lse = crs.lsh_attn(case["QK"], case["V"], bucket, perm, inv, case["valid_len"],
                           n_buckets=p["n_buckets"], chunk=p["chunk"], causal=p["causal"],
@@ -55,7 +55,10 @@ def _attn_and_check(crs, case, bucket, perm, inv, ob, op, oi, rows=None):
         gO = gO[:, :, rows]
         gl = gl[:, :, rows]
     tol = TOL[p["dtype"]]
-    err = np.abs(gO - oO) / np.maximum(1.0, np.abs(oO))
+    # `unit`: per (b, h) scale of V (the output is linear in V, so a head whose V is
+    # multiplied by 2^k is compared in units of 2^k)
+    u = 1.0 if unit is None else np.asarray(unit, dtype=np.float64)[:, :, None, None]
+    err = np.abs(gO - oO) / np.maximum(u, np.abs(oO))
     assert err.max() <= tol, f"max rel err {err.max():.3e} > {tol}"
     fin = np.isfinite(olse)
     assert (np.isfinite(gl) == fin).all()
@@ -100,6 +103,30 @@ def test_lsh_bf16_tensor_core_path(crs, cuda_dev, n, rounds, nb, causal, no_self
     r = _route_and_check(crs, case)
     _attn_and_check(crs, case, *r)
     assert "lsh_chunk_attn_tc" in crs.profile_collect()
+
+
+@pytest.mark.parametrize("variant", ["v_large_head", "v_large_one", "bound_mid", "bound_big"])
+def test_lsh_bf16_tc_precision_paths(crs, cuda_dev, variant):
+    """The tensor-core kernel's P formats: fp16 P (bounds <= 14 and V below 2^16 in
+    magnitude), the bf16 value + residual single pass (V not fp16-representable, or a row
+    bound in (14, 48]) and the two-pass path (bound > 48).  Each CTA picks its path alone:
+    one large V entry moves only the CTAs whose window holds it."""
+    case = workloads.lsh_clustered_case(B=1, H=2, n=1024, n_buckets=16, n_rounds=3, chunk=128,
+                                        n_centres=8, pad_frac=0.05, seed=77, device=cuda_dev)
+    V = case["V"].float()
+    unit = np.ones((1, 2))
+    if variant == "v_large_head":        # exact scaling: bf16(2^17 v) = 2^17 bf16(v)
+        V[0, 1] *= 2.0 ** 17
+        unit[0, 1] = 2.0 ** 17
+    elif variant == "v_large_one":
+        V[0, 0, 500, 3] = 1.0e6
+    elif variant == "bound_mid":          # |q| ~ 1.3: bound ~ 18.5 (log2 units)
+        case["params"]["scale"] = 10.0
+    else:                                 # bound ~ 370
+        case["params"]["scale"] = 200.0
+    case["V"] = V.to(torch.bfloat16)
+    r = _route_and_check(crs, case)
+    _attn_and_check(crs, case, *r, unit=unit)
 
 
 def test_lsh_fp32_variants(crs, cuda_dev):
