@@ -1446,6 +1446,7 @@ extern "C" int crs_block_select_ss(const crs_block_sel_params *p, const void *Q,
                                       (int)smem_a));
     {
         ProfScope _ps(K_BLK_SCORE, s);
+        _ps.more(1);                              // projection + scorer
         query_project_kernel<<<ceil_div(n_rows, 8), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Q), U, qx,
                                                                   n_rows, sd, p->scale);
         block_score_kernel<<<dim3(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv), kBsThreads, smem_a, s>>>(

@@ -159,11 +159,15 @@ enum KernelId {
 };
 void prof_begin(int id, cudaStream_t s, void **ev_start);
 void prof_end(int id, cudaStream_t s, void *ev_start);
+void prof_add_launches(int id, int k);
+// One scope counts one kernel launch; a scope that launches more kernels
+// calls more(k) for the k further launches.
 struct ProfScope {
     int id;
     cudaStream_t s;
     void *ev;
     ProfScope(int id_, cudaStream_t s_) : id(id_), s(s_), ev(nullptr) { prof_begin(id, s, &ev); }
     ~ProfScope() { prof_end(id, s, ev); }
+    void more(int k) { prof_add_launches(id, k); }
 };
 }  // namespace crs

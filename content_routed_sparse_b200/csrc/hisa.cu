@@ -421,6 +421,7 @@ extern "C" int crs_hisa_topk(const crs_hisa_params *p, const void *q_idx, const 
     case 8: hisa_pick_tokens_kernel<8><<<p->n_rows, kPickT, 0, s>>>(a); break;
     default: hisa_pick_tokens_kernel<16><<<p->n_rows, kPickT, 0, s>>>(a); break;
     }
+    _ps.more(max_blocks > 0 ? 3 : 2);             // coarse, block pick, fine, token pick
     CRS_CHECK_LAUNCH();
     return CRS_OK;
 }

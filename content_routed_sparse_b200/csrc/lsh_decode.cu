@@ -338,6 +338,7 @@ static int ld_run(const crs_lsh_decode_params *p, const crs_lsh_decode_state *st
     lsd_append_kernel<<<ceil_div(p->n_seq * p->n_heads * p->n_rounds, 8), 256, 0, s>>>(a);
     if (O) lsd_attend_kernel<<<p->n_seq * p->n_heads, kLdAttWarps * 32, 0, s>>>(a);
     lsd_advance_kernel<<<ceil_div(p->n_seq, 128), 128, 0, s>>>(st->seq_len, p->n_seq, n_new, p->max_len);
+    _ps.more(O ? 4 : 3);                          // hash, store, append, (attend,) advance
     CRS_CHECK_LAUNCH();
     return CRS_OK;
 }

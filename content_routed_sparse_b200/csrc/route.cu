@@ -583,6 +583,7 @@ extern "C" int crs_route_attn(const crs_route_params *p, const void *Q, const vo
         route_attn_kernel<<<dim3(p->C, BH), max(32, ceil_div(a.mm, 32) * 32), rt_attn_smem(a.mm), s>>>(a);
     }
     route_merge_kernel<<<(unsigned)ceil_div((long long)BH * p->n, 8), 256, 0, s>>>(a);
+    _ps.more(3);                                  // score, quota, attention, merge
     CRS_CHECK_LAUNCH();
     return CRS_OK;
 }
