@@ -25,9 +25,10 @@
 //   lsd_append_kernel      one warp per (row, head, round): tokens in position
 //                          order, lanes grouped by bucket (match_any), one
 //                          length update and page allocation per group
-//   lsd_attend_kernel      one CTA per (row, head): each lane takes a candidate
-//                          (online softmax in registers), lanes and warps merged
-//                          in shared memory
+//   lsd_attend_kernel      one CTA per (row, head): the lists' kept entries are
+//                          compacted into shared memory, then 8-lane groups
+//                          score and accumulate them (online softmax), groups
+//                          merged in order
 //   lsd_advance_kernel     seq_len += tokens appended
 #include "common.cuh"
 
@@ -35,7 +36,6 @@ namespace crs {
 
 constexpr int kLdD = 64;                  // head dim
 constexpr int kLdMaxRounds = 8;
-constexpr int kLdAttWarps = 4;
 
 struct LdState {
     __nv_bfloat16 *K, *V;
@@ -72,11 +72,22 @@ __global__ void __launch_bounds__(256) lsd_hash_kernel(LdArgs a) {
     const float *R = a.rot + ((size_t)h * a.R + r) * kLdD * half;
     float best = -INFINITY;
     int bi = 0x7fffffff;
-    for (int k = lane; k < half; k += 32) {
+    // the row in registers (two values per lane, broadcast by shuffles); the chain
+    // itself stays one FMA per term in index order
+    const float2 xl = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162 *>(x)[lane]);
+    for (int k0 = 0; k0 < half; k0 += 32) {             // same trip count in every lane
+        const int k = k0 + lane;
+        const bool kv = k < half;
         float u = 0.0f;
-        for (int i = 0; i < kLdD; ++i) u = fmaf(__bfloat162float(x[i]), R[(size_t)i * half + k], u);
-        if (u > best || (u == best && k < bi)) { best = u; bi = k; }
-        if (-u > best || (-u == best && k + half < bi)) { best = -u; bi = k + half; }
+#pragma unroll
+        for (int i = 0; i < kLdD; ++i) {
+            const float xi = __shfl_sync(0xffffffffu, (i & 1) ? xl.y : xl.x, i >> 1);
+            u = fmaf(xi, kv ? __ldg(R + (size_t)i * half + k) : 0.0f, u);
+        }
+        if (kv) {
+            if (u > best || (u == best && k < bi)) { best = u; bi = k; }
+            if (-u > best || (-u == best && k + half < bi)) { best = -u; bi = k + half; }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -163,19 +174,89 @@ __global__ void __launch_bounds__(256) lsd_append_kernel(LdArgs a) {
 }
 
 // One CTA per (row, head): the newest token t attends to its buckets' lists.
-// Candidates are taken round by round; entry j of round r is skipped when j == t
-// (no_self) or when j shares an earlier round's bucket with t (already met).
-// Lane = candidate: dot with q (registers), online softmax and a 64-wide value
-// accumulator per lane; lanes then warps are merged through shared memory.
-__global__ void __launch_bounds__(kLdAttWarps * 32) lsd_attend_kernel(LdArgs a) {
-    __shared__ float sq[kLdD];
-    __shared__ float sm[kLdAttWarps * 32], sl[kLdAttWarps * 32];
-    __shared__ float so[kLdAttWarps][kLdD];
-    __shared__ int scnt[kLdAttWarps];
+// Candidates are taken round by round; entry j of round r is skipped when j > t,
+// when j == t (no_self) or when j shares an earlier round's bucket with t
+// (already met).
+//   1. the 256 threads walk the rounds' lists as one sequence (round by round,
+//      entries in order), two entries each per pass (list page -> entry ->
+//      earlier buckets and block table), and the kept
+//      candidates' K/V row indices are compacted into shared memory in that order
+//      (warp ballots, warp offsets), up to kLdCap at a time;
+//   2. 32 groups of 8 lanes take the candidates in turn: lane g of a group loads
+//      16 bytes (columns [8g, 8g + 8)) of the K and the V row, three shuffles
+//      give the score, and the group keeps an online softmax (m, l, 8 outputs);
+//   3. the 32 group states are merged in group order.
+constexpr int kLdAttThreads = 256;
+constexpr int kLdCap = 2048;               // candidate rows held in shared memory
+constexpr int kLdGroups = kLdAttThreads / 8;
+
+struct LdGroup {
+    float m, l, acc[8];
+    int cnt;
+};
+
+// Scores and accumulates the candidates c = G, G + 32, ... < nc of the buffer,
+// four per pass (their K and V loads in flight together), in that order.  The
+// loop runs the same number of times in every lane (the score shuffles need the
+// whole warp); a group past the end loads nothing and keeps its state.
+constexpr int kLdUnroll = 4;
+
+__device__ __forceinline__ void lsd_consume(const LdArgs &a, const uint32_t *crow, int nc, int G, int g,
+                                            const float (&qv)[8], LdGroup &st) {
+    for (int c0 = 0; c0 < nc; c0 += kLdUnroll * kLdGroups) {
+        uint4 kraw[kLdUnroll], vraw[kLdUnroll];
+        bool valid[kLdUnroll];
+#pragma unroll
+        for (int u = 0; u < kLdUnroll; ++u) {
+            const int c = c0 + u * kLdGroups + G;
+            valid[u] = c < nc;
+            kraw[u] = vraw[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (valid[u]) {
+                const size_t row = (size_t)crow[c] * kLdD + 8 * g;
+                kraw[u] = __ldg(reinterpret_cast<const uint4 *>(a.st.K + row));
+                vraw[u] = __ldg(reinterpret_cast<const uint4 *>(a.st.V + row));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kLdUnroll; ++u) {
+            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kraw[u]);
+            float dot = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 kv = __bfloat1622float2(k2[e]);
+                dot = fmaf(qv[2 * e], kv.x, fmaf(qv[2 * e + 1], kv.y, dot));
+            }
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+            if (valid[u]) {
+                const float mn = fmaxf(st.m, dot);
+                const float corr = __expf(st.m - mn), p = __expf(dot - mn);
+                st.l = st.l * corr + p;
+                const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vraw[u]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 vv = __bfloat1622float2(v2[e]);
+                    st.acc[2 * e] = fmaf(p, vv.x, st.acc[2 * e] * corr);
+                    st.acc[2 * e + 1] = fmaf(p, vv.y, st.acc[2 * e + 1] * corr);
+                }
+                st.m = mn;
+                ++st.cnt;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kLdAttThreads, 4) lsd_attend_kernel(LdArgs a) {
+    __shared__ uint32_t crow[kLdCap];
+    __shared__ int wcount[kLdAttThreads / 32];
+    __shared__ float gm[kLdGroups], gl[kLdGroups];
+    __shared__ int gc[kLdGroups];
+    __shared__ float go[kLdGroups][kLdD];
     const int sh = blockIdx.x, s = sh / a.H, h = sh - s * a.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = tid >> 3, g = tid & 7;
     const int t = a.st.seq_len[s];                           // the newest token
-    const int nt = kLdAttWarps * 32;
     if (t >= a.max_len) {                                    // no room: flagged by the append
         if (tid < kLdD) a.O[((size_t)s * a.H + h) * kLdD + tid] = 0.0f;
         if (tid == 0) {
@@ -184,86 +265,115 @@ __global__ void __launch_bounds__(kLdAttWarps * 32) lsd_attend_kernel(LdArgs a) 
         }
         return;
     }
-    const size_t q_off = ((size_t)s * a.n_new * a.H + h) * kLdD;   // token 0 of the step
-    if (tid < kLdD) sq[tid] = a.scale * __bfloat162float(a.X[q_off + tid]);
-    __syncthreads();
+    float qv[8];
+    {
+        const size_t q_off = ((size_t)s * a.n_new * a.H + h) * kLdD + 8 * g;   // token 0 of the step
+        const uint4 raw = *reinterpret_cast<const uint4 *>(a.X + q_off);
+        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float2 f = __bfloat1622float2(p2[u]);
+            qv[2 * u] = a.scale * f.x;
+            qv[2 * u + 1] = a.scale * f.y;
+        }
+    }
     uint8_t tb[kLdMaxRounds];
     const uint8_t *bk = a.st.bucket + ((size_t)s * a.H + h) * a.R * a.max_len;
 #pragma unroll
     for (int r = 0; r < kLdMaxRounds; ++r) tb[r] = r < a.R ? bk[(size_t)r * a.max_len + t] : 0;
-    float m = -INFINITY, l = 0.0f, o[kLdD];
+    LdGroup st;
+    st.m = -INFINITY;
+    st.l = 0.0f;
+    st.cnt = 0;
 #pragma unroll
-    for (int c = 0; c < kLdD; ++c) o[c] = 0.0f;
-    int cnt = 0;
-    for (int r = 0; r < a.R; ++r) {
-        const size_t lid = ld_list_id(a, s, h, r, tb[r]);
-        const int len = min(a.st.list_len[lid], a.list_pages * a.Lp);
-        for (int e = tid; e < len; e += nt) {
-            const int pg = a.st.list_table[lid * a.list_pages + e / a.Lp];
-            if (pg < 0) continue;
-            const int j = a.st.list_pool[(size_t)pg * a.Lp + e % a.Lp];
-            if (j > t || (a.no_self && j == t)) continue;
-            bool met = false;
-            for (int r2 = 0; r2 < r; ++r2) met |= bk[(size_t)r2 * a.max_len + j] == tb[r2];
-            if (met) continue;
-            const int page = a.st.block_table[(size_t)s * a.max_pages + j / a.P];
-            const size_t row = (((size_t)page * a.P + j % a.P) * a.H + h) * kLdD;
-            const uint4 *kr = reinterpret_cast<const uint4 *>(a.st.K + row);
-            float dot = 0.0f;
+    for (int c = 0; c < 8; ++c) st.acc[c] = 0.0f;
+    // the rounds' entries as one sequence, round by round (cum = start of each round)
+    int cum[kLdMaxRounds + 1];
+    cum[0] = 0;
 #pragma unroll
-            for (int c = 0; c < kLdD / 8; ++c) {
-                const uint4 raw = __ldg(kr + c);
-                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    for (int r = 0; r < kLdMaxRounds; ++r)
+        cum[r + 1] = cum[r] + (r < a.R ? min(a.st.list_len[ld_list_id(a, s, h, r, tb[r])], a.list_pages * a.Lp) : 0);
+    const int total_entries = cum[kLdMaxRounds];
+    int nc = 0;                                              // candidates buffered (CTA-uniform)
+    for (int base = 0; base < total_entries; base += 2 * kLdAttThreads) {
+        bool keep[2];
+        uint32_t row[2];
+        int pg[2], j[2], rr[2], e[2];
+        size_t lid[2];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 kv = __bfloat1622float2(p2[u]);
-                    dot = fmaf(sq[c * 8 + 2 * u], kv.x, fmaf(sq[c * 8 + 2 * u + 1], kv.y, dot));
-                }
+        for (int u = 0; u < 2; ++u) {
+            const int f = base + u * kLdAttThreads + tid;
+            int r = 0;
+#pragma unroll
+            for (int q = 1; q < kLdMaxRounds; ++q) r += (q < a.R && f >= cum[q]) ? 1 : 0;
+            rr[u] = r;
+            e[u] = f - cum[r];
+            lid[u] = ld_list_id(a, s, h, r, tb[r]);
+            pg[u] = f < total_entries ? a.st.list_table[lid[u] * a.list_pages + e[u] / a.Lp] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) j[u] = pg[u] >= 0 ? a.st.list_pool[(size_t)pg[u] * a.Lp + e[u] % a.Lp] : -1;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            keep[u] = j[u] >= 0 && j[u] <= t && !(a.no_self && j[u] == t);
+            row[u] = 0u;
+            if (keep[u] && j[u] / a.P >= a.max_pages) {         // no page-table slot for it
+                raise_error(CRS_DEVERR_INDEX);
+                keep[u] = false;
             }
-            const float mn = fmaxf(m, dot);
-            const float corr = __expf(m - mn), p = __expf(dot - mn);
-            l = l * corr + p;
-            const uint4 *vr = reinterpret_cast<const uint4 *>(a.st.V + row);
-#pragma unroll
-            for (int c = 0; c < kLdD / 8; ++c) {
-                const uint4 raw = __ldg(vr + c);
-                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 vv = __bfloat1622float2(p2[u]);
-                    o[c * 8 + 2 * u] = fmaf(p, vv.x, o[c * 8 + 2 * u] * corr);
-                    o[c * 8 + 2 * u + 1] = fmaf(p, vv.y, o[c * 8 + 2 * u + 1] * corr);
-                }
+            if (keep[u]) {
+                bool met = false;
+                for (int r2 = 0; r2 < rr[u]; ++r2) met |= bk[(size_t)r2 * a.max_len + j[u]] == tb[r2];
+                const int page = a.st.block_table[(size_t)s * a.max_pages + j[u] / a.P];
+                keep[u] = !met;
+                row[u] = (uint32_t)(((size_t)page * a.P + j[u] % a.P) * a.H + h);
             }
-            m = mn;
-            ++cnt;
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            // compact in entry order: warp ballot, then the earlier warps' counts
+            const uint32_t bal = __ballot_sync(0xffffffffu, keep[u]);
+            if (lane == 0) wcount[warp] = __popc(bal);
+            __syncthreads();
+            int off = nc, total = 0;
+#pragma unroll
+            for (int w = 0; w < kLdAttThreads / 32; ++w) {
+                const int cw = wcount[w];
+                if (w < warp) off += cw;
+                total += cw;
+            }
+            if (keep[u]) crow[off + __popc(bal & ((1u << lane) - 1u))] = row[u];
+            nc += total;
+            __syncthreads();
+            if (nc > kLdCap - kLdAttThreads) {               // room for one more pass of 256
+                lsd_consume(a, crow, nc, G, g, qv, st);
+                nc = 0;
+                __syncthreads();
+            }
         }
     }
-    // merge: the CTA maximum, then each lane's rescaled (l, o) summed per warp, then per CTA
-    sm[tid] = m;
-    __syncthreads();
-    float M = -INFINITY;
-    for (int i = 0; i < nt; ++i) M = fmaxf(M, sm[i]);
-    const float f = m == -INFINITY ? 0.0f : __expf(m - M);
-    float lw = warp_sum(l * f);
-    const int cw = warp_sum_int(cnt);
+    lsd_consume(a, crow, nc, G, g, qv, st);
+    // merge the 32 group states in group order
+    if (g == 0) {
+        gm[G] = st.m;
+        gl[G] = st.l;
+        gc[G] = st.cnt;
+    }
 #pragma unroll
-    for (int c = 0; c < kLdD; ++c) {
-        const float v = warp_sum(o[c] * f);
-        if (lane == 0) so[warp][c] = v;
-    }
-    if (lane == 0) {
-        sl[warp] = lw;
-        scnt[warp] = cw;
-    }
+    for (int c = 0; c < 8; ++c) go[G][8 * g + c] = st.acc[c];
     __syncthreads();
     if (tid < kLdD) {
-        float L = 0.0f, acc = 0.0f;
+        float M = -INFINITY;
         int C = 0;
-        for (int w = 0; w < kLdAttWarps; ++w) {
-            L += sl[w];
-            acc += so[w][tid];
-            C += scnt[w];
+        for (int w = 0; w < kLdGroups; ++w) {
+            M = fmaxf(M, gm[w]);
+            C += gc[w];
+        }
+        float L = 0.0f, acc = 0.0f;
+        for (int w = 0; w < kLdGroups; ++w) {
+            const float f = gc[w] > 0 ? __expf(gm[w] - M) : 0.0f;
+            L += gl[w] * f;
+            acc += go[w][tid] * f;
         }
         a.O[((size_t)s * a.H + h) * kLdD + tid] = C > 0 ? acc / L : 0.0f;
         if (tid == 0) {
@@ -336,7 +446,7 @@ static int ld_run(const crs_lsh_decode_params *p, const crs_lsh_decode_state *st
     lsd_hash_kernel<<<dim3(p->n_seq * p->n_heads, ceil_div(n_new * p->n_rounds, 8)), 256, 0, s>>>(a);
     lsd_store_kv_kernel<<<dim3(ceil_div(n_new * p->n_heads, 8), p->n_seq), 256, 0, s>>>(a);
     lsd_append_kernel<<<ceil_div(p->n_seq * p->n_heads * p->n_rounds, 8), 256, 0, s>>>(a);
-    if (O) lsd_attend_kernel<<<p->n_seq * p->n_heads, kLdAttWarps * 32, 0, s>>>(a);
+    if (O) lsd_attend_kernel<<<p->n_seq * p->n_heads, kLdAttThreads, 0, s>>>(a);
     lsd_advance_kernel<<<ceil_div(p->n_seq, 128), 128, 0, s>>>(st->seq_len, p->n_seq, n_new, p->max_len);
     _ps.more(O ? 4 : 3);                          // hash, store, append, (attend,) advance
     CRS_CHECK_LAUNCH();

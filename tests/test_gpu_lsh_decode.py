@@ -78,3 +78,18 @@ def test_full_list_flags_capacity_and_keeps_running(crs, cuda_dev):
     torch.cuda.synchronize()
     assert crs.get_device_error() & 0x8
     assert torch.isfinite(O).all() and (cnt.cpu().numpy() <= 8).all()
+
+
+def test_many_candidates_per_row(crs, cuda_dev):
+    """Two buckets, two rounds, 3000-token rows: about 2250 candidates per (row, head),
+    more than the attend kernel buffers at once, so it scores them in several batches."""
+    S, n, H, d, b, R = 2, 3000, 2, 64, 2, 2
+    x, v, rot = _inputs(S, n + 1, H, d, b, R, seed=54, dev=cuda_dev)
+    cache = crs.LshDecodeCache(S, H, b, R, max_len=n + 64, device=cuda_dev)
+    cache.prefill(x[:, :n].contiguous(), v[:, :n].contiguous(), rot)
+    O, lse, cnt = cache.step(x[:, n:].contiguous(), v[:, n:].contiguous(), rot)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    o_O, o_lse, o_cnt = _oracle(x, v, rot, b, np.full(S, n + 1), True)
+    assert o_cnt.min() > 2048
+    _compare(O, lse, cnt, o_O, o_lse, o_cnt)
