@@ -15,7 +15,8 @@
 //                            listed ascending
 //   hisa_fine_kernel         r_s = sum_h w_h ReLU(q_h . k_s) for every key of
 //                            the kept blocks and of the open block, in
-//                            candidate order (= ascending position)
+//                            candidate order (= ascending position); a CTA
+//                            takes 256 / b blocks
 //   hisa_pick_tokens_kernel  the topk candidates by (r desc, position asc),
 //                            ascending, -1 padded
 // The two selections are exact; one 1024-thread CTA per row builds the k-th
@@ -194,56 +195,68 @@ __global__ void __launch_bounds__(kPickT) hisa_pick_blocks_kernel(HisaArgs a) {
     if (tid == 0) a.n_keep[row] = n_sel;
 }
 
-// grid (top_blocks + 1, rows): unit u < n_keep scores the keys of kept block
-// u, unit top_blocks the open block; thread = key.
-__global__ void __launch_bounds__(256) hisa_fine_kernel(HisaArgs a) {
+// grid (ceil((top_blocks + 1) / UP), rows), 256 threads: CTA x takes the UP =
+// max(1, 256 / blk) units [x UP, x UP + UP); unit u < n_keep scores the keys
+// of kept block u, unit top_blocks the open block; one key per thread and pass.
+constexpr int kHFineThreads = 256;
+
+__host__ __device__ inline int hisa_fine_units(int blk) { return blk >= kHFineThreads ? 1 : kHFineThreads / blk; }
+
+__global__ void __launch_bounds__(kHFineThreads) hisa_fine_kernel(HisaArgs a) {
     __shared__ float sq[kHMaxHeads][kHd];
     __shared__ float sw[kHMaxHeads];
-    const int row = blockIdx.y, u = blockIdx.x, t = threadIdx.x;
+    const int row = blockIdx.y, t = threadIdx.x;
     const int64_t k0 = a.k_off[row];
     if (a.k_off[row + 1] - k0 > a.max_keys) return;
     const int ctx = (int)(a.k_off[row + 1] - k0);
     const int nb = ctx / a.blk;
     const int nkeep = a.n_keep[row];
-    int pos0, len, slot0;
-    if (u < a.top_blocks) {
-        if (u >= nkeep) return;                              // CTA-uniform
-        pos0 = a.blocks[(size_t)row * a.top_blocks + u] * a.blk;
-        len = a.blk;
-        slot0 = u * a.blk;
-    } else {
-        pos0 = nb * a.blk;
-        len = ctx - pos0;
-        slot0 = nkeep * a.blk;
-        if (len <= 0) return;
-    }
-    for (int e = t; e < a.H * kHd; e += blockDim.x)
+    const int UP = hisa_fine_units(a.blk);
+    const int u_first = blockIdx.x * UP;
+    if (u_first >= nkeep && u_first + UP <= a.top_blocks) return;   // CTA-uniform: nothing kept here
+    for (int e = t; e < a.H * kHd; e += kHFineThreads)
         sq[e / kHd][e % kHd] = __bfloat162float(a.q[(size_t)row * a.H * kHd + e]);
     if (t < a.H) sw[t] = a.w[(size_t)row * a.H + t];
     __syncthreads();
-    if (t >= len) return;
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.k + (k0 + pos0 + t) * kHd);
-    float dot[kHMaxHeads];
-#pragma unroll
-    for (int h = 0; h < kHMaxHeads; ++h) dot[h] = 0.0f;
-#pragma unroll
-    for (int c = 0; c < kHd / 8; ++c) {
-        const uint4 raw = __ldg(src + c);
-        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 kv = __bfloat1622float2(p2[e]);
-            const int d = c * 8 + 2 * e;
-#pragma unroll
-            for (int h = 0; h < kHMaxHeads; ++h)
-                if (h < a.H) dot[h] = fmaf(sq[h][d], kv.x, fmaf(sq[h][d + 1], kv.y, dot[h]));
+    for (int e = t; e < UP * a.blk; e += kHFineThreads) {
+        const int u = u_first + e / a.blk, i = e % a.blk;
+        int pos0, len, slot0;
+        if (u < a.top_blocks) {
+            if (u >= nkeep) continue;
+            pos0 = a.blocks[(size_t)row * a.top_blocks + u] * a.blk;
+            len = a.blk;
+            slot0 = u * a.blk;
+        } else if (u == a.top_blocks) {
+            pos0 = nb * a.blk;
+            len = ctx - pos0;
+            slot0 = nkeep * a.blk;
+        } else {
+            continue;
         }
-    }
-    float r = 0.0f;
+        if (i >= len) continue;
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.k + (k0 + pos0 + i) * kHd);
+        float dot[kHMaxHeads];
 #pragma unroll
-    for (int h = 0; h < kHMaxHeads; ++h)
-        if (h < a.H) r += sw[h] * (dot[h] != dot[h] ? dot[h] : fmaxf(dot[h], 0.0f));
-    a.fine[(size_t)row * a.cand_cap + slot0 + t] = r;
+        for (int h = 0; h < kHMaxHeads; ++h) dot[h] = 0.0f;
+#pragma unroll
+        for (int c = 0; c < kHd / 8; ++c) {
+            const uint4 raw = __ldg(src + c);
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 kv = __bfloat1622float2(p2[q]);
+                const int d = c * 8 + 2 * q;
+#pragma unroll
+                for (int h = 0; h < kHMaxHeads; ++h)
+                    if (h < a.H) dot[h] = fmaf(sq[h][d], kv.x, fmaf(sq[h][d + 1], kv.y, dot[h]));
+            }
+        }
+        float r = 0.0f;
+#pragma unroll
+        for (int h = 0; h < kHMaxHeads; ++h)
+            if (h < a.H) r += sw[h] * (dot[h] != dot[h] ? dot[h] : fmaxf(dot[h], 0.0f));
+        a.fine[(size_t)row * a.cand_cap + slot0 + i] = r;
+    }
 }
 
 // one CTA per row: the topk candidates (slot order = ascending position)
@@ -413,7 +426,7 @@ extern "C" int crs_hisa_topk(const crs_hisa_params *p, const void *q_idx, const 
     case 4: hisa_pick_blocks_kernel<4><<<p->n_rows, kPickT, 0, s>>>(a); break;
     default: hisa_pick_blocks_kernel<8><<<p->n_rows, kPickT, 0, s>>>(a); break;
     }
-    hisa_fine_kernel<<<dim3(p->top_blocks + 1, p->n_rows), max(32, ceil_div(p->blk, 32) * 32), 0, s>>>(a);
+    hisa_fine_kernel<<<dim3(ceil_div(p->top_blocks + 1, hisa_fine_units(p->blk)), p->n_rows), kHFineThreads, 0, s>>>(a);
     switch (hisa_kpt(a.cand_cap)) {
     case 1: hisa_pick_tokens_kernel<1><<<p->n_rows, kPickT, 0, s>>>(a); break;
     case 2: hisa_pick_tokens_kernel<2><<<p->n_rows, kPickT, 0, s>>>(a); break;
