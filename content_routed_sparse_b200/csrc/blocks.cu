@@ -549,15 +549,13 @@ block_pick_kernel(const float *__restrict__ sc, int32_t *__restrict__ tok, int32
             key[u] = score_key(acc);
         }
     }
+    int ph = 0;
     auto count_ge = [&](uint32_t c) -> int {
         int local = 0;
 #pragma unroll
         for (int u = 0; u < KPT; ++u) local += (valid[u] && key[u] >= c) ? 1 : 0;
-        if (KPT == 1) return __syncthreads_count(local);
-        int total = 0;
-#pragma unroll
-        for (int bit = 0; (1 << bit) <= KPT; ++bit) total += __syncthreads_count(local & (1 << bit)) << bit;
-        return total;
+        if (KPT == 1) return __syncthreads_count(local);       // one barrier already
+        return cta_count(local, ph);
     };
     // exact top k by (key desc, block asc): Tk = the largest key with >= k keys at or above it
     const int k = min(top, n_full);

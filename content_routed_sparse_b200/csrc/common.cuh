@@ -118,6 +118,22 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
 }
+// CTA-wide sum of one count per thread (blockDim.x a multiple of 32): warp sums
+// go to one of two shared arrays and a single barrier publishes them.  Every
+// thread makes the same sequence of calls with its own parity ph (flipped
+// here), so an array is rewritten only after all threads passed the barrier of
+// the call that followed its last reading.
+__device__ __forceinline__ int cta_count(int local, int &ph) {
+    __shared__ int cbuf[2][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ws = __reduce_add_sync(0xffffffffu, local);
+    if (lane == 0) cbuf[ph][warp] = ws;
+    __syncthreads();
+    const int v = lane < (int)(blockDim.x >> 5) ? cbuf[ph][lane] : 0;
+    ph ^= 1;
+    return __reduce_add_sync(0xffffffffu, v);
+}
+
 __device__ __forceinline__ void cp_async16_zfill(void *smem, const void *gmem, bool valid) {
     int src_size = valid ? 16 : 0;
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),

@@ -121,15 +121,13 @@ __global__ void __launch_bounds__(kHCoarseWarps * 32) hisa_coarse_kernel(HisaArg
 template <int KPT>
 __device__ __forceinline__ void cta_topk(const uint32_t (&key)[KPT], const bool (&valid)[KPT], int k,
                                          bool (&take)[KPT], int &slot, int &n_sel, int2 *wtot) {
+    int ph = 0;
     auto count_ge = [&](uint32_t c) -> int {
         int local = 0;
 #pragma unroll
         for (int u = 0; u < KPT; ++u) local += (valid[u] && key[u] >= c) ? 1 : 0;
-        if (KPT == 1) return __syncthreads_count(local);
-        int total = 0;
-#pragma unroll
-        for (int bit = 0; (1 << bit) <= KPT; ++bit) total += __syncthreads_count(local & (1 << bit)) << bit;
-        return total;
+        if (KPT == 1) return __syncthreads_count(local);       // one barrier already
+        return cta_count(local, ph);
     };
     uint32_t Tk = 0u;
     for (int bit = 31; bit >= 0; --bit) {
