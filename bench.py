@@ -765,6 +765,20 @@ def _omp_threads():
 
 
 # --------------------------------------------------------------------- main --
+def reduce_max_over_ranks(values, device):
+    """Each entry's maximum over the ranks of the default process group: the job
+    takes as long as its slowest rank."""
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_throughput(units_per_step, steps, world, total_ms):
+    """Whole-job units per second: every rank processes its own batch (weak
+    scaling), timed as the slowest rank's total."""
+    return units_per_step * steps * world / (total_ms / 1e3)
+
+
 def run_reference(args, rank):
     """Oracle arm: the CPU oracle on the host cores, bounded sample per step."""
     if rank != 0:
@@ -833,12 +847,9 @@ def main():
     tot_ms = sum(res["times_ms"])
     e2e_ms = sum(res["e2e_times_ms"])
     if dist_on:
-        t = torch.tensor([tot_ms, e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        tot_ms, e2e_ms = float(t[0]), float(t[1])
-    units = wl.units_per_step * args.steps * world
-    value = units / (tot_ms / 1e3)
-    e2e_value = units / (e2e_ms / 1e3)
+        tot_ms, e2e_ms = reduce_max_over_ranks([tot_ms, e2e_ms], dev)
+    value = job_throughput(wl.units_per_step, args.steps, world, tot_ms)
+    e2e_value = job_throughput(wl.units_per_step, args.steps, world, e2e_ms)
 
     extras = {}
     if not args.no_extras and not dist_on:
