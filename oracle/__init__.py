@@ -11,7 +11,7 @@ Parity status per function (pins in ``tests/test_oracle_*.py``):
   block_describe / block_log_mass / block_select   -- pinned (rank 0 = mean-pool selector)
   quest_describe / quest_select                    -- pinned
   block_describe_ss / block_select_ss              -- pinned
-  hisa_describe / hisa_topk                        -- pinned
+  hisa_describe / hisa_topk / hisa_topk_prefill    -- pinned
   lsh_decode                                       -- pinned
   kmeans_route                                     -- pinned
   fp4_quantize / fp4_dequantize                    -- pinned
@@ -71,6 +71,7 @@ def _lib():
         lib.oracle_hisa_topk.argtypes = [I, I, I, I, I, I, _f64p, _f64p, _f64p, _i64p, _f64p, _i64p, _i32p,
                                          _i32p, _i32p, _i32p, _f64p]
         lib.oracle_quest_describe.argtypes = [I, I, I, I, I, _f64p, _f64p, _f64p]
+        lib.oracle_hisa_topk_prefill.argtypes = [I, I, I, I, I, I, _f64p, _f64p, _f64p, _f64p, _i32p, _i32p, _i32p]
         lib.oracle_quest_select.argtypes = [I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p, I,
                                             _i32p, _i32p, _i32p, _f64p]
         lib.oracle_sparse_attn.argtypes = [I, I, I, I, D, _f64p, _f64p, _f64p, _i64p, _i32p, I, I,
@@ -291,6 +292,26 @@ def hisa_topk(q, w, K, k_offsets, rep, blk_offsets, topk, blk, top_blocks, given
                             _p(ko, _i64p), _p(rep, _f64p), _p(bo, _i64p), None if gb is None else _p(gb, _i32p),
                             _p(blocks, _i32p), _p(idx, _i32p), _p(cnt, _i32p), _p(coarse, _f64p))
     return blocks, idx, cnt, coarse[: rep.shape[0]]
+
+
+def hisa_topk_prefill(q, w, K, rep, topk, blk, top_blocks):
+    """Hierarchical top-k for the n causal queries of one sequence: query i sees keys
+    0..i, its complete blocks are j < (i + 1) // blk (rep [n // blk, d] from
+    hisa_describe(K, [0, n], blk)).  Returns (blocks [n, top_blocks], idx [n, topk],
+    count [n]), ascending and -1 padded."""
+    q = _c(q, np.float64)
+    w = _c(w, np.float64)
+    K = _c(K, np.float64)
+    rep = _c(rep, np.float64)
+    n, heads, d = q.shape
+    if rep.shape[0] == 0:
+        rep = np.zeros((1, d), dtype=np.float64)
+    blocks = np.empty((n, top_blocks), dtype=np.int32)
+    idx = np.empty((n, topk), dtype=np.int32)
+    cnt = np.empty(n, dtype=np.int32)
+    _lib().oracle_hisa_topk_prefill(n, heads, d, topk, blk, top_blocks, _p(q, _f64p), _p(w, _f64p), _p(K, _f64p),
+                                    _p(rep, _f64p), _p(blocks, _i32p), _p(idx, _i32p), _p(cnt, _i32p))
+    return blocks, idx, cnt
 
 
 # -------------------------------------------------------------- blocks --

@@ -548,6 +548,67 @@ OAPI void oracle_hisa_describe(int n_rows, int d, int blk, const double *K, cons
     }
 }
 
+/* One row: query qt / weights wt, its keys Kr[0 .. ctx), the representatives
+ * rep_r of its ctx / blk complete blocks; given (or NULL) replaces the coarse
+ * selection; coarse_r (or NULL) receives the coarse scores. */
+static void hisa_row(int n_heads, int d, int topk, int blk, int top_blocks, const double *qt,
+                     const double *wt, const double *Kr, long ctx, const double *rep_r,
+                     const int32_t *given, int32_t *ob, int32_t *o, int32_t *count, double *coarse_r)
+{
+    const int nb = (int)(ctx / blk);
+    int nkeep = 0;
+    if (given) {
+        for (int c = 0; c < top_blocks; ++c)
+            if (given[c] >= 0)
+                ob[nkeep++] = given[c];
+    } else {
+        scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(nb > 0 ? nb : 1));
+        double *cs = (double *)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
+        oracle_indexer_score(n_heads, d, qt, wt, rep_r, nb, cs);
+        for (int j = 0; j < nb; ++j) {
+            sc[j].s = cs[j];
+            sc[j].i = j;
+            if (coarse_r) coarse_r[j] = cs[j];
+        }
+        qsort(sc, (size_t)nb, sizeof(scored_t), cmp_score_desc_idx_asc);
+        nkeep = nb < top_blocks ? nb : top_blocks;
+        for (int c = 0; c < nkeep; ++c)
+            ob[c] = sc[c].i;
+        free(sc);
+        free(cs);
+    }
+    qsort(ob, (size_t)nkeep, sizeof(int32_t), cmp_i32);
+    for (int c = nkeep; c < top_blocks; ++c)
+        ob[c] = -1;
+    /* candidates: the kept blocks' keys, then the open block's */
+    const long open0 = (long)nb * blk;
+    const long ncand = (long)nkeep * blk + (ctx - open0);
+    scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(ncand > 0 ? ncand : 1));
+    double one;
+    long c = 0;
+    for (int b = 0; b < nkeep; ++b)
+        for (int i = 0; i < blk; ++i, ++c) {
+            const long pos = (long)ob[b] * blk + i;
+            oracle_indexer_score(n_heads, d, qt, wt, Kr + pos * d, 1, &one);
+            sc[c].s = one;
+            sc[c].i = (int32_t)pos;
+        }
+    for (long pos = open0; pos < ctx; ++pos, ++c) {
+        oracle_indexer_score(n_heads, d, qt, wt, Kr + pos * d, 1, &one);
+        sc[c].s = one;
+        sc[c].i = (int32_t)pos;
+    }
+    qsort(sc, (size_t)ncand, sizeof(scored_t), cmp_score_desc_idx_asc);
+    const int kk = ncand < topk ? (int)ncand : topk;
+    for (int i = 0; i < kk; ++i)
+        o[i] = sc[i].i;
+    qsort(o, (size_t)kk, sizeof(int32_t), cmp_i32);
+    for (int i = kk; i < topk; ++i)
+        o[i] = -1;
+    *count = kk;
+    free(sc);
+}
+
 OAPI void oracle_hisa_topk(int n_rows, int n_heads, int d, int topk, int blk, int top_blocks,
                            const double *q, const double *w, const double *K, const int64_t *k_offsets,
                            const double *rep, const int64_t *blk_offsets, const int32_t *given_blocks,
@@ -555,64 +616,29 @@ OAPI void oracle_hisa_topk(int n_rows, int n_heads, int d, int topk, int blk, in
                            double *coarse_score)
 {
 #pragma omp parallel for schedule(dynamic, 1)
-    for (long t = 0; t < n_rows; ++t) {
-        const long ctx = (long)(k_offsets[t + 1] - k_offsets[t]);
-        const int nb = (int)(ctx / blk);
-        const double *qt = q + t * (long)n_heads * d, *wt = w + t * (long)n_heads;
-        int32_t *ob = out_blocks + t * (long)top_blocks;
-        int nkeep = 0;
-        if (given_blocks) {
-            for (int c = 0; c < top_blocks; ++c)
-                if (given_blocks[t * (long)top_blocks + c] >= 0)
-                    ob[nkeep++] = given_blocks[t * (long)top_blocks + c];
-        } else {
-            scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(nb > 0 ? nb : 1));
-            double *cs = (double *)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
-            oracle_indexer_score(n_heads, d, qt, wt, rep + blk_offsets[t] * (long)d, nb, cs);
-            for (int j = 0; j < nb; ++j) {
-                sc[j].s = cs[j];
-                sc[j].i = j;
-                if (coarse_score) coarse_score[blk_offsets[t] + j] = cs[j];
-            }
-            qsort(sc, (size_t)nb, sizeof(scored_t), cmp_score_desc_idx_asc);
-            nkeep = nb < top_blocks ? nb : top_blocks;
-            for (int c = 0; c < nkeep; ++c)
-                ob[c] = sc[c].i;
-            free(sc);
-            free(cs);
-        }
-        qsort(ob, (size_t)nkeep, sizeof(int32_t), cmp_i32);
-        for (int c = nkeep; c < top_blocks; ++c)
-            ob[c] = -1;
-        /* candidates: the kept blocks' keys, then the open block's */
-        const long open0 = (long)nb * blk;
-        const long ncand = (long)nkeep * blk + (ctx - open0);
-        scored_t *sc = (scored_t *)malloc(sizeof(scored_t) * (size_t)(ncand > 0 ? ncand : 1));
-        double one;
-        long c = 0;
-        for (int b = 0; b < nkeep; ++b)
-            for (int i = 0; i < blk; ++i, ++c) {
-                const long pos = (long)ob[b] * blk + i;
-                oracle_indexer_score(n_heads, d, qt, wt, K + (k_offsets[t] + pos) * d, 1, &one);
-                sc[c].s = one;
-                sc[c].i = (int32_t)pos;
-            }
-        for (long pos = open0; pos < ctx; ++pos, ++c) {
-            oracle_indexer_score(n_heads, d, qt, wt, K + (k_offsets[t] + pos) * d, 1, &one);
-            sc[c].s = one;
-            sc[c].i = (int32_t)pos;
-        }
-        qsort(sc, (size_t)ncand, sizeof(scored_t), cmp_score_desc_idx_asc);
-        const int kk = ncand < topk ? (int)ncand : topk;
-        int32_t *o = out_idx + t * (long)topk;
-        for (int i = 0; i < kk; ++i)
-            o[i] = sc[i].i;
-        qsort(o, (size_t)kk, sizeof(int32_t), cmp_i32);
-        for (int i = kk; i < topk; ++i)
-            o[i] = -1;
-        out_count[t] = kk;
-        free(sc);
-    }
+    for (long t = 0; t < n_rows; ++t)
+        hisa_row(n_heads, d, topk, blk, top_blocks, q + t * (long)n_heads * d, w + t * (long)n_heads,
+                 K + k_offsets[t] * (long)d, (long)(k_offsets[t + 1] - k_offsets[t]),
+                 rep + blk_offsets[t] * (long)d, given_blocks ? given_blocks + t * (long)top_blocks : NULL,
+                 out_blocks + t * (long)top_blocks, out_idx + t * (long)topk, out_count + t,
+                 coarse_score ? coarse_score + blk_offsets[t] : NULL);
+}
+
+/* O4h, prefill (causal) form: the n queries of one sequence, query i seeing
+ * keys 0..i as the flat indexer's prefill rows do ([P2] §2.1 Eq.(4), S_t over
+ * r_{t,0:t}).  Its complete blocks are the sequence's blocks j < (i + 1) / blk,
+ * whose representatives (rep, computed once for the sequence) do not depend on
+ * the query; the rest is the row rule above with ctx = i + 1.  Layout: q [n,
+ * heads, d]; w [n, heads]; K [n, d]; rep [n / blk, d]; outputs per query. */
+OAPI void oracle_hisa_topk_prefill(int n, int n_heads, int d, int topk, int blk, int top_blocks,
+                                   const double *q, const double *w, const double *K, const double *rep,
+                                   int32_t *out_blocks, int32_t *out_idx, int32_t *out_count)
+{
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long i = 0; i < n; ++i)
+        hisa_row(n_heads, d, topk, blk, top_blocks, q + i * (long)n_heads * d, w + i * (long)n_heads, K,
+                 i + 1, rep, NULL, out_blocks + i * (long)top_blocks, out_idx + i * (long)topk, out_count + i,
+                 NULL);
 }
 
 /* ======================================================================
