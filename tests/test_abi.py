@@ -64,3 +64,38 @@ def test_short_workspace_is_rejected_before_launch(crs):
     st = lib.crs_lsh_attn(ctypes.byref(a), dummy, dummy, dummy, dummy, dummy, None, dummy, None,
                           dummy, 16, None)
     assert st == 6
+
+
+def test_host_validation_of_the_later_entry_points(crs):
+    """HISA, LSH decode, routing, the compressed / subspace / Quest block selectors:
+    out-of-range parameters give CRS_ERR_INVALID_ARG (1), shapes the kernels do not
+    implement CRS_ERR_UNSUPPORTED (2), missing buffers CRS_ERR_INVALID_ARG, all
+    before any device work (these calls run on a machine without a GPU)."""
+    lib = crs.lib()
+    by = ctypes.byref
+    # HISA: no rows; index head dim other than 64; then NULL buffers
+    assert lib.crs_hisa_topk(by(crs.HisaParams(0, 4, 64, 2048, 64, 128, 131072)), *([None] * 10), 0, None) == 1
+    assert lib.crs_hisa_describe(by(crs.HisaParams(4, 4, 32, 2048, 64, 128, 131072)), *([None] * 5)) == 2
+    assert lib.crs_hisa_describe(by(crs.HisaParams(4, 4, 64, 2048, 64, 128, 131072)), *([None] * 5)) == 1
+    assert lib.crs_hisa_topk(by(crs.HisaParams(4, 4, 64, 2048, 64, 128, 131072)), *([None] * 10), 0, None) == 1
+    assert lib.crs_hisa_topk_workspace_size(by(crs.HisaParams(0, 4, 64, 2048, 64, 128, 131072))) == 0
+    # LSH decode: odd bucket count; d other than 64; valid parameters with an empty state
+    ld = dict(n_seq=2, n_heads=2, d=64, n_buckets=16, n_rounds=2, page_size=16, max_pages=8, list_page=8,
+              list_pages=8, n_list_pages=64, max_len=128, no_self=1, key_norm=1, scale=0.125)
+    st = crs.LshDecodeState()
+    assert lib.crs_lsh_decode_step(by(crs.LshDecodeParams(**{**ld, "n_buckets": 15})), by(st), *([None] * 7)) == 1
+    assert lib.crs_lsh_decode_step(by(crs.LshDecodeParams(**{**ld, "d": 32})), by(st), *([None] * 7)) == 2
+    assert lib.crs_lsh_decode_step(by(crs.LshDecodeParams(**ld)), by(st), *([None] * 7)) == 1
+    assert lib.crs_lsh_decode_prefill(by(crs.LshDecodeParams(**ld)), by(st), None, None, None, 4, None) == 1
+    # routing: no centres; head dim other than 64; then NULL inputs
+    assert lib.crs_route_attn(by(crs.RouteParams(1, 1, 256, 64, 0, 8, 1, 0, 0.125)), *([None] * 10), 0, None) == 1
+    assert lib.crs_route_attn(by(crs.RouteParams(1, 1, 256, 32, 4, 8, 1, 0, 0.125)), *([None] * 10), 0, None) == 2
+    assert lib.crs_route_attn(by(crs.RouteParams(1, 1, 256, 64, 4, 8, 1, 0, 0.125)), *([None] * 10), 0, None) == 1
+    # block selectors on FP4 codes, the query subspace and Quest boxes: NULL inputs
+    bp = crs.BlockParams(2, 2, 4096, 128, 32, 4, 0, 4096 // 32)
+    sp = crs.BlockSelParams(bp, 16, 16, 256, 0.0884)
+    assert lib.crs_block_select_fp4(by(sp), *([None] * 7), 0, None) == 1
+    assert lib.crs_block_select_ss(by(sp), None, None, 16, *([None] * 5), 0, None) == 1
+    assert lib.crs_block_select_quest(by(sp), *([None] * 6), 0, None) == 1
+    assert lib.crs_block_quest_describe(by(bp), None, None, None, None) == 1
+    assert lib.crs_block_quantize(by(bp), *([None] * 6)) == 1
