@@ -1,7 +1,8 @@
 """Pins for the query-subspace descriptors and selection of the oracle ("COBS 阅读笔记",
 "子空间方法", Eq.(17)-(18)): the identity subspace reproduces the full-space descriptors,
 the quadratic term equals the covariance quadratic form of the projected query computed
-from the keys themselves, and the eigenvalues are those of U^T Sigma U."""
+from the keys themselves, the eigenvalues are those of U^T Sigma U, and keys that lie in
+the subspace are selected exactly as by the full-space selector."""
 import numpy as np
 
 import oracle
@@ -52,3 +53,25 @@ def test_quadratic_term_is_the_projected_query_form():
     direct = np.array([q[0, 0] @ keys[b].mean(axis=0)
                        + 0.5 * np.mean(((keys[b] - keys[b].mean(axis=0)) @ pq) ** 2) for b in range(n_full)])
     np.testing.assert_allclose(lb - lb[0], direct - direct[0], rtol=0, atol=1e-10)
+
+
+def test_keys_inside_the_subspace_select_as_in_the_full_space():
+    """Keys m + U z (a full-space mean plus a component in span U): every block covariance
+    lies in span U, the full-space eigenvectors are U times the subspace ones, so the
+    subspace selector's scores and picks equal the full-space selector's ([P5] Eq.(17)-(18)
+    against Eq.(14)-(16))."""
+    rng = np.random.default_rng(14)
+    D, s, L, nb, rank = 10, 4, 8, 9, 3
+    U = _orthonormal(rng, D, s)
+    m = rng.standard_normal(D)
+    z = rng.standard_normal((nb * L, s)) * np.linspace(0.5, 2.0, s)
+    K = (m + z @ U.T).reshape(nb, L, D)
+    mu, xi, _ = oracle.block_describe(K, rank)
+    mu_s, xi_s, _ = oracle.block_describe_ss(K, U, rank)
+    Q = rng.standard_normal((1, 2, D))
+    T, top, win = nb * L, 3, 8
+    full = oracle.block_select(Q, mu[None, None], xi[None, None], T, L, top, win, scale=0.5)
+    sub = oracle.block_select_ss(Q, U, mu_s[None, None], xi_s[None, None], T, L, top, win, scale=0.5)
+    np.testing.assert_allclose(sub[3], full[3], rtol=1e-9, atol=1e-9)     # block scores
+    assert np.array_equal(sub[2], full[2])                                # picked blocks
+    assert np.array_equal(sub[0], full[0]) and np.array_equal(sub[1], full[1])
