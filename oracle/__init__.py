@@ -75,7 +75,7 @@ def _lib():
         lib.oracle_quest_select.argtypes = [I, I, I, I, I, I, I, I, I, D, _f64p, _f64p, _f64p, I,
                                             _i32p, _i32p, _i32p, _f64p]
         lib.oracle_sparse_attn.argtypes = [I, I, I, I, D, _f64p, _f64p, _f64p, _i64p, _i32p, I, I,
-                                           _f64p, _f64p]
+                                           _u8p, _i32p, _f64p, _f64p]
         _LIB = lib
     return _LIB
 
@@ -455,10 +455,12 @@ def fp4_dequantize(codes, scale):
 
 
 # ---------------------------------------------------------- attention --
-def sparse_attn(Q, K, V, I, kv_base=None, scale=None):
+def sparse_attn(Q, K, V, I, kv_base=None, scale=None, key_valid=None, q_pos=None):
     """Q [rows, n_q, D]; K, V [tokens, n_kv, D]; I [rows, n_lists, max_idx]
-    (n_lists = n_kv or 1); kv_base [rows] token offset of each row's sequence.
-    Returns (O [rows, n_q, D], lse [rows, n_q])."""
+    (n_lists = n_kv or 1); kv_base [rows] token offset of each row's sequence;
+    key_valid [tokens] (non-zero = the key may be attended; None = all) and
+    q_pos [rows] (entry j of row t is used only if j <= q_pos[t]; None = no
+    causal limit).  Returns (O [rows, n_q, D], lse [rows, n_q])."""
     Q = _c(Q, np.float64)
     K = _c(K, np.float64)
     V = _c(V, np.float64)
@@ -473,9 +475,13 @@ def sparse_attn(Q, K, V, I, kv_base=None, scale=None):
     kb = _c(kv_base, np.int64)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    kv = None if key_valid is None else _c(np.asarray(key_valid) != 0, np.uint8)
+    qp = None if q_pos is None else _c(q_pos, np.int32)
     O = np.empty((rows, n_q, D), dtype=np.float64)
     lse = np.empty((rows, n_q), dtype=np.float64)
     _lib().oracle_sparse_attn(rows, n_q, n_kv, D, float(scale), _p(Q, _f64p), _p(K, _f64p),
                               _p(V, _f64p), _p(kb, _i64p), _p(I, _i32p), n_lists, max_idx,
+                              None if kv is None else _p(kv, _u8p),
+                              None if qp is None else _p(qp, _i32p),
                               _p(O, _f64p), _p(lse, _f64p))
     return O, lse

@@ -1029,13 +1029,27 @@ OAPI void oracle_quest_select(int n_seq, int n_kv, int n_q, int D, int n_full, i
  *   O_{t,g} = sum_{j in I} softmax_j(scale * q_{t,g} . k_{j,kv(g)}) v_{j,kv(g)}
  * over the valid (>= 0) entries of the index list; an empty list gives 0 and
  * lse = -inf.  Duplicated entries are a caller error and are counted as given.
+ * Masks ([P1] §1.1 Eq.(2): the allowed set P(i) is cut by the causal and the
+ * padding mask before the softmax): an entry j of row t takes part only when
+ * j <= q_pos[t] (q_pos NULL: no causal limit) and key_valid[kv_base[t] + j]
+ * is non-zero (key_valid NULL: every key valid).
  * Layout: Q [rows, n_q, D]; K, V: token j of row t, head h at
  * ((kv_base[t] + j) * n_kv + h) * D; I [rows, n_lists, max_idx] where
  * n_lists = n_kv (a list per KV head) or 1 (one list shared by all heads).
  * ====================================================================== */
+static int oracle_entry_allowed(int32_t j, long t, const int64_t *kv_base,
+                                const uint8_t *key_valid, const int32_t *q_pos)
+{
+    if (j < 0) return 0;
+    if (q_pos && j > q_pos[t]) return 0;
+    if (key_valid && !key_valid[kv_base[t] + j]) return 0;
+    return 1;
+}
+
 OAPI void oracle_sparse_attn(int n_rows, int n_q, int n_kv, int D, double scale, const double *Q,
                              const double *K, const double *V, const int64_t *kv_base,
-                             const int32_t *I, int n_lists, int max_idx, double *O, double *lse)
+                             const int32_t *I, int n_lists, int max_idx, const uint8_t *key_valid,
+                             const int32_t *q_pos, double *O, double *lse)
 {
     const int G = n_q / n_kv;
 #pragma omp parallel
@@ -1052,7 +1066,7 @@ OAPI void oracle_sparse_attn(int n_rows, int n_q, int n_kv, int D, double scale,
                     o[k] = 0.0;
                 double mx = -INFINITY;
                 for (int c = 0; c < max_idx; ++c) {
-                    if (idx[c] < 0) continue;
+                    if (!oracle_entry_allowed(idx[c], t, kv_base, key_valid, q_pos)) continue;
                     const double *kj = K + ((kv_base[t] + idx[c]) * n_kv + h) * (long)D;
                     double dot = 0.0;
                     for (int k = 0; k < D; ++k)
@@ -1066,9 +1080,9 @@ OAPI void oracle_sparse_attn(int n_rows, int n_q, int n_kv, int D, double scale,
                 }
                 double z = 0.0;
                 for (int c = 0; c < max_idx; ++c)
-                    if (idx[c] >= 0) z += exp(logit[c] - mx);
+                    if (oracle_entry_allowed(idx[c], t, kv_base, key_valid, q_pos)) z += exp(logit[c] - mx);
                 for (int c = 0; c < max_idx; ++c) {
-                    if (idx[c] < 0) continue;
+                    if (!oracle_entry_allowed(idx[c], t, kv_base, key_valid, q_pos)) continue;
                     const double p = exp(logit[c] - mx) / z;
                     const double *vj = V + ((kv_base[t] + idx[c]) * n_kv + h) * (long)D;
                     for (int k = 0; k < D; ++k)

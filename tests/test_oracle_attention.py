@@ -54,6 +54,62 @@ def test_all_visible_is_dense_causal(n_q, n_kv):
     assert np.abs(O - ref).max() < 1e-12
 
 
+@pytest.mark.parametrize("n_q,n_kv", [(4, 1), (6, 2)])
+def test_masks_on_full_lists_are_dense_causal_with_padding(n_q, n_kv):
+    """PaperTrace 2.1.1 §1.1 Eq.(2): the allowed set is cut by the causal and the padding
+    masks.  Every row lists every key; q_pos and key_valid alone must then give dense
+    attention under the mask (j <= i) & valid(j) (torch SDPA, fp64), on two sequences
+    packed behind kv_base."""
+    rng = np.random.default_rng(n_q + 7 * n_kv)
+    lens, D = [23, 31], 16
+    base = np.array([0, lens[0]], np.int64)
+    tokens = sum(lens)
+    K = rng.standard_normal((tokens, n_kv, D))
+    V = rng.standard_normal((tokens, n_kv, D))
+    valid = rng.random(tokens) > 0.3
+    valid[[0, lens[0]]] = True                      # every row keeps at least one key
+    rows_q, rows_b, rows_p = [], [], []
+    for s_, n in enumerate(lens):
+        for t in range(n):
+            rows_b.append(base[s_])
+            rows_p.append(t)
+    rows = len(rows_b)
+    Q = rng.standard_normal((rows, n_q, D))
+    nmax = max(lens)
+    I = np.full((rows, 1, nmax), -1, np.int32)
+    for r in range(rows):
+        n = lens[0] if rows_b[r] == 0 else lens[1]
+        I[r, 0, :n] = rng.permutation(n)            # list order does not matter
+    O, lse = oracle.sparse_attn(Q, K, V, I, kv_base=np.array(rows_b), key_valid=valid,
+                                q_pos=np.array(rows_p, np.int32))
+    scale = 1.0 / math.sqrt(D)
+    r0 = 0
+    for s_, n in enumerate(lens):
+        b = int(base[s_])
+        i = np.arange(n)[:, None]
+        j = np.arange(n)[None]
+        mask = (j <= i) & valid[b:b + n][None]
+        ref = _dense_sdpa(Q[r0:r0 + n], K[b:b + n], V[b:b + n], mask, scale)
+        assert np.abs(O[r0:r0 + n] - ref).max() < 1e-12
+        r0 += n
+    # the unmasked call attends to every listed key
+    O2, _ = oracle.sparse_attn(Q[:lens[0]], K[:lens[0]], V[:lens[0]], I[:lens[0], :, :lens[0]])
+    ref2 = _dense_sdpa(Q[:lens[0]], K[:lens[0]], V[:lens[0]], np.ones((lens[0], lens[0]), bool), scale)
+    assert np.abs(O2 - ref2).max() < 1e-12
+
+
+def test_masks_that_remove_every_entry_give_zero():
+    rng = np.random.default_rng(9)
+    Q = rng.standard_normal((2, 2, 8))
+    K = rng.standard_normal((10, 1, 8))
+    V = rng.standard_normal((10, 1, 8))
+    I = np.array([[[5, 6, 7]], [[1, 2, -1]]], np.int32)
+    valid = np.ones(10, bool)
+    valid[[1, 2]] = False
+    O, lse = oracle.sparse_attn(Q, K, V, I, key_valid=valid, q_pos=np.array([4, 9], np.int32))
+    assert (O == 0).all() and (lse == -np.inf).all()
+
+
 def test_window_is_sliding_window_attention():
     rng = np.random.default_rng(1)
     n, D, W = 50, 8, 6
