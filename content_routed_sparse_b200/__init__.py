@@ -128,6 +128,8 @@ _sig("crs_lsh_route", ctypes.c_int, [ctypes.POINTER(LshParams), _VP, _VP, _VP, _
 _sig("crs_lsh_attn_workspace_size", _SZ, [ctypes.POINTER(LshAttnParams)])
 _sig("crs_lsh_attn", ctypes.c_int, [ctypes.POINTER(LshAttnParams), _VP, _VP, _VP, _VP, _VP, _VP,
                                      _VP, _VP, _VP, _SZ, _VP])
+_sig("crs_lsh_candidates_csr", ctypes.c_int, [ctypes.POINTER(LshAttnParams), _VP, _VP, _VP, _VP, _VP, _VP,
+                                               _VP])
 _sig("crs_indexer_topk_workspace_size", _SZ, [ctypes.POINTER(IndexerParams)])
 _sig("crs_indexer_topk", ctypes.c_int, [ctypes.POINTER(IndexerParams), _VP, _VP, _VP, _VP, _VP,
                                          _VP, _VP, _SZ, _VP])
@@ -161,7 +163,7 @@ _sig("crs_block_select_noalloc", ctypes.c_int, [ctypes.POINTER(BlockSelParams), 
                                                  _VP, _VP, _VP])
 _sig("crs_sparse_attn_workspace_size", _SZ, [ctypes.POINTER(AttnParams)])
 _sig("crs_sparse_attn", ctypes.c_int, [ctypes.POINTER(AttnParams), _VP, _VP, _VP, _VP, _VP, _VP,
-                                        _VP, _VP, _SZ, _VP])
+                                        _VP, _VP, _VP, _VP, _SZ, _VP])
 
 
 _sig("crs_profile_set", ctypes.c_int, [ctypes.c_int])
@@ -316,6 +318,27 @@ def lsh_attn(QK, V, bucket, perm, inv_perm, valid_len=None, *, n_buckets, chunk,
 
 
 # ---------------------------------------------------------------- indexer --
+def lsh_candidates_csr(bucket, perm, inv_perm, valid_len=None, *, chunk, causal=1, no_self=0,
+                       stream=None):
+    """The candidate sets U(i) of lsh_attn as CSR: (row_ptr [B*H*n + 1] int64,
+    col_idx int32), rows ordered (b, h, i), each row ascending.  Two library calls
+    (counts, then the rows) with one host read of the total in between."""
+    _need(bucket, "bucket", torch.int32)
+    B, H, R, n = bucket.shape
+    _need(perm, "perm", torch.int32, bucket.shape)
+    _need(inv_perm, "inv_perm", torch.int32, bucket.shape)
+    if valid_len is not None:
+        _need(valid_len, "valid_len", torch.int32, (B,))
+    a = LshAttnParams(LshParams(B, H, n, 8, 2, R, int(chunk), CRS_BF16), int(causal), int(no_self), 1, 1.0)
+    row_ptr = torch.empty(B * H * n + 1, dtype=torch.int64, device=bucket.device)
+    args = (ctypes.byref(a), _ptr(bucket), _ptr(perm), _ptr(inv_perm), _ptr(valid_len), _ptr(row_ptr))
+    _check("crs_lsh_candidates_csr", _lib.crs_lsh_candidates_csr(*args, None, _stream(stream)))
+    nnz = int(row_ptr[-1].item())
+    col = torch.empty(max(nnz, 1), dtype=torch.int32, device=bucket.device)
+    _check("crs_lsh_candidates_csr", _lib.crs_lsh_candidates_csr(*args, _ptr(col), _stream(stream)))
+    return row_ptr, col[:nnz]
+
+
 def indexer_topk(q_idx, w, k_idx, topk: int, mode: int = CRS_IDX_PREFILL, k_offsets=None,
                  max_keys: int = 0, out=None, count=None, workspace=None, stream=None):
     """Lightning-indexer top-k; returns (idx [rows, topk] int32 ascending, -1 pad; count [rows])."""
@@ -715,11 +738,13 @@ def block_select_noalloc(Q, mu, xi, T: int, L: int, top_blocks: int, window: int
 
 
 # -------------------------------------------------------------- attention --
-def sparse_attn(Q, K, V, I, kv_base=None, scale=None, n_keys: int = 0, out=None, lse=None,
-                workspace=None, stream=None):
+def sparse_attn(Q, K, V, I, kv_base=None, scale=None, key_valid=None, q_pos=None, out=None,
+                lse=None, workspace=None, stream=None):
     """Attention over index lists -> (O [rows, n_q, D] fp32, lse).  Q [rows, n_q, D];
     K, V [tokens, n_kv, D] (token j of row t at kv_base[t] + j); I [rows, n_lists,
-    max_idx] (n_lists 1 or n_kv)."""
+    max_idx] (n_lists 1 or n_kv).  key_valid [tokens] uint8/bool (0 = padding key)
+    and q_pos [rows] int32 (entries j > q_pos[t] skipped) are optional masks.  Every
+    entry is bounds-checked against K's token count on the device."""
     _need(Q, "Q", torch.bfloat16)
     rows, n_q, D = Q.shape
     _need(K, "K", torch.bfloat16)
@@ -731,6 +756,13 @@ def sparse_attn(Q, K, V, I, kv_base=None, scale=None, n_keys: int = 0, out=None,
     n_lists, max_idx = I.shape[1], I.shape[2]
     if kv_base is not None:
         _need(kv_base, "kv_base", torch.int64, (rows,))
+    n_keys = K.numel() // (n_kv * D)
+    if key_valid is not None:
+        if key_valid.dtype == torch.bool:
+            key_valid = key_valid.view(torch.uint8)
+        _need(key_valid, "key_valid", torch.uint8, (n_keys,))
+    if q_pos is not None:
+        _need(q_pos, "q_pos", torch.int32, (rows,))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     p = AttnParams(rows, n_q, n_kv, D, max_idx, n_lists, int(n_keys), float(scale))
@@ -742,6 +774,7 @@ def sparse_attn(Q, K, V, I, kv_base=None, scale=None, n_keys: int = 0, out=None,
     ws, wsb = _workspace(int(_lib.crs_sparse_attn_workspace_size(ctypes.byref(p))), Q.device,
                          workspace)
     st = _lib.crs_sparse_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(kv_base),
-                              _ptr(I), _ptr(out), _ptr(lse), _ptr(ws), wsb, _stream(stream))
+                              _ptr(I), _ptr(key_valid), _ptr(q_pos), _ptr(out), _ptr(lse),
+                              _ptr(ws), wsb, _stream(stream))
     _check("crs_sparse_attn", st)
     return out, lse

@@ -3,6 +3,7 @@
 #include "api.cu"
 #include "lsh_tc.cu"
 #include "lsh.cu"
+#include "lsh_csr.cu"
 #include "lsh_decode.cu"
 #include "sparse_attn.cu"
 #include "indexer.cu"

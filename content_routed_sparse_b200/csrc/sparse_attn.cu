@@ -67,6 +67,8 @@ struct SaArgs {
     const __nv_bfloat16 *Q, *K, *V;
     const int64_t *kv_base;
     const int32_t *I;
+    const uint8_t *key_valid;   // [n_keys] or null: padding mask
+    const int32_t *q_pos;       // [n_rows] or null: causal limit per row
     float *O;
     float *lse;
     float *part_o;      // [rows*n_q][splits][D] (splits > 1)
@@ -106,13 +108,18 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
         *reinterpret_cast<uint4 *>(sQ + sw_off(r, c)) = v;
     }
 
-    // the split's index list, once, into shared memory (padded with -1 to whole tiles)
+    // the split's index list, once, into shared memory (padded with -1 to whole
+    // tiles).  An entry outside K/V is flagged and skipped; masked entries (after
+    // the row's causal limit, or on a padding key) are skipped ([P1] §1.1 Eq.(2)).
+    const int qlim = a.q_pos ? a.q_pos[row] : 0x7fffffff;
     for (int i = tid; i < n_tiles * kSaKeys; i += kSaThreads) {
         int j = (s0 + i < s1) ? __ldg(idx + s0 + i) : -1;
-        if (j >= 0 && a.n_keys > 0 && j >= a.n_keys) {
+        if (j < -1 || (j >= 0 && kbase + j >= (int64_t)a.n_keys)) {
             raise_error(CRS_DEVERR_INDEX);
             j = -1;
         }
+        if (j > qlim) j = -1;
+        if (j >= 0 && a.key_valid && a.key_valid[kbase + j] == 0) j = -1;
         sIdx[i] = j;
     }
     __syncthreads();
@@ -394,7 +401,7 @@ static int sa_validate(const crs_attn_params *p) {
     if (p->n_q % p->n_kv != 0 || p->n_q / p->n_kv > 16) return CRS_ERR_UNSUPPORTED;
     if (p->D != kSaD) return CRS_ERR_UNSUPPORTED;
     if (p->n_lists != 1 && p->n_lists != p->n_kv) return CRS_ERR_INVALID_ARG;
-    if (p->n_keys < 0) return CRS_ERR_INVALID_ARG;
+    if (p->n_keys < 1) return CRS_ERR_INVALID_ARG;
     if ((long long)p->n_rows * p->n_kv > 0x7fffffffLL) return CRS_ERR_UNSUPPORTED;
     return CRS_OK;
 }
@@ -412,7 +419,8 @@ extern "C" size_t crs_sparse_attn_workspace_size(const crs_attn_params *p) {
 }
 
 extern "C" int crs_sparse_attn(const crs_attn_params *p, const void *Q, const void *K,
-                               const void *V, const int64_t *kv_base, const int32_t *I, void *O,
+                               const void *V, const int64_t *kv_base, const int32_t *I,
+                               const uint8_t *key_valid, const int32_t *q_pos, void *O,
                                float *lse, void *ws, size_t ws_bytes, void *stream) {
     int st = sa_validate(p);
     if (st) return st;
@@ -426,6 +434,8 @@ extern "C" int crs_sparse_attn(const crs_attn_params *p, const void *Q, const vo
     a.V = static_cast<const __nv_bfloat16 *>(V);
     a.kv_base = kv_base;
     a.I = I;
+    a.key_valid = key_valid;
+    a.q_pos = q_pos;
     a.O = static_cast<float *>(O);
     a.lse = lse;
     a.n_rows = p->n_rows;

@@ -159,6 +159,25 @@ int crs_lsh_attn(const crs_lsh_attn_params *p, const void *QK, const void *V,
                  const int32_t *valid_len, void *O, float *lse, void *ws, size_t ws_bytes,
                  void *stream);
 
+/* The candidate sets U(i) of crs_lsh_attn as an explicit CSR matrix, an
+ * inspection export for small inputs ([P1] §4: the index tensors row_ptr /
+ * col_idx, perm, inverse_perm; §2.1-2.2 and §1.1 Eq.(2) define the set: the
+ * keys j of i's chunk and the chunk before it, in some round, with i's bucket,
+ * j <= i when causal, j != i when no_self, j < valid_len[b]; each key once).
+ * A padded query (i >= valid_len[b]) gets its set like any other row
+ * (crs_lsh_attn gives such a row O = 0).  Rows are ordered (b, h, i).
+ *   row_ptr: [B*H*n + 1] int64; col_idx: [row_ptr[B*H*n]] int32, each row's
+ *   keys ascending.
+ * Two calls: with col_idx == NULL the call writes row_ptr (counts, then their
+ * prefix sum; read row_ptr[B*H*n] to size col_idx); with col_idx it fills the
+ * rows, reading row_ptr as the first call left it (same inputs).  Only the
+ * routing fields of p (B, H, n, n_rounds, chunk), causal and no_self are used.
+ * n <= 65536 and B*H*n <= 2^22 (else CRS_ERR_UNSUPPORTED); a permutation
+ * entry outside [0, n) sets CRS_DEVERR_INDEX and is skipped. */
+int crs_lsh_candidates_csr(const crs_lsh_attn_params *p, const int32_t *bucket, const int32_t *perm,
+                           const int32_t *inv_perm, const int32_t *valid_len, int64_t *row_ptr,
+                           int32_t *col_idx, void *stream);
+
 /* ====================================================================== *
  * LSH attention in decode.  [P1] §5.2 "Prefill、Decode 与 KV 状态": the hash is
  * fixed (R as crs_lsh_route); each new token's bucket ids (one per round, O(d R))
@@ -453,11 +472,13 @@ int crs_block_select_quest(const crs_block_sel_params *p, const void *Q, const v
 
 /* ====================================================================== *
  * Attention over explicit index lists.  [P1] §1.1 Eq.(1) restricted to the
- * candidate set; [P2] §1.1 (one selected set shared by the main heads);
+ * candidate set, with the allowed set P(i) of Eq.(2) cut by the causal and the
+ * padding mask; [P2] §1.1 (one selected set shared by the main heads);
  * [P4] §26.2 (query heads [h*G, (h+1)*G) share KV head h):
  *   O_{t,g} = sum_{j in I} softmax_j(scale * q_{t,g} . k_{j,h}) v_{j,h},  h = g / G,
- * over the entries of the row's list that are >= 0.  An empty list gives
- * O = 0 and lse = -inf.  Duplicated entries are a caller error.
+ * over the entries j of the row's list with j >= 0, j <= q_pos[t] and
+ * key_valid[kv_base[t] + j] != 0.  An empty set gives O = 0 and lse = -inf.
+ * Duplicated entries are a caller error.
  * ====================================================================== */
 typedef struct {
     int n_rows;     /* queries                                               */
@@ -467,20 +488,30 @@ typedef struct {
     int max_idx;    /* slots per index list                                  */
     int n_lists;    /* 1: one list per row shared by all KV heads;
                        n_kv: one list per (row, KV head)                     */
-    int n_keys;     /* entries must be < n_keys (bounds check); 0 = no check  */
+    int n_keys;     /* tokens held by K and V (their first dimension), >= 1:
+                       an entry j of row t with kv_base[t] + j >= n_keys, or
+                       j < -1, sets CRS_DEVERR_INDEX and is skipped, so no
+                       entry can reach outside K/V                          */
     float scale;    /* typically 1/sqrt(D)                                   */
 } crs_attn_params;
 
-/* Q: [n_rows, n_q, D] bf16.  K, V: bf16, token j of row t and KV head h at
- * element ((kv_base[t] + j) * n_kv + h) * D (kv_base: [n_rows] int64, NULL =
- * 0).  I: [n_rows, n_lists, max_idx] int32.  O: [n_rows, n_q, D] f32 (the
- * fp32 accumulator's precision; P.V runs on bf16 tensor cores with P split
- * into a bf16 value and a bf16 residual);
- * lse: [n_rows, n_q] f32 or NULL. */
+/* Q: [n_rows, n_q, D] bf16.  K, V: [n_keys, n_kv, D] bf16, token j of row t
+ * and KV head h at element ((kv_base[t] + j) * n_kv + h) * D (kv_base:
+ * [n_rows] int64, NULL = 0).  I: [n_rows, n_lists, max_idx] int32.
+ * Masks (either may be NULL = no mask):
+ *   key_valid: [n_keys] uint8, 0 marks a padding key never attended;
+ *   q_pos:     [n_rows] int32, the causal limit: entries j > q_pos[t] are
+ *              skipped (for a decode row of a sequence with c keys, c - 1).
+ * O: [n_rows, n_q, D] f32 (the fp32 accumulator's precision; P.V runs on bf16
+ * tensor cores with P split into a bf16 value and a bf16 residual);
+ * lse: [n_rows, n_q] f32 or NULL.
+ * Workspace: crs_sparse_attn_workspace_size(p), queried with the same device
+ * current as the call (the split count depends on the device's SM count). */
 size_t crs_sparse_attn_workspace_size(const crs_attn_params *p);
 int crs_sparse_attn(const crs_attn_params *p, const void *Q, const void *K, const void *V,
-                    const int64_t *kv_base, const int32_t *I, void *O, float *lse, void *ws,
-                    size_t ws_bytes, void *stream);
+                    const int64_t *kv_base, const int32_t *I, const uint8_t *key_valid,
+                    const int32_t *q_pos, void *O, float *lse, void *ws, size_t ws_bytes,
+                    void *stream);
 
 #ifdef __cplusplus
 }

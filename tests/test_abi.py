@@ -43,8 +43,10 @@ def test_host_validation_without_gpu(crs):
     assert lib.crs_lsh_attn(ctypes.byref(a), *([None] * 9), 0, None) == 1
     ip = crs.IndexerParams(0, 10, 4, 32, 16, 0)         # d_idx != 64
     assert lib.crs_indexer_topk(ctypes.byref(ip), *([None] * 6), None, 0, None) == 2
-    ap = crs.AttnParams(4, 48, 2, 128, 16, 1, 0, 0.1)    # G = 24 > 16
-    assert lib.crs_sparse_attn(ctypes.byref(ap), *([None] * 8), 0, None) == 2
+    ap = crs.AttnParams(4, 48, 2, 128, 16, 1, 100, 0.1)  # G = 24 > 16
+    assert lib.crs_sparse_attn(ctypes.byref(ap), *([None] * 10), 0, None) == 2
+    ap = crs.AttnParams(4, 16, 1, 128, 16, 1, 0, 0.1)    # no key count: no bound to check
+    assert lib.crs_sparse_attn(ctypes.byref(ap), *([None] * 10), 0, None) == 1
     bp = crs.BlockParams(1, 1, 64, 128, 31, 4, 0, 2)     # odd L
     assert lib.crs_block_describe(ctypes.byref(bp), None, None, None, None) == 2
 
@@ -99,3 +101,19 @@ def test_host_validation_of_the_later_entry_points(crs):
     assert lib.crs_block_select_quest(by(sp), *([None] * 6), 0, None) == 1
     assert lib.crs_block_quest_describe(by(bp), None, None, None, None) == 1
     assert lib.crs_block_quantize(by(bp), *([None] * 6)) == 1
+
+
+def test_host_validation_of_the_csr_export(crs):
+    """crs_lsh_candidates_csr: too many rounds, a chunk past 128, NULL routing arrays and
+    an input beyond the export's size limit are rejected before any launch."""
+    lib = crs.lib()
+    by = ctypes.byref
+    dummy = ctypes.c_void_p(0x1000)
+    bad_rounds = crs.LshAttnParams(crs.LshParams(1, 1, 64, 64, 16, 9, 8, 1), 1, 0, 1, 0.125)
+    assert lib.crs_lsh_candidates_csr(by(bad_rounds), dummy, dummy, dummy, None, dummy, None, None) == 1
+    bad_chunk = crs.LshAttnParams(crs.LshParams(1, 1, 64, 64, 16, 2, 256, 1), 1, 0, 1, 0.125)
+    assert lib.crs_lsh_candidates_csr(by(bad_chunk), dummy, dummy, dummy, None, dummy, None, None) == 1
+    ok = crs.LshAttnParams(crs.LshParams(1, 1, 64, 64, 16, 2, 32, 1), 1, 0, 1, 0.125)
+    assert lib.crs_lsh_candidates_csr(by(ok), None, dummy, dummy, None, dummy, None, None) == 1
+    big = crs.LshAttnParams(crs.LshParams(1, 1, 70000, 64, 16, 2, 32, 1), 1, 0, 1, 0.125)
+    assert lib.crs_lsh_candidates_csr(by(big), dummy, dummy, dummy, None, dummy, None, None) == 2

@@ -5,7 +5,7 @@ import torch
 
 import oracle
 import workloads
-from parity import rel_err
+from parity import cutoff_gaps, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -52,7 +52,10 @@ def test_describe_small(crs, cuda_dev):
 
 
 def _check_select(tok, cnt, o_tok, o_cnt, o_blk, o_bs, L, T, window, top, what):
+    """Token lists ascending and -1 padded; kept blocks equal to the oracle's except
+    blocks whose oracle score lies within 1e-5 relative of the cutoff."""
     n_seq, n_kv = cnt.shape
+    ndiff, worst = 0, 0.0
     for s in range(n_seq):
         for h in range(n_kv):
             gt = tok[s, h, : cnt[s, h]]
@@ -63,11 +66,14 @@ def _check_select(tok, cnt, o_tok, o_cnt, o_blk, o_bs, L, T, window, top, what):
             diff = np.setxor1d(gb, ob)
             if diff.size:
                 sc = o_bs[s, h]
-                cut = np.sort(sc)[::-1][top - 1]
-                assert np.all(np.abs(sc[diff] - cut) <= 1e-5 * abs(cut) + 1e-6), \
-                    f"{what} ({s},{h}): blocks {diff} not at the cutoff"
+                cut = float(np.sort(sc)[::-1][top - 1])
+                worst = max(worst, cutoff_gaps(sc[diff], cut, what=f"{what} ({s},{h}) blocks {diff}"))
+                ndiff += diff.size
             else:
                 assert cnt[s, h] == o_cnt[s, h]
+    print(f"{what}: {n_seq * n_kv} (sequence, KV head) sets, {ndiff} differing blocks, largest "
+          f"relative gap to the cutoff {worst:.3e}")
+    return ndiff
 
 
 def test_select_on_oracle_descriptors(crs, cuda_dev):
@@ -106,24 +112,27 @@ def test_select_ragged_block_count(crs, cuda_dev):
 
 
 def test_describe_select_end_to_end_small(crs, cuda_dev):
+    """Describe then select, checked stage by stage ([P1] "最小正确性测试": the same
+    inputs first).  The fp32 descriptors against the fp64 oracle within the fp32
+    Jacobi bounds of test_describe_small; the selection against the oracle run on
+    those GPU descriptors under the 1e-5 cutoff rule.  (The oracle's own fp64
+    descriptors move a block score by up to ~1e-4 relative when the fp32 eigen
+    decomposition differs at that level, which no cutoff rule on the selection
+    alone can separate from a selection fault.)"""
     case = workloads.block_decode_case(n_seq=2, T=2048, seed=6, device=cuda_dev)
     p = case["params"]
     L, r, top, win = p["L"], p["rank"], 8, 128
     mu, xi = crs.block_describe(case["K"], L, r)
     tok, cnt = crs.block_select(case["Q"], mu, xi, p["T"], L, top, win)
     torch.cuda.synchronize()
-    omu, oxi, _ = _oracle_describe(_np(case["K"]), L, r)
-    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), omu, oxi[..., :r, :], p["T"], L,
+    omu, oxi, olam = _oracle_describe(_np(case["K"]), L, r)
+    assert rel_err(_np(mu), omu).max() < 1e-5
+    glam = (_np(xi) ** 2).sum(-1)
+    assert np.abs(glam - olam[..., :r]).max() <= 1e-4 * olam[..., 0].max()
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), _np(mu), _np(xi), p["T"], L,
                                                     top, win)
-    g_tok, g_cnt = tok.cpu().numpy(), cnt.cpu().numpy()
-    # descriptors carry fp32 rounding: a differing block must sit within 1e-3 of the cutoff
-    for s in range(2):
-        for h in range(4):
-            gb = np.unique(g_tok[s, h, : g_cnt[s, h]] // L)
-            ob = np.unique(o_tok[s, h, : o_cnt[s, h]] // L)
-            d = np.setxor1d(gb, ob)
-            cut = np.sort(o_bs[s, h])[::-1][top - 1]
-            assert np.all(np.abs(o_bs[s, h][d] - cut) <= 1e-3 * abs(cut))
+    _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, p["T"], win,
+                  top, "describe+select")
 
 
 def test_quantize_matches_oracle_bit_exact(crs, cuda_dev):

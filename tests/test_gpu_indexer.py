@@ -17,14 +17,18 @@ def _np(t):
 def _check_rows(g_idx, g_cnt, qd, wd, Kd, key_base, n_vis, rows, topk, what):
     o_idx, o_cnt, o_cut, _ = oracle.indexer_topk(qd[rows], wd[rows], Kd, key_base[rows],
                                                  n_vis[rows], topk)
-    ndiff = 0
+    ndiff, worst = 0, 0.0
     for j, r in enumerate(rows):
         kb, nv = int(key_base[r]), int(n_vis[r])
         Kr = Kd[kb:kb + nv]
         sc = lambda pos: oracle.indexer_score(qd[r], wd[r], Kr[pos])
         bd = lambda pos: indexer_abs_bound(qd[r], wd[r], Kr[pos])
-        ndiff += check_topk_row(g_idx[r], g_cnt[r], o_idx[j], o_cnt[j], o_cut[j], sc, bd,
+        nd, wg = check_topk_row(g_idx[r], g_cnt[r], o_idx[j], o_cnt[j], o_cut[j], sc, bd,
                                 what=f"{what} row {r}")
+        ndiff += nd
+        worst = max(worst, wg)
+    print(f"{what}: {len(rows)} rows, {ndiff} differing positions, largest relative gap to the "
+          f"cutoff {worst:.3e}")
     return ndiff
 
 

@@ -158,3 +158,32 @@ def test_lsh_rejects_bad_args(crs, cuda_dev):
     R = torch.zeros(1, 1, 7, 8, device=cuda_dev)
     with pytest.raises(crs.CrsError):
         crs.lsh_route(X, R, 16)
+
+
+@pytest.mark.parametrize("n,chunk,rounds,nb,causal,no_self,vl_frac", [
+    (700, 64, 3, 16, 1, 0, 0.9),
+    (333, 128, 1, 8, 1, 1, 1.0),      # n < 3 chunks, ragged last chunk
+    (1024, 32, 8, 64, 0, 1, 0.95),    # 8 rounds, not causal
+])
+def test_lsh_candidates_csr_matches_oracle(crs, cuda_dev, n, chunk, rounds, nb, causal, no_self, vl_frac):
+    """The CSR export of U(i) (PaperTrace 2.1.1 §4 index tensors) equals the oracle's
+    candidate set for every row, bit for bit."""
+    case = workloads.lsh_clustered_case(B=2, H=2, n=n, n_rounds=rounds, n_buckets=nb, chunk=chunk,
+                                        pad_frac=1.0 - vl_frac, seed=n + rounds, device=cuda_dev)
+    bucket, perm, inv, ob, op, oi = _route_and_check(crs, case)
+    row_ptr, col = crs.lsh_candidates_csr(bucket, perm, inv, case["valid_len"], chunk=chunk,
+                                          causal=causal, no_self=no_self)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    rp, cl = row_ptr.cpu().numpy(), col.cpu().numpy()
+    vl = case["valid_len"].cpu().numpy()
+    B, H = 2, 2
+    assert rp[0] == 0 and (np.diff(rp) >= 0).all()
+    for b in range(B):
+        for h in range(H):
+            for i in range(n):
+                row = (b * H + h) * n + i
+                want = oracle.lsh_candidates(ob[b, h], op[b, h], oi[b, h], i, chunk, causal, no_self,
+                                             int(vl[b]))
+                got = cl[rp[row]:rp[row + 1]]
+                assert np.array_equal(got, want), f"(b={b}, h={h}, i={i}): {got[:8]} vs {want[:8]}"

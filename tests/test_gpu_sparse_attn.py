@@ -24,7 +24,7 @@ def _random_lists(rng, n_rows, n_lists, max_idx, n_keys, fill):
 
 
 def _run(crs, dev, n_rows, n_q, n_kv, max_idx, n_tok, n_lists, seed, kv_base=None, fill=None,
-         per_row_tokens=None):
+         per_row_tokens=None, masks=False):
     rng = np.random.default_rng(seed)
     g = torch.Generator(device=dev).manual_seed(seed)
     Q = torch.randn(n_rows, n_q, 128, generator=g, device=dev).to(torch.bfloat16)
@@ -34,10 +34,17 @@ def _run(crs, dev, n_rows, n_q, n_kv, max_idx, n_tok, n_lists, seed, kv_base=Non
     It = torch.from_numpy(I).to(dev)
     kb = None if kv_base is None else torch.from_numpy(kv_base).to(dev)
     lse = torch.empty(n_rows, n_q, device=dev)
-    O, _ = crs.sparse_attn(Q, K, V, It, kv_base=kb, lse=lse)
+    key_valid = q_pos = None
+    if masks:
+        key_valid = rng.random(n_tok) > 0.25
+        q_pos = rng.integers(0, per_row_tokens or n_tok, n_rows).astype(np.int32)
+    O, _ = crs.sparse_attn(Q, K, V, It, kv_base=kb, lse=lse,
+                           key_valid=None if key_valid is None else torch.from_numpy(key_valid).to(dev),
+                           q_pos=None if q_pos is None else torch.from_numpy(q_pos).to(dev))
     torch.cuda.synchronize()
     assert crs.get_device_error() == 0
-    oO, olse = oracle.sparse_attn(_np(Q), _np(K), _np(V), I, kv_base=kv_base)
+    oO, olse = oracle.sparse_attn(_np(Q), _np(K), _np(V), I, kv_base=kv_base, key_valid=key_valid,
+                                  q_pos=q_pos)
     err = rel_err(_np(O), oO)
     assert err.max() <= TOL, f"max rel err {err.max():.3e}"
     gl = lse.cpu().numpy().astype(np.float64)
@@ -70,14 +77,34 @@ def test_per_kv_lists_and_splits(crs, cuda_dev, n_q, n_kv):
          seed=n_q + n_kv, fill=2560)
 
 
+@pytest.mark.parametrize("n_q,n_kv,n_lists", [(16, 1, 1), (32, 4, 4)])
+def test_causal_and_padding_masks(crs, cuda_dev, n_q, n_kv, n_lists):
+    """[P1] §1.1 Eq.(2): q_pos (causal limit per row) and key_valid (padding keys) cut
+    the listed entries; compared with the oracle applying the same masks."""
+    lens = [700, 2100, 333]
+    base = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+    _run(crs, cuda_dev, n_rows=3, n_q=n_q, n_kv=n_kv, max_idx=300, n_tok=sum(lens),
+         n_lists=n_lists, seed=40 + n_q, kv_base=base, per_row_tokens=min(lens), masks=True)
+    _run(crs, cuda_dev, n_rows=50, n_q=n_q, n_kv=n_kv, max_idx=1500, n_tok=4000,
+         n_lists=n_lists, seed=41 + n_q, masks=True)
+
+
 def test_out_of_range_index_is_flagged_and_skipped(crs, cuda_dev):
-    Q = torch.randn(2, 16, 128, device=cuda_dev).to(torch.bfloat16)
+    """Every entry is checked against K's token count (kv_base included): an entry
+    past the end, or below -1, sets CRS_DEVERR_INDEX and is skipped."""
+    Q = torch.randn(3, 16, 128, device=cuda_dev).to(torch.bfloat16)
     K = torch.randn(100, 1, 128, device=cuda_dev).to(torch.bfloat16)
     V = torch.randn(100, 1, 128, device=cuda_dev).to(torch.bfloat16)
-    I = torch.tensor([[[3, 5, 150]], [[1, 2, -1]]], dtype=torch.int32, device=cuda_dev)
+    I = torch.tensor([[[3, 5, 150]], [[1, 2, -1]], [[0, 39, 40]]], dtype=torch.int32, device=cuda_dev)
+    kb = torch.tensor([0, 0, 60], dtype=torch.int64, device=cuda_dev)
     crs.get_device_error()
-    O, _ = crs.sparse_attn(Q, K, V, I, n_keys=100)
+    O, _ = crs.sparse_attn(Q, K, V, I, kv_base=kb)
     assert crs.get_device_error() & crs.DEVERR_INDEX
-    Ir = np.array([[[3, 5, -1]], [[1, 2, -1]]], np.int32)
-    oO, _ = oracle.sparse_attn(_np(Q), _np(K), _np(V), Ir)
+    Ir = np.array([[[3, 5, -1]], [[1, 2, -1]], [[0, 39, -1]]], np.int32)
+    oO, _ = oracle.sparse_attn(_np(Q), _np(K), _np(V), Ir, kv_base=np.array([0, 0, 60]))
     assert rel_err(_np(O), oO).max() <= TOL
+    I2 = torch.tensor([[[3, -7, 4]]], dtype=torch.int32, device=cuda_dev)
+    O2, _ = crs.sparse_attn(Q[:1], K, V, I2)
+    assert crs.get_device_error() & crs.DEVERR_INDEX
+    oO2, _ = oracle.sparse_attn(_np(Q[:1]), _np(K), _np(V), np.array([[[3, -1, 4]]], np.int32))
+    assert rel_err(_np(O2), oO2).max() <= TOL
