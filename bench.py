@@ -123,12 +123,27 @@ class LshWorkload(Workload):
         self._run(self.d_in)
         self.h_out.copy_(self.O, non_blocking=True)
 
+    def step_bytes(self):
+        """Algorithmic bytes of a whole step: per (batch, head) Q and V once per round,
+        O once and the routing integers of every round."""
+        p = self.p
+        B, H, n, d, R = p["B"], p["H"], p["n"], p["d"], p["n_rounds"]
+        esz = 2 if self.dtype == "bf16" else 4
+        return B * H * (R * n * d * esz * 2 + n * d * esz + R * n * 4 * 3)
+
+    def cpu_sample(self, frac):
+        p = self.p
+        segs = max(1, int(round(p["B"] * p["H"] * frac)))
+        return cpu_sample_lsh(self.case, segs)
+
     def roofline_spec(self):
         p = self.p
         B, H, n, d, R, m = p["B"], p["H"], p["n"], p["d"], p["n_rounds"], p["chunk"]
         rect_flops = B * H * R * n * (2 * m) * d * 4          # QK^T and P.V over own+previous chunk
         esz = 2 if self.dtype == "bf16" else 4
-        attn_bytes = B * H * R * n * d * esz * 2 + B * H * R * n * (d + 1) * 4
+        # algorithmic bytes of the attention: Q (= K) and V read once per round, and the
+        # three int32 routing arrays (bucket, perm, inv_perm) of every round
+        attn_bytes = B * H * R * n * d * esz * 2 + B * H * R * n * 4 * 3
         return {
             "lsh_chunk_attn": [("alu", rect_flops / 1e12, "TFLOP/s"),
                                ("hbm", attn_bytes / 1e9, "GB/s")],
@@ -256,6 +271,7 @@ class PrefillWorkload(Workload):
         self.idx = torch.empty((n, k), dtype=torch.int32, device=dev)
         self.cnt = torch.empty((n,), dtype=torch.int32, device=dev)
         self.O = torch.empty(c["Q"].shape, dtype=torch.float32, device=dev)
+        self.q_pos = torch.arange(n, dtype=torch.int32, device=dev)     # causal limit of row t
         import ctypes
         ip = crs.IndexerParams(crs.CRS_IDX_PREFILL, n, 4, 64, k, 0)
         self.ws = torch.empty(max(1, int(crs.lib().crs_indexer_topk_workspace_size(ctypes.byref(ip)))),
@@ -270,7 +286,8 @@ class PrefillWorkload(Workload):
         k = self.p["topk"]
         self.crs.indexer_topk(src["q_idx"], src["w"], src["k_idx"], k, self.crs.CRS_IDX_PREFILL,
                               out=self.idx, count=self.cnt, workspace=self.ws)
-        self.crs.sparse_attn(src["Q"], src["K"], src["V"], self.idx.view(-1, 1, k), out=self.O)
+        self.crs.sparse_attn(src["Q"], src["K"], src["V"], self.idx.view(-1, 1, k), q_pos=self.q_pos,
+                             out=self.O)
 
     def step(self):
         self._run(self.c)
@@ -280,6 +297,9 @@ class PrefillWorkload(Workload):
             self.d_in[k2].copy_(h, non_blocking=True)
         self._run(self.d_in)
         self.h_out.copy_(self.O, non_blocking=True)
+
+    def cpu_sample(self, frac):
+        return cpu_sample_prefill(self.c, max(16, int(512 * frac)))
 
     def roofline_spec(self):
         n, k = self.p["n"], self.p["topk"]
@@ -311,11 +331,12 @@ class DecodeWorkload(Workload):
         self.cnt = torch.empty((ns,), dtype=torch.int32, device=dev)
         self.O = torch.empty(c["Q"].shape, dtype=torch.float32, device=dev)
         self.kv_base = c["offsets"][:-1].contiguous()
+        self.q_pos = (c["ctx"] - 1).to(torch.int32).contiguous()     # row s sees [0, ctx_s)
         import ctypes
         ip = crs.IndexerParams(crs.CRS_IDX_DECODE, ns, 4, 64, k, 131072)
         self.ws = torch.empty(int(crs.lib().crs_indexer_topk_workspace_size(ctypes.byref(ip))),
                               dtype=torch.uint8, device=dev)
-        ap = crs.AttnParams(ns, 32, 8, 128, k, 1, 0, 0.0)
+        ap = crs.AttnParams(ns, 32, 8, 128, k, 1, int(c["offsets"][-1]), 0.0)
         self.ws2 = torch.empty(max(1, int(crs.lib().crs_sparse_attn_workspace_size(ctypes.byref(ap)))),
                                dtype=torch.uint8, device=dev)
         # end to end: the per-step inputs are the new queries (caches stay resident)
@@ -332,7 +353,7 @@ class DecodeWorkload(Workload):
                               k_offsets=self.c["offsets"], max_keys=131072, out=self.idx,
                               count=self.cnt, workspace=self.ws)
         self.crs.sparse_attn(Q, self.c["K"], self.c["V"], self.idx.view(-1, 1, k),
-                             kv_base=self.kv_base, out=self.O, workspace=self.ws2)
+                             kv_base=self.kv_base, q_pos=self.q_pos, out=self.O, workspace=self.ws2)
 
     def step(self):
         self._run(self.c["q_idx"], self.c["w"], self.c["Q"])
@@ -342,6 +363,9 @@ class DecodeWorkload(Workload):
             self.d_in[k2].copy_(h, non_blocking=True)
         self._run(self.d_in["q_idx"], self.d_in["w"], self.d_in["Q"])
         self.h_out.copy_(self.O, non_blocking=True)
+
+    def cpu_sample(self, frac):
+        return cpu_sample_decode(self.c, max(1, int(self.p["n_seq"] * frac)))
 
     def roofline_spec(self):
         ns, k = self.p["n_seq"], self.p["topk"]
@@ -358,6 +382,7 @@ class DecodeHisaWorkload(DecodeWorkload):
     64-key blocks (a cache, built once per filled block), 128 kept blocks per row, the
     token indexer on their keys and the open block, then the gather attention."""
     BLK, TOP_BLOCKS = 64, 128
+    cpu_sample = None
 
     def __init__(self, crs, dev):
         super().__init__(crs, dev)
@@ -376,7 +401,7 @@ class DecodeHisaWorkload(DecodeWorkload):
                            self.TOP_BLOCKS, 131072, out_blocks=self.blocks, out=self.idx, count=self.cnt,
                            workspace=self.ws)
         self.crs.sparse_attn(Q, self.c["K"], self.c["V"], self.idx.view(-1, 1, k),
-                             kv_base=self.kv_base, out=self.O, workspace=self.ws2)
+                             kv_base=self.kv_base, q_pos=self.q_pos, out=self.O, workspace=self.ws2)
 
     def roofline_spec(self):
         ns, k = self.p["n_seq"], self.p["topk"]
@@ -410,6 +435,7 @@ class BlockWorkload(Workload):
         self.Kf = c["K"].view(p["n_seq"] * p["T"], p["n_kv_heads"], p["D"])
         self.Vf = c["V"].view(p["n_seq"] * p["T"], p["n_kv_heads"], p["D"])
         self.kv_base = torch.arange(p["n_seq"], device=dev, dtype=torch.int64) * p["T"]
+        self.q_pos = torch.full((p["n_seq"],), p["T"] - 1, dtype=torch.int32, device=dev)
         import ctypes
         bp = crs.BlockSelParams(crs.BlockParams(p["n_seq"], p["n_kv_heads"], p["T"], p["D"], p["L"],
                                                 p["rank"], 0, p["T"] // p["L"]),
@@ -417,7 +443,7 @@ class BlockWorkload(Workload):
         self.ws = torch.empty(int(crs.lib().crs_block_select_workspace_size(ctypes.byref(bp))),
                               dtype=torch.uint8, device=dev)
         ap = crs.AttnParams(p["n_seq"], p["n_q_heads"], p["n_kv_heads"], p["D"], cap,
-                            p["n_kv_heads"], 0, 0.0)
+                            p["n_kv_heads"], p["n_seq"] * p["T"], 0.0)
         self.ws2 = torch.empty(max(1, int(crs.lib().crs_sparse_attn_workspace_size(ctypes.byref(ap)))),
                                dtype=torch.uint8, device=dev)
         self.h_in = {"Q": c["Q"].cpu().pin_memory()}
@@ -429,12 +455,15 @@ class BlockWorkload(Workload):
     def _build_cache(self):
         self.mu, self.xi = self.crs.block_describe(self.c["K"], self.p["L"], self.p["rank"])
 
+    def cpu_sample(self, frac):
+        return cpu_sample_block(self, max(1, int(self.p["n_seq"] * frac)))
+
     def _run(self, Q):
         p = self.p
         self.crs.block_select(Q, self.mu, self.xi, p["T"], p["L"], p["top_blocks"], p["window"],
                               tok=self.tok, count=self.cnt, workspace=self.ws)
-        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
-                             workspace=self.ws2)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, q_pos=self.q_pos,
+                             out=self.O, workspace=self.ws2)
 
     def step(self):
         self._run(self.c["Q"])
@@ -473,8 +502,8 @@ class BlockFp4Workload(BlockWorkload):
         p = self.p
         self.crs.block_select_fp4(Q, self.mu16, self.xi4, self.xs, p["T"], p["L"], p["top_blocks"],
                                   p["window"], tok=self.tok, count=self.cnt, workspace=self.ws)
-        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
-                             workspace=self.ws2)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, q_pos=self.q_pos,
+                             out=self.O, workspace=self.ws2)
 
     def roofline_spec(self):
         p = self.p
@@ -490,6 +519,7 @@ class BlockFp4Workload(BlockWorkload):
 class BlockQuestWorkload(BlockWorkload):
     """Baseline selector: Quest boxes (element-wise key min / max per block, bf16, 512 B
     per block) under the same selection rule, then the gather attention."""
+    cpu_sample = None
 
     def __init__(self, crs, dev):
         super().__init__(crs, dev)
@@ -502,8 +532,8 @@ class BlockQuestWorkload(BlockWorkload):
         p = self.p
         self.crs.block_select_quest(Q, self.kmin, self.kmax, p["T"], p["L"], p["top_blocks"], p["window"],
                                     tok=self.tok, count=self.cnt, workspace=self.ws)
-        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
-                             workspace=self.ws2)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, q_pos=self.q_pos,
+                             out=self.O, workspace=self.ws2)
 
     def roofline_spec(self):
         p = self.p
@@ -516,6 +546,7 @@ class BlockQuestWorkload(BlockWorkload):
 class BlockSubspaceWorkload(BlockWorkload):
     """COBS descriptors in a query subspace of s = 85 dims: fp32 mean (512 B) and four
     scaled eigenvectors of U^T Sigma U (4 x 85 x 4 B) per block."""
+    cpu_sample = None
     SD = 85
 
     def __init__(self, crs, dev):
@@ -538,8 +569,8 @@ class BlockSubspaceWorkload(BlockWorkload):
         p = self.p
         self.crs.block_select_ss(Q, self.U, self.mu, self.xi, p["T"], p["L"], p["top_blocks"], p["window"],
                                  tok=self.tok, count=self.cnt, workspace=self.ws)
-        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, out=self.O,
-                             workspace=self.ws2)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, q_pos=self.q_pos,
+                             out=self.O, workspace=self.ws2)
 
     def roofline_spec(self):
         p = self.p
@@ -552,6 +583,7 @@ class BlockSubspaceWorkload(BlockWorkload):
 
 class BlockMeanPoolWorkload(BlockWorkload):
     """Baseline selector: the block mean alone (first-order score, fp32, 512 B per block)."""
+    cpu_sample = None
 
     def __init__(self, crs, dev):
         super().__init__(crs, dev)
@@ -731,10 +763,30 @@ def measure(crs, wl, steps, warmup, flush_buf, dist_on, peaks, e2e=True):
 
 
 # ------------------------------------------------------------- CPU baseline --
-def cpu_baseline_lsh(case, n_segments=16):
-    """The oracle on a bounded sample: n_segments of the B*H (batch, head)
-    segments, each routed (hash + sort, all rounds) and attended for all n
-    query rows.  Returns (tokens/s scaled to the metric, seconds, sample text)."""
+# The oracle (plain C, fp64, OpenMP over rows), timed as it stands on the host
+# cores on a bounded sample of the same workload.  Only the oracle calls are
+# timed; copying inputs to the host (and, for the gather stages, collecting the
+# K/V rows a list names) happens outside the timed spans.  Each function returns
+# (units of the workload's metric covered by the sample, seconds, sample text).
+def _tnp(t):
+    import numpy as np
+    return t.detach().cpu().double().numpy().astype(np.float64)
+
+
+class _Clock:
+    def __init__(self):
+        self.s = 0.0
+
+    def __call__(self, fn, *a, **k):
+        t0 = time.perf_counter()
+        r = fn(*a, **k)
+        self.s += time.perf_counter() - t0
+        return r
+
+
+def cpu_sample_lsh(case, n_segments=16):
+    """n_segments of the B*H (batch, head) segments, each routed (hash + sort, all
+    rounds) and attended for all n query rows."""
     import numpy as np
 
     import oracle
@@ -745,18 +797,116 @@ def cpu_baseline_lsh(case, n_segments=16):
     R = case["R"].cpu().numpy()
     vl = case["valid_len"].cpu().numpy()
     segs = [(s // H, s % H) for s in range(min(n_segments, B * H))]
-    t0 = time.perf_counter()
+    clk = _Clock()
     for b, h in segs:
         x = QK[b:b + 1, h:h + 1]
-        bk = oracle.lsh_hash(x, R[h:h + 1], p["n_buckets"])
-        pm, ip = oracle.lsh_sort(bk)
-        oracle.lsh_attn(x.astype(np.float64), V[b:b + 1, h:h + 1], bk, pm, ip, vl[b:b + 1],
-                        p["chunk"], p["causal"], p["no_self"], p["key_norm"], p["scale"])
-    dt = time.perf_counter() - t0
+        bk = clk(oracle.lsh_hash, x, R[h:h + 1], p["n_buckets"])
+        pm, ip = clk(oracle.lsh_sort, bk)
+        clk(oracle.lsh_attn, x.astype(np.float64), V[b:b + 1, h:h + 1], bk, pm, ip, vl[b:b + 1],
+            p["chunk"], p["causal"], p["no_self"], p["key_norm"], p["scale"])
     tokens = B * n * len(segs) / (B * H)      # a (b, h) segment is 1/(B*H) of a step's work
     sample = (f"{len(segs)} of {B*H} (batch, head) segments: hash + sort + LSH attention for all "
               f"{n} query rows and {p['n_rounds']} rounds, scaled by segments/(B*H)")
+    return tokens, clk.s, sample
+
+
+def cpu_baseline_lsh(case, n_segments=16):
+    tokens, dt, sample = cpu_sample_lsh(case, n_segments)
     return tokens / dt, dt, sample
+
+
+def cpu_sample_prefill(c, n_rows=512):
+    """n_rows query rows spread evenly over the sequence (row t scores its t + 1 keys),
+    each: indexer top-k, then gather attention of the 16 heads over the oracle's own
+    list.  Tokens covered = rows."""
+    import numpy as np
+
+    import oracle
+    p = c["params"]
+    n, k = p["n"], p["topk"]
+    rows = ((np.arange(n_rows) + 0.5) * n / n_rows).astype(np.int64)
+    qd, wd, Kd = _tnp(c["q_idx"][rows]), _tnp(c["w"][rows]), _tnp(c["k_idx"])
+    Q, K, V = _tnp(c["Q"][rows]), _tnp(c["K"]), _tnp(c["V"])
+    clk = _Clock()
+    idx, cnt, _, _ = clk(oracle.indexer_topk, qd, wd, Kd, np.zeros(n_rows, np.int64),
+                         (rows + 1).astype(np.int32), k)
+    clk(oracle.sparse_attn, Q, K, V, idx[:, None, :], q_pos=rows.astype(np.int32))
+    return float(n_rows), clk.s, (f"{n_rows} of {n} query rows evenly spaced (indexer top-{k} over "
+                                  f"keys 0..t, then {p['n_q_heads']}-head attention over the list)")
+
+
+def cpu_sample_decode(c, n_seq=64):
+    """n_seq of the sequences: indexer top-k over the whole context, then the GQA
+    attention over the oracle's list (the listed K/V rows collected on the device,
+    untimed).  Steps covered = n_seq / sequences."""
+    import numpy as np
+
+    import oracle
+    p = c["params"]
+    S, k = p["n_seq"], p["topk"]
+    off = c["offsets"].cpu().numpy()
+    clk = _Clock()
+    for s in range(min(n_seq, S)):
+        Kr = _tnp(c["k_idx"][off[s]:off[s + 1]])
+        idx, cnt, _, _ = clk(oracle.indexer_topk, _tnp(c["q_idx"][s:s + 1]), _tnp(c["w"][s:s + 1]), Kr,
+                             np.zeros(1, np.int64), np.array([Kr.shape[0]], np.int32), k)
+        lst = torch.as_tensor(off[s] + idx[0, : cnt[0]], dtype=torch.int64, device=c["K"].device)
+        Kc, Vc = _tnp(c["K"][lst]), _tnp(c["V"][lst])
+        I = np.arange(int(cnt[0]), dtype=np.int32)[None, None]
+        clk(oracle.sparse_attn, _tnp(c["Q"][s:s + 1]), Kc, Vc, I)
+    m = min(n_seq, S)
+    return m / S, clk.s, (f"{m} of {S} sequences (indexer top-{k} over the context, then "
+                          f"{p['n_q_heads']}/{p['n_kv_heads']} GQA attention), scaled by sequences/{S}")
+
+
+def cpu_sample_block(wl, n_seq=32):
+    """n_seq of the sequences: block selection on the step's descriptors (fp32, or the
+    dequantised FP4 ones), then the attention over each KV head's token list (the listed
+    rows collected on the device, untimed).  Steps covered = n_seq / sequences."""
+    import numpy as np
+
+    import oracle
+    c, p = wl.c, wl.p
+    S, T, L, nkv = p["n_seq"], p["T"], p["L"], p["n_kv_heads"]
+    G = p["n_q_heads"] // nkv
+    clk = _Clock()
+    m = min(n_seq, S)
+    for s in range(m):
+        if hasattr(wl, "xi4"):
+            mu = _tnp(wl.mu16[s:s + 1])
+            xi = oracle.fp4_dequantize(wl.xi4[s:s + 1].cpu().numpy(), wl.xs[s:s + 1].cpu().numpy())
+        else:
+            mu, xi = _tnp(wl.mu[s:s + 1]), _tnp(wl.xi[s:s + 1])
+        Qs = _tnp(c["Q"][s:s + 1])
+        tok, cnt, _, _ = clk(oracle.block_select, Qs, mu, xi, T, L, p["top_blocks"], p["window"])
+        for h in range(nkv):
+            lst = torch.as_tensor(tok[0, h, : cnt[0, h]], dtype=torch.int64, device=c["K"].device)
+            Kc = _tnp(c["K"][s, lst, h])[:, None, :]
+            Vc = _tnp(c["V"][s, lst, h])[:, None, :]
+            I = np.arange(int(cnt[0, h]), dtype=np.int32)[None, None]
+            clk(oracle.sparse_attn, Qs[:, h * G:(h + 1) * G], Kc, Vc, I)
+    kind = "FP4 (dequantised)" if hasattr(wl, "xi4") else "fp32"
+    return m / S, clk.s, (f"{m} of {S} sequences (block selection on {kind} descriptors, then "
+                          f"attention over each KV head's list), scaled by sequences/{S}")
+
+
+def cpu_baseline(wl, single_thread_fraction):
+    """The oracle on all host cores (the workload's default sample) and on one core
+    (a smaller sample): value in the workload's unit, cores, per-core value."""
+    import oracle
+    fn = getattr(wl, "cpu_sample", None)
+    if fn is None:
+        return None
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    units, dt, sample = fn(1.0)
+    oracle.set_threads(1)
+    u1, dt1, sample1 = fn(single_thread_fraction)
+    oracle.set_threads(cores)
+    return {"value": round(units / dt, 3), "unit": wl.unit, "cores": cores, "kind": "oracle",
+            "sample": sample, "seconds": round(dt, 3),
+            "per_core": {"value": round(u1 / dt1, 3), "unit": wl.unit, "cores": 1, "sample": sample1,
+                         "seconds": round(dt1, 3)}}
 
 
 def _omp_threads():
@@ -866,6 +1016,8 @@ def main():
                                         "unit": w2.unit, "h2d_bytes_per_step": w2.h2d,
                                         "d2h_bytes_per_step": w2.d2h},
                                 "gpu_launches": r2["gpu_launches"]}
+                if not args.no_cpu_baseline:
+                    extras[name]["cpu_baseline"] = cpu_baseline(w2, 1.0 / 8)
                 if name == "block":
                     torch.cuda.synchronize()
                     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -885,10 +1037,13 @@ def main():
                 extras[name] = {"error": f"{type(e).__name__}: {e}"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "lsh":
-        v, dt, sample = cpu_baseline_lsh(wl.case)
-        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": _omp_threads(), "kind": "oracle",
-               "sample": sample, "seconds": round(dt, 3)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, 1.0 / 16)
+    step_rl = None
+    if hasattr(wl, "step_bytes"):
+        gbs = wl.step_bytes() / (tot_ms / args.steps / 1e3) / 1e9
+        step_rl = {"bound": "hbm", "bytes_per_step": wl.step_bytes(), "achieved": round(gbs, 3),
+                   "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}
 
     if rank == 0:
         p = getattr(wl, "p", {})
@@ -904,6 +1059,7 @@ def main():
                     "d2h_bytes_per_step": wl.d2h},
             "gpu_launches": res["gpu_launches"],
             "roofline": res["roofline"],
+            "step_roofline": step_rl,
             "stages_ms": res["stages_ms"],
             "cpu_baseline": cpu,
             "clocks": clocks,

@@ -43,6 +43,8 @@ def _lib():
         path = _build.build()
         lib = ctypes.CDLL(path)
         I, L, D = ctypes.c_int, ctypes.c_long, ctypes.c_double
+        lib.oracle_set_num_threads.argtypes = [I]
+        lib.oracle_max_threads.restype = I
         lib.oracle_lsh_hash.argtypes = [I, I, I, I, I, I, _f32p, _f32p, _i32p]
         lib.oracle_lsh_margin.argtypes = [I, I, I, I, I, I, _f32p, _f32p, _f64p]
         lib.oracle_lsh_sort.argtypes = [I, I, _i32p, _i32p, _i32p]
@@ -89,9 +91,13 @@ def _p(a, ctype):
 
 
 def set_threads(n: Optional[int]) -> None:
-    """Number of OpenMP threads used by later calls (None: library default)."""
-    if n is not None:
-        os.environ["OMP_NUM_THREADS"] = str(int(n))
+    """Number of OpenMP threads used by later calls (None: every core)."""
+    _lib().oracle_set_num_threads(int(n) if n is not None else (os.cpu_count() or 1))
+
+
+def threads() -> int:
+    """Number of OpenMP threads later calls use."""
+    return int(_lib().oracle_max_threads())
 
 
 # ---------------------------------------------------------------- LSH --

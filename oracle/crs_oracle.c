@@ -15,11 +15,17 @@
  *   [P5] "COBS 阅读笔记: 块稀疏注意力的选择器到底漏掉了什么"
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
 #define OAPI __attribute__((visibility("default")))
+
+/* Threads used by later calls (rows are split across them; no operation order
+ * depends on the count), and the current count. */
+OAPI void oracle_set_num_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+OAPI int oracle_max_threads(void) { return omp_get_max_threads(); }
 
 /* ======================================================================
  * O1  LSH bucket id.  [P1] §2.1 Eq.(4): u = x R with R in R^{d x b/2};
