@@ -243,6 +243,15 @@ def get_device_diag(stream=None) -> list:
     return [int(x) for x in buf]
 
 
+_sig("crs_debug_force_wait_timeout", ctypes.c_int, [ctypes.c_int])
+
+
+def debug_force_wait_timeout(on: bool) -> None:
+    """Make the first bounded wait of the tensor-core LSH kernels give up at once
+    (failure-path test switch; see include/crs.h)."""
+    _check("crs_debug_force_wait_timeout", _lib.crs_debug_force_wait_timeout(1 if on else 0))
+
+
 def profile_set(enabled: bool) -> None:
     """Turn per-launch CUDA-event timing on or off (launch counting is always on)."""
     _check("crs_profile_set", _lib.crs_profile_set(1 if enabled else 0))

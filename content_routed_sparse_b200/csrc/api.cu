@@ -114,6 +114,12 @@ extern "C" int crs_get_device_diag(void *stream, uint32_t *out, int n) {
     return CRS_OK;
 }
 
+extern "C" int crs_debug_force_wait_timeout(int on) {
+    const uint32_t v = on ? 1u : 0u;
+    CRS_TRY_CUDA(cudaMemcpyToSymbol(crs::g_force_wait_timeout, &v, sizeof(v)));
+    return CRS_OK;
+}
+
 extern "C" int crs_get_device_error(void *stream, uint32_t *flags) {
     if (!flags) return CRS_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

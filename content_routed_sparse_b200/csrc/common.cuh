@@ -15,6 +15,11 @@ __device__ uint32_t g_device_error = 0;
 
 __device__ __forceinline__ void raise_error(uint32_t bit) { atomicOr(&g_device_error, bit); }
 
+// Debug switch (crs_debug_force_wait_timeout): while non-zero, the bounded waits
+// marked as forceable give up at once, so a test can drive the timeout path
+// (error bit, diagnostic record, drain, early return) without a stuck barrier.
+__device__ uint32_t g_force_wait_timeout = 0;
+
 // Diagnostic record of the first failure a kernel reports about itself:
 // [0] = kernel id + 1 (0: none), [1] = where (kernel-defined site), [2..4] =
 // blockIdx.x/y/z, [5..] = kernel-defined values.  Read by crs_get_device_diag.

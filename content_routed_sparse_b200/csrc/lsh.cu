@@ -474,16 +474,9 @@ lsh_chunk_attn_kernel(const T *__restrict__ QK, const T *__restrict__ V,
 // Padded positions and queries with no edge in any round give 0 / -inf.
 // --------------------------------------------------------------------------
 template <int DH>
-__global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
-                                   const int32_t *__restrict__ valid_len, float *__restrict__ O,
-                                   float *__restrict__ lse_out, int BH, int H, int n, int rounds) {
-    constexpr int G4 = DH / 4;                  // float4 groups per row
-    const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gt >= (long long)BH * n * G4) return;
-    const int g = (int)(gt % G4);
-    const long long rowi = gt / G4;
-    const int bh = (int)(rowi / n), pos = (int)(rowi - (long long)bh * n);
-    const int vl = valid_len ? valid_len[bh / H] : n;
+__device__ __forceinline__ void lsh_merge_rounds(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
+                                                 float *__restrict__ O, float *__restrict__ lse_out, int BH,
+                                                 int n, int rounds, int bh, int pos, int g, bool padded) {
     // every round's lse and partial output are requested before any is used
     float l[kMaxRounds];
     float4 ov[kMaxRounds];
@@ -500,7 +493,7 @@ __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *
         mx = fmaxf(mx, l[r]);
     }
     float4 *o = reinterpret_cast<float4 *>(O + ((size_t)bh * n + pos) * DH) + g;
-    if (pos >= vl || mx == -INFINITY) {
+    if (padded || mx == -INFINITY) {
         *o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (lse_out && g == 0) lse_out[(size_t)bh * n + pos] = -INFINITY;
         return;
@@ -523,6 +516,55 @@ __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *
     }
     *o = acc;
     if (lse_out && g == 0) lse_out[(size_t)bh * n + pos] = LSE;
+}
+
+template <int DH>
+__global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
+                                   const int32_t *__restrict__ valid_len, float *__restrict__ O,
+                                   float *__restrict__ lse_out, int BH, int H, int n, int rounds) {
+    constexpr int G4 = DH / 4;                  // float4 groups per row
+    const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gt >= (long long)BH * n * G4) return;
+    const int g = (int)(gt % G4);
+    const long long rowi = gt / G4;
+    const int bh = (int)(rowi / n), pos = (int)(rowi - (long long)bh * n);
+    const int vl = valid_len ? valid_len[bh / H] : n;
+    lsh_merge_rounds<DH>(o_ws, lse_ws, O, lse_out, BH, n, rounds, bh, pos, g, pos >= vl);
+}
+
+// K4 after the fixed-shift round accumulation of the tensor-core attention: O holds
+// sum_j 2^(s_ij - M_i) v_j over the union of the rounds' candidates, acc_L the matching
+// sum of weights, acc_M the shift M_i (log2 units); O /= L and lse = (M_i + log2 L) ln 2.
+// Rows the attention kept in the per-round form (acc_M = +inf) are merged as above.
+template <int DH>
+__global__ void lsh_finish_kernel(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
+                                  const float *__restrict__ acc_L, const float *__restrict__ acc_M,
+                                  const int32_t *__restrict__ valid_len, float *__restrict__ O,
+                                  float *__restrict__ lse_out, int BH, int H, int n, int rounds) {
+    constexpr int G4 = DH / 4;
+    const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gt >= (long long)BH * n * G4) return;
+    const int g = (int)(gt % G4);
+    const long long rowi = gt / G4;
+    const int bh = (int)(rowi / n), pos = (int)(rowi - (long long)bh * n);
+    const int vl = valid_len ? valid_len[bh / H] : n;
+    const float m = acc_M[rowi];
+    if (m == INFINITY) {
+        lsh_merge_rounds<DH>(o_ws, lse_ws, O, lse_out, BH, n, rounds, bh, pos, g, pos >= vl);
+        return;
+    }
+    const float L = acc_L[rowi];
+    float4 *o = reinterpret_cast<float4 *>(O + (size_t)rowi * DH) + g;
+    if (pos >= vl || !(L > 0.0f)) {
+        *o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (lse_out && g == 0) lse_out[rowi] = -INFINITY;
+        return;
+    }
+    const float inv = 1.0f / L;
+    float4 v = *o;
+    v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+    *o = v;
+    if (lse_out && g == 0) lse_out[rowi] = (m + log2f(L)) * 0.6931471805599453f;
 }
 
 // ------------------------------------------------------------ host side --
@@ -556,7 +598,18 @@ extern "C" int crs_lsh_route(const crs_lsh_params *p, const void *X, const float
     const size_t smem = ((size_t)p->d * half + (size_t)kHashTok * (p->d + 1)) * sizeof(float);
     if (smem > 200 * 1024) return CRS_ERR_UNSUPPORTED;
     dim3 grid(ceil_div(p->n, kHashTok), p->n_rounds, p->B * p->H);
-    if (p->d == 64 && (half == 32 || half == 8)) {
+    if (p->dtype == CRS_BF16 && p->d == kHtD && half == kHtHalf && p->n_rounds <= 4) {
+        // tensor-core filter with the exact chain as fallback (identical bucket ids)
+        const int N = p->n_rounds * kHtHalf;
+        const size_t hsm = ht_smem_bytes(N) + 1024;
+        CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_hash_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)hsm));
+        const int tpc = ht_tiles_per_cta(p->n, p->B * p->H);
+        dim3 gh(ceil_div(ceil_div(p->n, kHtM), tpc), p->B * p->H);
+        ProfScope _ps(K_LSH_HASH, s);
+        lsh_hash_tc_kernel<<<gh, kHtThreads, hsm, s>>>(static_cast<const __nv_bfloat16 *>(X), R, bucket,
+                                                       p->H, p->n, p->n_rounds, tpc);
+    } else if (p->d == 64 && (half == 32 || half == 8)) {
         // specialised kernel: one CTA per 128 tokens covers every round
         dim3 g2(ceil_div(p->n, kHashTok), 1, p->B * p->H);
         ProfScope _ps(K_LSH_HASH, s);
@@ -612,7 +665,9 @@ extern "C" size_t crs_lsh_attn_workspace_size(const crs_lsh_attn_params *a) {
     if (!a || validate_lsh(&a->p)) return 0;
     const crs_lsh_params &p = a->p;
     const size_t rows = (size_t)p.n_rounds * p.B * p.H * p.n;
-    return align256(rows * p.d * sizeof(float)) + align256(rows * sizeof(float));
+    // per-round (o_r, lse_r), then the accumulated weight sums and shifts of each row
+    return align256(rows * p.d * sizeof(float)) + align256(rows * sizeof(float)) +
+           2 * align256((size_t)p.B * p.H * p.n * sizeof(float));
 }
 
 namespace crs {
@@ -620,7 +675,7 @@ template <typename T, int DH>
 static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const void *V,
                            const int32_t *bucket, const int32_t *perm, const int32_t *inv_perm,
                            const int32_t *valid_len, void *O, float *lse, float *o_ws,
-                           float *lse_ws, cudaStream_t s) {
+                           float *lse_ws, float *acc_L, float *acc_M, cudaStream_t s) {
     const crs_lsh_params &p = a->p;
     bool tc_done = false;
     if constexpr (std::is_same<T, __nv_bfloat16>::value && DH == kTcD) {
@@ -633,14 +688,33 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
                                               cudaFuncAttributePreferredSharedMemoryCarveout,
                                               (int)cudaSharedmemCarveoutMaxShared));
             dim3 grid(ceil_div(p.n, kTcM), p.n_rounds, p.B * p.H);
+            // normalised keys: the rounds accumulate into O with a fixed shift per row
+            const bool acc = a->key_norm != 0;
+            const size_t nrow = (size_t)p.B * p.H * p.n;
+            if (acc) {
+                CRS_TRY_CUDA(cudaMemsetAsync(O, 0, nrow * DH * sizeof(float), s));
+                CRS_TRY_CUDA(cudaMemsetAsync(acc_L, 0, 2 * align256(nrow * sizeof(float)), s));
+            }
             {
                 ProfScope _ps(K_LSH_ATTN_TC, s);
                 lsh_chunk_attn_tc_kernel<<<grid, kTcThreads, smem, s>>>(
                     static_cast<const __nv_bfloat16 *>(QK), static_cast<const __nv_bfloat16 *>(V),
-                    bucket, perm, inv_perm, valid_len, o_ws, lse_ws, p.H, p.n, p.n_rounds,
+                    bucket, perm, inv_perm, valid_len, o_ws, lse_ws, acc ? static_cast<float *>(O) : nullptr,
+                    acc ? acc_L : nullptr, acc ? acc_M : nullptr, p.H, p.n, p.n_rounds,
                     a->causal, a->no_self, a->key_norm, a->scale * 1.4426950408889634f);
             }
             CRS_CHECK_LAUNCH();
+            if (acc) {
+                const long long work = (long long)p.B * p.H * p.n * (DH / 4);
+                {
+                    ProfScope _ps(K_LSH_COMBINE, s);
+                    lsh_finish_kernel<DH><<<(unsigned)ceil_div_ll(work, 256), 256, 0, s>>>(
+                        o_ws, lse_ws, acc_L, acc_M, valid_len, static_cast<float *>(O), lse, p.B * p.H, p.H,
+                        p.n, p.n_rounds);
+                }
+                CRS_CHECK_LAUNCH();
+                return CRS_OK;
+            }
             tc_done = true;
         }
     }
@@ -691,20 +765,23 @@ extern "C" int crs_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const 
     float *o_ws = static_cast<float *>(ws);
     float *lse_ws = reinterpret_cast<float *>(static_cast<char *>(ws) +
                                               align256(rows * p.d * sizeof(float)));
+    float *acc_L = reinterpret_cast<float *>(reinterpret_cast<char *>(lse_ws) + align256(rows * sizeof(float)));
+    float *acc_M = reinterpret_cast<float *>(reinterpret_cast<char *>(acc_L) +
+                                             align256((size_t)p.B * p.H * p.n * sizeof(float)));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p.d == 64) {
         if (p.dtype == CRS_F32)
             return launch_lsh_attn<float, 64>(a, QK, V, bucket, perm, inv_perm, valid_len, O, lse,
-                                              o_ws, lse_ws, s);
+                                              o_ws, lse_ws, acc_L, acc_M, s);
         return launch_lsh_attn<__nv_bfloat16, 64>(a, QK, V, bucket, perm, inv_perm, valid_len, O,
-                                                  lse, o_ws, lse_ws, s);
+                                                  lse, o_ws, lse_ws, acc_L, acc_M, s);
     }
     if (p.d == 32) {
         if (p.dtype == CRS_F32)
             return launch_lsh_attn<float, 32>(a, QK, V, bucket, perm, inv_perm, valid_len, O, lse,
-                                              o_ws, lse_ws, s);
+                                              o_ws, lse_ws, acc_L, acc_M, s);
         return launch_lsh_attn<__nv_bfloat16, 32>(a, QK, V, bucket, perm, inv_perm, valid_len, O,
-                                                  lse, o_ws, lse_ws, s);
+                                                  lse, o_ws, lse_ws, acc_L, acc_M, s);
     }
     return CRS_ERR_UNSUPPORTED;
 }

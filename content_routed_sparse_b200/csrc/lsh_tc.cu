@@ -49,6 +49,7 @@ constexpr int kBktBefore = -1;                  // absent slot before the sequen
 constexpr int kBktAfter = 0x7fffffff;           // absent slot after the sequence
 constexpr float kTcBoundMax = 48.0f;            // single pass while 2^(-2 bound) stays normal
 constexpr float kTcBoundMax16 = 14.0f;          // fp16 P while 2^(15 - 2 bound) stays fp16-normal
+constexpr float kTcAccBoundMax = 63.0f;         // fixed-shift round accumulation while 2^(-2 bound) is normal
 
 struct LshTcSmem {
     // K tile (rows = keys; rows 128..255 = Q tile) until S is computed, then
@@ -68,9 +69,16 @@ struct LshTcSmem {
     int kcode[kMaxRounds - 1][kTcN];    // earlier rounds: bucket * C1 + chunk + 1
     float kscale[kTcN];                 // scale * log2(e) / |k_j|
     float rowmax[2][kTcM];
+    float rbound[kTcM];                 // scale |q_i| in log2 units (normalised keys)
     uint64_t bar[3];
     uint32_t tmem_base;
 };
+
+// o[0..3] += (a, b, c, d) in global memory, one vector reduction (no return value)
+__device__ __forceinline__ void red_add_v4(float *o, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(o), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {   // 2^x, PTX ex2.approx (rel. err ~2^-22)
     float r;
@@ -362,7 +370,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
                          const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
                          const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
-                         float *__restrict__ o_ws, float *__restrict__ lse_ws, int H, int n,
+                         float *__restrict__ o_ws, float *__restrict__ lse_ws, float *__restrict__ acc_O,
+                         float *__restrict__ acc_L, float *__restrict__ acc_M, int H, int n,
                          int rounds, int causal, int no_self, int key_norm, float scale_log2) {
     extern __shared__ unsigned char lsh_tc_raw[];
     const uint32_t mis = smem_u32(lsh_tc_raw) & 1023u;
@@ -486,6 +495,7 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         if (j >= kTcM) {
             const float bound = sqrtf(ss) * fabsf(scale_log2);
             S.rowmax[1][j - kTcM] = bound;
+            S.rbound[j - kTcM] = bound;
             big = bound > kTcBoundMax;
             no16 = no16 || !(bound <= kTcBoundMax16);
         }
@@ -513,7 +523,7 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         }
         tc::commit(&S.bar[0]);
     }
-    bool ok_wait = tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 1);
+    bool ok_wait = tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 1, 10000u, true);
     if (__syncthreads_or(!ok_wait)) {
         tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 2);   // let the MMA drain
         goto teardown;
@@ -617,7 +627,37 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         uint32_t v[32];
         tc::tmem_ld32(trow + wg * 32, v);
         tc::tmem_ld_wait();
-        if (q.pos_i >= 0) {
+        // Round accumulation with a fixed shift (normalised keys): every logit of row i
+        // is at most bound_i = scale |q_i| (log2 units), the same value in every round,
+        // so the rounds' numerators sum_j 2^(s_ij - bound_i) v_j and denominators add up
+        // directly; with bound_i <= 63 no term leaves the fp32 normal range.  This
+        // round's terms were taken relative to M (bound - 15 for fp16 P, bound in the
+        // single pass, the row maximum in the two-pass path): they are rescaled by
+        // 2^(M - bound).  Pairs are counted in their first round only, so the sums are
+        // over the union of the rounds' candidates ([P1] "重复候选和归一化").  Rows with
+        // a larger bound keep the per-round (o_r, lse_r) form, merged afterwards.
+        bool stored = false;
+        if (acc_O && q.pos_i >= 0) {
+            const float bnd = S.rbound[q.row];
+            if (bnd <= kTcAccBoundMax) {
+                const float L = S.u2.rowsum[0][q.row] + S.u2.rowsum[1][q.row];
+                const size_t orow = (size_t)bh * n + q.pos_i;
+                if (q.qvalid && L > 0.0f) {
+                    const float f = use16 ? 0x1p-15f : (single ? 1.0f : exp2f(M - bnd));
+                    float *o = acc_O + orow * kTcD + wg * 32;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        red_add_v4(o + u * 4, __uint_as_float(v[u * 4 + 0]) * f, __uint_as_float(v[u * 4 + 1]) * f,
+                                   __uint_as_float(v[u * 4 + 2]) * f, __uint_as_float(v[u * 4 + 3]) * f);
+                    if (wg == 0) atomicAdd(acc_L + orow, L * f);
+                }
+                if (wg == 0) acc_M[orow] = bnd;
+                stored = true;
+            } else if (wg == 0) {
+                acc_M[(size_t)bh * n + q.pos_i] = INFINITY;   // merged from the per-round form
+            }
+        }
+        if (q.pos_i >= 0 && !stored) {
             const float L = S.u2.rowsum[0][q.row] + S.u2.rowsum[1][q.row];
             float *o = o_ws + (((size_t)r * BH + bh) * n + q.pos_i) * kTcD + wg * 32;
             const bool has = q.qvalid && L > 0.0f;

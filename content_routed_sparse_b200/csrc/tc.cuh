@@ -138,9 +138,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *mbar, uint32_t parity, u
 // phase is polled with try_wait (each poll suspends at most `suspend_ns`); the
 // global timer is read only every 256 polls, because reading it is slow and a
 // read between polls would delay the wake-up of every pipeline handoff.
+// A forceable wait gives up before its first poll while g_force_wait_timeout is
+// set (the caller's failure path then drains with non-forceable waits).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parity,
                                                   uint64_t limit_ns, uint32_t kernel,
-                                                  uint32_t site, uint32_t suspend_ns = 10000u) {
+                                                  uint32_t site, uint32_t suspend_ns = 10000u,
+                                                  bool forceable = false) {
+    if (forceable && *reinterpret_cast<volatile uint32_t *>(&g_force_wait_timeout) != 0u) {
+        raise_error(CRS_DEVERR_TIMEOUT);
+        diag_record(kernel, site, 0u, threadIdx.x, 0u, 0u);
+        return false;
+    }
     uint64_t t0 = 0;
     for (uint32_t polls = 1;; ++polls) {
         if (mbar_try_wait(mbar, parity, suspend_ns)) return true;

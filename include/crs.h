@@ -80,6 +80,18 @@ int crs_get_device_error(void *stream, uint32_t *flags);
  * Synchronizes `stream`, copies min(n, 16) words and clears the record. */
 int crs_get_device_diag(void *stream, uint32_t *out, int n);
 
+/* Test switch for the failure path of the bounded waits (the pages have no
+ * counterpart: it exists to exercise this library's own fault handling).  While
+ * on (on != 0, current device), the first mbarrier wait of the tensor-core LSH
+ * kernels (the hash of crs_lsh_route and the chunk attention of crs_lsh_attn)
+ * gives up at once, as a wait that ran out would: the kernel sets
+ * CRS_DEVERR_TIMEOUT, records (kernel id, site 1) in the diagnostic record,
+ * waits for the tensor-core work it issued, frees its tensor memory and
+ * returns without writing its outputs (bucket ids, attention sums).  Turn it
+ * off (on = 0) before using the results of later calls.  Returns CRS_ERR_CUDA
+ * if the device global cannot be written. */
+int crs_debug_force_wait_timeout(int on);
+
 /* Launch tracing.  [P1] "一个可复现的评测矩阵" and [P2] §1.1 "性能轴" ask for the
  * time of every stage (routing, sort, selection, gather, attention) reported
  * separately; this is how the library provides it.  Every kernel

@@ -105,12 +105,13 @@ def test_lsh_bf16_tensor_core_path(crs, cuda_dev, n, rounds, nb, causal, no_self
     assert "lsh_chunk_attn_tc" in crs.profile_collect()
 
 
-@pytest.mark.parametrize("variant", ["v_large_head", "v_large_one", "bound_mid", "bound_big"])
+@pytest.mark.parametrize("variant", ["v_large_head", "v_large_one", "bound_mid", "bound_two_pass", "bound_big"])
 def test_lsh_bf16_tc_precision_paths(crs, cuda_dev, variant):
     """The tensor-core kernel's P formats: fp16 P (bounds <= 14 and V below 2^16 in
     magnitude), the bf16 value + residual single pass (V not fp16-representable, or a row
     bound in (14, 48]) and the two-pass path (bound > 48).  Each CTA picks its path alone:
-    one large V entry moves only the CTAs whose window holds it."""
+    one large V entry moves only the CTAs whose window holds it.  Rows with a bound up to
+    63 sum the rounds with a fixed shift; larger bounds keep the per-round form."""
     case = workloads.lsh_clustered_case(B=1, H=2, n=1024, n_buckets=16, n_rounds=3, chunk=128,
                                         n_centres=8, pad_frac=0.05, seed=77, device=cuda_dev)
     V = case["V"].float()
@@ -122,6 +123,8 @@ def test_lsh_bf16_tc_precision_paths(crs, cuda_dev, variant):
         V[0, 0, 500, 3] = 1.0e6
     elif variant == "bound_mid":          # |q| ~ 1.3: bound ~ 18.5 (log2 units)
         case["params"]["scale"] = 10.0
+    elif variant == "bound_two_pass":     # bound ~ 55: two passes, rows around 63 take either
+        case["params"]["scale"] = 29.0    # the fixed-shift sums or the per-round form
     else:                                 # bound ~ 370
         case["params"]["scale"] = 200.0
     case["V"] = V.to(torch.bfloat16)
@@ -187,3 +190,23 @@ def test_lsh_candidates_csr_matches_oracle(crs, cuda_dev, n, chunk, rounds, nb, 
                                              int(vl[b]))
                 got = cl[rp[row]:rp[row + 1]]
                 assert np.array_equal(got, want), f"(b={b}, h={h}, i={i}): {got[:8]} vs {want[:8]}"
+
+
+def test_lsh_hash_tensor_core_near_ties(crs, cuda_dev):
+    """bf16, d = 64, b = 64: the tensor-core hash decides a bucket only when the winner
+    leads by more than its error bound, else recomputes the fp32 chain.  Exact ties
+    (duplicated rotation columns: the first maximum wins), near ties (columns 1e-6
+    apart), zero rows and rows of mixed magnitude must all give the oracle's ids."""
+    case = workloads.lsh_clustered_case(B=2, H=2, n=3000, n_rounds=4, n_buckets=64, chunk=128,
+                                        seed=5, device=cuda_dev)
+    R = case["R"].clone()
+    R[:, :, :, 5] = R[:, :, :, 3]
+    R[:, :, :, 7] = R[:, :, :, 6] + 1e-6 * torch.randn_like(R[:, :, :, 6])
+    R[:, 1, :, 20] = -R[:, 1, :, 19]
+    X = case["QK"].clone()
+    X[0, 0, 100:140] = 0
+    X[1, 1, :50] *= 1000.0
+    case["R"], case["QK"] = R, X.contiguous()
+    crs.profile_collect()
+    _route_and_check(crs, case)
+    assert "lsh_hash" in crs.profile_collect()
