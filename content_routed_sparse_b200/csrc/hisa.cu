@@ -4,8 +4,8 @@
 // scores block representatives, prunes blocks, and runs the original token
 // indexer inside the kept blocks only, with the same top-k output), §2.2
 // Eq.(7) (recall of the two levels multiplies), the HISA cost
-// O(B d_c + k_b b d_r), and "未满块由局部或单独 open-block 路径处理" (the
-// incomplete trailing block is always searched).
+// O(B d_c + k_b b d_r), and its update discussion in §2.2 (a block without a
+// representative yet, the incomplete trailing one, is searched at token level).
 //
 // Steps per decode row (one query):
 //   hisa_describe_kernel     rep_j = mean of block j's index keys (once per

@@ -13,9 +13,13 @@
 // The array's name is only a host-side stand-in for the device object; the
 // device address is fetched once per device with cudaGetSymbolAddress (with
 // that device current) the first time this entry point runs on it, and then
-// reused.  The kernels (the same ones crs_block_select launches) overwrite
+// reused while the device's current context stays the same one (after a
+// cudaDeviceReset the module is loaded again and the address is fetched anew).
+// The kernels (the same ones crs_block_select launches) overwrite
 // every scratch entry before they read it, so nothing has to be cleared
 // between calls; the array keeps the last call's contents.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -28,18 +32,50 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 constexpr int kNoAllocMaxDevices = 64;
 static std::mutex g_noalloc_mu;
 static void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+static unsigned long long g_noalloc_ctx_id[kNoAllocMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (set up once per device).
+// Unique id of the current context (cuCtxGetCurrent + cuCtxGetId, looked up once
+// through the runtime: no link-time dependency on libcuda); 0 when unknown.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+static unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+        looked = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of g_noalloc_scratch on the current device: set up once per device
+// and context, fetched again when the current context is not the one it was set up
+// in (or cannot be identified).
 static int noalloc_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return CRS_ERR_CUDA;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return CRS_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    unsigned long long id = current_ctx_id();
+    if (!g_noalloc_ptr[dev] || id == 0 || id != g_noalloc_ctx_id[dev]) {
         void *ptr = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess || ptr == nullptr) return CRS_ERR_CUDA;
         g_noalloc_ptr[dev] = ptr;
+        if (id == 0) id = current_ctx_id();     // the lookup made the primary context current
+        g_noalloc_ctx_id[dev] = id;
     }
     *out = g_noalloc_ptr[dev];
     return CRS_OK;

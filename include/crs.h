@@ -402,8 +402,10 @@ int crs_block_select(const crs_block_sel_params *p, const void *Q, const float *
  *     (sequence, query head, block) scores; larger problems return
  *     CRS_ERR_WORKSPACE with nothing launched.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture on the device.
+ *     (cudaGetSymbolAddress, with that device current) and caches it with the
+ *     device's current context; a call under another context (after a
+ *     cudaDeviceReset, say) looks it up again.  Make the first call on a
+ *     device, and the first call after a reset, before any stream capture.
  *   - Every call, on any stream, shares the one array and it keeps the last
  *     call's contents: calls that overlap on the GPU (concurrent streams)
  *     race on it and must be serialized by the caller.  Nothing needs
