@@ -1,7 +1,8 @@
 """Throughput of content-routed sparse attention on B200 (one JSON line).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
-                  [--workload lsh|lsh_fp32|lsh_decode|route|prefill|decode|decode_hisa|block|block_fp4|block_ss|block_quest|block_meanpool] [--no-extras]
+                  [--workload lsh|lsh_fp32|lsh_decode|route|prefill|prefill_hisa|decode|decode_hisa|block|block_fp4|
+                              block_ss|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
@@ -13,6 +14,7 @@ A step is one pass of the hot path over one batch of the workload:
            lists (64 buckets x 4 rounds) and paged K/V; a step appends one token per row
            and attends with it.
   prefill  indexer prefill n=32768 (top-2048) + MQA gather attention (16 heads).
+  prefill_hisa  the same with the hierarchical indexer's prefill form (64-key blocks, 128 kept).
   decode   indexer decode, 64 sequences of ragged context + GQA gather attention.
   decode_hisa  the same with the hierarchical indexer (64-key blocks, 128 kept).
   block    block-mass decode: block select (top-64 + 512 window) + GQA attention;
@@ -315,6 +317,45 @@ class PrefillWorkload(Workload):
         }
 
 
+class PrefillHisaWorkload(PrefillWorkload):
+    """The indexer prefill workload with the hierarchical indexer in its prefill form:
+    mean representatives of 64-key blocks (built once per filled block, untimed), 128
+    kept blocks per query (all of them for the first 8192 + 64 queries), the token
+    top-2048 on the tensor cores over the kept blocks and the open block, then the
+    same gather attention."""
+    BLK, TOP_BLOCKS = 64, 128
+    cpu_sample = None
+
+    def __init__(self, crs, dev):
+        super().__init__(crs, dev)
+        n = self.p["n"]
+        self.name = self.c["workload"].replace("indexer_prefill_", f"hisa_b{self.BLK}_kb{self.TOP_BLOCKS}_prefill_", 1)
+        ko = torch.tensor([0, n], dtype=torch.int64, device=dev)
+        self.rep, _ = crs.hisa_describe(self.c["k_idx"], ko, self.BLK, n)
+        self.blocks = torch.empty((n, self.TOP_BLOCKS), dtype=torch.int32, device=dev)
+        import ctypes
+        hp = crs.HisaParams(n, 4, 64, self.p["topk"], self.BLK, self.TOP_BLOCKS, n)
+        self.ws = torch.empty(int(crs.lib().crs_hisa_topk_prefill_workspace_size(ctypes.byref(hp))),
+                              dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+
+    def _run(self, src):
+        k = self.p["topk"]
+        self.crs.hisa_topk_prefill(src["q_idx"], src["w"], src["k_idx"], self.rep, k, self.BLK, self.TOP_BLOCKS,
+                                   out_blocks=self.blocks, out=self.idx, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(src["Q"], src["K"], src["V"], self.idx.view(-1, 1, k), q_pos=self.q_pos,
+                             out=self.O)
+
+    def roofline_spec(self):
+        spec = super().roofline_spec()
+        n = self.p["n"]
+        nb = n // self.BLK
+        # coarse scores of the rows with more than TOP_BLOCKS complete blocks (CUDA cores)
+        coarse = sum(max(0, (t + 1) // self.BLK) for t in range(n) if (t + 1) // self.BLK > self.TOP_BLOCKS)
+        spec["hisa"] = [("alu", coarse * 4 * 64 * 2 / 1e12, "TFLOP/s")]
+        return spec
+
+
 class DecodeWorkload(Workload):
     unit = "steps/s"
 
@@ -603,7 +644,8 @@ class BlockMeanPoolWorkload(BlockWorkload):
 
 WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_fp32": lambda crs, dev: LshWorkload(crs, dev, fp32=True),
-             "prefill": PrefillWorkload, "decode": DecodeWorkload, "decode_hisa": DecodeHisaWorkload,
+             "prefill": PrefillWorkload, "prefill_hisa": PrefillHisaWorkload, "decode": DecodeWorkload,
+             "decode_hisa": DecodeHisaWorkload,
              "lsh_decode": LshDecodeWorkload, "route": RouteWorkload,
              "block": BlockWorkload,
              "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
@@ -1003,7 +1045,8 @@ def main():
 
     extras = {}
     if not args.no_extras and not dist_on:
-        for name in [w for w in ("lsh_fp32", "lsh_decode", "route", "prefill", "decode", "decode_hisa", "block", "block_fp4", "block_ss",
+        for name in [w for w in ("lsh_fp32", "lsh_decode", "route", "prefill", "prefill_hisa", "decode", "decode_hisa",
+                                  "block", "block_fp4", "block_ss",
                                   "block_quest", "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)

@@ -151,6 +151,9 @@ _sig("crs_hisa_describe", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _
 _sig("crs_hisa_topk_workspace_size", _SZ, [ctypes.POINTER(HisaParams)])
 _sig("crs_hisa_topk", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                       _VP, _SZ, _VP])
+_sig("crs_hisa_topk_prefill_workspace_size", _SZ, [ctypes.POINTER(HisaParams)])
+_sig("crs_hisa_topk_prefill", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                              _SZ, _VP])
 _sig("crs_block_describe_ss", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, ctypes.c_int, _VP, _VP,
                                               _VP])
 _sig("crs_block_select_ss_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams), ctypes.c_int])
@@ -521,6 +524,35 @@ def hisa_topk(q_idx, w, k_idx, k_offsets, rep, blk_offsets, topk: int, blk: int,
 
 
 # ----------------------------------------------------------------- blocks --
+def hisa_topk_prefill(q_idx, w, k_idx, rep, topk: int, blk: int, top_blocks: int, out_blocks=None, out=None,
+                      count=None, workspace=None, stream=None):
+    """Hierarchical top-k for the n causal queries of one sequence -> (blocks [n,
+    top_blocks], idx [n, topk], count [n]).  rep [n // blk, 64] from hisa_describe(k_idx,
+    [0, n], blk, n)."""
+    _need(q_idx, "q_idx", torch.bfloat16)
+    n, H, d = q_idx.shape
+    _need(w, "w", torch.float32, (n, H))
+    _need(k_idx, "k_idx", torch.bfloat16, (n, d))
+    _need(rep, "rep", torch.float32)
+    p = HisaParams(n, H, d, int(topk), int(blk), int(top_blocks), n)
+    if out_blocks is None:
+        out_blocks = torch.empty((n, top_blocks), dtype=torch.int32, device=q_idx.device)
+    if out is None:
+        out = torch.empty((n, topk), dtype=torch.int32, device=q_idx.device)
+    if count is None:
+        count = torch.empty((n,), dtype=torch.int32, device=q_idx.device)
+    _need(out_blocks, "out_blocks", torch.int32, (n, top_blocks))
+    _need(out, "out", torch.int32, (n, topk))
+    _need(count, "count", torch.int32, (n,))
+    ws, wsb = _workspace(int(_lib.crs_hisa_topk_prefill_workspace_size(ctypes.byref(p))), q_idx.device, workspace)
+    if wsb == 0:
+        raise CrsError("crs_hisa_topk_prefill", 2)
+    st = _lib.crs_hisa_topk_prefill(ctypes.byref(p), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(rep), _ptr(out_blocks),
+                                    _ptr(out), _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_hisa_topk_prefill", st)
+    return out_blocks, out, count
+
+
 def block_describe(K, L: int, rank: int, blk_range=None, mu=None, xi=None, stream=None):
     """Block descriptors of K [n_seq, T, n_kv, D] bf16 -> (mu, xi) fp32."""
     _need(K, "K", torch.bfloat16)

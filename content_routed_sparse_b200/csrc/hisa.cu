@@ -46,6 +46,7 @@ struct HisaArgs {
     int32_t *out_idx;           // [rows, topk]
     int32_t *out_count;         // [rows]
     int n_rows, H, topk, blk, top_blocks, cand_cap, max_keys;
+    int prefill;                // 1: row t is query t of one sequence (keys 0..t, shared reps)
 };
 
 // one warp per complete block: lane l averages dims 2l, 2l + 1 over the block
@@ -75,8 +76,17 @@ template <int HP>
 __global__ void __launch_bounds__(kHCoarseWarps * 32) hisa_coarse_kernel(HisaArgs a) {
     constexpr int BPW = 32 / HP;
     const int row = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t k0 = a.k_off[row];
-    const int nb = (int)(min(a.k_off[row + 1] - k0, (int64_t)a.max_keys) / a.blk);
+    int nb;
+    int64_t b0;
+    if (a.prefill) {             // query row of one sequence: complete blocks below row + 1
+        nb = (row + 1) / a.blk;
+        b0 = 0;
+        if (nb <= a.top_blocks) return;                      // every block is kept: no scores
+    } else {
+        const int64_t k0 = a.k_off[row];
+        nb = (int)(min(a.k_off[row + 1] - k0, (int64_t)a.max_keys) / a.blk);
+        b0 = a.b_off[row];
+    }
     const int j0 = (blockIdx.x * kHCoarseWarps + warp) * BPW;
     if (j0 >= nb) return;                                    // warp-uniform
     float q[HP][2];
@@ -88,7 +98,7 @@ __global__ void __launch_bounds__(kHCoarseWarps * 32) hisa_coarse_kernel(HisaArg
         q[h][0] = v.x;
         q[h][1] = v.y;
     }
-    const float *rep = a.rep + a.b_off[row] * kHd + 2 * lane;
+    const float *rep = a.rep + b0 * kHd + 2 * lane;
     float v[32];
 #pragma unroll
     for (int i = 0; i < BPW; ++i) {
@@ -191,6 +201,74 @@ __global__ void __launch_bounds__(kPickT) hisa_pick_blocks_kernel(HisaArgs a) {
     }
     for (int i = n_sel + tid; i < a.top_blocks; i += kPickT) out[i] = -1;
     if (tid == 0) a.n_keep[row] = n_sel;
+}
+
+// Prefill form, one warp per query row t: its complete blocks j < (t + 1) / blk
+// sit KPL per lane (j = 32 u + lane), so word u of the row's kept-block bitmap is
+// the warp's ballot for u.  The top_blocks blocks by (c desc, block asc): the k-th
+// largest order-preserving key T bit by bit (warp counts), then every key > T and
+// the first (in block order) of those equal to T.  Rows with at most top_blocks
+// blocks keep them all.  Writes the bitmap [rows, keep_words] and the ascending
+// list [rows, top_blocks] (-1 padded).
+constexpr int kHPickWarps = 8;
+
+template <int KPL>
+__global__ void __launch_bounds__(kHPickWarps * 32) hisa_prefill_pick_kernel(HisaArgs a, uint32_t *keep,
+                                                                           int keep_words) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kHPickWarps + warp;
+    if (row >= a.n_rows) return;                             // warp-uniform
+    const int nb = (row + 1) / a.blk;
+    uint32_t *kw = keep + (size_t)row * keep_words;
+    int32_t *out = a.blocks + (size_t)row * a.top_blocks;
+    if (nb <= a.top_blocks) {
+        for (int u = lane; u < keep_words; u += 32) {
+            const int lo = 32 * u;
+            kw[u] = nb >= lo + 32 ? 0xffffffffu : (nb <= lo ? 0u : ((1u << (nb - lo)) - 1u));
+        }
+        for (int i = lane; i < a.top_blocks; i += 32) out[i] = i < nb ? i : -1;
+        return;
+    }
+    const float *c = a.coarse + (size_t)row * (a.max_keys / a.blk);
+    uint32_t key[KPL];
+    bool nan = false;
+#pragma unroll
+    for (int u = 0; u < KPL; ++u) {
+        const int j = 32 * u + lane;
+        const float x = j < nb ? c[j] : 0.0f;
+        nan |= j < nb && x != x;
+        key[u] = j < nb ? score_key(x) : 0u;
+    }
+    if (__any_sync(0xffffffffu, nan) && lane == 0) raise_error(CRS_DEVERR_NONFINITE);
+    const int k = a.top_blocks;
+    uint32_t T = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cnd = T | (1u << bit);
+        int local = 0;
+#pragma unroll
+        for (int u = 0; u < KPL; ++u) local += (32 * u + lane < nb && key[u] >= cnd) ? 1 : 0;
+        if ((int)__reduce_add_sync(0xffffffffu, (unsigned)local) >= k) T = cnd;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int u = 0; u < KPL; ++u) gt += (32 * u + lane < nb && key[u] > T) ? 1 : 0;
+    const int need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+    const uint32_t below = (1u << lane) - 1u;
+    int eq_seen = 0, base = 0;
+#pragma unroll
+    for (int u = 0; u < KPL; ++u) {
+        const bool in = 32 * u + lane < nb;
+        const bool eq = in && key[u] == T;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const bool tk = (in && key[u] > T) || (eq && eq_seen + __popc(eqm & below) < need);
+        eq_seen += __popc(eqm);
+        const uint32_t tm = __ballot_sync(0xffffffffu, tk);
+        if (lane == 0 && u < keep_words) kw[u] = tm;
+        if (tk) out[base + __popc(tm & below)] = 32 * u + lane;
+        base += __popc(tm);
+    }
+    for (int u = KPL + lane; u < keep_words; u += 32) kw[u] = 0u;
+    for (int i = base + lane; i < a.top_blocks; i += 32) out[i] = -1;
 }
 
 // grid (ceil((top_blocks + 1) / UP), rows), 256 threads: CTA x takes the UP =
@@ -435,4 +513,102 @@ extern "C" int crs_hisa_topk(const crs_hisa_params *p, const void *q_idx, const 
     _ps.more(max_blocks > 0 ? 3 : 2);             // coarse, block pick, fine, token pick
     CRS_CHECK_LAUNCH();
     return CRS_OK;
+}
+
+// ------------------------------------------------------------ prefill form --
+namespace crs {
+constexpr int kHpBlk = 64;               // one block = one 64-key tile of the tensor-core indexer
+
+static int hisa_prefill_validate(const crs_hisa_params *p) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    if (p->n_rows < 1 || p->n_idx_heads < 1 || p->topk < 1 || p->blk < 1 || p->top_blocks < 1)
+        return CRS_ERR_INVALID_ARG;
+    if (p->d_idx != kHd || p->n_idx_heads != 4 || p->blk != kHpBlk || p->topk > 2048)
+        return CRS_ERR_UNSUPPORTED;
+    if ((long long)p->top_blocks * p->blk < p->topk) return CRS_ERR_UNSUPPORTED;
+    if (p->n_rows / p->blk > 1024 || p->n_rows > (1 << 19)) return CRS_ERR_UNSUPPORTED;
+    return CRS_OK;
+}
+
+struct HisaPrefillWs {
+    float *coarse;
+    int32_t *blocks;
+    uint32_t *keep;
+    void *tc;
+    int keep_words;
+    size_t total;
+};
+
+static void hisa_prefill_layout(const crs_hisa_params *p, HisaPrefillWs &w, char *base) {
+    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const int n = p->n_rows, nbk = n / p->blk;
+    w.keep_words = max(1, ceil_div(nbk, 32));
+    size_t off = 0;
+    auto take = [&](size_t bytes) { char *q = base ? base + off : nullptr; off += al(bytes); return q; };
+    w.coarse = reinterpret_cast<float *>(take((size_t)n * max(nbk, 1) * 4));
+    w.blocks = reinterpret_cast<int32_t *>(take((size_t)n * p->top_blocks * 4));
+    w.keep = reinterpret_cast<uint32_t *>(take((size_t)n * w.keep_words * 4));
+    crs_indexer_params ip{CRS_IDX_PREFILL, n, p->n_idx_heads, p->d_idx, p->topk, 0};
+    w.tc = take(prefill_tc_workspace(&ip));
+    w.total = off;
+}
+}  // namespace crs
+
+extern "C" size_t crs_hisa_topk_prefill_workspace_size(const crs_hisa_params *p) {
+    if (hisa_prefill_validate(p)) return 0;
+    HisaPrefillWs w;
+    hisa_prefill_layout(p, w, nullptr);
+    return w.total;
+}
+
+extern "C" int crs_hisa_topk_prefill(const crs_hisa_params *p, const void *q_idx, const float *w, const void *k_idx,
+                                     const float *rep, int32_t *out_blocks, int32_t *out_idx, int32_t *out_count,
+                                     void *ws, size_t ws_bytes, void *stream) {
+    int st = hisa_prefill_validate(p);
+    if (st) return st;
+    if (!q_idx || !w || !k_idx || !rep || !out_idx || !out_count) return CRS_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q_idx) & 15) || (reinterpret_cast<uintptr_t>(k_idx) & 15) ||
+        (reinterpret_cast<uintptr_t>(rep) & 7))
+        return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_hisa_topk_prefill_workspace_size(p);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    HisaPrefillWs hw;
+    hisa_prefill_layout(p, hw, static_cast<char *>(ws));
+    const int n = p->n_rows, nbk = n / p->blk;
+    HisaArgs a{};
+    a.q = static_cast<const __nv_bfloat16 *>(q_idx);
+    a.w = w;
+    a.k = static_cast<const __nv_bfloat16 *>(k_idx);
+    a.rep = const_cast<float *>(rep);
+    a.coarse = hw.coarse;
+    a.blocks = out_blocks ? out_blocks : hw.blocks;
+    a.n_rows = n;
+    a.H = p->n_idx_heads;
+    a.topk = p->topk;
+    a.blk = p->blk;
+    a.top_blocks = p->top_blocks;
+    a.max_keys = n;
+    a.prefill = 1;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        ProfScope _ps(K_HISA, s);
+        if (nbk > p->top_blocks) {
+            const dim3 gc(ceil_div(nbk, kHCoarseWarps * (32 / 4)), n);
+            hisa_coarse_kernel<4><<<gc, kHCoarseWarps * 32, 0, s>>>(a);
+            _ps.more(1);
+        }
+        const int kpl = ceil_div(max(nbk, 1), 32);
+        const unsigned gp = (unsigned)ceil_div(n, kHPickWarps);
+        if (kpl <= 1) hisa_prefill_pick_kernel<1><<<gp, kHPickWarps * 32, 0, s>>>(a, hw.keep, hw.keep_words);
+        else if (kpl <= 2) hisa_prefill_pick_kernel<2><<<gp, kHPickWarps * 32, 0, s>>>(a, hw.keep, hw.keep_words);
+        else if (kpl <= 4) hisa_prefill_pick_kernel<4><<<gp, kHPickWarps * 32, 0, s>>>(a, hw.keep, hw.keep_words);
+        else if (kpl <= 8) hisa_prefill_pick_kernel<8><<<gp, kHPickWarps * 32, 0, s>>>(a, hw.keep, hw.keep_words);
+        else if (kpl <= 16) hisa_prefill_pick_kernel<16><<<gp, kHPickWarps * 32, 0, s>>>(a, hw.keep, hw.keep_words);
+        else hisa_prefill_pick_kernel<32><<<gp, kHPickWarps * 32, 0, s>>>(a, hw.keep, hw.keep_words);
+    }
+    CRS_CHECK_LAUNCH();
+    // the token level: the tensor-core prefill indexer with every row's kept blocks
+    const crs_indexer_params ip{CRS_IDX_PREFILL, n, p->n_idx_heads, p->d_idx, p->topk, 0};
+    return launch_prefill_tc(&ip, q_idx, w, k_idx, out_idx, out_count, hw.tc, s, hw.keep, hw.keep_words,
+                             p->top_blocks);
 }

@@ -184,6 +184,8 @@ struct IdxArgs {
     const int32_t *row_list;      // optional: rows to process (blockIdx -> row_list[i])
     const int32_t *list_count;    //   and how many entries of row_list are live
     int list_cap;                 //   capacity of row_list
+    const uint32_t *keep;         // optional (prefill): kept 64-key blocks per row, a bit each;
+    int keep_words;               //   a complete block without its bit is not visible
 };
 
 __device__ __forceinline__ void row_range(const IdxArgs &a, int row, int64_t &kb, int &nv) {
@@ -238,7 +240,16 @@ __device__ __forceinline__ void idx_slice_row(const IdxArgs &a, const int slice,
 
     // ---- scores: one thread per key, 128-byte key rows read as 8 x 16 B
     bool nonfinite = false;
+    const uint32_t *keep_row = a.keep ? a.keep + (size_t)row * a.keep_words : nullptr;
+    const int n_full = nv >> 6;                  // complete 64-key blocks of the row
     for (int i = threadIdx.x; i < ns; i += kSelThreads) {
+        if (keep_row) {
+            const int blk = (s0 + i) >> 6;
+            if (blk < n_full && !((keep_row[blk >> 5] >> (blk & 31)) & 1u)) {
+                skey[i] = 0u;                    // not a candidate: ranks below every score
+                continue;
+            }
+        }
         const uint4 *kr = reinterpret_cast<const uint4 *>(a.k + (size_t)(kb + s0 + i) * kIdxDim);
         float kf[kIdxDim];
 #pragma unroll
@@ -710,7 +721,7 @@ static bool prefill_tc_applicable(const crs_indexer_params *p);
 static size_t prefill_tc_workspace(const crs_indexer_params *p);
 static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, const float *wgt,
                              const void *k_idx, int32_t *out_idx, int32_t *out_count, void *ws,
-                             cudaStream_t s);
+                             cudaStream_t s, const uint32_t *keep, int keep_words, int top_blocks);
 }  // namespace crs
 
 struct DecWs {
@@ -799,7 +810,7 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
         return CRS_OK;
     }
     if (prefill_tc_applicable(p))
-        return launch_prefill_tc(p, q_idx, w, k_idx, out_idx, out_count, ws, s);
+        return launch_prefill_tc(p, q_idx, w, k_idx, out_idx, out_count, ws, s, nullptr, 0, 0);
     int max_slices, ws_rows;
     idx_geometry(p, max_slices, ws_rows);
     if (max_slices > 64) return CRS_ERR_UNSUPPORTED;
@@ -807,6 +818,8 @@ extern "C" int crs_indexer_topk(const crs_indexer_params *p, const void *q_idx, 
     a.row_list = nullptr;
     a.list_count = nullptr;
     a.list_cap = 0;
+    a.keep = nullptr;
+    a.keep_words = 0;
     a.mode = p->mode;
     a.q = static_cast<const __nv_bfloat16 *>(q_idx);
     a.w = w;

@@ -73,6 +73,8 @@ struct IdxTcArgs {
     uint32_t *cand_key;       // [n, kIParts, kICap]
     int32_t *cand_idx;        // [n, kIParts, kICap]
     int32_t *cand_cnt;        // [n, kIParts]
+    const uint32_t *keep;     // optional: [n, keep_words] kept 64-key blocks (one bit each);
+    int keep_words;           //   a complete block without its bit is masked for that row
     int n, samp_slots, n_tiles_rows;
 };
 
@@ -258,7 +260,12 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             const int key0 = kt * kIkN + part * kIPartKeys;
             // keys > t (causal) exist only in the CTA's last two tiles
             const int lim = t - key0 + 1;            // keys [key0, key0 + lim) are visible
-            const uint32_t vis = lim >= kIPartKeys ? 0xffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+            uint32_t vis = lim >= kIPartKeys ? 0xffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+            // hierarchical mode: a key tile is one 64-key block; a complete block the
+            // row did not keep is not visible (the open block and later keys are)
+            if (a.keep != nullptr && row_ok && kt < ((t + 1) >> 6) &&
+                !((__ldg(a.keep + (size_t)t * a.keep_words + (kt >> 5)) >> (kt & 31)) & 1u))
+                vis = 0u;
             if constexpr (MODE == 0) {
                 if (row_ok) {
                     uint32_t pk[kIPartKeys / 2];
@@ -331,13 +338,17 @@ idx_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) idx_tc_tau_kernel(const uint16_t *__restrict__ samples,
                                                          uint32_t *__restrict__ tau, int n,
-                                                         int samp_slots, int topk) {
+                                                         int samp_slots, int topk, int top_blocks) {
     __shared__ int hist[8][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t >= n) return;
     int *hw = hist[warp];
-    if (t + 1 <= topk) {
+    // the row's candidate keys: all t + 1, or (hierarchical) the kept blocks + the open block
+    long long cand = t + 1;
+    const int nbt = (t + 1) >> 6;
+    if (top_blocks > 0 && nbt > top_blocks) cand = (long long)top_blocks * 64 + (t + 1 - nbt * 64);
+    if (cand <= topk) {
         if (lane == 0) tau[t] = 0u;
         return;
     }
@@ -357,7 +368,7 @@ __global__ void __launch_bounds__(256) idx_tc_tau_kernel(const uint16_t *__restr
     }
     nvalid = warp_sum_int(nvalid);
     __syncwarp();
-    const long long R = ((long long)nvalid * topk * 5 + 4LL * (t + 1) - 1) / (4LL * (t + 1));  // ceil(1.25 k nv/(t+1))
+    const long long R = ((long long)nvalid * topk * 5 + 4LL * cand - 1) / (4LL * cand);  // ceil(1.25 k nv/cand)
     if (R < 1 || R > nvalid) {
         if (lane == 0) tau[t] = 0u;
         return;
@@ -603,7 +614,7 @@ static size_t prefill_tc_workspace(const crs_indexer_params *p) {
 
 static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, const float *wgt,
                              const void *k_idx, int32_t *out_idx, int32_t *out_count, void *ws,
-                             cudaStream_t s) {
+                             cudaStream_t s, const uint32_t *keep, int keep_words, int top_blocks) {
     const int n = p->n_rows, topk = p->topk;
     PFN_cuTensorMapEncodeTiled_v12000 enc = tc::tensor_map_encoder();
     if (!enc) return CRS_ERR_CUDA;
@@ -639,6 +650,8 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
     a.cand_key = w.cand_key;
     a.cand_idx = w.cand_idx;
     a.cand_cnt = w.cand_cnt;
+    a.keep = keep;
+    a.keep_words = keep_words;
     a.n = n;
     a.samp_slots = w.samp_slots;
     a.n_tiles_rows = ceil_div(n, kIqM);
@@ -653,7 +666,7 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
     CRS_CHECK_LAUNCH();
     {
         ProfScope _ps(K_IDX_SELECT, s);
-        idx_tc_tau_kernel<<<ceil_div(n, 8), 256, 0, s>>>(w.samples, w.tau, n, w.samp_slots, topk);
+        idx_tc_tau_kernel<<<ceil_div(n, 8), 256, 0, s>>>(w.samples, w.tau, n, w.samp_slots, topk, top_blocks);
     }
     CRS_CHECK_LAUNCH();
     {
@@ -690,6 +703,8 @@ static int launch_prefill_tc(const crs_indexer_params *p, const void *q_idx, con
     f.max_slices = w.fb_slices;
     f.row_list = w.fb_list;
     f.list_count = w.fb_count;
+    f.keep = keep;
+    f.keep_words = keep_words;
     const int fbr = min(n, kIFallbackRows);
     f.list_cap = fbr;
     const int fb_grid = min(fbr, 2 * 148);      // CTAs stride over the live list entries

@@ -336,6 +336,28 @@ int crs_hisa_topk(const crs_hisa_params *p, const void *q_idx, const float *w, c
                   int32_t *out_blocks, int32_t *out_idx, int32_t *out_count, void *ws, size_t ws_bytes,
                   void *stream);
 
+/* HISA prefill (causal) form.  [P2] "索引器的三种降本方向", §2.1 Eq.(4) and §2.2
+ * Eq.(7): the n queries of one sequence; query t sees keys 0..t as the flat
+ * prefill indexer's rows do; its complete blocks are the sequence's blocks
+ * j < (t + 1) / blk, whose representatives rep_j do not depend on the query
+ * (crs_hisa_describe with n_rows = 1, k_offsets = {0, n}, blk_offsets = {0, n / blk});
+ * then the decode row rule with ctx = t + 1: the top_blocks blocks by
+ * (c desc, block asc) (all of them when there are at most top_blocks), and the
+ * token top-k (same score, ties, ascending, -1-padded output) over the kept
+ * blocks' keys and the open block (keys (t + 1) / blk * blk .. t).
+ * p: n_rows = n (queries = keys), n_idx_heads = 4, d_idx = 64, blk = 64,
+ * topk <= 2048, top_blocks * blk >= topk, n / blk <= 1024, n <= 2^19 (else
+ * CRS_ERR_UNSUPPORTED); max_keys is not used.
+ * q_idx [n, 4, 64] bf16, w [n, 4] f32, k_idx [n, 64] bf16 (16-byte aligned);
+ * rep [n / blk, 64] f32; out_blocks (optional) [n, top_blocks] int32; out_idx
+ * [n, topk] int32; out_count [n] int32.  The token level runs on the tensor
+ * cores (one 64-key block = one key tile; a row's unkept complete blocks are
+ * masked), with the exact selection of crs_indexer_topk. */
+size_t crs_hisa_topk_prefill_workspace_size(const crs_hisa_params *p);
+int crs_hisa_topk_prefill(const crs_hisa_params *p, const void *q_idx, const float *w, const void *k_idx,
+                          const float *rep, int32_t *out_blocks, int32_t *out_idx, int32_t *out_count,
+                          void *ws, size_t ws_bytes, void *stream);
+
 /* ====================================================================== *
  * Block descriptors.  [P5] Eq.(11), (16), (20) and Algorithm 2: for each
  * complete block of L consecutive keys of one (sequence, KV head):
