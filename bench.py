@@ -2,7 +2,7 @@
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl product|reference]
                   [--workload lsh|lsh_fp32|lsh_decode|route|prefill|prefill_hisa|decode|decode_hisa|block|block_fp4|
-                              block_ss|block_quest|block_meanpool] [--no-extras]
+                              block_ss|block_fp4_ss|block_quest|block_meanpool] [--no-extras]
 
 A step is one pass of the hot path over one batch of the workload:
   lsh      (headline) multi-round bf16 LSH attention, B=2, H=8, n=16384, d=64,
@@ -21,6 +21,8 @@ A step is one pass of the hot path over one batch of the workload:
            the descriptor build is timed separately (it runs once per filled block).
   block_fp4 the same on bf16 means + FP4 (E2M1) eigenvectors (528 B per block).
   block_ss  the same on descriptors in a query subspace of 85 dims (fp32).
+  block_fp4_ss  the deployed descriptor: bf16 means + FP4 eigenvectors in the 85-dim query
+           subspace, scored on the tensor cores.
   block_quest / block_meanpool  the same step with the baseline selectors (Quest boxes;
            block means alone).
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on
@@ -622,6 +624,58 @@ class BlockSubspaceWorkload(BlockWorkload):
         return spec
 
 
+class BlockFp4SubspaceWorkload(BlockWorkload):
+    """The pages' deployed descriptor (the delivered row of the COBS notes' Table 3):
+    bf16 block means and four FP4 (E2M1) scaled eigenvectors of the query-subspace
+    covariance (s = 85), scored on the tensor cores with the projected query.  Cache
+    build: subspace describe + quantise (untimed)."""
+    SD = 85
+    cpu_sample = None
+
+    def __init__(self, crs, dev):
+        import workloads
+        self.U = workloads.query_subspace(128, self.SD, device=dev)
+        super().__init__(crs, dev)
+        p = self.p
+        self.name = self.c["workload"].replace("block_", f"block_fp4_ss{self.SD}_", 1)
+        import ctypes
+        bp = crs.BlockSelParams(crs.BlockParams(p["n_seq"], p["n_kv_heads"], p["T"], p["D"], p["L"],
+                                                p["rank"], 0, p["T"] // p["L"]),
+                                p["n_q_heads"], p["top_blocks"], p["window"], p["scale"])
+        self.ws = torch.empty(int(crs.lib().crs_block_select_fp4_ss_workspace_size(ctypes.byref(bp), self.SD)),
+                              dtype=torch.uint8, device=dev)
+
+    def _build_cache(self):
+        mu, xi = self.crs.block_describe_ss(self.c["K"], self.p["L"], self.p["rank"], self.U)
+        self.mu16, self.xi4, self.xs = self.crs.block_quantize_ss(mu, xi, self.p["T"], self.p["L"])
+        torch.cuda.synchronize()
+        del mu, xi
+
+    def _run(self, Q):
+        p = self.p
+        self.crs.block_select_fp4_ss(Q, self.U, self.mu16, self.xi4, self.xs, p["T"], p["L"], p["top_blocks"],
+                                     p["window"], tok=self.tok, count=self.cnt, workspace=self.ws)
+        self.crs.sparse_attn(Q, self.Kf, self.Vf, self.tok, kv_base=self.kv_base, q_pos=self.q_pos,
+                             out=self.O, workspace=self.ws2)
+
+    def summary_bytes(self):
+        """Summary-key bytes of one sequence's step (4 KV heads x T/L blocks): the pages'
+        accounting (bf16 mean + 4 x (s/2 code bytes + a 4-byte scale)) and what is stored
+        (codes padded to 48 bytes per vector)."""
+        p = self.p
+        blocks = p["n_kv_heads"] * (p["T"] // p["L"])
+        alg = blocks * (p["D"] * 2 + p["rank"] * (self.SD / 2 + 4))
+        stored = blocks * (p["D"] * 2 + p["rank"] * (48 + 4))
+        return alg, stored
+
+    def roofline_spec(self):
+        p = self.p
+        spec = super().roofline_spec()
+        _, stored = self.summary_bytes()
+        spec["block_score"] = [("hbm", p["n_seq"] * stored / 1e9, "GB/s")]
+        return spec
+
+
 class BlockMeanPoolWorkload(BlockWorkload):
     """Baseline selector: the block mean alone (first-order score, fp32, 512 B per block)."""
     cpu_sample = None
@@ -649,7 +703,8 @@ WORKLOADS = {"lsh": lambda crs, dev: LshWorkload(crs, dev),
              "lsh_decode": LshDecodeWorkload, "route": RouteWorkload,
              "block": BlockWorkload,
              "block_fp4": BlockFp4Workload, "block_quest": BlockQuestWorkload,
-             "block_meanpool": BlockMeanPoolWorkload, "block_ss": BlockSubspaceWorkload}
+             "block_meanpool": BlockMeanPoolWorkload, "block_ss": BlockSubspaceWorkload,
+             "block_fp4_ss": BlockFp4SubspaceWorkload}
 
 
 # ------------------------------------------------------------------- timing --
@@ -1046,7 +1101,7 @@ def main():
     extras = {}
     if not args.no_extras and not dist_on:
         for name in [w for w in ("lsh_fp32", "lsh_decode", "route", "prefill", "prefill_hisa", "decode", "decode_hisa",
-                                  "block", "block_fp4", "block_ss",
+                                  "block", "block_fp4", "block_fp4_ss", "block_ss",
                                   "block_quest", "block_meanpool") if w != args.workload]:
             try:
                 w2 = WORKLOADS[name](crs, dev)
@@ -1061,6 +1116,11 @@ def main():
                                 "gpu_launches": r2["gpu_launches"]}
                 if not args.no_cpu_baseline:
                     extras[name]["cpu_baseline"] = cpu_baseline(w2, 1.0 / 8)
+                if hasattr(w2, "summary_bytes"):
+                    alg, stored = w2.summary_bytes()
+                    extras[name]["summary_key_kib_per_seq"] = {"algorithmic": round(alg / 1024, 1),
+                                                               "stored": round(stored / 1024, 1),
+                                                               "pages_table3": 1767}
                 if name == "block":
                     torch.cuda.synchronize()
                     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -154,6 +154,11 @@ _sig("crs_hisa_topk", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, 
 _sig("crs_hisa_topk_prefill_workspace_size", _SZ, [ctypes.POINTER(HisaParams)])
 _sig("crs_hisa_topk_prefill", ctypes.c_int, [ctypes.POINTER(HisaParams), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                               _SZ, _VP])
+_sig("crs_block_quantize_ss", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, ctypes.c_int, _VP, _VP, _VP,
+                                              _VP])
+_sig("crs_block_select_fp4_ss_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams), ctypes.c_int])
+_sig("crs_block_select_fp4_ss", ctypes.c_int, [ctypes.POINTER(BlockSelParams), _VP, _VP, ctypes.c_int, _VP, _VP,
+                                                _VP, _VP, _VP, _VP, _SZ, _VP])
 _sig("crs_block_describe_ss", ctypes.c_int, [ctypes.POINTER(BlockParams), _VP, _VP, ctypes.c_int, _VP, _VP,
                                               _VP])
 _sig("crs_block_select_ss_workspace_size", _SZ, [ctypes.POINTER(BlockSelParams), ctypes.c_int])
@@ -740,6 +745,61 @@ def block_select_fp4(Q, mu16, xi4, xi_scale, T: int, L: int, top_blocks: int, wi
     st = _lib.crs_block_select_fp4(ctypes.byref(p), _ptr(Q), _ptr(mu16), _ptr(xi4), _ptr(xi_scale),
                                    _ptr(tok), _ptr(count), _ptr(ws), wsb, _stream(stream))
     _check("crs_block_select_fp4", st)
+    return tok, count
+
+
+SS_CODE_BYTES = 48        # stored codes per subspace eigenvector (96 dims, those past sd zero)
+
+
+def block_quantize_ss(mu, xi_ss, T: int, L: int, out=None, stream=None):
+    """The deployed descriptor: mu -> bf16 (full space), the query-subspace eigenvectors
+    xi_ss [.., rank, sd] (sd <= 96) -> FP4 codes [.., rank, 48] + fp32 scales."""
+    _need(mu, "mu", torch.float32)
+    n_seq, n_kv, nfull, D = mu.shape
+    rank, sd = xi_ss.shape[3], xi_ss.shape[4]
+    _need(xi_ss, "xi_ss", torch.float32, (n_seq, n_kv, nfull, rank, sd))
+    if out is None:
+        out = (torch.empty((n_seq, n_kv, nfull, D), dtype=torch.bfloat16, device=mu.device),
+               torch.empty((n_seq, n_kv, nfull, rank, SS_CODE_BYTES), dtype=torch.uint8, device=mu.device),
+               torch.empty((n_seq, n_kv, nfull, rank), dtype=torch.float32, device=mu.device))
+    mu16, xi4, xs = out
+    _need(mu16, "mu16", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    _need(xi4, "xi4", torch.uint8, (n_seq, n_kv, nfull, rank, SS_CODE_BYTES))
+    _need(xs, "xi_scale", torch.float32, (n_seq, n_kv, nfull, rank))
+    p = BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull)
+    _check("crs_block_quantize_ss", _lib.crs_block_quantize_ss(ctypes.byref(p), _ptr(mu), _ptr(xi_ss), int(sd),
+                                                               _ptr(mu16), _ptr(xi4), _ptr(xs), _stream(stream)))
+    return mu16, xi4, xs
+
+
+def block_select_fp4_ss(Q, U, mu16, xi4, xi_scale, T: int, L: int, top_blocks: int, window: int, scale=None,
+                        tok=None, count=None, workspace=None, stream=None):
+    """block_select on the deployed descriptor (bf16 means, FP4 query-subspace
+    eigenvectors from block_quantize_ss); U [D, sd] the subspace basis."""
+    _need(Q, "Q", torch.bfloat16)
+    n_seq, n_q, D = Q.shape
+    _need(U, "U", torch.float32)
+    sd = U.shape[1]
+    n_kv, nfull, rank = mu16.shape[1], mu16.shape[2], xi4.shape[3]
+    _need(mu16, "mu16", torch.bfloat16, (n_seq, n_kv, nfull, D))
+    _need(xi4, "xi4", torch.uint8, (n_seq, n_kv, nfull, rank, SS_CODE_BYTES))
+    _need(xi_scale, "xi_scale", torch.float32, (n_seq, n_kv, nfull, rank))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    p = BlockSelParams(BlockParams(n_seq, n_kv, int(T), D, int(L), rank, 0, nfull), n_q,
+                       int(top_blocks), int(window), float(scale))
+    cap = top_blocks * L + window
+    if tok is None:
+        tok = torch.empty((n_seq, n_kv, cap), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((n_seq, n_kv), dtype=torch.int32, device=Q.device)
+    _need(tok, "tok", torch.int32, (n_seq, n_kv, cap))
+    _need(count, "count", torch.int32, (n_seq, n_kv))
+    ws, wsb = _workspace(int(_lib.crs_block_select_fp4_ss_workspace_size(ctypes.byref(p), int(sd))), Q.device,
+                         workspace)
+    st = _lib.crs_block_select_fp4_ss(ctypes.byref(p), _ptr(Q), _ptr(U), int(sd), _ptr(mu16), _ptr(xi4),
+                                      _ptr(xi_scale), _ptr(tok), _ptr(count), _ptr(ws), wsb, _stream(stream))
+    _check("crs_block_select_fp4_ss", st)
     return tok, count
 
 

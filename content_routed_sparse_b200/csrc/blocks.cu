@@ -300,7 +300,8 @@ query_project_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restric
     const __nv_bfloat16 *q = Q + (size_t)row * kBdD;
     for (int j = lane; j < sd; j += 32) {
         float acc = 0.0f;
-        for (int d = 0; d < kBdD; ++d) acc = fmaf(U[(size_t)d * sd + j], scale * __bfloat162float(q[d]), acc);
+#pragma unroll 16           // the loads of U run ahead of the dependent FMA chain
+        for (int d = 0; d < kBdD; ++d) acc = fmaf(__ldg(U + (size_t)d * sd + j), scale * __bfloat162float(q[d]), acc);
         qx[(size_t)row * sd + j] = acc;
     }
 }
@@ -872,6 +873,7 @@ struct FtSmem {
     unsigned char mu[kFtStages][2][kFtM * 128];    // [stage][K half]: 128 blocks x 64 dims, SW128
     unsigned char dec[kFtDecBufs][2][kFtM * 128];  // [buffer][K half]: one eigenvector as bf16
     unsigned char q[kFtStages][2][kFtN * 128];     // [stage][K half]: 16 rows x 64 dims, rows >= G zero
+    unsigned char p[kFtStages][2][kFtN * 128];     // subspace form: projected query, hi rows 0..G-1, lo G..2G-1
     uint64_t full[kFtStages], raw_empty[kFtStages], dec_full[kFtDecBufs], dec_empty[kFtDecBufs];
     uint64_t tm_full[2], tm_empty[2];
     uint32_t tmem_base;
@@ -884,12 +886,14 @@ struct FtArgs {
     const float *xi_scale;
     float *sc_out;
     int n_kv, n_q, G, R, n_full, tiles_per_sh, total_tiles, tiles_per_cta;
+    int code_bytes;     // bytes of codes per eigenvector: 64 (D = 128) or 48 (subspace, <= 96 dims)
+    int split;          // 1: the code products take the projected query (bf16 value + residual)
     float scale;
 };
 
 __global__ void __launch_bounds__(kFtThreads, 1)
 block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_constant__ CUtensorMap tq,
-                          FtArgs a) {
+                          const __grid_constant__ CUtensorMap tp, FtArgs a) {
     extern __shared__ unsigned char ft_raw[];
     const uint32_t mis = smem_u32(ft_raw) & 1023u;
     FtSmem &S = *reinterpret_cast<FtSmem *>(ft_raw + ((1024u - mis) & 1023u));
@@ -944,13 +948,17 @@ block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_
                 int sh, b0, nb;
                 tile_of(i, sh, b0, nb);
                 const int seq = sh / a.n_kv, h = sh - seq * a.n_kv;
-                tc::mbar_arrive_expect_tx(&S.full[s], 2 * kFtM * 128 + 2 * a.G * 128);
+                tc::mbar_arrive_expect_tx(&S.full[s], 2 * kFtM * 128 + 2 * a.G * 128 + (a.split ? 2 * kFtN * 128 : 0));
                 const int row = sh * a.n_full + b0;
                 tc::tma_load_2d(S.mu[s][0], &tmu, 0, row, &S.full[s]);
                 tc::tma_load_2d(S.mu[s][1], &tmu, 64, row, &S.full[s]);
                 const int qrow = seq * a.n_q + h * a.G;
                 tc::tma_load_2d(S.q[s][0], &tq, 0, qrow, &S.full[s]);
                 tc::tma_load_2d(S.q[s][1], &tq, 64, qrow, &S.full[s]);
+                if (a.split) {           // this (sequence, KV head)'s 16 projected rows
+                    tc::tma_load_2d(S.p[s][0], &tp, 0, sh * kFtN, &S.full[s]);
+                    tc::tma_load_2d(S.p[s][1], &tp, 64, sh * kFtN, &S.full[s]);
+                }
             }
         }
     } else if (warp == 1) {
@@ -968,24 +976,24 @@ block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_
                 if (!ok) break;
                 tc::fence_after();
                 const uint32_t d0 = tmem + acc * 128;
-                auto mma_tile = [&](unsigned char (*A)[kFtM * 128], uint32_t d) {
+                auto mma_tile = [&](unsigned char (*A)[kFtM * 128], unsigned char (*B)[kFtN * 128], uint32_t d) {
 #pragma unroll
                     for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint64_t ad = tc::smem_desc(smem_u32(A[kh]) + k * 32, 16, 1024, tc::kLayoutSW128);
-                            const uint64_t bd = tc::smem_desc(smem_u32(S.q[s][kh]) + k * 32, 16, 1024,
+                            const uint64_t bd = tc::smem_desc(smem_u32(B[kh]) + k * 32, 16, 1024,
                                                               tc::kLayoutSW128);
                             tc::mma_bf16(d, ad, bd, idesc, (kh | k) ? 1u : 0u);
                         }
                 };
-                mma_tile(S.mu[s], d0);
+                mma_tile(S.mu[s], S.q[s], d0);
                 for (int e = 0; e < R; ++e, ++j) {
                     const int b = j % kFtDecBufs, v = j / kFtDecBufs;
                     ok = tc::mbar_wait_bounded(&S.dec_full[b], v & 1, kBsWaitNs, K_BLK_SCORE, 13, kFtSuspendNs);
                     if (!ok) break;
                     tc::fence_after();
-                    mma_tile(S.dec[b], d0 + 16 * (1 + e));
+                    mma_tile(S.dec[b], a.split ? S.p[s] : S.q[s], d0 + 16 * (1 + e));
                     tc::commit(&S.dec_empty[b]);
                 }
                 if (!ok) break;
@@ -1007,13 +1015,14 @@ block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_
         auto fetch = [&](int i, uint4 (&dst)[kFtMaxR][2]) {
             int sh, b0, nb;
             tile_of(i, sh, b0, nb);
-            const uint8_t *src = a.xi4 + ((size_t)sh * a.n_full + b0 + r) * R * 64 + c0 * 4;
+            const uint8_t *src = a.xi4 + ((size_t)sh * a.n_full + b0 + r) * R * a.code_bytes + c0 * 4;
 #pragma unroll
             for (int e = 0; e < kFtMaxR; ++e)
 #pragma unroll
-                for (int kh = 0; kh < 2; ++kh)
-                    dst[e][kh] = (e < R && r < nb) ? __ldg(reinterpret_cast<const uint4 *>(src + e * 64 + kh * 32))
-                                                   : make_uint4(0, 0, 0, 0);
+                for (int kh = 0; kh < 2; ++kh)     // codes past code_bytes (dims the vector lacks) are zero
+                    dst[e][kh] = (e < R && r < nb && kh * 32 + c0 * 4 < a.code_bytes)
+                                     ? __ldg(reinterpret_cast<const uint4 *>(src + e * a.code_bytes + kh * 32))
+                                     : make_uint4(0, 0, 0, 0);
         };
         fetch(0, cur);
         int j = 0;
@@ -1101,7 +1110,9 @@ block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_
                     float quad2 = 0.0f;
 #pragma unroll
                     for (int e = 0; e < kFtMaxR; ++e) {      // sig[e] = 0 for e >= R
-                        const float pe = sig[e] * __uint_as_float(e < R ? d[1 + e][g] : 0u);
+                        float dot = __uint_as_float(e < R ? d[1 + e][g] : 0u);
+                        if (a.split) dot += __uint_as_float(e < R ? d[1 + e][a.G + g] : 0u);   // + residual
+                        const float pe = sig[e] * dot;
                         quad2 = fmaf(pe, pe, quad2);
                     }
                     a.sc_out[((size_t)sh * a.G + g) * a.n_full + b0 + row] =
@@ -1353,6 +1364,8 @@ extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q
     fa.tiles_per_sh = ceil_div(n_full, kFtM);
     fa.total_tiles = n_sh * fa.tiles_per_sh;
     fa.scale = p->scale;
+    fa.code_bytes = kBdD / 2;
+    fa.split = 0;
     int dev = 0, sms = 148;
     CRS_TRY_CUDA(cudaGetDevice(&dev));
     CRS_TRY_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
@@ -1363,7 +1376,7 @@ extern "C" int crs_block_select_fp4(const crs_block_sel_params *p, const void *Q
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
     {
         ProfScope _ps(K_BLK_SCORE, s);
-        block_score_fp4_tc_kernel<<<grid, kFtThreads, smem_s, s>>>(tmu, tq, fa);
+        block_score_fp4_tc_kernel<<<grid, kFtThreads, smem_s, s>>>(tmu, tq, tq, fa);
     }
     CRS_CHECK_LAUNCH();
     return launch_block_pick(p, sc, tok_idx, tok_count, s);
@@ -1450,6 +1463,193 @@ extern "C" int crs_block_select_ss(const crs_block_sel_params *p, const void *Q,
         block_score_kernel<<<dim3(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv), kBsThreads, smem_a, s>>>(
             static_cast<const __nv_bfloat16 *>(Q), mu, xi_ss, sc, p->b.n_kv, p->n_q, G, p->b.rank, n_full,
             p->scale, sd, qx);
+    }
+    CRS_CHECK_LAUNCH();
+    return launch_block_pick(p, sc, tok_idx, tok_count, s);
+}
+
+// ---------------------------------------------------------------------------
+// The pages' deployed descriptor ([P5] "子空间方法" Eq.(17)-(18) with "量化",
+// Table 3's delivered row): the bf16 block mean in the full space and the r
+// scaled eigenvectors of the query-subspace covariance U^T Sigma U (sd <= 96
+// dims) in E2M1 FP4, one fp32 scale each.  Codes are stored 48 bytes per
+// vector (96 dims, those past sd zero) so that every vector starts on a
+// 16-byte boundary.
+// ---------------------------------------------------------------------------
+namespace crs {
+constexpr int kSsPad = 96;                  // stored subspace dims
+constexpr int kSsCodeBytes = kSsPad / 2;
+
+// one warp per vector: vectors v < n_mu are means (bf16), the rest subspace
+// eigenvectors; lane l < 24 takes dims [4l, 4l + 4)
+__global__ void __launch_bounds__(256) block_quantize_ss_kernel(const float *__restrict__ mu,
+                                                                const float *__restrict__ xi,
+                                                                __nv_bfloat16 *__restrict__ mu16,
+                                                                uint8_t *__restrict__ xi4,
+                                                                float *__restrict__ xi_scale, long long n_mu,
+                                                                long long n_xi, int sd) {
+    const long long v = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (v < n_mu) {
+        const float4 x = reinterpret_cast<const float4 *>(mu + v * kBdD)[lane];
+        __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t *>(&a);
+        o.y = *reinterpret_cast<uint32_t *>(&b);
+        reinterpret_cast<uint2 *>(mu16 + v * kBdD)[lane] = o;
+        return;
+    }
+    const long long w = v - n_mu;
+    if (w >= n_xi) return;
+    float x[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int dd = 4 * lane + t;
+        x[t] = dd < sd ? xi[w * sd + dd] : 0.0f;
+    }
+    const float amax = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+    const float sc = amax / 6.0f;
+    const uint32_t c = e2m1_code(x[0], sc) | (e2m1_code(x[1], sc) << 4) | (e2m1_code(x[2], sc) << 8) |
+                       (e2m1_code(x[3], sc) << 12);
+    if (lane < kSsPad / 4) reinterpret_cast<uint16_t *>(xi4 + w * kSsCodeBytes)[lane] = (uint16_t)c;
+    if (lane == 0) xi_scale[w] = sc;
+}
+
+// P[sh][row][j]: per (sequence, KV head) the G projected queries p_g = U^T q_g
+// (fp32, one FMA per term in dim order) as a bf16 value (rows 0..G-1) and the
+// bf16 residual p_g - value (rows G..2G-1); dims past sd and rows past 2G zero.
+// One warp per (sh, g); lane l takes dims l, l + 32, l + 64 (< 96).
+__global__ void __launch_bounds__(256) query_project_split_kernel(const __nv_bfloat16 *__restrict__ Q,
+                                                                  const float *__restrict__ U,
+                                                                  __nv_bfloat16 *__restrict__ P, int n_sh,
+                                                                  int n_kv, int n_q, int G, int sd) {
+    const int item = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (item >= n_sh * kFtN) return;
+    const int sh = item / kFtN, rrow = item - sh * kFtN;
+    __nv_bfloat16 *out = P + ((size_t)sh * kFtN + rrow) * kBdD;
+    if (rrow >= G) {                             // residual rows are written by their g; zero the rest
+        if (rrow >= 2 * G)
+            for (int j = lane; j < kBdD; j += 32) out[j] = __float2bfloat16_rn(0.0f);
+        return;
+    }
+    const int seq = sh / n_kv, h = sh - seq * n_kv;
+    const __nv_bfloat16 *q = Q + ((size_t)seq * n_q + h * G + rrow) * kBdD;
+    __nv_bfloat16 *res = P + ((size_t)sh * kFtN + G + rrow) * kBdD;
+    for (int j = lane; j < kBdD; j += 32) {
+        float acc = 0.0f;
+        if (j < sd) {
+#pragma unroll 16           // the loads of U run ahead of the dependent FMA chain
+            for (int dd = 0; dd < kBdD; ++dd) acc = fmaf(__ldg(U + (size_t)dd * sd + j), __bfloat162float(q[dd]), acc);
+        }
+        const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+        out[j] = hi;
+        res[j] = __float2bfloat16_rn(acc - __bfloat162float(hi));
+    }
+}
+
+}  // namespace crs
+
+using namespace crs;
+
+extern "C" int crs_block_quantize_ss(const crs_block_params *p, const float *mu, const float *xi_ss, int sd,
+                                     void *mu16, uint8_t *xi4, float *xi_scale, void *stream) {
+    if (!p) return CRS_ERR_INVALID_ARG;
+    crs_block_params b = *p;
+    b.blk_begin = 0;
+    b.blk_end = 0;
+    int st = bd_validate(&b);
+    if (st) return st;
+    if (sd < 1 || sd > kBdD) return CRS_ERR_INVALID_ARG;
+    if (sd > kSsPad) return CRS_ERR_UNSUPPORTED;
+    if (!mu || !xi_ss || !mu16 || !xi4 || !xi_scale) return CRS_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mu) | reinterpret_cast<uintptr_t>(mu16) | reinterpret_cast<uintptr_t>(xi4)) &
+        15)
+        return CRS_ERR_INVALID_ARG;
+    const long long n_mu = (long long)p->n_seq * p->n_kv * (p->T / p->L);
+    const long long n_xi = n_mu * p->rank;
+    if (n_mu == 0) return CRS_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        ProfScope _ps(K_BLK_QUANTIZE, s);
+        block_quantize_ss_kernel<<<(unsigned)ceil_div_ll(n_mu + n_xi, 8), 256, 0, s>>>(
+            mu, xi_ss, static_cast<__nv_bfloat16 *>(mu16), xi4, xi_scale, n_mu, n_xi, sd);
+    }
+    CRS_CHECK_LAUNCH();
+    return CRS_OK;
+}
+
+extern "C" size_t crs_block_select_fp4_ss_workspace_size(const crs_block_sel_params *p, int sd) {
+    const size_t sc = crs_block_select_workspace_size(p);
+    if (sc == 0 || sd < 1 || sd > kSsPad) return 0;
+    return ((sc + 255) & ~size_t(255)) + (size_t)p->b.n_seq * p->b.n_kv * kFtN * kBdD * 2;
+}
+
+extern "C" int crs_block_select_fp4_ss(const crs_block_sel_params *p, const void *Q, const float *U, int sd,
+                                       const void *mu16, const uint8_t *xi4, const float *xi_scale,
+                                       int32_t *tok_idx, int32_t *tok_count, void *ws, size_t ws_bytes,
+                                       void *stream) {
+    int st = bs_validate(p);
+    if (st) return st;
+    if (!Q || !U || !mu16 || !xi4 || !xi_scale || !tok_idx || !tok_count) return CRS_ERR_INVALID_ARG;
+    const int G = p->n_q / p->b.n_kv, R = p->b.rank;
+    if (R < 1 || sd < 1 || sd > kBdD) return CRS_ERR_INVALID_ARG;
+    if (R > kFtMaxR || sd > kSsPad || 2 * G > kFtN) return CRS_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(mu16) | reinterpret_cast<uintptr_t>(xi4)) &
+        15)
+        return CRS_ERR_INVALID_ARG;
+    const size_t need = crs_block_select_fp4_ss_workspace_size(p, sd);
+    if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int n_full = p->b.T / p->b.L;
+    float *sc = static_cast<float *>(ws);
+    __nv_bfloat16 *P = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) +
+                                                         ((crs_block_select_workspace_size(p) + 255) & ~size_t(255)));
+    const int n_sh = p->b.n_seq * p->b.n_kv;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tc::tensor_map_encoder();
+    if (!enc) return CRS_ERR_CUDA;
+    CUtensorMap tmu, tq, tp;
+    auto encode = [&](CUtensorMap *m, const void *base, cuuint64_t rows, cuuint32_t box_rows) {
+        cuuint64_t dims[2] = {(cuuint64_t)kBdD, rows};
+        cuuint64_t strides[1] = {(cuuint64_t)kBdD * 2};
+        cuuint32_t box[2] = {64, box_rows};
+        cuuint32_t estr[2] = {1, 1};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!encode(&tmu, mu16, (cuuint64_t)n_sh * n_full, kFtM) ||
+        !encode(&tq, Q, (cuuint64_t)p->b.n_seq * p->n_q, (cuuint32_t)G) ||
+        !encode(&tp, P, (cuuint64_t)n_sh * kFtN, kFtN))
+        return CRS_ERR_CUDA;
+    FtArgs fa;
+    fa.mu16 = static_cast<const __nv_bfloat16 *>(mu16);
+    fa.xi4 = xi4;
+    fa.xi_scale = xi_scale;
+    fa.sc_out = sc;
+    fa.n_kv = p->b.n_kv;
+    fa.n_q = p->n_q;
+    fa.G = G;
+    fa.R = R;
+    fa.n_full = n_full;
+    fa.tiles_per_sh = ceil_div(n_full, kFtM);
+    fa.total_tiles = n_sh * fa.tiles_per_sh;
+    fa.scale = p->scale;
+    fa.code_bytes = kSsCodeBytes;
+    fa.split = 1;
+    int dev = 0, sms = 148;
+    CRS_TRY_CUDA(cudaGetDevice(&dev));
+    CRS_TRY_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    fa.tiles_per_cta = ceil_div(fa.total_tiles, max(1, sms));
+    const int grid = ceil_div(fa.total_tiles, fa.tiles_per_cta);
+    const size_t smem_s = sizeof(FtSmem) + 1024;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_fp4_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
+    {
+        ProfScope _ps(K_BLK_SCORE, s);
+        _ps.more(1);                              // projection + scorer
+        query_project_split_kernel<<<ceil_div(n_sh * kFtN, 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(Q), U, P, n_sh, p->b.n_kv, p->n_q, G, sd);
+        block_score_fp4_tc_kernel<<<grid, kFtThreads, smem_s, s>>>(tmu, tq, tp, fa);
     }
     CRS_CHECK_LAUNCH();
     return launch_block_pick(p, sc, tok_idx, tok_count, s);

@@ -486,6 +486,31 @@ int crs_block_select_ss(const crs_block_sel_params *p, const void *Q, const floa
                         const float *mu, const float *xi_ss, int32_t *tok_idx, int32_t *tok_count,
                         void *ws, size_t ws_bytes, void *stream);
 
+/* The pages' deployed descriptor ([P5] "子空间方法" Eq.(17)-(18) with §5.5
+ * "量化" and the delivered row of Table 3: s ~ 85, r = 4, FP4): the block mean
+ * in bf16 (full space) and the r scaled eigenvectors of U^T Sigma_b U in E2M1
+ * FP4 with one fp32 scale each, scored with the projected query.
+ * crs_block_quantize_ss: mu [n_seq, n_kv, T/L, D] f32 and xi_ss [n_seq, n_kv,
+ *   T/L, rank, sd] f32 (from crs_block_describe_ss) -> mu16 (bf16, round to
+ *   nearest even), xi4 [n_seq, n_kv, T/L, rank, 48] bytes (codes of dims
+ *   0..95, two per byte, the even dim in the low nibble, dims >= sd zero; the
+ *   code and scale rule of crs_block_quantize), xi_scale [.., rank] f32.
+ *   sd <= 96 (else CRS_ERR_UNSUPPORTED); mu, mu16, xi4 16-byte aligned.
+ * crs_block_select_fp4_ss: the crs_block_select rule with
+ *   s_{g,b} = qt . mu16_b + 1/2 sum_i (sigma_i code_i . U^T qt)^2, qt = scale q_g;
+ *   U [D, sd] f32 row-major.  The products run on the tensor cores: Q . mu16
+ *   (both exact in bf16) and code_i . p_g with p_g = U^T q_g (fp32, one FMA per
+ *   term in dim order) split into a bf16 value and a bf16 residual (two query
+ *   columns each), accumulated in fp32.  G = n_q / n_kv <= 8, rank <= 4 (else
+ *   CRS_ERR_UNSUPPORTED); Q, mu16, xi4 16-byte aligned.  Workspace:
+ *   crs_block_select_fp4_ss_workspace_size (scores + projected queries). */
+int crs_block_quantize_ss(const crs_block_params *p, const float *mu, const float *xi_ss, int sd, void *mu16,
+                          uint8_t *xi4, float *xi_scale, void *stream);
+size_t crs_block_select_fp4_ss_workspace_size(const crs_block_sel_params *p, int sd);
+int crs_block_select_fp4_ss(const crs_block_sel_params *p, const void *Q, const float *U, int sd, const void *mu16,
+                            const uint8_t *xi4, const float *xi_scale, int32_t *tok_idx, int32_t *tok_count,
+                            void *ws, size_t ws_bytes, void *stream);
+
 /* ====================================================================== *
  * Quest box selector ([P5] Quest section, Eq.(23)-(24), Table 1).
  * crs_block_quest_describe: per complete block b of L keys and KV head h the

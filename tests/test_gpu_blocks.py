@@ -362,3 +362,76 @@ def test_select_one_query_head_per_kv_head(crs, cuda_dev):
     o_tok, o_cnt, o_blk, o_bs = oracle.block_select(_np(case["Q"]), mu.double().cpu().numpy(),
                                                     xi.double().cpu().numpy(), p["T"], L, 12, 64)
     _check_select(tok.cpu().numpy(), cnt.cpu().numpy(), o_tok, o_cnt, o_blk, o_bs, L, p["T"], 64, 12, "G1")
+
+
+def _pad96(x):
+    out = np.zeros(x.shape[:-1] + (96,), dtype=np.float32)
+    out[..., : x.shape[-1]] = x
+    return out
+
+
+def test_quantize_ss_matches_oracle_bit_exact(crs, cuda_dev):
+    """The deployed descriptor's codes ([P5] "量化" on the subspace eigenvectors): the
+    codes and scales of each s = 85 vector equal the oracle's for the same vector padded
+    with zeros to the 96 stored dims (zeros change neither the scale nor any code);
+    the mean is bf16 round-to-nearest-even."""
+    case = workloads.block_decode_case(n_seq=2, T=32 * 41, seed=44, device=cuda_dev)
+    p = case["params"]
+    U = workloads.query_subspace(128, 85, device=cuda_dev)
+    mu, xi = crs.block_describe_ss(case["K"], p["L"], p["rank"], U)
+    mu16, xi4, xs = crs.block_quantize_ss(mu, xi, p["T"], p["L"])
+    torch.cuda.synchronize()
+    o_codes, o_scale = oracle.fp4_quantize(_pad96(xi.cpu().numpy()))
+    assert np.array_equal(xi4.cpu().numpy(), o_codes)
+    assert np.array_equal(xs.cpu().numpy(), o_scale)
+    assert torch.equal(mu16.cpu(), mu.cpu().to(torch.bfloat16))
+
+
+def _select_fp4_ss_and_check(crs, case, U, top, win, seqs=None, what=""):
+    p = case["params"]
+    T, L, r = p["T"], p["L"], p["rank"]
+    sd = U.shape[1]
+    mu, xi = crs.block_describe_ss(case["K"], L, r, U)
+    mu16, xi4, xs = crs.block_quantize_ss(mu, xi, T, L)
+    tok, cnt = crs.block_select_fp4_ss(case["Q"], U, mu16, xi4, xs, T, L, top, win)
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    seqs = list(range(p["n_seq"])) if seqs is None else seqs
+    omu = _np(mu16)[seqs]
+    oxi = oracle.fp4_dequantize(xi4.cpu().numpy()[seqs], xs.cpu().numpy()[seqs])[..., :sd]
+    o_tok, o_cnt, o_blk, o_bs = oracle.block_select_ss(_np(case["Q"])[seqs], U.double().cpu().numpy(), omu, oxi,
+                                                       T, L, top, win)
+    _check_select(tok.cpu().numpy()[seqs], cnt.cpu().numpy()[seqs], o_tok, o_cnt, o_blk, o_bs, L, T, win, top,
+                  what)
+
+
+@pytest.mark.parametrize("n_q,n_kv,T,top,win,sd", [(32, 4, 4096, 16, 256, 85), (16, 4, 32 * 300 + 5, 20, 64, 48),
+                                                   (4, 4, 32 * 90, 9, 100, 96), (8, 8, 32 * 129, 7, 0, 85)])
+def test_select_fp4_ss_matches_oracle(crs, cuda_dev, n_q, n_kv, T, top, win, sd):
+    """The deployed descriptor scored on the tensor cores equals the oracle's subspace
+    selection over the same dequantised descriptors (set rule at the cutoff)."""
+    case = workloads.block_decode_case(n_seq=3, T=T, n_kv_heads=n_kv, n_q_heads=n_q, seed=T + sd + 1,
+                                       device=cuda_dev)
+    U = workloads.query_subspace(128, sd, seed=sd, device=cuda_dev)
+    _select_fp4_ss_and_check(crs, case, U, top, win, what=f"fp4-ss{sd}-G{n_q // n_kv}")
+
+
+def test_select_fp4_ss_full_config_sampled(crs, cuda_dev):
+    """The block-sparse decode workload (32 sequences, T = 32768, 32 query heads over 4
+    KV heads) on the deployed descriptor (s = 85, r = 4, FP4): 6 sequences checked."""
+    case = workloads.block_decode_case(device=cuda_dev)
+    U = workloads.query_subspace(128, 85, device=cuda_dev)
+    p = case["params"]
+    _select_fp4_ss_and_check(crs, case, U, p["top_blocks"], p["window"], seqs=[0, 5, 11, 17, 26, 31],
+                             what="fp4-ss85-full")
+
+
+def test_select_fp4_ss_rejects_wide_groups(crs, cuda_dev):
+    """More than 8 query heads per KV head leave no room for the split query columns."""
+    case = workloads.block_decode_case(n_seq=1, T=32 * 64, n_kv_heads=2, n_q_heads=32, seed=3, device=cuda_dev)
+    p = case["params"]
+    U = workloads.query_subspace(128, 85, device=cuda_dev)
+    mu, xi = crs.block_describe_ss(case["K"], p["L"], p["rank"], U)
+    mu16, xi4, xs = crs.block_quantize_ss(mu, xi, p["T"], p["L"])
+    with pytest.raises(crs.CrsError):
+        crs.block_select_fp4_ss(case["Q"], U, mu16, xi4, xs, p["T"], p["L"], 8, 64)
