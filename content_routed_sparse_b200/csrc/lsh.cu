@@ -536,35 +536,44 @@ __global__ void lsh_combine_kernel(const float *__restrict__ o_ws, const float *
 // sum_j 2^(s_ij - M_i) v_j over the union of the rounds' candidates, acc_L the matching
 // sum of weights, acc_M the shift M_i (log2 units); O /= L and lse = (M_i + log2 L) ln 2.
 // Rows the attention kept in the per-round form (acc_M = +inf) are merged as above.
+// A thread takes four 16-byte groups of one row (a quarter row for d = 64) and
+// issues all of its loads before using any: the pass is bound by how many bytes
+// are in flight.
 template <int DH>
 __global__ void lsh_finish_kernel(const float *__restrict__ o_ws, const float *__restrict__ lse_ws,
                                   const float *__restrict__ acc_L, const float *__restrict__ acc_M,
                                   const int32_t *__restrict__ valid_len, float *__restrict__ O,
                                   float *__restrict__ lse_out, int BH, int H, int n, int rounds) {
-    constexpr int G4 = DH / 4;
+    constexpr int G4 = DH / 4;                  // float4 groups per row
+    constexpr int PER = G4 >= 4 ? 4 : G4;       // groups per thread
+    constexpr int TPR = G4 / PER;               // threads per row
     const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gt >= (long long)BH * n * G4) return;
-    const int g = (int)(gt % G4);
-    const long long rowi = gt / G4;
+    if (gt >= (long long)BH * n * TPR) return;
+    const int g0 = (int)(gt % TPR) * PER;
+    const long long rowi = gt / TPR;
     const int bh = (int)(rowi / n), pos = (int)(rowi - (long long)bh * n);
+    const float m = __ldcs(acc_M + rowi);
+    const float L = __ldcs(acc_L + rowi);
+    float4 *o = reinterpret_cast<float4 *>(O + (size_t)rowi * DH) + g0;
+    float4 v[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) v[u] = __ldcs(o + u);
     const int vl = valid_len ? valid_len[bh / H] : n;
-    const float m = acc_M[rowi];
     if (m == INFINITY) {
-        lsh_merge_rounds<DH>(o_ws, lse_ws, O, lse_out, BH, n, rounds, bh, pos, g, pos >= vl);
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+            lsh_merge_rounds<DH>(o_ws, lse_ws, O, u == 0 ? lse_out : nullptr, BH, n, rounds, bh, pos, g0 + u,
+                                 pos >= vl);
         return;
     }
-    const float L = acc_L[rowi];
-    float4 *o = reinterpret_cast<float4 *>(O + (size_t)rowi * DH) + g;
-    if (pos >= vl || !(L > 0.0f)) {
-        *o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (lse_out && g == 0) lse_out[rowi] = -INFINITY;
-        return;
+    const bool has = pos < vl && L > 0.0f;
+    const float inv = has ? 1.0f / L : 0.0f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        v[u].x *= inv; v[u].y *= inv; v[u].z *= inv; v[u].w *= inv;
+        o[u] = v[u];
     }
-    const float inv = 1.0f / L;
-    float4 v = *o;
-    v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
-    *o = v;
-    if (lse_out && g == 0) lse_out[rowi] = (m + log2f(L)) * 0.6931471805599453f;
+    if (lse_out && g0 == 0) lse_out[rowi] = has ? (m + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
 // ------------------------------------------------------------ host side --
@@ -598,17 +607,27 @@ extern "C" int crs_lsh_route(const crs_lsh_params *p, const void *X, const float
     const size_t smem = ((size_t)p->d * half + (size_t)kHashTok * (p->d + 1)) * sizeof(float);
     if (smem > 200 * 1024) return CRS_ERR_UNSUPPORTED;
     dim3 grid(ceil_div(p->n, kHashTok), p->n_rounds, p->B * p->H);
-    if (p->dtype == CRS_BF16 && p->d == kHtD && half == kHtHalf && p->n_rounds <= 4) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tc::tensor_map_encoder();
+    const long long rows_all = (long long)p->B * p->H * p->n;
+    if (p->dtype == CRS_BF16 && p->d == kHtD && half == kHtHalf && p->n_rounds <= 4 && enc &&
+        !(reinterpret_cast<uintptr_t>(X) & 15) && rows_all + kHtM < 0x7fffffffLL) {
         // tensor-core filter with the exact chain as fallback (identical bucket ids)
-        const int N = p->n_rounds * kHtHalf;
-        const size_t hsm = ht_smem_bytes(N) + 1024;
+        CUtensorMap tx;
+        cuuint64_t dims[2] = {(cuuint64_t)kHtD, (cuuint64_t)rows_all};
+        cuuint64_t strides[1] = {(cuuint64_t)kHtD * 2};
+        cuuint32_t box[2] = {(cuuint32_t)kHtD, (cuuint32_t)kHtM};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CRS_ERR_CUDA;
+        const size_t hsm = sizeof(HtSmem) + 1024;
         CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_hash_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)hsm));
         const int tpc = ht_tiles_per_cta(p->n, p->B * p->H);
         dim3 gh(ceil_div(ceil_div(p->n, kHtM), tpc), p->B * p->H);
         ProfScope _ps(K_LSH_HASH, s);
-        lsh_hash_tc_kernel<<<gh, kHtThreads, hsm, s>>>(static_cast<const __nv_bfloat16 *>(X), R, bucket,
-                                                       p->H, p->n, p->n_rounds, tpc);
+        lsh_hash_tc_kernel<<<gh, kHtThreads, hsm, s>>>(tx, R, bucket, p->H, p->n, p->n_rounds, tpc);
     } else if (p->d == 64 && (half == 32 || half == 8)) {
         // specialised kernel: one CTA per 128 tokens covers every round
         dim3 g2(ceil_div(p->n, kHashTok), 1, p->B * p->H);
@@ -705,7 +724,8 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
             }
             CRS_CHECK_LAUNCH();
             if (acc) {
-                const long long work = (long long)p.B * p.H * p.n * (DH / 4);
+                constexpr int kPer = DH / 4 >= 4 ? 4 : DH / 4;
+                const long long work = (long long)p.B * p.H * p.n * (DH / 4 / kPer);
                 {
                     ProfScope _ps(K_LSH_COMBINE, s);
                     lsh_finish_kernel<DH><<<(unsigned)ceil_div_ll(work, 256), 256, 0, s>>>(

@@ -9,10 +9,10 @@
 // fallback:
 //   1. approximate u~ = x (R_hi + R_lo) on tcgen05 (R split into two bf16
 //      parts, x exact in bf16, every product exact, fp32 accumulation in
-//      tensor memory), and S~ = |x| |R| (the absolute sums that bound every
-//      rounding error), for all rounds at once (N = 32 x rounds columns);
-//   2. per (token, round): with E_k = 2^-13 S~_k, the largest |u~_k| wins by
-//      more than E_k1 + E_k2 over the runner-up and by more than E_k1 over its own
+//      tensor memory) for all rounds at once (N = 32 x rounds columns);
+//   2. per (token, round): with E_k = 2^-12 |x| |r_k| (Cauchy-Schwarz bounds
+//      S_k = sum_i |x_i| |r_ik| by |x| |r_k|), the largest |u~_k| wins by more
+//      than E_k1 + E_k2 over the runner-up and by more than E_k1 over its own
 //      negation -> it is the argmax of the chain values as well (see the bound
 //      below), and its sign picks the +u or -u half;
 //   3. otherwise (a near tie, or all u~ ~ 0) the warp recomputes that token's
@@ -20,29 +20,40 @@
 //      maximum as the definition does.
 // The bound: |u~_k - u_k| <= |x . (R - R_hi - R_lo)| + (tensor-core
 // accumulation) + (chain rounding) <= (2^-16 + 128 * 2^-22 + gamma_64) S_k
-// < 5e-5 S_k, S_k = sum_i |x_i| |r_ik| <= 1.01 S~_k (|R| rounded to bf16 at
-// most 2^-8 relative); E_k = 2^-13 S~_k >= 1.2e-4 S~_k covers it with a factor
-// 2.4.  A winner by more than the two bounds therefore wins in the chain values.
+// < 5e-5 S_k <= 5e-5 |x| |r_k|; E_k = 2^-12 |x| |r_k| (norms in fp32) covers it
+// with a factor of about 4.9.  A winner by more than the two bounds therefore
+// wins in the chain values.
 //
-// One CTA (4 warps, one token row per thread in the epilogue) walks several
-// 128-token tiles of one (batch, head): R is split into its operand tiles once,
-// the next X tile is prefetched while the current one is in the epilogue.
+// Persistent, warp-specialised CTA walking the 128-token tiles of one
+// (batch, head): warp 0 loads X tiles with TMA into a 3-stage ring, warp 1
+// issues the MMAs into two tensor-memory buffers, warps 2..5 (one token row
+// per thread) read the scores, decide the buckets and release the buffers.
+// R is split into its operand tiles once per CTA.
 #include "common.cuh"
 #include "tc.cuh"
 
 namespace crs {
 
 constexpr int kHtM = 128;                 // tokens per tile (MMA M)
-constexpr int kHtThreads = 128;
 constexpr int kHtHalf = 32;               // b / 2
 constexpr int kHtD = 64;
-constexpr float kHtErr = 1.220703125e-4f; // 2^-13
+constexpr int kHtMaxN = 128;              // 32 x rounds, rounds <= 4
+constexpr int kHtStages = 3;
+constexpr int kHtEpiWarps = 4;
+constexpr int kHtThreads = 32 * (2 + kHtEpiWarps);
+constexpr float kHtErr = 2.44140625e-4f;  // 2^-12
 constexpr uint64_t kHtWaitNs = 1000000000ull;
+constexpr uint32_t kHtSuspendNs = 256;
 
-__host__ __device__ constexpr size_t ht_smem_bytes(int N) {
-    // X double buffer, |X|, three B tiles (R_hi, R_lo, |R|) of N rows, barrier + TMEM slot
-    return 2 * 16384 + 16384 + 3 * (size_t)N * 128 + 64;
-}
+struct HtSmem {
+    unsigned char x[kHtStages][kHtM * 128];   // X tiles, 128B swizzle
+    unsigned char bhi[kHtMaxN * 128];         // B operand: R_hi, row r*32 + k = column k of R_{h,r}
+    unsigned char blo[kHtMaxN * 128];         //            R_lo
+    float rnorm[kHtMaxN];                     // |r_k| per column
+    uint64_t xfull[kHtStages], xempty[kHtStages], tfull[2], tempty[2];
+    uint32_t tmem_base;
+    int fail;
+};
 
 __device__ __forceinline__ float ht_x(const unsigned char *xt, int row, int t) {
     const uint16_t b = *reinterpret_cast<const uint16_t *>(xt + tc::sw128(row, t >> 3) + (t & 7) * 2);
@@ -50,160 +61,204 @@ __device__ __forceinline__ float ht_x(const unsigned char *xt, int row, int t) {
 }
 
 __global__ void __launch_bounds__(kHtThreads, 2)
-lsh_hash_tc_kernel(const __nv_bfloat16 *__restrict__ X, const float *__restrict__ R,
+lsh_hash_tc_kernel(const __grid_constant__ CUtensorMap tx, const float *__restrict__ R,
                    int32_t *__restrict__ bucket, int H, int n, int rounds, int tiles_per_cta) {
     extern __shared__ unsigned char ht_raw[];
     const uint32_t mis = smem_u32(ht_raw) & 1023u;
-    unsigned char *base = ht_raw + ((1024u - mis) & 1023u);
+    HtSmem &S = *reinterpret_cast<HtSmem *>(ht_raw + ((1024u - mis) & 1023u));
     const int N = rounds * kHtHalf;
-    unsigned char *xbuf[2] = {base, base + 16384};
-    unsigned char *xab = base + 32768;
-    unsigned char *bhi = base + 49152;
-    unsigned char *blo = bhi + (size_t)N * 128;
-    unsigned char *bab = blo + (size_t)N * 128;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(bab + (size_t)N * 128);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
-
     const int bh = blockIdx.y, h = bh % H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_tiles = (n + kHtM - 1) / kHtM;
     const int t_first = blockIdx.x * tiles_per_cta;
-    const int t_end = min(n_tiles, t_first + tiles_per_cta);
-    if (t_first >= t_end) return;                 // uniform over the CTA
-    const __nv_bfloat16 *Xb = X + (size_t)bh * n * kHtD;
+    const int nt = min(n_tiles, t_first + tiles_per_cta) - t_first;
+    if (nt <= 0) return;                          // uniform over the CTA
     const float *Rh = R + (size_t)h * rounds * kHtD * kHtHalf;
 
-    auto load_x = [&](int tile, unsigned char *dst) {
-        const int i0 = tile * kHtM;
+    if (tid == 0) {
+        for (int i = 0; i < kHtStages; ++i) {
+            tc::mbar_init(&S.xfull[i], 1);
+            tc::mbar_init(&S.xempty[i], kHtEpiWarps);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&S.tfull[i], 1);
+            tc::mbar_init(&S.tempty[i], kHtEpiWarps);
+        }
+        tc::mbar_fence_init();
+        S.fail = 0;
+    }
+    // B operand tiles (K-major) and column norms; eight loads in flight per thread
+    for (int e0 = tid; e0 < N * kHtD; e0 += 8 * kHtThreads) {
+        float v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int e = tid + u * kHtThreads;
-            const int row = e >> 3, ch = e & 7;
-            const bool ok = i0 + row < n;
-            cp_async16_zfill(dst + tc::sw128(row, ch), Xb + (size_t)(ok ? i0 + row : 0) * kHtD + ch * 8, ok);
+            const int e = e0 + u * kHtThreads;
+            v[u] = e < N * kHtD ? __ldg(Rh + e) : 0.0f;
         }
-        cp_async_commit();
-    };
-    load_x(t_first, xbuf[0]);
-
-    // B operand tiles, K-major: row r*32 + k holds column k of R_{h,r} (64 values)
-    for (int e = tid; e < N * kHtD; e += kHtThreads) {
-        const int k = e & (kHtHalf - 1), t = (e >> 5) & (kHtD - 1), r = e >> 11;
-        const float v = Rh[e];
-        const uint32_t off = tc::sw128(r * kHtHalf + k, t >> 3) + (t & 7) * 2;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-        const __nv_bfloat16 ab = __float2bfloat16_rn(fabsf(v));
-        *reinterpret_cast<__nv_bfloat16 *>(bhi + off) = hi;
-        *reinterpret_cast<__nv_bfloat16 *>(blo + off) = lo;
-        *reinterpret_cast<__nv_bfloat16 *>(bab + off) = ab;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * kHtThreads;
+            if (e >= N * kHtD) break;
+            const int k = e & (kHtHalf - 1), t = (e >> 5) & (kHtD - 1), r = e >> 11;
+            const uint32_t off = tc::sw128(r * kHtHalf + k, t >> 3) + (t & 7) * 2;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v[u]);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(v[u] - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16 *>(S.bhi + off) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(S.blo + off) = lo;
+        }
     }
-    const uint32_t ncols = N * 2 <= 32 ? 32u : (N * 2 <= 64 ? 64u : (N * 2 <= 128 ? 128u : (N * 2 <= 256 ? 256u : 512u)));
-    if (warp == 0) tc::tmem_alloc(tslot, ncols);
-    if (tid == 0) {
-        tc::mbar_init(bar, 1);
-        tc::mbar_fence_init();
+    for (int c = tid; c < N; c += kHtThreads) {
+        const int r = c / kHtHalf, k = c - r * kHtHalf;
+        const float *col = Rh + (size_t)r * kHtD * kHtHalf + k;
+        float ss = 0.0f;
+#pragma unroll 16
+        for (int t = 0; t < kHtD; ++t) ss = fmaf(col[t * kHtHalf], col[t * kHtHalf], ss);
+        S.rnorm[c] = sqrtf(ss);
     }
+    if (warp == 1) tc::tmem_alloc(&S.tmem_base, 2 * kHtMaxN);
+    tc::fence_proxy_async();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
-    const uint32_t tmem = *tslot;
-    const uint32_t idesc = tc::idesc_bf16_f32(kHtM, (uint32_t)N, 0, 0);
+    const uint32_t tmem = S.tmem_base;
+    const volatile int *abort_flag = &S.fail;
 
-    for (int tile = t_first, it = 0; tile < t_end; ++tile, ++it) {
-        unsigned char *xa = xbuf[it & 1];
-        cp_async_wait<0>();
-        __syncthreads();                          // X tile landed; the last epilogue is done
-        // |X|: clear the sign bits
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = tid + u * kHtThreads;
-            const uint32_t off = tc::sw128(e >> 3, e & 7);
-            uint4 v = *reinterpret_cast<const uint4 *>(xa + off);
-            v.x &= 0x7fff7fffu; v.y &= 0x7fff7fffu; v.z &= 0x7fff7fffu; v.w &= 0x7fff7fffu;
-            *reinterpret_cast<uint4 *>(xab + off) = v;
-        }
-        tc::fence_proxy_async();
-        tc::fence_before();
-        __syncthreads();
-        tc::fence_after();
-        if (tid == 0) {
-            const uint32_t xs = smem_u32(xa), xb = smem_u32(xab);
-            const uint32_t hs = smem_u32(bhi), ls = smem_u32(blo), as = smem_u32(bab);
-#pragma unroll
-            for (int k = 0; k < kHtD / 16; ++k)
-                tc::mma_bf16(tmem, tc::smem_desc(xs + k * 32, 16, 1024, tc::kLayoutSW128),
-                             tc::smem_desc(hs + k * 32, 16, 1024, tc::kLayoutSW128), idesc, k > 0 ? 1u : 0u);
-#pragma unroll
-            for (int k = 0; k < kHtD / 16; ++k)
-                tc::mma_bf16(tmem, tc::smem_desc(xs + k * 32, 16, 1024, tc::kLayoutSW128),
-                             tc::smem_desc(ls + k * 32, 16, 1024, tc::kLayoutSW128), idesc, 1u);
-#pragma unroll
-            for (int k = 0; k < kHtD / 16; ++k)
-                tc::mma_bf16(tmem + (uint32_t)N, tc::smem_desc(xb + k * 32, 16, 1024, tc::kLayoutSW128),
-                             tc::smem_desc(as + k * 32, 16, 1024, tc::kLayoutSW128), idesc, k > 0 ? 1u : 0u);
-            tc::commit(bar);
-        }
-        // the other buffer was last read by the previous tile's MMAs, which completed
-        if (tile + 1 < t_end) load_x(tile + 1, xbuf[(it + 1) & 1]);
-        const bool ok = tc::mbar_wait_bounded(bar, (uint32_t)(it & 1), kHtWaitNs, K_LSH_HASH, 1, 10000u, true);
-        if (__syncthreads_or(!ok)) {
-            tc::mbar_wait_bounded(bar, (uint32_t)(it & 1), kHtWaitNs, K_LSH_HASH, 2);   // drain
-            cp_async_wait<0>();
-            break;
-        }
-        tc::fence_after();
-
-        const int row = warp * 32 + lane;
-        const int i = tile * kHtM + row;
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        for (int r = 0; r < rounds; ++r) {
-            uint32_t uv[32], sv[32];
-            tc::tmem_ld32(trow + (uint32_t)(r * kHtHalf), uv);
-            tc::tmem_ld32(trow + (uint32_t)(N + r * kHtHalf), sv);
-            tc::tmem_ld_wait();
-            // the two largest |u~_k| with their absolute sums (error scales)
-            float m1 = -1.0f, m2 = -1.0f, s1 = 0.0f, s2 = 0.0f, u1 = 0.0f;
-            int k1 = 0;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const float uk = __uint_as_float(uv[k]), sk = __uint_as_float(sv[k]);
-                const float a = fabsf(uk);
-                if (a > m1) { m2 = m1; s2 = s1; m1 = a; s1 = sk; k1 = k; u1 = uk; }
-                else if (a > m2) { m2 = a; s2 = sk; }
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            if (*reinterpret_cast<volatile uint32_t *>(&g_force_wait_timeout) != 0u) {
+                // test switch: give up before the first load (nothing is in flight)
+                raise_error(CRS_DEVERR_TIMEOUT);
+                diag_record(K_LSH_HASH, 1, 0u, threadIdx.x, 0u, 0u);
+                atomicOr(&S.fail, 1);
             }
-            // every other entry of [u~ ; -u~] is at most m2 (or -m1 for the winner's own
-            // negation); the winner is certain when it leads both by the two bounds
-            int bk = u1 > 0.0f ? k1 : kHtHalf + k1;
-            const float E1 = kHtErr * s1, E2 = kHtErr * s2;
-            const bool amb = (m2 >= m1 - (E1 + E2)) || (m1 <= E1);
-            // exact chains for the undecided tokens of this warp, one token at a time
-            uint32_t pend = __ballot_sync(0xffffffffu, amb && i < n);
-            const float *Rr = Rh + (size_t)r * kHtD * kHtHalf;
-            while (pend) {
-                const int l = __ffs(pend) - 1;
-                pend &= pend - 1;
-                const int rl = warp * 32 + l;
-                float rv[kHtD];                       // column `lane` of R_{h,r}, all loads in flight
-#pragma unroll
-                for (int t = 0; t < kHtD; ++t) rv[t] = __ldg(Rr + t * kHtHalf + lane);
-                float u = 0.0f;
-#pragma unroll
-                for (int t = 0; t < kHtD; ++t) u = __fmaf_rn(ht_x(xa, rl, t), rv[t], u);
-                const float bp = warp_max(u);
-                const int ap = __ffs(__ballot_sync(0xffffffffu, u == bp)) - 1;
-                const float bn = warp_max(-u);
-                const int an = __ffs(__ballot_sync(0xffffffffu, -u == bn)) - 1;
-                if (lane == l) bk = (bp >= bn) ? ap : kHtHalf + an;
+            for (int i = 0; i < nt && !*abort_flag; ++i) {
+                const int s = i % kHtStages, u = i / kHtStages;
+                if (u > 0 && !tc::mbar_wait_bounded(&S.xempty[s], (u - 1) & 1, kHtWaitNs, K_LSH_HASH, 2,
+                                                    kHtSuspendNs, false, abort_flag)) {
+                    atomicOr(&S.fail, 1);
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&S.xfull[s], kHtM * 128);
+                tc::tma_load_2d(S.x[s], &tx, 0, bh * n + (t_first + i) * kHtM, &S.xfull[s]);
+                ++issued;
             }
-            if (i < n) bucket[((size_t)bh * rounds + r) * n + i] = bk;
+            // the loads in flight land before the CTA may leave
+            for (int i = max(0, issued - kHtStages); i < issued; ++i)
+                tc::mbar_wait_bounded(&S.xfull[i % kHtStages], (i / kHtStages) & 1, kHtWaitNs, K_LSH_HASH, 3);
         }
-        tc::fence_before();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16_f32(kHtM, (uint32_t)N, 0, 0);
+            int last = -1;
+            for (int i = 0; i < nt; ++i) {
+                const int s = i % kHtStages, u = i / kHtStages, b = i & 1, v = i >> 1;
+                bool ok = tc::mbar_wait_bounded(&S.xfull[s], u & 1, kHtWaitNs, K_LSH_HASH, 4, kHtSuspendNs,
+                                                false, abort_flag);
+                if (ok && v > 0)
+                    ok = tc::mbar_wait_bounded(&S.tempty[b], (v - 1) & 1, kHtWaitNs, K_LSH_HASH, 5, kHtSuspendNs,
+                                               false, abort_flag);
+                if (!ok) {
+                    atomicOr(&S.fail, 1);
+                    break;
+                }
+                tc::fence_after();
+                const uint32_t xs = smem_u32(S.x[s]), hs = smem_u32(S.bhi), ls = smem_u32(S.blo);
+                const uint32_t d = tmem + (uint32_t)(b * kHtMaxN);
+#pragma unroll
+                for (int k = 0; k < kHtD / 16; ++k)
+                    tc::mma_bf16(d, tc::smem_desc(xs + k * 32, 16, 1024, tc::kLayoutSW128),
+                                 tc::smem_desc(hs + k * 32, 16, 1024, tc::kLayoutSW128), idesc, k > 0 ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < kHtD / 16; ++k)
+                    tc::mma_bf16(d, tc::smem_desc(xs + k * 32, 16, 1024, tc::kLayoutSW128),
+                                 tc::smem_desc(ls + k * 32, 16, 1024, tc::kLayoutSW128), idesc, 1u);
+                tc::commit(&S.tfull[b]);
+                last = i;
+            }
+            // the MMAs issued finish before the tensor memory may be freed
+            if (last >= 0) tc::mbar_wait_bounded(&S.tfull[last & 1], (last >> 1) & 1, kHtWaitNs, K_LSH_HASH, 6);
+        }
+    } else {
+        // ---------------- epilogue: thread = token row quad * 32 + lane of the tile
+        const int quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        for (int i = 0; i < nt; ++i) {
+            const int s = i % kHtStages, b = i & 1, v = i >> 1;
+            const bool ok = tc::mbar_wait_bounded(&S.tfull[b], v & 1, kHtWaitNs, K_LSH_HASH, 7, kHtSuspendNs,
+                                                  false, abort_flag);
+            if (__any_sync(0xffffffffu, !ok)) {
+                if (lane == 0) atomicOr(&S.fail, 1);
+                break;
+            }
+            tc::fence_after();
+            const unsigned char *xa = S.x[s];
+            const int tok = (t_first + i) * kHtM + row;
+            float ss = 0.0f;                      // |x|^2 of this row (16-byte reads of the swizzled tile)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 w4 = *reinterpret_cast<const uint4 *>(xa + tc::sw128(row, c));
+                const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float a0 = __uint_as_float(ww[q] << 16), a1 = __uint_as_float(ww[q] & 0xffff0000u);
+                    ss = fmaf(a0, a0, ss);
+                    ss = fmaf(a1, a1, ss);
+                }
+            }
+            const float xerr = kHtErr * sqrtf(ss);
+            for (int r = 0; r < rounds; ++r) {
+                uint32_t uv[32];
+                tc::tmem_ld32(tl + (uint32_t)(b * kHtMaxN + r * kHtHalf), uv);
+                tc::tmem_ld_wait();
+                if (r == rounds - 1) {            // the buffer is free for tile i + 2
+                    tc::fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&S.tempty[b]);
+                }
+                // the two largest |u~_k|
+                float m1 = -1.0f, m2 = -1.0f, u1 = 0.0f;
+                int k1 = 0, k2 = 0;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const float uk = __uint_as_float(uv[k]);
+                    const float a = fabsf(uk);
+                    if (a > m1) { m2 = m1; k2 = k1; m1 = a; k1 = k; u1 = uk; }
+                    else if (a > m2) { m2 = a; k2 = k; }
+                }
+                int bk = u1 > 0.0f ? k1 : kHtHalf + k1;
+                const float E1 = xerr * S.rnorm[r * kHtHalf + k1], E2 = xerr * S.rnorm[r * kHtHalf + k2];
+                const bool amb = (m2 >= m1 - (E1 + E2)) || (m1 <= E1);
+                // exact chains for the undecided tokens of this warp, one token at a time
+                uint32_t pend = __ballot_sync(0xffffffffu, amb && tok < n);
+                const float *Rr = Rh + (size_t)r * kHtD * kHtHalf;
+                while (pend) {
+                    const int l = __ffs(pend) - 1;
+                    pend &= pend - 1;
+                    const int rl = quad * 32 + l;
+                    float rv[kHtD];               // column `lane` of R_{h,r}, all loads in flight
+#pragma unroll
+                    for (int t = 0; t < kHtD; ++t) rv[t] = __ldg(Rr + t * kHtHalf + lane);
+                    float u = 0.0f;
+#pragma unroll
+                    for (int t = 0; t < kHtD; ++t) u = __fmaf_rn(ht_x(xa, rl, t), rv[t], u);
+                    const float bp = warp_max(u);
+                    const int ap = __ffs(__ballot_sync(0xffffffffu, u == bp)) - 1;
+                    const float bn = warp_max(-u);
+                    const int an = __ffs(__ballot_sync(0xffffffffu, -u == bn)) - 1;
+                    if (lane == l) bk = (bp >= bn) ? ap : kHtHalf + an;
+                }
+                if (tok < n) bucket[((size_t)bh * rounds + r) * n + tok] = bk;
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&S.xempty[s]);   // the X stage is free (MMA and fallbacks done)
+        }
     }
-    cp_async_wait<0>();
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, ncols);
+    if (warp == 1) tc::tmem_dealloc(tmem, 2 * kHtMaxN);
 }
 
 // Tiles per CTA so that the grid is about two CTAs per SM.

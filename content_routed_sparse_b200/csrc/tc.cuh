@@ -139,11 +139,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *mbar, uint32_t parity, u
 // global timer is read only every 256 polls, because reading it is slow and a
 // read between polls would delay the wake-up of every pipeline handoff.
 // A forceable wait gives up before its first poll while g_force_wait_timeout is
-// set (the caller's failure path then drains with non-forceable waits).
+// set (the caller's failure path then drains with non-forceable waits).  With an
+// abort flag (shared memory), the wait also returns false, silently, once the
+// flag is set by another warp of the CTA that gave up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parity,
                                                   uint64_t limit_ns, uint32_t kernel,
                                                   uint32_t site, uint32_t suspend_ns = 10000u,
-                                                  bool forceable = false) {
+                                                  bool forceable = false,
+                                                  const volatile int *abort_flag = nullptr) {
     if (forceable && *reinterpret_cast<volatile uint32_t *>(&g_force_wait_timeout) != 0u) {
         raise_error(CRS_DEVERR_TIMEOUT);
         diag_record(kernel, site, 0u, threadIdx.x, 0u, 0u);
@@ -152,6 +155,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parit
     uint64_t t0 = 0;
     for (uint32_t polls = 1;; ++polls) {
         if (mbar_try_wait(mbar, parity, suspend_ns)) return true;
+        // another role of the CTA gave up: stop waiting (it reported the failure)
+        if (abort_flag && *abort_flag) return false;
         if ((polls & 255u) == 0u) {
             const uint64_t now = globaltimer_ns();
             if (t0 == 0) t0 = now;
