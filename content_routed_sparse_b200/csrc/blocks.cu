@@ -291,18 +291,55 @@ block_score_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict_
     sc_out[((size_t)sh * G + g) * n_full + b0 + bl] = fmaf(0.5f, quad, lin);
 }
 
-// qx[row][j] = sum_d U[d][j] scale q[row][d]: one warp per query row, lanes over j.
+// Copies n floats global -> shared with 16-byte loads when both are 16-byte aligned
+// (every load of a thread is issued before the stores that use it).
+__device__ __forceinline__ void stage_floats(float *dst, const float *__restrict__ src, int n) {
+    if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0) {
+        const int n4 = n >> 2;
+        const float4 *s4 = reinterpret_cast<const float4 *>(src);
+        float4 *d4 = reinterpret_cast<float4 *>(dst);
+        for (int e0 = threadIdx.x; e0 < n4; e0 += 4 * blockDim.x) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * blockDim.x;
+                v[u] = e < n4 ? __ldg(s4 + e) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * blockDim.x;
+                if (e < n4) d4[e] = v[u];
+            }
+        }
+        for (int e = (n4 << 2) + threadIdx.x; e < n; e += blockDim.x) dst[e] = __ldg(src + e);
+    } else {
+        for (int e = threadIdx.x; e < n; e += blockDim.x) dst[e] = __ldg(src + e);
+    }
+}
+
+// qx[row][j] = sum_d U[d][j] scale q[row][d].
 __global__ void __launch_bounds__(256)
 query_project_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ U,
                      float *__restrict__ qx, int n_rows, int sd, float scale) {
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (row >= n_rows) return;
-    const __nv_bfloat16 *q = Q + (size_t)row * kBdD;
-    for (int j = lane; j < sd; j += 32) {
+    // 16 query rows per CTA; U (D x sd) and the rows staged in shared memory, then
+    // thread (row, j) forms qx[row][j] = sum_d U[d][j] scale q[d] as one FMA chain in d order
+    extern __shared__ float qp_smem[];
+    float *Us = qp_smem;                         // [D][sd]
+    float *qs = Us + (size_t)kBdD * sd;          // [16][D]
+    const int r0 = blockIdx.x * 16;
+    stage_floats(Us, U, kBdD * sd);
+    for (int e = threadIdx.x; e < 16 * kBdD; e += blockDim.x) {
+        const int r = e / kBdD, dd = e - r * kBdD;
+        qs[e] = r0 + r < n_rows ? scale * __bfloat162float(Q[(size_t)(r0 + r) * kBdD + dd]) : 0.0f;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < 16 * sd; e += blockDim.x) {
+        const int r = e / sd, j = e - r * sd;
+        if (r0 + r >= n_rows) continue;
         float acc = 0.0f;
-#pragma unroll 16           // the loads of U run ahead of the dependent FMA chain
-        for (int d = 0; d < kBdD; ++d) acc = fmaf(__ldg(U + (size_t)d * sd + j), scale * __bfloat162float(q[d]), acc);
-        qx[(size_t)row * sd + j] = acc;
+#pragma unroll 8
+        for (int dd = 0; dd < kBdD; ++dd) acc = fmaf(Us[dd * sd + j], qs[r * kBdD + dd], acc);
+        qx[(size_t)(r0 + r) * sd + j] = acc;
     }
 }
 
@@ -873,7 +910,7 @@ struct FtSmem {
     unsigned char mu[kFtStages][2][kFtM * 128];    // [stage][K half]: 128 blocks x 64 dims, SW128
     unsigned char dec[kFtDecBufs][2][kFtM * 128];  // [buffer][K half]: one eigenvector as bf16
     unsigned char q[kFtStages][2][kFtN * 128];     // [stage][K half]: 16 rows x 64 dims, rows >= G zero
-    unsigned char p[kFtStages][2][kFtN * 128];     // subspace form: projected query, hi rows 0..G-1, lo G..2G-1
+    unsigned char p[kFtStages][2][kFtN * 128];     // subspace form: projected query, value row g, residual 8 + g
     uint64_t full[kFtStages], raw_empty[kFtStages], dec_full[kFtDecBufs], dec_empty[kFtDecBufs];
     uint64_t tm_full[2], tm_empty[2];
     uint32_t tmem_base;
@@ -1111,7 +1148,8 @@ block_score_fp4_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_
 #pragma unroll
                     for (int e = 0; e < kFtMaxR; ++e) {      // sig[e] = 0 for e >= R
                         float dot = __uint_as_float(e < R ? d[1 + e][g] : 0u);
-                        if (a.split) dot += __uint_as_float(e < R ? d[1 + e][a.G + g] : 0u);   // + residual
+                        // + the residual column (rows 8 + g of the split query: a fixed index)
+                        if (a.split && g < kFtN / 2) dot += __uint_as_float(e < R ? d[1 + e][kFtN / 2 + g] : 0u);
                         const float pe = sig[e] * dot;
                         quad2 = fmaf(pe, pe, quad2);
                     }
@@ -1458,7 +1496,11 @@ extern "C" int crs_block_select_ss(const crs_block_sel_params *p, const void *Q,
     {
         ProfScope _ps(K_BLK_SCORE, s);
         _ps.more(1);                              // projection + scorer
-        query_project_kernel<<<ceil_div(n_rows, 8), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Q), U, qx,
+        const size_t psm = ((size_t)kBdD * sd + 16 * kBdD) * 4;
+        CRS_TRY_CUDA(cudaFuncSetAttribute(query_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)psm));
+        query_project_kernel<<<ceil_div(n_rows, 16), 256, psm, s>>>(
+            static_cast<const __nv_bfloat16 *>(Q), U, qx,
                                                                   n_rows, sd, p->scale);
         block_score_kernel<<<dim3(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv), kBsThreads, smem_a, s>>>(
             static_cast<const __nv_bfloat16 *>(Q), mu, xi_ss, sc, p->b.n_kv, p->n_q, G, p->b.rank, n_full,
@@ -1516,34 +1558,33 @@ __global__ void __launch_bounds__(256) block_quantize_ss_kernel(const float *__r
 }
 
 // P[sh][row][j]: per (sequence, KV head) the G projected queries p_g = U^T q_g
-// (fp32, one FMA per term in dim order) as a bf16 value (rows 0..G-1) and the
-// bf16 residual p_g - value (rows G..2G-1); dims past sd and rows past 2G zero.
-// One warp per (sh, g); lane l takes dims l, l + 32, l + 64 (< 96).
+// (fp32, one FMA per term in dim order) as a bf16 value (row g) and the bf16
+// residual p_g - value (row 8 + g); dims past sd and the other rows zero.
+// One CTA per (sequence, KV head): U and the G query rows staged in shared memory.
 __global__ void __launch_bounds__(256) query_project_split_kernel(const __nv_bfloat16 *__restrict__ Q,
                                                                   const float *__restrict__ U,
                                                                   __nv_bfloat16 *__restrict__ P, int n_sh,
                                                                   int n_kv, int n_q, int G, int sd) {
-    const int item = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (item >= n_sh * kFtN) return;
-    const int sh = item / kFtN, rrow = item - sh * kFtN;
-    __nv_bfloat16 *out = P + ((size_t)sh * kFtN + rrow) * kBdD;
-    if (rrow >= G) {                             // residual rows are written by their g; zero the rest
-        if (rrow >= 2 * G)
-            for (int j = lane; j < kBdD; j += 32) out[j] = __float2bfloat16_rn(0.0f);
-        return;
-    }
-    const int seq = sh / n_kv, h = sh - seq * n_kv;
-    const __nv_bfloat16 *q = Q + ((size_t)seq * n_q + h * G + rrow) * kBdD;
-    __nv_bfloat16 *res = P + ((size_t)sh * kFtN + G + rrow) * kBdD;
-    for (int j = lane; j < kBdD; j += 32) {
+    extern __shared__ float qs_smem[];
+    float *Us = qs_smem;                          // [D][sd]
+    float *qs = Us + (size_t)kBdD * sd;           // [G][D]
+    const int sh = blockIdx.x, seq = sh / n_kv, h = sh - seq * n_kv;
+    stage_floats(Us, U, kBdD * sd);
+    for (int e = threadIdx.x; e < G * kBdD; e += blockDim.x)
+        qs[e] = __bfloat162float(Q[((size_t)seq * n_q + h * G) * kBdD + e]);
+    __syncthreads();
+    __nv_bfloat16 *out = P + (size_t)sh * kFtN * kBdD;
+    constexpr int kHalf = kFtN / 2;               // value rows 0..7, residual rows 8..15
+    for (int e = threadIdx.x; e < kHalf * kBdD; e += blockDim.x) {
+        const int r = e / kBdD, j = e - r * kBdD;
         float acc = 0.0f;
-        if (j < sd) {
-#pragma unroll 16           // the loads of U run ahead of the dependent FMA chain
-            for (int dd = 0; dd < kBdD; ++dd) acc = fmaf(__ldg(U + (size_t)dd * sd + j), __bfloat162float(q[dd]), acc);
+        if (r < G && j < sd) {
+#pragma unroll 8
+            for (int dd = 0; dd < kBdD; ++dd) acc = fmaf(Us[dd * sd + j], qs[r * kBdD + dd], acc);
         }
         const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-        out[j] = hi;
-        res[j] = __float2bfloat16_rn(acc - __bfloat162float(hi));
+        out[e] = hi;
+        out[(size_t)(kHalf + r) * kBdD + j] = __float2bfloat16_rn(acc - __bfloat162float(hi));
     }
 }
 
@@ -1644,11 +1685,14 @@ extern "C" int crs_block_select_fp4_ss(const crs_block_sel_params *p, const void
     const size_t smem_s = sizeof(FtSmem) + 1024;
     CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_fp4_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
+    const size_t psm = ((size_t)kBdD * sd + (size_t)G * kBdD) * 4;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(query_project_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)psm));
     {
         ProfScope _ps(K_BLK_SCORE, s);
         _ps.more(1);                              // projection + scorer
-        query_project_split_kernel<<<ceil_div(n_sh * kFtN, 8), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(Q), U, P, n_sh, p->b.n_kv, p->n_q, G, sd);
+        query_project_split_kernel<<<n_sh, 256, psm, s>>>(static_cast<const __nv_bfloat16 *>(Q), U, P, n_sh,
+                                                         p->b.n_kv, p->n_q, G, sd);
         block_score_fp4_tc_kernel<<<grid, kFtThreads, smem_s, s>>>(tmu, tq, tp, fa);
     }
     CRS_CHECK_LAUNCH();

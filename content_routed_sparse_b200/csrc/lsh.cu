@@ -332,14 +332,18 @@ lsh_chunk_attn_kernel(const T *__restrict__ QK, const T *__restrict__ V,
                       const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
                       const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
                       float *__restrict__ o_ws, float *__restrict__ lse_ws, int H, int n, int m,
-                      int rounds, int causal, int no_self, int key_norm, float scale) {
+                      int rounds, int causal, int no_self, int key_norm, float scale, int q_splits) {
     extern __shared__ float smf[];
-    const int c = blockIdx.x, r = blockIdx.y, bh = blockIdx.z;
+    // blockIdx.x = chunk * q_splits + split: a small problem spreads a chunk's query
+    // rows over several CTAs (each gathers the chunk's key window)
+    const int c = blockIdx.x / q_splits, split = blockIdx.x - c * q_splits;
+    const int r = blockIdx.y, bh = blockIdx.z;
     const int b = bh / H;
     const int vl = valid_len ? valid_len[b] : n;
     const int ks0 = max(0, (c - 1) * m), ks1 = min((c + 1) * m, n);
     const int nk = ks1 - ks0;                    // <= 2m
-    const int qs0 = c * m, qs1 = min(qs0 + m, n);
+    const int rps = (m + q_splits - 1) / q_splits;
+    const int qs0 = min(c * m + split * rps, n), qs1 = min(min(c * m + m, n), qs0 + rps);
     const int KM = 2 * m;
     float *Ks = smf;                             // [KM][DH+1]
     float *Vs = Ks + KM * (DH + 1);              // [KM][DH]
@@ -746,13 +750,17 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
     if (smem > 227 * 1024) return CRS_ERR_UNSUPPORTED;
     auto kern = lsh_chunk_attn_kernel<T, DH>;
     CRS_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    dim3 grid(ceil_div(p.n, p.chunk), p.n_rounds, p.B * p.H);
+    // query splits per chunk: about two CTAs per SM when the problem is small, at
+    // least one warp's worth of rows (8) per CTA
+    const long long base_ctas = (long long)ceil_div(p.n, p.chunk) * p.n_rounds * p.B * p.H;
+    const int q_splits = (int)max(1LL, min((long long)max(1, p.chunk / kAttnWarps), ceil_div_ll(2 * 148, base_ctas)));
+    dim3 grid(ceil_div(p.n, p.chunk) * q_splits, p.n_rounds, p.B * p.H);
     {
         ProfScope _ps(K_LSH_ATTN, s);
         kern<<<grid, kAttnWarps * 32, smem, s>>>(static_cast<const T *>(QK), static_cast<const T *>(V),
                                                   bucket, perm, inv_perm, valid_len, o_ws, lse_ws, p.H,
                                                   p.n, p.chunk, p.n_rounds, a->causal, a->no_self,
-                                                  a->key_norm, a->scale);
+                                                  a->key_norm, a->scale, q_splits);
     }
     CRS_CHECK_LAUNCH();
     }

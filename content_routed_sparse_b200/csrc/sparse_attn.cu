@@ -27,6 +27,14 @@ constexpr int kSaTileBytes = kSaKeys * kSaRowBytes;   // 16 KB
 constexpr int kSaStages = 3;                          // K/V tiles in the ring
 constexpr float kLog2e = 1.4426950408889634f;
 
+// 2^x by the hardware approximation (relative error about 2^-22, far inside the
+// output tolerance); 2^-inf = 0
+__device__ __forceinline__ float sa_ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // swizzled byte offset of 16-byte chunk c (0..15) of row r inside a tile
 __device__ __forceinline__ int sw_off(int r, int c) { return r * kSaRowBytes + ((c ^ (r & 7)) << 4); }
 
@@ -212,15 +220,15 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
             mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
             mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
             const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-            const float c_lo = (mn_lo == -INFINITY) ? 1.0f : exp2f(m_lo - mn_lo);
-            const float c_hi = (mn_hi == -INFINITY) ? 1.0f : exp2f(m_hi - mn_hi);
+            const float c_lo = (mn_lo == -INFINITY) ? 1.0f : sa_ex2(m_lo - mn_lo);
+            const float c_hi = (mn_hi == -INFINITY) ? 1.0f : sa_ex2(m_hi - mn_hi);
             float ps_lo = 0.0f, ps_hi = 0.0f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    s[nt][e] = (s[nt][e] == -INFINITY) ? 0.0f : exp2f(s[nt][e] - mn_lo);
-                    s[nt][2 + e] = (s[nt][2 + e] == -INFINITY) ? 0.0f : exp2f(s[nt][2 + e] - mn_hi);
+                    s[nt][e] = (s[nt][e] == -INFINITY) ? 0.0f : sa_ex2(s[nt][e] - mn_lo);
+                    s[nt][2 + e] = (s[nt][2 + e] == -INFINITY) ? 0.0f : sa_ex2(s[nt][2 + e] - mn_hi);
                     ps_lo += s[nt][e];
                     ps_hi += s[nt][2 + e];
                 }
@@ -229,10 +237,13 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
             l_hi = l_hi * c_hi + ps_hi;
             m_lo = mn_lo;
             m_hi = mn_hi;
+            // the running maxima rarely move after the first tiles: rescale only when one did
+            if (c_lo != 1.0f || c_hi != 1.0f) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                o[j][0] *= c_lo; o[j][1] *= c_lo;
-                o[j][2] *= c_hi; o[j][3] *= c_hi;
+                for (int j = 0; j < 16; ++j) {
+                    o[j][0] *= c_lo; o[j][1] *= c_lo;
+                    o[j][2] *= c_hi; o[j][3] *= c_hi;
+                }
             }
             // P = P_hi + P_lo, both bf16: the pair carries ~16 significant bits, so
             // rounding P for the tensor core stays far below the output tolerance
