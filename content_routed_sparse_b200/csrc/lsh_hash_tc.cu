@@ -26,8 +26,9 @@
 //
 // Persistent, warp-specialised CTA walking the 128-token tiles of one
 // (batch, head): warp 0 loads X tiles with TMA into a 3-stage ring, warp 1
-// issues the MMAs into two tensor-memory buffers, warps 2..5 (one token row
-// per thread) read the scores, decide the buckets and release the buffers.
+// issues the MMAs into two tensor-memory buffers, warps 2..9 (one token row
+// per thread; two warps per row quadrant, each taking half of the rounds) read
+// the scores, decide the buckets and release the buffers.
 // R is split into its operand tiles once per CTA.
 #include "common.cuh"
 #include "tc.cuh"
@@ -39,7 +40,7 @@ constexpr int kHtHalf = 32;               // b / 2
 constexpr int kHtD = 64;
 constexpr int kHtMaxN = 128;              // 32 x rounds, rounds <= 4
 constexpr int kHtStages = 3;
-constexpr int kHtEpiWarps = 4;
+constexpr int kHtEpiWarps = 8;            // two per tensor-memory lane quadrant, each half the rounds
 constexpr int kHtThreads = 32 * (2 + kHtEpiWarps);
 constexpr float kHtErr = 2.44140625e-4f;  // 2^-12
 constexpr uint64_t kHtWaitNs = 1000000000ull;
@@ -182,8 +183,11 @@ lsh_hash_tc_kernel(const __grid_constant__ CUtensorMap tx, const float *__restri
             if (last >= 0) tc::mbar_wait_bounded(&S.tfull[last & 1], (last >> 1) & 1, kHtWaitNs, K_LSH_HASH, 6);
         }
     } else {
-        // ---------------- epilogue: thread = token row quad * 32 + lane of the tile
+        // ---------------- epilogue: thread = token row quad * 32 + lane of the tile;
+        // the two warps of a quadrant take rounds [r_lo, r_hi)
         const int quad = warp & 3, row = quad * 32 + lane;
+        const int half = (warp - 2) >> 2;
+        const int r_lo = half == 0 ? 0 : (rounds + 1) / 2, r_hi = half == 0 ? (rounds + 1) / 2 : rounds;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         for (int i = 0; i < nt; ++i) {
             const int s = i % kHtStages, b = i & 1, v = i >> 1;
@@ -209,28 +213,36 @@ lsh_hash_tc_kernel(const __grid_constant__ CUtensorMap tx, const float *__restri
                 }
             }
             const float xerr = kHtErr * sqrtf(ss);
-            for (int r = 0; r < rounds; ++r) {
+            if (r_lo >= r_hi) {                   // nothing for this warp (a single round)
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&S.tempty[b]);
+            }
+            for (int r = r_lo; r < r_hi; ++r) {
                 uint32_t uv[32];
                 tc::tmem_ld32(tl + (uint32_t)(b * kHtMaxN + r * kHtHalf), uv);
                 tc::tmem_ld_wait();
-                if (r == rounds - 1) {            // the buffer is free for tile i + 2
+                if (r == r_hi - 1) {              // this warp's reads of the buffer are done
                     tc::fence_before();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&S.tempty[b]);
                 }
-                // the two largest |u~_k|
-                float m1 = -1.0f, m2 = -1.0f, u1 = 0.0f;
-                int k1 = 0, k2 = 0;
+                // The two largest |u~_k| as integer keys: |u~| with its low 6 mantissa bits
+                // replaced by (sign, k), so one unsigned max finds value, sign and index
+                // (truncating |u~| moves it by less than 2^-17 of itself, added to the margin).
+                uint32_t best1 = 0u, best2 = 0u;
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
-                    const float uk = __uint_as_float(uv[k]);
-                    const float a = fabsf(uk);
-                    if (a > m1) { m2 = m1; k2 = k1; m1 = a; k1 = k; u1 = uk; }
-                    else if (a > m2) { m2 = a; k2 = k; }
+                    const uint32_t key = (uv[k] & 0x7FFFFFC0u) | ((uv[k] >> 26) & 32u) | (uint32_t)k;
+                    best2 = max(best2, min(best1, key));
+                    best1 = max(best1, key);
                 }
-                int bk = u1 > 0.0f ? k1 : kHtHalf + k1;
+                const int k1 = (int)(best1 & 31u), k2 = (int)(best2 & 31u);
+                const float m1 = __uint_as_float(best1 & 0xFFFFFFC0u), m2 = __uint_as_float(best2 & 0xFFFFFFC0u);
+                int bk = (best1 & 32u) ? kHtHalf + k1 : k1;
                 const float E1 = xerr * S.rnorm[r * kHtHalf + k1], E2 = xerr * S.rnorm[r * kHtHalf + k2];
-                const bool amb = (m2 >= m1 - (E1 + E2)) || (m1 <= E1);
+                // written as "not a clear winner" so that a NaN anywhere also takes the exact path
+                const bool amb = !((m1 - (E1 + E2) - m1 * 0x1p-16f > m2) && (m1 > E1));
                 // exact chains for the undecided tokens of this warp, one token at a time
                 uint32_t pend = __ballot_sync(0xffffffffu, amb && tok < n);
                 const float *Rr = Rh + (size_t)r * kHtD * kHtHalf;
