@@ -636,25 +636,44 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         // 2^(M - bound).  Pairs are counted in their first round only, so the sums are
         // over the union of the rounds' candidates ([P1] "重复候选和归一化").  Rows with
         // a larger bound keep the per-round (o_r, lse_r) form, merged afterwards.
-        bool stored = false;
+        bool stored = false, acc_row = false;
+        float f = 0.0f;
         if (acc_O && q.pos_i >= 0) {
             const float bnd = S.rbound[q.row];
             if (bnd <= kTcAccBoundMax) {
                 const float L = S.u2.rowsum[0][q.row] + S.u2.rowsum[1][q.row];
                 const size_t orow = (size_t)bh * n + q.pos_i;
                 if (q.qvalid && L > 0.0f) {
-                    const float f = use16 ? 0x1p-15f : (single ? 1.0f : exp2f(M - bnd));
-                    float *o = acc_O + orow * kTcD + wg * 32;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        red_add_v4(o + u * 4, __uint_as_float(v[u * 4 + 0]) * f, __uint_as_float(v[u * 4 + 1]) * f,
-                                   __uint_as_float(v[u * 4 + 2]) * f, __uint_as_float(v[u * 4 + 3]) * f);
+                    f = use16 ? 0x1p-15f : (single ? 1.0f : exp2f(M - bnd));
+                    acc_row = true;
                     if (wg == 0) atomicAdd(acc_L + orow, L * f);
                 }
                 if (wg == 0) acc_M[orow] = bnd;
                 stored = true;
             } else if (wg == 0) {
                 acc_M[(size_t)bh * n + q.pos_i] = INFINITY;   // merged from the per-round form
+            }
+        }
+        // The accumulated rows go through shared memory (the P buffer is free once P.V has
+        // completed): each warp stages its 32 rows x 32 columns, then every vector reduction
+        // covers 128 contiguous bytes of one row, four rows per instruction.
+        const uint32_t acc_mask = __ballot_sync(0xffffffffu, acc_row);
+        if (acc_mask) {
+            unsigned char *tile = &S.kp[0][0] + warp * 4096;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<float4 *>(tile + tc::sw128(lane, u)) =
+                    make_float4(__uint_as_float(v[u * 4 + 0]) * f, __uint_as_float(v[u * 4 + 1]) * f,
+                                __uint_as_float(v[u * 4 + 2]) * f, __uint_as_float(v[u * 4 + 3]) * f);
+            __syncwarp();
+#pragma unroll
+            for (int pp = 0; pp < 8; ++pp) {
+                const int rr = (lane >> 3) + 4 * pp, ch = lane & 7;
+                if ((acc_mask >> rr) & 1u) {
+                    const float4 x = *reinterpret_cast<const float4 *>(tile + tc::sw128(rr, ch));
+                    const int pos = S.kpos[kTcM + quad * 32 + rr];
+                    red_add_v4(acc_O + ((size_t)bh * n + pos) * kTcD + wg * 32 + ch * 4, x.x, x.y, x.z, x.w);
+                }
             }
         }
         if (q.pos_i >= 0 && !stored) {
