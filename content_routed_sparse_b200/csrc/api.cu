@@ -9,7 +9,7 @@ namespace crs {
 static const char *kKernelNames[K_COUNT] = {
     "lsh_hash", "lsh_sort", "lsh_chunk_attn", "lsh_combine", "idx_slice_topk", "idx_merge_topk",
     "sparse_attn", "sparse_attn_merge", "block_describe", "block_score", "block_pick",
-    "lsh_chunk_attn_tc", "idx_prefill_tc", "idx_select", "noalloc", "block_quantize", "hisa", "lsh_decode", "route", "lsh_csr"};
+    "lsh_chunk_attn_tc", "idx_prefill_tc", "idx_select", "noalloc", "block_quantize", "hisa", "lsh_decode", "route", "lsh_csr", "lsh_chunk_attn_ring"};
 struct PendingEv {
     int id;
     cudaEvent_t a, b;

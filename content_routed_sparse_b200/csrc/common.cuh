@@ -176,7 +176,7 @@ namespace crs {
 enum KernelId {
     K_LSH_HASH = 0, K_LSH_SORT, K_LSH_ATTN, K_LSH_COMBINE, K_IDX_SLICE, K_IDX_MERGE,
     K_SA_MAIN, K_SA_MERGE, K_BLK_DESCRIBE, K_BLK_SCORE, K_BLK_PICK, K_LSH_ATTN_TC,
-    K_IDX_PREFILL_TC, K_IDX_SELECT, K_NOALLOC, K_BLK_QUANTIZE, K_HISA, K_LSH_DECODE, K_ROUTE, K_LSH_CSR, K_COUNT
+    K_IDX_PREFILL_TC, K_IDX_SELECT, K_NOALLOC, K_BLK_QUANTIZE, K_HISA, K_LSH_DECODE, K_ROUTE, K_LSH_CSR, K_LSH_ATTN_RING, K_COUNT
 };
 void prof_begin(int id, cudaStream_t s, void **ev_start);
 void prof_end(int id, cudaStream_t s, void *ev_start);

@@ -688,9 +688,11 @@ extern "C" size_t crs_lsh_attn_workspace_size(const crs_lsh_attn_params *a) {
     if (!a || validate_lsh(&a->p)) return 0;
     const crs_lsh_params &p = a->p;
     const size_t rows = (size_t)p.n_rounds * p.B * p.H * p.n;
-    // per-round (o_r, lse_r), then the accumulated weight sums and shifts of each row
+    // per-round (o_r, lse_r), then the accumulated weight sums and shifts of each row,
+    // then the persistent kernel's counters and its list of items left to the per-item kernel
+    const size_t items = (size_t)ceil_div(p.n, kTcM) * p.n_rounds * p.B * p.H;
     return align256(rows * p.d * sizeof(float)) + align256(rows * sizeof(float)) +
-           2 * align256((size_t)p.B * p.H * p.n * sizeof(float));
+           2 * align256((size_t)p.B * p.H * p.n * sizeof(float)) + 256 + align256(items * sizeof(int32_t));
 }
 
 namespace crs {
@@ -718,13 +720,45 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
                 CRS_TRY_CUDA(cudaMemsetAsync(O, 0, nrow * DH * sizeof(float), s));
                 CRS_TRY_CUDA(cudaMemsetAsync(acc_L, 0, 2 * align256(nrow * sizeof(float)), s));
             }
-            {
+            if (acc && p.n_rounds <= kRgEarlier + 1) {
+                // persistent ring kernel, then the per-item kernel over the items it left
+                int *ctr = reinterpret_cast<int *>(reinterpret_cast<char *>(acc_M) + align256(nrow * sizeof(float)));
+                int32_t *deferred = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(ctr) + 256);
+                CRS_TRY_CUDA(cudaMemsetAsync(ctr, 0, 2 * sizeof(int), s));
+                int dev = 0, sms = 148;
+                CRS_TRY_CUDA(cudaGetDevice(&dev));
+                CRS_TRY_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+                const int nch = ceil_div(p.n, kTcM);
+                const long long units = (long long)(rg_big_units(nch) + rg_small_units(nch)) * p.n_rounds * p.B * p.H;
+                const size_t rsmem = sizeof(RgSmem) + 1024;
+                CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_chunk_attn_ring_kernel,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+                CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_chunk_attn_ring_kernel,
+                                                  cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                  (int)cudaSharedmemCarveoutMaxShared));
+                {
+                    ProfScope _ps(K_LSH_ATTN_RING, s);
+                    lsh_chunk_attn_ring_kernel<<<(unsigned)min((long long)2 * sms, units), kRgThreads, rsmem, s>>>(
+                        static_cast<const __nv_bfloat16 *>(QK), static_cast<const __nv_bfloat16 *>(V), bucket, perm,
+                        inv_perm, valid_len, static_cast<float *>(O), acc_L, acc_M, ctr, deferred, ctr + 1, p.H,
+                        p.B * p.H, p.n, p.n_rounds, a->causal, a->no_self, a->scale * 1.4426950408889634f);
+                }
+                CRS_CHECK_LAUNCH();
+                {
+                    ProfScope _ps(K_LSH_ATTN_TC, s);
+                    lsh_chunk_attn_tc_kernel<<<(unsigned)(2 * sms), kTcThreads, smem, s>>>(
+                        static_cast<const __nv_bfloat16 *>(QK), static_cast<const __nv_bfloat16 *>(V),
+                        bucket, perm, inv_perm, valid_len, o_ws, lse_ws, static_cast<float *>(O), acc_L, acc_M,
+                        p.H, p.B * p.H, p.n, p.n_rounds, a->causal, a->no_self, a->key_norm,
+                        a->scale * 1.4426950408889634f, deferred, ctr + 1);
+                }
+            } else {
                 ProfScope _ps(K_LSH_ATTN_TC, s);
                 lsh_chunk_attn_tc_kernel<<<grid, kTcThreads, smem, s>>>(
                     static_cast<const __nv_bfloat16 *>(QK), static_cast<const __nv_bfloat16 *>(V),
                     bucket, perm, inv_perm, valid_len, o_ws, lse_ws, acc ? static_cast<float *>(O) : nullptr,
-                    acc ? acc_L : nullptr, acc ? acc_M : nullptr, p.H, p.n, p.n_rounds,
-                    a->causal, a->no_self, a->key_norm, a->scale * 1.4426950408889634f);
+                    acc ? acc_L : nullptr, acc ? acc_M : nullptr, p.H, p.B * p.H, p.n, p.n_rounds,
+                    a->causal, a->no_self, a->key_norm, a->scale * 1.4426950408889634f, nullptr, nullptr);
             }
             CRS_CHECK_LAUNCH();
             if (acc) {

@@ -366,21 +366,19 @@ __device__ __forceinline__ void lsh_tc_issue_pv(LshTcSmem &S, uint32_t tmem, int
     }
 }
 
-__global__ void __launch_bounds__(kTcThreads, 2)
-lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
-                         const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
-                         const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
-                         float *__restrict__ o_ws, float *__restrict__ lse_ws, float *__restrict__ acc_O,
-                         float *__restrict__ acc_L, float *__restrict__ acc_M, int H, int n,
-                         int rounds, int causal, int no_self, int key_norm, float scale_log2) {
-    extern __shared__ unsigned char lsh_tc_raw[];
-    const uint32_t mis = smem_u32(lsh_tc_raw) & 1023u;
-    LshTcSmem &S = *reinterpret_cast<LshTcSmem *>(lsh_tc_raw + ((1024u - mis) & 1023u));
-
-    const int c = blockIdx.x, r = blockIdx.y, bh = blockIdx.z;
-    const int BH = gridDim.z;
+// One (chunk c, round r, batch*head bh) item of the CTA; false when a wait gave up.
+// ph holds the parity each barrier completes with next.
+__device__ __forceinline__ bool lsh_tc_item(LshTcSmem &S, uint32_t tmem, uint32_t (&ph)[3],
+                                            const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
+                                            const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
+                                            const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
+                                            float *__restrict__ o_ws, float *__restrict__ lse_ws, float *__restrict__ acc_O,
+                                            float *__restrict__ acc_L, float *__restrict__ acc_M, int H, int BH, int n,
+                                            int rounds, int causal, int no_self, int key_norm, float scale_log2,
+                                            int c, int r, int bh) {
     const int b = bh / H;
     const int vl = valid_len ? valid_len[b] : n;
+    __syncthreads();                              // the previous item's reads of shared memory are done
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int C1 = (n + kTcM - 1) / kTcM + 1;      // chunk-code stride
     const size_t seg_r = ((size_t)bh * rounds + r) * n;
@@ -410,12 +408,6 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
             S.kcode[rr][j] = code;
         }
     }
-    if (tid == 0) {
-        tc::mbar_init(&S.bar[0], 1);
-        tc::mbar_init(&S.bar[1], 1);
-        tc::mbar_init(&S.bar[2], 1);
-        tc::mbar_fence_init();
-    }
     __syncthreads();
 
     // ---- 2. gather K (= Q) and V rows; bucket runs of the window
@@ -434,7 +426,6 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         }
         cp_async_commit();
     }
-    if (warp == 0) tc::tmem_alloc(&S.tmem_base, kTcCols);
     {
         // the window's buckets are nondecreasing: binary searches give the run
         const int j = tid, bk = S.u1.kbkt[j];
@@ -509,7 +500,6 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(S.v + tc::sw128(tid, ch)) = v16[ch];
     }
     tc::fence_proxy_async();
-    const uint32_t tmem = S.tmem_base;
 
     // ---- 3. S = Q K^T into TMEM columns [0, 256)
     if (tid == 0) {
@@ -523,11 +513,12 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         }
         tc::commit(&S.bar[0]);
     }
-    bool ok_wait = tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 1, 10000u, true);
+    bool ok_wait = tc::mbar_wait_bounded(&S.bar[0], ph[0], kTcWaitNs, K_LSH_ATTN_TC, 1, 10000u, true);
     if (__syncthreads_or(!ok_wait)) {
-        tc::mbar_wait_bounded(&S.bar[0], 0, kTcWaitNs, K_LSH_ATTN_TC, 2);   // let the MMA drain
-        goto teardown;
+        tc::mbar_wait_bounded(&S.bar[0], ph[0], kTcWaitNs, K_LSH_ATTN_TC, 2);   // let the MMA drain
+        return false;
     }
+    ph[0] ^= 1u;
     tc::fence_after();
 
     {
@@ -591,8 +582,9 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         for (int half = 0; half < 2 && !use16; ++half) {
             if (half == 1) {
                 // the buffer is free once the first half's P.V has completed
-                ok_wait = tc::mbar_wait_bounded(&S.bar[1], 0, kTcWaitNs, K_LSH_ATTN_TC, 3);
-                if (__syncthreads_or(!ok_wait)) goto teardown;
+                ok_wait = tc::mbar_wait_bounded(&S.bar[1], ph[1], kTcWaitNs, K_LSH_ATTN_TC, 3);
+                if (__syncthreads_or(!ok_wait)) return false;
+                ph[1] ^= 1u;
                 tc::fence_after();
             }
             const int col0 = half * 128 + wg * 64;
@@ -617,8 +609,9 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
             }
         }
         S.u2.rowsum[wg][q.row] = sum;
-        ok_wait = tc::mbar_wait_bounded(&S.bar[2], 0, kTcWaitNs, K_LSH_ATTN_TC, 4);
-        if (__syncthreads_or(!ok_wait)) goto teardown;
+        ok_wait = tc::mbar_wait_bounded(&S.bar[2], ph[2], kTcWaitNs, K_LSH_ATTN_TC, 4);
+        if (__syncthreads_or(!ok_wait)) return false;
+        ph[2] ^= 1u;
         tc::fence_after();
 
         // ---- 6. epilogue: warpgroup wg writes output columns [32 wg, 32 wg + 32).
@@ -696,10 +689,53 @@ lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat
         }
     }
 
-teardown:
+    return true;
+}
+
+// Grid mode (items == nullptr): CTA (x, y, z) is the item (chunk x, round y, batch*head z).
+// List mode: the CTAs share the item ids items[0 .. *item_count), id = (bh * rounds + r) * chunks + c.
+__global__ void __launch_bounds__(kTcThreads, 2)
+lsh_chunk_attn_tc_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bfloat16 *__restrict__ V,
+                         const int32_t *__restrict__ bucket, const int32_t *__restrict__ perm,
+                         const int32_t *__restrict__ inv_perm, const int32_t *__restrict__ valid_len,
+                         float *__restrict__ o_ws, float *__restrict__ lse_ws, float *__restrict__ acc_O,
+                         float *__restrict__ acc_L, float *__restrict__ acc_M, int H, int BH, int n,
+                         int rounds, int causal, int no_self, int key_norm, float scale_log2,
+                         const int32_t *__restrict__ items, const int32_t *__restrict__ item_count) {
+    extern __shared__ unsigned char lsh_tc_raw[];
+    const uint32_t mis = smem_u32(lsh_tc_raw) & 1023u;
+    LshTcSmem &S = *reinterpret_cast<LshTcSmem *>(lsh_tc_raw + ((1024u - mis) & 1023u));
+    const int count = items ? *item_count : 1;
+    if (items && (int)blockIdx.x >= count) return;    // uniform over the CTA, before any setup
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&S.bar[0], 1);
+        tc::mbar_init(&S.bar[1], 1);
+        tc::mbar_init(&S.bar[2], 1);
+        tc::mbar_fence_init();
+    }
+    if (warp == 0) tc::tmem_alloc(&S.tmem_base, kTcCols);
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(S.tmem_base, kTcCols);
+    tc::fence_after();
+    const uint32_t tmem = S.tmem_base;
+    uint32_t ph[3] = {0u, 0u, 0u};
+    const int nch = (n + kTcM - 1) / kTcM;
+    for (int t = items ? (int)blockIdx.x : 0; t < count; t += items ? (int)gridDim.x : 1) {
+        int c = blockIdx.x, r = blockIdx.y, bh = blockIdx.z;
+        if (items) {
+            const int id = items[t];
+            c = id % nch;
+            r = (id / nch) % rounds;
+            bh = id / (nch * rounds);
+        }
+        if (!lsh_tc_item(S, tmem, ph, QK, V, bucket, perm, inv_perm, valid_len, o_ws, lse_ws, acc_O, acc_L,
+                         acc_M, H, BH, n, rounds, causal, no_self, key_norm, scale_log2, c, r, bh))
+            break;
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTcCols);
 }
 
 }  // namespace crs

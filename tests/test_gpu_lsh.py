@@ -92,6 +92,8 @@ def test_lsh_bf16_small(crs, cuda_dev, n, chunk, rounds, nb, vl_frac):
     (1280, 8, 4, 1, 1, 1, 0.2),     # 8 rounds: dedup against 7 earlier rounds
     (640, 3, 8, 0, 0, 0, 0.0),      # no causal mask, raw keys
     (129, 1, 2, 1, 1, 1, 0.0),      # two chunks, the second of one slot
+    (2200, 4, 16, 1, 0, 1, 0.1),    # 18 chunks: work units of 8, 8 and 2 chunks in the ring kernel
+    (3000, 4, 32, 0, 1, 1, 0.0),    # no causal mask, self excluded, 24 chunks
 ])
 def test_lsh_bf16_tensor_core_path(crs, cuda_dev, n, rounds, nb, causal, no_self, key_norm, vl_frac):
     """bf16, d = 64, chunk = 128 runs on the tcgen05 kernel."""
