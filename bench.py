@@ -153,6 +153,11 @@ class LshWorkload(Workload):
                                ("hbm", attn_bytes / 1e9, "GB/s")],
             "lsh_chunk_attn_tc": [("tensor", rect_flops / 1e12, "TFLOP/s"),
                                   ("hbm", attn_bytes / 1e9, "GB/s")],
+            # the persistent kernel; the per-item kernel then runs over the items it left
+            # (normally none) and its time is counted with it
+            "lsh_chunk_attn_ring": [("tensor", rect_flops / 1e12, "TFLOP/s"),
+                                    ("hbm", attn_bytes / 1e9, "GB/s")],
+            "_with": {"lsh_chunk_attn_ring": ["lsh_chunk_attn_tc"]},
             "lsh_hash": [("alu", B * H * R * n * d * (p["n_buckets"] // 2) * 2 / 1e12, "TFLOP/s")],
         }
 
@@ -801,7 +806,8 @@ def _traffic(kernel, workload):
 
 def roofline(wl, prof, peaks, traffic=None):
     """The dominant kernel (largest summed device time) with its algorithmic work."""
-    spec = wl.roofline_spec()
+    spec = dict(wl.roofline_spec())
+    companions = spec.pop("_with", {})
     timed = {k: v for k, v in prof.items() if v["timed_launches"] > 0}
     if not timed:
         return None, {}
@@ -810,7 +816,9 @@ def roofline(wl, prof, peaks, traffic=None):
     if top not in spec:
         return {"kernel": top, "bound": None, "achieved": None, "peak": None, "unit": None,
                 "frac": None, "traffic": None}, stages
-    per_launch_s = timed[top]["total_ms"] / timed[top]["timed_launches"] / 1e3
+    # kernels that always run right after the top one, on its leftovers, count with it
+    with_ms = sum(timed[c]["total_ms"] for c in companions.get(top, []) if c in timed)
+    per_launch_s = (timed[top]["total_ms"] + with_ms) / timed[top]["timed_launches"] / 1e3
 
     def peak_of(bound):
         if bound == "hbm":
@@ -828,6 +836,8 @@ def roofline(wl, prof, peaks, traffic=None):
            "unit": unit, "frac": round(achieved / peak, 4), "traffic": _traffic(top, wl.name),
            "peak_source": src,
            "per_launch_ms": round(per_launch_s * 1e3, 5)}
+    if companions.get(top):
+        out["includes"] = [c for c in companions[top] if c in timed]
     if len(entries) > 1:
         b2, a2, u2 = entries[1]
         p2 = peak_of(b2)[0]

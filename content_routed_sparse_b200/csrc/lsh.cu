@@ -746,7 +746,7 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
                 CRS_CHECK_LAUNCH();
                 {
                     ProfScope _ps(K_LSH_ATTN_TC, s);
-                    lsh_chunk_attn_tc_kernel<<<(unsigned)(2 * sms), kTcThreads, smem, s>>>(
+                    lsh_chunk_attn_tc_kernel<<<(unsigned)sms, kTcThreads, smem, s>>>(
                         static_cast<const __nv_bfloat16 *>(QK), static_cast<const __nv_bfloat16 *>(V),
                         bucket, perm, inv_perm, valid_len, o_ws, lse_ws, static_cast<float *>(O), acc_L, acc_M,
                         p.H, p.B * p.H, p.n, p.n_rounds, a->causal, a->no_self, a->key_norm,

@@ -28,9 +28,12 @@
 // are appended to a list for lsh_chunk_attn_tc_kernel's list mode (bf16 P with
 // a residual, or the two-pass form), which runs right after this kernel.
 //
-// Tensor memory (256 columns per CTA): S of window keys [0,128) in columns
-// [0,128) and of keys [128,256) in [128,256); P of keys [0,128) in [0,64) and
-// of keys [128,256) in [128,192); O in [64,128).
+// Tensor memory (256 columns per CTA): S of window key j in column j.  The two
+// warps that share a row's lanes split its eight 32-key chunks by parity (the
+// causal mask empties the high chunks of the low rows, so halves would be
+// unbalanced); the k-th chunk a warp handles (chunk 2k + wg) puts its P (16
+// columns) at rg_pcol(k, wg), inside the S columns that warp has already read.
+// P fills [0,128); O goes to [128,192).
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -248,21 +251,31 @@ __device__ __forceinline__ void rg_prep(RgSmem &S, int slot, int prev, int tid, 
     tc::fence_proxy_async();                      // the fp16 V rows are read by tcgen05.mma
 }
 
-// Masked fp16 P of one query row for the 128 window keys [128 wg, 128 wg + 128)
-// (slot metadata Mk), written over the S columns already read; returns the row's
-// partial sum.  NR = earlier rounds whose pairs are excluded.
+// Tensor-memory column of the P of the k-th chunk (0..3) of warp half wg: chunks
+// 2k + wg = 0, 2 | 1, 3 | 4, 6 | 5, 7 land in [0,32) | [32,64) | [64,96) | [96,128),
+// each inside the S columns of chunk 2 (k / 2) + wg, read by the same warp before.
+__host__ __device__ constexpr int rg_pcol(int k, int wg) { return 64 * (k >> 1) + 32 * wg + 16 * (k & 1); }
+
+// Masked fp16 P of one query row for the window chunks 2k + wg, k = 0..3 (keys of
+// the previous chunk's slot MP for k < 2, of the own chunk's MO after), written to
+// tensor memory at rg_pcol; returns the row's partial sum.  NR = earlier rounds
+// whose pairs are excluded.
 template <int NR>
-__device__ __forceinline__ float rg_softmax16(const RgMeta &Mk, const RgMeta &Mq, const LshTcRow &q,
+__device__ __forceinline__ float rg_softmax16(const RgMeta &MP, const RgMeta &MO, const LshTcRow &q,
                                               uint32_t trow, int wg, float M, const RgGather &g, bool gather,
                                               int tid) {
+    const RgMeta &Mq = MO;
     int ci[NR > 0 ? NR : 1];
 #pragma unroll
     for (int rr = 0; rr < NR; ++rr) ci[rr] = Mq.code[rr][q.row];
-    float2 sum2 = make_float2(0.0f, 0.0f);
+    float2 sum2[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                      make_float2(0.0f, 0.0f)};           // four independent chains
     const float2 negM = make_float2(-M, -M);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-        const int c0 = wg * 128 + cc * 32;        // window column
+        const int c0 = (2 * cc + wg) * 32;        // window column of the chunk
+        const RgMeta &Mk = cc < 2 ? MP : MO;
+        const int kr = c0 & (kTcM - 1);           // its first row in that slot
         uint32_t mb = q.qvalid ? range_bits(q.lo, q.hi, c0) : 0u;
         if (q.excl_self && q.jq >= c0 && q.jq < c0 + 32) mb &= ~(1u << (q.jq - c0));
         uint32_t ph[16];
@@ -270,7 +283,7 @@ __device__ __forceinline__ float rg_softmax16(const RgMeta &Mk, const RgMeta &Mq
             uint32_t v[32];
             tc::tmem_ld32(trow + c0, v);
             tc::tmem_ld_wait();
-            const float4 *ks = reinterpret_cast<const float4 *>(&Mk.kscale[cc * 32]);
+            const float4 *ks = reinterpret_cast<const float4 *>(&Mk.kscale[kr]);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const float4 k4 = ks[u];
@@ -279,7 +292,7 @@ __device__ __forceinline__ float rg_softmax16(const RgMeta &Mk, const RgMeta &Mq
                 for (int e = 0; e < 4; ++e) ok[e] = (mb >> (4 * u + e)) & 1u;
 #pragma unroll
                 for (int rr = 0; rr < NR; ++rr) {
-                    const int4 kc = reinterpret_cast<const int4 *>(&Mk.code[rr][cc * 32])[u];
+                    const int4 kc = reinterpret_cast<const int4 *>(&Mk.code[rr][kr])[u];
                     ok[0] = ok[0] && (uint32_t)(ci[rr] - kc.x) > 1u;
                     ok[1] = ok[1] && (uint32_t)(ci[rr] - kc.y) > 1u;
                     ok[2] = ok[2] && (uint32_t)(ci[rr] - kc.z) > 1u;
@@ -291,8 +304,8 @@ __device__ __forceinline__ float rg_softmax16(const RgMeta &Mk, const RgMeta &Mq
                                             make_float2(k4.z, k4.w), negM);
                 const float2 p01 = make_float2(ok[0] ? ex2_approx(a.x) : 0.0f, ok[1] ? ex2_approx(a.y) : 0.0f);
                 const float2 p23 = make_float2(ok[2] ? ex2_approx(b.x) : 0.0f, ok[3] ? ex2_approx(b.y) : 0.0f);
-                sum2 = __fadd2_rn(sum2, p01);
-                sum2 = __fadd2_rn(sum2, p23);
+                sum2[2 * (u & 1)] = __fadd2_rn(sum2[2 * (u & 1)], p01);
+                sum2[2 * (u & 1) + 1] = __fadd2_rn(sum2[2 * (u & 1) + 1], p23);
                 const __half2 h01 = __floats2half2_rn(p01.x, p01.y);
                 const __half2 h23 = __floats2half2_rn(p23.x, p23.y);
                 ph[2 * u] = *reinterpret_cast<const uint32_t *>(&h01);
@@ -302,11 +315,11 @@ __device__ __forceinline__ float rg_softmax16(const RgMeta &Mk, const RgMeta &Mq
 #pragma unroll
             for (int t2 = 0; t2 < 16; ++t2) ph[t2] = 0u;
         }
-        // keys [c0, c0 + 32) -> columns 128 wg + 16 cc + [0, 16): S columns this thread has read
-        tc::tmem_st16(trow + wg * 128 + cc * 16, ph);
+        tc::tmem_st16(trow + rg_pcol(cc, wg), ph);
         if (gather) rg_gather_piece(g, tid, cc);
     }
-    return sum2.x + sum2.y;
+    const float2 t = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
+    return t.x + t.y;
 }
 
 __global__ void __launch_bounds__(kRgThreads, 2)
@@ -454,13 +467,12 @@ lsh_chunk_attn_ring_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bflo
                 q.excl_self = (!causal) && no_self;
                 bnd = MO.bound[row];
                 const float Mx = bnd - 15.0f;
-                const RgMeta &Mk = wg == 0 ? MP : MO;
                 const RgGather g{S.kv[sF][0], S.kv[sF][1], S.meta[sF].pos, Kb, Vb};
                 switch (r) {
-                    case 0: sum = rg_softmax16<0>(Mk, MO, q, trow, wg, Mx, g, has_next, tid); break;
-                    case 1: sum = rg_softmax16<1>(Mk, MO, q, trow, wg, Mx, g, has_next, tid); break;
-                    case 2: sum = rg_softmax16<2>(Mk, MO, q, trow, wg, Mx, g, has_next, tid); break;
-                    default: sum = rg_softmax16<3>(Mk, MO, q, trow, wg, Mx, g, has_next, tid); break;
+                    case 0: sum = rg_softmax16<0>(MP, MO, q, trow, wg, Mx, g, has_next, tid); break;
+                    case 1: sum = rg_softmax16<1>(MP, MO, q, trow, wg, Mx, g, has_next, tid); break;
+                    case 2: sum = rg_softmax16<2>(MP, MO, q, trow, wg, Mx, g, has_next, tid); break;
+                    default: sum = rg_softmax16<3>(MP, MO, q, trow, wg, Mx, g, has_next, tid); break;
                 }
                 if (has_next) cp_async_commit();
                 tc::tmem_st_wait();
@@ -473,9 +485,9 @@ lsh_chunk_attn_ring_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bflo
                     constexpr uint32_t idesc = tc::idesc_f16_f32(kTcM, kTcD, 0, 1);
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk) {
-                        const int h = kk >> 3;
-                        const uint32_t vs = smem_u32(S.kv[h == 0 ? sP : sO][1]) + (kk & 7) * 16 * 128;
-                        tc::mma_f16_ts(tmem + 64, tmem + (uint32_t)(h * 128 + (kk & 7) * 8),
+                        const int j = kk >> 1, hh = kk & 1;   // keys [32 j + 16 hh, +16)
+                        const uint32_t vs = smem_u32(S.kv[j < 4 ? sP : sO][1]) + ((j & 3) * 32 + hh * 16) * 128;
+                        tc::mma_f16_ts(tmem + 128, tmem + (uint32_t)(rg_pcol(j >> 1, j & 1) + hh * 8),
                                        tc::smem_desc(vs, 32768, 1024, tc::kLayoutSW128), idesc, kk > 0 ? 1u : 0u);
                     }
                     tc::commit(&S.bar[1]);
@@ -510,7 +522,7 @@ lsh_chunk_attn_ring_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bflo
                 ph1 ^= 1u;
                 tc::fence_after();
                 uint32_t v[32];
-                tc::tmem_ld32(trow + 64 + wg * 32, v);
+                tc::tmem_ld32(trow + 128 + wg * 32, v);
                 tc::tmem_ld_wait();
                 const float L = S.rowsum[0][row] + S.rowsum[1][row];
                 const bool acc_row = q.qvalid && L > 0.0f;
