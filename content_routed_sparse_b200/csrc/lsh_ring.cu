@@ -54,8 +54,8 @@ struct RgMeta {
     int code[kRgEarlier][kTcM];     // earlier rounds: bucket * C1 + chunk + 1 (-8: none)
     float kscale[kTcM];             // scale * log2(e) / |k_j|
     float bound[kTcM];              // scale |k_j| in log2 units (the row bound as a query)
-    uint32_t run[kTcM];             // as a query: its bucket run in the window (previous chunk,
-                                    // this chunk), first | last with position < valid_len << 16
+    uint32_t run[kTcM];             // within the slot: first row of the row's bucket run | last row
+                                    // of the run's prefix with position < valid_len from it << 16
     int flags;
     int pad[3];
 };
@@ -63,6 +63,7 @@ struct RgMeta {
 struct RgSmem {
     unsigned char kv[3][2][kTcM * 128];   // ring slots: [0] K rows (128B swizzle), [1] V rows
     RgMeta meta[3];
+    int scan[2][4];                       // per warp of a slot's rows: last run start, first run stop
     int stage[1 + kRgEarlier][kTcM];      // next chunk's earlier-round slots and the chunk after's perm
                                           // entries, copied in by cp.async (its buckets go to its metadata)
     float rowsum[2][kTcM];
@@ -180,11 +181,10 @@ __device__ __forceinline__ void rg_gather_piece(const RgGather &g, int tid, int 
     cp_async16_zfill(g.vdst + tc::sw128(row, ch), g.Vb + off, ok);
 }
 
-// Prepare a slot whose rows have landed: V to fp16 in place (flagging values that
-// do not convert exactly), key norms and row bounds, and, when the slot of the
-// previous chunk is given (prev >= 0), the bucket runs of its rows as queries.
-// Two threads per row.
-__device__ __forceinline__ void rg_prep(RgSmem &S, int slot, int prev, int tid, float scale_log2, int vl) {
+// Prepare a slot whose rows have landed (metadata written): V to fp16 in place
+// (flagging values that do not convert exactly), key norms, row bounds and the
+// bucket runs inside the slot.  Two threads per row.
+__device__ __forceinline__ void rg_prep(RgSmem &S, int slot, int tid, float scale_log2, int vl) {
     const int row = tid >> 1, h = tid & 1;
     RgMeta &M = S.meta[slot];
     uint32_t vbad = 0u;
@@ -219,31 +219,26 @@ __device__ __forceinline__ void rg_prep(RgSmem &S, int slot, int prev, int tid, 
         M.kscale[row] = (ss > 0.0f ? rsqrtf(ss) : 0.0f) * scale_log2;
         M.bound[row] = bound;
     }
-    if (prev >= 0) {
-        // window key j < 128 is row j of the previous chunk's slot, j >= 128 row j - 128 of
-        // this one; the buckets are nondecreasing over the window
-        const RgMeta &MP = S.meta[prev];
-        const int jq = kTcM + row, bk = M.bkt[row];
-        int a, z;
-        if (h == 0) {
-            a = 0;                                // first window index with bucket >= bk
-            z = jq;
-            while (a < z) {
-                const int mid = (a + z) >> 1;
-                const int bm = mid < kTcM ? MP.bkt[mid] : M.bkt[mid - kTcM];
-                if (bm < bk) a = mid + 1; else z = mid;
-            }
-        } else {
-            a = jq;                               // last index of the run with position < vl
-            z = 2 * kTcM - 1;
-            while (a < z) {
-                const int mid = (a + z + 1) >> 1;
-                const int bm = mid < kTcM ? MP.bkt[mid] : M.bkt[mid - kTcM];
-                const int pm = mid < kTcM ? MP.pos[mid] : M.pos[mid - kTcM];
-                if (bm == bk && pm < vl) a = mid; else z = mid - 1;
-            }
+    // Bucket runs inside the slot (rows are sorted by bucket, then position): a run starts
+    // where the bucket changes; from row j its valid part goes on while the next row has
+    // the same bucket and a position below vl.  One row per thread of warps 0..3; a warp
+    // with no start (stop) of its own takes the nearest one of the warps before (after) it.
+    if (tid < kTcM) {
+        const int j = tid, w = j >> 5, l = j & 31;
+        const int bk = M.bkt[j];
+        const bool start = j == 0 || M.bkt[j - 1] != bk;
+        const bool stop = j == kTcM - 1 || M.bkt[j + 1] != bk || !(M.pos[j + 1] < vl);
+        const uint32_t sm = __ballot_sync(0xffffffffu, start), tm = __ballot_sync(0xffffffffu, stop);
+        if (l == 0) {
+            S.scan[0][w] = sm ? 32 * w + 31 - __clz(sm) : -1;
+            S.scan[1][w] = tm ? 32 * w + __ffs(tm) - 1 : kTcM;
         }
-        reinterpret_cast<uint16_t *>(&M.run[row])[h] = (uint16_t)a;
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        const uint32_t le = sm & (0xffffffffu >> (31 - l)), ge = tm & (0xffffffffu << l);
+        int first = le ? 32 * w + 31 - __clz(le) : -1, last = ge ? 32 * w + __ffs(ge) - 1 : kTcM;
+        for (int w2 = w - 1; first < 0; --w2) first = S.scan[0][w2];   // row 0 always starts a run
+        for (int w2 = w + 1; last == kTcM; ++w2) last = S.scan[1][w2];  // row 127 always stops one
+        M.run[j] = (uint32_t)first | ((uint32_t)last << 16);
     }
     const int fl = (vbad ? kRgFlagV : 0) | (!(bound <= kTcBoundMax16) ? kRgFlagBound : 0);
     const int wfl = __reduce_or_sync(0xffffffffu, fl);
@@ -393,9 +388,9 @@ lsh_chunk_attn_ring_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bflo
         if (tid < kTcM && c_begin + 1 < c_end) pos_next = rg_slot_pos(perm, seg_r, n, (c_begin + 1) * kTcM + tid);
         cp_async_wait<0>();
         __syncthreads();
-        rg_prep(S, 0, -1, tid, scale_log2, vl);
-        __syncthreads();                               // slot 0 is complete before slot 1's runs read it
-        rg_prep(S, 1, 0, tid, scale_log2, vl);
+        rg_prep(S, 0, tid, scale_log2, vl);
+        __syncthreads();                               // the run scratch is reused
+        rg_prep(S, 1, tid, scale_log2, vl);
 
         for (int c = c_begin; c < c_end; ++c) {
             const bool has_next = c + 1 < c_end, has_next2 = c + 2 < c_end;
@@ -461,9 +456,14 @@ lsh_chunk_attn_ring_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bflo
                 q.jq = kTcM + row;
                 q.pos_i = MO.pos[row];
                 q.qvalid = q.pos_i >= 0 && q.pos_i < vl;
+                // the query's bucket run in the window (key j < 128: row j of the previous
+                // chunk's slot, j >= 128: row j - 128 of its own): it starts in the own chunk,
+                // or, when the own chunk's first run continues the previous chunk's last,
+                // where that one starts; its valid part ends in the own chunk
                 const uint32_t run = MO.run[row];
-                q.lo = (int)(run & 0xffffu);
-                q.hi = causal ? (no_self ? q.jq - 1 : q.jq) : (int)(run >> 16);
+                const int f = (int)(run & 0xffffu);
+                q.lo = f > 0 || MP.bkt[kTcM - 1] != MO.bkt[row] ? kTcM + f : (int)(MP.run[kTcM - 1] & 0xffffu);
+                q.hi = causal ? (no_self ? q.jq - 1 : q.jq) : kTcM + (int)(run >> 16);
                 q.excl_self = (!causal) && no_self;
                 bnd = MO.bound[row];
                 const float Mx = bnd - 15.0f;
@@ -510,7 +510,7 @@ lsh_chunk_attn_ring_kernel(const __nv_bfloat16 *__restrict__ QK, const __nv_bflo
                 pos_next = want2 ? rg_checked_pos(S.stage[kRgEarlier][tid], n) : -1;
             }
             __syncthreads();
-            if (has_next) rg_prep(S, sF, sO, tid, scale_log2, vl);
+            if (has_next) rg_prep(S, sF, tid, scale_log2, vl);
             if (use16) {
                 // ---- F. epilogue: accumulate the round into O with the row's fixed shift
                 const bool ok = tc::mbar_wait_bounded(&S.bar[1], ph1, kTcWaitNs, K_LSH_ATTN_TC, 4);
