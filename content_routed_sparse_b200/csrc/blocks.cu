@@ -344,10 +344,13 @@ query_project_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restric
 }
 
 // K9a specialised for G query heads and rank R, streaming the descriptors
-// through shared memory.  A CTA owns a contiguous range of blocks of one
-// (sequence, KV head); chunks of 16 blocks (mu 8 KB + xi 32 KB, contiguous in
-// HBM) arrive by two bulk copies each into a 2-stage ring, so one chunk is in
-// flight while the previous is scored (two CTAs per SM).  Eight lanes share a block: lane s reads
+// through shared memory.  The work is the list of chunks of 16 blocks of every
+// (sequence, KV head) (mu 8 KB + xi 32 KB, contiguous in HBM; the last chunk of
+// a (sequence, KV head) may be short); a CTA owns a contiguous range of that list
+// (two CTAs per SM, equal ranges, so no partial last wave), reloading its scaled
+// queries when the range crosses into the next (sequence, KV head).  Chunks
+// arrive by two bulk copies each into a 2-stage ring, so one chunk is in flight
+// while the previous is scored.  Eight lanes share a block: lane s reads
 // 16-byte chunks s, s + 8, s + 16, s + 24 of each 512-byte row (a group's
 // reads are 128 contiguous bytes: no bank conflicts), forms its G x (1 + R)
 // partial dot products with the scaled queries (read the same way), and the
@@ -369,25 +372,22 @@ template <int G, int R>
 __global__ void __launch_bounds__(kBsThreadsT, 2)
 block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ mu,
                        const float *__restrict__ xi, float *__restrict__ sc_out, int n_kv, int n_q,
-                       int n_full, int blocks_per_cta, float scale) {
+                       int n_full, int total_chunks, int chunks_per_cta, float scale) {
     extern __shared__ __align__(128) unsigned char bs_raw[];
     BsSmem<G, R> &S = *reinterpret_cast<BsSmem<G, R> *>(bs_raw);
-    const int sh = blockIdx.y, seq = sh / n_kv, h = sh - seq * n_kv;
-    const int b_lo = blockIdx.x * blocks_per_cta;
-    const int b_hi = min(n_full, b_lo + blocks_per_cta);
-    if (b_lo >= b_hi) return;
-    const int n_chunks = ceil_div(b_hi - b_lo, kBsChunk);
+    const int cps = ceil_div(n_full, kBsChunk);    // chunks per (sequence, KV head)
+    const int c_lo = blockIdx.x * chunks_per_cta;
+    const int n_chunks = min(total_chunks, c_lo + chunks_per_cta) - c_lo;
+    if (n_chunks <= 0) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const float *mu_sh = mu + (size_t)sh * n_full * kBdD;
-    const float *xi_sh = xi + (size_t)sh * n_full * R * kBdD;
     auto issue = [&](int c) {                      // one thread
         const int st = c % kBsStages;
-        const int b0 = b_lo + c * kBsChunk;
-        const int nb = min(kBsChunk, b_hi - b0);
+        const int gc = c_lo + c, sh = gc / cps, b0 = (gc - sh * cps) * kBsChunk;
+        const int nb = min(kBsChunk, n_full - b0);
         const uint32_t mb = (uint32_t)nb * kBdD * 4, xb = mb * R;
         tc::mbar_arrive_expect_tx(&S.full[st], mb + xb);
-        tc::bulk_load(&S.mu[st][0][0], mu_sh + (size_t)b0 * kBdD, mb, &S.full[st]);
-        tc::bulk_load(&S.xi[st][0][0][0], xi_sh + (size_t)b0 * R * kBdD, xb, &S.full[st]);
+        tc::bulk_load(&S.mu[st][0][0], mu + ((size_t)sh * n_full + b0) * kBdD, mb, &S.full[st]);
+        tc::bulk_load(&S.xi[st][0][0][0], xi + ((size_t)sh * n_full + b0) * R * kBdD, xb, &S.full[st]);
     };
     if (tid == 0) {
         for (int st = 0; st < kBsStages; ++st) tc::mbar_init(&S.full[st], 1);
@@ -396,19 +396,25 @@ block_score_tma_kernel(const __nv_bfloat16 *__restrict__ Q, const float *__restr
     __syncthreads();
     if (tid == 0)
         for (int c = 0; c < min(kBsStages, n_chunks); ++c) issue(c);
-    for (int e = tid; e < G * kBdD; e += blockDim.x) {
-        const int g = e / kBdD, d = e - g * kBdD;
-        S.sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
-    }
-    __syncthreads();
     const int sub = lane & 7, grp = warp * 4 + (lane >> 3);     // block of the chunk
     const float4 *q4 = reinterpret_cast<const float4 *>(&S.sq[0][0]);
     bool ok = true;
+    int cur_sh = -1;
     for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kBsStages;
+        const int gc = c_lo + c, sh = gc / cps, b_hi = n_full;
+        const int b = (gc - sh * cps) * kBsChunk + grp;
+        if (sh != cur_sh) {                        // uniform: the scaled queries of this (sequence, KV head)
+            __syncthreads();                       // the previous ones are no longer read
+            const int seq = sh / n_kv, h = sh - seq * n_kv;
+            for (int e = tid; e < G * kBdD; e += blockDim.x) {
+                const int g = e / kBdD, d = e - g * kBdD;
+                S.sq[g][d] = scale * __bfloat162float(Q[((size_t)seq * n_q + h * G + g) * kBdD + d]);
+            }
+            cur_sh = sh;
+        }
         ok = ok && tc::mbar_wait_bounded(&S.full[st], (c / kBsStages) & 1, kBsWaitNs, K_BLK_SCORE, 1);
         if (__syncthreads_or(!ok)) break;
-        const int b = b_lo + c * kBsChunk + grp;
         {   // every lane computes (the group shuffles need all 32); invalid blocks only skip the store
             const float4 *m4 = reinterpret_cast<const float4 *>(&S.mu[st][grp][0]);
             const float4 *x4 = reinterpret_cast<const float4 *>(&S.xi[st][grp][0][0]);
@@ -1300,16 +1306,20 @@ extern "C" int crs_block_select(const crs_block_sel_params *p, const void *Q, co
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a));
     float *sc = static_cast<float *>(ws);
     if (G == 8 && p->b.rank == 4) {
-        const int n_sh = p->b.n_seq * p->b.n_kv;
-        const int per_sh = max(1, min(ceil_div(n_full, kBsChunk), ceil_div(148 * 4, n_sh)));
-        const int bpc = ceil_div(ceil_div(n_full, per_sh), kBsChunk) * kBsChunk;
+        const long long n_sh = (long long)p->b.n_seq * p->b.n_kv;
+        const long long total = n_sh * ceil_div(n_full, kBsChunk);
+        if (total > 0x7fffffffLL) return CRS_ERR_UNSUPPORTED;
+        int dev = 0, sms = 148;
+        CRS_TRY_CUDA(cudaGetDevice(&dev));
+        CRS_TRY_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+        const int grid = (int)min(total, (long long)2 * sms);          // two CTAs per SM, one wave
+        const int cpc = (int)ceil_div_ll(total, grid);
         const size_t smem_s = sizeof(BsSmem<8, 4>);
         CRS_TRY_CUDA(cudaFuncSetAttribute(block_score_tma_kernel<8, 4>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s));
-        dim3 gf(ceil_div(n_full, bpc), n_sh);
         ProfScope _ps(K_BLK_SCORE, s);
-        block_score_tma_kernel<8, 4><<<gf, kBsThreadsT, smem_s, s>>>(static_cast<const __nv_bfloat16 *>(Q), mu, xi,
-                                                            sc, p->b.n_kv, p->n_q, n_full, bpc, p->scale);
+        block_score_tma_kernel<8, 4><<<(unsigned)ceil_div_ll(total, cpc), kBsThreadsT, smem_s, s>>>(
+            static_cast<const __nv_bfloat16 *>(Q), mu, xi, sc, p->b.n_kv, p->n_q, n_full, (int)total, cpc, p->scale);
     } else {
     dim3 ga(ceil_div(n_full, nbt), p->b.n_seq * p->b.n_kv);
     {
