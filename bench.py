@@ -65,6 +65,25 @@ def _peaks():
             "source": "fallback"}
 
 
+def l2_gather_gbs(crs, dev, reps=5):
+    """The L2 read ceiling of 512-byte row gathers on this GPU, measured now: random rows
+    of a 16 MiB table (inside L2), one row per warp load, through crs_probe_l2_gather;
+    CUDA events around `reps` launches of 2^21 rows each, after two warm-up launches."""
+    table = torch.zeros(32768 * 128, dtype=torch.float32, device=dev)          # 32768 rows x 512 B
+    gen = torch.Generator(device=dev).manual_seed(7)
+    idx = torch.randint(0, 32768, (1 << 21,), dtype=torch.int32, device=dev, generator=gen)
+    sink = torch.zeros(4, dtype=torch.int32, device=dev)
+    for _ in range(2):
+        crs.probe_l2_gather(table, idx, sink)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        crs.probe_l2_gather(table, idx, sink)
+    b.record()
+    torch.cuda.synchronize()
+    return 512.0 * idx.numel() * reps / (a.elapsed_time(b) * 1e6)
+
+
 # ------------------------------------------------------------------ workloads --
 class Workload:
     name = ""
@@ -319,7 +338,9 @@ class PrefillWorkload(Workload):
             # two launches per step (sampled threshold pass + filter pass): the
             # step's causal score FLOPs split evenly over them
             "idx_prefill_tc": [("tensor", pairs * 4 * 64 * 2 / 2 / 1e12, "TFLOP/s")],
-            "sparse_attn": [("hbm", rows * 128 * 2 * 2 / 1e9, "GB/s"),
+            # the K/V cache (n x 512 B = 16.8 MB) stays in L2: its gathers are bound by the
+            # L2 read ceiling, measured by crs_probe_l2_gather in the same run
+            "sparse_attn": [("l2", rows * 128 * 2 * 2 / 1e9, "GB/s"),
                             ("tensor", rows * 16 * 128 * 4 / 1e12, "TFLOP/s")],
         }
 
@@ -825,6 +846,8 @@ def roofline(wl, prof, peaks, traffic=None):
             return peaks["hbm_gbs"], f"hbm_gbs ({peaks['source']})"
         if bound == "tensor":
             return peaks["bf16_tflops"], f"bf16_tflops ({peaks['source']})"
+        if bound == "l2":
+            return peaks["l2_gather_gbs"], "l2_gather_gbs (crs_probe_l2_gather on this GPU, this run)"
         return FP32_ALU_TFLOPS_NOMINAL, "fp32 FMA: 148 SM x 128 lanes x 2 x 1.965 GHz"
 
     # the binding roofline: the resource whose algorithmic work takes longest at its peak
@@ -1093,6 +1116,7 @@ def main():
     import content_routed_sparse_b200 as crs
 
     peaks = _peaks()
+    peaks["l2_gather_gbs"] = l2_gather_gbs(crs, dev)
     flush_buf = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB
     wl = WORKLOADS[args.workload](crs, dev)
     sampler = ClockSampler(local)

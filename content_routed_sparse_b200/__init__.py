@@ -260,6 +260,24 @@ def debug_force_wait_timeout(on: bool) -> None:
     _check("crs_debug_force_wait_timeout", _lib.crs_debug_force_wait_timeout(1 if on else 0))
 
 
+_sig("crs_probe_l2_gather", ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_void_p])
+
+
+def probe_l2_gather(table: torch.Tensor, idx: torch.Tensor, sink: torch.Tensor) -> None:
+    """Gather the 512-byte rows idx of table (rows x 512 bytes) once, on the current
+    stream; a measurement aid for the L2 gather ceiling (see include/crs.h)."""
+    if not (table.is_cuda and idx.is_cuda and sink.is_cuda) or idx.dtype != torch.int32:
+        raise ValueError("probe_l2_gather: CUDA table, int32 idx and sink expected")
+    if table.numel() * table.element_size() % 512 or not table.is_contiguous() or not idx.is_contiguous():
+        raise ValueError("probe_l2_gather: contiguous table of 512-byte rows expected")
+    if sink.numel() * sink.element_size() < 16:
+        raise ValueError("probe_l2_gather: sink of at least 16 bytes expected")
+    rows = table.numel() * table.element_size() // 512
+    _check("crs_probe_l2_gather", _lib.crs_probe_l2_gather(table.data_ptr(), rows, idx.data_ptr(), idx.numel(),
+                                                           sink.data_ptr(), _stream(None)))
+
+
 def profile_set(enabled: bool) -> None:
     """Turn per-launch CUDA-event timing on or off (launch counting is always on)."""
     _check("crs_profile_set", _lib.crs_profile_set(1 if enabled else 0))

@@ -8,10 +8,13 @@
 // One CTA = one (row, KV head, split of the list).  The G <= 16 query heads
 // of the KV head form the M = 16 side of mma.sync.m16n8k16 (bf16 in, fp32
 // accumulate).  Keys are gathered 64 per stage with 16-byte cp.async into
-// XOR-swizzled shared rows (a ring of 3 tiles, two in flight while one is
+// XOR-swizzled shared rows (a ring of 2 tiles, one in flight while the other is
 // consumed; one barrier per tile); each of the 4 warps owns 16
 // keys of a stage and keeps its own online-softmax state; the warps merge at
-// the end.  The path is bound by the gather bandwidth.
+// the end.  The path is bound by gather latency: with two tiles (64 KB) and the
+// query tile placed over the second ring slot until that slot's first gather,
+// three CTAs share an SM at a 2048-key list (a three-tile ring held two:
+// 6.6 -> 4.8 ms at prefill).
 #include <math.h>
 
 #include "common.cuh"
@@ -24,7 +27,7 @@ constexpr int kSaWarps = 4;
 constexpr int kSaThreads = kSaWarps * 32;
 constexpr int kSaRowBytes = kSaD * 2;                 // 256 B per K or V row
 constexpr int kSaTileBytes = kSaKeys * kSaRowBytes;   // 16 KB
-constexpr int kSaStages = 3;                          // K/V tiles in the ring
+constexpr int kSaStages = 2;                          // K/V tiles in the ring
 constexpr float kLog2e = 1.4426950408889634f;
 
 // 2^x by the hardware approximation (relative error about 2^-22, far inside the
@@ -89,8 +92,10 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
     extern __shared__ __align__(128) unsigned char sa_smem[];
     unsigned char *sK = sa_smem;                                  // [kSaStages][kSaTileBytes]
     unsigned char *sV = sK + kSaStages * kSaTileBytes;            // [kSaStages][kSaTileBytes]
-    unsigned char *sQ = sV + kSaStages * kSaTileBytes;            // [16 rows][256 B] swizzled
-    float *sRed = reinterpret_cast<float *>(sQ + 16 * kSaRowBytes);   // [4][16] m, [4][16] l
+    // [16 rows][256 B] swizzled, over ring slot 1: its first gather is issued after every
+    // warp has read the query fragments (they are read before the loop's first barrier)
+    unsigned char *sQ = sK + 1 * kSaTileBytes;
+    float *sRed = reinterpret_cast<float *>(sV + kSaStages * kSaTileBytes);   // [4][16] m, [4][16] l
     int *sIdx = reinterpret_cast<int *>(sRed + kSaWarps * 16 * 2);      // the split's list, -1 padded
 
     const int split = blockIdx.x;
@@ -358,7 +363,8 @@ constexpr int kSaMaxSplit = 4096;     // keys per split: the split's list sits i
 static size_t sa_smem_bytes(int split_len) {
     static_assert((size_t)kSaWarps * 16 * kSaD * 4 <= 2 * kSaStages * (size_t)kSaTileBytes,
                   "merge scratch must fit in the K/V ring");
-    return 2 * kSaStages * (size_t)kSaTileBytes + 16 * kSaRowBytes + (size_t)kSaWarps * 16 * 2 * 4 +
+    static_assert(kSaStages >= 2, "the query tile sits over ring slot 1");
+    return 2 * kSaStages * (size_t)kSaTileBytes + (size_t)kSaWarps * 16 * 2 * 4 +
            (size_t)split_len * 4;
 }
 

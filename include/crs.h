@@ -92,6 +92,18 @@ int crs_get_device_diag(void *stream, uint32_t *out, int n);
  * if the device global cannot be written. */
 int crs_debug_force_wait_timeout(int on);
 
+/* Measurement aid (no counterpart in the pages): the L2 read ceiling of row
+ * gathers, against which the gather attention over an L2-resident K/V set is
+ * reported.  Reads the `n_idx` rows idx[0 .. n_idx) (each 0 <= idx[i] < rows)
+ * of `table` (device, rows x 512 bytes, 16-byte aligned), one 512-byte row per
+ * warp load instruction (32 lanes x 16 bytes, L1 bypassed), from 8 CTAs of 512
+ * threads per SM; a warp writes the XOR of what it read to `sink` (device,
+ * 16 bytes) only when that XOR equals a fixed constant, which keeps the loads.  The caller times the launch on `stream`
+ * (a table of 16 MiB stays in L2).  CRS_ERR_INVALID_ARG for null pointers,
+ * rows < 1 or n_idx < 1; index values are the caller's to keep in range. */
+int crs_probe_l2_gather(const void *table, int64_t rows, const int32_t *idx, int64_t n_idx, void *sink,
+                        void *stream);
+
 /* Launch tracing.  [P1] "一个可复现的评测矩阵" and [P2] §1.1 "性能轴" ask for the
  * time of every stage (routing, sort, selection, gather, attention) reported
  * separately; this is how the library provides it.  Every kernel
