@@ -704,7 +704,9 @@ static int launch_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const v
     const crs_lsh_params &p = a->p;
     bool tc_done = false;
     if constexpr (std::is_same<T, __nv_bfloat16>::value && DH == kTcD) {
-        if (p.chunk == kTcM) {
+        // 16-byte row pieces are read from QK and V: both must be 16-byte aligned
+        const bool aligned = !(reinterpret_cast<uintptr_t>(QK) & 15) && !(reinterpret_cast<uintptr_t>(V) & 15);
+        if (p.chunk == kTcM && aligned) {
             // tensor-core path: bf16, d = 64, chunk = 128
             const size_t smem = sizeof(LshTcSmem) + 1024;
             CRS_TRY_CUDA(cudaFuncSetAttribute(lsh_chunk_attn_tc_kernel,
@@ -820,6 +822,7 @@ extern "C" int crs_lsh_attn(const crs_lsh_attn_params *a, const void *QK, const 
     const crs_lsh_params &p = a->p;
     if (p.chunk < 1 || p.chunk > 128) return CRS_ERR_INVALID_ARG;
     if (!QK || !V || !bucket || !perm || !inv_perm || !O) return CRS_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(O) & 15) return CRS_ERR_INVALID_ARG;   // 16-byte row stores
     if (!(a->scale == a->scale)) return CRS_ERR_INVALID_ARG;
     const size_t need = crs_lsh_attn_workspace_size(a);
     if (!ws || ws_bytes < need) return CRS_ERR_WORKSPACE;

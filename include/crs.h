@@ -176,7 +176,11 @@ typedef struct {
  * O: [B,H,n,d] f32, written in original token order (f32 whatever p.dtype:
  * the 2e-3 output tolerance for bf16 inputs is below bf16's unit roundoff
  * 2^-8, so the result keeps the fp32 accumulator's precision);
- * lse: [B,H,n] f32 natural-log normaliser of the merged softmax, or NULL. */
+ * lse: [B,H,n] f32 natural-log normaliser of the merged softmax, or NULL.
+ * O must start on a 16-byte boundary (rows are written as 16-byte vectors;
+ * else CRS_ERR_INVALID_ARG).  The tensor-core kernels also read QK and V rows
+ * as 16-byte pieces: with either not 16-byte aligned the call takes the
+ * CUDA-core kernel instead. */
 size_t crs_lsh_attn_workspace_size(const crs_lsh_attn_params *p);
 int crs_lsh_attn(const crs_lsh_attn_params *p, const void *QK, const void *V,
                  const int32_t *bucket, const int32_t *perm, const int32_t *inv_perm,

@@ -214,3 +214,21 @@ def test_lsh_hash_tensor_core_near_ties(crs, cuda_dev):
     crs.profile_collect()
     _route_and_check(crs, case)
     assert "lsh_hash" in crs.profile_collect()
+
+
+def test_lsh_bf16_unaligned_inputs_take_the_cuda_core_kernel(crs, cuda_dev):
+    """QK and V that do not start on a 16-byte boundary cannot feed the tensor-core
+    kernels' 16-byte row reads: the call takes the CUDA-core kernel, same results."""
+    case = workloads.lsh_clustered_case(B=1, H=2, n=700, n_buckets=16, n_rounds=2, chunk=128,
+                                        n_centres=8, pad_frac=0.1, seed=31, device=cuda_dev)
+    r = _route_and_check(crs, case)
+    for k in ("QK", "V"):                      # same values, storage shifted by one element (2 bytes)
+        t = case[k]
+        buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+        case[k] = buf[1:].view(t.shape)
+        case[k].copy_(t)
+        assert case[k].data_ptr() % 16 != 0
+    crs.profile_collect()
+    _attn_and_check(crs, case, *r)
+    prof = crs.profile_collect()
+    assert "lsh_chunk_attn" in prof and "lsh_chunk_attn_ring" not in prof and "lsh_chunk_attn_tc" not in prof
