@@ -442,6 +442,9 @@ extern "C" int crs_sparse_attn(const crs_attn_params *p, const void *Q, const vo
     int st = sa_validate(p);
     if (st) return st;
     if (!Q || !K || !V || !I || !O) return CRS_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) |
+         reinterpret_cast<uintptr_t>(ws)) & 15)
+        return CRS_ERR_INVALID_ARG;                       // 16-byte row pieces
     const size_t need = crs_sparse_attn_workspace_size(p);
     if (need > 0 && (!ws || ws_bytes < need)) return CRS_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

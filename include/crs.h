@@ -582,6 +582,8 @@ typedef struct {
  * O: [n_rows, n_q, D] f32 (the fp32 accumulator's precision; P.V runs on bf16
  * tensor cores with P split into a bf16 value and a bf16 residual);
  * lse: [n_rows, n_q] f32 or NULL.
+ * Q, K, V and the workspace must start on 16-byte boundaries (rows are read as
+ * 16-byte pieces; else CRS_ERR_INVALID_ARG).
  * Workspace: crs_sparse_attn_workspace_size(p), queried with the same device
  * current as the call (the split count depends on the device's SM count). */
 size_t crs_sparse_attn_workspace_size(const crs_attn_params *p);

@@ -49,6 +49,11 @@ def test_host_validation_without_gpu(crs):
     assert lib.crs_sparse_attn(ctypes.byref(ap), *([None] * 10), 0, None) == 1
     bp = crs.BlockParams(1, 1, 64, 128, 31, 4, 0, 2)     # odd L
     assert lib.crs_block_describe(ctypes.byref(bp), None, None, None, None) == 2
+    # Q, K or V off a 16-byte boundary: rejected before any launch
+    ap = crs.AttnParams(4, 16, 1, 128, 16, 1, 100, 0.1)
+    f16, f2 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10002)
+    assert lib.crs_sparse_attn(ctypes.byref(ap), f16, f2, f16, None, f16, None, None, f16, None, None, 0,
+                               None) == 1
     # O not on a 16-byte boundary: rejected before the workspace is looked at (no launch)
     a = crs.LshAttnParams(crs.LshParams(1, 1, 256, 64, 16, 2, 128, 1), 1, 0, 1, 0.125)
     fake = ctypes.c_void_p(0x10000)
