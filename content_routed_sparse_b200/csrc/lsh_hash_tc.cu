@@ -25,7 +25,7 @@
 // wins in the chain values.
 //
 // Persistent, warp-specialised CTA walking the 128-token tiles of one
-// (batch, head): warp 0 loads X tiles with TMA into a 3-stage ring, warp 1
+// (batch, head): warp 0 loads X tiles with TMA into a 2-stage ring, warp 1
 // issues the MMAs into two tensor-memory buffers, warps 2..9 (one token row
 // per thread; two warps per row quadrant, each taking half of the rounds) read
 // the scores, decide the buckets and release the buffers.
@@ -39,7 +39,7 @@ constexpr int kHtM = 128;                 // tokens per tile (MMA M)
 constexpr int kHtHalf = 32;               // b / 2
 constexpr int kHtD = 64;
 constexpr int kHtMaxN = 128;              // 32 x rounds, rounds <= 4
-constexpr int kHtStages = 3;
+constexpr int kHtStages = 2;                  // X tiles in flight (the fp32 R copy takes the third's room)
 constexpr int kHtEpiWarps = 8;            // two per tensor-memory lane quadrant, each half the rounds
 constexpr int kHtThreads = 32 * (2 + kHtEpiWarps);
 constexpr float kHtErr = 2.44140625e-4f;  // 2^-12
@@ -50,15 +50,40 @@ struct HtSmem {
     unsigned char x[kHtStages][kHtM * 128];   // X tiles, 128B swizzle
     unsigned char bhi[kHtMaxN * 128];         // B operand: R_hi, row r*32 + k = column k of R_{h,r}
     unsigned char blo[kHtMaxN * 128];         //            R_lo
+    float rf[kHtMaxN * kHtD];                 // R_{h,r} in fp32, [r][t][k] as in global memory: the
+                                              // exact chains of the near ties read it here
     float rnorm[kHtMaxN];                     // |r_k| per column
     uint64_t xfull[kHtStages], xempty[kHtStages], tfull[2], tempty[2];
     uint32_t tmem_base;
     int fail;
 };
 
-__device__ __forceinline__ float ht_x(const unsigned char *xt, int row, int t) {
-    const uint16_t b = *reinterpret_cast<const uint16_t *>(xt + tc::sw128(row, t >> 3) + (t & 7) * 2);
-    return __uint_as_float((uint32_t)b << 16);
+// The definition's bucket of token row rl of the X tile xa for one round (R_{h,r} at Rr,
+// fp32, [t][k]): lane k evaluates the chain u_k = fma(x_63, r_63k, ... fma(x_0, r_0k, 0)) in
+// index order, then the first maximum of [u ; -u].  Warp-collective; out of line so that
+// the common path of the epilogue keeps its registers.
+__device__ __noinline__ int ht_exact_bucket(const unsigned char *xa, int rl, const float *Rr, int lane) {
+    // token row rl: eight 16-byte broadcast reads; column `lane` of R from shared memory
+    uint32_t xw[kHtD / 2];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 w4 = *reinterpret_cast<const uint4 *>(xa + tc::sw128(rl, c));
+        xw[4 * c] = w4.x;
+        xw[4 * c + 1] = w4.y;
+        xw[4 * c + 2] = w4.z;
+        xw[4 * c + 3] = w4.w;
+    }
+    float u = 0.0f;
+#pragma unroll
+    for (int t = 0; t < kHtD; ++t) {
+        const float xt = __uint_as_float((t & 1) ? (xw[t >> 1] & 0xffff0000u) : (xw[t >> 1] << 16));
+        u = __fmaf_rn(xt, Rr[t * kHtHalf + lane], u);
+    }
+    const float bp = warp_max(u);
+    const int ap = __ffs(__ballot_sync(0xffffffffu, u == bp)) - 1;
+    const float bn = warp_max(-u);
+    const int an = __ffs(__ballot_sync(0xffffffffu, -u == bn)) - 1;
+    return (bp >= bn) ? ap : kHtHalf + an;
 }
 
 __global__ void __launch_bounds__(kHtThreads, 2)
@@ -102,6 +127,7 @@ lsh_hash_tc_kernel(const __grid_constant__ CUtensorMap tx, const float *__restri
             if (e >= N * kHtD) break;
             const int k = e & (kHtHalf - 1), t = (e >> 5) & (kHtD - 1), r = e >> 11;
             const uint32_t off = tc::sw128(r * kHtHalf + k, t >> 3) + (t & 7) * 2;
+            S.rf[e] = v[u];
             const __nv_bfloat16 hi = __float2bfloat16_rn(v[u]);
             const __nv_bfloat16 lo = __float2bfloat16_rn(v[u] - __bfloat162float(hi));
             *reinterpret_cast<__nv_bfloat16 *>(S.bhi + off) = hi;
@@ -245,22 +271,12 @@ lsh_hash_tc_kernel(const __grid_constant__ CUtensorMap tx, const float *__restri
                 const bool amb = !((m1 - (E1 + E2) - m1 * 0x1p-16f > m2) && (m1 > E1));
                 // exact chains for the undecided tokens of this warp, one token at a time
                 uint32_t pend = __ballot_sync(0xffffffffu, amb && tok < n);
-                const float *Rr = Rh + (size_t)r * kHtD * kHtHalf;
+                const float *Rr = S.rf + r * kHtD * kHtHalf;
                 while (pend) {
                     const int l = __ffs(pend) - 1;
                     pend &= pend - 1;
-                    const int rl = quad * 32 + l;
-                    float rv[kHtD];               // column `lane` of R_{h,r}, all loads in flight
-#pragma unroll
-                    for (int t = 0; t < kHtD; ++t) rv[t] = __ldg(Rr + t * kHtHalf + lane);
-                    float u = 0.0f;
-#pragma unroll
-                    for (int t = 0; t < kHtD; ++t) u = __fmaf_rn(ht_x(xa, rl, t), rv[t], u);
-                    const float bp = warp_max(u);
-                    const int ap = __ffs(__ballot_sync(0xffffffffu, u == bp)) - 1;
-                    const float bn = warp_max(-u);
-                    const int an = __ffs(__ballot_sync(0xffffffffu, -u == bn)) - 1;
-                    if (lane == l) bk = (bp >= bn) ? ap : kHtHalf + an;
+                    const int e = ht_exact_bucket(xa, quad * 32 + l, Rr, lane);
+                    if (lane == l) bk = e;
                 }
                 if (tok < n) bucket[((size_t)bh * rounds + r) * n + tok] = bk;
             }
