@@ -503,18 +503,18 @@ idx_tc_final_kernel(const uint32_t *__restrict__ cand_key, const int32_t *__rest
 #pragma unroll
         for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0u;
         __syncwarp();
-        // four keys per lane in flight per step (the passes are bound by load latency)
+        // eight keys per lane in flight per step (the passes are bound by load latency)
 #pragma unroll
         for (int q = 0; q < kIParts; ++q)
-            for (int i0 = lane; i0 < c[q]; i0 += 4 * 32) {
-                uint32_t kk[4];
+            for (int i0 = lane; i0 < c[q]; i0 += 8 * 32) {
+                uint32_t kk[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 8; ++u) {
                     const int i = i0 + u * 32;
                     kk[u] = i < c[q] ? __ldg(ck + q * kICap + i) : 0u;
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+                for (int u = 0; u < 8; ++u)
                     if (i0 + u * 32 < c[q] && (kk[u] & mask) == prefix) atomicAdd(&hist[(kk[u] >> shift) & 255u], 1u);
             }
         __syncwarp();
@@ -529,18 +529,18 @@ idx_tc_final_kernel(const uint32_t *__restrict__ cand_key, const int32_t *__rest
     __syncwarp();
 #pragma unroll
     for (int q = 0; q < kIParts; ++q)
-        for (int i0 = lane; i0 < c[q]; i0 += 4 * 32) {
-            uint32_t kk[4];
-            int pos[4];
+        for (int i0 = lane; i0 < c[q]; i0 += 8 * 32) {
+            uint32_t kk[8];
+            int pos[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int i = i0 + u * 32;
                 const bool in = i < c[q];
                 kk[u] = in ? __ldg(ck + q * kICap + i) : 0u;
                 pos[u] = in ? __ldg(ci + q * kICap + i) : 0;
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < 8; ++u)
                 if (i0 + u * 32 < c[q] && kk[u] >= T)
                     atomicOr(kk[u] > T ? &bm_gt[pos[u] >> 5] : &bm_eq[pos[u] >> 5], 1u << (pos[u] & 31));
         }
