@@ -88,6 +88,11 @@ struct SaArgs {
     float scale_log2;   // scale * log2(e)
 };
 
+// kOff32: the list holds each token's offset from K (and V) in 16-byte units, which fits
+// an int when the cache is below 32 GB (the host checks), so a gather piece needs one
+// 32-bit multiply instead of the 64-bit position arithmetic; -1 marks a skipped entry
+// either way.
+template <bool kOff32>
 __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
     extern __shared__ __align__(128) unsigned char sa_smem[];
     unsigned char *sK = sa_smem;                                  // [kSaStages][kSaTileBytes]
@@ -133,7 +138,8 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
         }
         if (j > qlim) j = -1;
         if (j >= 0 && a.key_valid && a.key_valid[kbase + j] == 0) j = -1;
-        sIdx[i] = j;
+        if constexpr (kOff32) sIdx[i] = j >= 0 ? (int)((kbase + j) * (int64_t)(tok_stride / 8)) : -1;
+        else sIdx[i] = j;
     }
     __syncthreads();
 
@@ -151,7 +157,9 @@ __global__ void __launch_bounds__(kSaThreads) sparse_attn_kernel(SaArgs a) {
                 const int r = e >> 4, c = e & 15;
                 const int j = si[r];
                 const bool ok = j >= 0;
-                const size_t off = ok ? ((size_t)(kbase + j) * tok_stride + c * 8) : 0;
+                size_t off;                            // elements from Kh / Vh
+                if constexpr (kOff32) off = ok ? ((size_t)(unsigned)j + (unsigned)c) * 8u : 0;
+                else off = ok ? ((size_t)(kbase + j) * tok_stride + c * 8) : 0;
                 cp_async16_zfill(k_dst + sw_off(r, c), Kh + off, ok);
                 cp_async16_zfill(v_dst + sw_off(r, c), Vh + off, ok);
             }
@@ -385,7 +393,7 @@ static int sa_splits(const crs_attn_params *p) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
-        cudaFuncGetAttributes(&fa, sparse_attn_kernel) != cudaSuccess) {
+        cudaFuncGetAttributes(&fa, sparse_attn_kernel<true>) != cudaSuccess) {
         cudaGetLastError();          // model with the defaults; the launch reports real errors
         sms = 148;
     }
@@ -476,12 +484,15 @@ extern "C" int crs_sparse_attn(const crs_attn_params *p, const void *Q, const vo
                                                           ~size_t(255)))
                              : nullptr;
     const size_t smem = sa_smem_bytes(a.split_len);
-    CRS_TRY_CUDA(cudaFuncSetAttribute(sparse_attn_kernel,
+    // 16-byte offsets of every token fit an int below 32 GB of K (or V)
+    const bool off32 = (long long)p->n_keys * p->n_kv * (kSaD / 8) <= 0x7fffffffLL;
+    auto kern = off32 ? sparse_attn_kernel<true> : sparse_attn_kernel<false>;
+    CRS_TRY_CUDA(cudaFuncSetAttribute(kern,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     dim3 grid(a.splits, p->n_rows * p->n_kv);
     {
         ProfScope _ps(K_SA_MAIN, s);
-        sparse_attn_kernel<<<grid, kSaThreads, smem, s>>>(a);
+        kern<<<grid, kSaThreads, smem, s>>>(a);
     }
     CRS_CHECK_LAUNCH();
     if (a.splits > 1) {
