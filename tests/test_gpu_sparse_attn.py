@@ -108,3 +108,32 @@ def test_out_of_range_index_is_flagged_and_skipped(crs, cuda_dev):
     assert crs.get_device_error() & crs.DEVERR_INDEX
     oO2, _ = oracle.sparse_attn(_np(Q[:1]), _np(K), _np(V), np.array([[[3, -1, 4]]], np.int32))
     assert rel_err(_np(O2), oO2).max() <= TOL
+
+
+def test_wide_offset_form_matches(crs, cuda_dev):
+    """Caches past 32 GB take the 64-bit position arithmetic; force that form by declaring a
+    larger token count (every index stays inside the real cache) and compare bitwise with
+    the 16-byte-offset form the real count selects."""
+    import ctypes
+    rng = np.random.default_rng(5)
+    g = torch.Generator(device=cuda_dev).manual_seed(5)
+    n_rows, n_q, n_kv, max_idx, n_tok = 12, 8, 2, 640, 3000
+    Q = torch.randn(n_rows, n_q, 128, generator=g, device=cuda_dev).to(torch.bfloat16)
+    K = torch.randn(n_tok, n_kv, 128, generator=g, device=cuda_dev).to(torch.bfloat16)
+    V = torch.randn(n_tok, n_kv, 128, generator=g, device=cuda_dev).to(torch.bfloat16)
+    I = torch.from_numpy(_random_lists(rng, n_rows, 1, max_idx, n_tok, None)).to(cuda_dev)
+    O32, _ = crs.sparse_attn(Q, K, V, I)
+    wide_keys = (1 << 31) // (n_kv * 16) + 1          # 16-byte offsets past the int range
+    p = crs.AttnParams(n_rows, n_q, n_kv, 128, max_idx, 1, wide_keys, 1.0 / np.sqrt(128))
+    lib = crs.lib()
+    wsb = int(lib.crs_sparse_attn_workspace_size(ctypes.byref(p)))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=cuda_dev)
+    O64 = torch.empty_like(O32)
+    st = lib.crs_sparse_attn(ctypes.byref(p), ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(K.data_ptr()),
+                             ctypes.c_void_p(V.data_ptr()), None, ctypes.c_void_p(I.data_ptr()), None, None,
+                             ctypes.c_void_p(O64.data_ptr()), None, ctypes.c_void_p(ws.data_ptr()), wsb,
+                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert crs.get_device_error() == 0
+    assert torch.equal(O32, O64)
