@@ -34,6 +34,20 @@
 // unbalanced); the k-th chunk a warp handles (chunk 2k + wg) puts its P (16
 // columns) at rg_pcol(k, wg), inside the S columns that warp has already read.
 // P fills [0,128); O goes to [128,192).
+//
+// One item, slots P (chunk c-1), O (chunk c), F (free), all 256 threads:
+//   A  positions of chunk c+1 into F's metadata; barrier (the previous item's
+//      epilogue reads of P's slot and of tensor memory are done);
+//   B  thread 0 issues S (mbarrier bar[0]); the rows of c+1 go to F by cp.async
+//      (during C for an fp16 item); F's buckets, earlier-round slots and the
+//      perm entries of c+2 by 4-byte cp.async into shared memory;
+//   C  wait bar[0] with a CTA vote; softmax of the item's rows, P stored to tensor
+//      memory; tcgen05.wait::st, barrier; thread 0 issues P V (bar[1]);
+//   E  cp.async wait; F's metadata finished from the staged words; barrier;
+//      F prepared (V to fp16, norms, bounds, bucket runs; proxy fence);
+//   F  wait bar[1] with a CTA vote; O rows staged in P's slot, reductions into O;
+//   G  barrier; the ring turns (P <- O <- F <- P).
+// Every wait is bounded; a CTA that gives up drains its MMA and leaves the loop.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
