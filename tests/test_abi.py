@@ -54,6 +54,11 @@ def test_host_validation_without_gpu(crs):
     f16, f2 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10002)
     assert lib.crs_sparse_attn(ctypes.byref(ap), f16, f2, f16, None, f16, None, None, f16, None, None, 0,
                                None) == 1
+    # the L2 probe: null pointers or empty sizes are rejected before any CUDA call
+    f16 = ctypes.c_void_p(0x10000)
+    assert lib.crs_probe_l2_gather(None, 1, f16, 1, f16, None) == 1
+    assert lib.crs_probe_l2_gather(f16, 0, f16, 1, f16, None) == 1
+    assert lib.crs_probe_l2_gather(f16, 1, f16, 0, f16, None) == 1
     # O not on a 16-byte boundary: rejected before the workspace is looked at (no launch)
     a = crs.LshAttnParams(crs.LshParams(1, 1, 256, 64, 16, 2, 128, 1), 1, 0, 1, 0.125)
     fake = ctypes.c_void_p(0x10000)
